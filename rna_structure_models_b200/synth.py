@@ -1,0 +1,203 @@
+"""Seeded synthetic inputs for the IPA core and the geometric attention variant.
+
+This module only draws random numbers in the shapes, distributions and
+structure of the workloads; it computes none of the attention arithmetic.
+Both the float64 oracle (tests only) and the CUDA path are fed from here.
+
+Structure of the inputs (stand-ins for the protein / RNA backbones that the
+Flash Invariant Point Attention paper trains on, Fig. 2-4, which are not
+available here):
+  * frames T_i = (R_i, t_i): R_i a proper rotation from the QR decomposition
+    of a Gaussian 3x3 matrix (sign fixed by diag(R), first column flipped if
+    det < 0); t_i a C-alpha-like random walk with 3.8 Angstrom steps in
+    directions uniform on the sphere, starting at the origin;
+  * q/k/v, query/key/value points and the pair factors z1/z2 ~ N(0, 1);
+  * w_bias ~ N(0, 0.1^2) (std 0.1); gamma = softplus(N(0, 1)) (already > 0).
+
+Draw order (fixed, one numpy PCG64 stream per call): rotations, walk,
+(jitter), q, k, v, q_pts, k_pts, v_pts, z1, z2, w_bias, gamma, masks.
+Arrays are drawn in float64 and returned as float32 (masks as bool); the
+oracle up-casts the same float32 values, so parity never measures input
+rounding.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+__all__ = [
+    "IpaDims", "GeoDims", "ipa_inputs", "geo_inputs", "ipa_preset", "geo_preset",
+    "IPA_PRESETS", "random_rotations", "random_walk",
+]
+
+
+@dataclass(frozen=True)
+class IpaDims:
+    B: int
+    L: int
+    H: int
+    C: int = 16
+    Pq: int = 4
+    Pv: int = 8
+    R: int = 2
+    Cz: int = 128
+
+    @property
+    def F(self) -> int:
+        """Output features per (residue, head): scalar | points xyz | point norms | pair."""
+        return self.C + 3 * self.Pv + self.Pv + self.Cz
+
+
+@dataclass(frozen=True)
+class GeoDims:
+    B: int
+    N: int
+    H: int
+    M: int
+    Cout: int
+
+
+def random_rotations(rng: np.random.Generator, n: int) -> np.ndarray:
+    """n proper rotations: QR of Gaussian 3x3, sign-fixed, det forced to +1."""
+    a = rng.standard_normal((n, 3, 3))
+    q, r = np.linalg.qr(a)
+    d = np.sign(np.diagonal(r, axis1=1, axis2=2))
+    d[d == 0] = 1.0
+    q = q * d[:, None, :]
+    neg = np.linalg.det(q) < 0
+    q[neg, :, 0] *= -1.0
+    return q
+
+
+def random_walk(rng: np.random.Generator, n: int, step: float = 3.8) -> np.ndarray:
+    """Positions of an n-point walk with fixed step length and isotropic directions."""
+    u = rng.standard_normal((max(n - 1, 0), 3))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    t = np.zeros((n, 3))
+    if n > 1:
+        t[1:] = np.cumsum(step * u, axis=0)
+    return t
+
+
+def _softplus_draw(x: np.ndarray) -> np.ndarray:
+    # distribution of gamma in the workloads: softplus of a standard normal draw
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+
+
+def ipa_inputs(dims: IpaDims, seed: int = 0, *, masked_tail_frac: float = 0.0,
+               ragged: tuple[int, int] | None = None, jitter: float = 0.0) -> dict:
+    """Seeded IPA-core inputs.
+
+    masked_tail_frac: the last round(frac * L) residues of every batch element
+      are masked out (mask False).
+    ragged: (lo, hi) -> per batch element a length L_b uniform in [lo, hi]
+      (inclusive); mask[b, i] = i < L_b.
+    jitter: std (Angstrom) of isotropic Gaussian noise added to the walk.
+    """
+    B, L, H, C, Pq, Pv, R, Cz = (dims.B, dims.L, dims.H, dims.C, dims.Pq,
+                                 dims.Pv, dims.R, dims.Cz)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rot = random_rotations(rng, B * L).reshape(B, L, 3, 3)
+    trans = np.stack([random_walk(rng, L) for _ in range(B)])
+    if jitter > 0.0:
+        trans = trans + jitter * rng.standard_normal(trans.shape)
+    q = rng.standard_normal((B, L, H, C))
+    k = rng.standard_normal((B, L, H, C))
+    v = rng.standard_normal((B, L, H, C))
+    q_pts = rng.standard_normal((B, L, H, Pq, 3))
+    k_pts = rng.standard_normal((B, L, H, Pq, 3))
+    v_pts = rng.standard_normal((B, L, H, Pv, 3))
+    z1 = rng.standard_normal((B, L, R, Cz))
+    z2 = rng.standard_normal((B, L, R, Cz))
+    w_bias = 0.1 * rng.standard_normal((Cz, H))
+    gamma = _softplus_draw(rng.standard_normal(H))
+    mask = np.ones((B, L), dtype=bool)
+    lengths = np.full(B, L)
+    if ragged is not None:
+        lengths = rng.integers(ragged[0], ragged[1] + 1, size=B)
+        mask = np.arange(L)[None, :] < lengths[:, None]
+    if masked_tail_frac > 0.0:
+        n_mask = int(round(masked_tail_frac * L))
+        if n_mask > 0:
+            mask[:, L - n_mask:] = False
+            lengths = np.minimum(lengths, L - n_mask)
+    f32 = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    return {
+        "dims": dims,
+        "q": f32(q), "k": f32(k), "v": f32(v),
+        "q_pts": f32(q_pts), "k_pts": f32(k_pts), "v_pts": f32(v_pts),
+        "rot": f32(rot), "trans": f32(trans),
+        "z1": f32(z1), "z2": f32(z2),
+        "w_bias": f32(w_bias), "gamma": f32(gamma),
+        "mask": np.ascontiguousarray(mask),
+        "lengths": lengths,
+    }
+
+
+def geo_inputs(dims: GeoDims, seed: int = 0, *, pair_drop: float = 0.2,
+               frame_drop: float = 0.05, with_pair_mask: bool = True,
+               with_bias: bool = True) -> dict:
+    """Seeded inputs of the direction/distance geometric attention variant.
+
+    Draw order: rotations, walk, q_direction, k_direction, q_point, k_point,
+    values, direction_scale, distance_scale, output_weight, output_bias,
+    frame_mask, pair_mask.  output_weight ~ N(0, 1/(H*M*3)) and
+    output_bias ~ N(0, 0.1^2) (the pages give no distribution for them).
+    """
+    B, N, H, M, Cout = dims.B, dims.N, dims.H, dims.M, dims.Cout
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rot = random_rotations(rng, B * N).reshape(B, N, 3, 3)
+    trans = np.stack([random_walk(rng, N) for _ in range(B)])
+    qd = rng.standard_normal((B, N, H, 3))
+    kd = rng.standard_normal((B, N, H, 3))
+    qp = rng.standard_normal((B, N, H, 3))
+    kp = rng.standard_normal((B, N, H, 3))
+    values = rng.standard_normal((B, N, H, M, 3))
+    dscale = rng.standard_normal(H)
+    xscale = rng.standard_normal(H)
+    w_out = rng.standard_normal((H * M * 3, Cout)) / math.sqrt(H * M * 3)
+    b_out = 0.1 * rng.standard_normal(Cout)
+    frame_mask = rng.random((B, N)) >= frame_drop
+    pair_mask = None
+    if with_pair_mask:
+        pair_mask = rng.random((B, H, N, N)) >= pair_drop
+    f32 = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    return {
+        "dims": dims,
+        "q_direction": f32(qd), "k_direction": f32(kd),
+        "q_point": f32(qp), "k_point": f32(kp), "values": f32(values),
+        "direction_scale": f32(dscale), "distance_scale": f32(xscale),
+        "output_weight": f32(w_out),
+        "output_bias": f32(b_out) if with_bias else None,
+        "rotation": f32(rot), "translation": f32(trans),
+        "frame_mask": np.ascontiguousarray(frame_mask),
+        "pair_mask": pair_mask,
+    }
+
+
+# Named workloads.  Sizes follow the IPA module of AlphaFold-2-style models
+# (12 heads, 16 scalar channels, 4 query / 8 value points) with a rank-2
+# factorised pair representation of 128 channels.
+IPA_PRESETS = {
+    "tiny": (IpaDims(B=1, L=64, H=4, C=16, Pq=4, Pv=8, R=2, Cz=16), {}),
+    "af2": (IpaDims(B=1, L=512, H=12, Cz=128), {"masked_tail_frac": 0.1}),
+    "long2048": (IpaDims(B=1, L=2048, H=12, Cz=128), {}),
+    "long4096": (IpaDims(B=1, L=4096, H=12, Cz=128), {}),
+    "long8192": (IpaDims(B=1, L=8192, H=12, Cz=128), {}),
+    "long16384": (IpaDims(B=1, L=16384, H=12, Cz=128), {}),
+    "batched": (IpaDims(B=32, L=128, H=8, Cz=64), {"ragged": (64, 128), "jitter": 1.0}),
+}
+
+
+def ipa_preset(name: str, seed: int = 0) -> dict:
+    dims, kw = IPA_PRESETS[name]
+    return ipa_inputs(dims, seed, **kw)
+
+
+GEO_PRESET = GeoDims(B=2, N=2048, H=8, M=4, Cout=256)
+
+
+def geo_preset(seed: int = 0, **kw) -> dict:
+    return geo_inputs(GEO_PRESET, seed, **kw)
