@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Throughput of the fused Invariant Point Attention core on B200.
+
+One step = one pass of the whole hot path over one batch element of the
+long-context workload (L = 4096 residues, 12 heads, 16 scalar channels,
+4 query / 8 value points, rank-2 x 128-channel factorised pair
+representation): frames applied and augmented operands built (prologue), then
+the fused attention pass (core).  Metric: algorithmic TFLOP/s of the fused
+core, 2 L^2 H (Dqk + Dv) flops per batch element with Dqk = C + 3 Pq + 1 + R Cz
+and Dv = C + 3 Pv + R Cz.
+
+Launch: `python bench.py --gpus N --steps K --warmup W` (N > 1 under
+torchrun; every rank runs its own batch element -- weak scaling, no
+collective on the data path).  Rank 0 prints one JSON line.
+`--impl reference` times the float64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from rna_structure_models_b200.synth import GeoDims, IpaDims, geo_inputs, ipa_inputs  # noqa: E402
+
+H, C, PQ, PV, R, CZ = 12, 16, 4, 8, 2, 128
+METRIC = "fused IPA attention TFLOP/s and % bf16 tensor-pipe peak at L=4096 (1xB200)"
+UNIT = "TFLOP/s"
+
+# DRAM traffic of one launch of the core kernel from an ncu capture, valid only
+# for the kernel source it was taken on (sha256 of csrc/ipa_kernels.cu).
+NCU_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None}
+
+
+def ipa_flops(B, L, n_valid=None):
+    """Algorithmic flops of the fused core (2 per multiply-add)."""
+    dqk = C + 3 * PQ + 1 + R * CZ
+    dv = C + 3 * PV + R * CZ
+    pairs = B * L * L if n_valid is None else float(np.sum(np.asarray(n_valid, float) ** 2))
+    return 2.0 * pairs * H * (dqk + dv)
+
+
+def kernel_sha():
+    p = os.path.join(ROOT, "rna_structure_models_b200", "csrc", "ipa_kernels.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x2: "applications_clocks_setting", 0x1: "gpu_idle",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+            self.ok = True
+        except Exception:  # noqa: BLE001 -- clocks are reported as unavailable
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def cpu_oracle_sample(L, seconds, max_rows, seed=0, inp=None):
+    """Time the float64 oracle on query-row blocks of the same workload
+    (input generation is outside the timed part)."""
+    from oracle import ipa_dense
+    if inp is None:
+        inp = ipa_inputs(IpaDims(B=1, L=L, H=H, C=C, Pq=PQ, Pv=PV, R=R, Cz=CZ), seed)
+    rows_done, t_total = 0, 0.0
+    while rows_done < max_rows and t_total < seconds:
+        rows = np.arange(rows_done, min(rows_done + 64, L, max_rows))
+        t0 = time.perf_counter()
+        ipa_dense(inp, rows=rows)
+        t_total += time.perf_counter() - t0
+        rows_done += len(rows)
+    flops = 2.0 * rows_done * L * H * (C + 3 * PQ + 1 + R * CZ + C + 3 * PV + R * CZ)
+    return flops / t_total / 1e12, rows_done, t_total
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    L = args.L
+    ms = []
+    rows_per_step = args.ref_rows
+    inp = ipa_inputs(IpaDims(B=1, L=L, H=H, C=C, Pq=PQ, Pv=PV, R=R, Cz=CZ), 0)
+    for s in range(args.warmup + args.steps):
+        _, nrows, dt = cpu_oracle_sample(L, 1e9, rows_per_step, inp=inp)
+        if s >= args.warmup:
+            ms.append(dt * 1e3)
+    flops_step = 2.0 * rows_per_step * L * H * (C + 3 * PQ + 1 + R * CZ + C + 3 * PV + R * CZ)
+    value = flops_step * len(ms) / (sum(ms) / 1e3) / 1e12
+    sample = f"{rows_per_step} query rows x all {L} keys x {H} heads of the L={L} workload per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(ms),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"IPA core B=1 L={L} H={H} C={C} Pq={PQ} Pv={PV} R={R} Cz={CZ}",
+                       "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--L", type=int, default=4096)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variant", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--core-only", action="store_true", help="profiling aid: time only, print nothing else")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from rna_structure_models_b200 import api
+
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    L = args.L
+    dims = IpaDims(B=1, L=L, H=H, C=C, Pq=PQ, Pv=PV, R=R, Cz=CZ)
+    inp = ipa_inputs(dims, seed=rank)                      # each rank its own batch element
+    names = api.IPA_INPUTS
+    host = {n: torch.from_numpy(inp[n]) for n in names}
+    dvc = {n: host[n].to(dev) for n in names}
+    plan = api.IpaPlan(1, L, H, C, PQ, PV, R, CZ, device=dev)
+    out = torch.empty((1, L, H, plan.F), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    args_in = [dvc[n] for n in names]
+
+    def step():
+        plan.prologue(*args_in)
+        plan.core(out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    plan.check()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        for k in range(K):
+            flush.zero_()                                  # L2 flushed between steps (untimed)
+            ev[k][0].record()
+            plan.prologue(*args_in)
+            ev[k][1].record()
+            plan.core(out)
+            ev[k][2].record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    plan.check()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    core_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    pro_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    if args.core_only:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    flops = ipa_flops(1, L)
+    value = world * flops * K / (total_ms / 1e3) / 1e12
+    peaks, peak_kind = measured_peaks()
+    core_mean = statistics.mean(core_ms)
+    achieved = flops / (core_mean / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])        # fp16 and bf16 share the dense tensor rate
+    traffic = NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["kernel_sha256"] == kernel_sha() else None
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": f"IPA core B=1 L={L} H={H} C={C} Pq={PQ} Pv={PV} R={R} Cz={CZ} per GPU",
+                   "global_batch": world, "seq_len": L, "parallelism": f"dp{world}",
+                   "l2": "flushed between steps (256 MB write, untimed)",
+                   "step": "prologue (frames, augmented fp16 operands) + fused attention core"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "ipa_attention_kernel",
+                     "peak_source": f"{peak_kind} bf16 dense (burst); fp16 has the same nominal rate",
+                     "core_ms": core_mean, "prologue_ms": statistics.mean(pro_ms),
+                     "issued_frac": achieved * 640.0 / 581.0 / peak},
+        "gpu_launches": 3 * K,
+        "clocks": clk.summary(),
+    }
+
+    # end to end through the public API with host buffers
+    if not args.no_e2e:
+        pinned = {n: host[n].pin_memory() for n in names}
+        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+        res = torch.empty((1, L, H, plan.F), dtype=torch.float32, pin_memory=True)
+        d2h = res.numel() * res.element_size()
+        for _ in range(max(1, min(args.warmup, 3))):
+            o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev)
+        torch.cuda.synchronize()
+        ke = max(3, min(K, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(ke):
+            o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev)
+        e1.record()
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        line["e2e"] = {"value": world * flops * ke / (float(te.item()) / 1e3) / 1e12, "unit": UNIT,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
+                       "ms_per_step": float(te.item()) / ke}
+
+    # second hot-path row: direction/distance geometric attention (B=2, N=2048)
+    if not args.no_variant and rank == 0:
+        g = geo_inputs(GeoDims(B=2, N=2048, H=8, M=4, Cout=256), 0)
+        gd = {k: (torch.from_numpy(v).to(dev) if isinstance(v, np.ndarray) else None) for k, v in g.items()
+              if k != "dims"}
+        gp = api.GeoPlan(2, 2048, 8, 4, 256, device=dev)
+        outs = {"vectors": torch.empty((2, 2048, 8, 4, 3), device=dev),
+                "output": torch.empty((2, 2048, 256), device=dev),
+                "attention": torch.empty((2, 8, 2048, 2048), device=dev)}
+        res = {}
+        for with_att in (False, True):
+            o2 = dict(outs)
+            if not with_att:
+                o2["attention"] = None
+            for _ in range(3):
+                gp(gd, out=o2)
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(20):
+                flush.zero_()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record()
+                gp(gd, out=o2)
+                a1.record()
+                torch.cuda.synchronize()
+                times.append(a0.elapsed_time(a1))
+            res[with_att] = statistics.mean(times)
+        gp.check()
+        pairs = 2 * 8 * 2048 * 2048
+        att_bytes = pairs * 4 + pairs * 1          # attention map written + pair mask read
+        line["variant"] = {
+            "workload": "geometric attention B=2 N=2048 H=8 M=4 Cout=256, 20% pair mask, 5% invalid frames",
+            "ms_no_attention_map": res[False], "ms_with_attention_map": res[True],
+            "pair_heads_per_s": pairs / (res[False] / 1e3),
+            "attention_map_GBps": att_bytes / ((res[True] - res[False]) / 1e3) / 1e9
+            if res[True] > res[False] else None,
+        }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, nrows, secs = cpu_oracle_sample(L, args.cpu_seconds, 4096)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": f"{nrows} query rows x {L} keys x {H} heads of the same workload, "
+                                          f"{secs:.1f} s of numpy float64 (single-threaded einsum)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,212 @@
+/*
+ * flashipa_b200.h -- C ABI of the B200 (sm_100a) fused Invariant Point
+ * Attention core and of the geometric direction/distance attention variant.
+ *
+ * Every buffer is owned by the caller.  The library never allocates or frees
+ * device memory and never writes to an input.  Work is enqueued on the
+ * caller's CUDA stream; a return of IPA_OK means "validated and launched".
+ * Argument errors are returned before anything is launched; errors that can
+ * only be seen on the device (a bounded wait that ran out) are written, first
+ * one wins, into the optional device word `dev_err` (0 = no error), which the
+ * caller reads after synchronising the stream.  No C++ exception crosses this
+ * boundary.
+ *
+ * Tensors are passed as ipa_tensor_t: a device pointer, a dtype code, and the
+ * logical sizes and element strides of every dimension (stride 0 expresses a
+ * broadcast where that is allowed).  Inputs may be non-contiguous; outputs
+ * must be contiguous.
+ */
+#ifndef FLASHIPA_B200_H_
+#define FLASHIPA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define IPA_API __attribute__((visibility("default")))
+#else
+#define IPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  IPA_OK = 0,
+  IPA_ERR_NULL = 1,         /* a required pointer is NULL                       */
+  IPA_ERR_SHAPE = 2,        /* sizes disagree with the params or are < 1        */
+  IPA_ERR_STRIDE_ALIGN = 3, /* negative stride, non-contiguous output, or a
+                               misaligned pointer                               */
+  IPA_ERR_DTYPE = 4,        /* wrong element type                               */
+  IPA_ERR_WORKSPACE = 5,    /* workspace too small or not 256-byte aligned      */
+  IPA_ERR_UNSUPPORTED = 6,  /* dims outside the supported envelope (below)      */
+  IPA_ERR_CUDA = 7,         /* a CUDA runtime call failed (launch, attribute)   */
+  IPA_ERR_TIMEOUT = 8       /* device: a bounded wait ran out (in dev_err only) */
+} ipa_status_t;
+
+/* Element type codes. */
+enum {
+  IPA_DTYPE_F32 = 0,
+  IPA_DTYPE_F64 = 1,
+  IPA_DTYPE_BOOL = 2, /* one byte per element, 0 = false */
+  IPA_DTYPE_F16 = 3
+};
+
+#define IPA_MAX_DIMS 6
+
+typedef struct {
+  const void* data;              /* device pointer                            */
+  int32_t dtype;                 /* IPA_DTYPE_*                               */
+  int32_t ndim;                  /* number of dimensions used                 */
+  int64_t size[IPA_MAX_DIMS];    /* logical sizes                             */
+  int64_t stride[IPA_MAX_DIMS];  /* strides in ELEMENTS (not bytes), >= 0     */
+} ipa_tensor_t;
+
+/* --------------------------------------------------------------------------
+ * Fused IPA core.
+ *
+ * Operation (Flash Invariant Point Attention, TL;DR and Abstract: IPA with
+ * the factorised pair representation z_ij = sum_r z1_i[r] * z2_j[r]; MEET,
+ * section 2.2 eq. (7)-(8) for the squared distance folded into augmented
+ * query/key columns).  For batch b, query residue i, key residue j, head h:
+ *   gq = R_i q_pts + t_i, gk = R_j k_pts + t_j, gv = R_j v_pts + t_j
+ *   logit = w_L * ( scalar_scale * q.k
+ *                   + sum_{r,c} w_bias[c,h] z1_i[r,c] z2_j[r,c]
+ *                   - gamma_h * w_C / 2 * sum_p |gq_p - gk_p|^2 )
+ *   a = softmax over keys j with mask_i && mask_j (no allowed key -> a = 0)
+ *   out[b,i,h,:] = [ sum_j a v_j                      (C)
+ *                  | R_i^T (sum_j a gv_j - t_i)       (Pv x 3, xyz inner)
+ *                  | norms of those Pv points         (Pv)
+ *                  | sum_r z1_i[r,:] * sum_j a z2_j[r,:] (Cz) ]
+ *   and every feature is 0 for a row with no allowed key.
+ * The L x L logits and the pair tensor are never materialised.
+ *
+ * Shapes (all float inputs IPA_DTYPE_F32, any non-negative strides):
+ *   q, k, v          [B, L, H, C]
+ *   q_pts, k_pts     [B, L, H, Pq, 3]
+ *   v_pts            [B, L, H, Pv, 3]
+ *   rot              [B, L, 3, 3]   rot[b,i] maps local column vectors to global
+ *   trans            [B, L, 3]
+ *   z1, z2           [B, L, R, Cz]
+ *   w_bias           [Cz, H]
+ *   gamma            [H]            already positive (e.g. softplus of a weight)
+ *   mask             [B, L]         IPA_DTYPE_BOOL
+ *   out              [B, L, H, C + 4 Pv + Cz], IPA_DTYPE_F32, contiguous
+ * Supported envelope: C == 16, Pq == 4, Pv == 8 (the AlphaFold-2 IPA head
+ * shape), 1 <= R * Cz <= 256 with Cz a multiple of 16, 1 <= L <= 1048576.
+ * Arithmetic: fp16 tensor-core operands with fp32 accumulation; point
+ * coordinates, key norms and value points carry a second fp16 term for the
+ * rounding residue.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t B, L, H, C, Pq, Pv, R, Cz;
+  float w_L;          /* weight of the whole logit, sqrt(1/3) in AlphaFold-2 */
+  float w_C;          /* point weight, sqrt(2 / (9 Pq)) in AlphaFold-2       */
+  float scalar_scale; /* 1 / sqrt(C) in AlphaFold-2                          */
+} ipa_params_t;
+
+/* Bytes of device workspace ipa_attn_fwd needs for these params (0 if the
+ * params are invalid).  Pure host function. */
+IPA_API size_t ipa_attn_workspace_size(const ipa_params_t* p);
+
+/* Enqueue the fused IPA core on `stream` (a cudaStream_t, NULL = legacy
+ * default stream).  workspace: device memory of at least
+ * ipa_attn_workspace_size(p) bytes, 256-byte aligned, not shared with a
+ * concurrent call.  dev_err: optional device int (NULL allowed). */
+IPA_API ipa_status_t ipa_attn_fwd(const ipa_params_t* p,
+                          const ipa_tensor_t* q, const ipa_tensor_t* k, const ipa_tensor_t* v,
+                          const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                          const ipa_tensor_t* v_pts,
+                          const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                          const ipa_tensor_t* z1, const ipa_tensor_t* z2,
+                          const ipa_tensor_t* w_bias, const ipa_tensor_t* gamma,
+                          const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                          void* workspace, size_t workspace_bytes,
+                          void* stream, int32_t* dev_err);
+
+/* The two stages of ipa_attn_fwd, callable separately (same arguments and
+ * rules).  ipa_attn_prologue applies the frames and writes the augmented
+ * fp16 operands into the workspace; ipa_attn_core runs the fused attention
+ * pass from that workspace into `out`.  The core reads only the workspace,
+ * so it must follow a prologue with the same params and workspace on the
+ * same stream.  ipa_attn_fwd == prologue then core. */
+IPA_API ipa_status_t ipa_attn_prologue(const ipa_params_t* p,
+                               const ipa_tensor_t* q, const ipa_tensor_t* k, const ipa_tensor_t* v,
+                               const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                               const ipa_tensor_t* v_pts,
+                               const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                               const ipa_tensor_t* z1, const ipa_tensor_t* z2,
+                               const ipa_tensor_t* w_bias, const ipa_tensor_t* gamma,
+                               const ipa_tensor_t* mask,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream, int32_t* dev_err);
+IPA_API ipa_status_t ipa_attn_core(const ipa_params_t* p, const ipa_tensor_t* out,
+                           void* workspace, size_t workspace_bytes,
+                           void* stream, int32_t* dev_err);
+
+/* --------------------------------------------------------------------------
+ * Geometric direction-and-distance attention ("Geometric direction-and-
+ * distance attention", Required behavior).  For query i, key j, head h:
+ *   qd = R_i q_direction_i, kd = R_j k_direction_j,
+ *   qp = R_i q_point_i + t_i, kp = R_j k_point_j + t_j
+ *   s = (softplus(direction_scale_h) qd.kd - softplus(distance_scale_h) |qp - kp|) / sqrt(3)
+ *   (unsquared distance, no epsilon; softplus evaluated stably)
+ *   allowed = frame_mask_i && frame_mask_j && pair_mask[b,h,i,j]
+ *   attention = masked softmax over j (a head row with no allowed key is 0)
+ *   vectors_i = R_i^T sum_j attention_ij (R_j values_j)   (no translation)
+ *   output_i = flatten(vectors_i in H, M, xyz order) . output_weight (+ output_bias),
+ *              forced to 0 when no head of query i has an allowed key.
+ *
+ * Shapes (float inputs IPA_DTYPE_F32 or IPA_DTYPE_F64, all the same; the
+ * kernels compute in fp32; any non-negative strides):
+ *   q_direction, k_direction, q_point, k_point [B, N, H, 3]
+ *   values            [B, N, H, M, 3]
+ *   direction_scale, distance_scale [H]   unconstrained logits
+ *   output_weight     [H*M*3, Cout]
+ *   output_bias       [Cout] or data == NULL (no bias)
+ *   rotation          [B, N, 3, 3]; translation [B, N, 3]
+ *   frame_mask        [B, N] IPA_DTYPE_BOOL
+ *   pair_mask         [B, H, N, N] IPA_DTYPE_BOOL, broadcast by stride 0, or
+ *                     NULL / data == NULL (all pairs allowed)
+ * Outputs (IPA_DTYPE_F32, contiguous):
+ *   out_vectors       [B, N, H, M, 3]
+ *   out_output        [B, N, Cout]
+ *   out_attention     [B, H, N, N] or NULL / data == NULL (not written)
+ * Supported envelope: H*M*3 <= 384, N <= 1048576.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t B, N, H, M, Cout;
+} geo_params_t;
+
+IPA_API size_t geo_attn_workspace_size(const geo_params_t* p);
+
+IPA_API ipa_status_t geo_attn_fwd(const geo_params_t* p,
+                          const ipa_tensor_t* q_direction, const ipa_tensor_t* k_direction,
+                          const ipa_tensor_t* q_point, const ipa_tensor_t* k_point,
+                          const ipa_tensor_t* values,
+                          const ipa_tensor_t* direction_scale,
+                          const ipa_tensor_t* distance_scale,
+                          const ipa_tensor_t* output_weight, const ipa_tensor_t* output_bias,
+                          const ipa_tensor_t* rotation, const ipa_tensor_t* translation,
+                          const ipa_tensor_t* frame_mask, const ipa_tensor_t* pair_mask,
+                          const ipa_tensor_t* out_vectors, const ipa_tensor_t* out_output,
+                          const ipa_tensor_t* out_attention,
+                          void* workspace, size_t workspace_bytes,
+                          void* stream, int32_t* dev_err);
+
+/* Static description of a status code (never NULL). */
+IPA_API const char* ipa_status_string(ipa_status_t s);
+
+/* Translate a device error word written by the kernels into a status:
+ * 0 -> IPA_OK, bounded-wait expiry -> IPA_ERR_TIMEOUT, else IPA_ERR_CUDA. */
+IPA_API ipa_status_t ipa_device_error_status(int32_t dev_err_value);
+
+/* Library build identifier, e.g. "flashipa_b200 sm_100a". */
+IPA_API const char* ipa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHIPA_B200_H_ */

@@ -1,0 +1,294 @@
+"""Python binding of the C ABI in include/flashipa_b200.h.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch provides device memory and streams.  The library must be
+built (`python -m rna_structure_models_b200.build`); if it is missing, the
+first call raises -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libflashipa_b200.so")
+
+IPA_DTYPE_F32, IPA_DTYPE_F64, IPA_DTYPE_BOOL, IPA_DTYPE_F16 = 0, 1, 2, 3
+STATUS = {0: "IPA_OK", 1: "IPA_ERR_NULL", 2: "IPA_ERR_SHAPE", 3: "IPA_ERR_STRIDE_ALIGN",
+          4: "IPA_ERR_DTYPE", 5: "IPA_ERR_WORKSPACE", 6: "IPA_ERR_UNSUPPORTED", 7: "IPA_ERR_CUDA",
+          8: "IPA_ERR_TIMEOUT"}
+EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa_attn_core",
+            "geo_attn_workspace_size", "geo_attn_fwd", "ipa_status_string",
+            "ipa_device_error_status", "ipa_version")
+
+
+class IpaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("size", ctypes.c_int64 * 6), ("stride", ctypes.c_int64 * 6)]
+
+
+class IpaParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("C", ctypes.c_int32), ("Pq", ctypes.c_int32), ("Pv", ctypes.c_int32),
+                ("R", ctypes.c_int32), ("Cz", ctypes.c_int32), ("w_L", ctypes.c_float),
+                ("w_C", ctypes.c_float), ("scalar_scale", ctypes.c_float)]
+
+
+class GeoParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("M", ctypes.c_int32), ("Cout", ctypes.c_int32)]
+
+
+class IpaError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{STATUS.get(code, code)}{': ' + what if what else ''}")
+
+
+_lib = None
+
+
+def library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} not found: build it with `python -m rna_structure_models_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER
+    T = P(IpaTensor)
+    lib.ipa_attn_workspace_size.argtypes = [P(IpaParams)]
+    lib.ipa_attn_workspace_size.restype = ctypes.c_size_t
+    lib.ipa_attn_fwd.argtypes = [P(IpaParams)] + [T] * 14 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                            ctypes.c_void_p, ctypes.c_void_p]
+    lib.ipa_attn_fwd.restype = ctypes.c_int
+    lib.ipa_attn_prologue.argtypes = [P(IpaParams)] + [T] * 13 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                                 ctypes.c_void_p, ctypes.c_void_p]
+    lib.ipa_attn_prologue.restype = ctypes.c_int
+    lib.ipa_attn_core.argtypes = [P(IpaParams), T, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                  ctypes.c_void_p]
+    lib.ipa_attn_core.restype = ctypes.c_int
+    lib.geo_attn_workspace_size.argtypes = [P(GeoParams)]
+    lib.geo_attn_workspace_size.restype = ctypes.c_size_t
+    lib.geo_attn_fwd.argtypes = [P(GeoParams)] + [T] * 16 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                            ctypes.c_void_p, ctypes.c_void_p]
+    lib.geo_attn_fwd.restype = ctypes.c_int
+    lib.ipa_status_string.argtypes = [ctypes.c_int]
+    lib.ipa_status_string.restype = ctypes.c_char_p
+    lib.ipa_device_error_status.argtypes = [ctypes.c_int32]
+    lib.ipa_device_error_status.restype = ctypes.c_int
+    lib.ipa_version.argtypes = []
+    lib.ipa_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+_DT = {torch.float32: IPA_DTYPE_F32, torch.float64: IPA_DTYPE_F64, torch.bool: IPA_DTYPE_BOOL,
+       torch.uint8: IPA_DTYPE_BOOL, torch.float16: IPA_DTYPE_F16}
+
+
+def tensor_desc(t: Optional[torch.Tensor]) -> IpaTensor:
+    """Describe a torch tensor (no copy; strides in elements)."""
+    d = IpaTensor()
+    if t is None:
+        d.data = None
+        return d
+    if t.dim() > 6:
+        raise ValueError("at most 6 dimensions")
+    d.data = t.data_ptr() if t.numel() > 0 else None
+    d.dtype = _DT.get(t.dtype, -1)
+    d.ndim = t.dim()
+    for i, (s, st) in enumerate(zip(t.shape, t.stride())):
+        d.size[i] = s
+        d.stride[i] = st
+    return d
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors (use ipa_attn_host for host buffers)")
+
+
+def ipa_defaults(C: int, Pq: int) -> dict:
+    """AlphaFold-2 IPA logit weights."""
+    return {"w_L": math.sqrt(1.0 / 3.0), "w_C": math.sqrt(2.0 / (9.0 * Pq)),
+            "scalar_scale": 1.0 / math.sqrt(C)}
+
+
+def ipa_params(B, L, H, C, Pq, Pv, R, Cz, w_L=None, w_C=None, scalar_scale=None) -> IpaParams:
+    d = ipa_defaults(C, Pq)
+    return IpaParams(B, L, H, C, Pq, Pv, R, Cz,
+                     d["w_L"] if w_L is None else w_L,
+                     d["w_C"] if w_C is None else w_C,
+                     d["scalar_scale"] if scalar_scale is None else scalar_scale)
+
+
+def ipa_workspace_bytes(p: IpaParams) -> int:
+    return int(library().ipa_attn_workspace_size(ctypes.byref(p)))
+
+
+class IpaPlan:
+    """Reusable launch state for one problem shape: params, workspace and a
+    device error word allocated once (by torch), so repeated calls allocate
+    nothing."""
+
+    def __init__(self, B, L, H, C=16, Pq=4, Pv=8, R=2, Cz=128, device="cuda", **consts):
+        self.params = ipa_params(B, L, H, C, Pq, Pv, R, Cz, **consts)
+        nbytes = ipa_workspace_bytes(self.params)
+        if nbytes == 0:
+            raise IpaError(6, "dimensions outside the supported envelope")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.F = C + 4 * Pv + Cz
+
+    def __call__(self, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask,
+                 out=None, stream=None):
+        p = self.params
+        _require_cuda(q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask)
+        if out is None:
+            out = torch.empty((p.B, p.L, p.H, self.F), dtype=torch.float32, device=q.device)
+        descs = [tensor_desc(t) for t in (q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2,
+                                          w_bias, gamma, mask, out)]
+        st = library().ipa_attn_fwd(ctypes.byref(p), *[ctypes.byref(d) for d in descs],
+                                    ctypes.c_void_p(self.workspace.data_ptr()),
+                                    ctypes.c_size_t(self.workspace.numel()),
+                                    ctypes.c_void_p(_stream_ptr(stream)),
+                                    ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return out
+
+    def prologue(self, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask,
+                 stream=None):
+        """Stage 1 only: frames applied, augmented operands written to the workspace."""
+        p = self.params
+        _require_cuda(q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask)
+        descs = [tensor_desc(t) for t in (q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2,
+                                          w_bias, gamma, mask)]
+        st = library().ipa_attn_prologue(ctypes.byref(p), *[ctypes.byref(d) for d in descs],
+                                         ctypes.c_void_p(self.workspace.data_ptr()),
+                                         ctypes.c_size_t(self.workspace.numel()),
+                                         ctypes.c_void_p(_stream_ptr(stream)),
+                                         ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+
+    def core(self, out, stream=None):
+        """Stage 2 only: the fused attention pass from the workspace into `out`."""
+        d = tensor_desc(out)
+        st = library().ipa_attn_core(ctypes.byref(self.params), ctypes.byref(d),
+                                     ctypes.c_void_p(self.workspace.data_ptr()),
+                                     ctypes.c_size_t(self.workspace.numel()),
+                                     ctypes.c_void_p(_stream_ptr(stream)),
+                                     ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return out
+
+    def check(self):
+        """Synchronise and raise if a kernel reported a device-side error."""
+        v = int(self.dev_err.item())
+        if v != 0:
+            self.dev_err.zero_()
+            raise IpaError(int(library().ipa_device_error_status(v)), f"device error code {v}")
+
+
+IPA_INPUTS = ("q", "k", "v", "q_pts", "k_pts", "v_pts", "rot", "trans", "z1", "z2", "w_bias",
+              "gamma", "mask")
+
+
+def ipa_attn(inp: dict, *, out=None, stream=None, check: bool = True, **consts):
+    """Fused IPA core on CUDA tensors given in a dict keyed like IPA_INPUTS."""
+    q = inp["q"]
+    B, L, H, C = q.shape
+    Pq, Pv = inp["q_pts"].shape[3], inp["v_pts"].shape[3]
+    R, Cz = inp["z1"].shape[2], inp["z1"].shape[3]
+    plan = IpaPlan(B, L, H, C, Pq, Pv, R, Cz, device=q.device, **consts)
+    res = plan(*[inp[n] for n in IPA_INPUTS], out=out, stream=stream)
+    if check:
+        plan.check()
+    return res
+
+
+def ipa_attn_host(inp: dict, plan: Optional[IpaPlan] = None, device="cuda", stream=None):
+    """End-to-end call on HOST tensors: copies the inputs to the device (from
+    pinned memory when they are pinned), runs the fused core, copies the
+    result back into a pinned host tensor.  Returns (out_host, plan)."""
+    q = inp["q"]
+    B, L, H, C = q.shape
+    if plan is None:
+        plan = IpaPlan(B, L, H, C, inp["q_pts"].shape[3], inp["v_pts"].shape[3],
+                       inp["z1"].shape[2], inp["z1"].shape[3], device=device)
+    dev = {n: inp[n].to(device, non_blocking=True) for n in IPA_INPUTS}
+    out = plan(*[dev[n] for n in IPA_INPUTS], stream=stream)
+    host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    host.copy_(out, non_blocking=True)
+    return host, plan
+
+
+# ------------------------------------------------------------------ variant
+GEO_INPUTS = ("q_direction", "k_direction", "q_point", "k_point", "values", "direction_scale",
+              "distance_scale", "output_weight", "output_bias", "rotation", "translation",
+              "frame_mask", "pair_mask")
+
+
+class GeoPlan:
+    def __init__(self, B, N, H, M, Cout, device="cuda"):
+        self.params = GeoParams(B, N, H, M, Cout)
+        nbytes = int(library().geo_attn_workspace_size(ctypes.byref(self.params)))
+        if nbytes == 0:
+            raise IpaError(6, "dimensions outside the supported envelope")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def __call__(self, inp: dict, *, with_attention: bool = True, out: Optional[dict] = None, stream=None):
+        p = self.params
+        dev = inp["q_direction"].device
+        _require_cuda(*[inp.get(n) for n in GEO_INPUTS])
+        if out is None:
+            out = {"vectors": torch.empty((p.B, p.N, p.H, p.M, 3), dtype=torch.float32, device=dev),
+                   "output": torch.empty((p.B, p.N, p.Cout), dtype=torch.float32, device=dev),
+                   "attention": (torch.empty((p.B, p.H, p.N, p.N), dtype=torch.float32, device=dev)
+                                 if with_attention else None)}
+        pm = inp.get("pair_mask")
+        if pm is not None and pm.dim() == 4 and tuple(pm.shape) != (p.B, p.H, p.N, p.N):
+            pm = pm.expand(p.B, p.H, p.N, p.N)
+        descs = [tensor_desc(inp.get(n)) for n in GEO_INPUTS[:-1]] + [tensor_desc(pm)]
+        descs += [tensor_desc(out["vectors"]), tensor_desc(out["output"]), tensor_desc(out.get("attention"))]
+        st = library().geo_attn_fwd(ctypes.byref(p), *[ctypes.byref(d) for d in descs],
+                                    ctypes.c_void_p(self.workspace.data_ptr()),
+                                    ctypes.c_size_t(self.workspace.numel()),
+                                    ctypes.c_void_p(_stream_ptr(stream)),
+                                    ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return out
+
+    def check(self):
+        v = int(self.dev_err.item())
+        if v != 0:
+            self.dev_err.zero_()
+            raise IpaError(int(library().ipa_device_error_status(v)), f"device error code {v}")
+
+
+def geo_attn(inp: dict, *, with_attention: bool = True, stream=None, check: bool = True):
+    B, N, H, _ = inp["q_direction"].shape
+    M = inp["values"].shape[3]
+    Cout = inp["output_weight"].shape[1]
+    plan = GeoPlan(B, N, H, M, Cout, device=inp["q_direction"].device)
+    res = plan(inp, with_attention=with_attention, stream=stream)
+    if check:
+        plan.check()
+    return res

@@ -1,0 +1,67 @@
+"""Build the sm_100a C-ABI library (and the test-only probe library) in tree
+with nvcc.  `python -m rna_structure_models_b200.build` or build_all()."""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libflashipa_b200.so")
+PROBE_SRC = os.path.join(ROOT, "tests", "csrc", "umma_probe.cu")
+PROBE_LIB = os.path.join(ROOT, "tests", "libflashipa_probe.so")
+
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
+         "--expt-relaxed-constexpr", "-Xcompiler", "-fvisibility=hidden"]
+SOURCES = ["api.cu", "ipa_kernels.cu", "geo_kernels.cu"]
+
+
+def nvcc() -> str:
+    exe = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(exe):
+        raise RuntimeError("nvcc not found")
+    return exe
+
+
+def _run(cmd, verbose):
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
+    return r.stdout + r.stderr
+
+
+def build_lib(verbose: bool = False, ptxas_info: bool = False) -> str:
+    srcs = [os.path.join(CSRC, s) for s in SOURCES]
+    cmd = [nvcc(), *ARCH, *FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", "-Xcompiler",
+           "-DFLASHIPA_EXPORTS", *srcs, "-o", LIB]
+    if ptxas_info:
+        cmd.insert(1, "-Xptxas=-v")
+    out = _run(cmd, verbose)
+    if ptxas_info:
+        print(out)
+    return LIB
+
+
+def build_probe(verbose: bool = False) -> str:
+    cmd = [nvcc(), *ARCH, *FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", PROBE_SRC, "-o", PROBE_LIB]
+    _run(cmd, verbose)
+    return PROBE_LIB
+
+
+def build_all(verbose: bool = False) -> None:
+    build_lib(verbose)
+    if os.path.exists(PROBE_SRC):
+        build_probe(verbose)
+
+
+if __name__ == "__main__":
+    build_all(verbose=True)
+    if "--ptxas" in sys.argv:
+        build_lib(ptxas_info=True)

@@ -1,0 +1,340 @@
+// Host side of the C ABI declared in include/flashipa_b200.h: argument
+// validation, workspace carving, tensor-map encoding and launches.  No device
+// memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "flashipa_b200.h"
+#include "internal.h"
+
+namespace fipa {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool check_tensor(const ipa_tensor_t* t, int dtype, int ndim, const int64_t* sizes, ipa_status_t* st,
+                  bool allow_f64 = false) {
+  if (t == nullptr || t->data == nullptr) { *st = IPA_ERR_NULL; return false; }
+  if (!(t->dtype == dtype || (allow_f64 && t->dtype == IPA_DTYPE_F64))) { *st = IPA_ERR_DTYPE; return false; }
+  if (t->ndim != ndim) { *st = IPA_ERR_SHAPE; return false; }
+  for (int d = 0; d < ndim; ++d) {
+    if (t->size[d] != sizes[d] || sizes[d] < 1) { *st = IPA_ERR_SHAPE; return false; }
+    if (t->stride[d] < 0) { *st = IPA_ERR_STRIDE_ALIGN; return false; }
+  }
+  const int esz = t->dtype == IPA_DTYPE_F64 ? 8 : t->dtype == IPA_DTYPE_BOOL ? 1 : t->dtype == IPA_DTYPE_F16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(t->data) % esz != 0) { *st = IPA_ERR_STRIDE_ALIGN; return false; }
+  return true;
+}
+
+bool check_contiguous_out(const ipa_tensor_t* t, int ndim, const int64_t* sizes, ipa_status_t* st) {
+  if (!check_tensor(t, IPA_DTYPE_F32, ndim, sizes, st)) return false;
+  int64_t expect = 1;
+  for (int d = ndim - 1; d >= 0; --d) {
+    if (sizes[d] > 1 && t->stride[d] != expect) { *st = IPA_ERR_STRIDE_ALIGN; return false; }
+    expect *= sizes[d];
+  }
+  if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0) { *st = IPA_ERR_STRIDE_ALIGN; return false; }
+  return true;
+}
+
+View view_of(const ipa_tensor_t* t) {
+  View v{};
+  v.p = t ? t->data : nullptr;
+  for (int d = 0; d < 6; ++d) v.s[d] = (t && d < t->ndim) ? t->stride[d] : 0;
+  v.dtype = !t ? 0 : t->dtype == IPA_DTYPE_F64 ? 1 : t->dtype == IPA_DTYPE_BOOL ? 2 : 0;
+  return v;
+}
+
+bool ipa_dims_ok(const ipa_params_t* p, ipa_status_t* st) {
+  if (p == nullptr) { *st = IPA_ERR_NULL; return false; }
+  if (p->B < 1 || p->L < 1 || p->H < 1 || p->C < 1 || p->Pq < 1 || p->Pv < 1 || p->R < 1 || p->Cz < 1) {
+    *st = IPA_ERR_SHAPE;
+    return false;
+  }
+  if (p->C != IPA_C || p->Pq != IPA_PQ || p->Pv != IPA_PV || p->Cz % 16 != 0 ||
+      static_cast<int64_t>(p->R) * p->Cz > MAX_DZ || p->L > (1 << 20) ||
+      static_cast<int64_t>(p->B) * p->H * p->L > (int64_t{1} << 31) / 64) {
+    *st = IPA_ERR_UNSUPPORTED;
+    return false;
+  }
+  return true;
+}
+
+int pair_width(const ipa_params_t* p) { return ((p->R * p->Cz + 63) / 64) * 64; }
+
+bool geo_dims_ok(const geo_params_t* p, ipa_status_t* st) {
+  if (p == nullptr) { *st = IPA_ERR_NULL; return false; }
+  if (p->B < 1 || p->N < 1 || p->H < 1 || p->M < 1 || p->Cout < 1) { *st = IPA_ERR_SHAPE; return false; }
+  if (p->M > 8 || p->H * p->M * 3 > 384 || p->N > (1 << 20) || p->H > 65535 || p->B > 65535) {
+    *st = IPA_ERR_UNSUPPORTED;
+    return false;
+  }
+  return true;
+}
+
+}  // namespace
+
+bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace fipa
+
+using namespace fipa;
+
+extern "C" {
+
+const char* ipa_status_string(ipa_status_t s) {
+  switch (s) {
+    case IPA_OK: return "ok";
+    case IPA_ERR_NULL: return "null pointer";
+    case IPA_ERR_SHAPE: return "shape mismatch";
+    case IPA_ERR_STRIDE_ALIGN: return "bad stride or alignment";
+    case IPA_ERR_DTYPE: return "bad dtype";
+    case IPA_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case IPA_ERR_UNSUPPORTED: return "dimensions outside the supported envelope";
+    case IPA_ERR_CUDA: return "CUDA runtime error";
+    case IPA_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+ipa_status_t ipa_device_error_status(int32_t v) {
+  if (v == 0) return IPA_OK;
+  if (v >= 1 && v <= 5) return IPA_ERR_TIMEOUT;
+  return IPA_ERR_CUDA;
+}
+
+const char* ipa_version(void) { return "flashipa_b200 sm_100a 0.1"; }
+
+size_t ipa_attn_workspace_size(const ipa_params_t* p) {
+  ipa_status_t st;
+  if (!ipa_dims_ok(p, &st)) return 0;
+  return ipa_workspace_layout(p->B, p->L, p->H, pair_width(p), p->R * p->Cz).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Validation + launch description shared by the three IPA entry points.
+// inputs == false: only the params, `out` and the workspace are checked.
+ipa_status_t ipa_prepare(const ipa_params_t* p, const ipa_tensor_t* const* in, const ipa_tensor_t* out,
+                         void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err,
+                         bool inputs, bool reset_err, IpaLaunch* a) {
+  ipa_status_t st = IPA_OK;
+  if (!ipa_dims_ok(p, &st)) return st;
+  const int64_t B = p->B, L = p->L, H = p->H, C = p->C, Pq = p->Pq, Pv = p->Pv, R = p->R, Cz = p->Cz;
+  const int64_t F = C + 4 * Pv + Cz;
+  if (inputs) {
+    const int64_t s_qkv[4] = {B, L, H, C};
+    const int64_t s_qp[5] = {B, L, H, Pq, 3};
+    const int64_t s_vp[5] = {B, L, H, Pv, 3};
+    const int64_t s_rot[4] = {B, L, 3, 3};
+    const int64_t s_tr[3] = {B, L, 3};
+    const int64_t s_z[4] = {B, L, R, Cz};
+    const int64_t s_w[2] = {Cz, H};
+    const int64_t s_g[1] = {H};
+    const int64_t s_m[2] = {B, L};
+    const int64_t* shp[13] = {s_qkv, s_qkv, s_qkv, s_qp, s_qp, s_vp, s_rot, s_tr, s_z, s_z, s_w, s_g, s_m};
+    const int nd[13] = {4, 4, 4, 5, 5, 5, 4, 3, 4, 4, 2, 1, 2};
+    for (int t = 0; t < 13; ++t)
+      if (!check_tensor(in[t], t == 12 ? IPA_DTYPE_BOOL : IPA_DTYPE_F32, nd[t], shp[t], &st)) return st;
+  }
+  if (out != nullptr || !inputs) {
+    const int64_t s_o[4] = {B, L, H, F};
+    if (!check_contiguous_out(out, 4, s_o, &st)) return st;
+  }
+  const int DZ = pair_width(p);
+  const IpaWorkspace lay = ipa_workspace_layout(p->B, p->L, p->H, DZ, p->R * p->Cz);
+  if (workspace == nullptr) return IPA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
+
+  *a = IpaLaunch{};
+  a->B = p->B; a->L = p->L; a->H = p->H; a->C = p->C; a->Pq = p->Pq; a->Pv = p->Pv; a->R = p->R; a->Cz = p->Cz;
+  a->DZ = DZ; a->RCz = p->R * p->Cz; a->F = static_cast<int>(F);
+  a->nqt = (p->L + QT - 1) / QT; a->nkt = (p->L + KT - 1) / KT;
+  a->w_L = p->w_L; a->w_C = p->w_C; a->scalar_scale = p->scalar_scale;
+  if (inputs) {
+    View* vs[13] = {&a->q, &a->k, &a->v, &a->q_pts, &a->k_pts, &a->v_pts, &a->rot, &a->trans,
+                    &a->z1, &a->z2, &a->w_bias, &a->gamma, &a->mask};
+    for (int t = 0; t < 13; ++t) *vs[t] = view_of(in[t]);
+  }
+  a->out = out ? static_cast<float*>(const_cast<void*>(out->data)) : nullptr;
+  a->ws = static_cast<unsigned char*>(workspace);
+  a->lay = lay;
+  if (dev_err != nullptr) {
+    a->err = dev_err;
+  } else {
+    a->err = reinterpret_cast<int*>(a->ws + lay.err);
+    if (reset_err && cudaMemsetAsync(a->err, 0, sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return IPA_ERR_CUDA;
+  }
+  return IPA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ipa_status_t ipa_attn_prologue(const ipa_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,
+                               const ipa_tensor_t* v, const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                               const ipa_tensor_t* v_pts, const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                               const ipa_tensor_t* z1, const ipa_tensor_t* z2, const ipa_tensor_t* w_bias,
+                               const ipa_tensor_t* gamma, const ipa_tensor_t* mask, void* workspace,
+                               size_t workspace_bytes, void* stream, int32_t* dev_err) {
+  const ipa_tensor_t* in[13] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask};
+  IpaLaunch a;
+  const ipa_status_t st = ipa_prepare(p, in, nullptr, workspace, workspace_bytes, stream, dev_err, true, true, &a);
+  if (st != IPA_OK) return st;
+  return ipa_launch_prologue(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? IPA_OK : IPA_ERR_CUDA;
+}
+
+ipa_status_t ipa_attn_core(const ipa_params_t* p, const ipa_tensor_t* out, void* workspace,
+                           size_t workspace_bytes, void* stream, int32_t* dev_err) {
+  IpaLaunch a;
+  const ipa_status_t st = ipa_prepare(p, nullptr, out, workspace, workspace_bytes, stream, dev_err, false, false, &a);
+  if (st != IPA_OK) return st;
+  return ipa_launch_core(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? IPA_OK : IPA_ERR_CUDA;
+}
+
+ipa_status_t ipa_attn_fwd(const ipa_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,
+                          const ipa_tensor_t* v, const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                          const ipa_tensor_t* v_pts, const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                          const ipa_tensor_t* z1, const ipa_tensor_t* z2, const ipa_tensor_t* w_bias,
+                          const ipa_tensor_t* gamma, const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                          void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err) {
+  const ipa_tensor_t* in[13] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask};
+  IpaLaunch a;
+  if (out == nullptr) return IPA_ERR_NULL;
+  const ipa_status_t st = ipa_prepare(p, in, out, workspace, workspace_bytes, stream, dev_err, true, true, &a);
+  if (st != IPA_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ipa_launch_prologue(a, s) != cudaSuccess) return IPA_ERR_CUDA;
+  if (ipa_launch_core(a, s) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
+size_t geo_attn_workspace_size(const geo_params_t* p) {
+  ipa_status_t st;
+  if (!geo_dims_ok(p, &st)) return 0;
+  return geo_workspace_layout(p->B, p->N, p->H, p->M, p->Cout).total;
+}
+
+ipa_status_t geo_attn_fwd(const geo_params_t* p, const ipa_tensor_t* q_direction,
+                          const ipa_tensor_t* k_direction, const ipa_tensor_t* q_point,
+                          const ipa_tensor_t* k_point, const ipa_tensor_t* values,
+                          const ipa_tensor_t* direction_scale, const ipa_tensor_t* distance_scale,
+                          const ipa_tensor_t* output_weight, const ipa_tensor_t* output_bias,
+                          const ipa_tensor_t* rotation, const ipa_tensor_t* translation,
+                          const ipa_tensor_t* frame_mask, const ipa_tensor_t* pair_mask,
+                          const ipa_tensor_t* out_vectors, const ipa_tensor_t* out_output,
+                          const ipa_tensor_t* out_attention, void* workspace, size_t workspace_bytes,
+                          void* stream, int32_t* dev_err) {
+  ipa_status_t st = IPA_OK;
+  if (!geo_dims_ok(p, &st)) return st;
+  const int64_t B = p->B, N = p->N, H = p->H, M = p->M, Cout = p->Cout;
+  const int fdt = q_direction ? q_direction->dtype : IPA_DTYPE_F32;
+  if (fdt != IPA_DTYPE_F32 && fdt != IPA_DTYPE_F64) return q_direction ? IPA_ERR_DTYPE : IPA_ERR_NULL;
+  const bool has_bias = output_bias != nullptr && output_bias->data != nullptr;
+  const bool has_pm = pair_mask != nullptr && pair_mask->data != nullptr;
+  const bool has_att = out_attention != nullptr && out_attention->data != nullptr;
+  {
+    const int64_t s_v3[4] = {B, N, H, 3};
+    const int64_t s_val[5] = {B, N, H, M, 3};
+    const int64_t s_h[1] = {H};
+    const int64_t s_w[2] = {H * M * 3, Cout};
+    const int64_t s_b[1] = {Cout};
+    const int64_t s_rot[4] = {B, N, 3, 3};
+    const int64_t s_tr[3] = {B, N, 3};
+    const int64_t s_fm[2] = {B, N};
+    const int64_t s_pm[4] = {B, H, N, N};
+    const int64_t s_out[2] = {B * N, Cout};
+    const int64_t s_o3[3] = {B, N, Cout};
+    const int64_t s_att[4] = {B, H, N, N};
+    (void)s_out;
+    if (!check_tensor(q_direction, fdt, 4, s_v3, &st) || !check_tensor(k_direction, fdt, 4, s_v3, &st) ||
+        !check_tensor(q_point, fdt, 4, s_v3, &st) || !check_tensor(k_point, fdt, 4, s_v3, &st) ||
+        !check_tensor(values, fdt, 5, s_val, &st) || !check_tensor(direction_scale, fdt, 1, s_h, &st) ||
+        !check_tensor(distance_scale, fdt, 1, s_h, &st) || !check_tensor(output_weight, fdt, 2, s_w, &st) ||
+        (has_bias && !check_tensor(output_bias, fdt, 1, s_b, &st)) ||
+        !check_tensor(rotation, fdt, 4, s_rot, &st) || !check_tensor(translation, fdt, 3, s_tr, &st) ||
+        !check_tensor(frame_mask, IPA_DTYPE_BOOL, 2, s_fm, &st) ||
+        !check_contiguous_out(out_vectors, 5, s_val, &st) || !check_contiguous_out(out_output, 3, s_o3, &st) ||
+        (has_att && !check_contiguous_out(out_attention, 4, s_att, &st)))
+      return st;
+    if (has_pm) {
+      // broadcastable to [B, H, N, N]: each size equals the full size or is 1 (stride ignored then)
+      if (pair_mask->dtype != IPA_DTYPE_BOOL) return IPA_ERR_DTYPE;
+      if (pair_mask->ndim != 4) return IPA_ERR_SHAPE;
+      for (int d = 0; d < 4; ++d) {
+        if (pair_mask->size[d] != s_pm[d] && pair_mask->size[d] != 1) return IPA_ERR_SHAPE;
+        if (pair_mask->stride[d] < 0) return IPA_ERR_STRIDE_ALIGN;
+      }
+    }
+  }
+  const GeoWorkspace lay = geo_workspace_layout(p->B, p->N, p->H, p->M, p->Cout);
+  if (workspace == nullptr) return IPA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
+
+  GeoLaunch a{};
+  a.B = p->B; a.N = p->N; a.H = p->H; a.M = p->M; a.Cout = p->Cout; a.HM3 = p->H * p->M * 3;
+  a.q_direction = view_of(q_direction); a.k_direction = view_of(k_direction);
+  a.q_point = view_of(q_point); a.k_point = view_of(k_point); a.values = view_of(values);
+  a.direction_scale = view_of(direction_scale); a.distance_scale = view_of(distance_scale);
+  a.output_weight = view_of(output_weight); a.output_bias = view_of(has_bias ? output_bias : nullptr);
+  a.output_bias.dtype = has_bias ? a.output_bias.dtype : a.output_weight.dtype;
+  a.rotation = view_of(rotation); a.translation = view_of(translation); a.frame_mask = view_of(frame_mask);
+  a.pair_mask = view_of(has_pm ? pair_mask : nullptr);
+  if (has_pm)
+    for (int d = 0; d < 4; ++d)
+      if (pair_mask->size[d] == 1) a.pair_mask.s[d] = 0;  // broadcast dimension
+  a.has_bias = has_bias; a.has_pair_mask = has_pm;
+  a.out_vectors = static_cast<float*>(const_cast<void*>(out_vectors->data));
+  a.out_output = static_cast<float*>(const_cast<void*>(out_output->data));
+  a.out_attention = has_att ? static_cast<float*>(const_cast<void*>(out_attention->data)) : nullptr;
+  a.ws = static_cast<unsigned char*>(workspace);
+  a.lay = lay;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dev_err != nullptr) {
+    a.err = dev_err;
+  } else {
+    a.err = reinterpret_cast<int*>(a.ws + lay.err);
+    if (cudaMemsetAsync(a.err, 0, sizeof(int), s) != cudaSuccess) return IPA_ERR_CUDA;
+  }
+  if (geo_launch_all(a, s) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,477 @@
+// Geometric direction-and-distance attention for sm_100a ("Geometric
+// direction-and-distance attention", Required behavior).
+//
+// The score uses the UNSQUARED distance |qp_i - kp_j|, which does not
+// factorise into query and key columns, so the per-pair score is evaluated on
+// CUDA cores inside the key loop (fp32, MUFU sqrt / exp2).  Launches:
+//   1. geo_weights_kernel -- softplus scales per head, readout weight / bias
+//      converted to fp32.
+//   2. geo_prep_kernel    -- per (b, n, h): rotated directions, transformed
+//      points, R_j-rotated values (no translation), frame-mask bias.
+//   3. geo_attn_kernel<M> -- per (b, h, 128 queries) x 4 key splits: online
+//      masked softmax in the log2 domain and aggregation of the rotated
+//      values; splits merged through shared memory; R_i^T back-rotation.
+//   4. geo_map_kernel     -- optional: recomputes each score and writes the
+//      normalised attention row with coalesced stores.
+//   5. geo_readout_kernel -- output = flatten(vectors) . W (+ b), forced to
+//      zero for queries where no head has an allowed key.
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fipa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int GEO_ROWS = 128;
+constexpr int GEO_SPLIT = 4;
+constexpr int GEO_CHUNK = 32;
+
+__device__ __forceinline__ float ldf(const View& v, int64_t off) {
+  if (v.dtype == 1) return static_cast<float>(reinterpret_cast<const double*>(v.p)[off]);
+  return reinterpret_cast<const float*>(v.p)[off];
+}
+__device__ __forceinline__ bool ldb(const View& v, int64_t off) {
+  return reinterpret_cast<const unsigned char*>(v.p)[off] != 0;
+}
+
+// log(1 + exp(x)) without overflow: max(x, 0) + log1p(exp(-|x|))
+__device__ __forceinline__ float softplus_stable(float x) {
+  return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
+}
+
+struct WArgs {
+  int H, HM3, Cout;
+  bool has_bias;
+  View dscale, xscale, w, bias;
+  float2* sc;   // [H]: (log2e softplus(direction)/sqrt3, log2e softplus(distance)/sqrt3)
+  float* wf;    // [HM3, Cout]
+  float* bf;    // [Cout]
+};
+
+__global__ void geo_weights_kernel(const WArgs a) {
+  const int64_t n = static_cast<int64_t>(a.HM3) * a.Cout;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t < n) {
+    const int r = static_cast<int>(t / a.Cout), c = static_cast<int>(t % a.Cout);
+    a.wf[t] = ldf(a.w, r * a.w.s[0] + c * a.w.s[1]);
+  }
+  if (t < a.Cout) a.bf[t] = a.has_bias ? ldf(a.bias, t * a.bias.s[0]) : 0.f;
+  if (t < a.H) {
+    const float k = kLog2e * 0.57735026918962576f;  // log2(e) / sqrt(3)
+    a.sc[t] = make_float2(k * softplus_stable(ldf(a.dscale, t * a.dscale.s[0])),
+                          k * softplus_stable(ldf(a.xscale, t * a.xscale.s[0])));
+  }
+}
+
+struct PrepArgs {
+  int B, N, H, M, VW;
+  View qd, kd, qp, kp, val, rot, trans, fmask;
+  float4* qg;   // [B*H, N, 2]: (qd, bias) (qp, 0)
+  float4* kg;   // [B*H, N, 2]: (kd, bias) (kp, 0)
+  float* vg;    // [B*H, N, VW]
+  float* rotf;  // [B, N, 9]
+};
+
+__global__ void geo_prep_kernel(const PrepArgs a) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(a.B) * a.N * a.H;
+  if (t >= total) return;
+  const int h = static_cast<int>(t % a.H);
+  const int n = static_cast<int>((t / a.H) % a.N);
+  const int b = static_cast<int>(t / (static_cast<int64_t>(a.H) * a.N));
+  float R[9];
+  const int64_t ro = b * a.rot.s[0] + n * a.rot.s[1];
+#pragma unroll
+  for (int x = 0; x < 3; ++x)
+#pragma unroll
+    for (int y = 0; y < 3; ++y) R[x * 3 + y] = ldf(a.rot, ro + x * a.rot.s[2] + y * a.rot.s[3]);
+  const int64_t to = b * a.trans.s[0] + n * a.trans.s[1];
+  const float T[3] = {ldf(a.trans, to), ldf(a.trans, to + a.trans.s[2]), ldf(a.trans, to + 2 * a.trans.s[2])};
+  const bool valid = ldb(a.fmask, b * a.fmask.s[0] + n * a.fmask.s[1]);
+  const float bias = valid ? 0.f : -INFINITY;
+
+  auto rot3 = [&](const View& v, int64_t base, float out[3]) {
+    const float p0 = ldf(v, base), p1 = ldf(v, base + v.s[3]), p2 = ldf(v, base + 2 * v.s[3]);
+#pragma unroll
+    for (int x = 0; x < 3; ++x) out[x] = fmaf(R[x * 3], p0, fmaf(R[x * 3 + 1], p1, R[x * 3 + 2] * p2));
+  };
+  float qd[3], kd[3], qp[3], kp[3];
+  rot3(a.qd, b * a.qd.s[0] + n * a.qd.s[1] + h * a.qd.s[2], qd);
+  rot3(a.kd, b * a.kd.s[0] + n * a.kd.s[1] + h * a.kd.s[2], kd);
+  rot3(a.qp, b * a.qp.s[0] + n * a.qp.s[1] + h * a.qp.s[2], qp);
+  rot3(a.kp, b * a.kp.s[0] + n * a.kp.s[1] + h * a.kp.s[2], kp);
+  const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.N + n;
+  a.qg[2 * row] = make_float4(qd[0], qd[1], qd[2], bias);
+  a.qg[2 * row + 1] = make_float4(qp[0] + T[0], qp[1] + T[1], qp[2] + T[2], 0.f);
+  a.kg[2 * row] = make_float4(kd[0], kd[1], kd[2], bias);
+  a.kg[2 * row + 1] = make_float4(kp[0] + T[0], kp[1] + T[1], kp[2] + T[2], 0.f);
+  float* vo = a.vg + row * a.VW;
+  for (int m = 0; m < a.M; ++m) {
+    float vr[3];
+    const int64_t vb = b * a.val.s[0] + n * a.val.s[1] + h * a.val.s[2] + m * a.val.s[3];
+    const float p0 = ldf(a.val, vb), p1 = ldf(a.val, vb + a.val.s[4]), p2 = ldf(a.val, vb + 2 * a.val.s[4]);
+#pragma unroll
+    for (int x = 0; x < 3; ++x) vr[x] = fmaf(R[x * 3], p0, fmaf(R[x * 3 + 1], p1, R[x * 3 + 2] * p2));
+    vo[3 * m] = vr[0];
+    vo[3 * m + 1] = vr[1];
+    vo[3 * m + 2] = vr[2];
+  }
+  for (int e = 3 * a.M; e < a.VW; ++e) vo[e] = 0.f;
+  if (h == 0) {
+    float* rf = a.rotf + (static_cast<int64_t>(b) * a.N + n) * 9;
+#pragma unroll
+    for (int e = 0; e < 9; ++e) rf[e] = R[e];
+  }
+}
+
+// Score in the log2 domain.  The same instruction sequence is used by the
+// aggregation kernel and by the attention-map kernel so both see identical
+// values.
+__device__ __forceinline__ float geo_score(const float4 q0, const float4 q1, const float4 k0,
+                                           const float4 k1, float A, float Bd) {
+  const float dot = fmaf(q0.x, k0.x, fmaf(q0.y, k0.y, __fmul_rn(q0.z, k0.z)));
+  const float dx = __fsub_rn(q1.x, k1.x), dy = __fsub_rn(q1.y, k1.y), dz = __fsub_rn(q1.z, k1.z);
+  const float d2 = fmaf(dx, dx, fmaf(dy, dy, __fmul_rn(dz, dz)));
+  const float dist = __fsqrt_rn(d2);
+  return __fadd_rn(__fadd_rn(fmaf(A, dot, -__fmul_rn(Bd, dist)), q0.w), k0.w);
+}
+
+struct AttnArgs {
+  int B, N, H, VW;
+  float tau;
+  const float4* qg;
+  const float4* kg;
+  const float* vg;
+  const float2* sc;
+  const float* rotf;
+  const unsigned char* pm;   // may be null
+  int64_t pms[4];            // element (byte) strides b, h, i, j
+  float* out_vectors;        // [B, N, H, M, 3]
+  float2* ml;                // [B*H, N]
+  unsigned char* live;       // [B, N, H]
+};
+
+template <int M>
+__global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT) geo_attn_kernel(const AttnArgs a) {
+  constexpr int V = 3 * M;
+  const int tid = threadIdx.x;
+  const int r = tid % GEO_ROWS, split = tid / GEO_ROWS;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int i = blockIdx.x * GEO_ROWS + r;
+  const int N = a.N;
+  const int64_t bh = static_cast<int64_t>(b) * a.H + h;
+  const bool in_range = i < N;
+  const float2 sc = a.sc[h];
+
+  float4 q0 = make_float4(0, 0, 0, -INFINITY), q1 = make_float4(0, 0, 0, 0);
+  if (in_range) {
+    q0 = a.qg[2 * (bh * N + i)];
+    q1 = a.qg[2 * (bh * N + i) + 1];
+  }
+  const unsigned char* pmrow =
+      a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(in_range ? i : 0) * a.pms[2] : nullptr;
+  const int64_t pj = a.pms[3];
+
+  float m = -INFINITY, l = 0.f;
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+
+  const int nchunk = (N + GEO_CHUNK - 1) / GEO_CHUNK;
+  for (int ch = split; ch < nchunk; ch += GEO_SPLIT) {
+    const int j0 = ch * GEO_CHUNK;
+    uint32_t allowed = 0xffffffffu;
+    if (pmrow) {
+      allowed = 0u;
+      const unsigned char* p = pmrow + static_cast<int64_t>(j0) * pj;
+      if (pj == 1 && j0 + GEO_CHUNK <= N && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+        const uint4 u0 = *reinterpret_cast<const uint4*>(p);
+        const uint4 u1 = *reinterpret_cast<const uint4*>(p + 16);
+        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int k = 0; k < 32; ++k) allowed |= ((w[k >> 2] >> (8 * (k & 3))) & 0xffu) ? (1u << k) : 0u;
+      } else {
+        for (int k = 0; k < GEO_CHUNK && j0 + k < N; ++k) allowed |= p[k * pj] ? (1u << k) : 0u;
+      }
+    }
+    float s[GEO_CHUNK];
+    float cm = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < GEO_CHUNK; ++k) {
+      const int j = j0 + k;
+      float v = -INFINITY;
+      if (j < N) {
+        const float4 k0 = a.kg[2 * (bh * N + j)];
+        const float4 k1 = a.kg[2 * (bh * N + j) + 1];
+        v = geo_score(q0, q1, k0, k1, sc.x, sc.y);
+        if (!((allowed >> k) & 1u)) v = -INFINITY;
+      }
+      s[k] = v;
+      cm = fmaxf(cm, v);
+    }
+    if (cm > m + a.tau) {
+      if (m != -INFINITY) {
+        const float f = ex2(m - cm);
+        l *= f;
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] *= f;
+      }
+      m = cm;
+    }
+    if (m == -INFINITY) continue;
+#pragma unroll
+    for (int k = 0; k < GEO_CHUNK; ++k) {
+      const float p = ex2(s[k] - m);
+      l += p;
+      const float* vr = a.vg + (bh * N + j0 + k) * a.VW;
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] = fmaf(p, vr[e], acc[e]);
+    }
+  }
+
+  // merge the key splits
+  extern __shared__ float geo_merge[];  // [GEO_SPLIT][2 + V][GEO_ROWS]
+  auto sm_at = [&](int s2, int e) -> float& { return geo_merge[(s2 * (2 + V) + e) * GEO_ROWS + r]; };
+  sm_at(split, 0) = m;
+  sm_at(split, 1) = l;
+#pragma unroll
+  for (int e = 0; e < V; ++e) sm_at(split, 2 + e) = acc[e];
+  __syncthreads();
+  if (split != 0 || !in_range) return;
+  float mf = -INFINITY;
+#pragma unroll
+  for (int s2 = 0; s2 < GEO_SPLIT; ++s2) mf = fmaxf(mf, sm_at(s2, 0));
+  float lf = 0.f, af[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) af[e] = 0.f;
+  if (mf != -INFINITY) {
+#pragma unroll
+    for (int s2 = 0; s2 < GEO_SPLIT; ++s2) {
+      const float ms = sm_at(s2, 0);
+      if (ms == -INFINITY) continue;
+      const float f = ex2(ms - mf);
+      lf = fmaf(sm_at(s2, 1), f, lf);
+#pragma unroll
+      for (int e = 0; e < V; ++e) af[e] = fmaf(sm_at(s2, 2 + e), f, af[e]);
+    }
+  }
+  const bool has = lf > 0.f;
+  const float inv = has ? 1.f / lf : 0.f;
+  const float* R = a.rotf + (static_cast<int64_t>(b) * N + i) * 9;
+  float* dst = a.out_vectors + ((static_cast<int64_t>(b) * N + i) * a.H + h) * V;
+#pragma unroll
+  for (int mm = 0; mm < M; ++mm) {
+    const float gx = af[3 * mm] * inv, gy = af[3 * mm + 1] * inv, gz = af[3 * mm + 2] * inv;
+#pragma unroll
+    for (int x = 0; x < 3; ++x)  // R^T g
+      dst[3 * mm + x] = has ? fmaf(R[x], gx, fmaf(R[3 + x], gy, R[6 + x] * gz)) : 0.f;
+  }
+  a.ml[bh * N + i] = make_float2(mf, lf);
+  a.live[(static_cast<int64_t>(b) * N + i) * a.H + h] = has ? 1 : 0;
+}
+
+struct MapArgs {
+  int B, N, H;
+  const float4* qg;
+  const float4* kg;
+  const float2* sc;
+  const float2* ml;
+  const unsigned char* pm;
+  int64_t pms[4];
+  float* att;   // [B, H, N, N]
+};
+
+__global__ void __launch_bounds__(256) geo_map_kernel(const MapArgs a) {
+  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int N = a.N;
+  const int64_t bh = static_cast<int64_t>(b) * a.H + h;
+  const float4 q0 = a.qg[2 * (bh * N + i)];
+  const float4 q1 = a.qg[2 * (bh * N + i) + 1];
+  const float2 sc = a.sc[h];
+  const float2 st = a.ml[bh * N + i];
+  const bool has = st.y > 0.f;
+  const float inv = has ? 1.f / st.y : 0.f;
+  float* dst = a.att + (bh * N + i) * static_cast<int64_t>(N);
+  const unsigned char* pmrow = a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(i) * a.pms[2] : nullptr;
+  for (int j = threadIdx.x; j < N; j += blockDim.x) {
+    float v = 0.f;
+    if (has && (!pmrow || pmrow[static_cast<int64_t>(j) * a.pms[3]])) {
+      const float4 k0 = a.kg[2 * (bh * N + j)];
+      const float4 k1 = a.kg[2 * (bh * N + j) + 1];
+      const float s = geo_score(q0, q1, k0, k1, sc.x, sc.y);
+      v = ex2(s - st.x) * inv;
+    }
+    dst[j] = v;
+  }
+}
+
+struct ReadArgs {
+  int B, N, H, HM3, Cout;
+  const float* vec;   // [B*N, HM3]
+  const unsigned char* live;
+  const float* wf;
+  const float* bf;
+  float* out;         // [B*N, Cout]
+};
+
+constexpr int RD_ROWS = 32;
+
+__global__ void __launch_bounds__(256) geo_readout_kernel(const ReadArgs a) {
+  extern __shared__ float vs[];  // [RD_ROWS][HM3]
+  __shared__ int any_live[RD_ROWS];
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * RD_ROWS;
+  const int64_t nrows = static_cast<int64_t>(a.B) * a.N;
+  for (int t = threadIdx.x; t < RD_ROWS * a.HM3; t += blockDim.x) {
+    const int rr = t / a.HM3, k = t % a.HM3;
+    vs[t] = row0 + rr < nrows ? a.vec[(row0 + rr) * a.HM3 + k] : 0.f;
+  }
+  if (threadIdx.x < RD_ROWS) {
+    int anyl = 0;
+    if (row0 + threadIdx.x < nrows)
+      for (int h = 0; h < a.H; ++h) anyl |= a.live[(row0 + threadIdx.x) * a.H + h];
+    any_live[threadIdx.x] = anyl;
+  }
+  __syncthreads();
+  const int col = blockIdx.y * blockDim.x + threadIdx.x;
+  if (col >= a.Cout) return;
+  float acc[RD_ROWS];
+#pragma unroll
+  for (int rr = 0; rr < RD_ROWS; ++rr) acc[rr] = 0.f;
+  for (int k = 0; k < a.HM3; ++k) {
+    const float w = a.wf[static_cast<int64_t>(k) * a.Cout + col];
+#pragma unroll
+    for (int rr = 0; rr < RD_ROWS; ++rr) acc[rr] = fmaf(vs[rr * a.HM3 + k], w, acc[rr]);
+  }
+  const float bias = a.bf[col];
+#pragma unroll
+  for (int rr = 0; rr < RD_ROWS; ++rr) {
+    const int64_t row = row0 + rr;
+    if (row < nrows) a.out[row * a.Cout + col] = any_live[rr] ? acc[rr] + bias : 0.f;
+  }
+}
+
+template <int M>
+cudaError_t launch_attn(const AttnArgs& t, int B, int N, int H, cudaStream_t st) {
+  dim3 grid((N + GEO_ROWS - 1) / GEO_ROWS, H, B);
+  const size_t smem = sizeof(float) * GEO_SPLIT * (2 + 3 * M) * GEO_ROWS;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(geo_attn_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  geo_attn_kernel<M><<<grid, GEO_ROWS * GEO_SPLIT, smem, st>>>(t);
+  return cudaSuccess;
+}
+
+}  // namespace
+
+GeoWorkspace geo_workspace_layout(int B, int N, int H, int M, int Cout) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  GeoWorkspace w{};
+  size_t o = 0;
+  const size_t bhn = static_cast<size_t>(B) * H * N;
+  const int VW = 3 * M;
+  const int HM3 = H * M * 3;
+  w.qg = o; o = up(o + bhn * 32);
+  w.kg = o; o = up(o + bhn * 32);
+  w.vg = o; o = up(o + bhn * VW * 4);
+  w.rotf = o; o = up(o + static_cast<size_t>(B) * N * 36);
+  w.ml = o; o = up(o + bhn * 8);
+  w.live = o; o = up(o + bhn);
+  w.wf = o; o = up(o + static_cast<size_t>(HM3) * Cout * 4);
+  w.bf = o; o = up(o + static_cast<size_t>(Cout) * 4);
+  w.sc = o; o = up(o + static_cast<size_t>(H) * 8);
+  w.err = o; o = up(o + 16);
+  w.total = o;
+  return w;
+}
+
+cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
+  unsigned char* ws = a.ws;
+  const GeoWorkspace& w = a.lay;
+  const int VW = 3 * a.M;
+
+  WArgs wa{};
+  wa.H = a.H; wa.HM3 = a.HM3; wa.Cout = a.Cout; wa.has_bias = a.has_bias;
+  wa.dscale = a.direction_scale; wa.xscale = a.distance_scale; wa.w = a.output_weight; wa.bias = a.output_bias;
+  wa.sc = reinterpret_cast<float2*>(ws + w.sc);
+  wa.wf = reinterpret_cast<float*>(ws + w.wf);
+  wa.bf = reinterpret_cast<float*>(ws + w.bf);
+  {
+    int64_t n = static_cast<int64_t>(a.HM3) * a.Cout;
+    if (n < a.Cout) n = a.Cout;
+    if (n < a.H) n = a.H;
+    geo_weights_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(wa);
+  }
+
+  PrepArgs pa{};
+  pa.B = a.B; pa.N = a.N; pa.H = a.H; pa.M = a.M; pa.VW = VW;
+  pa.qd = a.q_direction; pa.kd = a.k_direction; pa.qp = a.q_point; pa.kp = a.k_point;
+  pa.val = a.values; pa.rot = a.rotation; pa.trans = a.translation; pa.fmask = a.frame_mask;
+  pa.qg = reinterpret_cast<float4*>(ws + w.qg);
+  pa.kg = reinterpret_cast<float4*>(ws + w.kg);
+  pa.vg = reinterpret_cast<float*>(ws + w.vg);
+  pa.rotf = reinterpret_cast<float*>(ws + w.rotf);
+  {
+    const int64_t n = static_cast<int64_t>(a.B) * a.N * a.H;
+    geo_prep_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(pa);
+  }
+
+  AttnArgs t{};
+  t.B = a.B; t.N = a.N; t.H = a.H; t.VW = VW; t.tau = 8.f;
+  t.qg = pa.qg; t.kg = pa.kg; t.vg = pa.vg; t.sc = wa.sc; t.rotf = pa.rotf;
+  t.pm = a.has_pair_mask ? reinterpret_cast<const unsigned char*>(a.pair_mask.p) : nullptr;
+  for (int d = 0; d < 4; ++d) t.pms[d] = a.has_pair_mask ? a.pair_mask.s[d] : 0;
+  t.out_vectors = a.out_vectors;
+  t.ml = reinterpret_cast<float2*>(ws + w.ml);
+  t.live = ws + w.live;
+  cudaError_t le = cudaErrorInvalidValue;
+  switch (a.M) {
+    case 1: le = launch_attn<1>(t, a.B, a.N, a.H, st); break;
+    case 2: le = launch_attn<2>(t, a.B, a.N, a.H, st); break;
+    case 3: le = launch_attn<3>(t, a.B, a.N, a.H, st); break;
+    case 4: le = launch_attn<4>(t, a.B, a.N, a.H, st); break;
+    case 5: le = launch_attn<5>(t, a.B, a.N, a.H, st); break;
+    case 6: le = launch_attn<6>(t, a.B, a.N, a.H, st); break;
+    case 7: le = launch_attn<7>(t, a.B, a.N, a.H, st); break;
+    case 8: le = launch_attn<8>(t, a.B, a.N, a.H, st); break;
+    default: break;
+  }
+  if (le != cudaSuccess) return le;
+
+  if (a.out_attention) {
+    MapArgs ma{};
+    ma.B = a.B; ma.N = a.N; ma.H = a.H;
+    ma.qg = pa.qg; ma.kg = pa.kg; ma.sc = wa.sc; ma.ml = t.ml;
+    ma.pm = t.pm;
+    for (int d = 0; d < 4; ++d) ma.pms[d] = t.pms[d];
+    ma.att = a.out_attention;
+    geo_map_kernel<<<dim3(a.N, a.H, a.B), 256, 0, st>>>(ma);
+  }
+
+  ReadArgs ra{};
+  ra.B = a.B; ra.N = a.N; ra.H = a.H; ra.HM3 = a.HM3; ra.Cout = a.Cout;
+  ra.vec = a.out_vectors; ra.live = t.live; ra.wf = wa.wf; ra.bf = wa.bf; ra.out = a.out_output;
+  {
+    const int64_t rows = static_cast<int64_t>(a.B) * a.N;
+    dim3 grid(static_cast<unsigned>((rows + RD_ROWS - 1) / RD_ROWS), (a.Cout + 255) / 256);
+    const size_t smem = static_cast<size_t>(RD_ROWS) * a.HM3 * sizeof(float);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(geo_readout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    geo_readout_kernel<<<grid, 256, smem, st>>>(ra);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fipa

@@ -1,0 +1,73 @@
+// Internal (non-exported) declarations shared by the host API and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace fipa {
+
+// Geometry of the fused IPA kernels.
+constexpr int QT = 128;      // query rows per CTA (tcgen05 M)
+constexpr int KT = 64;       // keys per tile (N of Q K^T, K of P V)
+constexpr int DH = 64;       // width of the per-head augmented rows (fp16)
+constexpr int NSTAGE = 3;    // K/V shared-memory stages
+constexpr int MAX_DZ = 256;  // widest pair block (R * Cz padded to 64)
+constexpr int IPA_C = 16, IPA_PQ = 4, IPA_PV = 8;
+
+// Strided fp32 / byte view of a caller tensor (strides in elements).
+struct View {
+  const void* p;
+  int64_t s[6];
+  int dtype;  // 0 f32, 1 f64, 2 u8
+};
+
+struct IpaWorkspace {
+  size_t qh, kh, vh, qp, z2, rowq, colk, frame, z1f, oq, ok, headc, err, total;
+};
+
+IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz);
+
+struct IpaLaunch {
+  int B, L, H, C, Pq, Pv, R, Cz, DZ, RCz, F, nqt, nkt;
+  float w_L, w_C, scalar_scale;
+  View q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask;
+  float* out;
+  unsigned char* ws;
+  IpaWorkspace lay;
+  int* err;
+};
+
+// Stage launches; each returns the cudaError_t of its last launch.
+cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream);
+cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream);
+
+struct GeoWorkspace {
+  size_t qg, kg, vg, rotf, ml, live, wf, bf, sc, err, total;
+};
+
+GeoWorkspace geo_workspace_layout(int B, int N, int H, int M, int Cout);
+
+struct GeoLaunch {
+  int B, N, H, M, Cout, HM3;
+  View q_direction, k_direction, q_point, k_point, values, direction_scale, distance_scale,
+      output_weight, output_bias, rotation, translation, frame_mask, pair_mask;
+  bool has_bias, has_pair_mask;
+  float* out_vectors;
+  float* out_output;
+  float* out_attention;  // may be null
+  unsigned char* ws;
+  GeoWorkspace lay;
+  int* err;
+};
+
+cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled obtained through the runtime's driver entry point.
+bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                        uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
+                        uint32_t box0, uint32_t box1);
+
+}  // namespace fipa

@@ -1,0 +1,193 @@
+"""CPU-only checks of the C ABI boundary: the library loads, exports every
+function include/flashipa_b200.h declares, and rejects bad arguments before
+launching anything.  No test here runs device code."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from rna_structure_models_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flashipa_b200.h")
+
+FAKE = 1 << 20  # a non-null, 256-aligned address that is never dereferenced
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"IPA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"ipa_attn_fwd", "ipa_attn_workspace_size", "geo_attn_fwd", "geo_attn_workspace_size",
+            "ipa_status_string"} <= names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = api.library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(api.EXPORTED) == set(declared_functions())
+
+
+def test_status_strings_and_version():
+    lib = api.library()
+    for code in range(9):
+        assert lib.ipa_status_string(code)
+    assert b"sm_100a" in lib.ipa_version()
+    assert lib.ipa_device_error_status(0) == 0
+    assert lib.ipa_device_error_status(1) == 8       # bounded wait expired -> IPA_ERR_TIMEOUT
+    assert lib.ipa_device_error_status(7) == 7
+
+
+def desc(shape, dtype=api.IPA_DTYPE_F32, ptr=FAKE, strides=None):
+    d = api.IpaTensor()
+    d.data = ptr
+    d.dtype = dtype
+    d.ndim = len(shape)
+    if strides is None:
+        strides, acc = [], 1
+        for s in reversed(shape):
+            strides.insert(0, acc)
+            acc *= s
+    for i, (s, st) in enumerate(zip(shape, strides)):
+        d.size[i] = s
+        d.stride[i] = st
+    return d
+
+
+def ipa_args(B=1, L=64, H=4, C=16, Pq=4, Pv=8, R=2, Cz=16, **over):
+    F = C + 4 * Pv + Cz
+    shapes = {"q": (B, L, H, C), "k": (B, L, H, C), "v": (B, L, H, C),
+              "q_pts": (B, L, H, Pq, 3), "k_pts": (B, L, H, Pq, 3), "v_pts": (B, L, H, Pv, 3),
+              "rot": (B, L, 3, 3), "trans": (B, L, 3), "z1": (B, L, R, Cz), "z2": (B, L, R, Cz),
+              "w_bias": (Cz, H), "gamma": (H,), "mask": (B, L), "out": (B, L, H, F)}
+    ds = {k: desc(s, api.IPA_DTYPE_BOOL if k == "mask" else api.IPA_DTYPE_F32) for k, s in shapes.items()}
+    ds.update(over)
+    return api.ipa_params(B, L, H, C, Pq, Pv, R, Cz), ds
+
+
+ORDER = ("q", "k", "v", "q_pts", "k_pts", "v_pts", "rot", "trans", "z1", "z2", "w_bias", "gamma",
+         "mask", "out")
+
+
+def call_ipa(p, ds, ws_bytes=None, ws_ptr=FAKE):
+    lib = api.library()
+    if ws_bytes is None:
+        ws_bytes = lib.ipa_attn_workspace_size(ctypes.byref(p))
+    return lib.ipa_attn_fwd(ctypes.byref(p), *[ctypes.byref(ds[k]) if ds[k] is not None else None
+                                               for k in ORDER],
+                            ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes), None,
+                            ctypes.c_void_p(FAKE))
+
+
+def test_workspace_size_is_linear_in_L_and_zero_when_invalid():
+    lib = api.library()
+    sizes = []
+    for L in (2048, 4096, 8192, 16384):
+        p = api.ipa_params(1, L, 12, 16, 4, 8, 2, 128)
+        sizes.append(lib.ipa_attn_workspace_size(ctypes.byref(p)))
+    per = [s / L for s, L in zip(sizes, (2048, 4096, 8192, 16384))]
+    assert max(per) / min(per) < 1.01
+    bad = api.ipa_params(1, 64, 4, 32, 4, 8, 2, 16)      # C = 32 is outside the envelope
+    assert lib.ipa_attn_workspace_size(ctypes.byref(bad)) == 0
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("null_tensor", 1), ("shape", 2), ("neg_stride", 3), ("dtype", 4), ("workspace", 5),
+    ("ws_align", 5), ("unsupported", 6), ("mask_dtype", 4), ("out_noncontig", 3), ("null_params", 1),
+])
+def test_ipa_rejects_bad_arguments_before_launch(case, expect):
+    p, ds = ipa_args()
+    ws = None
+    ws_ptr = FAKE
+    if case == "null_tensor":
+        ds["k"] = desc((1, 64, 4, 16), ptr=None)
+    elif case == "shape":
+        ds["v"] = desc((1, 63, 4, 16))
+    elif case == "neg_stride":
+        ds["q"] = desc((1, 64, 4, 16), strides=(4096, 64, -16, 1))
+    elif case == "dtype":
+        ds["z1"] = desc((1, 64, 2, 16), dtype=api.IPA_DTYPE_F64)
+    elif case == "workspace":
+        ws = 1024
+    elif case == "ws_align":
+        ws_ptr = FAKE + 8
+    elif case == "unsupported":
+        p, ds = ipa_args(Pv=4)
+    elif case == "mask_dtype":
+        ds["mask"] = desc((1, 64), dtype=api.IPA_DTYPE_F32)
+    elif case == "out_noncontig":
+        ds["out"] = desc((1, 64, 4, 64), strides=(64 * 4 * 128, 4 * 128, 128, 1))
+    if case == "null_params":
+        lib = api.library()
+        st = lib.ipa_attn_fwd(None, *[ctypes.byref(ds[k]) for k in ORDER], ctypes.c_void_p(FAKE),
+                              ctypes.c_size_t(1 << 30), None, ctypes.c_void_p(FAKE))
+    else:
+        st = call_ipa(p, ds, ws, ws_ptr)
+    assert st == expect
+
+
+def geo_args(B=1, N=32, H=2, M=2, Cout=8, dt=api.IPA_DTYPE_F32, **over):
+    shapes = {"q_direction": (B, N, H, 3), "k_direction": (B, N, H, 3), "q_point": (B, N, H, 3),
+              "k_point": (B, N, H, 3), "values": (B, N, H, M, 3), "direction_scale": (H,),
+              "distance_scale": (H,), "output_weight": (H * M * 3, Cout), "output_bias": (Cout,),
+              "rotation": (B, N, 3, 3), "translation": (B, N, 3)}
+    ds = {k: desc(s, dt) for k, s in shapes.items()}
+    ds["frame_mask"] = desc((B, N), api.IPA_DTYPE_BOOL)
+    ds["pair_mask"] = desc((B, H, N, N), api.IPA_DTYPE_BOOL)
+    ds["out_vectors"] = desc((B, N, H, M, 3))
+    ds["out_output"] = desc((B, N, Cout))
+    ds["out_attention"] = desc((B, H, N, N))
+    ds.update(over)
+    return api.GeoParams(B, N, H, M, Cout), ds
+
+
+GEO_ORDER = api.GEO_INPUTS + ("out_vectors", "out_output", "out_attention")
+
+
+def call_geo(p, ds, ws_bytes=None):
+    lib = api.library()
+    if ws_bytes is None:
+        ws_bytes = lib.geo_attn_workspace_size(ctypes.byref(p))
+    return lib.geo_attn_fwd(ctypes.byref(p), *[ctypes.byref(ds[k]) if ds[k] is not None else None
+                                               for k in GEO_ORDER],
+                            ctypes.c_void_p(FAKE), ctypes.c_size_t(ws_bytes), None, ctypes.c_void_p(FAKE))
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("mixed_dtype", 4), ("pair_mask_shape", 2), ("values_shape", 2), ("workspace", 5),
+    ("too_many_channels", 6), ("frame_mask_dtype", 4), ("att_noncontig", 3),
+])
+def test_geo_rejects_bad_arguments_before_launch(case, expect):
+    p, ds = geo_args()
+    ws = None
+    if case == "mixed_dtype":
+        ds["k_point"] = desc((1, 32, 2, 3), api.IPA_DTYPE_F64)
+    elif case == "pair_mask_shape":
+        ds["pair_mask"] = desc((1, 2, 32, 31), api.IPA_DTYPE_BOOL)
+    elif case == "values_shape":
+        ds["values"] = desc((1, 32, 2, 3, 3))
+    elif case == "workspace":
+        ws = 100
+    elif case == "too_many_channels":
+        p, ds = geo_args(H=40, M=4)
+    elif case == "frame_mask_dtype":
+        ds["frame_mask"] = desc((1, 32))
+    elif case == "att_noncontig":
+        ds["out_attention"] = desc((1, 2, 32, 32), strides=(4096, 2048, 64, 1))
+    assert call_geo(p, ds, ws) == expect
+
+
+def test_package_import_does_not_load_the_library():
+    import importlib
+    import subprocess
+    import sys
+    code = ("import rna_structure_models_b200, rna_structure_models_b200.synth, sys;"
+            "print(any('libflashipa' in l for l in open('/proc/self/maps')))")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT)
+    assert out.stdout.strip() == "False", out.stderr
+    importlib.import_module("rna_structure_models_b200")
