@@ -40,7 +40,7 @@ METRIC = "fused IPA attention TFLOP/s and % bf16 tensor-pipe peak at L=4096 (1xB
 UNIT = "TFLOP/s"
 
 # DRAM traffic of one launch of the core kernel from an ncu capture, valid only
-# for the kernel source it was taken on (sha256 of csrc/ipa_kernels.cu).
+# for the kernel source it was taken on (sha256 of csrc/ipa_attention.cu).
 NCU_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None}
 
 
@@ -53,7 +53,7 @@ def ipa_flops(B, L, n_valid=None):
 
 
 def kernel_sha():
-    p = os.path.join(ROOT, "rna_structure_models_b200", "csrc", "ipa_kernels.cu")
+    p = os.path.join(ROOT, "rna_structure_models_b200", "csrc", "ipa_attention.cu")
     return hashlib.sha256(open(p, "rb").read()).hexdigest()
 
 

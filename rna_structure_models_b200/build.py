@@ -18,7 +18,7 @@ PROBE_LIB = os.path.join(ROOT, "tests", "libflashipa_probe.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
          "--expt-relaxed-constexpr", "-Xcompiler", "-fvisibility=hidden"]
-SOURCES = ["api.cu", "ipa_kernels.cu", "geo_kernels.cu"]
+SOURCES = ["api.cu", "ipa_prologue.cu", "ipa_attention.cu", "geo_kernels.cu"]
 
 
 def nvcc() -> str:
@@ -47,6 +47,14 @@ def build_lib(verbose: bool = False, ptxas_info: bool = False) -> str:
     if ptxas_info:
         print(out)
     return LIB
+
+
+def build_traced(out_path: str, verbose: bool = False) -> str:
+    """Same library with per-tile event tracing compiled in (IPA_TRACE)."""
+    srcs = [os.path.join(CSRC, s) for s in SOURCES]
+    cmd = [nvcc(), *ARCH, *FLAGS, "-DIPA_TRACE", f"-I{INCLUDE}", f"-I{CSRC}", *srcs, "-o", out_path]
+    _run(cmd, verbose)
+    return out_path
 
 
 def build_probe(verbose: bool = False) -> str:

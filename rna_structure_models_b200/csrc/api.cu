@@ -338,3 +338,10 @@ ipa_status_t geo_attn_fwd(const geo_params_t* p, const ipa_tensor_t* q_direction
 }
 
 }  // extern "C"
+
+#ifdef IPA_TRACE
+// Tracing build only: copy the per-tile event timestamps to the host.
+extern "C" __attribute__((visibility("default"))) int ipa_trace_copy(void* host, size_t bytes) {
+  return fipa::ipa_trace_read(host, bytes) ? 0 : 1;
+}
+#endif

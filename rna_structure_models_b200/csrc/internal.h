@@ -25,7 +25,7 @@ struct View {
 };
 
 struct IpaWorkspace {
-  size_t qh, kh, vh, qp, z2, rowq, colk, frame, z1f, oq, ok, headc, err, total;
+  size_t qh, kh, vh, z2, z1f, rowq, colk, frame, part, cen, oq, ok, headc, wqp, err, total;
 };
 
 IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz);
@@ -64,6 +64,10 @@ struct GeoLaunch {
 };
 
 cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t stream);
+
+#ifdef IPA_TRACE
+bool ipa_trace_read(void* host, size_t bytes);
+#endif
 
 // cuTensorMapEncodeTiled obtained through the runtime's driver entry point.
 bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,

@@ -1,0 +1,413 @@
+// Prologue of the fused IPA core: applies the residue frames and writes the
+// fp16 augmented operands that the attention kernel streams with TMA.
+//
+//   ipa_tile_kernel   -- one CTA per (batch, 64-residue key tile): frame rows
+//                        (R, t, valid), partial sums of the valid origins, and
+//                        the pair factors z2 (fp16) / z1 (fp32) padded to DZ.
+//   ipa_reduce_kernel -- one CTA per batch: centroid of the valid origins,
+//                        query-tile (128) and key-tile (64) origins relative
+//                        to it; per-head point coefficient and pair-bias
+//                        weights w_L log2(e) w_bias[c, h] (batch 0's CTA).
+//   ipa_rows_kernel   -- one thread per (b, h, i): Q_h, K_h, V_h rows (64
+//                        fp16 each) and the two small fp32 row terms.
+//
+// Augmented row layout for the (C, Pq, Pv) = (16, 4, 8) head shape, with
+// c = log2(e) w_L gamma_h w_C / 2, gq' / gk' the global query / key points
+// relative to their tile origin and gv the value points relative to the
+// centroid (hi = fp16(x), lo = fp16(x - hi)):
+//   Q_h: [ log2(e) w_L s q (16) | gq'hi (12) | gq'hi (12) | gq'lo (12) | -1 -1 | 0 (10) ]
+//   K_h: [ k (16) | 2c gk' hi (12) | lo (12) | hi (12) | c|gk'|^2 hi, lo | 0 (10) ]
+//   V_h: [ v (16) | gv hi (24) | gv lo (24) ]
+// so Q_h . K_h = log2(e) w_L s q.k + 2c gq'.gk' - c sum_p |gk'_p|^2 (the
+// lo*lo product is dropped; every kept product is exact in fp32).
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fipa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float ldf(const View& v, int64_t off) {
+  return reinterpret_cast<const float*>(v.p)[off];
+}
+__device__ __forceinline__ bool ldb(const View& v, int64_t off) {
+  return reinterpret_cast<const unsigned char*>(v.p)[off] != 0;
+}
+
+struct TileArgs {
+  int B, L, R, Cz, RCz, DZ, nkt;
+  View rot, trans, mask, z1, z2;
+  float4* frame;   // [B, L, 4]: (R00 R01 R02 R10) (R11 R12 R20 R21) (R22 tx ty tz) (valid 0 0 0)
+  float4* part;    // [B, nkt]: sum of valid origins, count
+  float* z1f;      // [B, L, DZ]
+  __half* z2h;     // [B, L, DZ]
+};
+
+// Pair factors of 64 residues x one 64-column panel, zero-padded beyond
+// R*Cz and zero for masked residues: 4 residues x 64 columns per pass, all
+// loads of a thread issued before its stores.
+__device__ __forceinline__ void ipa_tile_copy_pairs(const TileArgs& a, int b, int i0, int panel, int tid) {
+  const int col = panel * 64 + (tid & 63);
+  const bool inpair = col < a.RCz;
+  const int rr = inpair ? col / a.Cz : 0, cc = inpair ? col % a.Cz : 0;
+  constexpr int NR = KT / 4;
+  float v1[NR], v2[NR];
+#pragma unroll
+  for (int q = 0; q < NR; ++q) {
+    const int i = i0 + 4 * q + (tid >> 6);
+    v1[q] = 0.f;
+    v2[q] = 0.f;
+    if (i < a.L && inpair && ldb(a.mask, b * a.mask.s[0] + i * a.mask.s[1])) {
+      v1[q] = ldf(a.z1, b * a.z1.s[0] + i * a.z1.s[1] + rr * a.z1.s[2] + cc * a.z1.s[3]);
+      v2[q] = ldf(a.z2, b * a.z2.s[0] + i * a.z2.s[1] + rr * a.z2.s[2] + cc * a.z2.s[3]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < NR; ++q) {
+    const int i = i0 + 4 * q + (tid >> 6);
+    if (i < a.L) {
+      const int64_t o = (static_cast<int64_t>(b) * a.L + i) * a.DZ + col;
+      a.z1f[o] = v1[q];
+      a.z2h[o] = __float2half_rn(v2[q]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) ipa_tile_kernel(const TileArgs a) {
+  const int J = blockIdx.x, b = blockIdx.y, panel = blockIdx.z, tid = threadIdx.x;
+  const int i0 = J * KT;
+  __shared__ float red[2][4];
+  if (panel > 0) {
+    ipa_tile_copy_pairs(a, b, i0, panel, tid);
+    return;
+  }
+  if (tid < KT) {
+    const int i = i0 + tid;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < a.L) {
+      const bool valid = ldb(a.mask, b * a.mask.s[0] + i * a.mask.s[1]);
+      const int64_t ro = b * a.rot.s[0] + i * a.rot.s[1];
+      float Rm[9];
+#pragma unroll
+      for (int x = 0; x < 3; ++x)
+#pragma unroll
+        for (int y = 0; y < 3; ++y) Rm[3 * x + y] = ldf(a.rot, ro + x * a.rot.s[2] + y * a.rot.s[3]);
+      const int64_t to = b * a.trans.s[0] + i * a.trans.s[1];
+      const float tx = ldf(a.trans, to), ty = ldf(a.trans, to + a.trans.s[2]), tz = ldf(a.trans, to + 2 * a.trans.s[2]);
+      float4* f = a.frame + (static_cast<int64_t>(b) * a.L + i) * 4;
+      f[0] = make_float4(Rm[0], Rm[1], Rm[2], Rm[3]);
+      f[1] = make_float4(Rm[4], Rm[5], Rm[6], Rm[7]);
+      f[2] = make_float4(Rm[8], tx, ty, tz);
+      f[3] = make_float4(valid ? 1.f : 0.f, 0.f, 0.f, 0.f);
+      if (valid) s = make_float4(tx, ty, tz, 1.f);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      s.x += __shfl_xor_sync(0xffffffffu, s.x, off);
+      s.y += __shfl_xor_sync(0xffffffffu, s.y, off);
+      s.z += __shfl_xor_sync(0xffffffffu, s.z, off);
+      s.w += __shfl_xor_sync(0xffffffffu, s.w, off);
+    }
+    if ((tid & 31) == 0) {
+      red[tid >> 5][0] = s.x; red[tid >> 5][1] = s.y; red[tid >> 5][2] = s.z; red[tid >> 5][3] = s.w;
+    }
+  }
+  __syncthreads();
+  if (tid == 0)
+    a.part[b * a.nkt + J] = make_float4(red[0][0] + red[1][0], red[0][1] + red[1][1],
+                                        red[0][2] + red[1][2], red[0][3] + red[1][3]);
+  ipa_tile_copy_pairs(a, b, i0, 0, tid);
+}
+
+struct ReduceArgs {
+  int B, L, H, Cz, RCz, DZ, nqt, nkt;
+  float w_L, w_C;
+  View gamma, w_bias;
+  const float4* part;
+  float4* cen;     // [B]
+  float4* oq;      // [B, nqt]
+  float4* ok;      // [B, nkt]
+  float* headc;    // [H]
+  float* wqp;      // [H, DZ]
+};
+
+__global__ void __launch_bounds__(256) ipa_reduce_kernel(const ReduceArgs a) {
+  const int b = blockIdx.x, tid = threadIdx.x;
+  __shared__ double red[4][8];
+  __shared__ float cen[3];
+  double sx = 0, sy = 0, sz = 0, sn = 0;
+  for (int J = tid; J < a.nkt; J += blockDim.x) {
+    const float4 p = a.part[b * a.nkt + J];
+    sx += p.x; sy += p.y; sz += p.z; sn += p.w;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    sx += __shfl_xor_sync(0xffffffffu, sx, off);
+    sy += __shfl_xor_sync(0xffffffffu, sy, off);
+    sz += __shfl_xor_sync(0xffffffffu, sz, off);
+    sn += __shfl_xor_sync(0xffffffffu, sn, off);
+  }
+  const int w = tid >> 5, lane = tid & 31;
+  if (lane == 0) { red[0][w] = sx; red[1][w] = sy; red[2][w] = sz; red[3][w] = sn; }
+  __syncthreads();
+  if (tid == 0) {
+    double tx = 0, ty = 0, tz = 0, tn = 0;
+    for (int k = 0; k < static_cast<int>(blockDim.x >> 5); ++k) {
+      tx += red[0][k]; ty += red[1][k]; tz += red[2][k]; tn += red[3][k];
+    }
+    const double inv = tn > 0 ? 1.0 / tn : 0.0;
+    cen[0] = static_cast<float>(tx * inv);
+    cen[1] = static_cast<float>(ty * inv);
+    cen[2] = static_cast<float>(tz * inv);
+    a.cen[b] = make_float4(cen[0], cen[1], cen[2], static_cast<float>(tn));
+  }
+  __syncthreads();
+  const float cx = cen[0], cy = cen[1], cz = cen[2];
+  for (int J = tid; J < a.nkt; J += blockDim.x) {
+    const float4 p = a.part[b * a.nkt + J];
+    const float inv = p.w > 0.f ? 1.f / p.w : 0.f;
+    a.ok[b * a.nkt + J] = p.w > 0.f ? make_float4(p.x * inv - cx, p.y * inv - cy, p.z * inv - cz, 0.f)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int I = tid; I < a.nqt; I += blockDim.x) {
+    float4 p = a.part[b * a.nkt + 2 * I];
+    if (2 * I + 1 < a.nkt) {
+      const float4 p2 = a.part[b * a.nkt + 2 * I + 1];
+      p.x += p2.x; p.y += p2.y; p.z += p2.z; p.w += p2.w;
+    }
+    const float inv = p.w > 0.f ? 1.f / p.w : 0.f;
+    a.oq[b * a.nqt + I] = p.w > 0.f ? make_float4(p.x * inv - cx, p.y * inv - cy, p.z * inv - cz, 0.f)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if (b == 0) {
+    for (int h = tid; h < a.H; h += blockDim.x)
+      a.headc[h] = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
+    for (int e = tid; e < a.H * a.DZ; e += blockDim.x) {
+      const int h = e / a.DZ, col = e % a.DZ;
+      float val = 0.f;
+      if (col < a.RCz) val = kLog2e * a.w_L * ldf(a.w_bias, (col % a.Cz) * a.w_bias.s[0] + h * a.w_bias.s[1]);
+      a.wqp[e] = val;
+    }
+  }
+}
+
+struct RowArgs {
+  int B, L, H, nqt, nkt;
+  float qscale;    // log2(e) w_L scalar_scale
+  View q, k, v, q_pts, k_pts, v_pts;
+  const float4* frame;
+  const float4* cen;
+  const float4* oq;
+  const float4* ok;
+  const float* headc;
+  uint4* qh;       // [B*H, L, 64] fp16 (8 x uint4 per row)
+  uint4* kh;
+  uint4* vh;
+  float4* rowq;    // [B*H, L]
+  float4* colk;    // [B*H, L]
+  int* err;
+};
+
+template <int N>
+__device__ __forceinline__ void load_row(const View& v, int64_t base, int64_t st, float (&out)[N]) {
+#pragma unroll
+  for (int e = 0; e < N; ++e) out[e] = ldf(v, base + e * st);
+}
+
+template <int C, int PQ, int PV>
+__global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
+  static_assert(C + 9 * PQ + 2 <= DH && C + 6 * PV <= DH, "augmented rows wider than 64");
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(a.B) * a.H * a.L;
+  if (t >= total) return;
+  const int i = static_cast<int>(t % a.L);
+  const int bh = static_cast<int>(t / a.L);
+  const int h = bh % a.H, b = bh / a.H;
+
+  const float4* fr = a.frame + (static_cast<int64_t>(b) * a.L + i) * 4;
+  const float4 f0 = fr[0], f1 = fr[1], f2 = fr[2], f3 = fr[3];
+  const float4 cn = a.cen[b];
+  const float Rm[9] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w, f2.x};
+  const float tc[3] = {f2.y - cn.x, f2.z - cn.y, f2.w - cn.z};
+  const bool valid = f3.x != 0.f;
+  const float4 oqv = a.oq[b * a.nqt + i / QT];
+  const float4 okv = a.ok[b * a.nkt + i / KT];
+  const float oqa[3] = {oqv.x, oqv.y, oqv.z}, oka[3] = {okv.x, okv.y, okv.z};
+  const float c = a.headc[h];
+
+  float qs[C], ks[C], vs[C], qp[PQ * 3], kp[PQ * 3], vp[PV * 3];
+  load_row(a.q, b * a.q.s[0] + i * a.q.s[1] + h * a.q.s[2], a.q.s[3], qs);
+  load_row(a.k, b * a.k.s[0] + i * a.k.s[1] + h * a.k.s[2], a.k.s[3], ks);
+  load_row(a.v, b * a.v.s[0] + i * a.v.s[1] + h * a.v.s[2], a.v.s[3], vs);
+#pragma unroll
+  for (int p = 0; p < PQ; ++p)
+#pragma unroll
+    for (int y = 0; y < 3; ++y) {
+      qp[3 * p + y] = ldf(a.q_pts, b * a.q_pts.s[0] + i * a.q_pts.s[1] + h * a.q_pts.s[2] + p * a.q_pts.s[3] + y * a.q_pts.s[4]);
+      kp[3 * p + y] = ldf(a.k_pts, b * a.k_pts.s[0] + i * a.k_pts.s[1] + h * a.k_pts.s[2] + p * a.k_pts.s[3] + y * a.k_pts.s[4]);
+    }
+#pragma unroll
+  for (int p = 0; p < PV; ++p)
+#pragma unroll
+    for (int y = 0; y < 3; ++y)
+      vp[3 * p + y] = ldf(a.v_pts, b * a.v_pts.s[0] + i * a.v_pts.s[1] + h * a.v_pts.s[2] + p * a.v_pts.s[3] + y * a.v_pts.s[4]);
+
+  // frames applied: gq' = R q + t' - o_I, gk' = R k + t' - o_J, gv = R v + t'
+  float gq[PQ * 3], gk[PQ * 3], gv[PV * 3];
+#pragma unroll
+  for (int p = 0; p < PQ; ++p)
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      gq[3 * p + x] = fmaf(Rm[3 * x], qp[3 * p], fmaf(Rm[3 * x + 1], qp[3 * p + 1], Rm[3 * x + 2] * qp[3 * p + 2])) + tc[x] - oqa[x];
+      gk[3 * p + x] = fmaf(Rm[3 * x], kp[3 * p], fmaf(Rm[3 * x + 1], kp[3 * p + 1], Rm[3 * x + 2] * kp[3 * p + 2])) + tc[x] - oka[x];
+    }
+#pragma unroll
+  for (int p = 0; p < PV; ++p)
+#pragma unroll
+    for (int x = 0; x < 3; ++x)
+      gv[3 * p + x] = fmaf(Rm[3 * x], vp[3 * p], fmaf(Rm[3 * x + 1], vp[3 * p + 1], Rm[3 * x + 2] * vp[3 * p + 2])) + tc[x];
+
+  // rows are built and stored one after the other to keep few values live
+  float sq[3] = {0.f, 0.f, 0.f}, sk[3] = {0.f, 0.f, 0.f}, nk = 0.f;
+#pragma unroll
+  for (int e = 0; e < 3 * PQ; ++e) {
+    sq[e % 3] += gq[e];
+    sk[e % 3] += gk[e];
+    nk = fmaf(gk[e], gk[e], nk);
+  }
+  bool overflow = false;
+  auto store_row = [&](uint4* dst, auto value_of) {
+#pragma unroll
+    for (int u = 0; u < DH / 8; ++u) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w[e] = valid ? pack_half2(value_of(8 * u + 2 * e), value_of(8 * u + 2 * e + 1)) : 0u;
+        // |x| >= 65520 rounds to infinity in fp16 (exponent field all ones)
+        overflow |= ((w[e] & 0x7c00u) == 0x7c00u) || ((w[e] & 0x7c000000u) == 0x7c000000u);
+      }
+      dst[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  };
+  auto hi_of = [](float x) { return __half2float(__float2half_rn(x)); };
+  // Q_h: [ scaled q | gq' hi | gq' hi | gq' lo | -1 -1 | 0 ]
+  store_row(a.qh + t * 8, [&](int col) -> float {
+    if (col < C) return a.qscale * qs[col];
+    if (col < C + 9 * PQ) {
+      const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
+      const float hi = hi_of(gq[e]);
+      return part < 2 ? hi : gq[e] - hi;
+    }
+    return col < C + 9 * PQ + 2 ? -1.f : 0.f;
+  });
+  // K_h: [ k | 2c gk' hi | lo | hi | c|gk'|^2 hi, lo | 0 ]
+  store_row(a.kh + t * 8, [&](int col) -> float {
+    if (col < C) return ks[col];
+    if (col < C + 9 * PQ) {
+      const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
+      const float g = 2.f * c * gk[e], hi = hi_of(g);
+      return part == 1 ? g - hi : hi;
+    }
+    if (col < C + 9 * PQ + 2) {
+      const float n = c * nk, hi = hi_of(n);
+      return col == C + 9 * PQ ? hi : n - hi;
+    }
+    return 0.f;
+  });
+  // V_h: [ v | gv hi | gv lo ]
+  store_row(a.vh + t * 8, [&](int col) -> float {
+    if (col < C) return vs[col];
+    if (col < C + 6 * PV) {
+      const int u = col - C, part = u / (3 * PV), e = u % (3 * PV);
+      const float hi = hi_of(gv[e]);
+      return part == 0 ? hi : gv[e] - hi;
+    }
+    return 0.f;
+  });
+  if (!valid) {
+    sq[0] = sq[1] = sq[2] = 0.f;
+    sk[0] = sk[1] = sk[2] = 0.f;
+  }
+  a.rowq[t] = make_float4(sq[0], sq[1], sq[2], 0.f);
+  a.colk[t] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
+  if (overflow) record_error(a.err, DEV_NONFINITE);
+}
+
+}  // namespace
+
+cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
+  unsigned char* ws = a.ws;
+  const IpaWorkspace& w = a.lay;
+
+  TileArgs ta{};
+  ta.B = a.B; ta.L = a.L; ta.R = a.R; ta.Cz = a.Cz; ta.RCz = a.RCz; ta.DZ = a.DZ; ta.nkt = a.nkt;
+  ta.rot = a.rot; ta.trans = a.trans; ta.mask = a.mask; ta.z1 = a.z1; ta.z2 = a.z2;
+  ta.frame = reinterpret_cast<float4*>(ws + w.frame);
+  ta.part = reinterpret_cast<float4*>(ws + w.part);
+  ta.z1f = reinterpret_cast<float*>(ws + w.z1f);
+  ta.z2h = reinterpret_cast<__half*>(ws + w.z2);
+  ipa_tile_kernel<<<dim3(a.nkt, a.B, a.DZ / 64), 256, 0, stream>>>(ta);
+
+  ReduceArgs ra{};
+  ra.B = a.B; ra.L = a.L; ra.H = a.H; ra.Cz = a.Cz; ra.RCz = a.RCz; ra.DZ = a.DZ; ra.nqt = a.nqt; ra.nkt = a.nkt;
+  ra.w_L = a.w_L; ra.w_C = a.w_C; ra.gamma = a.gamma; ra.w_bias = a.w_bias;
+  ra.part = ta.part;
+  ra.cen = reinterpret_cast<float4*>(ws + w.cen);
+  ra.oq = reinterpret_cast<float4*>(ws + w.oq);
+  ra.ok = reinterpret_cast<float4*>(ws + w.ok);
+  ra.headc = reinterpret_cast<float*>(ws + w.headc);
+  ra.wqp = reinterpret_cast<float*>(ws + w.wqp);
+  ipa_reduce_kernel<<<a.B, 256, 0, stream>>>(ra);
+
+  RowArgs r{};
+  r.B = a.B; r.L = a.L; r.H = a.H; r.nqt = a.nqt; r.nkt = a.nkt;
+  r.qscale = kLog2e * a.w_L * a.scalar_scale;
+  r.q = a.q; r.k = a.k; r.v = a.v; r.q_pts = a.q_pts; r.k_pts = a.k_pts; r.v_pts = a.v_pts;
+  r.frame = ta.frame; r.cen = ra.cen; r.oq = ra.oq; r.ok = ra.ok; r.headc = ra.headc;
+  r.qh = reinterpret_cast<uint4*>(ws + w.qh);
+  r.kh = reinterpret_cast<uint4*>(ws + w.kh);
+  r.vh = reinterpret_cast<uint4*>(ws + w.vh);
+  r.rowq = reinterpret_cast<float4*>(ws + w.rowq);
+  r.colk = reinterpret_cast<float4*>(ws + w.colk);
+  r.err = a.err;
+  const int64_t n = static_cast<int64_t>(a.B) * a.H * a.L;
+  ipa_rows_kernel<IPA_C, IPA_PQ, IPA_PV><<<static_cast<unsigned>((n + 127) / 128), 128, 0, stream>>>(r);
+  return cudaGetLastError();
+}
+
+IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz) {
+  (void)RCz;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  IpaWorkspace w{};
+  size_t o = 0;
+  const size_t bhl = static_cast<size_t>(B) * H * L, bl = static_cast<size_t>(B) * L;
+  const int nqt = (L + QT - 1) / QT, nkt = (L + KT - 1) / KT;
+  w.qh = o; o = up(o + bhl * DH * 2);
+  w.kh = o; o = up(o + bhl * DH * 2);
+  w.vh = o; o = up(o + bhl * DH * 2);
+  w.z2 = o; o = up(o + bl * DZ * 2);
+  w.z1f = o; o = up(o + bl * DZ * 4);
+  w.rowq = o; o = up(o + bhl * 16);
+  w.colk = o; o = up(o + bhl * 16);
+  w.frame = o; o = up(o + bl * 64);
+  w.part = o; o = up(o + static_cast<size_t>(B) * nkt * 16);
+  w.cen = o; o = up(o + static_cast<size_t>(B) * 16);
+  w.oq = o; o = up(o + static_cast<size_t>(B) * nqt * 16);
+  w.ok = o; o = up(o + static_cast<size_t>(B) * nkt * 16);
+  w.headc = o; o = up(o + static_cast<size_t>(H) * 4);
+  w.wqp = o; o = up(o + static_cast<size_t>(H) * DZ * 4);
+  w.err = o; o = up(o + 16);
+  w.total = o;
+  return w;
+}
+
+}  // namespace fipa

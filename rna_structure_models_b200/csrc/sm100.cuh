@@ -247,6 +247,16 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Round a non-negative fp32 value to the nearest value with an fp16-sized
+// significand (10 explicit bits), ties to even, using integer operations
+// only.  For values in fp16's normal range this is exactly the value that a
+// round-to-nearest fp32 -> fp16 conversion produces.
+__device__ __forceinline__ float round_f16_precision(float x) {
+  const uint32_t u = __float_as_uint(x);
+  const uint32_t r = (u + 0x0FFFu + ((u >> 13) & 1u)) & 0xFFFFE000u;
+  return __uint_as_float(r);
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);

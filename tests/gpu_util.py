@@ -1,5 +1,7 @@
 """Helpers shared by the GPU tests: move seeded inputs to the device and
 compare against the oracle with the tolerances the fused path is held to."""
+import os
+
 import numpy as np
 import torch
 
@@ -37,5 +39,9 @@ def errors(gpu, ref):
 def assert_parity(gpu, ref, max_abs=IPA_MAX_ABS, rel_fro=IPA_REL_FRO, what=""):
     assert np.all(np.isfinite(gpu)), f"{what}: non-finite values"
     m, r = errors(gpu, ref)
+    log = os.environ.get("PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(f"{what}\tmax_abs={m:.3e}\trel_fro={r:.3e}\tbound=({max_abs}, {rel_fro})\n")
     assert m <= max_abs and r <= rel_fro, f"{what}: max-abs {m:.3e} (<= {max_abs}), rel-Fro {r:.3e} (<= {rel_fro})"
     return m, r
