@@ -41,7 +41,8 @@ UNIT = "TFLOP/s"
 
 # DRAM traffic of one launch of the core kernel from an ncu capture, valid only
 # for the kernel source it was taken on (sha256 of csrc/ipa_attention.cu).
-NCU_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None}
+NCU_TRAFFIC = {"kernel_sha256": "ea1ad3fdcdd7547ea56f59b3ac154dcb3403459fea25f67214690e2068a35b48",
+               "bytes_per_launch": 28.86e6}
 
 
 def ipa_flops(B, L, n_valid=None):
