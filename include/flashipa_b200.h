@@ -195,6 +195,44 @@ IPA_API ipa_status_t geo_attn_fwd(const geo_params_t* p,
                           void* workspace, size_t workspace_bytes,
                           void* stream, int32_t* dev_err);
 
+/* --------------------------------------------------------------------------
+ * geo_attn_fwd without a workspace argument (no counterpart on the pages:
+ * this is an interface convenience of this library, not part of the method).
+ *
+ * For callers that may not allocate device memory where they run this
+ * operator -- e.g. an operator hook inside a host framework that provides no
+ * scratch buffer and forbids cudaMalloc on that path, or a plain C program
+ * linking this library without an allocator.  It allocates nothing: its
+ * scratch is a fixed array of GEO_STATIC_SCRATCH_BYTES inside this library,
+ * reserved on every GPU that loads the library until the process exits.
+ *   - Same arguments, results and errors as geo_attn_fwd, minus the
+ *     workspace; returns IPA_ERR_WORKSPACE when geo_attn_workspace_size(p)
+ *     exceeds GEO_STATIC_SCRATCH_BYTES (e.g. B*H*N above roughly 64 K rows
+ *     of 128 bytes for M = 4).
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress); make that first call outside any stream
+ *     capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents: calls whose executions overlap on the GPU (other
+ *     streams, other host threads) race on it and must be serialised by the
+ *     caller.  Every byte a call reads from it is written earlier in the same
+ *     call.
+ * ------------------------------------------------------------------------ */
+#define GEO_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+IPA_API ipa_status_t geo_attn_fwd_static(const geo_params_t* p,
+                                 const ipa_tensor_t* q_direction, const ipa_tensor_t* k_direction,
+                                 const ipa_tensor_t* q_point, const ipa_tensor_t* k_point,
+                                 const ipa_tensor_t* values,
+                                 const ipa_tensor_t* direction_scale,
+                                 const ipa_tensor_t* distance_scale,
+                                 const ipa_tensor_t* output_weight, const ipa_tensor_t* output_bias,
+                                 const ipa_tensor_t* rotation, const ipa_tensor_t* translation,
+                                 const ipa_tensor_t* frame_mask, const ipa_tensor_t* pair_mask,
+                                 const ipa_tensor_t* out_vectors, const ipa_tensor_t* out_output,
+                                 const ipa_tensor_t* out_attention,
+                                 void* stream, int32_t* dev_err);
+
 /* Static description of a status code (never NULL). */
 IPA_API const char* ipa_status_string(ipa_status_t s);
 

@@ -22,7 +22,7 @@ STATUS = {0: "IPA_OK", 1: "IPA_ERR_NULL", 2: "IPA_ERR_SHAPE", 3: "IPA_ERR_STRIDE
           4: "IPA_ERR_DTYPE", 5: "IPA_ERR_WORKSPACE", 6: "IPA_ERR_UNSUPPORTED", 7: "IPA_ERR_CUDA",
           8: "IPA_ERR_TIMEOUT"}
 EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa_attn_core",
-            "geo_attn_workspace_size", "geo_attn_fwd", "ipa_status_string",
+            "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static", "ipa_status_string",
             "ipa_device_error_status", "ipa_version")
 
 
