@@ -96,7 +96,8 @@ bool geo_dims_ok(const geo_params_t* p, ipa_status_t* st) {
 }  // namespace
 
 bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1) {
+                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                        int swizzle_bytes) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
@@ -104,7 +105,8 @@ bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_
   const cuuint32_t box[3] = {box0, box1, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -343,5 +345,8 @@ ipa_status_t geo_attn_fwd(const geo_params_t* p, const ipa_tensor_t* q_direction
 // Tracing build only: copy the per-tile event timestamps to the host.
 extern "C" __attribute__((visibility("default"))) int ipa_trace_copy(void* host, size_t bytes) {
   return fipa::ipa_trace_read(host, bytes) ? 0 : 1;
+}
+extern "C" __attribute__((visibility("default"))) int ipa_pair_trace_copy(void* host, size_t bytes) {
+  return fipa::ipa_pair_trace_read(host, bytes) ? 0 : 1;
 }
 #endif

@@ -70,8 +70,16 @@ bool ipa_trace_read(void* host, size_t bytes);
 #endif
 
 // cuTensorMapEncodeTiled obtained through the runtime's driver entry point.
+// swizzle_bytes: 128 or 64 (the inner box must then be exactly that many bytes).
 bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                         uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
-                        uint32_t box0, uint32_t box1);
+                        uint32_t box0, uint32_t box1, int swizzle_bytes = 128);
+
+// CTA-pair core kernel (cta_group::2): pair-dimension widths it supports and its launch.
+bool ipa_pair_supported(int DZ);
+cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream);
+#ifdef IPA_TRACE
+bool ipa_pair_trace_read(void* host, size_t bytes);
+#endif
 
 }  // namespace fipa

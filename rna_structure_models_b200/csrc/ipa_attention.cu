@@ -31,6 +31,8 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -530,7 +532,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace
 
+// FLASHIPA_CORE=single forces the single-CTA kernel (for comparisons); by
+// default the CTA-pair kernel runs whenever it supports the pair width.
+static bool force_single_cta() {
+  static const bool v = [] {
+    const char* e = std::getenv("FLASHIPA_CORE");
+    return e != nullptr && std::strcmp(e, "single") == 0;
+  }();
+  return v;
+}
+
 cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream) {
+  if (ipa_pair_supported(a.DZ) && !force_single_cta()) return ipa_launch_core_pair(a, stream);
   unsigned char* ws = a.ws;
   const IpaWorkspace& w = a.lay;
   CUtensorMap tqh, tkh, tvh, tz2;

@@ -1,0 +1,598 @@
+// Fused attention pass of the IPA core on a CTA pair (cta_group::2).
+//
+// A cluster of two CTAs owns 256 query rows of one (batch, head); CTA r of
+// the pair owns rows [256 I + 128 r, +128).  Key tiles are 128 keys.  The MMAs
+// are issued by one thread of CTA 0 for both CTAs (M = 256): each CTA
+// supplies its own 128 rows of A and HALF of every B operand from its own
+// shared memory, which halves the per-CTA shared-memory footprint and the
+// operand traffic of a key tile and allows N = 128 keys per Q.K^T MMA
+// (N = 64 MMAs run well below the tensor rate on this GPU).
+//
+//   S = [Q_h | Q_pair] . [K_h | Z2]^T      N = 128: CTA r supplies keys [64 r, 64 r + 64)
+//   O_pair += P . Z2                        N = DZ: CTA r supplies features [r DZ/2, (r+1) DZ/2)
+//   O_v    += P . V_h                       N = 64: CTA r supplies V_h columns [32 r, 32 r + 32)
+//
+// P (fp16, 128 keys) lives in tensor memory and is the A operand of the P.V
+// MMAs.  Per CTA, tensor memory: O_pair [0, DZ) | O_v [DZ, DZ+64) | S [320, 448)
+// | P [448, 512); shared memory: Q_h 16 KB | Q_pair DZ*256 B | 2 x K slot
+// (own 64 keys: K_h 8 KB + Z2 DZ*128 B) | 1 x V slot (all 128 keys: own Z2
+// panels DZ*128 B + own V_h columns 8 KB, 64-byte swizzle).
+//
+// Synchronisation: barriers the MMA thread waits on live in CTA 0 (K/V slots
+// full: TMA bytes of both CTAs; S read and P written: one arrival per softmax
+// warp of both CTAs); barriers the softmax and producer warps wait on live in
+// each CTA and are signalled by multicast tcgen05.commit.  Every wait is
+// bounded (2 s) and reports into the error word.
+//
+// The softmax, lazy rescaling, rounded row sums, tile-local point terms and
+// the epilogue are those of the single-CTA kernel (ipa_attention.cu).
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+#ifdef IPA_TRACE
+__device__ unsigned long long g_pair_trace[2][64][32];
+#define PAIR_TR(j, ev)                                                               \
+  do {                                                                               \
+    if (trace_slot >= 0 && (j) < 64) g_pair_trace[trace_slot][(j)][(ev)] = clock64(); \
+  } while (0)
+#else
+#define PAIR_TR(j, ev) \
+  do {                 \
+  } while (0)
+#endif
+
+namespace fipa {
+
+using namespace sm100;
+
+namespace {
+
+struct PairArgs {
+  int B, L, H, DZ, RCz, Cz, nqt, nkt, nqp, nkp, F;  // nqt/nkt: 128-row / 64-key tiles; nqp/nkp: 256 / 128
+  float tau;
+  const float4* rowq;
+  const float4* colk;
+  const float4* oq;     // [B, nqt]   128-row query tile origins
+  const float4* ok;     // [B, nkt]   64-key tile origins
+  const float4* cen;
+  const float* headc;
+  const float* wqp;     // [H, DZ]
+  const float4* frame;
+  const float* z1f;     // [B, L, DZ]
+  float* out;
+  int* err;
+  int trace_cta0, trace_cta1;
+};
+
+constexpr int NT = 320;            // 8 softmax warps, producer warp, MMA warp
+constexpr int NSOFT = 256;
+constexpr int W_PROD = 8, W_MMA = 9;
+constexpr int NCOL = 4;            // column-term ring
+
+// shared memory (offsets from a 1024-byte aligned base)
+constexpr uint32_t SP_QH = 0;
+constexpr uint32_t SP_QP = 16384;                 // DZ/64 panels x 16 KB
+constexpr uint32_t KSLOT = 8192 + 4 * 8192;       // K_h half + Z2 half (<= 4 panels)
+constexpr uint32_t SP_K = SP_QP + 4 * 16384;      // 2 slots
+constexpr uint32_t SP_V = SP_K + 2 * KSLOT;       // Z2 own panels (<= 2 x 16 KB) | V_h 8 KB
+constexpr uint32_t V_VH = 32768;
+constexpr uint32_t VSLOT = V_VH + 8192;
+constexpr uint32_t SP_AUX = SP_V + VSLOT;
+constexpr uint32_t AX_COL = 0;                    // float [NCOL][128]
+constexpr uint32_t AX_D = 2048;                   // float4 [NCOL][2]
+constexpr uint32_t AX_XCH = 2304;                 // float [2][2][128] maxima + [2][128] sums
+constexpr uint32_t AX_BAR = 5376;
+constexpr uint32_t SP_BYTES = SP_AUX + 6144;
+constexpr uint32_t SP_ALLOC = SP_BYTES + 1024;
+
+enum {
+  // local barriers (waited on in each CTA)
+  P_QFULL = 0, P_SFULL, P_PFREE, P_KEMPTY0, P_VEMPTY = P_KEMPTY0 + 2, P_COLFULL0, P_DRAIN = P_COLFULL0 + NCOL,
+  // barriers waited on by the MMA thread (used in CTA 0)
+  P_KFULL0, P_VFULL = P_KFULL0 + 2, P_SFREE, P_PFULL, P_QREADY, P_COUNT
+};
+constexpr uint32_t AX_TMEM = AX_BAR + 8 * P_COUNT;
+constexpr uint32_t AX_ABORT = AX_TMEM + 8;
+
+constexpr uint32_t TM_S = 320, TM_P = 448, TM_COLS = 512;
+
+__device__ __forceinline__ uint64_t k128(uint32_t a) { return smem_desc(a, 16, 1024, 2); }           // K-major SW128
+__device__ __forceinline__ uint64_t mn128(uint32_t a) { return smem_desc(a, 16384, 1024, 2); }       // MN-major SW128, 16 KB panels
+__device__ __forceinline__ uint64_t mn64(uint32_t a) { return smem_desc(a, 16384, 512, 4); }         // MN-major SW64
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
+    ipa_attention_pair_kernel(const __grid_constant__ CUtensorMap tm_qh,
+                              const __grid_constant__ CUtensorMap tm_kh,
+                              const __grid_constant__ CUtensorMap tm_z2k,
+                              const __grid_constant__ CUtensorMap tm_z2v,
+                              const __grid_constant__ CUtensorMap tm_vh, const PairArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (sb - raw_u32);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int I2 = pair % a.nqp;
+  const int bh = pair / a.nqp;
+  const int b = bh / a.H, h = bh % a.H;
+  const int L = a.L, nt = a.nkp, DZ = a.DZ, np = DZ / 64;
+  const int row0 = 256 * I2 + 128 * static_cast<int>(rank);   // first query row of this CTA
+  const int I = row0 / QT;                                      // its 128-row query tile
+#ifdef IPA_TRACE
+  const int trace_slot = (blockIdx.x == a.trace_cta0) ? 0 : (blockIdx.x == a.trace_cta1) ? 1 : -1;
+#endif
+
+  float* col_s = reinterpret_cast<float*>(smem + SP_AUX + AX_COL);
+  float4* dinfo = reinterpret_cast<float4*>(smem + SP_AUX + AX_D);
+  float* xch = reinterpret_cast<float*>(smem + SP_AUX + AX_XCH);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SP_AUX + AX_ABORT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SP_AUX + AX_TMEM);
+  auto bar = [&](int k) -> uint32_t { return sb + SP_AUX + AX_BAR + 8u * k; };
+  auto bar0 = [&](int k) -> uint32_t { return mapa_shared(bar(k), 0); };   // the barrier in CTA 0
+
+  if (tid == 0) {
+    mbar_init(bar(P_QFULL), 1);
+    mbar_init(bar(P_SFULL), 1);
+    mbar_init(bar(P_PFREE), 1);
+    mbar_init(bar(P_KEMPTY0), 1);
+    mbar_init(bar(P_KEMPTY0 + 1), 1);
+    mbar_init(bar(P_VEMPTY), 1);
+    for (int s = 0; s < NCOL; ++s) mbar_init(bar(P_COLFULL0 + s), 1);
+    mbar_init(bar(P_DRAIN), 1);
+    mbar_init(bar(P_KFULL0), 2);
+    mbar_init(bar(P_KFULL0 + 1), 2);
+    mbar_init(bar(P_VFULL), 2);
+    mbar_init(bar(P_SFREE), 16);
+    mbar_init(bar(P_PFULL), 16);
+    mbar_init(bar(P_QREADY), 2);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == W_MMA) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == W_PROD && lane == 0) {
+    tma_prefetch_desc(&tm_qh);
+    tma_prefetch_desc(&tm_kh);
+    tma_prefetch_desc(&tm_z2k);
+    tma_prefetch_desc(&tm_z2v);
+    tma_prefetch_desc(&tm_vh);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&](int code) {
+    record_error(a.err, code);
+    *abort_flag = 1;
+  };
+  const int start = (2 * I2) % nt;   // diagonal key tile first
+
+  if (warp == W_PROD) {
+    // ------------------------------------------------ producer (each CTA)
+    const float4 oqv = a.oq[b * a.nqt + (I < a.nqt ? I : a.nqt - 1)];
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(P_QFULL), 16384);
+      tma_load_3d(sb + SP_QH, &tm_qh, bar(P_QFULL), 0, row0, bh);
+    }
+    const uint32_t kbytes = 8192u + static_cast<uint32_t>(np) * 8192u;
+    const uint32_t vbytes = static_cast<uint32_t>(np / 2) * 16384u + 8192u;
+    auto load_k = [&](int j) {
+      const int J2 = (start + j) % nt;
+      const int s = j & 1;
+      // column terms of this CTA's rows for the 128 keys of the tile
+      const int cs = j % NCOL;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int kk = lane + 32 * t;
+        const int key = J2 * 128 + kk;
+        float cv = -INFINITY;
+        if (key < L) {
+          const float4 okv = a.ok[b * a.nkt + key / KT];
+          const float4 ck = a.colk[static_cast<int64_t>(bh) * L + key];
+          cv = ck.w - fmaf(ck.x, okv.x - oqv.x, fmaf(ck.y, okv.y - oqv.y, ck.z * (okv.z - oqv.z)));
+        }
+        col_s[cs * 128 + kk] = cv;
+      }
+      if (lane < 2) {
+        const int jt = 2 * J2 + lane;
+        const float4 okv = jt < a.nkt ? a.ok[b * a.nkt + jt] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float dx = okv.x - oqv.x, dy = okv.y - oqv.y, dz = okv.z - oqv.z;
+        dinfo[cs * 2 + lane] = make_float4(dx, dy, dz, fmaf(dx, dx, fmaf(dy, dy, dz * dz)));
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(P_COLFULL0 + cs));
+        const uint32_t kf = bar0(P_KFULL0 + s);
+        const uint32_t st = sb + SP_K + s * KSLOT;
+        const int krow = J2 * 128 + 64 * static_cast<int>(rank);
+        mbar_arrive_expect_tx_cluster(kf, kbytes);
+        tma_load_3d_pair(st, &tm_kh, kf, 0, krow, bh);
+        for (int p = 0; p < np; ++p) tma_load_3d_pair(st + 8192 + 8192 * p, &tm_z2k, kf, 64 * p, krow, b);
+        PAIR_TR(j, 13);
+      }
+      __syncwarp();
+    };
+    auto load_v = [&](int j) {
+      const int J2 = (start + j) % nt;
+      if (lane == 0) {
+        const uint32_t vf = bar0(P_VFULL);
+        const uint32_t st = sb + SP_V;
+        mbar_arrive_expect_tx_cluster(vf, vbytes);
+        for (int p = 0; p < np / 2; ++p)
+          tma_load_3d_pair(st + 16384 * p, &tm_z2v, vf, 64 * (static_cast<int>(rank) * (np / 2) + p), J2 * 128, b);
+        tma_load_3d_pair(st + V_VH, &tm_vh, vf, 32 * static_cast<int>(rank), J2 * 128, bh);
+        PAIR_TR(j, 14);
+      }
+      __syncwarp();
+    };
+    auto wait_local = [&](int barid, uint32_t parity, int code) -> bool {
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait_bounded(bar(barid), parity, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok && lane == 0) fail(code);
+      return ok != 0;
+    };
+    // K(0), K(1), V(0); then per tile j >= 1: K(j+1) (after QK(j-1)), V(j) (after PV(j-1))
+    load_k(0);
+    if (nt > 1) load_k(1);
+    load_v(0);
+    for (int j = 1; j < nt; ++j) {
+      if (j + 1 < nt) {
+        if (!wait_local(P_KEMPTY0 + ((j + 1) & 1), ((j - 1) >> 1) & 1, DEV_TIMEOUT_EMPTY)) break;
+        load_k(j + 1);
+      }
+      if (!wait_local(P_VEMPTY, (j - 1) & 1, DEV_TIMEOUT_EMPTY)) break;
+      load_v(j);
+    }
+  } else if (warp == W_MMA) {
+    // ------------------------------------------------ MMA issuer (CTA 0, one thread)
+    if (rank == 0 && lane == 0) {
+      bool ok = mbar_wait_bounded_cluster(bar(P_QREADY), 0, abort_flag);
+      if (!ok) fail(DEV_TIMEOUT_SOFTMAX);
+      tc_fence_after();
+      const uint32_t idq = idesc_f16(256, 128, false);
+      const uint32_t idz = idesc_f16(256, DZ, true);
+      const uint32_t idv = idesc_f16(256, 64, true);
+      const uint32_t tS = tmem + TM_S, tP = tmem + TM_P, tOz = tmem, tOv = tmem + DZ;
+      bool issued_any = false;
+      for (int j = 0; ok && j <= nt; ++j) {
+        if (j < nt) {
+          const int s = j & 1;
+          ok = mbar_wait_bounded_cluster(bar(P_KFULL0 + s), (j >> 1) & 1, abort_flag);
+          PAIR_TR(j, 0);
+          if (ok && j > 0) ok = mbar_wait_bounded_cluster(bar(P_SFREE), (j - 1) & 1, abort_flag);
+          PAIR_TR(j, 1);
+          if (!ok) { fail(DEV_TIMEOUT_FULL); break; }
+          tc_fence_after();
+          const uint32_t st = sb + SP_K + s * KSLOT;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma2_ss(tS, k128(sb + SP_QH + 32 * k), k128(st + 32 * k), idq, k > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4 * np; ++kk)
+            umma2_ss(tS, k128(sb + SP_QP + 16384 * (kk >> 2) + 32 * (kk & 3)),
+                     k128(st + 8192 + 8192 * (kk >> 2) + 32 * (kk & 3)), idq, 1u);
+          umma2_commit_both(bar(P_SFULL));
+          umma2_commit_both(bar(P_KEMPTY0 + s));
+          PAIR_TR(j, 2);
+          issued_any = true;
+        }
+        if (j > 0) {
+          const int jj = j - 1;
+          ok = mbar_wait_bounded_cluster(bar(P_PFULL), jj & 1, abort_flag);
+          if (ok) ok = mbar_wait_bounded_cluster(bar(P_VFULL), jj & 1, abort_flag);
+          PAIR_TR(jj, 3);
+          if (!ok) { fail(DEV_TIMEOUT_SOFTMAX); break; }
+          tc_fence_after();
+          const uint32_t st = sb + SP_V;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
+            umma2_ts(tOz, tP + 8 * k, mn128(st + 2048 * k), idz, acc);
+            umma2_ts(tOv, tP + 8 * k, mn64(st + V_VH + 1024 * k), idv, acc);
+          }
+          umma2_commit_both(bar(P_PFREE));
+          umma2_commit_both(bar(P_VEMPTY));
+          PAIR_TR(jj, 4);
+        }
+      }
+      if (!ok && issued_any) {
+        umma2_commit_both(bar(P_DRAIN));
+        mbar_wait_bounded(bar(P_DRAIN), 0, nullptr, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------ softmax + epilogue (256 threads)
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const int row = row0 + r;
+    const bool in_range = row < L;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t pair_bar = 2 + quarter;
+    const float ch = a.headc[h];
+    const float4 sq = in_range ? a.rowq[static_cast<int64_t>(bh) * L + row] : make_float4(0, 0, 0, 0);
+    const float pq = static_cast<float>(IPA_PQ);
+    const int tev = (tid == 0) ? 0 : (tid == 96) ? 1 : -1;
+    (void)tev;
+
+    // Q_pair rows (log2(e) w_L w_bias[:, h] * z1_i) into shared memory, 128-byte
+    // swizzled K-major panels; this thread writes half of the panels of row r
+    {
+      const float* zr = a.z1f + (static_cast<int64_t>(b) * L + (in_range ? row : 0)) * DZ;
+      const float* wr = a.wqp + static_cast<int64_t>(h) * DZ;
+      for (int p = half * (np / 2); p < (half + 1) * (np / 2); ++p) {
+        unsigned char* prow = smem + SP_QP + 16384 * p + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 z0 = in_range ? *reinterpret_cast<const float4*>(zr + 64 * p + 8 * c) : make_float4(0, 0, 0, 0);
+          const float4 z1 = in_range ? *reinterpret_cast<const float4*>(zr + 64 * p + 8 * c + 4) : make_float4(0, 0, 0, 0);
+          const float4 w0 = *reinterpret_cast<const float4*>(wr + 64 * p + 8 * c);
+          const float4 w1 = *reinterpret_cast<const float4*>(wr + 64 * p + 8 * c + 4);
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+              make_uint4(pack_half2(z0.x * w0.x, z0.y * w0.y), pack_half2(z0.z * w0.z, z0.w * w0.w),
+                         pack_half2(z1.x * w1.x, z1.y * w1.y), pack_half2(z1.z * w1.z, z1.w * w1.w));
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, NSOFT);
+      if (tid == 0) {
+        const bool okq = mbar_wait_bounded(bar(P_QFULL), 0, abort_flag);
+        if (!okq) fail(DEV_TIMEOUT_FULL);
+        mbar_arrive_cluster(bar0(P_QREADY));
+      }
+    }
+
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    const int OW = DZ + 64;
+    const int o_lo = half * (OW / 2), o_hi = o_lo + OW / 2;
+    for (int j = 0; j < nt && ok; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_SFULL), j & 1, abort_flag))) {
+        if (lane == 0) fail(DEV_TIMEOUT_MMA);
+        ok = false;
+        break;
+      }
+      if (tev >= 0) PAIR_TR(j, tev ? 26 : 16);
+      tc_fence_after();
+      uint32_t sr[64];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tmem + TM_S + 64 * half + lane_off, r0);
+        tmem_ld32(tmem + TM_S + 64 * half + 32 + lane_off, r1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) { sr[e] = r0[e]; sr[32 + e] = r1[e]; }
+      }
+      tc_fence_before();
+      if (tid == 0) PAIR_TR(j, 17);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(bar0(P_SFREE));
+      if (tid == 0) PAIR_TR(j, 18);
+      const int cs = j % NCOL;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_COLFULL0 + cs), (j / NCOL) & 1, abort_flag))) {
+        if (lane == 0) fail(DEV_TIMEOUT_FULL);
+        ok = false;
+        break;
+      }
+      if (tid == 0) PAIR_TR(j, 19);
+      const float4* colv = reinterpret_cast<const float4*>(col_s + cs * 128 + 64 * half);
+      const float4 dd = dinfo[cs * 2 + half];
+      const float rt = ch * (2.f * fmaf(sq.x, dd.x, fmaf(sq.y, dd.y, sq.z * dd.z)) - pq * dd.w);
+      float x[64];
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int k4 = 0; k4 < 16; ++k4) {
+        const float4 cv = colv[k4];
+        x[4 * k4 + 0] = __uint_as_float(sr[4 * k4 + 0]) + cv.x;
+        x[4 * k4 + 1] = __uint_as_float(sr[4 * k4 + 1]) + cv.y;
+        x[4 * k4 + 2] = __uint_as_float(sr[4 * k4 + 2]) + cv.z;
+        x[4 * k4 + 3] = __uint_as_float(sr[4 * k4 + 3]) + cv.w;
+        mx4[0] = fmaxf(mx4[0], x[4 * k4 + 0]);
+        mx4[1] = fmaxf(mx4[1], x[4 * k4 + 1]);
+        mx4[2] = fmaxf(mx4[2], x[4 * k4 + 2]);
+        mx4[3] = fmaxf(mx4[3], x[4 * k4 + 3]);
+      }
+      // this half's max in full logit units (the row term differs between the key halves)
+      const float mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) + rt;
+      float* xb = xch + (j & 1) * 256;
+      xb[half * 128 + r] = mine;
+      if (tid == 0) PAIR_TR(j, 20);
+      named_bar_sync(pair_bar, 64);
+      if (tid == 0) PAIR_TR(j, 21);
+      const float mt = fmaxf(mine, xb[(1 - half) * 128 + r]);
+      const bool need = mt > m_used + a.tau;
+      const bool resc = need && (m_used != -INFINITY);
+      const float scale = resc ? ex2(m_used - mt) : 1.f;
+      if (need) m_used = mt;
+      l *= scale;
+      const float base = m_used - rt;
+      const bool live = m_used != -INFINITY;
+      uint32_t pk[32];
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float p0 = round_f16_precision(live ? ex2(x[2 * k] - base) : 0.f);
+        const float p1 = round_f16_precision(live ? ex2(x[2 * k + 1] - base) : 0.f);
+        pk[k] = pack_half2(p0, p1);
+        ls4[k & 3] += p0 + p1;
+      }
+      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+      if (tid == 0) PAIR_TR(j, 22);
+      // PV(j-1) must have finished reading P and accumulating O
+      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_PFREE), (j - 1) & 1, abort_flag))) {
+        if (lane == 0) fail(DEV_TIMEOUT_MMA);
+        ok = false;
+        break;
+      }
+      if (tid == 0) PAIR_TR(j, 23);
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, resc)) {
+        for (int c0 = o_lo; c0 < o_hi; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tmem + c0 + lane_off, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * scale);
+          tmem_st32(tmem + c0 + lane_off, o);
+        }
+      }
+      tmem_st32(tmem + TM_P + 32 * half + lane_off, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      if (tid == 0) PAIR_TR(j, 24);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(bar0(P_PFULL));
+      if (tid == 0) PAIR_TR(j, 25);
+      if (tid == 96) PAIR_TR(j, 27);
+    }
+
+    // ------------------------------------------------ epilogue
+    if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_PFREE), (nt - 1) & 1, abort_flag))) {
+      if (lane == 0) fail(DEV_TIMEOUT_MMA);
+      ok = false;
+    }
+    const bool all_ok = __all_sync(0xffffffffu, ok);
+    xch[512 + half * 128 + r] = l;
+    named_bar_sync(pair_bar, 64);
+    const float lt = l + xch[512 + (1 - half) * 128 + r];
+    const float4 f3 = a.frame[(static_cast<int64_t>(b) * L + (in_range ? row : 0)) * 4 + 3];
+    const bool dead = !(in_range && f3.x != 0.f && lt > 0.f);
+    const int pitch = OW + 4;
+    float* stage = reinterpret_cast<float*>(smem + SP_QP);
+    if (all_ok) {
+      tc_fence_after();
+      const float inv = dead ? 0.f : 1.f / lt;
+      float* orow = stage + r * pitch;
+      // staged row layout: [O_v (64) | O_pair (DZ)]; tensor memory holds [O_pair | O_v]
+      for (int c0 = o_lo; c0 < o_hi; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(tmem + c0 + lane_off, o);
+        tmem_ld_wait();
+        const int dstc = c0 < DZ ? 64 + c0 : c0 - DZ;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(orow + dstc + e) =
+              make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                          __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+      }
+      if (half == 0) orow[OW] = dead ? 1.f : 0.f;
+    }
+    tc_fence_before();
+    named_bar_sync(1, NSOFT);
+    if (!*abort_flag) {
+      const int C = IPA_C, Pv = IPA_PV, Cz = a.Cz, R = a.RCz / a.Cz;
+      const int F = a.F;
+      const float4 cn = a.cen[b];
+      for (int rr = 0; rr < 16; ++rr) {
+        const int rloc = warp * 16 + rr;
+        const int grow = row0 + rloc;
+        if (grow >= L) break;
+        const float* O = stage + rloc * pitch;
+        const bool rdead = O[OW] != 0.f;
+        const float4* fg = a.frame + (static_cast<int64_t>(b) * L + grow) * 4;
+        const float4 g0 = fg[0], g1 = fg[1], g2 = fg[2];
+        const float Rm[9] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w, g2.x};
+        const float tcx[3] = {g2.y - cn.x, g2.z - cn.y, g2.w - cn.z};
+        float* dst = a.out + ((static_cast<int64_t>(b) * L + grow) * a.H + h) * F;
+        const float* z1r = a.z1f + (static_cast<int64_t>(b) * L + grow) * DZ;
+        for (int f = lane; f < F; f += 32) {
+          float val = 0.f;
+          if (!rdead) {
+            if (f < C) {
+              val = O[f];
+            } else if (f < C + 4 * Pv) {
+              const bool is_norm = f >= C + 3 * Pv;
+              const int p = is_norm ? f - C - 3 * Pv : (f - C) / 3;
+              float op[3];
+#pragma unroll
+              for (int xx = 0; xx < 3; ++xx) {
+                float acc = 0.f;
+#pragma unroll
+                for (int y = 0; y < 3; ++y) {
+                  const float og = O[C + 3 * p + y] + O[C + 3 * Pv + 3 * p + y];
+                  acc = fmaf(Rm[y * 3 + xx], og - tcx[y], acc);   // (R^T (og - t'))_xx
+                }
+                op[xx] = acc;
+              }
+              const int xc = (f - C) % 3;
+              val = is_norm ? sqrtf(fmaf(op[0], op[0], fmaf(op[1], op[1], op[2] * op[2])))
+                            : (xc == 0 ? op[0] : xc == 1 ? op[1] : op[2]);
+            } else {
+              const int cc = f - C - 4 * Pv;
+              for (int r2 = 0; r2 < R; ++r2) val = fmaf(z1r[r2 * Cz + cc], O[64 + r2 * Cz + cc], val);
+            }
+          }
+          dst[f] = val;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == W_MMA) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TM_COLS);
+  }
+}
+
+}  // namespace
+
+bool ipa_pair_supported(int DZ) { return DZ == 128 || DZ == 256; }
+
+cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
+  unsigned char* ws = a.ws;
+  const IpaWorkspace& w = a.lay;
+  CUtensorMap tqh, tkh, tz2k, tz2v, tvh;
+  const uint64_t bh = static_cast<uint64_t>(a.B) * a.H;
+  const uint64_t rowb = static_cast<uint64_t>(a.L) * DH * 2;
+  const uint64_t zrow = static_cast<uint64_t>(a.DZ) * 2, zb = static_cast<uint64_t>(a.L) * a.DZ * 2;
+  bool ok = encode_tmap_f16_3d(&tqh, ws + w.qh, DH, a.L, bh, DH * 2, rowb, 64, QT) &&
+            encode_tmap_f16_3d(&tkh, ws + w.kh, DH, a.L, bh, DH * 2, rowb, 64, 64) &&
+            encode_tmap_f16_3d(&tz2k, ws + w.z2, a.DZ, a.L, a.B, zrow, zb, 64, 64) &&
+            encode_tmap_f16_3d(&tz2v, ws + w.z2, a.DZ, a.L, a.B, zrow, zb, 64, 128) &&
+            encode_tmap_f16_3d(&tvh, ws + w.vh, DH, a.L, bh, DH * 2, rowb, 32, 128, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(ipa_attention_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(SP_ALLOC));
+  if (e != cudaSuccess) return e;
+  PairArgs t{};
+  t.B = a.B; t.L = a.L; t.H = a.H; t.DZ = a.DZ; t.RCz = a.RCz; t.Cz = a.Cz;
+  t.nqt = a.nqt; t.nkt = a.nkt; t.nqp = (a.L + 255) / 256; t.nkp = (a.L + 127) / 128; t.F = a.F; t.tau = 8.f;
+  t.rowq = reinterpret_cast<const float4*>(ws + w.rowq);
+  t.colk = reinterpret_cast<const float4*>(ws + w.colk);
+  t.oq = reinterpret_cast<const float4*>(ws + w.oq);
+  t.ok = reinterpret_cast<const float4*>(ws + w.ok);
+  t.cen = reinterpret_cast<const float4*>(ws + w.cen);
+  t.headc = reinterpret_cast<const float*>(ws + w.headc);
+  t.wqp = reinterpret_cast<const float*>(ws + w.wqp);
+  t.frame = reinterpret_cast<const float4*>(ws + w.frame);
+  t.z1f = reinterpret_cast<const float*>(ws + w.z1f);
+  t.out = a.out; t.err = a.err;
+  const int pairs = static_cast<int>(bh) * t.nqp;
+  t.trace_cta0 = 0;
+  t.trace_cta1 = 2 * (pairs / 2);
+  ipa_attention_pair_kernel<<<static_cast<unsigned>(2 * pairs), NT, SP_ALLOC, stream>>>(tqh, tkh, tz2k, tz2v, tvh, t);
+  return cudaGetLastError();
+}
+
+#ifdef IPA_TRACE
+bool ipa_pair_trace_read(void* host, size_t bytes) {
+  if (bytes < sizeof(g_pair_trace)) return false;
+  return cudaMemcpyFromSymbol(host, g_pair_trace, sizeof(g_pair_trace)) == cudaSuccess;
+}
+#endif
+
+}  // namespace fipa

@@ -65,14 +65,15 @@ def test_invariance_under_global_rigid_motion(cuda_device):
     assert rel <= 1e-3, rel
 
 
-@pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 127, 129, 200])
-def test_ragged_lengths(cuda_device, L):
-    inp = ipa_inputs(IpaDims(B=2, L=L, H=3, Cz=32), 3)
+@pytest.mark.parametrize("Cz", [32, 64])     # R*Cz = 64: single-CTA kernel; 128: CTA-pair kernel
+@pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 127, 129, 200, 257, 383])
+def test_ragged_lengths(cuda_device, L, Cz):
+    inp = ipa_inputs(IpaDims(B=2, L=L, H=3, Cz=Cz), 3)
     if L > 3:
         inp["mask"][1, L // 2:] = False
     gpu = run_gpu(inp)
     ref = ipa_dense(inp)
-    assert_parity(gpu, ref, what=f"L={L}")
+    assert_parity(gpu, ref, what=f"L={L} Cz={Cz}")
 
 
 def test_masks_all_masked_batch_and_single_valid(cuda_device):

@@ -24,6 +24,9 @@ def probe(cuda_device):
     lib.probe_umma.restype = ctypes.c_int
     lib.probe_bounded_wait.argtypes = [ctypes.c_void_p, ctypes.c_ulonglong, ctypes.c_void_p]
     lib.probe_bounded_wait.restype = ctypes.c_int
+    lib.probe_umma_pair.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_void_p]
+    lib.probe_umma_pair.restype = ctypes.c_int
     return lib
 
 
@@ -62,3 +65,24 @@ def test_bounded_wait_reports_instead_of_hanging(probe):
     # the context is still usable afterwards
     x = torch.ones(4, device="cuda")
     assert float((x * 2).sum()) == 8.0
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_cta_pair_building_block(probe, mode):
+    g = torch.Generator(device="cpu").manual_seed(10 + mode)
+    A = torch.randn(256, 64, generator=g).half().cuda()
+    if mode == 0:
+        B = torch.randn(128, 64, generator=g).half().cuda()     # [N, K]
+        ref = A.float() @ B.float().t()
+    else:
+        nn = 256 if mode == 1 else 64
+        B = torch.randn(64, nn, generator=g).half().cuda()      # [K, N]
+        ref = A.float() @ B.float()
+    D = torch.zeros(ref.shape, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = probe.probe_umma_pair(mode, A.data_ptr(), B.data_ptr(), D.data_ptr(), err.data_ptr(),
+                               torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert rc == 0
+    assert int(err.item()) == 0
+    assert torch.allclose(D, ref, rtol=1e-5, atol=1e-4), (D - ref).abs().max().item()
