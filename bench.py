@@ -39,10 +39,12 @@ H, C, PQ, PV, R, CZ = 12, 16, 4, 8, 2, 128
 METRIC = "fused IPA attention TFLOP/s and % bf16 tensor-pipe peak at L=4096 (1xB200)"
 UNIT = "TFLOP/s"
 
-# DRAM traffic of one launch of the core kernel from an ncu capture, valid only
-# for the kernel source it was taken on (sha256 of csrc/ipa_attention.cu).
-NCU_TRAFFIC = {"kernel_sha256": "ea1ad3fdcdd7547ea56f59b3ac154dcb3403459fea25f67214690e2068a35b48",
-               "bytes_per_launch": 28.86e6}
+# DRAM traffic of one launch of the core kernel (the CTA-pair kernel at this
+# workload's R Cz = 256) from an ncu capture, valid only for the kernel source
+# it was taken on (sha256 over the sources listed in CORE_SOURCES).
+CORE_KERNEL = "ipa_attention_pair_kernel"
+CORE_SOURCES = ("ipa_attention_pair.cu", "ipa_epilogue.cuh", "sm100.cuh")
+NCU_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None}
 
 
 def ipa_flops(B, L, n_valid=None):
@@ -53,9 +55,33 @@ def ipa_flops(B, L, n_valid=None):
     return 2.0 * pairs * H * (dqk + dv)
 
 
+def rank_inputs(rank, L):
+    """Each rank times its own batch element of the workload (weak scaling):
+    same shapes, seed = rank."""
+    return ipa_inputs(IpaDims(B=1, L=L, H=H, C=C, Pq=PQ, Pv=PV, R=R, Cz=CZ), seed=rank)
+
+
+def max_over_ranks(ms, world, dist=None, device="cpu"):
+    """The job's time is the slowest rank's (every rank calls this, in the
+    same order, also when it has nothing to report)."""
+    if world == 1:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world, flops_per_rank_step, steps, total_ms):
+    """Whole-job throughput: all ranks' work over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (total_ms / 1e3) / 1e12
+
+
 def kernel_sha():
-    p = os.path.join(ROOT, "rna_structure_models_b200", "csrc", "ipa_attention.cu")
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()
+    h = hashlib.sha256()
+    for f in CORE_SOURCES:
+        h.update(open(os.path.join(ROOT, "rna_structure_models_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
 
 
 def measured_peaks():
@@ -197,8 +223,7 @@ def main():
     dev = torch.device("cuda", local)
 
     L = args.L
-    dims = IpaDims(B=1, L=L, H=H, C=C, Pq=PQ, Pv=PV, R=R, Cz=CZ)
-    inp = ipa_inputs(dims, seed=rank)                      # each rank its own batch element
+    inp = rank_inputs(rank, L)                             # each rank its own batch element
     names = api.IPA_INPUTS
     host = {n: torch.from_numpy(inp[n]) for n in names}
     dvc = {n: host[n].to(dev) for n in names}
@@ -236,18 +261,14 @@ def main():
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     core_ms = [e[1].elapsed_time(e[2]) for e in ev]
     pro_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dist, dev)
     if args.core_only:
         if world > 1:
             dist.destroy_process_group()
         return
 
     flops = ipa_flops(1, L)
-    value = world * flops * K / (total_ms / 1e3) / 1e12
+    value = aggregate_tflops(world, flops, K, total_ms)
     peaks, peak_kind = measured_peaks()
     core_mean = statistics.mean(core_ms)
     achieved = flops / (core_mean / 1e3) / 1e12
@@ -264,11 +285,11 @@ def main():
                    "step": "prologue (frames, augmented fp16 operands) + fused attention core"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "ipa_attention_kernel",
+                     "kernel": CORE_KERNEL,
                      "peak_source": f"{peak_kind} bf16 dense (burst); fp16 has the same nominal rate",
                      "core_ms": core_mean, "prologue_ms": statistics.mean(pro_ms),
                      "issued_frac": achieved * 640.0 / 581.0 / peak},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 4 * K,                             # tile, reduce, rows, core
         "clocks": clk.summary(),
     }
 
@@ -291,12 +312,10 @@ def main():
             o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev)
         e1.record()
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        line["e2e"] = {"value": world * flops * ke / (float(te.item()) / 1e3) / 1e12, "unit": UNIT,
+        te = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
+        line["e2e"] = {"value": aggregate_tflops(world, flops, ke, te), "unit": UNIT,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
-                       "ms_per_step": float(te.item()) / ke}
+                       "ms_per_step": te / ke}
 
     # second hot-path row: direction/distance geometric attention (B=2, N=2048)
     if not args.no_variant and rank == 0:

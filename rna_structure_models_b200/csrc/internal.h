@@ -25,7 +25,7 @@ struct View {
 };
 
 struct IpaWorkspace {
-  size_t qh, kh, vh, z2, z1f, rowq, colk, frame, part, cen, oq, ok, headc, wqp, err, total;
+  size_t qh, kh, vh, z2, z1h, z1f, rowq, colk, frame, part, cen, oq, ok, headc, wqp, err, total;
 };
 
 IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz);
@@ -80,6 +80,8 @@ bool ipa_pair_supported(int DZ);
 cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream);
 #ifdef IPA_TRACE
 bool ipa_pair_trace_read(void* host, size_t bytes);
+bool ipa_pair_span_read(void* host, size_t bytes);
+int ipa_pair_max_clusters();
 #endif
 
 }  // namespace fipa

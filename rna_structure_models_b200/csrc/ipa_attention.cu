@@ -35,6 +35,7 @@
 #include <cstring>
 
 #include "internal.h"
+#include "ipa_epilogue.cuh"
 #include "sm100.cuh"
 
 #ifdef IPA_TRACE
@@ -86,6 +87,8 @@ constexpr uint32_t AUX_BAR = 1152;                     // mbarriers
 constexpr uint32_t AUX_XCH = 2048;                     // float [2][2][128] row maxima + [2][128] row sums
 constexpr uint32_t SMEM_BYTES = SM_AUX + AUX_XCH + 4096;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;     // + alignment slack
+// the epilogue stage (128 rows x stage_pitch(DZ) floats) reuses the K/V stages and P
+static_assert(SM_STG + 128u * stage_pitch(MAX_DZ) * 4u <= SM_AUX, "epilogue stage overlaps the aux area");
 
 // barrier slots
 enum { B_Q = 0, B_QP, B_SFULL, B_SFREE, B_FULL0, B_EMPTY0 = B_FULL0 + NSTAGE,
@@ -359,22 +362,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float4* colv = reinterpret_cast<const float4*>(col_s + s * KT + 32 * half);
       const float4 dd = dinfo[s];
       const float rt = ch * (2.f * fmaf(sq.x, dd.x, fmaf(sq.y, dd.y, sq.z * dd.z)) - pq * dd.w);
-      float x[32];
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float2 x[16];
+      float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
       for (int k4 = 0; k4 < 8; ++k4) {
         const float4 cv = colv[k4];
-        x[4 * k4 + 0] = __uint_as_float(sr[4 * k4 + 0]) + cv.x;
-        x[4 * k4 + 1] = __uint_as_float(sr[4 * k4 + 1]) + cv.y;
-        x[4 * k4 + 2] = __uint_as_float(sr[4 * k4 + 2]) + cv.z;
-        x[4 * k4 + 3] = __uint_as_float(sr[4 * k4 + 3]) + cv.w;
-        mx4[0] = fmaxf(mx4[0], x[4 * k4 + 0]);
-        mx4[1] = fmaxf(mx4[1], x[4 * k4 + 1]);
-        mx4[2] = fmaxf(mx4[2], x[4 * k4 + 2]);
-        mx4[3] = fmaxf(mx4[3], x[4 * k4 + 3]);
+        x[2 * k4] = add_f32x2(make_float2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
+                              make_float2(cv.x, cv.y));
+        x[2 * k4 + 1] = add_f32x2(make_float2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
+                                  make_float2(cv.z, cv.w));
+        mxa = fmax3(mxa, x[2 * k4].x, x[2 * k4].y);
+        mxb = fmax3(mxb, x[2 * k4 + 1].x, x[2 * k4 + 1].y);
       }
       // row max over both halves (exchange through shared memory)
-      const float mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      const float mine = fmaxf(mxa, mxb);
       float* xb = xch + (j & 1) * 256;
       xb[half * 128 + r] = mine;
       named_bar_sync(pair_bar, 64);
@@ -384,19 +385,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float scale = resc ? ex2(m_used - mt) : 1.f;
       if (need) m_used = mt;
       l *= scale;
-      const float base = m_used - rt;
-      const bool live = m_used != -INFINITY;
+      // while no key of the row has been allowed, every x is -inf and the
+      // exponent base 0 gives P = 0
+      const float nbase = (m_used != -INFINITY) ? rt - m_used : 0.f;
+      const float2 nb2 = make_float2(nbase, nbase);
       uint32_t pk[16];
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        // p rounded to fp16 precision on the integer pipe (the value the
-        // tensor core will multiply), then packed; the row sum uses exactly
-        // those values
-        const float p0 = round_f16_precision(live ? ex2(x[2 * k] - base) : 0.f);
-        const float p1 = round_f16_precision(live ? ex2(x[2 * k + 1] - base) : 0.f);
-        pk[k] = pack_half2(p0, p1);
-        ls4[k & 3] += p0 + p1;
+        // P rounded to fp16 (nearest even) by the pack: the value the tensor
+        // core multiplies; the row sum adds exactly those values
+        const float2 y = add_f32x2(x[k], nb2);
+        pk[k] = pack_half2(ex2(y.x), ex2(y.y));
+        ls4[k & 3] = add_half2_to_f32(pk[k], ls4[k & 3]);
       }
       l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       if (tid == 0) IPA_TR(0, j, 8);
@@ -441,6 +442,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 
     // ------------------------------------------------ epilogue
+    // frame of this row (rotation, translation, valid), loaded while the last
+    // P.V runs
+    const float4* fgr = a.frame + (static_cast<int64_t>(b) * L + (in_range ? row : 0)) * 4;
+    const float4 f3 = fgr[3];
+    float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, g2 = g0, cn = g0;
+    if (half == 0) {
+      g0 = fgr[0];
+      g1 = fgr[1];
+      g2 = fgr[2];
+      cn = a.cen[b];
+    }
     if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_PFREE0 + ((nt - 1) & 1)),
                                                           ((nt - 1) >> 1) & 1, abort_flag))) {
       if (lane == 0) fail(DEV_TIMEOUT_MMA);
@@ -451,9 +463,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     xch[512 + half * 128 + r] = l;
     named_bar_sync(pair_bar, 64);
     const float lt = l + xch[512 + (1 - half) * 128 + r];
-    const float4 f3 = a.frame[(static_cast<int64_t>(b) * L + (in_range ? row : 0)) * 4 + 3];
     const bool dead = !(in_range && f3.x != 0.f && lt > 0.f);
-    const int pitch = OW + 4;
+    const int pitch = stage_pitch(DZ);
     float* stage = reinterpret_cast<float*>(smem + SM_STG);
     if (all_ok) {
       tc_fence_after();
@@ -469,56 +480,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
                           __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
       }
-      if (half == 0) orow[OW] = dead ? 1.f : 0.f;
+      if (half == 0) stage_frame(orow + 64 + DZ, g0, g1, g2, cn, dead);
     }
     tc_fence_before();
     named_bar_sync(1, NSOFT);
     if (!*abort_flag) {
-      const int C = IPA_C, Pv = IPA_PV, Cz = a.Cz, R = a.RCz / a.Cz;
-      const int F = a.F;
-      const float4 cn = a.cen[b];
-      for (int rr = 0; rr < 16; ++rr) {
-        const int rloc = warp * 16 + rr;
-        const int grow = I * QT + rloc;
-        if (grow >= L) break;
-        const float* O = stage + rloc * pitch;
-        const bool rdead = O[OW] != 0.f;
-        const float4* fg = a.frame + (static_cast<int64_t>(b) * L + grow) * 4;
-        const float4 g0 = fg[0], g1 = fg[1], g2 = fg[2];
-        const float Rm[9] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w, g2.x};
-        const float tcx[3] = {g2.y - cn.x, g2.z - cn.y, g2.w - cn.z};
-        float* dst = a.out + ((static_cast<int64_t>(b) * L + grow) * a.H + h) * F;
-        const float* z1r = a.z1f + (static_cast<int64_t>(b) * L + grow) * DZ;
-        for (int f = lane; f < F; f += 32) {
-          float val = 0.f;
-          if (!rdead) {
-            if (f < C) {
-              val = O[f];
-            } else if (f < C + 4 * Pv) {
-              const bool is_norm = f >= C + 3 * Pv;
-              const int p = is_norm ? f - C - 3 * Pv : (f - C) / 3;
-              float op[3];
-#pragma unroll
-              for (int xx = 0; xx < 3; ++xx) {
-                float acc = 0.f;
-#pragma unroll
-                for (int y = 0; y < 3; ++y) {
-                  const float og = O[C + 3 * p + y] + O[C + 3 * Pv + 3 * p + y];
-                  acc = fmaf(Rm[y * 3 + xx], og - tcx[y], acc);   // (R^T (og - t'))_xx
-                }
-                op[xx] = acc;
-              }
-              const int xc = (f - C) % 3;
-              val = is_norm ? sqrtf(fmaf(op[0], op[0], fmaf(op[1], op[1], op[2] * op[2])))
-                            : (xc == 0 ? op[0] : xc == 1 ? op[1] : op[2]);
-            } else {
-              const int cc = f - C - 4 * Pv;
-              for (int r2 = 0; r2 < R; ++r2) val = fmaf(z1r[r2 * Cz + cc], O[64 + r2 * Cz + cc], val);
-            }
-          }
-          dst[f] = val;
-        }
-      }
+      const EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, I * QT, a.z1f, a.out};
+      write_rows<IPA_C, IPA_PV>(ea, warp, lane);
     }
   }
 

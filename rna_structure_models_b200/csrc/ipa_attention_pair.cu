@@ -18,6 +18,11 @@
 // (own 64 keys: K_h 8 KB + Z2 DZ*128 B) | 1 x V slot (all 128 keys: own Z2
 // panels DZ*128 B + own V_h columns 8 KB, 64-byte swizzle).
 //
+// Warps: 0-7 softmax and epilogue (two threads per query row), 8 K producer
+// (K_h / Z2 key-half copies, then the fp32 column terms), 9 MMA issuer (one
+// thread of CTA 0) and tensor-memory owner, 10 V producer.  K and V copies
+// have their own threads so that neither waits for the other's slot.
+//
 // Synchronisation: barriers the MMA thread waits on live in CTA 0 (K/V slots
 // full: TMA bytes of both CTAs; S read and P written: one arrival per softmax
 // warp of both CTAs); barriers the softmax and producer warps wait on live in
@@ -32,10 +37,16 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "ipa_epilogue.cuh"
 #include "sm100.cuh"
 
 #ifdef IPA_TRACE
 __device__ unsigned long long g_pair_trace[2][64][32];
+__device__ unsigned long long g_pair_span[4096][64];  // per CTA: globaltimer start/end, clock64 start/end, smid, phase clocks
+#define PAIR_SPAN(k)                                                  \
+  do {                                                                \
+    if (blockIdx.x < 4096) g_pair_span[blockIdx.x][(k)] = clock64();  \
+  } while (0)
 #define PAIR_TR(j, ev)                                                               \
   do {                                                                               \
     if (trace_slot >= 0 && (j) < 64) g_pair_trace[trace_slot][(j)][(ev)] = clock64(); \
@@ -43,6 +54,9 @@ __device__ unsigned long long g_pair_trace[2][64][32];
 #else
 #define PAIR_TR(j, ev) \
   do {                 \
+  } while (0)
+#define PAIR_SPAN(k) \
+  do {               \
   } while (0)
 #endif
 
@@ -69,9 +83,9 @@ struct PairArgs {
   int trace_cta0, trace_cta1;
 };
 
-constexpr int NT = 320;            // 8 softmax warps, producer warp, MMA warp
+constexpr int NT = 352;            // 8 softmax warps, K producer, MMA warp, V producer
 constexpr int NSOFT = 256;
-constexpr int W_PROD = 8, W_MMA = 9;
+constexpr int W_PROD = 8, W_MMA = 9, W_VPROD = 10;
 constexpr int NCOL = 4;            // column-term ring
 
 // shared memory (offsets from a 1024-byte aligned base)
@@ -89,6 +103,8 @@ constexpr uint32_t AX_XCH = 2304;                 // float [2][2][128] maxima + 
 constexpr uint32_t AX_BAR = 5376;
 constexpr uint32_t SP_BYTES = SP_AUX + 6144;
 constexpr uint32_t SP_ALLOC = SP_BYTES + 1024;
+// the epilogue stage (128 rows x (64 + DZ + 20) floats) reuses Q_pair, K and V
+static_assert(SP_QP + 128u * stage_pitch(MAX_DZ) * 4u <= SP_AUX, "epilogue stage overlaps the aux area");
 
 enum {
   // local barriers (waited on in each CTA)
@@ -110,8 +126,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
                               const __grid_constant__ CUtensorMap tm_kh,
                               const __grid_constant__ CUtensorMap tm_z2k,
                               const __grid_constant__ CUtensorMap tm_z2v,
-                              const __grid_constant__ CUtensorMap tm_vh, const PairArgs a) {
+                              const __grid_constant__ CUtensorMap tm_vh,
+                              const __grid_constant__ CUtensorMap tm_z1, const PairArgs a) {
   extern __shared__ unsigned char smem_raw[];
+#ifdef IPA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 4096) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    g_pair_span[blockIdx.x][0] = globaltimer_ns();
+    g_pair_span[blockIdx.x][2] = clock64();
+    g_pair_span[blockIdx.x][4] = smid;
+  }
+#endif
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (sb - raw_u32);
@@ -165,12 +191,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     tma_prefetch_desc(&tm_z2k);
     tma_prefetch_desc(&tm_z2v);
     tma_prefetch_desc(&tm_vh);
+    tma_prefetch_desc(&tm_z1);
   }
   tc_fence_before();
   __syncthreads();
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (tid == 0) PAIR_SPAN(5);
 
   auto fail = [&](int code) {
     record_error(a.err, code);
@@ -182,14 +210,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     // ------------------------------------------------ producer (each CTA)
     const float4 oqv = a.oq[b * a.nqt + (I < a.nqt ? I : a.nqt - 1)];
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(P_QFULL), 16384);
+      // Q_h rows and the fp16 z1 rows of this CTA (scaled into Q_pair in place)
+      mbar_arrive_expect_tx(bar(P_QFULL), 16384u * static_cast<uint32_t>(1 + np));
       tma_load_3d(sb + SP_QH, &tm_qh, bar(P_QFULL), 0, row0, bh);
+      for (int p = 0; p < np; ++p) tma_load_3d(sb + SP_QP + 16384 * p, &tm_z1, bar(P_QFULL), 64 * p, row0, b);
     }
     const uint32_t kbytes = 8192u + static_cast<uint32_t>(np) * 8192u;
-    const uint32_t vbytes = static_cast<uint32_t>(np / 2) * 16384u + 8192u;
     auto load_k = [&](int j) {
       const int J2 = (start + j) % nt;
       const int s = j & 1;
+      // the copies first: the column terms below wait on global loads
+      if (lane == 0) {
+        const uint32_t kf = bar0(P_KFULL0 + s);
+        const uint32_t st = sb + SP_K + s * KSLOT;
+        const int krow = J2 * 128 + 64 * static_cast<int>(rank);
+        mbar_arrive_expect_tx_remote(kf, kbytes);
+        tma_load_3d_pair(st, &tm_kh, kf, 0, krow, bh);
+        for (int p = 0; p < np; ++p) tma_load_3d_pair(st + 8192 + 8192 * p, &tm_z2k, kf, 64 * p, krow, b);
+        PAIR_TR(j, 13);
+      }
       // column terms of this CTA's rows for the 128 keys of the tile
       const int cs = j % NCOL;
 #pragma unroll
@@ -211,29 +250,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         dinfo[cs * 2 + lane] = make_float4(dx, dy, dz, fmaf(dx, dx, fmaf(dy, dy, dz * dz)));
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(P_COLFULL0 + cs));
-        const uint32_t kf = bar0(P_KFULL0 + s);
-        const uint32_t st = sb + SP_K + s * KSLOT;
-        const int krow = J2 * 128 + 64 * static_cast<int>(rank);
-        mbar_arrive_expect_tx_cluster(kf, kbytes);
-        tma_load_3d_pair(st, &tm_kh, kf, 0, krow, bh);
-        for (int p = 0; p < np; ++p) tma_load_3d_pair(st + 8192 + 8192 * p, &tm_z2k, kf, 64 * p, krow, b);
-        PAIR_TR(j, 13);
-      }
-      __syncwarp();
-    };
-    auto load_v = [&](int j) {
-      const int J2 = (start + j) % nt;
-      if (lane == 0) {
-        const uint32_t vf = bar0(P_VFULL);
-        const uint32_t st = sb + SP_V;
-        mbar_arrive_expect_tx_cluster(vf, vbytes);
-        for (int p = 0; p < np / 2; ++p)
-          tma_load_3d_pair(st + 16384 * p, &tm_z2v, vf, 64 * (static_cast<int>(rank) * (np / 2) + p), J2 * 128, b);
-        tma_load_3d_pair(st + V_VH, &tm_vh, vf, 32 * static_cast<int>(rank), J2 * 128, bh);
-        PAIR_TR(j, 14);
-      }
+      if (lane == 0) mbar_arrive(bar(P_COLFULL0 + cs));
       __syncwarp();
     };
     auto wait_local = [&](int barid, uint32_t parity, int code) -> bool {
@@ -243,23 +260,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       if (!ok && lane == 0) fail(code);
       return ok != 0;
     };
-    // K(0), K(1), V(0); then per tile j >= 1: K(j+1) (after QK(j-1)), V(j) (after PV(j-1))
+    // K(0), K(1); then K(j) as soon as QK(j-2) has released its slot.  The
+    // column terms of tile j reuse ring entry j mod 4: QK(j-2) was issued
+    // after the softmax released S(j-3), so it has finished tile j-4.
     load_k(0);
     if (nt > 1) load_k(1);
-    load_v(0);
-    for (int j = 1; j < nt; ++j) {
-      if (j + 1 < nt) {
-        if (!wait_local(P_KEMPTY0 + ((j + 1) & 1), ((j - 1) >> 1) & 1, DEV_TIMEOUT_EMPTY)) break;
-        load_k(j + 1);
-      }
-      if (!wait_local(P_VEMPTY, (j - 1) & 1, DEV_TIMEOUT_EMPTY)) break;
-      load_v(j);
+    for (int j = 2; j < nt; ++j) {
+      if (!wait_local(P_KEMPTY0 + (j & 1), ((j - 2) >> 1) & 1, DEV_TIMEOUT_EMPTY)) break;
+      load_k(j);
     }
+  } else if (warp == W_VPROD) {
+    // ------------------------------------------------ V producer (each CTA, one thread)
+    if (lane == 0) {
+      const uint32_t vbytes = static_cast<uint32_t>(np / 2) * 16384u + 8192u;
+      for (int j = 0; j < nt; ++j) {
+        if (j > 0 && !mbar_wait_bounded(bar(P_VEMPTY), (j - 1) & 1, abort_flag)) {
+          fail(DEV_TIMEOUT_EMPTY);
+          break;
+        }
+        const int J2 = (start + j) % nt;
+        const uint32_t vf = bar0(P_VFULL);
+        const uint32_t st = sb + SP_V;
+        mbar_arrive_expect_tx_remote(vf, vbytes);
+        for (int p = 0; p < np / 2; ++p)
+          tma_load_3d_pair(st + 16384 * p, &tm_z2v, vf, 64 * (static_cast<int>(rank) * (np / 2) + p), J2 * 128, b);
+        tma_load_3d_pair(st + V_VH, &tm_vh, vf, 32 * static_cast<int>(rank), J2 * 128, bh);
+        PAIR_TR(j, 14);
+      }
+    }
+    __syncwarp();
   } else if (warp == W_MMA) {
     // ------------------------------------------------ MMA issuer (CTA 0, one thread)
     if (rank == 0 && lane == 0) {
       bool ok = mbar_wait_bounded_cluster(bar(P_QREADY), 0, abort_flag);
       if (!ok) fail(DEV_TIMEOUT_SOFTMAX);
+      PAIR_SPAN(7);
       tc_fence_after();
       const uint32_t idq = idesc_f16(256, 128, false);
       const uint32_t idz = idesc_f16(256, DZ, true);
@@ -269,9 +304,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
           const int s = j & 1;
-          ok = mbar_wait_bounded_cluster(bar(P_KFULL0 + s), (j >> 1) & 1, abort_flag);
+          ok = mbar_wait_bounded(bar(P_KFULL0 + s), (j >> 1) & 1, abort_flag);
           PAIR_TR(j, 0);
-          if (ok && j > 0) ok = mbar_wait_bounded_cluster(bar(P_SFREE), (j - 1) & 1, abort_flag);
+          if (ok && j > 0) ok = mbar_wait_bounded(bar(P_SFREE), (j - 1) & 1, abort_flag);
           PAIR_TR(j, 1);
           if (!ok) { fail(DEV_TIMEOUT_FULL); break; }
           tc_fence_after();
@@ -285,12 +320,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           umma2_commit_both(bar(P_SFULL));
           umma2_commit_both(bar(P_KEMPTY0 + s));
           PAIR_TR(j, 2);
+          if (j == 0) PAIR_SPAN(8);
           issued_any = true;
         }
         if (j > 0) {
           const int jj = j - 1;
-          ok = mbar_wait_bounded_cluster(bar(P_PFULL), jj & 1, abort_flag);
-          if (ok) ok = mbar_wait_bounded_cluster(bar(P_VFULL), jj & 1, abort_flag);
+          ok = mbar_wait_bounded(bar(P_PFULL), jj & 1, abort_flag);
+          if (ok) ok = mbar_wait_bounded(bar(P_VFULL), jj & 1, abort_flag);
           PAIR_TR(jj, 3);
           if (!ok) { fail(DEV_TIMEOUT_SOFTMAX); break; }
           tc_fence_after();
@@ -306,6 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           PAIR_TR(jj, 4);
         }
       }
+      PAIR_SPAN(9);
       if (!ok && issued_any) {
         umma2_commit_both(bar(P_DRAIN));
         mbar_wait_bounded(bar(P_DRAIN), 0, nullptr, 100000000ull);
@@ -326,31 +363,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     const int tev = (tid == 0) ? 0 : (tid == 96) ? 1 : -1;
     (void)tev;
 
-    // Q_pair rows (log2(e) w_L w_bias[:, h] * z1_i) into shared memory, 128-byte
-    // swizzled K-major panels; this thread writes half of the panels of row r
+    // Q_pair = (log2(e) w_L w_bias[:, h]) * z1_i: the z1 rows arrive by TMA in
+    // the 128-byte swizzled K-major panels the MMA reads; each thread scales
+    // half of the panels of its row in place (fp32 product, one fp16 rounding)
     {
-      const float* zr = a.z1f + (static_cast<int64_t>(b) * L + (in_range ? row : 0)) * DZ;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_QFULL), 0, abort_flag)) && lane == 0)
+        fail(DEV_TIMEOUT_FULL);
       const float* wr = a.wqp + static_cast<int64_t>(h) * DZ;
       for (int p = half * (np / 2); p < (half + 1) * (np / 2); ++p) {
         unsigned char* prow = smem + SP_QP + 16384 * p + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const float4 z0 = in_range ? *reinterpret_cast<const float4*>(zr + 64 * p + 8 * c) : make_float4(0, 0, 0, 0);
-          const float4 z1 = in_range ? *reinterpret_cast<const float4*>(zr + 64 * p + 8 * c + 4) : make_float4(0, 0, 0, 0);
-          const float4 w0 = *reinterpret_cast<const float4*>(wr + 64 * p + 8 * c);
-          const float4 w1 = *reinterpret_cast<const float4*>(wr + 64 * p + 8 * c + 4);
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-              make_uint4(pack_half2(z0.x * w0.x, z0.y * w0.y), pack_half2(z0.z * w0.z, z0.w * w0.w),
-                         pack_half2(z1.x * w1.x, z1.y * w1.y), pack_half2(z1.z * w1.z, z1.w * w1.w));
+          uint4* ptr = reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4));
+          uint4 u = *ptr;
+          const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr + 64 * p + 8 * c));
+          const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr + 64 * p + 8 * c + 4));
+          const float2 z0 = unpack_half2(u.x), z1 = unpack_half2(u.y), z2 = unpack_half2(u.z), z3 = unpack_half2(u.w);
+          u = make_uint4(pack_half2(z0.x * w0.x, z0.y * w0.y), pack_half2(z1.x * w0.z, z1.y * w0.w),
+                         pack_half2(z2.x * w1.x, z2.y * w1.y), pack_half2(z3.x * w1.z, z3.y * w1.w));
+          *ptr = u;
         }
       }
       fence_proxy_async_smem();
       named_bar_sync(1, NSOFT);
-      if (tid == 0) {
-        const bool okq = mbar_wait_bounded(bar(P_QFULL), 0, abort_flag);
-        if (!okq) fail(DEV_TIMEOUT_FULL);
-        mbar_arrive_cluster(bar0(P_QREADY));
-      }
+      if (tid == 0) PAIR_SPAN(6);
+      if (tid == 0) mbar_arrive_cluster(bar0(P_QREADY));
     }
 
     float m_used = -INFINITY, l = 0.f;
@@ -377,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       tc_fence_before();
       if (tid == 0) PAIR_TR(j, 17);
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(bar0(P_SFREE));
+      if (lane == 0) mbar_arrive_remote(bar0(P_SFREE));
       if (tid == 0) PAIR_TR(j, 18);
       const int cs = j % NCOL;
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_COLFULL0 + cs), (j / NCOL) & 1, abort_flag))) {
@@ -389,22 +426,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       const float4* colv = reinterpret_cast<const float4*>(col_s + cs * 128 + 64 * half);
       const float4 dd = dinfo[cs * 2 + half];
       const float rt = ch * (2.f * fmaf(sq.x, dd.x, fmaf(sq.y, dd.y, sq.z * dd.z)) - pq * dd.w);
-      float x[64];
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // x = S + column term (packed pairs), running maximum over this half's keys
+      float2 x[32];
+      float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
       for (int k4 = 0; k4 < 16; ++k4) {
         const float4 cv = colv[k4];
-        x[4 * k4 + 0] = __uint_as_float(sr[4 * k4 + 0]) + cv.x;
-        x[4 * k4 + 1] = __uint_as_float(sr[4 * k4 + 1]) + cv.y;
-        x[4 * k4 + 2] = __uint_as_float(sr[4 * k4 + 2]) + cv.z;
-        x[4 * k4 + 3] = __uint_as_float(sr[4 * k4 + 3]) + cv.w;
-        mx4[0] = fmaxf(mx4[0], x[4 * k4 + 0]);
-        mx4[1] = fmaxf(mx4[1], x[4 * k4 + 1]);
-        mx4[2] = fmaxf(mx4[2], x[4 * k4 + 2]);
-        mx4[3] = fmaxf(mx4[3], x[4 * k4 + 3]);
+        x[2 * k4] = add_f32x2(make_float2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
+                              make_float2(cv.x, cv.y));
+        x[2 * k4 + 1] = add_f32x2(make_float2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
+                                  make_float2(cv.z, cv.w));
+        mxa = fmax3(mxa, x[2 * k4].x, x[2 * k4].y);
+        mxb = fmax3(mxb, x[2 * k4 + 1].x, x[2 * k4 + 1].y);
       }
       // this half's max in full logit units (the row term differs between the key halves)
-      const float mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) + rt;
+      const float mine = fmaxf(mxa, mxb) + rt;
       float* xb = xch + (j & 1) * 256;
       xb[half * 128 + r] = mine;
       if (tid == 0) PAIR_TR(j, 20);
@@ -416,16 +452,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       const float scale = resc ? ex2(m_used - mt) : 1.f;
       if (need) m_used = mt;
       l *= scale;
-      const float base = m_used - rt;
-      const bool live = m_used != -INFINITY;
+      // while no key of the row has been allowed, every x is -inf and the
+      // exponent base 0 gives P = 0
+      const float nbase = (m_used != -INFINITY) ? rt - m_used : 0.f;
+      const float2 nb2 = make_float2(nbase, nbase);
+      // P = 2^(x - base) rounded to fp16 (round to nearest even) in the pack;
+      // the row sum adds exactly the fp16 values the P.V MMA consumes
       uint32_t pk[32];
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const float p0 = round_f16_precision(live ? ex2(x[2 * k] - base) : 0.f);
-        const float p1 = round_f16_precision(live ? ex2(x[2 * k + 1] - base) : 0.f);
-        pk[k] = pack_half2(p0, p1);
-        ls4[k & 3] += p0 + p1;
+        const float2 y = add_f32x2(x[k], nb2);
+        pk[k] = pack_half2(ex2(y.x), ex2(y.y));
+        ls4[k & 3] = add_half2_to_f32(pk[k], ls4[k & 3]);
       }
       l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       if (tid == 0) PAIR_TR(j, 22);
@@ -452,29 +491,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       tc_fence_before();
       if (tid == 0) PAIR_TR(j, 24);
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(bar0(P_PFULL));
+      if (lane == 0) mbar_arrive_remote(bar0(P_PFULL));
       if (tid == 0) PAIR_TR(j, 25);
       if (tid == 96) PAIR_TR(j, 27);
     }
 
     // ------------------------------------------------ epilogue
+    // frame of this row (rotation, translation, valid), loaded while the last
+    // P.V runs
+    const float4* fgr = a.frame + (static_cast<int64_t>(b) * L + (in_range ? row : 0)) * 4;
+    const float4 f3 = fgr[3];
+    float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, g2 = g0, cn = g0;
+    if (half == 0) {
+      g0 = fgr[0];
+      g1 = fgr[1];
+      g2 = fgr[2];
+      cn = a.cen[b];
+    }
     if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_PFREE), (nt - 1) & 1, abort_flag))) {
       if (lane == 0) fail(DEV_TIMEOUT_MMA);
       ok = false;
     }
+    if (tid == 0) PAIR_SPAN(10);
     const bool all_ok = __all_sync(0xffffffffu, ok);
     xch[512 + half * 128 + r] = l;
     named_bar_sync(pair_bar, 64);
     const float lt = l + xch[512 + (1 - half) * 128 + r];
-    const float4 f3 = a.frame[(static_cast<int64_t>(b) * L + (in_range ? row : 0)) * 4 + 3];
     const bool dead = !(in_range && f3.x != 0.f && lt > 0.f);
-    const int pitch = OW + 4;
+    const int pitch = stage_pitch(DZ);
     float* stage = reinterpret_cast<float*>(smem + SP_QP);
     if (all_ok) {
       tc_fence_after();
       const float inv = dead ? 0.f : 1.f / lt;
       float* orow = stage + r * pitch;
-      // staged row layout: [O_v (64) | O_pair (DZ)]; tensor memory holds [O_pair | O_v]
+      // tensor memory holds [O_pair | O_v]; the stage row is [O_v | O_pair | frame]
       for (int c0 = o_lo; c0 < o_hi; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tmem + c0 + lane_off, o);
@@ -486,66 +536,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
               make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
                           __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
       }
-      if (half == 0) orow[OW] = dead ? 1.f : 0.f;
+      if (half == 0) stage_frame(orow + 64 + DZ, g0, g1, g2, cn, dead);
     }
     tc_fence_before();
     named_bar_sync(1, NSOFT);
+    if (tid == 0) PAIR_SPAN(11);
     if (!*abort_flag) {
-      const int C = IPA_C, Pv = IPA_PV, Cz = a.Cz, R = a.RCz / a.Cz;
-      const int F = a.F;
-      const float4 cn = a.cen[b];
-      for (int rr = 0; rr < 16; ++rr) {
-        const int rloc = warp * 16 + rr;
-        const int grow = row0 + rloc;
-        if (grow >= L) break;
-        const float* O = stage + rloc * pitch;
-        const bool rdead = O[OW] != 0.f;
-        const float4* fg = a.frame + (static_cast<int64_t>(b) * L + grow) * 4;
-        const float4 g0 = fg[0], g1 = fg[1], g2 = fg[2];
-        const float Rm[9] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w, g2.x};
-        const float tcx[3] = {g2.y - cn.x, g2.z - cn.y, g2.w - cn.z};
-        float* dst = a.out + ((static_cast<int64_t>(b) * L + grow) * a.H + h) * F;
-        const float* z1r = a.z1f + (static_cast<int64_t>(b) * L + grow) * DZ;
-        for (int f = lane; f < F; f += 32) {
-          float val = 0.f;
-          if (!rdead) {
-            if (f < C) {
-              val = O[f];
-            } else if (f < C + 4 * Pv) {
-              const bool is_norm = f >= C + 3 * Pv;
-              const int p = is_norm ? f - C - 3 * Pv : (f - C) / 3;
-              float op[3];
-#pragma unroll
-              for (int xx = 0; xx < 3; ++xx) {
-                float acc = 0.f;
-#pragma unroll
-                for (int y = 0; y < 3; ++y) {
-                  const float og = O[C + 3 * p + y] + O[C + 3 * Pv + 3 * p + y];
-                  acc = fmaf(Rm[y * 3 + xx], og - tcx[y], acc);   // (R^T (og - t'))_xx
-                }
-                op[xx] = acc;
-              }
-              const int xc = (f - C) % 3;
-              val = is_norm ? sqrtf(fmaf(op[0], op[0], fmaf(op[1], op[1], op[2] * op[2])))
-                            : (xc == 0 ? op[0] : xc == 1 ? op[1] : op[2]);
-            } else {
-              const int cc = f - C - 4 * Pv;
-              for (int r2 = 0; r2 < R; ++r2) val = fmaf(z1r[r2 * Cz + cc], O[64 + r2 * Cz + cc], val);
-            }
-          }
-          dst[f] = val;
-        }
-      }
+      EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, row0, a.z1f, a.out};
+#ifdef IPA_TRACE
+      ea.trace = (blockIdx.x < 4096 && warp == 0) ? &g_pair_span[blockIdx.x][16] : nullptr;
+#endif
+      write_rows<IPA_C, IPA_PV>(ea, warp, lane);
     }
   }
 
+  if (tid == 0) PAIR_SPAN(12);
   tc_fence_before();
   __syncthreads();
+  if (tid == 0) PAIR_SPAN(13);
   cluster_sync();
+  if (tid == 0) PAIR_SPAN(14);
   if (warp == W_MMA) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, TM_COLS);
   }
+#ifdef IPA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 4096) {
+    g_pair_span[blockIdx.x][3] = clock64();
+    g_pair_span[blockIdx.x][1] = globaltimer_ns();
+  }
+#endif
 }
 
 }  // namespace
@@ -555,7 +575,7 @@ bool ipa_pair_supported(int DZ) { return DZ == 128 || DZ == 256; }
 cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
   unsigned char* ws = a.ws;
   const IpaWorkspace& w = a.lay;
-  CUtensorMap tqh, tkh, tz2k, tz2v, tvh;
+  CUtensorMap tqh, tkh, tz2k, tz2v, tvh, tz1;
   const uint64_t bh = static_cast<uint64_t>(a.B) * a.H;
   const uint64_t rowb = static_cast<uint64_t>(a.L) * DH * 2;
   const uint64_t zrow = static_cast<uint64_t>(a.DZ) * 2, zb = static_cast<uint64_t>(a.L) * a.DZ * 2;
@@ -563,7 +583,8 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
             encode_tmap_f16_3d(&tkh, ws + w.kh, DH, a.L, bh, DH * 2, rowb, 64, 64) &&
             encode_tmap_f16_3d(&tz2k, ws + w.z2, a.DZ, a.L, a.B, zrow, zb, 64, 64) &&
             encode_tmap_f16_3d(&tz2v, ws + w.z2, a.DZ, a.L, a.B, zrow, zb, 64, 128) &&
-            encode_tmap_f16_3d(&tvh, ws + w.vh, DH, a.L, bh, DH * 2, rowb, 32, 128, 64);
+            encode_tmap_f16_3d(&tvh, ws + w.vh, DH, a.L, bh, DH * 2, rowb, 32, 128, 64) &&
+            encode_tmap_f16_3d(&tz1, ws + w.z1h, a.DZ, a.L, a.B, zrow, zb, 64, 128);
   if (!ok) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(ipa_attention_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(SP_ALLOC));
@@ -584,7 +605,7 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
   const int pairs = static_cast<int>(bh) * t.nqp;
   t.trace_cta0 = 0;
   t.trace_cta1 = 2 * (pairs / 2);
-  ipa_attention_pair_kernel<<<static_cast<unsigned>(2 * pairs), NT, SP_ALLOC, stream>>>(tqh, tkh, tz2k, tz2v, tvh, t);
+  ipa_attention_pair_kernel<<<static_cast<unsigned>(2 * pairs), NT, SP_ALLOC, stream>>>(tqh, tkh, tz2k, tz2v, tvh, tz1, t);
   return cudaGetLastError();
 }
 
@@ -592,6 +613,27 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
 bool ipa_pair_trace_read(void* host, size_t bytes) {
   if (bytes < sizeof(g_pair_trace)) return false;
   return cudaMemcpyFromSymbol(host, g_pair_trace, sizeof(g_pair_trace)) == cudaSuccess;
+}
+bool ipa_pair_span_read(void* host, size_t bytes) {
+  if (bytes < sizeof(g_pair_span)) return false;
+  return cudaMemcpyFromSymbol(host, g_pair_span, sizeof(g_pair_span)) == cudaSuccess;
+}
+int ipa_pair_max_clusters() {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * 192);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = SP_ALLOC;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = -1;
+  cudaFuncSetAttribute(ipa_attention_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SP_ALLOC));
+  if (cudaOccupancyMaxActiveClusters(&n, ipa_attention_pair_kernel, &cfg) != cudaSuccess) return -1;
+  return n;
 }
 #endif
 

@@ -1,0 +1,216 @@
+// Output pass of the fused IPA core, shared by the single-CTA and the
+// CTA-pair attention kernels.
+//
+// The softmax threads stage, per query row of a 128-row tile, the normalised
+// accumulators and the row's frame in shared memory:
+//
+//   [ O_v (64) | O_pair (DZ) | R (9, row-major) | t - centroid (3) | dead (1) | pad ]
+//
+// with O_v = [o (C) | gv hi (3 Pv) | gv lo (3 Pv)] (value points relative to
+// the centroid) and O_pair = sum_j a_ij z2_j.  Eight warps then write the
+// rows of the tile, one row per warp at a time, consecutive lanes on
+// consecutive output features (coalesced stores):
+//
+//   out[b, i, h, :] = [ o (C) | R_i^T (gv - t_i) (3 Pv) | |.| per point (Pv) |
+//                       sum_r z1_i[r] (.) O_pair[r] (Cz) ]
+//
+// (Flash Invariant Point Attention, TL;DR: the factorised pair output; the
+// point output is mapped back into the residue's local frame as in the IPA
+// formulation.)  A row with no allowed key is written as zeros.
+#pragma once
+
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace fipa {
+
+// Frame columns of a staged row start at 64 + DZ; the pitch is 4 x odd floats
+// so that per-thread float4 stores of consecutive rows are conflict-free.
+__host__ __device__ constexpr int stage_pitch(int DZ) { return 64 + DZ + 20; }
+
+__device__ __forceinline__ void stage_frame(float* orow_frame, float4 g0, float4 g1, float4 g2, float4 cn,
+                                            bool dead) {
+  *reinterpret_cast<float4*>(orow_frame) = g0;
+  *reinterpret_cast<float4*>(orow_frame + 4) = g1;
+  *reinterpret_cast<float4*>(orow_frame + 8) = make_float4(g2.x, g2.y - cn.x, g2.z - cn.y, g2.w - cn.z);
+  orow_frame[12] = dead ? 1.f : 0.f;
+}
+
+struct EpilogueArgs {
+  float* stage;          // 128 staged rows
+  int DZ, Cz, RCz, F, H, L;
+  int b, h, row0;        // first query row of the tile
+  const float* z1f;      // [B, L, DZ] fp32, zero-padded
+  float* out;            // [B, L, H, F]
+#ifdef IPA_TRACE
+  unsigned long long* trace = nullptr;   // phase clocks of warp 0 (tracing build only)
+#endif
+};
+
+// One output row, written by one warp from its staged row O (the pair sums
+// sum_r z1 (.) O_pair already reduced into O[64 .. 64 + Cz)):
+//   * point p, coordinate x on lane 3p + x: g = gv - t' (hi + lo), the three
+//     coordinates of a point meet by shuffles, R^T g, then the norm on lane p;
+//   * pair feature cc on the lane of its output position.
+// The lane-to-feature map below is written for C = 16, PV = 8: output chunk 0
+// is [o (16) | coordinates 0..15], chunk 1 is [coordinates 16..23 | norms (8) |
+// pair 0..15], later chunks are pair features.  No loop here has a runtime
+// trip count, so the loads of a row issue together.
+template <int C, int PV>
+__device__ __forceinline__ void write_row(const float* O, float* dst, int lane, int DZ, int F) {
+  static_assert(C == 16 && PV == 8, "output lane map assumes the (16, 8) head shape");
+  const int FR = 64 + DZ;
+  const int l = lane < 3 * PV ? lane : 0;
+  const int x = l % 3, p3 = l - x;
+  const float gd = O[C + l] + O[C + 3 * PV + l] - O[FR + 9 + x];
+  const float r0 = O[FR + x], r1 = O[FR + 3 + x], r2 = O[FR + 6 + x];
+  const float own = O[lane];
+  const bool rdead = O[FR + 12] != 0.f;
+  float pv[9];                          // pair features of output chunks 1..9 (F = 48 + Cz <= 304)
+#pragma unroll
+  for (int k = 1; k < 10; ++k) {
+    const int f = 32 * k + lane;
+    const int cc = f - C - 4 * PV;
+    pv[k - 1] = (cc >= 0 && f < F) ? O[64 + cc] : 0.f;
+  }
+  const float g0 = __shfl_sync(0xffffffffu, gd, p3);
+  const float g1 = __shfl_sync(0xffffffffu, gd, p3 + 1);
+  const float g2 = __shfl_sync(0xffffffffu, gd, p3 + 2);
+  const float op = fmaf(r0, g0, fmaf(r1, g1, r2 * g2));   // (R^T g)_x
+  const float sq = op * op;
+  const int pp = (lane < PV ? lane : 0) * 3;
+  const float nrm = sqrtf(__shfl_sync(0xffffffffu, sq, pp) + __shfl_sync(0xffffffffu, sq, pp + 1) +
+                          __shfl_sync(0xffffffffu, sq, pp + 2));
+  const float c_lo = __shfl_sync(0xffffffffu, op, (lane - 16) & 31);   // coordinates 0..15 on lanes 16..31
+  const float c_hi = __shfl_sync(0xffffffffu, op, (lane + 16) & 31);   // coordinates 16..23 on lanes 0..7
+  const float n_p = __shfl_sync(0xffffffffu, nrm, (lane - 8) & 31);    // norms on lanes 8..15
+#pragma unroll
+  for (int k = 0; k < 10; ++k) {
+    const int f = 32 * k + lane;
+    float val;
+    if (k == 0) val = lane < C ? own : c_lo;
+    else if (k == 1 && lane < 8) val = c_hi;
+    else if (k == 1 && lane < 16) val = n_p;
+    else val = pv[k - 1];
+    if (f < F) dst[f] = rdead ? 0.f : val;
+  }
+}
+
+// Phase A for the 16 rows of one warp: z1 (.) O_pair summed over the R
+// factors into O_pair[0 .. Cz) of each staged row.  z1 rows load coalesced,
+// 4 rows per group, the next group's loads in flight while the current one is
+// folded.  NCZ = Cz / 32 > 0: a lane's columns c = lane + 32 t (all R factors)
+// fold into pair feature lane + 32 (t mod NCZ) in registers (every column a
+// lane reads or writes is its own).  NCZ = 0 (Cz not a multiple of 32): the
+// products are written in place and reduced in a second pass.
+template <int NCZ>
+__device__ __noinline__ void fold_pairs_rows(const EpilogueArgs& e, int warp, int lane) {
+  const int pitch = stage_pitch(e.DZ);
+  const int nz = (e.RCz + 31) >> 5;   // z1 values per lane per row (<= 8)
+  float zc[4][8], zn[4][8];
+  auto load_group = [&](int g, float (&zz)[4][8]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int grow = e.row0 + warp * 16 + 4 * g + q;
+      const float* zr = e.z1f + (static_cast<int64_t>(e.b) * e.L + (grow < e.L ? grow : 0)) * e.DZ;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int c = lane + 32 * t;
+        zz[q][t] = (t < nz && c < e.RCz && grow < e.L) ? __ldg(zr + c) : 0.f;
+      }
+    }
+  };
+  load_group(0, zc);
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    if (g < 3) load_group(g + 1, zn);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float* P = e.stage + (warp * 16 + 4 * g + q) * pitch + 64;
+      if (NCZ > 0) {
+        float acc[NCZ > 0 ? NCZ : 1];
+#pragma unroll
+        for (int j = 0; j < (NCZ > 0 ? NCZ : 1); ++j) acc[j] = 0.f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          if (t < nz) acc[t % (NCZ > 0 ? NCZ : 1)] = fmaf(zc[q][t], P[lane + 32 * t], acc[t % (NCZ > 0 ? NCZ : 1)]);
+#pragma unroll
+        for (int j = 0; j < (NCZ > 0 ? NCZ : 1); ++j) P[lane + 32 * j] = acc[j];
+      } else {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int c = lane + 32 * t;
+          if (t < nz && c < e.RCz) P[c] *= zc[q][t];
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) zc[q][t] = zn[q][t];
+  }
+  __syncwarp();
+  const int R = e.RCz / e.Cz;
+  if (NCZ == 0 && R > 1) {
+    for (int rr = 0; rr < 16; ++rr) {
+      float* P = e.stage + (warp * 16 + rr) * pitch + 64;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int cc = lane + 32 * u;
+        if (cc < e.Cz) {
+          float acc = P[cc];
+          for (int r2 = 1; r2 < R; ++r2) acc += P[r2 * e.Cz + cc];
+          P[cc] = acc;
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// Called by all 8 warps (warp = 0..7) after the staged rows are complete;
+// warp w handles rows 16 w .. 16 w + 15 of the tile: phase A (above, one
+// instantiation chosen per call), then phase B: the output rows with
+// coalesced stores.  No global load is issued after a global store.
+template <int C, int PV>
+__device__ __forceinline__ void write_rows(const EpilogueArgs& e, int warp, int lane) {
+  const int pitch = stage_pitch(e.DZ);
+#ifdef IPA_TRACE
+#define EPI_TR(k)                                                  \
+  do {                                                             \
+    if (e.trace != nullptr && lane == 0) e.trace[(k)] = clock64(); \
+  } while (0)
+#else
+#define EPI_TR(k) \
+  do {            \
+  } while (0)
+#endif
+  EPI_TR(0);
+  switch ((e.Cz & 31) == 0 ? e.Cz >> 5 : 0) {
+    case 1: fold_pairs_rows<1>(e, warp, lane); break;
+    case 2: fold_pairs_rows<2>(e, warp, lane); break;
+    case 3: fold_pairs_rows<3>(e, warp, lane); break;
+    case 4: fold_pairs_rows<4>(e, warp, lane); break;
+    case 5: fold_pairs_rows<5>(e, warp, lane); break;
+    case 6: fold_pairs_rows<6>(e, warp, lane); break;
+    case 7: fold_pairs_rows<7>(e, warp, lane); break;
+    case 8: fold_pairs_rows<8>(e, warp, lane); break;
+    default: fold_pairs_rows<0>(e, warp, lane); break;
+  }
+  EPI_TR(1);
+#pragma unroll 1
+  for (int rr = 0; rr < 16; ++rr) {
+    const int rloc = warp * 16 + rr;
+    const int grow = e.row0 + rloc;
+    if (grow < e.L)
+      write_row<C, PV>(e.stage + rloc * pitch, e.out + ((static_cast<int64_t>(e.b) * e.L + grow) * e.H + e.h) * e.F,
+                       lane, e.DZ, e.F);
+    EPI_TR(3 + rr);
+  }
+  EPI_TR(2);
+}
+
+#undef EPI_TR
+
+}  // namespace fipa

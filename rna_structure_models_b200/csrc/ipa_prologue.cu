@@ -3,7 +3,8 @@
 //
 //   ipa_tile_kernel   -- one CTA per (batch, 64-residue key tile): frame rows
 //                        (R, t, valid), partial sums of the valid origins, and
-//                        the pair factors z2 (fp16) / z1 (fp32) padded to DZ.
+//                        the pair factors z2 (fp16) and z1 (fp32 and fp16)
+//                        padded to DZ.
 //   ipa_reduce_kernel -- one CTA per batch: centroid of the valid origins,
 //                        query-tile (128) and key-tile (64) origins relative
 //                        to it; per-head point coefficient and pair-bias
@@ -49,6 +50,7 @@ struct TileArgs {
   float4* frame;   // [B, L, 4]: (R00 R01 R02 R10) (R11 R12 R20 R21) (R22 tx ty tz) (valid 0 0 0)
   float4* part;    // [B, nkt]: sum of valid origins, count
   float* z1f;      // [B, L, DZ]
+  __half* z1h;     // [B, L, DZ]
   __half* z2h;     // [B, L, DZ]
 };
 
@@ -77,6 +79,7 @@ __device__ __forceinline__ void ipa_tile_copy_pairs(const TileArgs& a, int b, in
     if (i < a.L) {
       const int64_t o = (static_cast<int64_t>(b) * a.L + i) * a.DZ + col;
       a.z1f[o] = v1[q];
+      a.z1h[o] = __float2half_rn(v1[q]);
       a.z2h[o] = __float2half_rn(v2[q]);
     }
   }
@@ -355,6 +358,7 @@ cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
   ta.part = reinterpret_cast<float4*>(ws + w.part);
   ta.z1f = reinterpret_cast<float*>(ws + w.z1f);
   ta.z2h = reinterpret_cast<__half*>(ws + w.z2);
+  ta.z1h = reinterpret_cast<__half*>(ws + w.z1h);
   ipa_tile_kernel<<<dim3(a.nkt, a.B, a.DZ / 64), 256, 0, stream>>>(ta);
 
   ReduceArgs ra{};
@@ -395,6 +399,7 @@ IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz) {
   w.kh = o; o = up(o + bhl * DH * 2);
   w.vh = o; o = up(o + bhl * DH * 2);
   w.z2 = o; o = up(o + bl * DZ * 2);
+  w.z1h = o; o = up(o + bl * DZ * 2);
   w.z1f = o; o = up(o + bl * DZ * 4);
   w.rowq = o; o = up(o + bhl * 16);
   w.colk = o; o = up(o + bhl * 16);
