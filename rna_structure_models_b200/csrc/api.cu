@@ -111,6 +111,25 @@ bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_
   return r == CUDA_SUCCESS;
 }
 
+// [B, L, DZ] fp16 seen as 64-column panels: dims (64 columns, L rows, DZ/64
+// panels, B) with strides (DZ*2, 128, L*DZ*2) bytes.  One box of
+// (64, box_rows, box_panels) lands in shared memory as box_panels consecutive
+// 128-byte swizzled K-major panels of box_rows rows, the layout the MMA
+// descriptors read, so a whole multi-panel tile is one copy.
+bool encode_tmap_f16_panels(CUtensorMap* map, const void* base, uint64_t DZ, uint64_t L, uint64_t B,
+                            uint32_t box_rows, uint32_t box_panels) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr || DZ % 64 != 0) return false;
+  const cuuint64_t dims[4] = {64, L, DZ / 64, B};
+  const cuuint64_t strides[3] = {DZ * 2, 128, L * DZ * 2};
+  const cuuint32_t box[4] = {64, box_rows, box_panels, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fipa
 
 using namespace fipa;

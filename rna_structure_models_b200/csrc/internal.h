@@ -74,6 +74,8 @@ bool ipa_trace_read(void* host, size_t bytes);
 bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                         uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
                         uint32_t box0, uint32_t box1, int swizzle_bytes = 128);
+bool encode_tmap_f16_panels(CUtensorMap* map, const void* base, uint64_t DZ, uint64_t L, uint64_t B,
+                            uint32_t box_rows, uint32_t box_panels);
 
 // CTA-pair core kernel (cta_group::2): pair-dimension widths it supports and its launch.
 bool ipa_pair_supported(int DZ);

@@ -83,7 +83,7 @@ struct PairArgs {
   int trace_cta0, trace_cta1;
 };
 
-constexpr int NT = 352;            // 8 softmax warps, K producer, MMA warp, V producer
+constexpr int NT = 352;            // 8 softmax warps, K producer, MMA issuer, V producer
 constexpr int NSOFT = 256;
 constexpr int W_PROD = 8, W_MMA = 9, W_VPROD = 10;
 constexpr int NCOL = 4;            // column-term ring
@@ -213,45 +213,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       // Q_h rows and the fp16 z1 rows of this CTA (scaled into Q_pair in place)
       mbar_arrive_expect_tx(bar(P_QFULL), 16384u * static_cast<uint32_t>(1 + np));
       tma_load_3d(sb + SP_QH, &tm_qh, bar(P_QFULL), 0, row0, bh);
-      for (int p = 0; p < np; ++p) tma_load_3d(sb + SP_QP + 16384 * p, &tm_z1, bar(P_QFULL), 64 * p, row0, b);
+      tma_load_4d(sb + SP_QP, &tm_z1, bar(P_QFULL), 0, row0, 0, b);   // all np panels
     }
     const uint32_t kbytes = 8192u + static_cast<uint32_t>(np) * 8192u;
+    // inputs of the column terms of the next tile, loaded one tile ahead so
+    // that their global-load latency overlaps the wait for a free K slot
+    float4 ckn[4], okn[4], odn = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto fetch_cols = [&](int j) {
+      const int J2 = (start + j) % nt;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int key = J2 * 128 + lane + 32 * t;
+        const bool in = j < nt && key < L;
+        ckn[t] = in ? a.colk[static_cast<int64_t>(bh) * L + key] : make_float4(0.f, 0.f, 0.f, -INFINITY);
+        okn[t] = in ? a.ok[b * a.nkt + key / KT] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      const int jt = 2 * J2 + (lane & 1);
+      odn = (j < nt && jt < a.nkt) ? a.ok[b * a.nkt + jt] : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
     auto load_k = [&](int j) {
       const int J2 = (start + j) % nt;
       const int s = j & 1;
-      // the copies first: the column terms below wait on global loads
       if (lane == 0) {
         const uint32_t kf = bar0(P_KFULL0 + s);
         const uint32_t st = sb + SP_K + s * KSLOT;
         const int krow = J2 * 128 + 64 * static_cast<int>(rank);
         mbar_arrive_expect_tx_remote(kf, kbytes);
+        PAIR_TR(j, 10);
         tma_load_3d_pair(st, &tm_kh, kf, 0, krow, bh);
-        for (int p = 0; p < np; ++p) tma_load_3d_pair(st + 8192 + 8192 * p, &tm_z2k, kf, 64 * p, krow, b);
+        PAIR_TR(j, 9);
+        tma_load_4d_pair(st + 8192, &tm_z2k, kf, 0, krow, 0, b);   // all np panels of the key half
         PAIR_TR(j, 13);
       }
-      // column terms of this CTA's rows for the 128 keys of the tile
+      // column terms of this CTA's rows for the 128 keys of the tile (-inf
+      // for keys past L and for masked keys, whose colk.w is -inf)
       const int cs = j % NCOL;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const int kk = lane + 32 * t;
-        const int key = J2 * 128 + kk;
-        float cv = -INFINITY;
-        if (key < L) {
-          const float4 okv = a.ok[b * a.nkt + key / KT];
-          const float4 ck = a.colk[static_cast<int64_t>(bh) * L + key];
-          cv = ck.w - fmaf(ck.x, okv.x - oqv.x, fmaf(ck.y, okv.y - oqv.y, ck.z * (okv.z - oqv.z)));
-        }
-        col_s[cs * 128 + kk] = cv;
+        const float4 ck = ckn[t], okv = okn[t];
+        col_s[cs * 128 + lane + 32 * t] =
+            ck.w - fmaf(ck.x, okv.x - oqv.x, fmaf(ck.y, okv.y - oqv.y, ck.z * (okv.z - oqv.z)));
       }
       if (lane < 2) {
-        const int jt = 2 * J2 + lane;
-        const float4 okv = jt < a.nkt ? a.ok[b * a.nkt + jt] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float dx = okv.x - oqv.x, dy = okv.y - oqv.y, dz = okv.z - oqv.z;
+        const float dx = odn.x - oqv.x, dy = odn.y - oqv.y, dz = odn.z - oqv.z;
         dinfo[cs * 2 + lane] = make_float4(dx, dy, dz, fmaf(dx, dx, fmaf(dy, dy, dz * dz)));
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(P_COLFULL0 + cs));
       __syncwarp();
+      fetch_cols(j + 1);
     };
     auto wait_local = [&](int barid, uint32_t parity, int code) -> bool {
       int ok = 1;
@@ -260,6 +270,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       if (!ok && lane == 0) fail(code);
       return ok != 0;
     };
+    fetch_cols(0);
     // K(0), K(1); then K(j) as soon as QK(j-2) has released its slot.  The
     // column terms of tile j reuse ring entry j mod 4: QK(j-2) was issued
     // after the softmax released S(j-3), so it has finished tile j-4.
@@ -267,9 +278,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     if (nt > 1) load_k(1);
     for (int j = 2; j < nt; ++j) {
       if (!wait_local(P_KEMPTY0 + (j & 1), ((j - 2) >> 1) & 1, DEV_TIMEOUT_EMPTY)) break;
+      if (lane == 0) PAIR_TR(j, 12);
       load_k(j);
     }
   } else if (warp == W_VPROD) {
+#ifdef IPA_TRACE
+    // tracing build only: one idle lane of CTA 0 records when each K slot fills
+    if (lane == 1 && rank == 0 && trace_slot >= 0) {
+      for (int j = 0; j < nt; ++j) {
+        if (!mbar_wait_bounded_cluster(bar(P_KFULL0 + (j & 1)), (j >> 1) & 1, abort_flag)) break;
+        PAIR_TR(j, 11);
+      }
+    }
+#endif
     // ------------------------------------------------ V producer (each CTA, one thread)
     if (lane == 0) {
       const uint32_t vbytes = static_cast<uint32_t>(np / 2) * 16384u + 8192u;
@@ -278,12 +299,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           fail(DEV_TIMEOUT_EMPTY);
           break;
         }
+        PAIR_TR(j, 15);
         const int J2 = (start + j) % nt;
         const uint32_t vf = bar0(P_VFULL);
         const uint32_t st = sb + SP_V;
         mbar_arrive_expect_tx_remote(vf, vbytes);
-        for (int p = 0; p < np / 2; ++p)
-          tma_load_3d_pair(st + 16384 * p, &tm_z2v, vf, 64 * (static_cast<int>(rank) * (np / 2) + p), J2 * 128, b);
+        tma_load_4d_pair(st, &tm_z2v, vf, 0, J2 * 128, static_cast<int>(rank) * (np / 2), b);   // own np/2 panels
         tma_load_3d_pair(st + V_VH, &tm_vh, vf, 32 * static_cast<int>(rank), J2 * 128, bh);
         PAIR_TR(j, 14);
       }
@@ -301,6 +322,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       const uint32_t idv = idesc_f16(256, 64, true);
       const uint32_t tS = tmem + TM_S, tP = tmem + TM_P, tOz = tmem, tOv = tmem + DZ;
       bool issued_any = false;
+      // Q.K(j) as soon as its K tile is in and S(j-1) has been read, then
+      // P.V(j-1) once P(j-1) and V(j-1) are in
       for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
           const int s = j & 1;
@@ -578,13 +601,12 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
   CUtensorMap tqh, tkh, tz2k, tz2v, tvh, tz1;
   const uint64_t bh = static_cast<uint64_t>(a.B) * a.H;
   const uint64_t rowb = static_cast<uint64_t>(a.L) * DH * 2;
-  const uint64_t zrow = static_cast<uint64_t>(a.DZ) * 2, zb = static_cast<uint64_t>(a.L) * a.DZ * 2;
   bool ok = encode_tmap_f16_3d(&tqh, ws + w.qh, DH, a.L, bh, DH * 2, rowb, 64, QT) &&
             encode_tmap_f16_3d(&tkh, ws + w.kh, DH, a.L, bh, DH * 2, rowb, 64, 64) &&
-            encode_tmap_f16_3d(&tz2k, ws + w.z2, a.DZ, a.L, a.B, zrow, zb, 64, 64) &&
-            encode_tmap_f16_3d(&tz2v, ws + w.z2, a.DZ, a.L, a.B, zrow, zb, 64, 128) &&
+            encode_tmap_f16_panels(&tz2k, ws + w.z2, a.DZ, a.L, a.B, 64, a.DZ / 64) &&
+            encode_tmap_f16_panels(&tz2v, ws + w.z2, a.DZ, a.L, a.B, 128, a.DZ / 128) &&
             encode_tmap_f16_3d(&tvh, ws + w.vh, DH, a.L, bh, DH * 2, rowb, 32, 128, 64) &&
-            encode_tmap_f16_3d(&tz1, ws + w.z1h, a.DZ, a.L, a.B, zrow, zb, 64, 128);
+            encode_tmap_f16_panels(&tz1, ws + w.z1h, a.DZ, a.L, a.B, 128, a.DZ / 64);
   if (!ok) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(ipa_attention_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(SP_ALLOC));
@@ -604,7 +626,7 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
   t.out = a.out; t.err = a.err;
   const int pairs = static_cast<int>(bh) * t.nqp;
   t.trace_cta0 = 0;
-  t.trace_cta1 = 2 * (pairs / 2);
+  t.trace_cta1 = 1;   // the peer CTA of the first pair
   ipa_attention_pair_kernel<<<static_cast<unsigned>(2 * pairs), NT, SP_ALLOC, stream>>>(tqh, tkh, tz2k, tz2v, tvh, tz1, t);
   return cudaGetLastError();
 }

@@ -98,70 +98,61 @@ __device__ __forceinline__ void write_row(const float* O, float* dst, int lane, 
 }
 
 // Phase A for the 16 rows of one warp: z1 (.) O_pair summed over the R
-// factors into O_pair[0 .. Cz) of each staged row.  z1 rows load coalesced,
-// 4 rows per group, the next group's loads in flight while the current one is
-// folded.  NCZ = Cz / 32 > 0: a lane's columns c = lane + 32 t (all R factors)
-// fold into pair feature lane + 32 (t mod NCZ) in registers (every column a
-// lane reads or writes is its own).  NCZ = 0 (Cz not a multiple of 32): the
-// products are written in place and reduced in a second pass.
-template <int NCZ>
-__device__ __noinline__ void fold_pairs_rows(const EpilogueArgs& e, int warp, int lane) {
+// factors into O_pair[0 .. Cz) of each staged row.  z1 rows are read as
+// float4 (lane q holds columns 4q .. 4q + 3 and 128 + 4q ..), two rows ahead of
+// the row being folded: wide loads keep the number of outstanding L1 requests
+// low, which is what bounds this phase.  When Cz % 128 == 0 all R factors of
+// a pair feature sit on one lane and fold in registers; otherwise the
+// products are written in place and reduced in a second, float4 pass.
+static __device__ __noinline__ void fold_pairs_rows(const EpilogueArgs& e, int warp, int lane) {
   const int pitch = stage_pitch(e.DZ);
-  const int nz = (e.RCz + 31) >> 5;   // z1 values per lane per row (<= 8)
-  float zc[4][8], zn[4][8];
-  auto load_group = [&](int g, float (&zz)[4][8]) {
+  const int nq = e.RCz >> 2;                  // float4 columns holding pair factors (RCz % 16 == 0)
+  const int R = e.RCz / e.Cz, cq = e.Cz >> 2;
+  const bool lane_local = (e.Cz & 127) == 0;
+  const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 zb[3][2];
+  auto load_row = [&](int rr, float4 (&z)[2]) {
+    const int grow = e.row0 + warp * 16 + rr;
+    const bool in = rr < 16 && grow < e.L;
+    const float4* zr =
+        reinterpret_cast<const float4*>(e.z1f + (static_cast<int64_t>(e.b) * e.L + (in ? grow : 0)) * e.DZ);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int grow = e.row0 + warp * 16 + 4 * g + q;
-      const float* zr = e.z1f + (static_cast<int64_t>(e.b) * e.L + (grow < e.L ? grow : 0)) * e.DZ;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const int c = lane + 32 * t;
-        zz[q][t] = (t < nz && c < e.RCz && grow < e.L) ? __ldg(zr + c) : 0.f;
-      }
+    for (int u = 0; u < 2; ++u) {
+      const int q = lane + 32 * u;
+      z[u] = (in && q < nq) ? __ldg(zr + q) : zero4;
     }
   };
-  load_group(0, zc);
-#pragma unroll 1
-  for (int g = 0; g < 4; ++g) {
-    if (g < 3) load_group(g + 1, zn);
+  auto mul4 = [](float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); };
+  load_row(0, zb[0]);
+  load_row(1, zb[1]);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float* P = e.stage + (warp * 16 + 4 * g + q) * pitch + 64;
-      if (NCZ > 0) {
-        float acc[NCZ > 0 ? NCZ : 1];
-#pragma unroll
-        for (int j = 0; j < (NCZ > 0 ? NCZ : 1); ++j) acc[j] = 0.f;
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          if (t < nz) acc[t % (NCZ > 0 ? NCZ : 1)] = fmaf(zc[q][t], P[lane + 32 * t], acc[t % (NCZ > 0 ? NCZ : 1)]);
-#pragma unroll
-        for (int j = 0; j < (NCZ > 0 ? NCZ : 1); ++j) P[lane + 32 * j] = acc[j];
-      } else {
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int c = lane + 32 * t;
-          if (t < nz && c < e.RCz) P[c] *= zc[q][t];
-        }
-      }
+  for (int rr = 0; rr < 16; ++rr) {
+    load_row(rr + 2, zb[(rr + 2) % 3]);
+    float4* P = reinterpret_cast<float4*>(e.stage + (warp * 16 + rr) * pitch + 64);
+    const float4 z0 = zb[rr % 3][0], z1 = zb[rr % 3][1];
+    if (lane_local && R == 2) {              // Cz = 128: columns lane and 32 + lane hold factors 0 and 1
+      const float4 o0 = P[lane], o1 = P[32 + lane];
+      P[lane] = make_float4(fmaf(z1.x, o1.x, z0.x * o0.x), fmaf(z1.y, o1.y, z0.y * o0.y),
+                            fmaf(z1.z, o1.z, z0.z * o0.z), fmaf(z1.w, o1.w, z0.w * o0.w));
+    } else {                                 // R == 1, or products in place before the reduction
+      if (lane < nq) P[lane] = mul4(P[lane], z0);
+      if (32 + lane < nq) P[32 + lane] = mul4(P[32 + lane], z1);
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int t = 0; t < 8; ++t) zc[q][t] = zn[q][t];
   }
   __syncwarp();
-  const int R = e.RCz / e.Cz;
-  if (NCZ == 0 && R > 1) {
+  if (!lane_local && R > 1) {
     for (int rr = 0; rr < 16; ++rr) {
-      float* P = e.stage + (warp * 16 + rr) * pitch + 64;
+      float4* P = reinterpret_cast<float4*>(e.stage + (warp * 16 + rr) * pitch + 64);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int cc = lane + 32 * u;
-        if (cc < e.Cz) {
-          float acc = P[cc];
-          for (int r2 = 1; r2 < R; ++r2) acc += P[r2 * e.Cz + cc];
-          P[cc] = acc;
+      for (int u = 0; u < 2; ++u) {
+        const int c4 = lane + 32 * u;
+        if (c4 < cq) {
+          float4 acc = P[c4];
+          for (int r2 = 1; r2 < R; ++r2) {
+            const float4 v = P[r2 * cq + c4];
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+          }
+          P[c4] = acc;
         }
       }
     }
@@ -170,9 +161,8 @@ __device__ __noinline__ void fold_pairs_rows(const EpilogueArgs& e, int warp, in
 }
 
 // Called by all 8 warps (warp = 0..7) after the staged rows are complete;
-// warp w handles rows 16 w .. 16 w + 15 of the tile: phase A (above, one
-// instantiation chosen per call), then phase B: the output rows with
-// coalesced stores.  No global load is issued after a global store.
+// warp w handles rows 16 w .. 16 w + 15 of the tile: phase A (above), then
+// phase B: the output rows with coalesced stores.  No global load is issued after a global store.
 template <int C, int PV>
 __device__ __forceinline__ void write_rows(const EpilogueArgs& e, int warp, int lane) {
   const int pitch = stage_pitch(e.DZ);
@@ -187,17 +177,7 @@ __device__ __forceinline__ void write_rows(const EpilogueArgs& e, int warp, int 
   } while (0)
 #endif
   EPI_TR(0);
-  switch ((e.Cz & 31) == 0 ? e.Cz >> 5 : 0) {
-    case 1: fold_pairs_rows<1>(e, warp, lane); break;
-    case 2: fold_pairs_rows<2>(e, warp, lane); break;
-    case 3: fold_pairs_rows<3>(e, warp, lane); break;
-    case 4: fold_pairs_rows<4>(e, warp, lane); break;
-    case 5: fold_pairs_rows<5>(e, warp, lane); break;
-    case 6: fold_pairs_rows<6>(e, warp, lane); break;
-    case 7: fold_pairs_rows<7>(e, warp, lane); break;
-    case 8: fold_pairs_rows<8>(e, warp, lane); break;
-    default: fold_pairs_rows<0>(e, warp, lane); break;
-  }
+  fold_pairs_rows(e, warp, lane);
   EPI_TR(1);
 #pragma unroll 1
   for (int rr = 0; rr < 16; ++rr) {
