@@ -44,7 +44,8 @@ UNIT = "TFLOP/s"
 # it was taken on (sha256 over the sources listed in CORE_SOURCES).
 CORE_KERNEL = "ipa_attention_pair_kernel"
 CORE_SOURCES = ("ipa_attention_pair.cu", "ipa_epilogue.cuh", "sm100.cuh")
-NCU_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None}
+NCU_TRAFFIC = {"kernel_sha256": "0f5b328582d70debf43612647001a9ef5309a184971ec7a338d824fa4c5f1252",
+               "bytes_per_launch": 30.45e6}
 
 
 def ipa_flops(B, L, n_valid=None):
