@@ -38,6 +38,7 @@ from rna_structure_models_b200.synth import GeoDims, IpaDims, geo_inputs, ipa_in
 H, C, PQ, PV, R, CZ = 12, 16, 4, 8, 2, 128
 METRIC = "fused IPA attention TFLOP/s and % bf16 tensor-pipe peak at L=4096 (1xB200)"
 UNIT = "TFLOP/s"
+REF_BUDGET_S = 90.0
 
 # DRAM traffic of one launch of the core kernel (the CTA-pair kernel at this
 # workload's R Cz = 256) from an ncu capture, valid only for the kernel source
@@ -169,8 +170,14 @@ def run_reference(args, rank, world):
         return
     L = args.L
     ms = []
-    rows_per_step = args.ref_rows
     inp = ipa_inputs(IpaDims(B=1, L=L, H=H, C=C, Pq=PQ, Pv=PV, R=R, Cz=CZ), 0)
+    rows_per_step = args.ref_rows
+    if rows_per_step is None:
+        # size each step so that the whole --steps K --warmup W run takes about
+        # REF_BUDGET_S seconds of oracle time (calibrated on 8 rows, untimed)
+        _, _, t8 = cpu_oracle_sample(L, 1e9, 8, inp=inp)
+        per_row = t8 / 8
+        rows_per_step = int(max(1, min(64, REF_BUDGET_S / max(1, args.steps + args.warmup) / per_row)))
     for s in range(args.warmup + args.steps):
         _, nrows, dt = cpu_oracle_sample(L, 1e9, rows_per_step, inp=inp)
         if s >= args.warmup:
@@ -197,7 +204,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--L", type=int, default=4096)
-    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--ref-rows", type=int, default=None,
+                    help="query rows per reference step (default: sized to ~90 s for the whole run)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variant", action="store_true")
@@ -301,7 +309,7 @@ def main():
         res = torch.empty((1, L, H, plan.F), dtype=torch.float32, pin_memory=True)
         d2h = res.numel() * res.element_size()
         for _ in range(max(1, min(args.warmup, 3))):
-            o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev)
+            o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev, out=res)
         torch.cuda.synchronize()
         ke = max(3, min(K, 50))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -310,7 +318,7 @@ def main():
         torch.cuda.synchronize()
         e0.record()
         for _ in range(ke):
-            o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev)
+            o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev, out=res)
         e1.record()
         torch.cuda.synchronize()
         te = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
