@@ -5,12 +5,15 @@
 //                        (R, t, valid), partial sums of the valid origins, and
 //                        the pair factors z2 (fp16) and z1 (fp32 and fp16)
 //                        padded to DZ.
-//   ipa_reduce_kernel -- one CTA per batch: centroid of the valid origins,
-//                        query-tile (128) and key-tile (64) origins relative
-//                        to it; per-head point coefficient and pair-bias
-//                        weights w_L log2(e) w_bias[c, h] (batch 0's CTA).
-//   ipa_rows_kernel   -- one thread per (b, h, i): Q_h, K_h, V_h rows (64
-//                        fp16 each) and the two small fp32 row terms.
+//   ipa_rows_kernel   -- one thread per (b, i, h), heads fastest: the
+//                        centroid of the valid origins (each block reduces
+//                        the tile partial sums of its batches), query-tile
+//                        (128) and key-tile (64) origins relative to it, the
+//                        Q_h, K_h, V_h rows (64 fp16 each) and the two small
+//                        fp32 row terms; designated threads also write the
+//                        centroid, tile origins, per-head point coefficient
+//                        and pair-bias weights w_L log2(e) w_bias[c, h] that
+//                        the core kernel reads.
 //
 // Augmented row layout for the (C, Pq, Pv) = (16, 4, 8) head shape, with
 // c = log2(e) w_L gamma_h w_C / 2, gq' / gk' the global query / key points
@@ -131,87 +134,18 @@ __global__ void __launch_bounds__(256) ipa_tile_kernel(const TileArgs a) {
   ipa_tile_copy_pairs(a, b, i0, 0, tid);
 }
 
-struct ReduceArgs {
-  int B, L, H, Cz, RCz, DZ, nqt, nkt;
+struct RowArgs {
+  int B, L, H, nqt, nkt, Cz, RCz, DZ;
+  float qscale;    // log2(e) w_L scalar_scale
   float w_L, w_C;
-  View gamma, w_bias;
-  const float4* part;
-  float4* cen;     // [B]
+  View q, k, v, q_pts, k_pts, v_pts, gamma, w_bias;
+  const float4* frame;
+  const float4* part;   // [B, nkt] sum of valid origins and count per 64-residue tile
+  float4* cen;     // [B]        written here for the core kernel
   float4* oq;      // [B, nqt]
   float4* ok;      // [B, nkt]
   float* headc;    // [H]
   float* wqp;      // [H, DZ]
-};
-
-__global__ void __launch_bounds__(256) ipa_reduce_kernel(const ReduceArgs a) {
-  const int b = blockIdx.x, tid = threadIdx.x;
-  __shared__ double red[4][8];
-  __shared__ float cen[3];
-  double sx = 0, sy = 0, sz = 0, sn = 0;
-  for (int J = tid; J < a.nkt; J += blockDim.x) {
-    const float4 p = a.part[b * a.nkt + J];
-    sx += p.x; sy += p.y; sz += p.z; sn += p.w;
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    sx += __shfl_xor_sync(0xffffffffu, sx, off);
-    sy += __shfl_xor_sync(0xffffffffu, sy, off);
-    sz += __shfl_xor_sync(0xffffffffu, sz, off);
-    sn += __shfl_xor_sync(0xffffffffu, sn, off);
-  }
-  const int w = tid >> 5, lane = tid & 31;
-  if (lane == 0) { red[0][w] = sx; red[1][w] = sy; red[2][w] = sz; red[3][w] = sn; }
-  __syncthreads();
-  if (tid == 0) {
-    double tx = 0, ty = 0, tz = 0, tn = 0;
-    for (int k = 0; k < static_cast<int>(blockDim.x >> 5); ++k) {
-      tx += red[0][k]; ty += red[1][k]; tz += red[2][k]; tn += red[3][k];
-    }
-    const double inv = tn > 0 ? 1.0 / tn : 0.0;
-    cen[0] = static_cast<float>(tx * inv);
-    cen[1] = static_cast<float>(ty * inv);
-    cen[2] = static_cast<float>(tz * inv);
-    a.cen[b] = make_float4(cen[0], cen[1], cen[2], static_cast<float>(tn));
-  }
-  __syncthreads();
-  const float cx = cen[0], cy = cen[1], cz = cen[2];
-  for (int J = tid; J < a.nkt; J += blockDim.x) {
-    const float4 p = a.part[b * a.nkt + J];
-    const float inv = p.w > 0.f ? 1.f / p.w : 0.f;
-    a.ok[b * a.nkt + J] = p.w > 0.f ? make_float4(p.x * inv - cx, p.y * inv - cy, p.z * inv - cz, 0.f)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int I = tid; I < a.nqt; I += blockDim.x) {
-    float4 p = a.part[b * a.nkt + 2 * I];
-    if (2 * I + 1 < a.nkt) {
-      const float4 p2 = a.part[b * a.nkt + 2 * I + 1];
-      p.x += p2.x; p.y += p2.y; p.z += p2.z; p.w += p2.w;
-    }
-    const float inv = p.w > 0.f ? 1.f / p.w : 0.f;
-    a.oq[b * a.nqt + I] = p.w > 0.f ? make_float4(p.x * inv - cx, p.y * inv - cy, p.z * inv - cz, 0.f)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  if (b == 0) {
-    for (int h = tid; h < a.H; h += blockDim.x)
-      a.headc[h] = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
-    for (int e = tid; e < a.H * a.DZ; e += blockDim.x) {
-      const int h = e / a.DZ, col = e % a.DZ;
-      float val = 0.f;
-      if (col < a.RCz) val = kLog2e * a.w_L * ldf(a.w_bias, (col % a.Cz) * a.w_bias.s[0] + h * a.w_bias.s[1]);
-      a.wqp[e] = val;
-    }
-  }
-}
-
-struct RowArgs {
-  int B, L, H, nqt, nkt;
-  float qscale;    // log2(e) w_L scalar_scale
-  View q, k, v, q_pts, k_pts, v_pts;
-  const float4* frame;
-  const float4* cen;
-  const float4* oq;
-  const float4* ok;
-  const float* headc;
   uint4* qh;       // [B*H, L, 64] fp16 (8 x uint4 per row)
   uint4* kh;
   uint4* vh;
@@ -220,49 +154,133 @@ struct RowArgs {
   int* err;
 };
 
+// N consecutive elements of a row: float4 loads when the row is contiguous
+// and 16-byte aligned (the common dense layout), element loads otherwise.
 template <int N>
 __device__ __forceinline__ void load_row(const View& v, int64_t base, int64_t st, float (&out)[N]) {
+  const float* p = reinterpret_cast<const float*>(v.p) + base;
+  if (N % 4 == 0 && st == 1 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
 #pragma unroll
-  for (int e = 0; e < N; ++e) out[e] = ldf(v, base + e * st);
+    for (int e = 0; e < N; e += 4) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(p) + e / 4);
+      out[e] = x.x; out[e + 1] = x.y; out[e + 2] = x.z; out[e + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < N; ++e) out[e] = p[e * st];
+  }
+}
+
+// Origin (mean of the valid centred frame origins) of a run of 64-residue
+// tiles [J0, J1) of batch b, from their partial sums; 0 for an empty run.
+__device__ __forceinline__ float4 tile_origin(const float4* part, int J0, int J1, float4 cen) {
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int J = J0; J < J1; ++J) {
+    const float4 p = part[J];
+    s.x += p.x; s.y += p.y; s.z += p.z; s.w += p.w;
+  }
+  if (!(s.w > 0.f)) return make_float4(0.f, 0.f, 0.f, 0.f);
+  const float inv = 1.f / s.w;
+  return make_float4(s.x * inv - cen.x, s.y * inv - cen.y, s.z * inv - cen.z, 0.f);
 }
 
 template <int C, int PQ, int PV>
 __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   static_assert(C + 9 * PQ + 2 <= DH && C + 6 * PV <= DH, "augmented rows wider than 64");
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  // heads fastest: the threads of a residue read its contiguous [H, ...]
+  // input rows together
   const int64_t total = static_cast<int64_t>(a.B) * a.H * a.L;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x;
+  const int64_t t = t0 + threadIdx.x;
+  const int64_t hl = static_cast<int64_t>(a.H) * a.L;
+
+  // centroid of the valid origins of every batch this block touches (double
+  // sums over the per-tile partial sums; at most 128 batches per block)
+  __shared__ float4 cen_s[128];
+  __shared__ double red[4][4];
+  const int bfirst = static_cast<int>(t0 / hl);
+  const int blast = static_cast<int>((t0 + blockDim.x - 1 < total ? t0 + blockDim.x - 1 : total - 1) / hl);
+  for (int bb = bfirst; bb <= blast; ++bb) {
+    double sx = 0, sy = 0, sz = 0, sn = 0;
+    for (int J = threadIdx.x; J < a.nkt; J += blockDim.x) {
+      const float4 p = a.part[static_cast<int64_t>(bb) * a.nkt + J];
+      sx += p.x; sy += p.y; sz += p.z; sn += p.w;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sx += __shfl_xor_sync(0xffffffffu, sx, off);
+      sy += __shfl_xor_sync(0xffffffffu, sy, off);
+      sz += __shfl_xor_sync(0xffffffffu, sz, off);
+      sn += __shfl_xor_sync(0xffffffffu, sn, off);
+    }
+    if ((threadIdx.x & 31) == 0) {
+      const int w = threadIdx.x >> 5;
+      red[w][0] = sx; red[w][1] = sy; red[w][2] = sz; red[w][3] = sn;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double tx = 0, ty = 0, tz = 0, tn = 0;
+      for (int w = 0; w < 4; ++w) { tx += red[w][0]; ty += red[w][1]; tz += red[w][2]; tn += red[w][3]; }
+      const double inv = tn > 0 ? 1.0 / tn : 0.0;
+      cen_s[bb - bfirst] = make_float4(static_cast<float>(tx * inv), static_cast<float>(ty * inv),
+                                       static_cast<float>(tz * inv), static_cast<float>(tn));
+    }
+    __syncthreads();
+  }
   if (t >= total) return;
-  const int i = static_cast<int>(t % a.L);
-  const int bh = static_cast<int>(t / a.L);
-  const int h = bh % a.H, b = bh / a.H;
+  const int h = static_cast<int>(t % a.H);
+  const int i = static_cast<int>((t / a.H) % a.L);
+  const int b = static_cast<int>(t / hl);
+  const int bh = b * a.H + h;
+  const int64_t orow = static_cast<int64_t>(bh) * a.L + i;   // row of the [B*H, L] outputs
+
+  const float4 cn = cen_s[b - bfirst];
+  const float4* partb = a.part + static_cast<int64_t>(b) * a.nkt;
+  const int Jq = (i / QT) * (QT / KT);
+  const float4 oqv = tile_origin(partb, Jq, Jq + QT / KT < a.nkt ? Jq + QT / KT : a.nkt, cn);
+  const float4 okv = tile_origin(partb, i / KT, i / KT + 1, cn);
+  // the values the core kernel reads per batch / tile / head, one writer each
+  if (h == 0) {
+    if (i == 0) a.cen[b] = cn;
+    if (i % QT == 0) a.oq[b * a.nqt + i / QT] = oqv;
+    if (i % KT == 0) a.ok[b * a.nkt + i / KT] = okv;
+  }
+  const float c = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
+  if (b == 0) {
+    if (i == 0) a.headc[h] = c;
+    // the [H, DZ] pair-bias weights, one entry per thread of batch 0
+    for (int64_t e = t; e < static_cast<int64_t>(a.H) * a.DZ; e += hl) {
+      const int he = static_cast<int>(e / a.DZ), col = static_cast<int>(e % a.DZ);
+      a.wqp[e] = col < a.RCz ? kLog2e * a.w_L * ldf(a.w_bias, (col % a.Cz) * a.w_bias.s[0] + he * a.w_bias.s[1]) : 0.f;
+    }
+  }
 
   const float4* fr = a.frame + (static_cast<int64_t>(b) * a.L + i) * 4;
   const float4 f0 = fr[0], f1 = fr[1], f2 = fr[2], f3 = fr[3];
-  const float4 cn = a.cen[b];
   const float Rm[9] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w, f2.x};
   const float tc[3] = {f2.y - cn.x, f2.z - cn.y, f2.w - cn.z};
   const bool valid = f3.x != 0.f;
-  const float4 oqv = a.oq[b * a.nqt + i / QT];
-  const float4 okv = a.ok[b * a.nkt + i / KT];
   const float oqa[3] = {oqv.x, oqv.y, oqv.z}, oka[3] = {okv.x, okv.y, okv.z};
-  const float c = a.headc[h];
 
   float qs[C], ks[C], vs[C], qp[PQ * 3], kp[PQ * 3], vp[PV * 3];
   load_row(a.q, b * a.q.s[0] + i * a.q.s[1] + h * a.q.s[2], a.q.s[3], qs);
   load_row(a.k, b * a.k.s[0] + i * a.k.s[1] + h * a.k.s[2], a.k.s[3], ks);
   load_row(a.v, b * a.v.s[0] + i * a.v.s[1] + h * a.v.s[2], a.v.s[3], vs);
+  auto load_pts = [&](const View& v, auto& dst) {
+    const int64_t base = b * v.s[0] + i * v.s[1] + h * v.s[2];
+    if (v.s[4] == 1 && v.s[3] == 3) {
+      load_row(v, base, 1, dst);             // [points, xyz] dense
+    } else {
+      constexpr int NP = sizeof(dst) / sizeof(float) / 3;
 #pragma unroll
-  for (int p = 0; p < PQ; ++p)
+      for (int p = 0; p < NP; ++p)
 #pragma unroll
-    for (int y = 0; y < 3; ++y) {
-      qp[3 * p + y] = ldf(a.q_pts, b * a.q_pts.s[0] + i * a.q_pts.s[1] + h * a.q_pts.s[2] + p * a.q_pts.s[3] + y * a.q_pts.s[4]);
-      kp[3 * p + y] = ldf(a.k_pts, b * a.k_pts.s[0] + i * a.k_pts.s[1] + h * a.k_pts.s[2] + p * a.k_pts.s[3] + y * a.k_pts.s[4]);
+        for (int y = 0; y < 3; ++y) dst[3 * p + y] = ldf(v, base + p * v.s[3] + y * v.s[4]);
     }
-#pragma unroll
-  for (int p = 0; p < PV; ++p)
-#pragma unroll
-    for (int y = 0; y < 3; ++y)
-      vp[3 * p + y] = ldf(a.v_pts, b * a.v_pts.s[0] + i * a.v_pts.s[1] + h * a.v_pts.s[2] + p * a.v_pts.s[3] + y * a.v_pts.s[4]);
+  };
+  load_pts(a.q_pts, qp);
+  load_pts(a.k_pts, kp);
+  load_pts(a.v_pts, vp);
 
   // frames applied: gq' = R q + t' - o_I, gk' = R k + t' - o_J, gv = R v + t'
   float gq[PQ * 3], gk[PQ * 3], gv[PV * 3];
@@ -303,7 +321,7 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   };
   auto hi_of = [](float x) { return __half2float(__float2half_rn(x)); };
   // Q_h: [ scaled q | gq' hi | gq' hi | gq' lo | -1 -1 | 0 ]
-  store_row(a.qh + t * 8, [&](int col) -> float {
+  store_row(a.qh + orow * 8, [&](int col) -> float {
     if (col < C) return a.qscale * qs[col];
     if (col < C + 9 * PQ) {
       const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
@@ -313,7 +331,7 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     return col < C + 9 * PQ + 2 ? -1.f : 0.f;
   });
   // K_h: [ k | 2c gk' hi | lo | hi | c|gk'|^2 hi, lo | 0 ]
-  store_row(a.kh + t * 8, [&](int col) -> float {
+  store_row(a.kh + orow * 8, [&](int col) -> float {
     if (col < C) return ks[col];
     if (col < C + 9 * PQ) {
       const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
@@ -327,7 +345,7 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     return 0.f;
   });
   // V_h: [ v | gv hi | gv lo ]
-  store_row(a.vh + t * 8, [&](int col) -> float {
+  store_row(a.vh + orow * 8, [&](int col) -> float {
     if (col < C) return vs[col];
     if (col < C + 6 * PV) {
       const int u = col - C, part = u / (3 * PV), e = u % (3 * PV);
@@ -340,8 +358,8 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     sq[0] = sq[1] = sq[2] = 0.f;
     sk[0] = sk[1] = sk[2] = 0.f;
   }
-  a.rowq[t] = make_float4(sq[0], sq[1], sq[2], 0.f);
-  a.colk[t] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
+  a.rowq[orow] = make_float4(sq[0], sq[1], sq[2], 0.f);
+  a.colk[orow] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
   if (overflow) record_error(a.err, DEV_NONFINITE);
 }
 
@@ -361,22 +379,18 @@ cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
   ta.z1h = reinterpret_cast<__half*>(ws + w.z1h);
   ipa_tile_kernel<<<dim3(a.nkt, a.B, a.DZ / 64), 256, 0, stream>>>(ta);
 
-  ReduceArgs ra{};
-  ra.B = a.B; ra.L = a.L; ra.H = a.H; ra.Cz = a.Cz; ra.RCz = a.RCz; ra.DZ = a.DZ; ra.nqt = a.nqt; ra.nkt = a.nkt;
-  ra.w_L = a.w_L; ra.w_C = a.w_C; ra.gamma = a.gamma; ra.w_bias = a.w_bias;
-  ra.part = ta.part;
-  ra.cen = reinterpret_cast<float4*>(ws + w.cen);
-  ra.oq = reinterpret_cast<float4*>(ws + w.oq);
-  ra.ok = reinterpret_cast<float4*>(ws + w.ok);
-  ra.headc = reinterpret_cast<float*>(ws + w.headc);
-  ra.wqp = reinterpret_cast<float*>(ws + w.wqp);
-  ipa_reduce_kernel<<<a.B, 256, 0, stream>>>(ra);
-
   RowArgs r{};
-  r.B = a.B; r.L = a.L; r.H = a.H; r.nqt = a.nqt; r.nkt = a.nkt;
+  r.B = a.B; r.L = a.L; r.H = a.H; r.nqt = a.nqt; r.nkt = a.nkt; r.Cz = a.Cz; r.RCz = a.RCz; r.DZ = a.DZ;
   r.qscale = kLog2e * a.w_L * a.scalar_scale;
+  r.w_L = a.w_L; r.w_C = a.w_C;
   r.q = a.q; r.k = a.k; r.v = a.v; r.q_pts = a.q_pts; r.k_pts = a.k_pts; r.v_pts = a.v_pts;
-  r.frame = ta.frame; r.cen = ra.cen; r.oq = ra.oq; r.ok = ra.ok; r.headc = ra.headc;
+  r.gamma = a.gamma; r.w_bias = a.w_bias;
+  r.frame = ta.frame; r.part = ta.part;
+  r.cen = reinterpret_cast<float4*>(ws + w.cen);
+  r.oq = reinterpret_cast<float4*>(ws + w.oq);
+  r.ok = reinterpret_cast<float4*>(ws + w.ok);
+  r.headc = reinterpret_cast<float*>(ws + w.headc);
+  r.wqp = reinterpret_cast<float*>(ws + w.wqp);
   r.qh = reinterpret_cast<uint4*>(ws + w.qh);
   r.kh = reinterpret_cast<uint4*>(ws + w.kh);
   r.vh = reinterpret_cast<uint4*>(ws + w.vh);
