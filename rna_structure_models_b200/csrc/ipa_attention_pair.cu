@@ -108,7 +108,7 @@ static_assert(SP_QP + 128u * stage_pitch(MAX_DZ) * 4u <= SP_AUX, "epilogue stage
 
 enum {
   // local barriers (waited on in each CTA)
-  P_QFULL = 0, P_SFULL, P_PFREE, P_KEMPTY0, P_VEMPTY = P_KEMPTY0 + 2, P_COLFULL0, P_DRAIN = P_COLFULL0 + NCOL,
+  P_QFULL = 0, P_SFULL, P_PFREE, P_KEMPTY0, P_COLFULL0 = P_KEMPTY0 + 2, P_DRAIN = P_COLFULL0 + NCOL,
   // barriers waited on by the MMA thread (used in CTA 0)
   P_KFULL0, P_VFULL = P_KFULL0 + 2, P_SFREE, P_PFULL, P_QREADY, P_COUNT
 };
@@ -169,7 +169,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     mbar_init(bar(P_PFREE), 1);
     mbar_init(bar(P_KEMPTY0), 1);
     mbar_init(bar(P_KEMPTY0 + 1), 1);
-    mbar_init(bar(P_VEMPTY), 1);
     for (int s = 0; s < NCOL; ++s) mbar_init(bar(P_COLFULL0 + s), 1);
     mbar_init(bar(P_DRAIN), 1);
     mbar_init(bar(P_KFULL0), 2);
@@ -295,7 +294,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     if (lane == 0) {
       const uint32_t vbytes = static_cast<uint32_t>(np / 2) * 16384u + 8192u;
       for (int j = 0; j < nt; ++j) {
-        if (j > 0 && !mbar_wait_bounded(bar(P_VEMPTY), (j - 1) & 1, abort_flag)) {
+        // the V slot is free once P.V(j-1) has completed, which PFREE
+        // signals; this thread cannot fall two phases behind because P.V(j)
+        // needs V(j) first
+        if (j > 0 && !mbar_wait_bounded(bar(P_PFREE), (j - 1) & 1, abort_flag)) {
           fail(DEV_TIMEOUT_EMPTY);
           break;
         }
@@ -360,8 +362,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
             umma2_ts(tOz, tP + 8 * k, mn128(st + 2048 * k), idz, acc);
             umma2_ts(tOv, tP + 8 * k, mn64(st + V_VH + 1024 * k), idv, acc);
           }
-          umma2_commit_both(bar(P_PFREE));
-          umma2_commit_both(bar(P_VEMPTY));
+          umma2_commit_both(bar(P_PFREE));   // P and the V slot are free
           PAIR_TR(jj, 4);
         }
       }

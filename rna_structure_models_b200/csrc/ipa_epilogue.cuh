@@ -179,7 +179,7 @@ __device__ __forceinline__ void write_rows(const EpilogueArgs& e, int warp, int 
   EPI_TR(0);
   fold_pairs_rows(e, warp, lane);
   EPI_TR(1);
-#pragma unroll 1
+#pragma unroll 2
   for (int rr = 0; rr < 16; ++rr) {
     const int rloc = warp * 16 + rr;
     const int grow = e.row0 + rloc;
