@@ -29,7 +29,7 @@ import numpy as np
 
 __all__ = [
     "IpaDims", "GeoDims", "ipa_inputs", "geo_inputs", "ipa_preset", "geo_preset",
-    "IPA_PRESETS", "random_rotations", "random_walk",
+    "IPA_PRESETS", "random_rotations", "random_walk", "MeetDims", "meet_inputs",
 ]
 
 
@@ -57,6 +57,16 @@ class GeoDims:
     H: int
     M: int
     Cout: int
+
+
+@dataclass(frozen=True)
+class MeetDims:
+    """Distance-aware attention (MEET §2.2): B batch, L atoms, H heads, C
+    query/key/value channels per head."""
+    B: int = 1
+    L: int = 512
+    H: int = 8
+    C: int = 16
 
 
 def random_rotations(rng: np.random.Generator, n: int) -> np.ndarray:
@@ -175,6 +185,32 @@ def geo_inputs(dims: GeoDims, seed: int = 0, *, pair_drop: float = 0.2,
         "frame_mask": np.ascontiguousarray(frame_mask),
         "pair_mask": pair_mask,
     }
+
+
+def meet_inputs(dims: MeetDims, seed: int = 0, *, masked_tail_frac: float = 0.0) -> dict:
+    """Seeded inputs of the distance-aware attention of MEET §2.2.
+
+    Draw order: walk (coordinates x, 3.8 A steps), q, k, v ~ N(0, 1),
+    rho_h ~ U(0.5, 1.5) / sqrt(C) (attention scale), s_h ~ U(0.05, 0.3)
+    (distance scale, per A), masks.  The pages give no distributions for
+    rho and s; these keep the distance term and the dot product of similar
+    size for neighbours a few residues apart.
+    """
+    B, L, H, C = dims.B, dims.L, dims.H, dims.C
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = np.stack([random_walk(rng, L) for _ in range(B)])
+    q = rng.standard_normal((B, L, H, C))
+    k = rng.standard_normal((B, L, H, C))
+    v = rng.standard_normal((B, L, H, C))
+    rho = rng.uniform(0.5, 1.5, H) / math.sqrt(C)
+    s = rng.uniform(0.05, 0.3, H)
+    mask = np.ones((B, L), dtype=bool)
+    nmask = int(round(masked_tail_frac * L))
+    if nmask:
+        mask[:, L - nmask:] = False
+    f32 = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    return {"dims": dims, "q": f32(q), "k": f32(k), "v": f32(v), "x": f32(x),
+            "rho": f32(rho), "s": f32(s), "mask": mask}
 
 
 # Named workloads.  Sizes follow the IPA module of AlphaFold-2-style models
