@@ -233,6 +233,41 @@ IPA_API ipa_status_t geo_attn_fwd_static(const geo_params_t* p,
                                  const ipa_tensor_t* out_attention,
                                  void* stream, int32_t* dev_err);
 
+/* --------------------------------------------------------------------------
+ * Distance-aware attention (MEET, §2.2 "distance-aware attention",
+ * eq. (6)-(8)), run on the fused IPA core:
+ *
+ *   A_ij^h = rho_h * ( <q_i^h, k_j^h> - s_h^2 * ||x_i - x_j||^2 )
+ *   o_i^h  = sum_j softmax_j(A_i.^h) * v_j^h   over keys with mask_i and mask_j
+ *
+ * rows with no allowed key are 0 (the passage defines the logits; the value
+ * aggregation and the masking are this library's reading).  The distance is
+ * folded into the augmented query/key columns like the IPA point term
+ * (eq. (7)-(8)): each coordinate enters as a frame origin with identity
+ * rotation, the pair term is zero.
+ *
+ * Inputs (element strides, any layout):
+ *   q, k, v   [B, L, H, C] IPA_DTYPE_F32, C == 16 (the core's scalar width)
+ *   x         [B, L, 3]    IPA_DTYPE_F32 coordinates
+ *   rho, s    [H]          IPA_DTYPE_F32 attention and distance scales
+ *   mask      [B, L]       IPA_DTYPE_BOOL
+ * Output: out [B, L, H, C] IPA_DTYPE_F32, contiguous.
+ * Workspace: meet_attn_workspace_size(p) bytes, 256-byte aligned, caller
+ * owned; errors as for ipa_attn_fwd.  Supported: C == 16, L <= 1048576.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t B, L, H, C;
+} meet_params_t;
+
+IPA_API size_t meet_attn_workspace_size(const meet_params_t* p);
+
+IPA_API ipa_status_t meet_attn_fwd(const meet_params_t* p,
+                           const ipa_tensor_t* q, const ipa_tensor_t* k, const ipa_tensor_t* v,
+                           const ipa_tensor_t* x, const ipa_tensor_t* rho, const ipa_tensor_t* s,
+                           const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                           void* workspace, size_t workspace_bytes,
+                           void* stream, int32_t* dev_err);
+
 /* Static description of a status code (never NULL). */
 IPA_API const char* ipa_status_string(ipa_status_t s);
 

@@ -22,7 +22,8 @@ STATUS = {0: "IPA_OK", 1: "IPA_ERR_NULL", 2: "IPA_ERR_SHAPE", 3: "IPA_ERR_STRIDE
           4: "IPA_ERR_DTYPE", 5: "IPA_ERR_WORKSPACE", 6: "IPA_ERR_UNSUPPORTED", 7: "IPA_ERR_CUDA",
           8: "IPA_ERR_TIMEOUT"}
 EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa_attn_core",
-            "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static", "ipa_status_string",
+            "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static",
+            "meet_attn_workspace_size", "meet_attn_fwd", "ipa_status_string",
             "ipa_device_error_status", "ipa_version")
 
 
@@ -41,6 +42,11 @@ class IpaParams(ctypes.Structure):
 class GeoParams(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("M", ctypes.c_int32), ("Cout", ctypes.c_int32)]
+
+
+class MeetParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("C", ctypes.c_int32)]
 
 
 class IpaError(RuntimeError):
@@ -78,6 +84,11 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.geo_attn_fwd.argtypes = [P(GeoParams)] + [T] * 16 + [ctypes.c_void_p, ctypes.c_size_t,
                                                             ctypes.c_void_p, ctypes.c_void_p]
     lib.geo_attn_fwd.restype = ctypes.c_int
+    lib.meet_attn_workspace_size.argtypes = [P(MeetParams)]
+    lib.meet_attn_workspace_size.restype = ctypes.c_size_t
+    lib.meet_attn_fwd.argtypes = [P(MeetParams)] + [T] * 8 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                              ctypes.c_void_p, ctypes.c_void_p]
+    lib.meet_attn_fwd.restype = ctypes.c_int
     lib.ipa_status_string.argtypes = [ctypes.c_int]
     lib.ipa_status_string.restype = ctypes.c_char_p
     lib.ipa_device_error_status.argtypes = [ctypes.c_int32]
@@ -309,5 +320,56 @@ def geo_attn(inp: dict, *, with_attention: bool = True, stream=None, check: bool
     plan = GeoPlan(B, N, H, M, Cout, device=inp["q_direction"].device)
     res = plan(inp, with_attention=with_attention, stream=stream)
     if check:
+        plan.check()
+    return res
+
+
+# ------------------------------------------------------------------ MEET
+MEET_INPUTS = ("q", "k", "v", "x", "rho", "s", "mask")
+
+
+class MeetPlan:
+    """Distance-aware attention of MEET (§2.2, eq. (6)) on the fused core:
+    workspace owned by the plan, reused across calls of the same shape."""
+
+    def __init__(self, B: int, L: int, H: int, C: int = 16, device="cuda"):
+        self.params = MeetParams(B, L, H, C)
+        nbytes = int(library().meet_attn_workspace_size(ctypes.byref(self.params)))
+        if nbytes == 0:
+            raise IpaError(6, "dimensions outside the supported envelope (C must be 16)")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def __call__(self, q, k, v, x, rho, s, mask, out=None, stream=None):
+        p = self.params
+        _require_cuda(q, k, v, x, rho, s, mask)
+        if out is None:
+            out = torch.empty((p.B, p.L, p.H, p.C), dtype=torch.float32, device=q.device)
+        descs = [tensor_desc(t) for t in (q, k, v, x, rho, s, mask, out)]
+        st = library().meet_attn_fwd(ctypes.byref(p), *[ctypes.byref(d) for d in descs],
+                                     ctypes.c_void_p(self.workspace.data_ptr()),
+                                     ctypes.c_size_t(self.workspace.numel()),
+                                     ctypes.c_void_p(_stream_ptr(stream)),
+                                     ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return out
+
+    def check(self):
+        """Raise if a device-side bounded wait expired (call after a sync)."""
+        v = int(self.dev_err.item())
+        if v != 0:
+            st = library().ipa_device_error_status(v)
+            raise IpaError(st, f"device error word {v}")
+
+
+def meet_attn(inp: dict, *, out=None, stream=None, check: bool = True):
+    """One call of the distance-aware attention on CUDA tensors `inp`
+    (keys MEET_INPUTS); returns o [B, L, H, C]."""
+    B, L, H, C = inp["q"].shape
+    plan = MeetPlan(B, L, H, C, device=inp["q"].device)
+    res = plan(*[inp[n] for n in MEET_INPUTS], out=out, stream=stream)
+    if check:
+        torch.cuda.synchronize()
         plan.check()
     return res

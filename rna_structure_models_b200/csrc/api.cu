@@ -6,6 +6,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "flashipa_b200.h"
@@ -264,6 +265,89 @@ ipa_status_t ipa_attn_fwd(const ipa_params_t* p, const ipa_tensor_t* q, const ip
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (ipa_launch_prologue(a, s) != cudaSuccess) return IPA_ERR_CUDA;
   if (ipa_launch_core(a, s) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
+size_t meet_attn_workspace_size(const meet_params_t* p) {
+  if (p == nullptr || p->B < 1 || p->L < 1 || p->H < 1 || p->C != MEET_C || p->L > (1 << 20) ||
+      static_cast<int64_t>(p->B) * p->H * p->L > (int64_t{1} << 31) / 64)
+    return 0;
+  return meet_workspace_layout(p->B, p->L, p->H).total;
+}
+
+ipa_status_t meet_attn_fwd(const meet_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,
+                           const ipa_tensor_t* v, const ipa_tensor_t* x, const ipa_tensor_t* rho,
+                           const ipa_tensor_t* s, const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                           void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err) {
+  if (p == nullptr) return IPA_ERR_NULL;
+  if (p->B < 1 || p->L < 1 || p->H < 1 || p->C < 1) return IPA_ERR_SHAPE;
+  if (p->C != MEET_C || p->L > (1 << 20) || static_cast<int64_t>(p->B) * p->H * p->L > (int64_t{1} << 31) / 64)
+    return IPA_ERR_UNSUPPORTED;
+  const int64_t B = p->B, L = p->L, H = p->H, C = p->C;
+  ipa_status_t st = IPA_OK;
+  const int64_t s_qkv[4] = {B, L, H, C}, s_x[3] = {B, L, 3}, s_h[1] = {H}, s_m[2] = {B, L};
+  if (!check_tensor(q, IPA_DTYPE_F32, 4, s_qkv, &st) || !check_tensor(k, IPA_DTYPE_F32, 4, s_qkv, &st) ||
+      !check_tensor(v, IPA_DTYPE_F32, 4, s_qkv, &st) || !check_tensor(x, IPA_DTYPE_F32, 3, s_x, &st) ||
+      !check_tensor(rho, IPA_DTYPE_F32, 1, s_h, &st) || !check_tensor(s, IPA_DTYPE_F32, 1, s_h, &st) ||
+      !check_tensor(mask, IPA_DTYPE_BOOL, 2, s_m, &st) || !check_contiguous_out(out, 4, s_qkv, &st))
+    return st;
+  const MeetWorkspace lay = meet_workspace_layout(p->B, p->L, p->H);
+  if (workspace == nullptr) return IPA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+  MeetPrep m{};
+  m.B = p->B; m.L = p->L; m.H = p->H;
+  m.q = view_of(q); m.rho = view_of(rho); m.s = view_of(s);
+  m.qs = reinterpret_cast<float*>(ws + lay.qs);
+  m.gamma = reinterpret_cast<float*>(ws + lay.gamma);
+  m.consts = reinterpret_cast<float*>(ws + lay.consts);
+
+  // the IPA problem: C = 16, Pq = 4, Pv = 8, R = 1, Cz = 16; w_L = 1,
+  // w_C = 1/2, scalar scale 1
+  IpaLaunch a{};
+  a.B = p->B; a.L = p->L; a.H = p->H; a.C = MEET_C; a.Pq = IPA_PQ; a.Pv = IPA_PV; a.R = 1; a.Cz = MEET_RCZ;
+  a.DZ = MEET_DZ; a.RCz = MEET_RCZ; a.F = MEET_F;
+  a.nqt = (p->L + QT - 1) / QT; a.nkt = (p->L + KT - 1) / KT;
+  a.w_L = 1.f; a.w_C = 0.5f; a.scalar_scale = 1.f;
+  auto dense = [](const void* ptr, std::initializer_list<int64_t> strides) {
+    View vv{};
+    vv.p = ptr;
+    int d = 0;
+    for (int64_t st2 : strides) vv.s[d++] = st2;
+    return vv;
+  };
+  const float* zeros = m.consts;
+  const float* ident = m.consts + MEET_ZEROS;
+  a.q = dense(m.qs, {L * H * C, H * C, C, 1});
+  a.k = view_of(k);
+  a.v = view_of(v);
+  a.q_pts = dense(zeros, {0, 0, 0, 0, 0});
+  a.k_pts = dense(zeros, {0, 0, 0, 0, 0});
+  a.v_pts = dense(zeros, {0, 0, 0, 0, 0});
+  a.rot = dense(ident, {0, 0, 3, 1});
+  a.trans = view_of(x);
+  a.z1 = dense(zeros, {0, 0, 0, 0});
+  a.z2 = dense(zeros, {0, 0, 0, 0});
+  a.w_bias = dense(zeros, {0, 0});
+  a.gamma = dense(m.gamma, {1});
+  a.mask = view_of(mask);
+  a.mask.dtype = 2;
+  a.ws = ws + lay.ipa;
+  a.lay = ipa_workspace_layout(p->B, p->L, p->H, MEET_DZ, MEET_RCZ);
+  a.out = reinterpret_cast<float*>(ws + lay.out);
+  if (dev_err != nullptr) {
+    a.err = dev_err;
+  } else {
+    a.err = reinterpret_cast<int*>(a.ws + a.lay.err);
+    if (cudaMemsetAsync(a.err, 0, sizeof(int), cs) != cudaSuccess) return IPA_ERR_CUDA;
+  }
+  if (meet_launch_prep(m, cs) != cudaSuccess) return IPA_ERR_CUDA;
+  if (ipa_launch_prologue(a, cs) != cudaSuccess) return IPA_ERR_CUDA;
+  if (ipa_launch_core(a, cs) != cudaSuccess) return IPA_ERR_CUDA;
+  if (meet_launch_extract(a.out, static_cast<float*>(const_cast<void*>(out->data)), B * L * H, cs) != cudaSuccess)
+    return IPA_ERR_CUDA;
   return IPA_OK;
 }
 

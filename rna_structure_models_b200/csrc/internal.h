@@ -44,6 +44,25 @@ struct IpaLaunch {
 cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream);
 cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream);
 
+// Distance-aware attention (MEET) on the IPA core: C = 16, Pq = 4, Pv = 8,
+// one 16-channel pair factor (DZ = 64), output row F = 64.
+constexpr int MEET_C = 16, MEET_RCZ = 16, MEET_DZ = 64, MEET_F = 16 + 4 * 8 + 16, MEET_ZEROS = 128;
+
+struct MeetWorkspace {
+  size_t ipa, qs, gamma, consts, out, total;
+};
+MeetWorkspace meet_workspace_layout(int B, int L, int H);
+
+struct MeetPrep {
+  int B, L, H;
+  View q, rho, s;
+  float* qs;       // [B, L, H, 16] rho_h q
+  float* gamma;    // [H] rho_h s_h^2
+  float* consts;   // MEET_ZEROS zeros, then the 3x3 identity
+};
+cudaError_t meet_launch_prep(const MeetPrep& m, cudaStream_t stream);
+cudaError_t meet_launch_extract(const float* core_out, float* out, int64_t rows, cudaStream_t stream);
+
 struct GeoWorkspace {
   size_t qg, kg, vg, rotf, ml, live, wf, bf, sc, err, total;
 };

@@ -191,3 +191,47 @@ def test_package_import_does_not_load_the_library():
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT)
     assert out.stdout.strip() == "False", out.stderr
     importlib.import_module("rna_structure_models_b200")
+
+
+def meet_call(B=2, L=64, H=3, C=16, ws_bytes=None, ws_ptr=FAKE, **over):
+    lib = api.library()
+    p = api.MeetParams(B, L, H, C)
+    shapes = {"q": (B, L, H, C), "k": (B, L, H, C), "v": (B, L, H, C), "x": (B, L, 3), "rho": (H,), "s": (H,),
+              "mask": (B, L), "out": (B, L, H, C)}
+    ds = {k: desc(sh, api.IPA_DTYPE_BOOL if k == "mask" else api.IPA_DTYPE_F32) for k, sh in shapes.items()}
+    ds.update(over)
+    if ws_bytes is None:
+        ws_bytes = lib.meet_attn_workspace_size(ctypes.byref(p))
+    return lib.meet_attn_fwd(ctypes.byref(p), *[ctypes.byref(ds[k]) for k in api.MEET_INPUTS + ("out",)],
+                             ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes), None, ctypes.c_void_p(FAKE))
+
+
+def test_meet_workspace_linear_in_L_and_zero_outside_envelope():
+    lib = api.library()
+    per = []
+    for L in (2048, 4096, 8192):
+        per.append(lib.meet_attn_workspace_size(ctypes.byref(api.MeetParams(1, L, 8, 16))) / L)
+    assert max(per) / min(per) < 1.01
+    assert lib.meet_attn_workspace_size(ctypes.byref(api.MeetParams(1, 64, 8, 32))) == 0   # C must be 16
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("unsupported_C", 6), ("shape_x", 2), ("dtype_mask", 4), ("null_rho", 1), ("workspace", 5),
+    ("out_noncontig", 3),
+])
+def test_meet_rejects_bad_arguments_before_launch(case, expect):
+    if case == "unsupported_C":
+        assert meet_call(C=32, ws_bytes=1 << 30) == expect
+        return
+    over, ws_bytes = {}, None
+    if case == "shape_x":
+        over["x"] = desc((2, 64, 4))
+    elif case == "dtype_mask":
+        over["mask"] = desc((2, 64), api.IPA_DTYPE_F32)
+    elif case == "null_rho":
+        over["rho"] = desc((3,), ptr=None)
+    elif case == "workspace":
+        ws_bytes = 1024
+    elif case == "out_noncontig":
+        over["out"] = desc((2, 64, 3, 16), strides=(64 * 3 * 16, 1, 64, 3 * 64))
+    assert meet_call(ws_bytes=ws_bytes, **over) == expect
