@@ -364,6 +364,34 @@ def main():
             if res[True] > res[False] else None,
         }
 
+    # distance-aware attention of MEET (§2.2) on the same core (B=1, L=4096, H=8)
+    if not args.no_variant and rank == 0:
+        from rna_structure_models_b200.synth import MeetDims, meet_inputs
+        mi = meet_inputs(MeetDims(B=1, L=L, H=8, C=16), 0)
+        md = {n: torch.from_numpy(mi[n]).to(dev) for n in api.MEET_INPUTS}
+        mp = api.MeetPlan(1, L, 8, 16, device=dev)
+        mout = torch.empty((1, L, 8, 16), device=dev)
+        for _ in range(3):
+            mp(*[md[n] for n in api.MEET_INPUTS], out=mout)
+        torch.cuda.synchronize()
+        mt = []
+        for _ in range(20):
+            flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            mp(*[md[n] for n in api.MEET_INPUTS], out=mout)
+            a1.record()
+            torch.cuda.synchronize()
+            mt.append(a0.elapsed_time(a1))
+        mp.check()
+        ms_meet = statistics.mean(mt)
+        triples = L * L * 8
+        line["meet"] = {
+            "workload": f"MEET distance-aware attention B=1 L={L} H=8 C=16 (all four kernels of a call)",
+            "ms": ms_meet, "pair_heads_per_s": triples / (ms_meet / 1e3),
+            "tflops_algorithmic": triples * 2 * (2 * 16 + 9) / (ms_meet / 1e3) / 1e12,
+        }
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, nrows, secs = cpu_oracle_sample(L, args.cpu_seconds, 4096)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
