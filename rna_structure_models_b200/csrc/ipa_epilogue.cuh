@@ -99,8 +99,8 @@ __device__ __forceinline__ void write_row(const float* O, float* dst, int lane, 
 
 // Phase A for the 16 rows of one warp: z1 (.) O_pair summed over the R
 // factors into O_pair[0 .. Cz) of each staged row.  z1 rows are read as
-// float4 (lane q holds columns 4q .. 4q + 3 and 128 + 4q ..), two rows ahead of
-// the row being folded: wide loads keep the number of outstanding L1 requests
+// float4 (lane q holds columns 4q .. 4q + 3 and 128 + 4q ..), four rows ahead
+// of the row being folded: wide loads keep the number of outstanding L1 requests
 // low, which is what bounds this phase.  When Cz % 128 == 0 all R factors of
 // a pair feature sit on one lane and fold in registers; otherwise the
 // products are written in place and reduced in a second, float4 pass.
@@ -110,7 +110,8 @@ static __device__ __noinline__ void fold_pairs_rows(const EpilogueArgs& e, int w
   const int R = e.RCz / e.Cz, cq = e.Cz >> 2;
   const bool lane_local = (e.Cz & 127) == 0;
   const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  float4 zb[3][2];
+  constexpr int AHEAD = 4;                    // rows of z1 in flight ahead of the row being folded
+  float4 zb[AHEAD + 1][2];
   auto load_row = [&](int rr, float4 (&z)[2]) {
     const int grow = e.row0 + warp * 16 + rr;
     const bool in = rr < 16 && grow < e.L;
@@ -123,13 +124,13 @@ static __device__ __noinline__ void fold_pairs_rows(const EpilogueArgs& e, int w
     }
   };
   auto mul4 = [](float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); };
-  load_row(0, zb[0]);
-  load_row(1, zb[1]);
+#pragma unroll
+  for (int rr = 0; rr < AHEAD; ++rr) load_row(rr, zb[rr]);
 #pragma unroll
   for (int rr = 0; rr < 16; ++rr) {
-    load_row(rr + 2, zb[(rr + 2) % 3]);
+    load_row(rr + AHEAD, zb[(rr + AHEAD) % (AHEAD + 1)]);
     float4* P = reinterpret_cast<float4*>(e.stage + (warp * 16 + rr) * pitch + 64);
-    const float4 z0 = zb[rr % 3][0], z1 = zb[rr % 3][1];
+    const float4 z0 = zb[rr % (AHEAD + 1)][0], z1 = zb[rr % (AHEAD + 1)][1];
     if (lane_local && R == 2) {              // Cz = 128: columns lane and 32 + lane hold factors 0 and 1
       const float4 o0 = P[lane], o1 = P[32 + lane];
       P[lane] = make_float4(fmaf(z1.x, o1.x, z0.x * o0.x), fmaf(z1.y, o1.y, z0.y * o0.y),
