@@ -211,6 +211,8 @@ def main():
     ap.add_argument("--no-variant", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--core-only", action="store_true", help="profiling aid: time only, print nothing else")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the step's kernels directly instead of replaying a CUDA graph")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -250,8 +252,31 @@ def main():
     torch.cuda.synchronize()
     plan.check()
 
+    # the step as a CUDA graph (tile, rows and core kernels replayed without
+    # host launch gaps), and the core alone for its roofline time
+    graphs = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g_step, g_core = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step):
+            step()
+        with torch.cuda.graph(g_core):
+            plan.core(out)
+        torch.cuda.synchronize()
+        graphs = (g_step, g_core)
+        for _ in range(3):
+            g_step.replay()
+        torch.cuda.synchronize()
+        plan.check()
+
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    evc = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -259,17 +284,31 @@ def main():
         for k in range(K):
             flush.zero_()                                  # L2 flushed between steps (untimed)
             ev[k][0].record()
-            plan.prologue(*args_in)
-            ev[k][1].record()
-            plan.core(out)
+            if graphs:
+                graphs[0].replay()
+            else:
+                plan.prologue(*args_in)
+                ev[k][1].record()
+                plan.core(out)
             ev[k][2].record()
         torch.cuda.synchronize()
+        if graphs:                                         # the core alone, same flush between runs
+            for k in range(K):
+                flush.zero_()
+                evc[k][0].record()
+                graphs[1].replay()
+                evc[k][1].record()
+            torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     plan.check()
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    core_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    pro_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    if graphs:
+        core_ms = [e[0].elapsed_time(e[1]) for e in evc]
+        pro_ms = [max(0.0, sm - cm) for sm, cm in zip(step_ms, core_ms)]
+    else:
+        core_ms = [e[1].elapsed_time(e[2]) for e in ev]
+        pro_ms = [e[0].elapsed_time(e[1]) for e in ev]
     total_ms = max_over_ranks(sum(step_ms), world, dist, dev)
     if args.core_only:
         if world > 1:
@@ -291,12 +330,15 @@ def main():
         "config": {"workload": f"IPA core B=1 L={L} H={H} C={C} Pq={PQ} Pv={PV} R={R} Cz={CZ} per GPU",
                    "global_batch": world, "seq_len": L, "parallelism": f"dp{world}",
                    "l2": "flushed between steps (256 MB write, untimed)",
-                   "step": "prologue (frames, augmented fp16 operands) + fused attention core"},
+                   "step": "prologue (frames, augmented fp16 operands) + fused attention core",
+                   "launch": "direct launches" if args.no_graph else
+                             "CUDA graph replay of the step's 3 kernels; core time from a core-only graph"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": CORE_KERNEL,
                      "peak_source": f"{peak_kind} bf16 dense (burst); fp16 has the same nominal rate",
-                     "core_ms": core_mean, "prologue_ms": statistics.mean(pro_ms),
+                     "core_ms": core_mean,
+                     "prologue_ms": statistics.mean(pro_ms),   # step minus core with graphs
                      "issued_frac": achieved * 640.0 / 581.0 / peak},
         "gpu_launches": 3 * K,                             # tile, rows, core
         "clocks": clk.summary(),

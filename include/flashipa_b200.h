@@ -94,7 +94,8 @@ typedef struct {
  *   mask             [B, L]         IPA_DTYPE_BOOL
  *   out              [B, L, H, C + 4 Pv + Cz], IPA_DTYPE_F32, contiguous
  * Supported envelope: C == 16, Pq == 4, Pv == 8 (the AlphaFold-2 IPA head
- * shape), 1 <= R * Cz <= 256 with Cz a multiple of 16, 1 <= L <= 1048576.
+ * shape), 1 <= R * Cz <= 256 with Cz a multiple of 16, 1 <= L <= 1048576,
+ * 1 <= H <= 128.
  * Arithmetic: fp16 tensor-core operands with fp32 accumulation; point
  * coordinates, key norms and value points carry a second fp16 term for the
  * rounding residue.
@@ -253,7 +254,8 @@ IPA_API ipa_status_t geo_attn_fwd_static(const geo_params_t* p,
  *   mask      [B, L]       IPA_DTYPE_BOOL
  * Output: out [B, L, H, C] IPA_DTYPE_F32, contiguous.
  * Workspace: meet_attn_workspace_size(p) bytes, 256-byte aligned, caller
- * owned; errors as for ipa_attn_fwd.  Supported: C == 16, L <= 1048576.
+ * owned; errors as for ipa_attn_fwd.  Supported: C == 16, H <= 128,
+ * L <= 1048576.
  * ------------------------------------------------------------------------ */
 typedef struct {
   int32_t B, L, H, C;

@@ -73,7 +73,7 @@ bool ipa_dims_ok(const ipa_params_t* p, ipa_status_t* st) {
     *st = IPA_ERR_SHAPE;
     return false;
   }
-  if (p->C != IPA_C || p->Pq != IPA_PQ || p->Pv != IPA_PV || p->Cz % 16 != 0 ||
+  if (p->C != IPA_C || p->Pq != IPA_PQ || p->Pv != IPA_PV || p->Cz % 16 != 0 || p->H > 128 ||
       static_cast<int64_t>(p->R) * p->Cz > MAX_DZ || p->L > (1 << 20) ||
       static_cast<int64_t>(p->B) * p->H * p->L > (int64_t{1} << 31) / 64) {
     *st = IPA_ERR_UNSUPPORTED;
@@ -269,7 +269,7 @@ ipa_status_t ipa_attn_fwd(const ipa_params_t* p, const ipa_tensor_t* q, const ip
 }
 
 size_t meet_attn_workspace_size(const meet_params_t* p) {
-  if (p == nullptr || p->B < 1 || p->L < 1 || p->H < 1 || p->C != MEET_C || p->L > (1 << 20) ||
+  if (p == nullptr || p->B < 1 || p->L < 1 || p->H < 1 || p->C != MEET_C || p->H > 128 || p->L > (1 << 20) ||
       static_cast<int64_t>(p->B) * p->H * p->L > (int64_t{1} << 31) / 64)
     return 0;
   return meet_workspace_layout(p->B, p->L, p->H).total;
@@ -281,7 +281,8 @@ ipa_status_t meet_attn_fwd(const meet_params_t* p, const ipa_tensor_t* q, const 
                            void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err) {
   if (p == nullptr) return IPA_ERR_NULL;
   if (p->B < 1 || p->L < 1 || p->H < 1 || p->C < 1) return IPA_ERR_SHAPE;
-  if (p->C != MEET_C || p->L > (1 << 20) || static_cast<int64_t>(p->B) * p->H * p->L > (int64_t{1} << 31) / 64)
+  if (p->C != MEET_C || p->H > 128 || p->L > (1 << 20) ||
+      static_cast<int64_t>(p->B) * p->H * p->L > (int64_t{1} << 31) / 64)
     return IPA_ERR_UNSUPPORTED;
   const int64_t B = p->B, L = p->L, H = p->H, C = p->C;
   ipa_status_t st = IPA_OK;

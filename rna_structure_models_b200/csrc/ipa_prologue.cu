@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(256) ipa_tile_kernel(const TileArgs a) {
 
 struct RowArgs {
   int B, L, H, nqt, nkt, Cz, RCz, DZ;
+  int rb;          // residues per block (128 / H)
   float qscale;    // log2(e) w_L scalar_scale
   float w_L, w_C;
   View q, k, v, q_pts, k_pts, v_pts, gamma, w_bias;
@@ -187,23 +188,27 @@ __device__ __forceinline__ float4 tile_origin(const float4* part, int J0, int J1
 template <int C, int PQ, int PV>
 __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   static_assert(C + 9 * PQ + 2 <= DH && C + 6 * PV <= DH, "augmented rows wider than 64");
-  // heads fastest: the threads of a residue read its contiguous [H, ...]
-  // input rows together
-  const int64_t total = static_cast<int64_t>(a.B) * a.H * a.L;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x;
-  const int64_t t = t0 + threadIdx.x;
-  const int64_t hl = static_cast<int64_t>(a.H) * a.L;
+  // a block owns rb consecutive residues of one batch, all heads (heads
+  // fastest: the threads of a residue read its contiguous [H, ...] input
+  // rows together); its output rows are staged in shared memory and written
+  // as one contiguous run of rb rows per head plane
+  extern __shared__ uint4 stage_rows[];    // [3][H][rb][8] fp16 rows, then [2][H][rb] float4 terms
+  const int rb = a.rb, H = a.H;
+  const int b = blockIdx.y;
+  const int i0 = blockIdx.x * rb;
+  const int il = threadIdx.x / H, h = threadIdx.x % H;
+  const int i = i0 + il;
+  const bool active = il < rb && i < a.L;
+  const int nrow = a.L - i0 < rb ? a.L - i0 : rb;
 
-  // centroid of the valid origins of every batch this block touches (double
-  // sums over the per-tile partial sums; at most 128 batches per block)
-  __shared__ float4 cen_s[128];
+  // centroid of the batch's valid origins (double sums over the per-tile
+  // partial sums of the tile kernel)
   __shared__ double red[4][4];
-  const int bfirst = static_cast<int>(t0 / hl);
-  const int blast = static_cast<int>((t0 + blockDim.x - 1 < total ? t0 + blockDim.x - 1 : total - 1) / hl);
-  for (int bb = bfirst; bb <= blast; ++bb) {
+  __shared__ float4 cen_s;
+  {
     double sx = 0, sy = 0, sz = 0, sn = 0;
     for (int J = threadIdx.x; J < a.nkt; J += blockDim.x) {
-      const float4 p = a.part[static_cast<int64_t>(bb) * a.nkt + J];
+      const float4 p = a.part[static_cast<int64_t>(b) * a.nkt + J];
       sx += p.x; sy += p.y; sz += p.z; sn += p.w;
     }
 #pragma unroll
@@ -222,19 +227,25 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
       double tx = 0, ty = 0, tz = 0, tn = 0;
       for (int w = 0; w < 4; ++w) { tx += red[w][0]; ty += red[w][1]; tz += red[w][2]; tn += red[w][3]; }
       const double inv = tn > 0 ? 1.0 / tn : 0.0;
-      cen_s[bb - bfirst] = make_float4(static_cast<float>(tx * inv), static_cast<float>(ty * inv),
-                                       static_cast<float>(tz * inv), static_cast<float>(tn));
+      cen_s = make_float4(static_cast<float>(tx * inv), static_cast<float>(ty * inv), static_cast<float>(tz * inv),
+                          static_cast<float>(tn));
     }
     __syncthreads();
   }
-  if (t >= total) return;
-  const int h = static_cast<int>(t % a.H);
-  const int i = static_cast<int>((t / a.H) % a.L);
-  const int b = static_cast<int>(t / hl);
-  const int bh = b * a.H + h;
-  const int64_t orow = static_cast<int64_t>(bh) * a.L + i;   // row of the [B*H, L] outputs
-
-  const float4 cn = cen_s[b - bfirst];
+  const int slot = h * rb + il;                                   // row of this thread in a staged plane
+  uint4* sq_rows = stage_rows + static_cast<size_t>(0 * H * rb + slot) * 8;
+  uint4* sk_rows = stage_rows + static_cast<size_t>(1 * H * rb + slot) * 8;
+  uint4* sv_rows = stage_rows + static_cast<size_t>(2 * H * rb + slot) * 8;
+  float4* sterm = reinterpret_cast<float4*>(stage_rows + static_cast<size_t>(3 * H * rb) * 8);
+  // the [H, DZ] pair-bias weights, one entry per thread of batch 0
+  if (b == 0 && active)
+    for (int64_t e = static_cast<int64_t>(i) * H + h; e < static_cast<int64_t>(H) * a.DZ;
+         e += static_cast<int64_t>(H) * a.L) {
+      const int he = static_cast<int>(e / a.DZ), col = static_cast<int>(e % a.DZ);
+      a.wqp[e] = col < a.RCz ? kLog2e * a.w_L * ldf(a.w_bias, (col % a.Cz) * a.w_bias.s[0] + he * a.w_bias.s[1]) : 0.f;
+    }
+  if (active) {
+  const float4 cn = cen_s;
   const float4* partb = a.part + static_cast<int64_t>(b) * a.nkt;
   const int Jq = (i / QT) * (QT / KT);
   const float4 oqv = tile_origin(partb, Jq, Jq + QT / KT < a.nkt ? Jq + QT / KT : a.nkt, cn);
@@ -245,15 +256,8 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     if (i % QT == 0) a.oq[b * a.nqt + i / QT] = oqv;
     if (i % KT == 0) a.ok[b * a.nkt + i / KT] = okv;
   }
+  if (b == 0 && i == 0) a.headc[h] = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
   const float c = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
-  if (b == 0) {
-    if (i == 0) a.headc[h] = c;
-    // the [H, DZ] pair-bias weights, one entry per thread of batch 0
-    for (int64_t e = t; e < static_cast<int64_t>(a.H) * a.DZ; e += hl) {
-      const int he = static_cast<int>(e / a.DZ), col = static_cast<int>(e % a.DZ);
-      a.wqp[e] = col < a.RCz ? kLog2e * a.w_L * ldf(a.w_bias, (col % a.Cz) * a.w_bias.s[0] + he * a.w_bias.s[1]) : 0.f;
-    }
-  }
 
   const float4* fr = a.frame + (static_cast<int64_t>(b) * a.L + i) * 4;
   const float4 f0 = fr[0], f1 = fr[1], f2 = fr[2], f3 = fr[3];
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   };
   auto hi_of = [](float x) { return __half2float(__float2half_rn(x)); };
   // Q_h: [ scaled q | gq' hi | gq' hi | gq' lo | -1 -1 | 0 ]
-  store_row(a.qh + orow * 8, [&](int col) -> float {
+  store_row(sq_rows, [&](int col) -> float {
     if (col < C) return a.qscale * qs[col];
     if (col < C + 9 * PQ) {
       const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     return col < C + 9 * PQ + 2 ? -1.f : 0.f;
   });
   // K_h: [ k | 2c gk' hi | lo | hi | c|gk'|^2 hi, lo | 0 ]
-  store_row(a.kh + orow * 8, [&](int col) -> float {
+  store_row(sk_rows, [&](int col) -> float {
     if (col < C) return ks[col];
     if (col < C + 9 * PQ) {
       const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
@@ -345,7 +349,7 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     return 0.f;
   });
   // V_h: [ v | gv hi | gv lo ]
-  store_row(a.vh + orow * 8, [&](int col) -> float {
+  store_row(sv_rows, [&](int col) -> float {
     if (col < C) return vs[col];
     if (col < C + 6 * PV) {
       const int u = col - C, part = u / (3 * PV), e = u % (3 * PV);
@@ -358,9 +362,29 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     sq[0] = sq[1] = sq[2] = 0.f;
     sk[0] = sk[1] = sk[2] = 0.f;
   }
-  a.rowq[orow] = make_float4(sq[0], sq[1], sq[2], 0.f);
-  a.colk[orow] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
+  sterm[slot] = make_float4(sq[0], sq[1], sq[2], 0.f);
+  sterm[H * rb + slot] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
   if (overflow) record_error(a.err, DEV_NONFINITE);
+  }
+  __syncthreads();
+  // each head plane's run of nrow rows, 16-byte stores, consecutive threads on
+  // consecutive addresses
+  uint4* const outs[3] = {a.qh, a.kh, a.vh};
+  const int run = nrow * 8;                                        // uint4 per plane run
+#pragma unroll
+  for (int kind = 0; kind < 3; ++kind) {
+    const uint4* src = stage_rows + static_cast<size_t>(kind * H * rb) * 8;
+    for (int e = threadIdx.x; e < H * run; e += blockDim.x) {
+      const int hh = e / run, r = e % run;
+      outs[kind][(static_cast<int64_t>(b * H + hh) * a.L + i0) * 8 + r] = src[hh * rb * 8 + r];
+    }
+  }
+  for (int e = threadIdx.x; e < 2 * H * nrow; e += blockDim.x) {
+    const int which = e / (H * nrow), rem = e % (H * nrow);
+    const int hh = rem / nrow, r = rem % nrow;
+    float4* dst = which == 0 ? a.rowq : a.colk;
+    dst[static_cast<int64_t>(b * H + hh) * a.L + i0 + r] = sterm[which * H * rb + hh * rb + r];
+  }
 }
 
 }  // namespace
@@ -397,8 +421,14 @@ cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
   r.rowq = reinterpret_cast<float4*>(ws + w.rowq);
   r.colk = reinterpret_cast<float4*>(ws + w.colk);
   r.err = a.err;
-  const int64_t n = static_cast<int64_t>(a.B) * a.H * a.L;
-  ipa_rows_kernel<IPA_C, IPA_PQ, IPA_PV><<<static_cast<unsigned>((n + 127) / 128), 128, 0, stream>>>(r);
+  r.rb = 128 / a.H;
+  const size_t smem = static_cast<size_t>(a.H) * r.rb * (3 * DH * 2 + 2 * 16);
+  // the largest request is 128 rows x 416 B
+  const cudaError_t e = cudaFuncSetAttribute(ipa_rows_kernel<IPA_C, IPA_PQ, IPA_PV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * (3 * DH * 2 + 2 * 16));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>((a.L + r.rb - 1) / r.rb), static_cast<unsigned>(a.B));
+  ipa_rows_kernel<IPA_C, IPA_PQ, IPA_PV><<<grid, 128, smem, stream>>>(r);
   return cudaGetLastError();
 }
 
