@@ -268,6 +268,69 @@ def ipa_attn_host(inp: dict, plan: Optional[IpaPlan] = None, device="cuda", stre
     return out, plan
 
 
+class IpaHostPipeline:
+    """Many calls on HOST buffers with the transfers overlapped across calls:
+    call k's inputs go up on a copy stream while call k-1 computes and call
+    k-2's result comes down on a second copy stream (PCIe carries both
+    directions at once).  Two device staging sets; events order every reuse.
+    Each call's copies and kernels are the same as ipa_attn_host's."""
+
+    def __init__(self, plan: IpaPlan, device="cuda"):
+        self.plan = plan
+        self.device = torch.device(device)
+        self.up, self.comp, self.down = (torch.cuda.Stream(self.device) for _ in range(3))
+        self.sets = [{}, {}]
+        self.outs = [None, None]
+        ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]  # noqa: E731
+        self.uploaded, self.consumed, self.computed, self.downloaded = ev(), ev(), ev(), ev()
+
+    def _stage(self, s, inp):
+        d = self.sets[s]
+        for n in IPA_INPUTS:
+            t = inp[n]
+            buf = d.get(n)
+            if buf is None or buf.shape != t.shape or buf.stride() != t.stride() or buf.dtype != t.dtype:
+                buf = d[n] = torch.empty_strided(t.shape, t.stride(), dtype=t.dtype, device=self.device)
+            buf.copy_(t, non_blocking=True)
+        return d
+
+    def run(self, inputs, outputs, stream=None):
+        """inputs: list of dicts of pinned host tensors (IPA_INPUTS); outputs:
+        list of pinned host tensors [B, L, H, F].  Work starts after what is
+        already queued on `stream` (default: current) and `stream` waits for
+        the last result at the end."""
+        caller = stream if stream is not None else torch.cuda.current_stream(self.device)
+        start = torch.cuda.Event()
+        start.record(caller)
+        for st in (self.up, self.comp, self.down):
+            st.wait_event(start)
+        p = self.plan.params
+        for k, (inp, out_host) in enumerate(zip(inputs, outputs)):
+            s = k % 2
+            with torch.cuda.stream(self.up):
+                self.up.wait_event(self.consumed[s])         # call k-2 has read staging set s
+                dev = self._stage(s, inp)
+                self.uploaded[s].record(self.up)
+            with torch.cuda.stream(self.comp):
+                self.comp.wait_event(self.uploaded[s])
+                self.comp.wait_event(self.downloaded[s])     # call k-2's result has left buffer s
+                if self.outs[s] is None:
+                    self.outs[s] = torch.empty((p.B, p.L, p.H, self.plan.F), dtype=torch.float32,
+                                               device=self.device)
+                self.plan.prologue(*[dev[n] for n in IPA_INPUTS])
+                self.consumed[s].record(self.comp)
+                self.plan.core(self.outs[s])
+                self.computed[s].record(self.comp)
+            with torch.cuda.stream(self.down):
+                self.down.wait_event(self.computed[s])
+                out_host.copy_(self.outs[s], non_blocking=True)
+                self.downloaded[s].record(self.down)
+        end = torch.cuda.Event()
+        end.record(self.down)
+        caller.wait_event(end)
+        return outputs
+
+
 # ------------------------------------------------------------------ variant
 GEO_INPUTS = ("q_direction", "k_direction", "q_point", "k_point", "values", "direction_scale",
               "distance_scale", "output_weight", "output_bias", "rotation", "translation",

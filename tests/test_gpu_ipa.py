@@ -176,3 +176,17 @@ def test_host_buffer_entry_matches_device_path_and_reuses_staging(cuda_device):
         ref = run_gpu(inp)
         assert out_host.is_pinned()
         assert np.array_equal(out_host.numpy(), ref)
+
+
+def test_host_pipeline_matches_device_path_per_call(cuda_device):
+    # several calls with different inputs through the overlapped host
+    # pipeline: every result equals that call's device-path result
+    inps = [ipa_inputs(IpaDims(B=1, L=257, H=4, Cz=64), seed) for seed in (21, 22, 23, 24, 25)]
+    plan = api.IpaPlan(1, 257, 4, 16, 4, 8, 2, 64, device="cuda")
+    hosts = [{k: torch.from_numpy(inp[k]).pin_memory() for k in api.IPA_INPUTS} for inp in inps]
+    outs = [torch.empty((1, 257, 4, plan.F), dtype=torch.float32, pin_memory=True) for _ in inps]
+    api.IpaHostPipeline(plan, device="cuda").run(hosts, outs)
+    torch.cuda.synchronize()
+    plan.check()
+    for inp, out in zip(inps, outs):
+        assert np.array_equal(out.numpy(), run_gpu(inp))
