@@ -60,7 +60,43 @@ struct TileArgs {
 // Pair factors of 64 residues x one 64-column panel, zero-padded beyond
 // R*Cz and zero for masked residues: 4 residues x 64 columns per pass, all
 // loads of a thread issued before its stores.
+// Vector form of the copy below for the dense layout (unit column stride,
+// Cz % 4 == 0, 16-byte aligned rows): 16 residues x 64 columns per pass,
+// four columns per thread.
+__device__ __forceinline__ bool ipa_tile_copy_pairs_vec(const TileArgs& a, int b, int i0, int panel, int tid) {
+  if (a.z1.s[3] != 1 || a.z2.s[3] != 1 || (a.Cz & 3) != 0 || a.z1.s[2] != a.Cz || a.z2.s[2] != a.Cz ||
+      ((reinterpret_cast<uintptr_t>(a.z1.p) | reinterpret_cast<uintptr_t>(a.z2.p)) & 15) != 0 ||
+      ((a.z1.s[0] | a.z1.s[1] | a.z2.s[0] | a.z2.s[1]) & 3) != 0)
+    return false;
+  const int col = panel * 64 + 4 * (tid & 15);       // first of this thread's 4 columns
+  const bool inpair = col < a.RCz;                    // RCz % 16 == 0: all 4 or none
+  constexpr int NP = KT / 16;
+  float4 v1[NP], v2[NP];
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    const int i = i0 + 16 * q + (tid >> 4);
+    v1[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    v2[q] = v1[q];
+    if (i < a.L && inpair && ldb(a.mask, b * a.mask.s[0] + i * a.mask.s[1])) {
+      v1[q] = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(a.z1.p) + b * a.z1.s[0] + i * a.z1.s[1] + col));
+      v2[q] = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(a.z2.p) + b * a.z2.s[0] + i * a.z2.s[1] + col));
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    const int i = i0 + 16 * q + (tid >> 4);
+    if (i < a.L) {
+      const int64_t o = (static_cast<int64_t>(b) * a.L + i) * a.DZ + col;
+      *reinterpret_cast<float4*>(a.z1f + o) = v1[q];
+      *reinterpret_cast<uint2*>(a.z1h + o) = make_uint2(pack_half2(v1[q].x, v1[q].y), pack_half2(v1[q].z, v1[q].w));
+      *reinterpret_cast<uint2*>(a.z2h + o) = make_uint2(pack_half2(v2[q].x, v2[q].y), pack_half2(v2[q].z, v2[q].w));
+    }
+  }
+  return true;
+}
+
 __device__ __forceinline__ void ipa_tile_copy_pairs(const TileArgs& a, int b, int i0, int panel, int tid) {
+  if (ipa_tile_copy_pairs_vec(a, b, i0, panel, tid)) return;
   const int col = panel * 64 + (tid & 63);
   const bool inpair = col < a.RCz;
   const int rr = inpair ? col / a.Cz : 0, cc = inpair ? col % a.Cz : 0;
