@@ -208,6 +208,13 @@ __device__ __forceinline__ void load_row(const View& v, int64_t base, int64_t st
   }
 }
 
+// max that propagates NaN (so a NaN operand is reported like an overflow)
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // Origin (mean of the valid centred frame origins) of a run of 64-residue
 // tiles [J0, J1) of batch b, from their partial sums; 0 for an empty run.
 __device__ __forceinline__ float4 tile_origin(const float4* part, int J0, int J1, float4 cen) {
@@ -345,16 +352,16 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     sk[e % 3] += gk[e];
     nk = fmaf(gk[e], gk[e], nk);
   }
-  bool overflow = false;
+  float vmax = 0.f;   // largest |value| written (NaN if any value is NaN)
   auto store_row = [&](uint4* dst, auto value_of) {
 #pragma unroll
     for (int u = 0; u < DH / 8; ++u) {
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        w[e] = valid ? pack_half2(value_of(8 * u + 2 * e), value_of(8 * u + 2 * e + 1)) : 0u;
-        // |x| >= 65520 rounds to infinity in fp16 (exponent field all ones)
-        overflow |= ((w[e] & 0x7c00u) == 0x7c00u) || ((w[e] & 0x7c000000u) == 0x7c000000u);
+        const float x0 = value_of(8 * u + 2 * e), x1 = value_of(8 * u + 2 * e + 1);
+        vmax = fmax_nan(vmax, fmax_nan(fabsf(x0), fabsf(x1)));
+        w[e] = valid ? pack_half2(x0, x1) : 0u;
       }
       dst[u] = make_uint4(w[0], w[1], w[2], w[3]);
     }
@@ -400,7 +407,8 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   }
   sterm[slot] = make_float4(sq[0], sq[1], sq[2], 0.f);
   sterm[H * rb + slot] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
-  if (overflow) record_error(a.err, DEV_NONFINITE);
+  // |x| >= 65520 (or NaN) does not survive the fp16 rounding
+  if (valid && !(vmax < 65520.f)) record_error(a.err, DEV_NONFINITE);
   }
   __syncthreads();
   // each head plane's run of nrow rows, 16-byte stores, consecutive threads on

@@ -190,3 +190,17 @@ def test_host_pipeline_matches_device_path_per_call(cuda_device):
     plan.check()
     for inp, out in zip(inps, outs):
         assert np.array_equal(out.numpy(), run_gpu(inp))
+
+
+@pytest.mark.parametrize("bad", [1e7, float("nan")])
+def test_operand_outside_fp16_range_is_reported(cuda_device, bad):
+    # a scalar channel that cannot be represented in the fp16 operands (or is
+    # NaN) is reported through the device error word, not silently used
+    inp = ipa_preset("tiny")
+    inp["q"][0, 5, 1, 3] = bad
+    dev = to_dev({k: inp[k] for k in api.IPA_INPUTS})
+    plan = api.IpaPlan(1, 64, 4, 16, 4, 8, 2, 16, device="cuda")
+    plan(*[dev[n] for n in api.IPA_INPUTS])
+    torch.cuda.synchronize()
+    with pytest.raises(api.IpaError):
+        plan.check()
