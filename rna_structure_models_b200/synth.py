@@ -29,7 +29,7 @@ import numpy as np
 
 __all__ = [
     "IpaDims", "GeoDims", "ipa_inputs", "geo_inputs", "ipa_preset", "geo_preset",
-    "IPA_PRESETS", "random_rotations", "random_walk", "MeetDims", "meet_inputs",
+    "IPA_PRESETS", "random_rotations", "random_walk", "MeetDims", "meet_inputs", "backbone_inputs",
 ]
 
 
@@ -211,6 +211,27 @@ def meet_inputs(dims: MeetDims, seed: int = 0, *, masked_tail_frac: float = 0.0)
     f32 = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
     return {"dims": dims, "q": f32(q), "k": f32(k), "v": f32(v), "x": f32(x),
             "rho": f32(rho), "s": f32(s), "mask": mask}
+
+
+def backbone_inputs(B: int, L: int, seed: int = 0, *, jitter: float = 0.0) -> dict:
+    """Seeded backbone atoms N, CA, C [B, L, 3] and the frames they were
+    built from: CA on the 3.8 A walk, C at 1.52 A along the local x axis, N
+    at 1.46 A in the local xy plane at 111 degrees from it (rounded textbook
+    bond lengths and N-CA-C angle), then optional N(0, jitter) noise on N
+    and C.  Draw order: rotations, walk, noise."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    R = random_rotations(rng, B * L).reshape(B, L, 3, 3)
+    ca = np.stack([random_walk(rng, L) for _ in range(B)])
+    ang = math.radians(111.0)
+    c_loc = np.array([1.52, 0.0, 0.0])
+    n_loc = 1.46 * np.array([math.cos(ang), math.sin(ang), 0.0])
+    c = ca + np.einsum("blxy,y->blx", R, c_loc)
+    n = ca + np.einsum("blxy,y->blx", R, n_loc)
+    if jitter:
+        n = n + jitter * rng.standard_normal(n.shape)
+        c = c + jitter * rng.standard_normal(c.shape)
+    f32 = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    return {"n": f32(n), "ca": f32(ca), "c": f32(c), "rot": R, "trans": ca}
 
 
 # Named workloads.  Sizes follow the IPA module of AlphaFold-2-style models
