@@ -270,6 +270,27 @@ IPA_API ipa_status_t meet_attn_fwd(const meet_params_t* p,
                            void* workspace, size_t workspace_bytes,
                            void* stream, int32_t* dev_err);
 
+/* --------------------------------------------------------------------------
+ * Residue frames from backbone atoms (Flash Invariant Point Attention,
+ * Figure 1: the frame is centred on C_alpha and spanned by C_alpha -> C and
+ * C_alpha -> N through Gram-Schmidt; this library's reading of the order and
+ * handedness):
+ *   e1 = (C - CA) / |C - CA|
+ *   e2 = normalise((N - CA) - (e1 . (N - CA)) e1)
+ *   e3 = e1 x e2,  rot = [e1 | e2 | e3] (columns),  trans = CA
+ * so that rot maps local column vectors to global ones, as ipa_attn_fwd's
+ * `rot` expects.
+ * Inputs n, ca, c [B, L, 3] IPA_DTYPE_F32 (any strides); outputs rot
+ * [B, L, 3, 3] and trans [B, L, 3] IPA_DTYPE_F32, contiguous.  No workspace.
+ * Collinear N, CA, C give non-finite frames (outside the domain, not
+ * checked).  Enqueued on `stream`; errors as for ipa_attn_fwd.
+ * ------------------------------------------------------------------------ */
+IPA_API ipa_status_t ipa_frames_from_backbone(int32_t B, int32_t L,
+                                      const ipa_tensor_t* n, const ipa_tensor_t* ca,
+                                      const ipa_tensor_t* c,
+                                      const ipa_tensor_t* rot_out, const ipa_tensor_t* trans_out,
+                                      void* stream);
+
 /* Static description of a status code (never NULL). */
 IPA_API const char* ipa_status_string(ipa_status_t s);
 

@@ -23,7 +23,7 @@ STATUS = {0: "IPA_OK", 1: "IPA_ERR_NULL", 2: "IPA_ERR_SHAPE", 3: "IPA_ERR_STRIDE
           8: "IPA_ERR_TIMEOUT"}
 EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa_attn_core",
             "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static",
-            "meet_attn_workspace_size", "meet_attn_fwd", "ipa_status_string",
+            "meet_attn_workspace_size", "meet_attn_fwd", "ipa_frames_from_backbone", "ipa_status_string",
             "ipa_device_error_status", "ipa_version")
 
 
@@ -89,6 +89,8 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.meet_attn_fwd.argtypes = [P(MeetParams)] + [T] * 8 + [ctypes.c_void_p, ctypes.c_size_t,
                                                               ctypes.c_void_p, ctypes.c_void_p]
     lib.meet_attn_fwd.restype = ctypes.c_int
+    lib.ipa_frames_from_backbone.argtypes = [ctypes.c_int32, ctypes.c_int32] + [T] * 5 + [ctypes.c_void_p]
+    lib.ipa_frames_from_backbone.restype = ctypes.c_int
     lib.ipa_status_string.argtypes = [ctypes.c_int]
     lib.ipa_status_string.restype = ctypes.c_char_p
     lib.ipa_device_error_status.argtypes = [ctypes.c_int32]
@@ -436,3 +438,21 @@ def meet_attn(inp: dict, *, out=None, stream=None, check: bool = True):
         torch.cuda.synchronize()
         plan.check()
     return res
+
+
+# ------------------------------------------------------------------ frames
+def frames_from_backbone(n, ca, c, rot=None, trans=None, stream=None):
+    """Residue frames (rot [B, L, 3, 3], trans [B, L, 3]) from backbone atoms
+    n, ca, c [B, L, 3] on the GPU (Gram-Schmidt on C_alpha)."""
+    _require_cuda(n, ca, c)
+    B, L = n.shape[0], n.shape[1]
+    if rot is None:
+        rot = torch.empty((B, L, 3, 3), dtype=torch.float32, device=n.device)
+    if trans is None:
+        trans = torch.empty((B, L, 3), dtype=torch.float32, device=n.device)
+    descs = [tensor_desc(t) for t in (n, ca, c, rot, trans)]
+    st = library().ipa_frames_from_backbone(B, L, *[ctypes.byref(d) for d in descs],
+                                            ctypes.c_void_p(_stream_ptr(stream)))
+    if st != 0:
+        raise IpaError(st, library().ipa_status_string(st).decode())
+    return rot, trans

@@ -352,6 +352,33 @@ ipa_status_t meet_attn_fwd(const meet_params_t* p, const ipa_tensor_t* q, const 
   return IPA_OK;
 }
 
+ipa_status_t ipa_frames_from_backbone(int32_t B, int32_t L, const ipa_tensor_t* n, const ipa_tensor_t* ca,
+                                      const ipa_tensor_t* c, const ipa_tensor_t* rot_out,
+                                      const ipa_tensor_t* trans_out, void* stream) {
+  if (B < 1 || L < 1) return IPA_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * L > (int64_t{1} << 31) / 16) return IPA_ERR_UNSUPPORTED;
+  ipa_status_t st = IPA_OK;
+  const int64_t s_a[3] = {B, L, 3}, s_r[4] = {B, L, 3, 3};
+  if (!check_tensor(n, IPA_DTYPE_F32, 3, s_a, &st) || !check_tensor(ca, IPA_DTYPE_F32, 3, s_a, &st) ||
+      !check_tensor(c, IPA_DTYPE_F32, 3, s_a, &st) || !check_tensor(rot_out, IPA_DTYPE_F32, 4, s_r, &st) ||
+      !check_tensor(trans_out, IPA_DTYPE_F32, 3, s_a, &st))
+    return st;
+  for (const ipa_tensor_t* o : {rot_out, trans_out}) {    // outputs dense row-major
+    int64_t expect = 1;
+    for (int d = o->ndim - 1; d >= 0; --d) {
+      if (o->size[d] > 1 && o->stride[d] != expect) return IPA_ERR_STRIDE_ALIGN;
+      expect *= o->size[d];
+    }
+  }
+  FramesArgs a{};
+  a.B = B; a.L = L;
+  a.n = view_of(n); a.ca = view_of(ca); a.c = view_of(c);
+  a.rot = static_cast<float*>(const_cast<void*>(rot_out->data));
+  a.trans = static_cast<float*>(const_cast<void*>(trans_out->data));
+  if (frames_launch(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
 size_t geo_attn_workspace_size(const geo_params_t* p) {
   ipa_status_t st;
   if (!geo_dims_ok(p, &st)) return 0;

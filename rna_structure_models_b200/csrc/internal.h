@@ -63,6 +63,15 @@ struct MeetPrep {
 cudaError_t meet_launch_prep(const MeetPrep& m, cudaStream_t stream);
 cudaError_t meet_launch_extract(const float* core_out, float* out, int64_t rows, cudaStream_t stream);
 
+// Residue frames from backbone atoms.
+struct FramesArgs {
+  int B, L;
+  View n, ca, c;   // [B, L, 3]
+  float* rot;      // [B, L, 3, 3]
+  float* trans;    // [B, L, 3]
+};
+cudaError_t frames_launch(const FramesArgs& a, cudaStream_t stream);
+
 struct GeoWorkspace {
   size_t qg, kg, vg, rotf, ml, live, wf, bf, sc, err, total;
 };

@@ -235,3 +235,33 @@ def test_meet_rejects_bad_arguments_before_launch(case, expect):
     elif case == "out_noncontig":
         over["out"] = desc((2, 64, 3, 16), strides=(64 * 3 * 16, 1, 64, 3 * 64))
     assert meet_call(ws_bytes=ws_bytes, **over) == expect
+
+
+def frames_call(B=2, L=64, **over):
+    lib = api.library()
+    ds = {"n": desc((B, L, 3)), "ca": desc((B, L, 3)), "c": desc((B, L, 3)),
+          "rot": desc((B, L, 3, 3)), "trans": desc((B, L, 3))}
+    ds.update(over)
+    return lib.ipa_frames_from_backbone(B, L, *[ctypes.byref(ds[k]) for k in ("n", "ca", "c", "rot", "trans")],
+                                        ctypes.c_void_p(FAKE))
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("empty", 2), ("shape_ca", 2), ("dtype_c", 4), ("null_n", 1), ("rot_noncontig", 3), ("trans_shape", 2),
+])
+def test_frames_rejects_bad_arguments_before_launch(case, expect):
+    if case == "empty":
+        assert frames_call(B=0) == expect
+        return
+    over = {}
+    if case == "shape_ca":
+        over["ca"] = desc((2, 63, 3))
+    elif case == "dtype_c":
+        over["c"] = desc((2, 64, 3), api.IPA_DTYPE_BOOL)
+    elif case == "null_n":
+        over["n"] = desc((2, 64, 3), ptr=None)
+    elif case == "rot_noncontig":
+        over["rot"] = desc((2, 64, 3, 3), strides=(576, 9, 1, 3))
+    elif case == "trans_shape":
+        over["trans"] = desc((2, 64, 4))
+    assert frames_call(**over) == expect
