@@ -187,6 +187,21 @@ def geo_inputs(dims: GeoDims, seed: int = 0, *, pair_drop: float = 0.2,
     }
 
 
+def geo_upstream(dims: GeoDims, seed: int = 0, *, with_attention: bool = True,
+                 with_vectors: bool = True) -> dict:
+    """Seeded upstream gradients of the variant's three results, N(0, 1):
+    g_output [B, N, Cout], g_attention [B, H, N, N], g_vectors
+    [B, N, H, M, 3] (the last two None when not requested).  Draw order as
+    listed."""
+    B, N, H, M, Cout = dims.B, dims.N, dims.H, dims.M, dims.Cout
+    rng = np.random.Generator(np.random.PCG64(seed))
+    f32 = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    g_out = f32(rng.standard_normal((B, N, Cout)))
+    g_att = f32(rng.standard_normal((B, H, N, N))) if with_attention else None
+    g_vec = f32(rng.standard_normal((B, N, H, M, 3))) if with_vectors else None
+    return {"g_output": g_out, "g_attention": g_att, "g_vectors": g_vec}
+
+
 def meet_inputs(dims: MeetDims, seed: int = 0, *, masked_tail_frac: float = 0.0) -> dict:
     """Seeded inputs of the distance-aware attention of MEET §2.2.
 
