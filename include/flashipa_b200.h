@@ -197,6 +197,47 @@ IPA_API ipa_status_t geo_attn_fwd(const geo_params_t* p,
                           void* stream, int32_t* dev_err);
 
 /* --------------------------------------------------------------------------
+ * Gradients of the geometric attention ("Geometric direction-and-distance
+ * attention", Required behavior: the operator is differentiated, with the
+ * derivative of the distance at a zero displacement defined as the zero
+ * vector).  Given the forward's inputs (as for geo_attn_fwd) and upstream
+ * gradients of its results, writes the gradients of
+ *   sum(g_output * output) + sum(g_attention * attention) + sum(g_vectors * vectors)
+ * with respect to every floating input.  The forward statistics are
+ * recomputed inside the call; no N x N array is stored.
+ *   g_output     [B, N, Cout]        same dtype as the inputs, any strides
+ *   g_attention  [B, H, N, N] or NULL / data == NULL (zero)
+ *   g_vectors    [B, N, H, M, 3] or NULL / data == NULL (zero)
+ *   grads        one IPA_DTYPE_F32 contiguous buffer per floating input, of
+ *                the input's shape; grads->output_bias.data may be NULL only
+ *                when output_bias is absent.
+ * Queries with no allowed key in any head pass no g_output on (their output
+ * is forced to zero).  The caller owns every buffer; errors as for
+ * geo_attn_fwd.  Workspace: geo_attn_bwd_workspace_size(p) bytes, 256-byte
+ * aligned.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  ipa_tensor_t q_direction, k_direction, q_point, k_point, values;
+  ipa_tensor_t direction_scale, distance_scale, output_weight, output_bias;
+  ipa_tensor_t rotation, translation;
+} geo_grads_t;
+
+IPA_API size_t geo_attn_bwd_workspace_size(const geo_params_t* p);
+
+IPA_API ipa_status_t geo_attn_bwd(const geo_params_t* p,
+                          const ipa_tensor_t* q_direction, const ipa_tensor_t* k_direction,
+                          const ipa_tensor_t* q_point, const ipa_tensor_t* k_point,
+                          const ipa_tensor_t* values,
+                          const ipa_tensor_t* direction_scale,
+                          const ipa_tensor_t* distance_scale,
+                          const ipa_tensor_t* output_weight, const ipa_tensor_t* output_bias,
+                          const ipa_tensor_t* rotation, const ipa_tensor_t* translation,
+                          const ipa_tensor_t* frame_mask, const ipa_tensor_t* pair_mask,
+                          const ipa_tensor_t* g_output, const ipa_tensor_t* g_attention,
+                          const ipa_tensor_t* g_vectors, const geo_grads_t* grads,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
  * geo_attn_fwd without a workspace argument (no counterpart on the pages:
  * this is an interface convenience of this library, not part of the method).
  *

@@ -23,6 +23,7 @@ STATUS = {0: "IPA_OK", 1: "IPA_ERR_NULL", 2: "IPA_ERR_SHAPE", 3: "IPA_ERR_STRIDE
           8: "IPA_ERR_TIMEOUT"}
 EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa_attn_core",
             "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static",
+            "geo_attn_bwd_workspace_size", "geo_attn_bwd",
             "meet_attn_workspace_size", "meet_attn_fwd", "ipa_frames_from_backbone", "ipa_status_string",
             "ipa_device_error_status", "ipa_version")
 
@@ -42,6 +43,14 @@ class IpaParams(ctypes.Structure):
 class GeoParams(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("M", ctypes.c_int32), ("Cout", ctypes.c_int32)]
+
+
+GEO_GRADS = ("q_direction", "k_direction", "q_point", "k_point", "values", "direction_scale",
+             "distance_scale", "output_weight", "output_bias", "rotation", "translation")
+
+
+class GeoGrads(ctypes.Structure):
+    _fields_ = [(n, IpaTensor) for n in GEO_GRADS]
 
 
 class MeetParams(ctypes.Structure):
@@ -91,6 +100,11 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.meet_attn_fwd.restype = ctypes.c_int
     lib.ipa_frames_from_backbone.argtypes = [ctypes.c_int32, ctypes.c_int32] + [T] * 5 + [ctypes.c_void_p]
     lib.ipa_frames_from_backbone.restype = ctypes.c_int
+    lib.geo_attn_bwd_workspace_size.argtypes = [P(GeoParams)]
+    lib.geo_attn_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.geo_attn_bwd.argtypes = [P(GeoParams)] + [T] * 16 + [P(GeoGrads), ctypes.c_void_p, ctypes.c_size_t,
+                                                             ctypes.c_void_p]
+    lib.geo_attn_bwd.restype = ctypes.c_int
     lib.ipa_status_string.argtypes = [ctypes.c_int]
     lib.ipa_status_string.restype = ctypes.c_char_p
     lib.ipa_device_error_status.argtypes = [ctypes.c_int32]
@@ -387,6 +401,51 @@ def geo_attn(inp: dict, *, with_attention: bool = True, stream=None, check: bool
     if check:
         plan.check()
     return res
+
+
+class GeoGradPlan:
+    """Gradients of the variant (Required behavior: the operator is
+    differentiated, zero distance derivative at a zero displacement); the
+    workspace is owned by the plan and reused across calls of one shape."""
+
+    def __init__(self, B, N, H, M, Cout, device="cuda"):
+        self.params = GeoParams(B, N, H, M, Cout)
+        nbytes = int(library().geo_attn_bwd_workspace_size(ctypes.byref(self.params)))
+        if nbytes == 0:
+            raise IpaError(6, "dimensions outside the supported envelope")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def __call__(self, inp: dict, g_output, g_attention=None, g_vectors=None, *, out: Optional[dict] = None,
+                 stream=None):
+        p = self.params
+        dev = inp["q_direction"].device
+        _require_cuda(*[inp.get(n) for n in GEO_INPUTS], g_output, g_attention, g_vectors)
+        if out is None:
+            out = {n: (torch.empty(tuple(inp[n].shape), dtype=torch.float32, device=dev)
+                       if inp.get(n) is not None else None) for n in GEO_GRADS}
+        pm = inp.get("pair_mask")
+        if pm is not None and pm.dim() == 4 and tuple(pm.shape) != (p.B, p.H, p.N, p.N):
+            pm = pm.expand(p.B, p.H, p.N, p.N)
+        descs = [tensor_desc(inp.get(n)) for n in GEO_INPUTS[:-1]] + [tensor_desc(pm)]
+        descs += [tensor_desc(g_output), tensor_desc(g_attention), tensor_desc(g_vectors)]
+        grads = GeoGrads(*[tensor_desc(out.get(n)) for n in GEO_GRADS])
+        st = library().geo_attn_bwd(ctypes.byref(p), *[ctypes.byref(d) for d in descs], ctypes.byref(grads),
+                                    ctypes.c_void_p(self.workspace.data_ptr()),
+                                    ctypes.c_size_t(self.workspace.numel()),
+                                    ctypes.c_void_p(_stream_ptr(stream)))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return out
+
+
+def geo_attn_backward(inp: dict, g_output, g_attention=None, g_vectors=None, *, stream=None) -> dict:
+    """Gradients of sum(g_output * output) + sum(g_attention * attention)
+    + sum(g_vectors * vectors) with respect to every floating input (fp32)."""
+    B, N, H, _ = inp["q_direction"].shape
+    M = inp["values"].shape[3]
+    Cout = inp["output_weight"].shape[1]
+    plan = GeoGradPlan(B, N, H, M, Cout, device=inp["q_direction"].device)
+    return plan(inp, g_output, g_attention, g_vectors, stream=stream)
 
 
 # ------------------------------------------------------------------ MEET

@@ -385,6 +385,71 @@ size_t geo_attn_workspace_size(const geo_params_t* p) {
   return geo_workspace_layout(p->B, p->N, p->H, p->M, p->Cout).total;
 }
 
+namespace {
+
+// Checks the variant's inputs (shared by the forward and the gradient) and
+// fills the input part of a launch.
+ipa_status_t geo_inputs(const geo_params_t* p, const ipa_tensor_t* q_direction,
+                        const ipa_tensor_t* k_direction, const ipa_tensor_t* q_point,
+                        const ipa_tensor_t* k_point, const ipa_tensor_t* values,
+                        const ipa_tensor_t* direction_scale, const ipa_tensor_t* distance_scale,
+                        const ipa_tensor_t* output_weight, const ipa_tensor_t* output_bias,
+                        const ipa_tensor_t* rotation, const ipa_tensor_t* translation,
+                        const ipa_tensor_t* frame_mask, const ipa_tensor_t* pair_mask, fipa::GeoLaunch* a,
+                        int* fdt_out) {
+  ipa_status_t st = IPA_OK;
+  if (!geo_dims_ok(p, &st)) return st;
+  const int64_t B = p->B, N = p->N, H = p->H, M = p->M, Cout = p->Cout;
+  const int fdt = q_direction ? q_direction->dtype : IPA_DTYPE_F32;
+  if (fdt != IPA_DTYPE_F32 && fdt != IPA_DTYPE_F64) return q_direction ? IPA_ERR_DTYPE : IPA_ERR_NULL;
+  const bool has_bias = output_bias != nullptr && output_bias->data != nullptr;
+  const bool has_pm = pair_mask != nullptr && pair_mask->data != nullptr;
+  const int64_t s_v3[4] = {B, N, H, 3};
+  const int64_t s_val[5] = {B, N, H, M, 3};
+  const int64_t s_h[1] = {H};
+  const int64_t s_w[2] = {H * M * 3, Cout};
+  const int64_t s_b[1] = {Cout};
+  const int64_t s_rot[4] = {B, N, 3, 3};
+  const int64_t s_tr[3] = {B, N, 3};
+  const int64_t s_fm[2] = {B, N};
+  const int64_t s_pm[4] = {B, H, N, N};
+  if (!check_tensor(q_direction, fdt, 4, s_v3, &st) || !check_tensor(k_direction, fdt, 4, s_v3, &st) ||
+      !check_tensor(q_point, fdt, 4, s_v3, &st) || !check_tensor(k_point, fdt, 4, s_v3, &st) ||
+      !check_tensor(values, fdt, 5, s_val, &st) || !check_tensor(direction_scale, fdt, 1, s_h, &st) ||
+      !check_tensor(distance_scale, fdt, 1, s_h, &st) || !check_tensor(output_weight, fdt, 2, s_w, &st) ||
+      (has_bias && !check_tensor(output_bias, fdt, 1, s_b, &st)) ||
+      !check_tensor(rotation, fdt, 4, s_rot, &st) || !check_tensor(translation, fdt, 3, s_tr, &st) ||
+      !check_tensor(frame_mask, IPA_DTYPE_BOOL, 2, s_fm, &st))
+    return st;
+  if (has_pm) {
+    // broadcastable to [B, H, N, N]: each size equals the full size or is 1 (stride ignored then)
+    if (pair_mask->dtype != IPA_DTYPE_BOOL) return IPA_ERR_DTYPE;
+    if (pair_mask->ndim != 4) return IPA_ERR_SHAPE;
+    for (int d = 0; d < 4; ++d) {
+      if (pair_mask->size[d] != s_pm[d] && pair_mask->size[d] != 1) return IPA_ERR_SHAPE;
+      if (pair_mask->stride[d] < 0) return IPA_ERR_STRIDE_ALIGN;
+    }
+  }
+  fipa::GeoLaunch& g = *a;
+  g = fipa::GeoLaunch{};
+  g.B = p->B; g.N = p->N; g.H = p->H; g.M = p->M; g.Cout = p->Cout; g.HM3 = p->H * p->M * 3;
+  g.q_direction = view_of(q_direction); g.k_direction = view_of(k_direction);
+  g.q_point = view_of(q_point); g.k_point = view_of(k_point); g.values = view_of(values);
+  g.direction_scale = view_of(direction_scale); g.distance_scale = view_of(distance_scale);
+  g.output_weight = view_of(output_weight); g.output_bias = view_of(has_bias ? output_bias : nullptr);
+  g.output_bias.dtype = has_bias ? g.output_bias.dtype : g.output_weight.dtype;
+  g.rotation = view_of(rotation); g.translation = view_of(translation); g.frame_mask = view_of(frame_mask);
+  g.pair_mask = view_of(has_pm ? pair_mask : nullptr);
+  if (has_pm)
+    for (int d = 0; d < 4; ++d)
+      if (pair_mask->size[d] == 1) g.pair_mask.s[d] = 0;  // broadcast dimension
+  g.has_bias = has_bias; g.has_pair_mask = has_pm;
+  *fdt_out = fdt;
+  return IPA_OK;
+}
+
+}  // namespace
+
 ipa_status_t geo_attn_fwd(const geo_params_t* p, const ipa_tensor_t* q_direction,
                           const ipa_tensor_t* k_direction, const ipa_tensor_t* q_point,
                           const ipa_tensor_t* k_point, const ipa_tensor_t* values,
@@ -395,65 +460,23 @@ ipa_status_t geo_attn_fwd(const geo_params_t* p, const ipa_tensor_t* q_direction
                           const ipa_tensor_t* out_vectors, const ipa_tensor_t* out_output,
                           const ipa_tensor_t* out_attention, void* workspace, size_t workspace_bytes,
                           void* stream, int32_t* dev_err) {
-  ipa_status_t st = IPA_OK;
-  if (!geo_dims_ok(p, &st)) return st;
+  GeoLaunch a{};
+  int fdt = 0;
+  ipa_status_t st = geo_inputs(p, q_direction, k_direction, q_point, k_point, values, direction_scale,
+                               distance_scale, output_weight, output_bias, rotation, translation, frame_mask,
+                               pair_mask, &a, &fdt);
+  if (st != IPA_OK) return st;
   const int64_t B = p->B, N = p->N, H = p->H, M = p->M, Cout = p->Cout;
-  const int fdt = q_direction ? q_direction->dtype : IPA_DTYPE_F32;
-  if (fdt != IPA_DTYPE_F32 && fdt != IPA_DTYPE_F64) return q_direction ? IPA_ERR_DTYPE : IPA_ERR_NULL;
-  const bool has_bias = output_bias != nullptr && output_bias->data != nullptr;
-  const bool has_pm = pair_mask != nullptr && pair_mask->data != nullptr;
   const bool has_att = out_attention != nullptr && out_attention->data != nullptr;
-  {
-    const int64_t s_v3[4] = {B, N, H, 3};
-    const int64_t s_val[5] = {B, N, H, M, 3};
-    const int64_t s_h[1] = {H};
-    const int64_t s_w[2] = {H * M * 3, Cout};
-    const int64_t s_b[1] = {Cout};
-    const int64_t s_rot[4] = {B, N, 3, 3};
-    const int64_t s_tr[3] = {B, N, 3};
-    const int64_t s_fm[2] = {B, N};
-    const int64_t s_pm[4] = {B, H, N, N};
-    const int64_t s_out[2] = {B * N, Cout};
-    const int64_t s_o3[3] = {B, N, Cout};
-    const int64_t s_att[4] = {B, H, N, N};
-    (void)s_out;
-    if (!check_tensor(q_direction, fdt, 4, s_v3, &st) || !check_tensor(k_direction, fdt, 4, s_v3, &st) ||
-        !check_tensor(q_point, fdt, 4, s_v3, &st) || !check_tensor(k_point, fdt, 4, s_v3, &st) ||
-        !check_tensor(values, fdt, 5, s_val, &st) || !check_tensor(direction_scale, fdt, 1, s_h, &st) ||
-        !check_tensor(distance_scale, fdt, 1, s_h, &st) || !check_tensor(output_weight, fdt, 2, s_w, &st) ||
-        (has_bias && !check_tensor(output_bias, fdt, 1, s_b, &st)) ||
-        !check_tensor(rotation, fdt, 4, s_rot, &st) || !check_tensor(translation, fdt, 3, s_tr, &st) ||
-        !check_tensor(frame_mask, IPA_DTYPE_BOOL, 2, s_fm, &st) ||
-        !check_contiguous_out(out_vectors, 5, s_val, &st) || !check_contiguous_out(out_output, 3, s_o3, &st) ||
-        (has_att && !check_contiguous_out(out_attention, 4, s_att, &st)))
-      return st;
-    if (has_pm) {
-      // broadcastable to [B, H, N, N]: each size equals the full size or is 1 (stride ignored then)
-      if (pair_mask->dtype != IPA_DTYPE_BOOL) return IPA_ERR_DTYPE;
-      if (pair_mask->ndim != 4) return IPA_ERR_SHAPE;
-      for (int d = 0; d < 4; ++d) {
-        if (pair_mask->size[d] != s_pm[d] && pair_mask->size[d] != 1) return IPA_ERR_SHAPE;
-        if (pair_mask->stride[d] < 0) return IPA_ERR_STRIDE_ALIGN;
-      }
-    }
-  }
+  const int64_t s_val[5] = {B, N, H, M, 3};
+  const int64_t s_o3[3] = {B, N, Cout};
+  const int64_t s_att[4] = {B, H, N, N};
+  if (!check_contiguous_out(out_vectors, 5, s_val, &st) || !check_contiguous_out(out_output, 3, s_o3, &st) ||
+      (has_att && !check_contiguous_out(out_attention, 4, s_att, &st)))
+    return st;
   const GeoWorkspace lay = geo_workspace_layout(p->B, p->N, p->H, p->M, p->Cout);
   if (workspace == nullptr) return IPA_ERR_NULL;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
-
-  GeoLaunch a{};
-  a.B = p->B; a.N = p->N; a.H = p->H; a.M = p->M; a.Cout = p->Cout; a.HM3 = p->H * p->M * 3;
-  a.q_direction = view_of(q_direction); a.k_direction = view_of(k_direction);
-  a.q_point = view_of(q_point); a.k_point = view_of(k_point); a.values = view_of(values);
-  a.direction_scale = view_of(direction_scale); a.distance_scale = view_of(distance_scale);
-  a.output_weight = view_of(output_weight); a.output_bias = view_of(has_bias ? output_bias : nullptr);
-  a.output_bias.dtype = has_bias ? a.output_bias.dtype : a.output_weight.dtype;
-  a.rotation = view_of(rotation); a.translation = view_of(translation); a.frame_mask = view_of(frame_mask);
-  a.pair_mask = view_of(has_pm ? pair_mask : nullptr);
-  if (has_pm)
-    for (int d = 0; d < 4; ++d)
-      if (pair_mask->size[d] == 1) a.pair_mask.s[d] = 0;  // broadcast dimension
-  a.has_bias = has_bias; a.has_pair_mask = has_pm;
   a.out_vectors = static_cast<float*>(const_cast<void*>(out_vectors->data));
   a.out_output = static_cast<float*>(const_cast<void*>(out_output->data));
   a.out_attention = has_att ? static_cast<float*>(const_cast<void*>(out_attention->data)) : nullptr;
@@ -467,6 +490,82 @@ ipa_status_t geo_attn_fwd(const geo_params_t* p, const ipa_tensor_t* q_direction
     if (cudaMemsetAsync(a.err, 0, sizeof(int), s) != cudaSuccess) return IPA_ERR_CUDA;
   }
   if (geo_launch_all(a, s) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
+size_t geo_attn_bwd_workspace_size(const geo_params_t* p) {
+  ipa_status_t st = IPA_OK;
+  if (!geo_dims_ok(p, &st)) return 0;
+  return geo_bwd_workspace_layout(p->B, p->N, p->H, p->M, p->Cout).total;
+}
+
+ipa_status_t geo_attn_bwd(const geo_params_t* p, const ipa_tensor_t* q_direction,
+                          const ipa_tensor_t* k_direction, const ipa_tensor_t* q_point,
+                          const ipa_tensor_t* k_point, const ipa_tensor_t* values,
+                          const ipa_tensor_t* direction_scale, const ipa_tensor_t* distance_scale,
+                          const ipa_tensor_t* output_weight, const ipa_tensor_t* output_bias,
+                          const ipa_tensor_t* rotation, const ipa_tensor_t* translation,
+                          const ipa_tensor_t* frame_mask, const ipa_tensor_t* pair_mask,
+                          const ipa_tensor_t* g_output, const ipa_tensor_t* g_attention,
+                          const ipa_tensor_t* g_vectors, const geo_grads_t* grads, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  GeoBwdLaunch a{};
+  int fdt = 0;
+  ipa_status_t st = geo_inputs(p, q_direction, k_direction, q_point, k_point, values, direction_scale,
+                               distance_scale, output_weight, output_bias, rotation, translation, frame_mask,
+                               pair_mask, &a.f, &fdt);
+  if (st != IPA_OK) return st;
+  if (grads == nullptr) return IPA_ERR_NULL;
+  const int64_t B = p->B, N = p->N, H = p->H, M = p->M, Cout = p->Cout;
+  const int64_t s_v3[4] = {B, N, H, 3};
+  const int64_t s_val[5] = {B, N, H, M, 3};
+  const int64_t s_h[1] = {H};
+  const int64_t s_w[2] = {H * M * 3, Cout};
+  const int64_t s_b[1] = {Cout};
+  const int64_t s_rot[4] = {B, N, 3, 3};
+  const int64_t s_tr[3] = {B, N, 3};
+  const int64_t s_o3[3] = {B, N, Cout};
+  const int64_t s_att[4] = {B, H, N, N};
+  const bool has_ga = g_attention != nullptr && g_attention->data != nullptr;
+  const bool has_gv = g_vectors != nullptr && g_vectors->data != nullptr;
+  if (!check_tensor(g_output, fdt, 3, s_o3, &st) || (has_ga && !check_tensor(g_attention, fdt, 4, s_att, &st)) ||
+      (has_gv && !check_tensor(g_vectors, fdt, 5, s_val, &st)))
+    return st;
+  const bool want_bias = a.f.has_bias;
+  if (want_bias != (grads->output_bias.data != nullptr)) return grads->output_bias.data ? IPA_ERR_SHAPE : IPA_ERR_NULL;
+  if (!check_contiguous_out(&grads->q_direction, 4, s_v3, &st) ||
+      !check_contiguous_out(&grads->k_direction, 4, s_v3, &st) ||
+      !check_contiguous_out(&grads->q_point, 4, s_v3, &st) || !check_contiguous_out(&grads->k_point, 4, s_v3, &st) ||
+      !check_contiguous_out(&grads->values, 5, s_val, &st) ||
+      !check_contiguous_out(&grads->direction_scale, 1, s_h, &st) ||
+      !check_contiguous_out(&grads->distance_scale, 1, s_h, &st) ||
+      !check_contiguous_out(&grads->output_weight, 2, s_w, &st) ||
+      (want_bias && !check_contiguous_out(&grads->output_bias, 1, s_b, &st)) ||
+      !check_contiguous_out(&grads->rotation, 4, s_rot, &st) ||
+      !check_contiguous_out(&grads->translation, 3, s_tr, &st))
+    return st;
+  const GeoBwdWorkspace lay = geo_bwd_workspace_layout(p->B, p->N, p->H, p->M, p->Cout);
+  if (workspace == nullptr) return IPA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
+  auto outp = [](const ipa_tensor_t& t) { return static_cast<float*>(const_cast<void*>(t.data)); };
+  a.g_output = view_of(g_output);
+  a.g_attention = view_of(has_ga ? g_attention : nullptr);
+  a.g_vectors = view_of(has_gv ? g_vectors : nullptr);
+  a.g_attention.dtype = a.g_vectors.dtype = a.g_output.dtype;
+  a.has_g_attention = has_ga;
+  a.has_g_vectors = has_gv;
+  a.d_q_direction = outp(grads->q_direction); a.d_k_direction = outp(grads->k_direction);
+  a.d_q_point = outp(grads->q_point); a.d_k_point = outp(grads->k_point); a.d_values = outp(grads->values);
+  a.d_direction_scale = outp(grads->direction_scale); a.d_distance_scale = outp(grads->distance_scale);
+  a.d_output_weight = outp(grads->output_weight);
+  a.d_output_bias = want_bias ? outp(grads->output_bias) : nullptr;
+  a.d_rotation = outp(grads->rotation); a.d_translation = outp(grads->translation);
+  a.ws = static_cast<unsigned char*>(workspace);
+  a.lay = lay;
+  a.f.ws = a.ws;
+  a.f.lay = lay.fwd;
+  a.f.err = reinterpret_cast<int*>(a.ws + lay.fwd.err);
+  if (geo_launch_bwd(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return IPA_ERR_CUDA;
   return IPA_OK;
 }
 

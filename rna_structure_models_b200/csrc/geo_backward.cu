@@ -1,0 +1,599 @@
+// Gradients of the geometric direction-and-distance attention for sm_100a
+// ("Geometric direction-and-distance attention", Required behavior: the
+// operator is differentiated with the derivative of the unsquared distance
+// at a zero displacement defined as the zero vector).
+//
+// With s_ij = (A <qd_i, kd_j> - B |qp_i - kp_j|) / sqrt(3), a = masked
+// softmax_j(s), agg_i = sum_j a_ij vr_j and upstream gradients g_output,
+// g_attention, g_vectors:
+//   g_vec_i  = g_vectors_i + [i has an allowed key] g_output_i W^T
+//   dagg_i   = R_i g_vec_i,   da_ij = <dagg_i, vr_j> + g_attention_ij
+//   ds_ij    = a_ij (da_ij - D_i),  D_i = sum_j a_ij da_ij
+//            = <dagg_i, agg_i> + sum_j a_ij g_attention_ij
+//   d qd_i   =  A/sqrt3 sum_j ds_ij kd_j,   d qp_i = -B/sqrt3 sum_j ds_ij u_ij
+//   d kd_j   =  A/sqrt3 sum_i ds_ij qd_i,   d kp_j =  B/sqrt3 sum_i ds_ij u_ij
+//   d vr_j   =  sum_i a_ij dagg_i,  u_ij = (qp_i - kp_j) / |qp_i - kp_j| or 0
+// Launches (all fp32 on CUDA cores; the per-pair terms are recomputed, no
+// N x N array is stored):
+//   0. the forward statistics (scales, rotated inputs, row max / sum, agg)
+//   1. geo_gvec_kernel     -- per (b, n): g_vec and whether any head is live
+//   2. geo_dagg_kernel     -- per (b, n, h): dagg = R g_vec, <dagg, agg>
+//   3. geo_dw_kernel       -- dW = vec^T g_output, db = sum g_output (live rows)
+//   4. geo_bwd_rows_kernel -- per (b, h, 128 queries) x 4 key splits: D_i,
+//                             then d qd, d qp and the per-head sums of
+//                             ds <qd, kd> and ds |qp - kp|
+//   5. geo_bwd_cols_kernel -- per (b, h, 128 keys) x 4 query splits: d kd,
+//                             d kp, d vr
+//   6. geo_bwd_frame_kernel -- per (b, n): local gradients R^T (...), the
+//                             rotation and translation gradients summed over
+//                             heads; block 0 also writes the scale gradients.
+#include <cmath>
+#include <cstdint>
+
+#include "geo_common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fipa {
+
+using namespace sm100;
+using namespace geo;
+
+namespace {
+
+constexpr int BW_ROWS = 128;
+constexpr int BW_SPLIT = 4;
+constexpr int BW_CHUNK = 32;
+constexpr float kInvSqrt3 = 0.57735026918962576f;
+
+struct GvecArgs {
+  int B, N, H, HM3, Cout;
+  View g_output, g_vectors;
+  bool has_g_vectors;
+  const unsigned char* live;   // [B, N, H]
+  const float* wt;             // [Cout, HM3]
+  float* gvec;                 // [B*N, HM3]
+  unsigned char* rowlive;      // [B*N]
+};
+
+// g_vec = g_vectors + [row live] g_output W^T.  Block: 32 k-columns x 8 row
+// groups; each thread covers 4 rows of one column.
+__global__ void __launch_bounds__(256) geo_gvec_kernel(const GvecArgs a) {
+  const int kx = blockIdx.y * 32 + threadIdx.x;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.N;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32 + threadIdx.y * 4;
+  bool lv[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int64_t row = row0 + q;
+    bool l = false;
+    if (row < rows)
+      for (int h = 0; h < a.H; ++h) l |= a.live[row * a.H + h] != 0;
+    lv[q] = l;
+    if (blockIdx.y == 0 && threadIdx.x == 0 && row < rows) a.rowlive[row] = l ? 1 : 0;
+  }
+  if (kx >= a.HM3) return;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int c = 0; c < a.Cout; ++c) {
+    const float w = a.wt[static_cast<int64_t>(c) * a.HM3 + kx];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t row = row0 + q;
+      if (row < rows && lv[q]) {
+        const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
+        acc[q] = fmaf(ldf(a.g_output, b * a.g_output.s[0] + n * a.g_output.s[1] + c * a.g_output.s[2]), w, acc[q]);
+      }
+    }
+  }
+  const int h = kx / (a.HM3 / a.H), mx = kx % (a.HM3 / a.H), m = mx / 3, x = mx % 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int64_t row = row0 + q;
+    if (row >= rows) continue;
+    float g = acc[q];
+    if (a.has_g_vectors) {
+      const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
+      const View& v = a.g_vectors;
+      g += ldf(v, b * v.s[0] + n * v.s[1] + h * v.s[2] + m * v.s[3] + x * v.s[4]);
+    }
+    a.gvec[row * a.HM3 + kx] = g;
+  }
+}
+
+struct DaggArgs {
+  int B, N, H, M, VW, HM3;
+  const float* gvec;   // [B*N, HM3]
+  const float* rotf;   // [B, N, 9]
+  const float* agg;    // [B*H, N, VW]
+  float* dagg;         // [B*H, N, VW]
+  float4* rowinfo;     // [B*H, N]: .z <- <dagg, agg>
+};
+
+__global__ void __launch_bounds__(256) geo_dagg_kernel(const DaggArgs a) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<int64_t>(a.B) * a.N * a.H) return;
+  const int h = static_cast<int>(t % a.H);
+  const int64_t bn = t / a.H;
+  const int b = static_cast<int>(bn / a.N), n = static_cast<int>(bn % a.N);
+  const float* R = a.rotf + bn * 9;
+  const float* g = a.gvec + bn * a.HM3 + h * 3 * a.M;
+  const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.N + n;
+  const float* ag = a.agg + row * a.VW;
+  float* dst = a.dagg + row * a.VW;
+  float d1 = 0.f;
+  for (int m = 0; m < a.M; ++m) {
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      const float v = fmaf(R[3 * x], g[3 * m], fmaf(R[3 * x + 1], g[3 * m + 1], R[3 * x + 2] * g[3 * m + 2]));
+      dst[3 * m + x] = v;
+      d1 = fmaf(v, ag[3 * m + x], d1);
+    }
+  }
+  a.rowinfo[row] = make_float4(0.f, 0.f, d1, 0.f);
+}
+
+struct DwArgs {
+  int64_t rows;
+  int HM3, Cout;
+  View g_output;
+  int N;
+  const float* vec;                // [rows, HM3]
+  const unsigned char* rowlive;    // [rows]
+  float* d_w;                      // [HM3, Cout]
+  float* d_b;                      // [Cout] or null
+};
+
+// One thread per (k, c): a deterministic sum over all rows.
+__global__ void __launch_bounds__(256) geo_dw_kernel(const DwArgs a) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int k = blockIdx.y;
+  if (c >= a.Cout) return;
+  float acc = 0.f, accb = 0.f;
+  for (int64_t row = 0; row < a.rows; ++row) {
+    if (!a.rowlive[row]) continue;
+    const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
+    const float g = ldf(a.g_output, b * a.g_output.s[0] + n * a.g_output.s[1] + c * a.g_output.s[2]);
+    acc = fmaf(a.vec[row * a.HM3 + k], g, acc);
+    accb += g;
+  }
+  a.d_w[static_cast<int64_t>(k) * a.Cout + c] = acc;
+  if (k == 0 && a.d_b) a.d_b[c] = accb;
+}
+
+struct PairArgs {
+  int B, N, H, VW;
+  const float4* qg;      // [B*H, N, 2]
+  const float4* kg;      // [B*H, N, 2]
+  const float* vg;       // [B*H, N, VW]
+  const float2* sc;      // [H]
+  const float2* ml;      // [B*H, N]
+  const float* dagg;     // [B*H, N, VW]
+  float4* rowinfo;       // [B*H, N]: (m, 1/l or 0, D, 0)
+  const unsigned char* pm;
+  int64_t pms[4];
+  View g_att;
+  bool has_g_att;
+  float4* dq;            // [B*H, N, 2]: (d qd, 0), (d qp, 0) in the global frame
+  float4* dk;            // [B*H, N, 2]
+  float* dvr;            // [B*H, N, VW]
+  float* acc;            // [2H]: sum ds <qd, kd>, sum ds |qp - kp|
+};
+
+__device__ __forceinline__ float g_att_at(const PairArgs& a, int b, int h, int i, int j) {
+  const View& v = a.g_att;
+  return ldf(v, b * v.s[0] + h * v.s[1] + static_cast<int64_t>(i) * v.s[2] + static_cast<int64_t>(j) * v.s[3]);
+}
+
+template <int M>
+__global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_rows_kernel(const PairArgs a) {
+  constexpr int V = 3 * M;
+  const int tid = threadIdx.x;
+  const int r = tid % BW_ROWS, split = tid / BW_ROWS;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int i = blockIdx.x * BW_ROWS + r;
+  const int N = a.N;
+  const int64_t bh = static_cast<int64_t>(b) * a.H + h;
+  const float2 sc = a.sc[h];
+  const bool in_range = i < N;
+  float4 q0 = make_float4(0, 0, 0, 0), q1 = q0;
+  float m = 0.f, inv = 0.f, d1 = 0.f;
+  float dg[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) dg[e] = 0.f;
+  if (in_range) {
+    const float2 st = a.ml[bh * N + i];
+    if (st.y > 0.f) {
+      m = st.x;
+      inv = 1.f / st.y;
+      q0 = a.qg[2 * (bh * N + i)];
+      q1 = a.qg[2 * (bh * N + i) + 1];
+      d1 = a.rowinfo[bh * N + i].z;
+#pragma unroll
+      for (int e = 0; e < V; ++e) dg[e] = a.dagg[(bh * N + i) * a.VW + e];
+    }
+  }
+  const bool live = inv > 0.f;
+  const unsigned char* pmrow =
+      a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(in_range ? i : 0) * a.pms[2] : nullptr;
+  const int nchunk = (N + BW_CHUNK - 1) / BW_CHUNK;
+  extern __shared__ float bw_merge[];   // [BW_SPLIT][8][BW_ROWS]
+  auto sm_at = [&](int s2, int e) -> float& { return bw_merge[(s2 * 8 + e) * BW_ROWS + r]; };
+
+  // D_i = <dagg_i, agg_i> + sum_j a_ij g_attention_ij
+  float dsum = 0.f;
+  if (a.has_g_att && live) {
+    for (int ch = split; ch < nchunk; ch += BW_SPLIT)
+      for (int k = 0; k < BW_CHUNK; ++k) {
+        const int j = ch * BW_CHUNK + k;
+        if (j >= N) break;
+        if (pmrow && !pmrow[static_cast<int64_t>(j) * a.pms[3]]) continue;
+        const float4 k0 = a.kg[2 * (bh * N + j)], k1 = a.kg[2 * (bh * N + j) + 1];
+        const float p = ex2(geo_score(q0, q1, k0, k1, sc.x, sc.y) - m) * inv;
+        dsum = fmaf(p, g_att_at(a, b, h, i, j), dsum);
+      }
+  }
+  sm_at(split, 0) = dsum;
+  __syncthreads();
+  float D = d1;
+#pragma unroll
+  for (int s2 = 0; s2 < BW_SPLIT; ++s2) D += sm_at(s2, 0);
+  __syncthreads();
+
+  float cq[3] = {0.f, 0.f, 0.f}, cp[3] = {0.f, 0.f, 0.f}, sdot = 0.f, sdist = 0.f;
+  if (live) {
+    for (int ch = split; ch < nchunk; ch += BW_SPLIT)
+      for (int k = 0; k < BW_CHUNK; ++k) {
+        const int j = ch * BW_CHUNK + k;
+        if (j >= N) break;
+        if (pmrow && !pmrow[static_cast<int64_t>(j) * a.pms[3]]) continue;
+        const float4 k0 = a.kg[2 * (bh * N + j)], k1 = a.kg[2 * (bh * N + j) + 1];
+        const GeoPair g = geo_pair(q0, q1, k0, k1, sc.x, sc.y);
+        const float p = ex2(g.s - m) * inv;
+        if (p == 0.f) continue;
+        const float* vr = a.vg + (bh * N + j) * a.VW;
+        float da = a.has_g_att ? g_att_at(a, b, h, i, j) : 0.f;
+#pragma unroll
+        for (int e = 0; e < V; ++e) da = fmaf(dg[e], vr[e], da);
+        const float ds = p * (da - D);
+        cq[0] = fmaf(ds, k0.x, cq[0]);
+        cq[1] = fmaf(ds, k0.y, cq[1]);
+        cq[2] = fmaf(ds, k0.z, cq[2]);
+        const float ru = g.dist > 0.f ? ds / g.dist : 0.f;   // zero displacement: zero derivative
+        cp[0] = fmaf(ru, g.dx, cp[0]);
+        cp[1] = fmaf(ru, g.dy, cp[1]);
+        cp[2] = fmaf(ru, g.dz, cp[2]);
+        sdot = fmaf(ds, g.dot, sdot);
+        sdist = fmaf(ds, g.dist, sdist);
+      }
+  }
+  sm_at(split, 0) = cq[0]; sm_at(split, 1) = cq[1]; sm_at(split, 2) = cq[2];
+  sm_at(split, 3) = cp[0]; sm_at(split, 4) = cp[1]; sm_at(split, 5) = cp[2];
+  sm_at(split, 6) = sdot;  sm_at(split, 7) = sdist;
+  __syncthreads();
+  if (split != 0) return;
+  float t[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    t[e] = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < BW_SPLIT; ++s2) t[e] += sm_at(s2, e);
+  }
+  const float Ar = sc.x / kLog2e, Br = sc.y / kLog2e;   // A / sqrt3, B / sqrt3
+  if (in_range) {
+    a.dq[2 * (bh * N + i)] = make_float4(Ar * t[0], Ar * t[1], Ar * t[2], 0.f);
+    a.dq[2 * (bh * N + i) + 1] = make_float4(-Br * t[3], -Br * t[4], -Br * t[5], 0.f);
+    a.rowinfo[bh * N + i] = make_float4(m, inv, D, 0.f);
+  }
+  // per-head sums over the block's rows (warps 0-3 hold split 0)
+  float s6 = t[6], s7 = t[7];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s6 += __shfl_xor_sync(0xffffffffu, s6, o);
+    s7 += __shfl_xor_sync(0xffffffffu, s7, o);
+  }
+  if ((tid & 31) == 0) {
+    atomicAdd(a.acc + h, s6);
+    atomicAdd(a.acc + a.H + h, s7);
+  }
+}
+
+template <int M>
+__global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_cols_kernel(const PairArgs a) {
+  constexpr int V = 3 * M;
+  const int tid = threadIdx.x;
+  const int r = tid % BW_ROWS, split = tid / BW_ROWS;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int j = blockIdx.x * BW_ROWS + r;
+  const int N = a.N;
+  const int64_t bh = static_cast<int64_t>(b) * a.H + h;
+  const float2 sc = a.sc[h];
+  const bool in_range = j < N;
+  float4 k0 = make_float4(0, 0, 0, -INFINITY), k1 = make_float4(0, 0, 0, 0);
+  float vr[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) vr[e] = 0.f;
+  if (in_range) {
+    k0 = a.kg[2 * (bh * N + j)];
+    k1 = a.kg[2 * (bh * N + j) + 1];
+#pragma unroll
+    for (int e = 0; e < V; ++e) vr[e] = a.vg[(bh * N + j) * a.VW + e];
+  }
+  float ck[3] = {0.f, 0.f, 0.f}, cp[3] = {0.f, 0.f, 0.f}, dv[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) dv[e] = 0.f;
+  const unsigned char* pmcol =
+      a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(in_range ? j : 0) * a.pms[3] : nullptr;
+  const int nchunk = (N + BW_CHUNK - 1) / BW_CHUNK;
+  if (in_range && k0.w == 0.f) {
+    for (int ch = split; ch < nchunk; ch += BW_SPLIT)
+      for (int k = 0; k < BW_CHUNK; ++k) {
+        const int i = ch * BW_CHUNK + k;
+        if (i >= N) break;
+        const float4 info = a.rowinfo[bh * N + i];     // same i across the warp: one broadcast load
+        if (info.y == 0.f) continue;                   // query without an allowed key
+        if (pmcol && !pmcol[static_cast<int64_t>(i) * a.pms[2]]) continue;
+        const float4 q0 = a.qg[2 * (bh * N + i)], q1 = a.qg[2 * (bh * N + i) + 1];
+        const GeoPair g = geo_pair(q0, q1, k0, k1, sc.x, sc.y);
+        const float p = ex2(g.s - info.x) * info.y;
+        if (p == 0.f) continue;
+        const float* dg = a.dagg + (bh * N + i) * a.VW;
+        float da = a.has_g_att ? g_att_at(a, b, h, i, j) : 0.f;
+        float dgv[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          dgv[e] = dg[e];
+          da = fmaf(dgv[e], vr[e], da);
+        }
+        const float ds = p * (da - info.z);
+        ck[0] = fmaf(ds, q0.x, ck[0]);
+        ck[1] = fmaf(ds, q0.y, ck[1]);
+        ck[2] = fmaf(ds, q0.z, ck[2]);
+        const float ru = g.dist > 0.f ? ds / g.dist : 0.f;
+        cp[0] = fmaf(ru, g.dx, cp[0]);
+        cp[1] = fmaf(ru, g.dy, cp[1]);
+        cp[2] = fmaf(ru, g.dz, cp[2]);
+#pragma unroll
+        for (int e = 0; e < V; ++e) dv[e] = fmaf(p, dgv[e], dv[e]);
+      }
+  }
+  extern __shared__ float bw_merge[];   // [BW_SPLIT][6 + V][BW_ROWS]
+  auto sm_at = [&](int s2, int e) -> float& { return bw_merge[(s2 * (6 + V) + e) * BW_ROWS + r]; };
+#pragma unroll
+  for (int e = 0; e < 3; ++e) {
+    sm_at(split, e) = ck[e];
+    sm_at(split, 3 + e) = cp[e];
+  }
+#pragma unroll
+  for (int e = 0; e < V; ++e) sm_at(split, 6 + e) = dv[e];
+  __syncthreads();
+  if (split != 0 || !in_range) return;
+  float t[6 + V];
+#pragma unroll
+  for (int e = 0; e < 6 + V; ++e) {
+    t[e] = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < BW_SPLIT; ++s2) t[e] += sm_at(s2, e);
+  }
+  const float Ar = sc.x / kLog2e, Br = sc.y / kLog2e;
+  a.dk[2 * (bh * N + j)] = make_float4(Ar * t[0], Ar * t[1], Ar * t[2], 0.f);
+  a.dk[2 * (bh * N + j) + 1] = make_float4(Br * t[3], Br * t[4], Br * t[5], 0.f);   // u points from kp to qp
+#pragma unroll
+  for (int e = 0; e < V; ++e) a.dvr[(bh * N + j) * a.VW + e] = t[6 + e];
+}
+
+struct FrameArgs {
+  int B, N, H, M, VW, HM3;
+  View qd, kd, qp, kp, val, dscale, xscale;
+  const float* rotf;
+  const float* agg;      // [B*H, N, VW]
+  const float* gvec;     // [B*N, HM3]
+  const float4* dq;
+  const float4* dk;
+  const float* dvr;
+  const float* acc;      // [2H]
+  float *d_qd, *d_kd, *d_qp, *d_kp, *d_val, *d_rot, *d_trans, *d_dscale, *d_xscale;
+};
+
+__global__ void __launch_bounds__(128) geo_bwd_frame_kernel(const FrameArgs a) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (blockIdx.x == 0)
+    for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+      // d scale = dA sigmoid(scale); dA = sum ds dot / sqrt3, dB = -sum ds dist / sqrt3
+      const float xd = ldf(a.dscale, h * a.dscale.s[0]), xx = ldf(a.xscale, h * a.xscale.s[0]);
+      a.d_dscale[h] = a.acc[h] * kInvSqrt3 / (1.f + expf(-xd));
+      a.d_xscale[h] = -a.acc[a.H + h] * kInvSqrt3 / (1.f + expf(-xx));
+    }
+  if (t >= static_cast<int64_t>(a.B) * a.N) return;
+  const int b = static_cast<int>(t / a.N), n = static_cast<int>(t % a.N);
+  const float* R = a.rotf + t * 9;
+  float dR[9], dT[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < 9; ++e) dR[e] = 0.f;
+  // local gradient R^T g and dR += g x^T for one rotated 3-vector x
+  auto back = [&](const float g[3], const View& v, int64_t base, int64_t sx, float* out) {
+    const float x0 = ldf(v, base), x1 = ldf(v, base + sx), x2 = ldf(v, base + 2 * sx);
+#pragma unroll
+    for (int y = 0; y < 3; ++y) out[y] = fmaf(R[y], g[0], fmaf(R[3 + y], g[1], R[6 + y] * g[2]));
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      dR[3 * x] = fmaf(g[x], x0, dR[3 * x]);
+      dR[3 * x + 1] = fmaf(g[x], x1, dR[3 * x + 1]);
+      dR[3 * x + 2] = fmaf(g[x], x2, dR[3 * x + 2]);
+    }
+  };
+  for (int h = 0; h < a.H; ++h) {
+    const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.N + n;
+    const int64_t o3 = (t * a.H + h) * 3;
+    const float4 q0 = a.dq[2 * row], q1 = a.dq[2 * row + 1], k0 = a.dk[2 * row], k1 = a.dk[2 * row + 1];
+    const float gqd[3] = {q0.x, q0.y, q0.z}, gqp[3] = {q1.x, q1.y, q1.z};
+    const float gkd[3] = {k0.x, k0.y, k0.z}, gkp[3] = {k1.x, k1.y, k1.z};
+    back(gqd, a.qd, b * a.qd.s[0] + n * a.qd.s[1] + h * a.qd.s[2], a.qd.s[3], a.d_qd + o3);
+    back(gkd, a.kd, b * a.kd.s[0] + n * a.kd.s[1] + h * a.kd.s[2], a.kd.s[3], a.d_kd + o3);
+    back(gqp, a.qp, b * a.qp.s[0] + n * a.qp.s[1] + h * a.qp.s[2], a.qp.s[3], a.d_qp + o3);
+    back(gkp, a.kp, b * a.kp.s[0] + n * a.kp.s[1] + h * a.kp.s[2], a.kp.s[3], a.d_kp + o3);
+#pragma unroll
+    for (int x = 0; x < 3; ++x) dT[x] += gqp[x] + gkp[x];
+    for (int m = 0; m < a.M; ++m) {
+      const float* dv = a.dvr + row * a.VW + 3 * m;
+      const float gv[3] = {dv[0], dv[1], dv[2]};
+      back(gv, a.val, b * a.val.s[0] + n * a.val.s[1] + h * a.val.s[2] + m * a.val.s[3], a.val.s[4],
+           a.d_val + (t * a.H + h) * a.VW + 3 * m);
+      // vectors = R^T agg: dR += agg g_vec^T
+      const float* ag = a.agg + row * a.VW + 3 * m;
+      const float* gq = a.gvec + t * a.HM3 + h * a.VW + 3 * m;
+#pragma unroll
+      for (int x = 0; x < 3; ++x)
+#pragma unroll
+        for (int y = 0; y < 3; ++y) dR[3 * x + y] = fmaf(ag[x], gq[y], dR[3 * x + y]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 9; ++e) a.d_rot[t * 9 + e] = dR[e];
+#pragma unroll
+  for (int x = 0; x < 3; ++x) a.d_trans[t * 3 + x] = dT[x];
+}
+
+struct TransposeArgs {
+  int HM3, Cout;
+  View w;
+  float* wt;   // [Cout, HM3]
+};
+
+__global__ void geo_wt_kernel(const TransposeArgs a) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<int64_t>(a.HM3) * a.Cout) return;
+  const int c = static_cast<int>(t / a.HM3), k = static_cast<int>(t % a.HM3);
+  a.wt[t] = ldf(a.w, k * a.w.s[0] + c * a.w.s[1]);
+}
+
+template <int M>
+cudaError_t launch_pairs(const PairArgs& p, int B, int N, int H, cudaStream_t st) {
+  dim3 grid((N + BW_ROWS - 1) / BW_ROWS, H, B);
+  const size_t smem_r = sizeof(float) * BW_SPLIT * 8 * BW_ROWS;
+  const size_t smem_c = sizeof(float) * BW_SPLIT * (6 + 3 * M) * BW_ROWS;
+  if (smem_c > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(geo_bwd_cols_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_c));
+    if (e != cudaSuccess) return e;
+  }
+  geo_bwd_rows_kernel<M><<<grid, BW_ROWS * BW_SPLIT, smem_r, st>>>(p);
+  geo_bwd_cols_kernel<M><<<grid, BW_ROWS * BW_SPLIT, smem_c, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+GeoBwdWorkspace geo_bwd_workspace_layout(int B, int N, int H, int M, int Cout) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  GeoBwdWorkspace w{};
+  w.fwd = geo_workspace_layout(B, N, H, M, Cout);
+  size_t o = w.fwd.total;
+  const size_t bn = static_cast<size_t>(B) * N, bhn = bn * H;
+  const size_t VW = 3 * static_cast<size_t>(M), HM3 = static_cast<size_t>(H) * VW;
+  w.vec = o; o = up(o + bn * HM3 * 4);
+  w.agg = o; o = up(o + bhn * VW * 4);
+  w.gvec = o; o = up(o + bn * HM3 * 4);
+  w.rowlive = o; o = up(o + bn);
+  w.dagg = o; o = up(o + bhn * VW * 4);
+  w.rowinfo = o; o = up(o + bhn * 16);
+  w.dq = o; o = up(o + bhn * 32);
+  w.dk = o; o = up(o + bhn * 32);
+  w.dvr = o; o = up(o + bhn * VW * 4);
+  w.acc = o; o = up(o + static_cast<size_t>(H) * 8);
+  w.wt = o; o = up(o + HM3 * static_cast<size_t>(Cout) * 4);
+  w.total = o;
+  return w;
+}
+
+cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
+  const GeoBwdWorkspace& w = a.lay;
+  unsigned char* ws = a.ws;
+  const int B = a.f.B, N = a.f.N, H = a.f.H, M = a.f.M, HM3 = a.f.HM3, Cout = a.f.Cout, VW = 3 * M;
+  const int64_t rows = static_cast<int64_t>(B) * N;
+
+  // 0. forward statistics: scales, rotated inputs, (m, l), agg, vectors
+  GeoLaunch f = a.f;
+  f.ws = ws;
+  f.lay = w.fwd;
+  f.out_vectors = reinterpret_cast<float*>(ws + w.vec);
+  f.out_output = nullptr;
+  f.out_attention = nullptr;
+  f.out_agg = reinterpret_cast<float*>(ws + w.agg);
+  f.skip_readout = true;
+  cudaError_t e = geo_launch_all(f, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(ws + w.acc, 0, static_cast<size_t>(H) * 8, st);
+  if (e != cudaSuccess) return e;
+
+  {
+    TransposeArgs ta{HM3, Cout, a.f.output_weight, reinterpret_cast<float*>(ws + w.wt)};
+    const int64_t n = static_cast<int64_t>(HM3) * Cout;
+    geo_wt_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(ta);
+  }
+  GvecArgs ga{};
+  ga.B = B; ga.N = N; ga.H = H; ga.HM3 = HM3; ga.Cout = Cout;
+  ga.g_output = a.g_output; ga.g_vectors = a.g_vectors; ga.has_g_vectors = a.has_g_vectors;
+  ga.live = ws + w.fwd.live;
+  ga.wt = reinterpret_cast<const float*>(ws + w.wt);
+  ga.gvec = reinterpret_cast<float*>(ws + w.gvec);
+  ga.rowlive = ws + w.rowlive;
+  geo_gvec_kernel<<<dim3(static_cast<unsigned>((rows + 31) / 32), (HM3 + 31) / 32), dim3(32, 8), 0, st>>>(ga);
+
+  DaggArgs da{};
+  da.B = B; da.N = N; da.H = H; da.M = M; da.VW = VW; da.HM3 = HM3;
+  da.gvec = ga.gvec;
+  da.rotf = reinterpret_cast<const float*>(ws + w.fwd.rotf);
+  da.agg = f.out_agg;
+  da.dagg = reinterpret_cast<float*>(ws + w.dagg);
+  da.rowinfo = reinterpret_cast<float4*>(ws + w.rowinfo);
+  geo_dagg_kernel<<<static_cast<unsigned>((rows * H + 255) / 256), 256, 0, st>>>(da);
+
+  DwArgs dw{};
+  dw.rows = rows; dw.HM3 = HM3; dw.Cout = Cout; dw.g_output = a.g_output; dw.N = N;
+  dw.vec = f.out_vectors; dw.rowlive = ga.rowlive; dw.d_w = a.d_output_weight; dw.d_b = a.d_output_bias;
+  geo_dw_kernel<<<dim3((Cout + 255) / 256, HM3), 256, 0, st>>>(dw);
+
+  PairArgs p{};
+  p.B = B; p.N = N; p.H = H; p.VW = VW;
+  p.qg = reinterpret_cast<const float4*>(ws + w.fwd.qg);
+  p.kg = reinterpret_cast<const float4*>(ws + w.fwd.kg);
+  p.vg = reinterpret_cast<const float*>(ws + w.fwd.vg);
+  p.sc = reinterpret_cast<const float2*>(ws + w.fwd.sc);
+  p.ml = reinterpret_cast<const float2*>(ws + w.fwd.ml);
+  p.dagg = da.dagg;
+  p.rowinfo = da.rowinfo;
+  p.pm = a.f.has_pair_mask ? reinterpret_cast<const unsigned char*>(a.f.pair_mask.p) : nullptr;
+  for (int d = 0; d < 4; ++d) p.pms[d] = a.f.has_pair_mask ? a.f.pair_mask.s[d] : 0;
+  p.g_att = a.g_attention;
+  p.has_g_att = a.has_g_attention;
+  p.dq = reinterpret_cast<float4*>(ws + w.dq);
+  p.dk = reinterpret_cast<float4*>(ws + w.dk);
+  p.dvr = reinterpret_cast<float*>(ws + w.dvr);
+  p.acc = reinterpret_cast<float*>(ws + w.acc);
+  switch (M) {
+    case 1: e = launch_pairs<1>(p, B, N, H, st); break;
+    case 2: e = launch_pairs<2>(p, B, N, H, st); break;
+    case 3: e = launch_pairs<3>(p, B, N, H, st); break;
+    case 4: e = launch_pairs<4>(p, B, N, H, st); break;
+    case 5: e = launch_pairs<5>(p, B, N, H, st); break;
+    case 6: e = launch_pairs<6>(p, B, N, H, st); break;
+    case 7: e = launch_pairs<7>(p, B, N, H, st); break;
+    case 8: e = launch_pairs<8>(p, B, N, H, st); break;
+    default: e = cudaErrorInvalidValue; break;
+  }
+  if (e != cudaSuccess) return e;
+
+  FrameArgs fa{};
+  fa.B = B; fa.N = N; fa.H = H; fa.M = M; fa.VW = VW; fa.HM3 = HM3;
+  fa.qd = a.f.q_direction; fa.kd = a.f.k_direction; fa.qp = a.f.q_point; fa.kp = a.f.k_point;
+  fa.val = a.f.values; fa.dscale = a.f.direction_scale; fa.xscale = a.f.distance_scale;
+  fa.rotf = da.rotf; fa.agg = f.out_agg; fa.gvec = ga.gvec;
+  fa.dq = p.dq; fa.dk = p.dk; fa.dvr = p.dvr; fa.acc = p.acc;
+  fa.d_qd = a.d_q_direction; fa.d_kd = a.d_k_direction; fa.d_qp = a.d_q_point; fa.d_kp = a.d_k_point;
+  fa.d_val = a.d_values; fa.d_rot = a.d_rotation; fa.d_trans = a.d_translation;
+  fa.d_dscale = a.d_direction_scale; fa.d_xscale = a.d_distance_scale;
+  geo_bwd_frame_kernel<<<static_cast<unsigned>((rows + 127) / 128), 128, 0, st>>>(fa);
+  return cudaGetLastError();
+}
+
+}  // namespace fipa

@@ -20,32 +20,20 @@
 #include <cmath>
 #include <cstdint>
 
+#include "geo_common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
 namespace fipa {
 
 using namespace sm100;
+using namespace geo;
 
 namespace {
 
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr int GEO_ROWS = 128;
 constexpr int GEO_SPLIT = 4;
 constexpr int GEO_CHUNK = 32;
-
-__device__ __forceinline__ float ldf(const View& v, int64_t off) {
-  if (v.dtype == 1) return static_cast<float>(reinterpret_cast<const double*>(v.p)[off]);
-  return reinterpret_cast<const float*>(v.p)[off];
-}
-__device__ __forceinline__ bool ldb(const View& v, int64_t off) {
-  return reinterpret_cast<const unsigned char*>(v.p)[off] != 0;
-}
-
-// log(1 + exp(x)) without overflow: max(x, 0) + log1p(exp(-|x|))
-__device__ __forceinline__ float softplus_stable(float x) {
-  return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
-}
 
 struct WArgs {
   int H, HM3, Cout;
@@ -132,18 +120,6 @@ __global__ void geo_prep_kernel(const PrepArgs a) {
   }
 }
 
-// Score in the log2 domain.  The same instruction sequence is used by the
-// aggregation kernel and by the attention-map kernel so both see identical
-// values.
-__device__ __forceinline__ float geo_score(const float4 q0, const float4 q1, const float4 k0,
-                                           const float4 k1, float A, float Bd) {
-  const float dot = fmaf(q0.x, k0.x, fmaf(q0.y, k0.y, __fmul_rn(q0.z, k0.z)));
-  const float dx = __fsub_rn(q1.x, k1.x), dy = __fsub_rn(q1.y, k1.y), dz = __fsub_rn(q1.z, k1.z);
-  const float d2 = fmaf(dx, dx, fmaf(dy, dy, __fmul_rn(dz, dz)));
-  const float dist = __fsqrt_rn(d2);
-  return __fadd_rn(__fadd_rn(fmaf(A, dot, -__fmul_rn(Bd, dist)), q0.w), k0.w);
-}
-
 struct AttnArgs {
   int B, N, H, VW;
   float tau;
@@ -157,6 +133,7 @@ struct AttnArgs {
   float* out_vectors;        // [B, N, H, M, 3]
   float2* ml;                // [B*H, N]
   unsigned char* live;       // [B, N, H]
+  float* agg;                // [B*H, N, VW] aggregated global-frame values, or null
 };
 
 template <int M>
@@ -267,6 +244,11 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT) geo_attn_kernel(const At
   const float inv = has ? 1.f / lf : 0.f;
   const float* R = a.rotf + (static_cast<int64_t>(b) * N + i) * 9;
   float* dst = a.out_vectors + ((static_cast<int64_t>(b) * N + i) * a.H + h) * V;
+  if (a.agg) {
+    float* ag = a.agg + (bh * N + i) * a.VW;
+#pragma unroll
+    for (int e = 0; e < V; ++e) ag[e] = has ? af[e] * inv : 0.f;
+  }
 #pragma unroll
   for (int mm = 0; mm < M; ++mm) {
     const float gx = af[3 * mm] * inv, gy = af[3 * mm + 1] * inv, gz = af[3 * mm + 2] * inv;
@@ -433,6 +415,7 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
   t.out_vectors = a.out_vectors;
   t.ml = reinterpret_cast<float2*>(ws + w.ml);
   t.live = ws + w.live;
+  t.agg = a.out_agg;
   cudaError_t le = cudaErrorInvalidValue;
   switch (a.M) {
     case 1: le = launch_attn<1>(t, a.B, a.N, a.H, st); break;
@@ -456,6 +439,8 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
     ma.att = a.out_attention;
     geo_map_kernel<<<dim3(a.N, a.H, a.B), 256, 0, st>>>(ma);
   }
+
+  if (a.skip_readout) return cudaGetLastError();
 
   ReadArgs ra{};
   ra.B = a.B; ra.N = a.N; ra.H = a.H; ra.HM3 = a.HM3; ra.Cout = a.Cout;

@@ -86,12 +86,34 @@ struct GeoLaunch {
   float* out_vectors;
   float* out_output;
   float* out_attention;  // may be null
+  float* out_agg;        // [B*H, N, 3M] global-frame aggregate, or null
+  bool skip_readout;     // stop after the vectors (gradient pass)
   unsigned char* ws;
   GeoWorkspace lay;
   int* err;
 };
 
 cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t stream);
+
+// Gradients of the variant: the forward statistics are recomputed into the
+// forward part of the workspace, then the adjoint kernels run.
+struct GeoBwdWorkspace {
+  GeoWorkspace fwd;   // offsets relative to the start of the gradient workspace
+  size_t vec, agg, gvec, rowlive, dagg, rowinfo, dq, dk, dvr, acc, wt, total;
+};
+GeoBwdWorkspace geo_bwd_workspace_layout(int B, int N, int H, int M, int Cout);
+
+struct GeoBwdLaunch {
+  GeoLaunch f;             // forward inputs; its ws / lay point into the gradient workspace
+  View g_output, g_attention, g_vectors;
+  bool has_g_attention, has_g_vectors;
+  // gradients (contiguous fp32); d_output_bias may be null
+  float *d_q_direction, *d_k_direction, *d_q_point, *d_k_point, *d_values, *d_direction_scale,
+      *d_distance_scale, *d_output_weight, *d_output_bias, *d_rotation, *d_translation;
+  unsigned char* ws;
+  GeoBwdWorkspace lay;
+};
+cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t stream);
 
 #ifdef IPA_TRACE
 bool ipa_trace_read(void* host, size_t bytes);

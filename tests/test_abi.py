@@ -265,3 +265,59 @@ def test_frames_rejects_bad_arguments_before_launch(case, expect):
     elif case == "trans_shape":
         over["trans"] = desc((2, 64, 4))
     assert frames_call(**over) == expect
+
+
+def geo_bwd_call(p, ds, grads_over=None, ws_bytes=None, **up_over):
+    lib = api.library()
+    B, N, H, M, Cout = p.B, p.N, p.H, p.M, p.Cout
+    up = {"g_output": desc((B, N, Cout)), "g_attention": desc((B, H, N, N)), "g_vectors": desc((B, N, H, M, 3))}
+    up.update(up_over)
+    shapes = {"q_direction": (B, N, H, 3), "k_direction": (B, N, H, 3), "q_point": (B, N, H, 3),
+              "k_point": (B, N, H, 3), "values": (B, N, H, M, 3), "direction_scale": (H,),
+              "distance_scale": (H,), "output_weight": (H * M * 3, Cout), "output_bias": (Cout,),
+              "rotation": (B, N, 3, 3), "translation": (B, N, 3)}
+    gd = {k: desc(s) for k, s in shapes.items()}
+    gd.update(grads_over or {})
+    grads = api.GeoGrads(*[gd[k] for k in api.GEO_GRADS])
+    if ws_bytes is None:
+        ws_bytes = lib.geo_attn_bwd_workspace_size(ctypes.byref(p))
+    return lib.geo_attn_bwd(ctypes.byref(p), *[ctypes.byref(ds[k]) if ds[k] is not None else None
+                                               for k in api.GEO_INPUTS],
+                            *[ctypes.byref(up[k]) if up[k] is not None else None
+                              for k in ("g_output", "g_attention", "g_vectors")],
+                            ctypes.byref(grads), ctypes.c_void_p(FAKE), ctypes.c_size_t(ws_bytes),
+                            ctypes.c_void_p(FAKE))
+
+
+def test_geo_bwd_workspace_grows_with_the_problem_and_is_zero_outside_envelope():
+    lib = api.library()
+    small = lib.geo_attn_bwd_workspace_size(ctypes.byref(api.GeoParams(1, 256, 8, 4, 256)))
+    big = lib.geo_attn_bwd_workspace_size(ctypes.byref(api.GeoParams(2, 2048, 8, 4, 256)))
+    assert 0 < small < big
+    assert big > lib.geo_attn_workspace_size(ctypes.byref(api.GeoParams(2, 2048, 8, 4, 256)))
+    assert lib.geo_attn_bwd_workspace_size(ctypes.byref(api.GeoParams(1, 64, 40, 4, 8))) == 0
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("g_output_shape", 2), ("g_att_dtype", 4), ("grad_noncontig", 3), ("bias_grad_missing", 1),
+    ("bias_grad_without_bias", 2), ("workspace", 5), ("input_shape", 2),
+])
+def test_geo_bwd_rejects_bad_arguments_before_launch(case, expect):
+    p, ds = geo_args()
+    grads_over, up, ws = {}, {}, None
+    if case == "g_output_shape":
+        up["g_output"] = desc((1, 32, 7))
+    elif case == "g_att_dtype":
+        up["g_attention"] = desc((1, 2, 32, 32), api.IPA_DTYPE_F64)
+    elif case == "grad_noncontig":
+        grads_over["values"] = desc((1, 32, 2, 2, 3), strides=(384, 12, 6, 1, 2))
+    elif case == "bias_grad_missing":
+        grads_over["output_bias"] = desc((8,), ptr=None)
+    elif case == "bias_grad_without_bias":
+        ds["output_bias"] = desc((8,), ptr=None)
+    elif case == "workspace":
+        ws = 4096
+    elif case == "input_shape":
+        ds["translation"] = desc((1, 32, 4))
+    assert geo_bwd_call(p, ds, grads_over, ws, **up) == expect
+
