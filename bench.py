@@ -420,6 +420,32 @@ def main():
             "attention_map_GBps": att_bytes / ((res[True] - res[False]) / 1e3) / 1e9
             if res[True] > res[False] else None,
         }
+        # gradients of the variant (forward statistics recomputed inside the call)
+        from rna_structure_models_b200.synth import geo_upstream
+        ug = {k: (torch.from_numpy(v).to(dev) if v is not None else None)
+              for k, v in geo_upstream(g["dims"], 1).items()}
+        gg = api.GeoGradPlan(2, 2048, 8, 4, 256, device=dev)
+        gout = {n: torch.empty(tuple(gd[n].shape), device=dev) for n in api.GEO_GRADS}
+        bres = {}
+        for with_ga in (False, True):
+            ga = ug["g_attention"] if with_ga else None
+            for _ in range(3):
+                gg(gd, ug["g_output"], ga, ug["g_vectors"], out=gout)
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(10):
+                flush.zero_()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record()
+                gg(gd, ug["g_output"], ga, ug["g_vectors"], out=gout)
+                a1.record()
+                torch.cuda.synchronize()
+                times.append(a0.elapsed_time(a1))
+            bres[with_ga] = statistics.mean(times)
+        line["variant"].update({
+            "backward_ms": bres[False], "backward_ms_with_attention_grad": bres[True],
+            "backward_pair_heads_per_s": pairs / (bres[False] / 1e3),
+        })
 
     # distance-aware attention of MEET (§2.2) on the same core (B=1, L=4096, H=8)
     if not args.no_variant and rank == 0:

@@ -18,7 +18,9 @@
 //   0. the forward statistics (scales, rotated inputs, row max / sum, agg)
 //   1. geo_gvec_kernel     -- per (b, n): g_vec and whether any head is live
 //   2. geo_dagg_kernel     -- per (b, n, h): dagg = R g_vec, <dagg, agg>
-//   3. geo_dw_kernel       -- dW = vec^T g_output, db = sum g_output (live rows)
+//   3. geo_dw_part_kernel / geo_dw_sum_kernel -- dW = vec^T g_output and
+//                             db = sum g_output over live rows, per 128-row
+//                             chunk, then summed in a fixed order
 //   4. geo_bwd_rows_kernel -- per (b, h, 128 queries) x 4 key splits: D_i,
 //                             then d qd, d qp and the per-head sums of
 //                             ds <qd, kd> and ds |qp - kp|
@@ -74,16 +76,22 @@ __global__ void __launch_bounds__(256) geo_gvec_kernel(const GvecArgs a) {
   }
   if (kx >= a.HM3) return;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int64_t go[4];   // g_output offset of each row (its live rows only)
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int64_t row = row0 + q;
+    go[q] = -1;
+    if (row < rows && lv[q]) {
+      const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
+      go[q] = b * a.g_output.s[0] + n * a.g_output.s[1];
+    }
+  }
+  const int64_t sc = a.g_output.s[2];
   for (int c = 0; c < a.Cout; ++c) {
     const float w = a.wt[static_cast<int64_t>(c) * a.HM3 + kx];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int64_t row = row0 + q;
-      if (row < rows && lv[q]) {
-        const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
-        acc[q] = fmaf(ldf(a.g_output, b * a.g_output.s[0] + n * a.g_output.s[1] + c * a.g_output.s[2]), w, acc[q]);
-      }
-    }
+    for (int q = 0; q < 4; ++q)
+      if (go[q] >= 0) acc[q] = fmaf(ldf(a.g_output, go[q] + c * sc), w, acc[q]);
   }
   const int h = kx / (a.HM3 / a.H), mx = kx % (a.HM3 / a.H), m = mx / 3, x = mx % 3;
 #pragma unroll
@@ -132,32 +140,76 @@ __global__ void __launch_bounds__(256) geo_dagg_kernel(const DaggArgs a) {
   a.rowinfo[row] = make_float4(0.f, 0.f, d1, 0.f);
 }
 
+constexpr int DW_ROWS = 128, DW_K = 32;
+
 struct DwArgs {
   int64_t rows;
-  int HM3, Cout;
+  int HM3, Cout, N, nchunk;
   View g_output;
-  int N;
   const float* vec;                // [rows, HM3]
   const unsigned char* rowlive;    // [rows]
+  float* part_w;                   // [nchunk, HM3, Cout]
+  float* part_b;                   // [nchunk, Cout]
   float* d_w;                      // [HM3, Cout]
   float* d_b;                      // [Cout] or null
 };
 
-// One thread per (k, c): a deterministic sum over all rows.
-__global__ void __launch_bounds__(256) geo_dw_kernel(const DwArgs a) {
+// Partial dW over one chunk of 128 rows: a thread owns one output column c
+// and 32 rows k of W; the chunk's vec values sit in shared memory.
+__global__ void __launch_bounds__(256) geo_dw_part_kernel(const DwArgs a) {
+  __shared__ float vs[DW_ROWS][DW_K];
+  __shared__ int64_t goff[DW_ROWS];   // g_output offset of each row, -1 if it passes nothing on
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  const int k = blockIdx.y;
-  if (c >= a.Cout) return;
-  float acc = 0.f, accb = 0.f;
-  for (int64_t row = 0; row < a.rows; ++row) {
-    if (!a.rowlive[row]) continue;
-    const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
-    const float g = ldf(a.g_output, b * a.g_output.s[0] + n * a.g_output.s[1] + c * a.g_output.s[2]);
-    acc = fmaf(a.vec[row * a.HM3 + k], g, acc);
-    accb += g;
+  const int k0 = blockIdx.y * DW_K;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.z) * DW_ROWS;
+  for (int e = threadIdx.x; e < DW_ROWS * DW_K; e += blockDim.x) {
+    const int rr = e / DW_K, kk = e % DW_K;
+    const int64_t row = r0 + rr;
+    vs[rr][kk] = (row < a.rows && k0 + kk < a.HM3) ? a.vec[row * a.HM3 + k0 + kk] : 0.f;
   }
-  a.d_w[static_cast<int64_t>(k) * a.Cout + c] = acc;
-  if (k == 0 && a.d_b) a.d_b[c] = accb;
+  for (int rr = threadIdx.x; rr < DW_ROWS; rr += blockDim.x) {
+    const int64_t row = r0 + rr;
+    int64_t off = -1;
+    if (row < a.rows && a.rowlive[row]) {
+      const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
+      off = b * a.g_output.s[0] + n * a.g_output.s[1];
+    }
+    goff[rr] = off;
+  }
+  __syncthreads();
+  if (c >= a.Cout) return;
+  float acc[DW_K], accb = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < DW_K; ++kk) acc[kk] = 0.f;
+  const int64_t sc = static_cast<int64_t>(c) * a.g_output.s[2];
+  for (int rr = 0; rr < DW_ROWS; ++rr) {
+    if (goff[rr] < 0) continue;
+    const float g = ldf(a.g_output, goff[rr] + sc);
+    accb += g;
+#pragma unroll
+    for (int kk = 0; kk < DW_K; ++kk) acc[kk] = fmaf(vs[rr][kk], g, acc[kk]);
+  }
+  float* pw = a.part_w + static_cast<int64_t>(blockIdx.z) * a.HM3 * a.Cout;
+#pragma unroll
+  for (int kk = 0; kk < DW_K; ++kk)
+    if (k0 + kk < a.HM3) pw[static_cast<int64_t>(k0 + kk) * a.Cout + c] = acc[kk];
+  if (blockIdx.y == 0) a.part_b[static_cast<int64_t>(blockIdx.z) * a.Cout + c] = accb;
+}
+
+// dW and db: the chunk partials summed in a fixed order (deterministic).
+__global__ void __launch_bounds__(256) geo_dw_sum_kernel(const DwArgs a) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nw = static_cast<int64_t>(a.HM3) * a.Cout;
+  if (t < nw) {
+    float s = 0.f;
+    for (int z = 0; z < a.nchunk; ++z) s += a.part_w[z * nw + t];
+    a.d_w[t] = s;
+  }
+  if (t < a.Cout && a.d_b) {
+    float s = 0.f;
+    for (int z = 0; z < a.nchunk; ++z) s += a.part_b[static_cast<int64_t>(z) * a.Cout + t];
+    a.d_b[t] = s;
+  }
 }
 
 struct PairArgs {
@@ -216,7 +268,7 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_rows_kernel(const 
   const unsigned char* pmrow =
       a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(in_range ? i : 0) * a.pms[2] : nullptr;
   const int nchunk = (N + BW_CHUNK - 1) / BW_CHUNK;
-  extern __shared__ float bw_merge[];   // [BW_SPLIT][8][BW_ROWS]
+  extern __shared__ float bw_merge[];   // [BW_SPLIT][8][BW_ROWS], then the staged keys
   auto sm_at = [&](int s2, int e) -> float& { return bw_merge[(s2 * 8 + e) * BW_ROWS + r]; };
 
   // D_i = <dagg_i, agg_i> + sum_j a_ij g_attention_ij
@@ -240,31 +292,53 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_rows_kernel(const 
   __syncthreads();
 
   float cq[3] = {0.f, 0.f, 0.f}, cp[3] = {0.f, 0.f, 0.f}, sdot = 0.f, sdist = 0.f;
-  if (live) {
-    for (int ch = split; ch < nchunk; ch += BW_SPLIT)
-      for (int k = 0; k < BW_CHUNK; ++k) {
-        const int j = ch * BW_CHUNK + k;
-        if (j >= N) break;
-        if (pmrow && !pmrow[static_cast<int64_t>(j) * a.pms[3]]) continue;
-        const float4 k0 = a.kg[2 * (bh * N + j)], k1 = a.kg[2 * (bh * N + j) + 1];
-        const GeoPair g = geo_pair(q0, q1, k0, k1, sc.x, sc.y);
-        const float p = ex2(g.s - m) * inv;
-        if (p == 0.f) continue;
-        const float* vr = a.vg + (bh * N + j) * a.VW;
-        float da = a.has_g_att ? g_att_at(a, b, h, i, j) : 0.f;
-#pragma unroll
-        for (int e = 0; e < V; ++e) da = fmaf(dg[e], vr[e], da);
-        const float ds = p * (da - D);
-        cq[0] = fmaf(ds, k0.x, cq[0]);
-        cq[1] = fmaf(ds, k0.y, cq[1]);
-        cq[2] = fmaf(ds, k0.z, cq[2]);
-        const float ru = g.dist > 0.f ? ds / g.dist : 0.f;   // zero displacement: zero derivative
-        cp[0] = fmaf(ru, g.dx, cp[0]);
-        cp[1] = fmaf(ru, g.dy, cp[1]);
-        cp[2] = fmaf(ru, g.dz, cp[2]);
-        sdot = fmaf(ds, g.dot, sdot);
-        sdist = fmaf(ds, g.dist, sdist);
+  // keys of one 32-key chunk staged per split group: [k0 | k1 | vr (padded)]
+  constexpr int SW = 8 + ((V + 3) & ~3);
+  float* stg = bw_merge + BW_SPLIT * 8 * BW_ROWS + split * BW_CHUNK * SW;
+  const uint32_t gbar = 1 + split;
+  for (int ch = split; ch < nchunk; ch += BW_SPLIT) {
+    const int j0 = ch * BW_CHUNK;
+    named_bar_sync(gbar, BW_ROWS);                 // the previous chunk has been read
+    for (int e = r; e < BW_CHUNK * SW; e += BW_ROWS) {
+      const int it = e / SW, f = e % SW, j = j0 + it;
+      float v = 0.f;
+      if (j < N) {
+        if (f < 8) v = reinterpret_cast<const float*>(a.kg)[8 * (bh * N + j) + f];
+        else if (f - 8 < V) v = a.vg[(bh * N + j) * a.VW + (f - 8)];
+      } else if (f == 3) {
+        v = -INFINITY;                             // beyond N: never allowed
       }
+      stg[e] = v;
+    }
+    named_bar_sync(gbar, BW_ROWS);
+    if (!live) continue;
+    uint32_t allowed = 0xffffffffu;
+    if (pmrow) {
+      allowed = 0u;
+      const unsigned char* pr = pmrow + static_cast<int64_t>(j0) * a.pms[3];
+      for (int k = 0; k < BW_CHUNK && j0 + k < N; ++k) allowed |= pr[k * a.pms[3]] ? (1u << k) : 0u;
+    }
+    for (int k = 0; k < BW_CHUNK; ++k) {
+      if (!((allowed >> k) & 1u)) continue;
+      const float* kk = stg + k * SW;
+      const float4 k0 = *reinterpret_cast<const float4*>(kk), k1 = *reinterpret_cast<const float4*>(kk + 4);
+      const GeoPair g = geo_pair(q0, q1, k0, k1, sc.x, sc.y);
+      const float p = ex2(g.s - m) * inv;
+      if (p == 0.f) continue;
+      float da = a.has_g_att && j0 + k < N ? g_att_at(a, b, h, i, j0 + k) : 0.f;
+#pragma unroll
+      for (int e = 0; e < V; ++e) da = fmaf(dg[e], kk[8 + e], da);
+      const float ds = p * (da - D);
+      cq[0] = fmaf(ds, k0.x, cq[0]);
+      cq[1] = fmaf(ds, k0.y, cq[1]);
+      cq[2] = fmaf(ds, k0.z, cq[2]);
+      const float ru = g.dist > 0.f ? __fdividef(ds, g.dist) : 0.f;   // zero displacement: zero derivative
+      cp[0] = fmaf(ru, g.dx, cp[0]);
+      cp[1] = fmaf(ru, g.dy, cp[1]);
+      cp[2] = fmaf(ru, g.dz, cp[2]);
+      sdot = fmaf(ds, g.dot, sdot);
+      sdist = fmaf(ds, g.dist, sdist);
+    }
   }
   sm_at(split, 0) = cq[0]; sm_at(split, 1) = cq[1]; sm_at(split, 2) = cq[2];
   sm_at(split, 3) = cp[0]; sm_at(split, 4) = cp[1]; sm_at(split, 5) = cp[2];
@@ -324,39 +398,53 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_cols_kernel(const 
   const unsigned char* pmcol =
       a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(in_range ? j : 0) * a.pms[3] : nullptr;
   const int nchunk = (N + BW_CHUNK - 1) / BW_CHUNK;
-  if (in_range && k0.w == 0.f) {
-    for (int ch = split; ch < nchunk; ch += BW_SPLIT)
-      for (int k = 0; k < BW_CHUNK; ++k) {
-        const int i = ch * BW_CHUNK + k;
-        if (i >= N) break;
-        const float4 info = a.rowinfo[bh * N + i];     // same i across the warp: one broadcast load
-        if (info.y == 0.f) continue;                   // query without an allowed key
-        if (pmcol && !pmcol[static_cast<int64_t>(i) * a.pms[2]]) continue;
-        const float4 q0 = a.qg[2 * (bh * N + i)], q1 = a.qg[2 * (bh * N + i) + 1];
-        const GeoPair g = geo_pair(q0, q1, k0, k1, sc.x, sc.y);
-        const float p = ex2(g.s - info.x) * info.y;
-        if (p == 0.f) continue;
-        const float* dg = a.dagg + (bh * N + i) * a.VW;
-        float da = a.has_g_att ? g_att_at(a, b, h, i, j) : 0.f;
-        float dgv[V];
-#pragma unroll
-        for (int e = 0; e < V; ++e) {
-          dgv[e] = dg[e];
-          da = fmaf(dgv[e], vr[e], da);
-        }
-        const float ds = p * (da - info.z);
-        ck[0] = fmaf(ds, q0.x, ck[0]);
-        ck[1] = fmaf(ds, q0.y, ck[1]);
-        ck[2] = fmaf(ds, q0.z, ck[2]);
-        const float ru = g.dist > 0.f ? ds / g.dist : 0.f;
-        cp[0] = fmaf(ru, g.dx, cp[0]);
-        cp[1] = fmaf(ru, g.dy, cp[1]);
-        cp[2] = fmaf(ru, g.dz, cp[2]);
-#pragma unroll
-        for (int e = 0; e < V; ++e) dv[e] = fmaf(p, dgv[e], dv[e]);
+  const bool active = in_range && k0.w == 0.f;
+  extern __shared__ float bw_merge[];   // [BW_SPLIT][6 + V][BW_ROWS], then the staged queries
+  // queries of one 32-query chunk staged per split group: [rowinfo | q0 | q1 | dagg (padded)]
+  constexpr int SW = 12 + ((V + 3) & ~3);
+  float* stg = bw_merge + BW_SPLIT * (6 + V) * BW_ROWS + split * BW_CHUNK * SW;
+  const uint32_t gbar = 1 + split;
+  for (int ch = split; ch < nchunk; ch += BW_SPLIT) {
+    const int i0 = ch * BW_CHUNK;
+    named_bar_sync(gbar, BW_ROWS);
+    for (int e = r; e < BW_CHUNK * SW; e += BW_ROWS) {
+      const int it = e / SW, f = e % SW, i = i0 + it;
+      float v = 0.f;
+      if (i < N) {
+        if (f < 4) v = reinterpret_cast<const float*>(a.rowinfo)[4 * (bh * N + i) + f];
+        else if (f < 12) v = reinterpret_cast<const float*>(a.qg)[8 * (bh * N + i) + (f - 4)];
+        else if (f - 12 < V) v = a.dagg[(bh * N + i) * a.VW + (f - 12)];
       }
+      stg[e] = v;                                  // beyond N: rowinfo.y = 0, skipped
+    }
+    named_bar_sync(gbar, BW_ROWS);
+    if (!active) continue;
+    for (int k = 0; k < BW_CHUNK; ++k) {
+      const float* qq = stg + k * SW;
+      const float4 info = *reinterpret_cast<const float4*>(qq);
+      if (info.y == 0.f) continue;                 // query without an allowed key
+      const int i = i0 + k;
+      if (pmcol && !pmcol[static_cast<int64_t>(i) * a.pms[2]]) continue;
+      const float4 q0 = *reinterpret_cast<const float4*>(qq + 4), q1 = *reinterpret_cast<const float4*>(qq + 8);
+      const GeoPair g = geo_pair(q0, q1, k0, k1, sc.x, sc.y);
+      const float p = ex2(g.s - info.x) * info.y;
+      if (p == 0.f) continue;
+      float da = a.has_g_att ? g_att_at(a, b, h, i, j) : 0.f;
+#pragma unroll
+      for (int e = 0; e < V; ++e) da = fmaf(qq[12 + e], vr[e], da);
+      const float ds = p * (da - info.z);
+      ck[0] = fmaf(ds, q0.x, ck[0]);
+      ck[1] = fmaf(ds, q0.y, ck[1]);
+      ck[2] = fmaf(ds, q0.z, ck[2]);
+      const float ru = g.dist > 0.f ? __fdividef(ds, g.dist) : 0.f;
+      cp[0] = fmaf(ru, g.dx, cp[0]);
+      cp[1] = fmaf(ru, g.dy, cp[1]);
+      cp[2] = fmaf(ru, g.dz, cp[2]);
+#pragma unroll
+      for (int e = 0; e < V; ++e) dv[e] = fmaf(p, qq[12 + e], dv[e]);
+    }
   }
-  extern __shared__ float bw_merge[];   // [BW_SPLIT][6 + V][BW_ROWS]
+  __syncthreads();
   auto sm_at = [&](int s2, int e) -> float& { return bw_merge[(s2 * (6 + V) + e) * BW_ROWS + r]; };
 #pragma unroll
   for (int e = 0; e < 3; ++e) {
@@ -469,8 +557,14 @@ __global__ void geo_wt_kernel(const TransposeArgs a) {
 template <int M>
 cudaError_t launch_pairs(const PairArgs& p, int B, int N, int H, cudaStream_t st) {
   dim3 grid((N + BW_ROWS - 1) / BW_ROWS, H, B);
-  const size_t smem_r = sizeof(float) * BW_SPLIT * 8 * BW_ROWS;
-  const size_t smem_c = sizeof(float) * BW_SPLIT * (6 + 3 * M) * BW_ROWS;
+  constexpr int V4 = (3 * M + 3) & ~3;
+  const size_t smem_r = sizeof(float) * BW_SPLIT * (8 * BW_ROWS + BW_CHUNK * (8 + V4));
+  const size_t smem_c = sizeof(float) * BW_SPLIT * ((6 + 3 * M) * BW_ROWS + BW_CHUNK * (12 + V4));
+  if (smem_r > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(geo_bwd_rows_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_r));
+    if (e != cudaSuccess) return e;
+  }
   if (smem_c > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(geo_bwd_cols_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_c));
@@ -501,6 +595,9 @@ GeoBwdWorkspace geo_bwd_workspace_layout(int B, int N, int H, int M, int Cout) {
   w.dvr = o; o = up(o + bhn * VW * 4);
   w.acc = o; o = up(o + static_cast<size_t>(H) * 8);
   w.wt = o; o = up(o + HM3 * static_cast<size_t>(Cout) * 4);
+  const size_t nchunk = (bn + 127) / 128;
+  w.dwpart = o; o = up(o + nchunk * HM3 * static_cast<size_t>(Cout) * 4);
+  w.dbpart = o; o = up(o + nchunk * static_cast<size_t>(Cout) * 4);
   w.total = o;
   return w;
 }
@@ -550,8 +647,16 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
 
   DwArgs dw{};
   dw.rows = rows; dw.HM3 = HM3; dw.Cout = Cout; dw.g_output = a.g_output; dw.N = N;
-  dw.vec = f.out_vectors; dw.rowlive = ga.rowlive; dw.d_w = a.d_output_weight; dw.d_b = a.d_output_bias;
-  geo_dw_kernel<<<dim3((Cout + 255) / 256, HM3), 256, 0, st>>>(dw);
+  dw.nchunk = static_cast<int>((rows + DW_ROWS - 1) / DW_ROWS);
+  dw.vec = f.out_vectors; dw.rowlive = ga.rowlive;
+  dw.part_w = reinterpret_cast<float*>(ws + w.dwpart);
+  dw.part_b = reinterpret_cast<float*>(ws + w.dbpart);
+  dw.d_w = a.d_output_weight; dw.d_b = a.d_output_bias;
+  geo_dw_part_kernel<<<dim3((Cout + 255) / 256, (HM3 + DW_K - 1) / DW_K, dw.nchunk), 256, 0, st>>>(dw);
+  {
+    int64_t n = static_cast<int64_t>(HM3) * Cout;
+    geo_dw_sum_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(dw);
+  }
 
   PairArgs p{};
   p.B = B; p.N = N; p.H = H; p.VW = VW;

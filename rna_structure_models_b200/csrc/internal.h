@@ -99,7 +99,7 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t stream);
 // forward part of the workspace, then the adjoint kernels run.
 struct GeoBwdWorkspace {
   GeoWorkspace fwd;   // offsets relative to the start of the gradient workspace
-  size_t vec, agg, gvec, rowlive, dagg, rowinfo, dq, dk, dvr, acc, wt, total;
+  size_t vec, agg, gvec, rowlive, dagg, rowinfo, dq, dk, dvr, acc, wt, dwpart, dbpart, total;
 };
 GeoBwdWorkspace geo_bwd_workspace_layout(int B, int N, int H, int M, int Cout);
 
