@@ -8,7 +8,8 @@
 //      converted to fp32.
 //   2. geo_prep_kernel    -- per (b, n, h): rotated directions, transformed
 //      points, R_j-rotated values (no translation), frame-mask bias.
-//   3. geo_attn_kernel<M> -- per (b, h, 128 queries) x 4 key splits: online
+//   3. geo_attn_kernel<M> -- per (b, h, 128 queries) x 4 key splits (each split
+//      group of four warps stages its 32-key chunk in shared memory): online
 //      masked softmax in the log2 domain and aggregation of the rotated
 //      values; splits merged through shared memory; R_i^T back-rotation.
 //   4. geo_map_kernel     -- optional: recomputes each score and writes the
@@ -162,9 +163,25 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT) geo_attn_kernel(const At
 #pragma unroll
   for (int e = 0; e < V; ++e) acc[e] = 0.f;
 
+  extern __shared__ float geo_merge[];  // [GEO_SPLIT][2 + V][GEO_ROWS], then the staged keys
+  // keys of one chunk staged per split group (four warps): [k0 | k1 | vr (padded)]
+  constexpr int SW = 8 + ((V + 3) & ~3);
+  float* stg = geo_merge + GEO_SPLIT * (2 + V) * GEO_ROWS + split * GEO_CHUNK * SW;
+  const uint32_t gbar = 1 + split;
   const int nchunk = (N + GEO_CHUNK - 1) / GEO_CHUNK;
   for (int ch = split; ch < nchunk; ch += GEO_SPLIT) {
     const int j0 = ch * GEO_CHUNK;
+    named_bar_sync(gbar, GEO_ROWS);              // the previous chunk has been read
+    for (int e = r; e < GEO_CHUNK * SW; e += GEO_ROWS) {
+      const int it = e / SW, f = e % SW, j = j0 + it;
+      float v = 0.f;
+      if (j < N) {
+        if (f < 8) v = reinterpret_cast<const float*>(a.kg)[8 * (bh * N + j) + f];
+        else if (f - 8 < V) v = a.vg[(bh * N + j) * a.VW + (f - 8)];
+      }
+      stg[e] = v;
+    }
+    named_bar_sync(gbar, GEO_ROWS);
     uint32_t allowed = 0xffffffffu;
     if (pmrow) {
       allowed = 0u;
@@ -186,8 +203,8 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT) geo_attn_kernel(const At
       const int j = j0 + k;
       float v = -INFINITY;
       if (j < N) {
-        const float4 k0 = a.kg[2 * (bh * N + j)];
-        const float4 k1 = a.kg[2 * (bh * N + j) + 1];
+        const float4 k0 = *reinterpret_cast<const float4*>(stg + k * SW);
+        const float4 k1 = *reinterpret_cast<const float4*>(stg + k * SW + 4);
         v = geo_score(q0, q1, k0, k1, sc.x, sc.y);
         if (!((allowed >> k) & 1u)) v = -INFINITY;
       }
@@ -208,14 +225,13 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT) geo_attn_kernel(const At
     for (int k = 0; k < GEO_CHUNK; ++k) {
       const float p = ex2(s[k] - m);
       l += p;
-      const float* vr = a.vg + (bh * N + j0 + k) * a.VW;
+      const float* vr = stg + k * SW + 8;
 #pragma unroll
       for (int e = 0; e < V; ++e) acc[e] = fmaf(p, vr[e], acc[e]);
     }
   }
 
   // merge the key splits
-  extern __shared__ float geo_merge[];  // [GEO_SPLIT][2 + V][GEO_ROWS]
   auto sm_at = [&](int s2, int e) -> float& { return geo_merge[(s2 * (2 + V) + e) * GEO_ROWS + r]; };
   sm_at(split, 0) = m;
   sm_at(split, 1) = l;
@@ -343,7 +359,7 @@ __global__ void __launch_bounds__(256) geo_readout_kernel(const ReadArgs a) {
 template <int M>
 cudaError_t launch_attn(const AttnArgs& t, int B, int N, int H, cudaStream_t st) {
   dim3 grid((N + GEO_ROWS - 1) / GEO_ROWS, H, B);
-  const size_t smem = sizeof(float) * GEO_SPLIT * (2 + 3 * M) * GEO_ROWS;
+  const size_t smem = sizeof(float) * GEO_SPLIT * ((2 + 3 * M) * GEO_ROWS + GEO_CHUNK * (8 + ((3 * M + 3) & ~3)));
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(geo_attn_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
