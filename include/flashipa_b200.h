@@ -332,6 +332,26 @@ IPA_API ipa_status_t ipa_frames_from_backbone(int32_t B, int32_t L,
                                       const ipa_tensor_t* rot_out, const ipa_tensor_t* trans_out,
                                       void* stream);
 
+/* --------------------------------------------------------------------------
+ * Dense projection y = x W + b on the tensor cores, the building block of the
+ * layer around the core (Flash Invariant Point Attention keeps the IPA layer's
+ * query / key / value / point projections of the single representation and
+ * its output projection; the factorised core sits between them).
+ *   x [M, K] IPA_DTYPE_F32, any strides; W [K, N] IPA_DTYPE_F32, any strides;
+ *   b [N] IPA_DTYPE_F32 contiguous, or NULL / data == NULL (no bias);
+ *   y [M, N] IPA_DTYPE_F32 contiguous (written).
+ * x and W are rounded to fp16 (into the workspace) and multiplied with fp32
+ * accumulation; the result is fp32.  Workspace: ipa_linear_workspace_size
+ * bytes, 256-byte aligned, caller-owned.  Envelope: 1 <= K <= 65536,
+ * M, N >= 1.  Errors as for ipa_attn_fwd; dev_err (optional) receives a
+ * device error code if a bounded wait expires.
+ * ------------------------------------------------------------------------ */
+IPA_API size_t ipa_linear_workspace_size(int32_t M, int32_t K, int32_t N);
+
+IPA_API ipa_status_t ipa_linear_fwd(int32_t M, int32_t K, int32_t N, const ipa_tensor_t* x,
+                            const ipa_tensor_t* w, const ipa_tensor_t* b, const ipa_tensor_t* y,
+                            void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err);
+
 /* Static description of a status code (never NULL). */
 IPA_API const char* ipa_status_string(ipa_status_t s);
 

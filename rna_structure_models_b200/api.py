@@ -24,7 +24,8 @@ STATUS = {0: "IPA_OK", 1: "IPA_ERR_NULL", 2: "IPA_ERR_SHAPE", 3: "IPA_ERR_STRIDE
 EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa_attn_core",
             "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static",
             "geo_attn_bwd_workspace_size", "geo_attn_bwd",
-            "meet_attn_workspace_size", "meet_attn_fwd", "ipa_frames_from_backbone", "ipa_status_string",
+            "meet_attn_workspace_size", "meet_attn_fwd", "ipa_frames_from_backbone", "ipa_linear_workspace_size",
+            "ipa_linear_fwd", "ipa_status_string",
             "ipa_device_error_status", "ipa_version")
 
 
@@ -105,6 +106,11 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.geo_attn_bwd.argtypes = [P(GeoParams)] + [T] * 16 + [P(GeoGrads), ctypes.c_void_p, ctypes.c_size_t,
                                                              ctypes.c_void_p]
     lib.geo_attn_bwd.restype = ctypes.c_int
+    lib.ipa_linear_workspace_size.argtypes = [ctypes.c_int32] * 3
+    lib.ipa_linear_workspace_size.restype = ctypes.c_size_t
+    lib.ipa_linear_fwd.argtypes = [ctypes.c_int32] * 3 + [T] * 4 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                                  ctypes.c_void_p, ctypes.c_void_p]
+    lib.ipa_linear_fwd.restype = ctypes.c_int
     lib.ipa_status_string.argtypes = [ctypes.c_int]
     lib.ipa_status_string.restype = ctypes.c_char_p
     lib.ipa_device_error_status.argtypes = [ctypes.c_int32]
@@ -515,3 +521,46 @@ def frames_from_backbone(n, ca, c, rot=None, trans=None, stream=None):
     if st != 0:
         raise IpaError(st, library().ipa_status_string(st).decode())
     return rot, trans
+
+
+# ------------------------------------------------------------------ projections
+class LinearPlan:
+    """y = x W + b on the tensor cores (fp16 operands, fp32 accumulation);
+    the plan owns the workspace for one (M, K, N)."""
+
+    def __init__(self, M: int, K: int, N: int, device="cuda"):
+        self.M, self.K, self.N = M, K, N
+        nbytes = int(library().ipa_linear_workspace_size(M, K, N))
+        if nbytes == 0:
+            raise IpaError(6, "dimensions outside the supported envelope")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def __call__(self, x, w, b=None, *, out=None, stream=None):
+        _require_cuda(x, w, b)
+        if out is None:
+            out = torch.empty((self.M, self.N), dtype=torch.float32, device=x.device)
+        descs = [tensor_desc(t) for t in (x, w, b, out)]
+        st = library().ipa_linear_fwd(self.M, self.K, self.N, *[ctypes.byref(d) for d in descs],
+                                      ctypes.c_void_p(self.workspace.data_ptr()),
+                                      ctypes.c_size_t(self.workspace.numel()),
+                                      ctypes.c_void_p(_stream_ptr(stream)),
+                                      ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return out
+
+    def check(self):
+        v = int(self.dev_err.item())
+        if v != 0:
+            self.dev_err.zero_()
+            raise IpaError(int(library().ipa_device_error_status(v)), f"device error code {v}")
+
+
+def linear(x, w, b=None, *, stream=None, check: bool = True):
+    """y = x W + b for x [M, K], W [K, N] (fp32 tensors on the GPU)."""
+    plan = LinearPlan(x.shape[0], x.shape[1], w.shape[1], device=x.device)
+    y = plan(x, w, b, stream=stream)
+    if check:
+        plan.check()
+    return y

@@ -493,6 +493,38 @@ ipa_status_t geo_attn_fwd(const geo_params_t* p, const ipa_tensor_t* q_direction
   return IPA_OK;
 }
 
+size_t ipa_linear_workspace_size(int32_t M, int32_t K, int32_t N) {
+  if (M < 1 || K < 1 || N < 1 || K > 65536 || M > (1 << 23)) return 0;
+  return linear_workspace_layout(M, K, N).total;
+}
+
+ipa_status_t ipa_linear_fwd(int32_t M, int32_t K, int32_t N, const ipa_tensor_t* x, const ipa_tensor_t* w,
+                            const ipa_tensor_t* b, const ipa_tensor_t* y, void* workspace,
+                            size_t workspace_bytes, void* stream, int32_t* dev_err) {
+  if (M < 1 || K < 1 || N < 1) return IPA_ERR_SHAPE;
+  if (K > 65536 || M > (1 << 23)) return IPA_ERR_UNSUPPORTED;
+  ipa_status_t st = IPA_OK;
+  const int64_t s_x[2] = {M, K}, s_w[2] = {K, N}, s_b[1] = {N}, s_y[2] = {M, N};
+  const bool has_b = b != nullptr && b->data != nullptr;
+  if (!check_tensor(x, IPA_DTYPE_F32, 2, s_x, &st) || !check_tensor(w, IPA_DTYPE_F32, 2, s_w, &st) ||
+      (has_b && !check_contiguous_out(b, 1, s_b, &st)) || !check_contiguous_out(y, 2, s_y, &st))
+    return st;
+  const LinearWorkspace lay = linear_workspace_layout(M, K, N);
+  if (workspace == nullptr) return IPA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
+  LinearLaunch a{};
+  a.M = M; a.K = K; a.N = N;
+  a.x = view_of(x); a.w = view_of(w);
+  a.bias = has_b ? static_cast<const float*>(b->data) : nullptr;
+  a.y = static_cast<float*>(const_cast<void*>(y->data));
+  a.ldy = N;
+  a.ws = static_cast<unsigned char*>(workspace);
+  a.lay = lay;
+  a.err = dev_err;
+  if (linear_launch(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
 size_t geo_attn_bwd_workspace_size(const geo_params_t* p) {
   ipa_status_t st = IPA_OK;
   if (!geo_dims_ok(p, &st)) return 0;

@@ -63,6 +63,24 @@ struct MeetPrep {
 cudaError_t meet_launch_prep(const MeetPrep& m, cudaStream_t stream);
 cudaError_t meet_launch_extract(const float* core_out, float* out, int64_t rows, cudaStream_t stream);
 
+// Dense projection y = x W + b (tcgen05, fp16 operands, fp32 accumulation).
+struct LinearWorkspace {
+  size_t x16, w16, total;
+};
+LinearWorkspace linear_workspace_layout(int M, int K, int N);
+
+struct LinearLaunch {
+  int M, K, N;
+  View x, w;            // [M, K], [K, N] fp32
+  const float* bias;    // [N] contiguous or null
+  float* y;             // [M, ldy] fp32
+  int64_t ldy;
+  unsigned char* ws;
+  LinearWorkspace lay;
+  int* err;
+};
+cudaError_t linear_launch(const LinearLaunch& a, cudaStream_t stream);
+
 // Residue frames from backbone atoms.
 struct FramesArgs {
   int B, L;

@@ -1,0 +1,260 @@
+// Dense projection y = x W + b on the tensor cores (tcgen05, fp16 operands,
+// fp32 accumulation in tensor memory).  The module around the IPA core uses it
+// for the q / k / v / point projections of the single representation and for
+// the output projection (Flash Invariant Point Attention keeps the IPA layer's
+// projections; the factorised core sits between them).
+//   linear_pack_x_kernel -- x (fp32, any row / column strides) -> fp16 [M, Kp],
+//                           K zero-padded to a multiple of 64
+//   linear_pack_w_kernel -- W [K, N] fp32 -> W^T fp16 [N, Kp] through a
+//                           shared-memory transpose
+//   linear_kernel        -- one CTA per 128 x 128 tile of y: a four-stage TMA
+//                           ring of 128 x 64 tiles of x and W^T, one thread
+//                           issuing tcgen05.mma (M = N = 128, K = 16), four
+//                           warps reading the accumulator back (+ b).
+// Every mbarrier wait is bounded; on expiry the CTA records an error code,
+// drains what it started, frees tensor memory and exits.
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fipa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int LBM = 128, LBN = 128, LBK = 64, LST = 4;
+constexpr uint32_t L_TILE = 16384;                 // 128 rows x 64 fp16
+constexpr uint32_t L_STAGE = 2 * L_TILE;           // x tile | W^T tile
+constexpr uint32_t L_AUX = LST * L_STAGE;
+constexpr uint32_t L_SMEM = L_AUX + 256;
+constexpr uint32_t L_ALLOC = L_SMEM + 1024;
+enum { LB_FULL0 = 0, LB_EMPTY0 = LST, LB_DONE = 2 * LST, LB_DRAIN, LB_COUNT };
+constexpr uint32_t L_TMEM_SLOT = 8 * LB_COUNT;
+constexpr uint32_t L_ABORT = L_TMEM_SLOT + 8;
+
+struct LinArgs {
+  int M, N, nk;
+  const float* bias;   // [N] or null
+  float* y;            // [M, ldy]
+  int64_t ldy;
+  int* err;
+};
+
+__device__ __forceinline__ uint64_t kmaj(uint32_t saddr) { return smem_desc_sw128(saddr, 16, 1024); }
+
+__global__ void __launch_bounds__(192, 1)
+    linear_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                  const LinArgs a) {
+  extern __shared__ unsigned char lin_smem_raw[];
+  const uint32_t raw = smem_u32(lin_smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  unsigned char* smem = lin_smem_raw + (sb - raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.y * LBM, n0 = blockIdx.x * LBN;
+  auto bar = [&](int k) -> uint32_t { return sb + L_AUX + 8u * k; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L_AUX + L_ABORT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L_AUX + L_TMEM_SLOT);
+
+  if (tid == 0) {
+    for (int s = 0; s < LST; ++s) {
+      mbar_init(bar(LB_FULL0 + s), 1);
+      mbar_init(bar(LB_EMPTY0 + s), 1);
+    }
+    mbar_init(bar(LB_DONE), 1);
+    mbar_init(bar(LB_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), LBN);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&](int code) {
+    record_error(a.err, code);
+    *abort_flag = 1;
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int kt = 0; kt < a.nk; ++kt) {
+        const int s = kt % LST;
+        if (kt >= LST && !mbar_wait_bounded(bar(LB_EMPTY0 + s), ((kt / LST) - 1) & 1, abort_flag)) {
+          fail(DEV_TIMEOUT_EMPTY);
+          break;
+        }
+        const uint32_t st = sb + s * L_STAGE;
+        mbar_arrive_expect_tx(bar(LB_FULL0 + s), L_STAGE);
+        tma_load_3d(st, &tm_x, bar(LB_FULL0 + s), kt * LBK, m0, 0);
+        tma_load_3d(st + L_TILE, &tm_w, bar(LB_FULL0 + s), kt * LBK, n0, 0);
+        issued = kt + 1;
+      }
+      if (*abort_flag)   // let the copies already started land before the CTA exits
+        for (int kt = (issued > LST ? issued - LST : 0); kt < issued; ++kt)
+          mbar_wait_bounded(bar(LB_FULL0 + kt % LST), (kt / LST) & 1, nullptr, 100000000ull);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(LBM, LBN, false);
+      bool ok = true, issued_any = false;
+      for (int kt = 0; kt < a.nk; ++kt) {
+        const int s = kt % LST;
+        if (!mbar_wait_bounded(bar(LB_FULL0 + s), (kt / LST) & 1, abort_flag)) {
+          fail(DEV_TIMEOUT_FULL);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = sb + s * L_STAGE;
+#pragma unroll
+        for (int k = 0; k < LBK / 16; ++k)
+          umma_ss(tmem, kmaj(st + 32 * k), kmaj(st + L_TILE + 32 * k), idesc, (kt > 0 || k > 0) ? 1u : 0u);
+        umma_commit(bar(LB_EMPTY0 + s));
+        issued_any = true;
+      }
+      if (ok) {
+        umma_commit(bar(LB_DONE));
+      } else if (issued_any) {
+        umma_commit(bar(LB_DRAIN));
+        mbar_wait_bounded(bar(LB_DRAIN), 0, nullptr, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue: rows m0 + 32 warp + lane
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(LB_DONE), 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      const int row = m0 + warp * 32 + lane;
+      const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+      float* yr = a.y + static_cast<int64_t>(row < a.M ? row : 0) * a.ldy;
+      for (int c0 = 0; c0 < LBN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + c0 + lane_off, v);
+        tmem_ld_wait();
+        const int col0 = n0 + c0;
+        if (row >= a.M || col0 >= a.N) continue;
+        if (col0 + 32 <= a.N && (a.ldy & 3) == 0) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float4 o = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                                   __uint_as_float(v[e + 3]));
+            if (a.bias) {
+              o.x += a.bias[col0 + e];
+              o.y += a.bias[col0 + e + 1];
+              o.z += a.bias[col0 + e + 2];
+              o.w += a.bias[col0 + e + 3];
+            }
+            *reinterpret_cast<float4*>(yr + col0 + e) = o;
+          }
+        } else {
+          for (int e = 0; e < 32 && col0 + e < a.N; ++e)
+            yr[col0 + e] = __uint_as_float(v[e]) + (a.bias ? a.bias[col0 + e] : 0.f);
+        }
+      }
+    } else if (lane == 0) {
+      fail(DEV_TIMEOUT_MMA);
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, LBN);
+  }
+}
+
+struct PackX {
+  int M, K, Kp;
+  View x;          // [M, K] fp32 (strides s[0], s[1])
+  __half* out;     // [M, Kp]
+};
+
+__global__ void linear_pack_x_kernel(const PackX a) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(a.M) * (a.Kp / 2);
+  if (t >= n) return;
+  const int m = static_cast<int>(t / (a.Kp / 2)), k = 2 * static_cast<int>(t % (a.Kp / 2));
+  const float* x = static_cast<const float*>(a.x.p) + m * a.x.s[0];
+  const float v0 = k < a.K ? x[k * a.x.s[1]] : 0.f, v1 = k + 1 < a.K ? x[(k + 1) * a.x.s[1]] : 0.f;
+  reinterpret_cast<__half2*>(a.out)[t] = __floats2half2_rn(v0, v1);
+}
+
+struct PackW {
+  int K, N, Kp;
+  View w;          // [K, N] fp32
+  __half* out;     // [N, Kp]
+};
+
+// 32 x 32 tiles: read along n (contiguous in W), write along k (contiguous in W^T)
+__global__ void __launch_bounds__(256) linear_pack_w_kernel(const PackW a) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
+  const float* w = static_cast<const float*>(a.w.p);
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int k = k0 + r, n = n0 + threadIdx.x;
+    tile[r][threadIdx.x] = (k < a.K && n < a.N) ? w[k * a.w.s[0] + n * a.w.s[1]] : 0.f;
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int n = n0 + r, k = k0 + threadIdx.x;
+    if (n < a.N && k < a.Kp) a.out[static_cast<int64_t>(n) * a.Kp + k] = __float2half_rn(tile[threadIdx.x][r]);
+  }
+}
+
+}  // namespace
+
+LinearWorkspace linear_workspace_layout(int M, int K, int N) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  LinearWorkspace w{};
+  const size_t Kp = (static_cast<size_t>(K) + 63) / 64 * 64;
+  size_t o = 0;
+  w.x16 = o; o = up(o + static_cast<size_t>(M) * Kp * 2);
+  w.w16 = o; o = up(o + static_cast<size_t>(N) * Kp * 2);
+  w.total = o;
+  return w;
+}
+
+cudaError_t linear_launch(const LinearLaunch& a, cudaStream_t st) {
+  const int Kp = (a.K + 63) / 64 * 64;
+  __half* x16 = reinterpret_cast<__half*>(a.ws + a.lay.x16);
+  __half* w16 = reinterpret_cast<__half*>(a.ws + a.lay.w16);
+  {
+    PackX p{a.M, a.K, Kp, a.x, x16};
+    const int64_t n = static_cast<int64_t>(a.M) * (Kp / 2);
+    linear_pack_x_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p);
+  }
+  {
+    PackW p{a.K, a.N, Kp, a.w, w16};
+    linear_pack_w_kernel<<<dim3(Kp / 32, (a.N + 31) / 32), dim3(32, 8), 0, st>>>(p);
+  }
+  CUtensorMap tx, tw;
+  if (!encode_tmap_f16_3d(&tx, x16, Kp, a.M, 1, static_cast<uint64_t>(Kp) * 2,
+                          static_cast<uint64_t>(Kp) * 2 * a.M, LBK, LBM) ||
+      !encode_tmap_f16_3d(&tw, w16, Kp, a.N, 1, static_cast<uint64_t>(Kp) * 2,
+                          static_cast<uint64_t>(Kp) * 2 * a.N, LBK, LBN))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L_ALLOC));
+  if (e != cudaSuccess) return e;
+  LinArgs la{a.M, a.N, Kp / LBK, a.bias, a.y, a.ldy, a.err};
+  linear_kernel<<<dim3((a.N + LBN - 1) / LBN, (a.M + LBM - 1) / LBM), 192, L_ALLOC, st>>>(tx, tw, la);
+  return cudaGetLastError();
+}
+
+}  // namespace fipa

@@ -321,3 +321,41 @@ def test_geo_bwd_rejects_bad_arguments_before_launch(case, expect):
         ds["translation"] = desc((1, 32, 4))
     assert geo_bwd_call(p, ds, grads_over, ws, **up) == expect
 
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("shape_w", 2), ("dtype_x", 4), ("y_noncontig", 3), ("bias_shape", 2), ("workspace", 5), ("big_k", 6),
+    ("zero_m", 2),
+])
+def test_linear_rejects_bad_arguments_before_launch(case, expect):
+    lib = api.library()
+    M, K, N = 200, 96, 70
+    ds = {"x": desc((M, K)), "w": desc((K, N)), "b": desc((N,)), "y": desc((M, N))}
+    ws = None
+    if case == "shape_w":
+        ds["w"] = desc((K + 1, N))
+    elif case == "dtype_x":
+        ds["x"] = desc((M, K), api.IPA_DTYPE_F64)
+    elif case == "y_noncontig":
+        ds["y"] = desc((M, N), strides=(1, M))
+    elif case == "bias_shape":
+        ds["b"] = desc((N + 1,))
+    elif case == "workspace":
+        ws = 512
+    elif case == "big_k":
+        K = 70000
+        ds["x"], ds["w"] = desc((M, K)), desc((K, N))
+        ws = 1 << 30
+    elif case == "zero_m":
+        M = 0
+    if ws is None:
+        ws = lib.ipa_linear_workspace_size(max(M, 1), K, N)
+    st = lib.ipa_linear_fwd(M, K, N, *[ctypes.byref(ds[k]) for k in ("x", "w", "b", "y")],
+                            ctypes.c_void_p(FAKE), ctypes.c_size_t(ws), None, None)
+    assert st == expect
+
+
+def test_linear_workspace_holds_both_fp16_operands():
+    lib = api.library()
+    assert lib.ipa_linear_workspace_size(4096, 384, 1152) >= 2 * (4096 + 1152) * 384
+    assert lib.ipa_linear_workspace_size(10, 70000, 10) == 0
