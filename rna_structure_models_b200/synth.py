@@ -249,6 +249,43 @@ def backbone_inputs(B: int, L: int, seed: int = 0, *, jitter: float = 0.0) -> di
     return {"n": f32(n), "ca": f32(ca), "c": f32(c), "rot": R, "trans": ca}
 
 
+@dataclass(frozen=True)
+class ModuleDims:
+    """IPA layer around the core: the core's dims plus the width c_s of the
+    single representation."""
+    B: int = 1
+    L: int = 512
+    H: int = 12
+    C: int = 16
+    Pq: int = 4
+    Pv: int = 8
+    R: int = 2
+    Cz: int = 128
+    c_s: int = 384
+
+
+def module_inputs(dims: ModuleDims, seed: int = 0, *, masked_tail_frac: float = 0.0, jitter: float = 0.0) -> dict:
+    """Seeded inputs of the IPA layer: the core's frames, pair factors,
+    w_bias, gamma and mask (as ipa_inputs draws them; its q / k / v / points
+    are dropped), then s ~ N(0, 1) [B, L, c_s], W_in ~ N(0, 1 / c_s)
+    [c_s, H (3 C + 3 (2 Pq + Pv))], b_in ~ N(0, 0.1^2), W_out ~ N(0, 1 / (H F))
+    [H F, c_s] with F = C + 4 Pv + Cz, b_out ~ N(0, 0.1^2), in that order."""
+    core = ipa_inputs(IpaDims(B=dims.B, L=dims.L, H=dims.H, C=dims.C, Pq=dims.Pq, Pv=dims.Pv, R=dims.R,
+                              Cz=dims.Cz), seed, masked_tail_frac=masked_tail_frac, jitter=jitter)
+    rng = np.random.Generator(np.random.PCG64(seed + 7919))
+    width = dims.H * (3 * dims.C + 3 * (2 * dims.Pq + dims.Pv))
+    F = dims.C + 4 * dims.Pv + dims.Cz
+    f32 = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    out = {k: core[k] for k in ("rot", "trans", "z1", "z2", "w_bias", "gamma", "mask")}
+    out["s"] = f32(rng.standard_normal((dims.B, dims.L, dims.c_s)))
+    out["w_in"] = f32(rng.standard_normal((dims.c_s, width)) / math.sqrt(dims.c_s))
+    out["b_in"] = f32(0.1 * rng.standard_normal(width))
+    out["w_out"] = f32(rng.standard_normal((dims.H * F, dims.c_s)) / math.sqrt(dims.H * F))
+    out["b_out"] = f32(0.1 * rng.standard_normal(dims.c_s))
+    out["dims"] = dims
+    return out
+
+
 # Named workloads.  Sizes follow the IPA module of AlphaFold-2-style models
 # (12 heads, 16 scalar channels, 4 query / 8 value points) with a rank-2
 # factorised pair representation of 128 channels.
