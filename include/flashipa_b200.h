@@ -352,6 +352,44 @@ IPA_API ipa_status_t ipa_linear_fwd(int32_t M, int32_t K, int32_t N, const ipa_t
                             const ipa_tensor_t* w, const ipa_tensor_t* b, const ipa_tensor_t* y,
                             void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err);
 
+/* --------------------------------------------------------------------------
+ * The IPA layer around the factorised core (Flash Invariant Point Attention
+ * keeps the IPA layer's projections; this library's reading of them):
+ *   Y = s W_in + b_in, s the single representation [B, L, c_s];
+ *   Y's columns, in order: q (H x C), k (H x C), v (H x C), q_pts (H x Pq x 3),
+ *   k_pts (H x Pq x 3), v_pts (H x Pv x 3), head-major, innermost the
+ *   channel (or the point, then xyz): width H (3 C + 3 (2 Pq + Pv));
+ *   o = ipa_attn_fwd on those (strided views of Y, no copy) with the frames,
+ *   z1, z2, w_bias, gamma and mask; F = C + 4 Pv + Cz features per head;
+ *   out = flatten(o) W_out + b_out  [B, L, c_s].
+ *   s      [B, L, c_s] IPA_DTYPE_F32, rows flattenable: stride(B) = L stride(L)
+ *   w_in   [c_s, width] IPA_DTYPE_F32; b_in [width] contiguous or NULL
+ *   w_out  [H F, c_s] IPA_DTYPE_F32;   b_out [c_s] contiguous or NULL
+ *   rot .. mask as for ipa_attn_fwd
+ *   out    [B, L, c_s] IPA_DTYPE_F32 contiguous
+ *   core_out [B, L, H, F] IPA_DTYPE_F32 contiguous, or NULL (then held in the
+ *          workspace)
+ * Projections run in fp16 with fp32 accumulation (ipa_linear_fwd), the core
+ * as ipa_attn_fwd.  Workspace: ipa_module_workspace_size bytes, 256-byte
+ * aligned.  Errors as for ipa_attn_fwd.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  ipa_params_t core;
+  int32_t c_s;
+} ipa_module_params_t;
+
+IPA_API size_t ipa_module_workspace_size(const ipa_module_params_t* p);
+
+IPA_API ipa_status_t ipa_module_fwd(const ipa_module_params_t* p, const ipa_tensor_t* s,
+                            const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                            const ipa_tensor_t* z1, const ipa_tensor_t* z2,
+                            const ipa_tensor_t* w_bias, const ipa_tensor_t* gamma,
+                            const ipa_tensor_t* mask, const ipa_tensor_t* w_in,
+                            const ipa_tensor_t* b_in, const ipa_tensor_t* w_out,
+                            const ipa_tensor_t* b_out, const ipa_tensor_t* out,
+                            const ipa_tensor_t* core_out, void* workspace, size_t workspace_bytes,
+                            void* stream, int32_t* dev_err);
+
 /* Static description of a status code (never NULL). */
 IPA_API const char* ipa_status_string(ipa_status_t s);
 

@@ -25,7 +25,7 @@ EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa
             "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static",
             "geo_attn_bwd_workspace_size", "geo_attn_bwd",
             "meet_attn_workspace_size", "meet_attn_fwd", "ipa_frames_from_backbone", "ipa_linear_workspace_size",
-            "ipa_linear_fwd", "ipa_status_string",
+            "ipa_linear_fwd", "ipa_module_workspace_size", "ipa_module_fwd", "ipa_status_string",
             "ipa_device_error_status", "ipa_version")
 
 
@@ -57,6 +57,10 @@ class GeoGrads(ctypes.Structure):
 class MeetParams(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("C", ctypes.c_int32)]
+
+
+class ModuleParams(ctypes.Structure):
+    _fields_ = [("core", IpaParams), ("c_s", ctypes.c_int32)]
 
 
 class IpaError(RuntimeError):
@@ -111,6 +115,11 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ipa_linear_fwd.argtypes = [ctypes.c_int32] * 3 + [T] * 4 + [ctypes.c_void_p, ctypes.c_size_t,
                                                                   ctypes.c_void_p, ctypes.c_void_p]
     lib.ipa_linear_fwd.restype = ctypes.c_int
+    lib.ipa_module_workspace_size.argtypes = [P(ModuleParams)]
+    lib.ipa_module_workspace_size.restype = ctypes.c_size_t
+    lib.ipa_module_fwd.argtypes = [P(ModuleParams)] + [T] * 14 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                                  ctypes.c_void_p, ctypes.c_void_p]
+    lib.ipa_module_fwd.restype = ctypes.c_int
     lib.ipa_status_string.argtypes = [ctypes.c_int]
     lib.ipa_status_string.restype = ctypes.c_char_p
     lib.ipa_device_error_status.argtypes = [ctypes.c_int32]
@@ -564,3 +573,61 @@ def linear(x, w, b=None, *, stream=None, check: bool = True):
     if check:
         plan.check()
     return y
+
+
+# ------------------------------------------------------------------ IPA layer
+MODULE_INPUTS = ("s", "rot", "trans", "z1", "z2", "w_bias", "gamma", "mask", "w_in", "b_in", "w_out", "b_out")
+
+
+class ModulePlan:
+    """The IPA layer around the core: input projection to q, k, v and the
+    local points, the fused core, output projection (one C-ABI call)."""
+
+    def __init__(self, B, L, H, C, Pq, Pv, R, Cz, c_s, device="cuda", **consts):
+        self.params = ModuleParams(ipa_params(B, L, H, C, Pq, Pv, R, Cz, **consts), c_s)
+        nbytes = int(library().ipa_module_workspace_size(ctypes.byref(self.params)))
+        if nbytes == 0:
+            raise IpaError(6, "dimensions outside the supported envelope")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.F = C + 4 * Pv + Cz
+
+    def __call__(self, inp: dict, *, out=None, core_out=None, stream=None):
+        p = self.params
+        _require_cuda(*[inp.get(n) for n in MODULE_INPUTS], core_out)
+        if out is None:
+            out = torch.empty((p.core.B, p.core.L, p.c_s), dtype=torch.float32, device=inp["s"].device)
+        descs = [tensor_desc(inp.get(n)) for n in MODULE_INPUTS] + [tensor_desc(out), tensor_desc(core_out)]
+        st = library().ipa_module_fwd(ctypes.byref(p), *[ctypes.byref(d) for d in descs],
+                                      ctypes.c_void_p(self.workspace.data_ptr()),
+                                      ctypes.c_size_t(self.workspace.numel()),
+                                      ctypes.c_void_p(_stream_ptr(stream)),
+                                      ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return out
+
+    def check(self):
+        v = int(self.dev_err.item())
+        if v != 0:
+            self.dev_err.zero_()
+            raise IpaError(int(library().ipa_device_error_status(v)), f"device error code {v}")
+
+
+def ipa_module(inp: dict, *, with_core: bool = False, stream=None, check: bool = True, **consts):
+    """IPA layer forward; with_core also returns the core output [B, L, H, F]."""
+    B, L, c_s = inp["s"].shape
+    H = inp["gamma"].shape[0]
+    z1 = inp["z1"]
+    R, Cz = z1.shape[2], z1.shape[3]
+    width = inp["w_in"].shape[1]
+    per_head = width // H                      # 3 C + 3 (2 Pq + Pv) with C = 16, Pq = 4, Pv = 8 supported
+    C, Pq, Pv = 16, 4, 8
+    if per_head != 3 * C + 3 * (2 * Pq + Pv):
+        raise IpaError(6, "the core supports C = 16, Pq = 4, Pv = 8")
+    plan = ModulePlan(B, L, H, C, Pq, Pv, R, Cz, c_s, device=inp["s"].device, **consts)
+    core = (torch.empty((B, L, H, plan.F), dtype=torch.float32, device=inp["s"].device) if with_core else None)
+    out = plan(inp, core_out=core, stream=stream)
+    if check:
+        plan.check()
+    return (out, core) if with_core else out

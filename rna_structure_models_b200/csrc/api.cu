@@ -525,6 +525,139 @@ ipa_status_t ipa_linear_fwd(int32_t M, int32_t K, int32_t N, const ipa_tensor_t*
   return IPA_OK;
 }
 
+namespace {
+
+struct ModuleLayout {
+  int64_t M, width, HF;
+  size_t y, o, lin, core, total;
+};
+
+bool module_layout(const ipa_module_params_t* p, ModuleLayout* m) {
+  if (p == nullptr || p->c_s < 1) return false;
+  const ipa_params_t& c = p->core;
+  const size_t core_ws = ipa_attn_workspace_size(&c);
+  if (core_ws == 0) return false;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  m->M = static_cast<int64_t>(c.B) * c.L;
+  m->width = static_cast<int64_t>(c.H) * (3 * c.C + 3 * (2 * c.Pq + c.Pv));
+  m->HF = static_cast<int64_t>(c.H) * (c.C + 4 * c.Pv + c.Cz);
+  if (m->M > (1 << 23) || p->c_s > 65536 || m->width > (1 << 20) || m->HF > 65536) return false;
+  const size_t lin_in = ipa_linear_workspace_size(static_cast<int32_t>(m->M), p->c_s, static_cast<int32_t>(m->width));
+  const size_t lin_out = ipa_linear_workspace_size(static_cast<int32_t>(m->M), static_cast<int32_t>(m->HF), p->c_s);
+  if (lin_in == 0 || lin_out == 0) return false;
+  size_t o = 0;
+  m->y = o; o = up(o + static_cast<size_t>(m->M) * m->width * 4);
+  m->o = o; o = up(o + static_cast<size_t>(m->M) * m->HF * 4);
+  m->lin = o; o = up(o + (lin_in > lin_out ? lin_in : lin_out));
+  m->core = o; o = up(o + core_ws);
+  m->total = o;
+  return true;
+}
+
+ipa_tensor_t dense_desc(const void* data, int ndim, const int64_t* size, const int64_t* stride) {
+  ipa_tensor_t t{};
+  t.data = data;
+  t.dtype = IPA_DTYPE_F32;
+  t.ndim = ndim;
+  for (int d = 0; d < ndim; ++d) {
+    t.size[d] = size[d];
+    t.stride[d] = stride[d];
+  }
+  return t;
+}
+
+}  // namespace
+
+size_t ipa_module_workspace_size(const ipa_module_params_t* p) {
+  ModuleLayout m{};
+  return module_layout(p, &m) ? m.total : 0;
+}
+
+ipa_status_t ipa_module_fwd(const ipa_module_params_t* p, const ipa_tensor_t* s, const ipa_tensor_t* rot,
+                            const ipa_tensor_t* trans, const ipa_tensor_t* z1, const ipa_tensor_t* z2,
+                            const ipa_tensor_t* w_bias, const ipa_tensor_t* gamma, const ipa_tensor_t* mask,
+                            const ipa_tensor_t* w_in, const ipa_tensor_t* b_in, const ipa_tensor_t* w_out,
+                            const ipa_tensor_t* b_out, const ipa_tensor_t* out, const ipa_tensor_t* core_out,
+                            void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err) {
+  if (p == nullptr) return IPA_ERR_NULL;
+  ipa_status_t st = IPA_OK;
+  if (!ipa_dims_ok(&p->core, &st)) return st;
+  if (p->c_s < 1) return IPA_ERR_SHAPE;
+  ModuleLayout m{};
+  if (!module_layout(p, &m)) return IPA_ERR_UNSUPPORTED;
+  const ipa_params_t& c = p->core;
+  const int64_t B = c.B, L = c.L, H = c.H, cs = p->c_s;
+  const int64_t F = c.C + 4 * c.Pv + c.Cz;
+  const int64_t s_s[3] = {B, L, cs}, s_wi[2] = {cs, m.width}, s_bi[1] = {m.width}, s_wo[2] = {m.HF, cs},
+                s_bo[1] = {cs}, s_o[4] = {B, L, H, F};
+  const bool has_bi = b_in != nullptr && b_in->data != nullptr;
+  const bool has_bo = b_out != nullptr && b_out->data != nullptr;
+  const bool has_co = core_out != nullptr && core_out->data != nullptr;
+  if (!check_tensor(s, IPA_DTYPE_F32, 3, s_s, &st) || !check_tensor(w_in, IPA_DTYPE_F32, 2, s_wi, &st) ||
+      (has_bi && !check_contiguous_out(b_in, 1, s_bi, &st)) || !check_tensor(w_out, IPA_DTYPE_F32, 2, s_wo, &st) ||
+      (has_bo && !check_contiguous_out(b_out, 1, s_bo, &st)) || !check_contiguous_out(out, 3, s_s, &st) ||
+      (has_co && !check_contiguous_out(core_out, 4, s_o, &st)))
+    return st;
+  if (B > 1 && s->stride[0] != L * s->stride[1]) return IPA_ERR_STRIDE_ALIGN;   // rows must flatten
+  {
+    // the core's own arguments, checked here too so that nothing is launched on a bad call
+    const int64_t s_rot[4] = {B, L, 3, 3}, s_tr[3] = {B, L, 3}, s_z[4] = {B, L, c.R, c.Cz},
+                  s_wb[2] = {c.Cz, H}, s_g[1] = {H}, s_m[2] = {B, L};
+    if (!check_tensor(rot, IPA_DTYPE_F32, 4, s_rot, &st) || !check_tensor(trans, IPA_DTYPE_F32, 3, s_tr, &st) ||
+        !check_tensor(z1, IPA_DTYPE_F32, 4, s_z, &st) || !check_tensor(z2, IPA_DTYPE_F32, 4, s_z, &st) ||
+        !check_tensor(w_bias, IPA_DTYPE_F32, 2, s_wb, &st) || !check_tensor(gamma, IPA_DTYPE_F32, 1, s_g, &st) ||
+        !check_tensor(mask, IPA_DTYPE_BOOL, 2, s_m, &st))
+      return st;
+  }
+  if (workspace == nullptr) return IPA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < m.total) return IPA_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  float* Y = reinterpret_cast<float*>(ws + m.y);
+  float* O = has_co ? static_cast<float*>(const_cast<void*>(core_out->data)) : reinterpret_cast<float*>(ws + m.o);
+
+  // 1. Y = s W_in + b_in
+  LinearLaunch l1{};
+  l1.M = static_cast<int>(m.M); l1.K = p->c_s; l1.N = static_cast<int>(m.width);
+  l1.x = view_of(s);
+  l1.x.s[0] = s->stride[1];      // [B*L, c_s] rows
+  l1.x.s[1] = s->stride[2];
+  l1.w = view_of(w_in);
+  l1.bias = has_bi ? static_cast<const float*>(b_in->data) : nullptr;
+  l1.y = Y; l1.ldy = m.width;
+  l1.ws = ws + m.lin; l1.lay = linear_workspace_layout(l1.M, l1.K, l1.N); l1.err = dev_err;
+  if (linear_launch(l1, strm) != cudaSuccess) return IPA_ERR_CUDA;
+
+  // 2. the core on strided views of Y
+  const int64_t rs = m.width;
+  const int64_t HC = H * c.C, HQ = H * c.Pq * 3;
+  const int64_t sz_s[4] = {B, L, H, c.C}, st_s[4] = {L * rs, rs, c.C, 1};
+  const int64_t sz_q[5] = {B, L, H, c.Pq, 3}, st_q[5] = {L * rs, rs, c.Pq * 3, 3, 1};
+  const int64_t sz_v[5] = {B, L, H, c.Pv, 3}, st_v[5] = {L * rs, rs, c.Pv * 3, 3, 1};
+  const ipa_tensor_t tq = dense_desc(Y, 4, sz_s, st_s), tk = dense_desc(Y + HC, 4, sz_s, st_s),
+                     tv = dense_desc(Y + 2 * HC, 4, sz_s, st_s), tqp = dense_desc(Y + 3 * HC, 5, sz_q, st_q),
+                     tkp = dense_desc(Y + 3 * HC + HQ, 5, sz_q, st_q),
+                     tvp = dense_desc(Y + 3 * HC + 2 * HQ, 5, sz_v, st_v);
+  const int64_t st_o[4] = {L * H * F, H * F, F, 1};
+  const ipa_tensor_t to = dense_desc(O, 4, s_o, st_o);
+  st = ipa_attn_fwd(&c, &tq, &tk, &tv, &tqp, &tkp, &tvp, rot, trans, z1, z2, w_bias, gamma, mask, &to,
+                    ws + m.core, workspace_bytes - m.core, stream, dev_err);
+  if (st != IPA_OK) return st;
+
+  // 3. out = flatten(o) W_out + b_out
+  LinearLaunch l2{};
+  l2.M = static_cast<int>(m.M); l2.K = static_cast<int>(m.HF); l2.N = p->c_s;
+  const int64_t sz_o2[2] = {m.M, m.HF}, st_o2[2] = {m.HF, 1};
+  const ipa_tensor_t to2 = dense_desc(O, 2, sz_o2, st_o2);
+  l2.x = view_of(&to2);
+  l2.w = view_of(w_out);
+  l2.bias = has_bo ? static_cast<const float*>(b_out->data) : nullptr;
+  l2.y = static_cast<float*>(const_cast<void*>(out->data)); l2.ldy = cs;
+  l2.ws = ws + m.lin; l2.lay = linear_workspace_layout(l2.M, l2.K, l2.N); l2.err = dev_err;
+  if (linear_launch(l2, strm) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
 size_t geo_attn_bwd_workspace_size(const geo_params_t* p) {
   ipa_status_t st = IPA_OK;
   if (!geo_dims_ok(p, &st)) return 0;

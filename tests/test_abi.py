@@ -359,3 +359,46 @@ def test_linear_workspace_holds_both_fp16_operands():
     lib = api.library()
     assert lib.ipa_linear_workspace_size(4096, 384, 1152) >= 2 * (4096 + 1152) * 384
     assert lib.ipa_linear_workspace_size(10, 70000, 10) == 0
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("s_rows_not_flat", 3), ("w_in_shape", 2), ("out_noncontig", 3), ("workspace", 5), ("core_C", 6),
+    ("c_s_zero", 2), ("core_out_shape", 2), ("rot_shape", 2), ("mask_dtype", 4),
+])
+def test_module_rejects_bad_arguments_before_launch(case, expect):
+    lib = api.library()
+    B, L, H, Cz, cs = 2, 64, 3, 32, 40
+    C, Pq, Pv, R = 16, 4, 8, 2
+    width, F = H * (3 * C + 3 * (2 * Pq + Pv)), C + 4 * Pv + Cz
+    p = api.ModuleParams(api.ipa_params(B, L, H, C, Pq, Pv, R, Cz), cs)
+    ds = {"s": desc((B, L, cs)), "rot": desc((B, L, 3, 3)), "trans": desc((B, L, 3)), "z1": desc((B, L, R, Cz)),
+          "z2": desc((B, L, R, Cz)), "w_bias": desc((Cz, H)), "gamma": desc((H,)),
+          "mask": desc((B, L), api.IPA_DTYPE_BOOL), "w_in": desc((cs, width)), "b_in": desc((width,)),
+          "w_out": desc((H * F, cs)), "b_out": desc((cs,)), "out": desc((B, L, cs)), "core_out": None}
+    ws = None
+    if case == "s_rows_not_flat":
+        ds["s"] = desc((B, L, cs), strides=(L * cs + 8, cs, 1))
+    elif case == "w_in_shape":
+        ds["w_in"] = desc((cs, width + 1))
+    elif case == "out_noncontig":
+        ds["out"] = desc((B, L, cs), strides=(L * cs, 1, L))
+    elif case == "workspace":
+        ws = 1 << 10
+    elif case == "core_C":
+        p = api.ModuleParams(api.ipa_params(B, L, H, 32, Pq, Pv, R, Cz), cs)
+        ws = 1 << 30
+    elif case == "c_s_zero":
+        p = api.ModuleParams(api.ipa_params(B, L, H, C, Pq, Pv, R, Cz), 0)
+        ws = 1 << 30
+    elif case == "core_out_shape":
+        ds["core_out"] = desc((B, L, H, F + 1))
+    elif case == "rot_shape":
+        ds["rot"] = desc((B, L, 3, 4))
+    elif case == "mask_dtype":
+        ds["mask"] = desc((B, L))
+    if ws is None:
+        ws = lib.ipa_module_workspace_size(ctypes.byref(p))
+    order = api.MODULE_INPUTS + ("out", "core_out")
+    st = lib.ipa_module_fwd(ctypes.byref(p), *[ctypes.byref(ds[k]) if ds[k] is not None else None for k in order],
+                            ctypes.c_void_p(FAKE), ctypes.c_size_t(ws), None, None)
+    assert st == expect
