@@ -475,6 +475,51 @@ def main():
             "tflops_algorithmic": triples * 2 * (2 * 16 + 9) / (ms_meet / 1e3) / 1e12,
         }
 
+    # the IPA layer around the core (projections + core), same sizes, c_s = 384
+    if not args.no_variant and rank == 0:
+        from rna_structure_models_b200.synth import ModuleDims, module_inputs
+        md_ = ModuleDims(B=1, L=L, H=12, Cz=128, c_s=384)
+        mi_ = module_inputs(md_, 0)
+        mdev = {k: torch.from_numpy(mi_[k]).to(dev) for k in api.MODULE_INPUTS}
+        mplan = api.ModulePlan(1, L, 12, 16, 4, 8, 2, 128, 384, device=dev)
+        mo = torch.empty((1, L, 384), device=dev)
+
+        def timed(fn, n=20):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(n):
+                flush.zero_()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record()
+                fn()
+                a1.record()
+                torch.cuda.synchronize()
+                ts.append(a0.elapsed_time(a1))
+            return statistics.mean(ts)
+
+        ms_layer = timed(lambda: mplan(mdev, out=mo))
+        mplan.check()
+        width = 12 * (3 * 16 + 3 * (2 * 4 + 8))
+        HF = 12 * (16 + 32 + 128)
+        lin_in = api.LinearPlan(L, 384, width, device=dev)
+        lin_out = api.LinearPlan(L, HF, 384, device=dev)
+        xo = torch.randn((L, HF), device=dev)
+        wo = torch.randn((HF, 384), device=dev)
+        ms_in = timed(lambda: lin_in(mdev["s"].view(L, 384), mdev["w_in"], mdev["b_in"]))
+        ms_out = timed(lambda: lin_out(xo, wo, mdev["b_out"]))
+        lin_in.check()
+        lin_out.check()
+        f_in, f_out = 2.0 * L * 384 * width, 2.0 * L * HF * 384
+        line["layer"] = {
+            "workload": f"IPA layer B=1 L={L} H=12 Cz=128 c_s=384: input projection, core, output projection",
+            "ms": ms_layer,
+            "linear_in_ms": ms_in, "linear_in_tflops": f_in / (ms_in / 1e3) / 1e12,
+            "linear_out_ms": ms_out, "linear_out_tflops": f_out / (ms_out / 1e3) / 1e12,
+            "linear_note": "each call packs x and W to fp16 (two kernels) before the tcgen05 GEMM",
+        }
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, nrows, secs = cpu_oracle_sample(L, args.cpu_seconds, 4096)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
