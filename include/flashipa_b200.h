@@ -1,6 +1,9 @@
 /*
  * flashipa_b200.h -- C ABI of the B200 (sm_100a) fused Invariant Point
- * Attention core and of the geometric direction/distance attention variant.
+ * Attention core, of the geometric direction/distance attention variant and
+ * its gradients, of MEET's distance-aware attention, and of the pieces of the
+ * IPA layer around the core (residue frames from backbone atoms, tensor-core
+ * projections, the whole layer).
  *
  * Every buffer is owned by the caller.  The library never allocates or frees
  * device memory and never writes to an input.  Work is enqueued on the
