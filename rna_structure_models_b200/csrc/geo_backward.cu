@@ -268,36 +268,19 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_rows_kernel(const 
   const unsigned char* pmrow =
       a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(in_range ? i : 0) * a.pms[2] : nullptr;
   const int nchunk = (N + BW_CHUNK - 1) / BW_CHUNK;
-  extern __shared__ float bw_merge[];   // [BW_SPLIT][8][BW_ROWS], then the staged keys
+  extern __shared__ float bw_merge[];   // [BW_SPLIT][8][BW_ROWS], the staged keys, the g_attention tiles
   auto sm_at = [&](int s2, int e) -> float& { return bw_merge[(s2 * 8 + e) * BW_ROWS + r]; };
 
-  // D_i = <dagg_i, agg_i> + sum_j a_ij g_attention_ij
-  float dsum = 0.f;
-  if (a.has_g_att && live) {
-    for (int ch = split; ch < nchunk; ch += BW_SPLIT)
-      for (int k = 0; k < BW_CHUNK; ++k) {
-        const int j = ch * BW_CHUNK + k;
-        if (j >= N) break;
-        if (pmrow && !pmrow[static_cast<int64_t>(j) * a.pms[3]]) continue;
-        const float4 k0 = a.kg[2 * (bh * N + j)], k1 = a.kg[2 * (bh * N + j) + 1];
-        const float p = ex2(geo_score(q0, q1, k0, k1, sc.x, sc.y) - m) * inv;
-        dsum = fmaf(p, g_att_at(a, b, h, i, j), dsum);
-      }
-  }
-  sm_at(split, 0) = dsum;
-  __syncthreads();
-  float D = d1;
-#pragma unroll
-  for (int s2 = 0; s2 < BW_SPLIT; ++s2) D += sm_at(s2, 0);
-  __syncthreads();
-
-  float cq[3] = {0.f, 0.f, 0.f}, cp[3] = {0.f, 0.f, 0.f}, sdot = 0.f, sdist = 0.f;
-  // keys of one 32-key chunk staged per split group: [k0 | k1 | vr (padded)]
+  // keys of one 32-key chunk staged per split group: [k0 | k1 | vr (padded)];
+  // with g_attention, also the group's 128 x 32 tile of it (rows padded to 33
+  // floats), loaded row-contiguous so a warp reads 128 consecutive bytes
   constexpr int SW = 8 + ((V + 3) & ~3);
+  constexpr int GP = BW_CHUNK + 1;
   float* stg = bw_merge + BW_SPLIT * 8 * BW_ROWS + split * BW_CHUNK * SW;
+  float* gst = bw_merge + BW_SPLIT * (8 * BW_ROWS + BW_CHUNK * SW) + split * BW_ROWS * GP;
   const uint32_t gbar = 1 + split;
-  for (int ch = split; ch < nchunk; ch += BW_SPLIT) {
-    const int j0 = ch * BW_CHUNK;
+  const int row0 = blockIdx.x * BW_ROWS;
+  auto stage_chunk = [&](int j0) {
     named_bar_sync(gbar, BW_ROWS);                 // the previous chunk has been read
     for (int e = r; e < BW_CHUNK * SW; e += BW_ROWS) {
       const int it = e / SW, f = e % SW, j = j0 + it;
@@ -310,14 +293,53 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_rows_kernel(const 
       }
       stg[e] = v;
     }
+    if (a.has_g_att)
+      for (int e = r; e < BW_ROWS * BW_CHUNK; e += BW_ROWS) {
+        const int rr = e / BW_CHUNK, kk = e % BW_CHUNK, ii = row0 + rr, jj = j0 + kk;
+        gst[rr * GP + kk] = (ii < N && jj < N) ? g_att_at(a, b, h, ii, jj) : 0.f;
+      }
     named_bar_sync(gbar, BW_ROWS);
-    if (!live) continue;
+  };
+  auto chunk_mask = [&](int j0) -> uint32_t {
     uint32_t allowed = 0xffffffffu;
     if (pmrow) {
       allowed = 0u;
       const unsigned char* pr = pmrow + static_cast<int64_t>(j0) * a.pms[3];
       for (int k = 0; k < BW_CHUNK && j0 + k < N; ++k) allowed |= pr[k * a.pms[3]] ? (1u << k) : 0u;
     }
+    return allowed;
+  };
+
+  // D_i = <dagg_i, agg_i> + sum_j a_ij g_attention_ij
+  float dsum = 0.f;
+  if (a.has_g_att) {
+    for (int ch = split; ch < nchunk; ch += BW_SPLIT) {
+      const int j0 = ch * BW_CHUNK;
+      stage_chunk(j0);
+      if (!live) continue;
+      const uint32_t allowed = chunk_mask(j0);
+      for (int k = 0; k < BW_CHUNK; ++k) {
+        if (!((allowed >> k) & 1u)) continue;
+        const float4 k0 = *reinterpret_cast<const float4*>(stg + k * SW);
+        const float4 k1 = *reinterpret_cast<const float4*>(stg + k * SW + 4);
+        const float p = ex2(geo_score(q0, q1, k0, k1, sc.x, sc.y) - m) * inv;   // 0 beyond N
+        dsum = fmaf(p, gst[r * GP + k], dsum);
+      }
+    }
+  }
+  sm_at(split, 0) = dsum;
+  __syncthreads();
+  float D = d1;
+#pragma unroll
+  for (int s2 = 0; s2 < BW_SPLIT; ++s2) D += sm_at(s2, 0);
+  __syncthreads();
+
+  float cq[3] = {0.f, 0.f, 0.f}, cp[3] = {0.f, 0.f, 0.f}, sdot = 0.f, sdist = 0.f;
+  for (int ch = split; ch < nchunk; ch += BW_SPLIT) {
+    const int j0 = ch * BW_CHUNK;
+    stage_chunk(j0);
+    if (!live) continue;
+    const uint32_t allowed = chunk_mask(j0);
     for (int k = 0; k < BW_CHUNK; ++k) {
       if (!((allowed >> k) & 1u)) continue;
       const float* kk = stg + k * SW;
@@ -325,7 +347,7 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_rows_kernel(const 
       const GeoPair g = geo_pair(q0, q1, k0, k1, sc.x, sc.y);
       const float p = ex2(g.s - m) * inv;
       if (p == 0.f) continue;
-      float da = a.has_g_att && j0 + k < N ? g_att_at(a, b, h, i, j0 + k) : 0.f;
+      float da = a.has_g_att ? gst[r * GP + k] : 0.f;
 #pragma unroll
       for (int e = 0; e < V; ++e) da = fmaf(dg[e], kk[8 + e], da);
       const float ds = p * (da - D);
@@ -558,7 +580,8 @@ template <int M>
 cudaError_t launch_pairs(const PairArgs& p, int B, int N, int H, cudaStream_t st) {
   dim3 grid((N + BW_ROWS - 1) / BW_ROWS, H, B);
   constexpr int V4 = (3 * M + 3) & ~3;
-  const size_t smem_r = sizeof(float) * BW_SPLIT * (8 * BW_ROWS + BW_CHUNK * (8 + V4));
+  const size_t smem_r = sizeof(float) * BW_SPLIT *
+                        (8 * BW_ROWS + BW_CHUNK * (8 + V4) + (p.has_g_att ? BW_ROWS * (BW_CHUNK + 1) : 0));
   const size_t smem_c = sizeof(float) * BW_SPLIT * ((6 + 3 * M) * BW_ROWS + BW_CHUNK * (12 + V4));
   if (smem_r > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(geo_bwd_rows_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
