@@ -236,8 +236,9 @@ __device__ __forceinline__ float g_att_at(const PairArgs& a, int b, int h, int i
   return ldf(v, b * v.s[0] + h * v.s[1] + static_cast<int64_t>(i) * v.s[2] + static_cast<int64_t>(j) * v.s[3]);
 }
 
+// two 512-thread blocks per SM (<= 64 registers) where the accumulators allow it
 template <int M>
-__global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_rows_kernel(const PairArgs a) {
+__global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_rows_kernel(const PairArgs a) {
   constexpr int V = 3 * M;
   const int tid = threadIdx.x;
   const int r = tid % BW_ROWS, split = tid / BW_ROWS;
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_rows_kernel(const 
 }
 
 template <int M>
-__global__ void __launch_bounds__(BW_ROWS * BW_SPLIT) geo_bwd_cols_kernel(const PairArgs a) {
+__global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_cols_kernel(const PairArgs a) {
   constexpr int V = 3 * M;
   const int tid = threadIdx.x;
   const int r = tid % BW_ROWS, split = tid / BW_ROWS;
