@@ -138,7 +138,7 @@ struct AttnArgs {
 };
 
 template <int M>
-__global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT) geo_attn_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, M <= 4 ? 2 : 1) geo_attn_kernel(const AttnArgs a) {
   constexpr int V = 3 * M;
   const int tid = threadIdx.x;
   const int r = tid % GEO_ROWS, split = tid / GEO_ROWS;
