@@ -31,8 +31,13 @@ def hi_lo(x):
     return h, f16(np.asarray(x, dtype=np.float64) - h)
 
 
-def ipa_bwd_model(inp: dict, g_out, fwd_out, *, w_L, w_C, scalar_scale) -> dict:
-    """Gradients of sum(g_out * core(inp)); fwd_out is the core's output."""
+def ipa_bwd_model(inp: dict, g_out, fwd_out, *, w_L, w_C, scalar_scale, stages: dict | None = None) -> dict:
+    """Gradients of sum(g_out * core(inp)); fwd_out is the core's output.
+
+    If `stages` is a dict, it receives, per (b, h), the intermediate arrays of
+    each planned kernel stage (operand rows, log2 logits, log-sum-exp, pair
+    aggregate, dS, the two passes' accumulators and row / column sums), so a
+    kernel can be compared stage by stage."""
     q, k, v = (np.asarray(inp[n], np.float64) for n in ("q", "k", "v"))
     qp, kp, vp = (np.asarray(inp[n], np.float64) for n in ("q_pts", "k_pts", "v_pts"))
     rot, trans = np.asarray(inp["rot"], np.float64), np.asarray(inp["trans"], np.float64)
@@ -132,6 +137,12 @@ def ipa_bwd_model(inp: dict, g_out, fwd_out, *, w_L, w_C, scalar_scale) -> dict:
             dVa = a.T @ dO
             cs = dS.sum(axis=0)
             CSo = dS.T @ o_res
+            if stages is not None:
+                stages[(b, h)] = {
+                    "Qrow": Qrow, "Krow": Krow, "QP": QP, "Z2": Z2, "Qrow_keyside": Qrow2, "Va": Va, "dO": dO,
+                    "dU": dU, "origin": o_res, "x": x, "lse": lse2 * LN2, "U": U, "D": D, "dS": dS,
+                    "dQrow": dQrow, "dQP": dQP, "rs": rs, "RSo": RSo, "dKrow": dKrow, "dZ2": dZ2, "dVa": dVa,
+                    "cs": cs, "CSo": CSo}
             # -- mapping back
             grads["q"][b, :, h] = L2E * w_L * ss * dQrow[:, :C]
             grads["k"][b, :, h] = dKrow[:, :C]

@@ -22,3 +22,26 @@ def test_planned_decomposition_matches_the_oracle(L, H, Cz, kw):
     for key, r in ref.items():
         err = np.linalg.norm(got[key] - r) / max(np.linalg.norm(r), 1e-30)
         assert err <= 2e-3, (key, err)
+
+
+def test_stage_references_are_consistent():
+    # the per-stage arrays a kernel will be compared with: softmax rows sum to 1,
+    # the log-sum-exp is the oracle's, dS rows sum to ~0 on live rows
+    inp = ipa_inputs(IpaDims(B=1, L=130, H=2, Cz=16), 3, masked_tail_frac=0.1)
+    consts = ipa_constants(16, 4)
+    out = ipa_dense(inp)
+    g = np.random.default_rng(4).standard_normal(out.shape)
+    stages = {}
+    ipa_bwd_model(inp, g, out, stages=stages, **consts)
+    assert set(stages) == {(0, 0), (0, 1)}
+    st = stages[(0, 1)]
+    live = np.isfinite(st["lse"]) & (inp["mask"][0])
+    a = np.where(np.isfinite(st["x"]), np.exp2(st["x"] - (st["lse"] / np.log(2))[:, None]), 0.0)
+    assert np.allclose(a[live].sum(axis=1), 1.0, atol=1e-9)
+    # natural log-sum-exp of the true logits, from the oracle's own attention
+    _, attn = ipa_dense(inp, return_attn=True)
+    logits_nat = st["x"] * np.log(2)
+    i = np.flatnonzero(live)[5]
+    j = np.flatnonzero(attn[0, 1, i] > 0)[0]
+    assert abs(np.exp(logits_nat[i, j] - st["lse"][i]) - attn[0, 1, i, j]) <= 2e-3 * attn[0, 1, i, j]
+    assert np.max(np.abs(st["rs"][live])) <= 1e-3 * np.max(np.abs(st["dS"]))
