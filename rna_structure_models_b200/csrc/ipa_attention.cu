@@ -31,8 +31,6 @@
 
 #include <cmath>
 #include <cstdint>
-#include <cstdlib>
-#include <cstring>
 
 #include "internal.h"
 #include "ipa_epilogue.cuh"
@@ -71,6 +69,8 @@ struct AttnArgs {
   const float4* frame; // [B, L, 4]
   const float* z1f;    // [B, L, DZ]
   float* out;
+  float* lse;           // training forward: [B, H, L] log-sum-exp (natural log), else null
+  float* uagg;          // training forward: [B, L, H, R Cz] pair aggregate, else null
   int* err;
   int trace_cta0, trace_cta1;
 };
@@ -317,17 +317,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float4* zr = reinterpret_cast<const float4*>(a.z1f + (static_cast<int64_t>(b) * L + (in_range ? row : 0)) * DZ);
       const float4* wr = reinterpret_cast<const float4*>(a.wqp + static_cast<int64_t>(h) * DZ);
       const int c_lo = half * (DZ / 4), c_hi = c_lo + DZ / 4;   // packed columns of this half
+      float qmax = 0.f;   // largest |Q_pair| before rounding (NaN if any is NaN)
       for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
         uint32_t rg[32];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float4 z = in_range ? zr[c0 / 2 + e] : make_float4(0, 0, 0, 0);
           const float4 w = wr[c0 / 2 + e];
-          rg[2 * e] = pack_half2(z.x * w.x, z.y * w.y);
-          rg[2 * e + 1] = pack_half2(z.z * w.z, z.w * w.w);
+          const float4 y = make_float4(z.x * w.x, z.y * w.y, z.z * w.z, z.w * w.w);
+          qmax = fmax_nan(qmax, fmax_nan(fmax_nan(fabsf(y.x), fabsf(y.y)), fmax_nan(fabsf(y.z), fabsf(y.w))));
+          rg[2 * e] = pack_half2(y.x, y.y);
+          rg[2 * e + 1] = pack_half2(y.z, y.w);
         }
         tmem_st32(tmem + TM_QP + c0 + lane_off, rg);
       }
+      if (!(qmax < 65520.f)) record_error(a.err, DEV_NONFINITE);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(B_QP));
@@ -464,6 +468,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     named_bar_sync(pair_bar, 64);
     const float lt = l + xch[512 + (1 - half) * 128 + r];
     const bool dead = !(in_range && f3.x != 0.f && lt > 0.f);
+    // training forward: log-sum-exp of the true logits; the pass left the row
+    // constant c sum_p |gq'_p|^2 (rowq.w) out of its logits
+    if (a.lse != nullptr && half == 0 && in_range)
+      a.lse[static_cast<int64_t>(bh) * L + row] = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
     const int pitch = stage_pitch(DZ);
     float* stage = reinterpret_cast<float*>(smem + SM_STG);
     if (all_ok) {
@@ -485,7 +493,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_before();
     named_bar_sync(1, NSOFT);
     if (!*abort_flag) {
-      const EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, I * QT, a.z1f, a.out};
+      EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, I * QT, a.z1f, a.out};
+      ea.uagg = a.uagg;
       write_rows<IPA_C, IPA_PV>(ea, warp, lane);
     }
   }
@@ -500,18 +509,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace
 
-// FLASHIPA_CORE=single forces the single-CTA kernel (for comparisons); by
-// default the CTA-pair kernel runs whenever it supports the pair width.
-static bool force_single_cta() {
-  static const bool v = [] {
-    const char* e = std::getenv("FLASHIPA_CORE");
-    return e != nullptr && std::strcmp(e, "single") == 0;
-  }();
-  return v;
-}
-
 cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream) {
-  if (ipa_pair_supported(a.DZ) && !force_single_cta()) return ipa_launch_core_pair(a, stream);
+  // the CTA-pair kernel covers pair widths 128 and 256; this kernel the rest
+  if (ipa_pair_supported(a.DZ)) return ipa_launch_core_pair(a, stream);
   unsigned char* ws = a.ws;
   const IpaWorkspace& w = a.lay;
   CUtensorMap tqh, tkh, tvh, tz2;
@@ -538,7 +538,7 @@ cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream) {
   t.wqp = reinterpret_cast<const float*>(ws + w.wqp);
   t.frame = reinterpret_cast<const float4*>(ws + w.frame);
   t.z1f = reinterpret_cast<const float*>(ws + w.z1f);
-  t.out = a.out; t.err = a.err;
+  t.out = a.out; t.err = a.err; t.lse = a.lse; t.uagg = a.uagg;
   t.trace_cta0 = 0;
   t.trace_cta1 = static_cast<int>(bh * a.nqt) / 2;
   ipa_attention_kernel<<<static_cast<unsigned>(bh * a.nqt), NTHREADS, SMEM_ALLOC, stream>>>(tqh, tkh, tvh, tz2, t);

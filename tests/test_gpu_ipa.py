@@ -28,14 +28,23 @@ def test_preset_parity_full(cuda_device, name):
     assert_parity(gpu, ref, what=name)
 
 
-@pytest.mark.parametrize("L", [2048, 4096])
+def sampled_rows(inp, L, n_far, n_random, seed=1):
+    """Rows to compare at long L: the residues farthest from the centroid
+    (largest point coordinates), the first / last rows of query and key
+    tiles around the start, middle and end, and a seeded random sample."""
+    t = inp["trans"][0] - inp["trans"][0].mean(0)
+    far = np.argsort(-np.linalg.norm(t, axis=1))[:n_far]
+    edges = [0, 1, 63, 64, 127, 128, 255, 256, L // 2 - 1, L // 2, L - 129, L - 128, L - 65, L - 64, L - 2, L - 1]
+    rnd = np.random.default_rng(seed).choice(L, n_random, replace=False)
+    return np.unique(np.concatenate([far, edges, rnd]))
+
+
+@pytest.mark.parametrize("L", [2048, 4096, 8192])
 def test_long_context_sampled_rows(cuda_device, L):
+    # configs of the long-context workload (L = 2048 ... 16384, H = 12, R Cz = 256)
     inp = ipa_inputs(IpaDims(B=1, L=L, H=12), 0)
     gpu = run_gpu(inp)
-    t = inp["trans"][0] - inp["trans"][0].mean(0)
-    far = np.argsort(-np.linalg.norm(t, axis=1))[:32]       # residues farthest from the centroid
-    rows = np.unique(np.concatenate([far, [0, 1, 127, 128, L // 2, L - 2, L - 1],
-                                     np.random.default_rng(1).choice(L, 64, replace=False)]))
+    rows = sampled_rows(inp, L, 32, 64)
     ref = ipa_dense_blocked(inp, rows=rows, block=64)
     assert_parity(gpu[:, rows], ref, what=f"L={L}")
 
@@ -44,9 +53,8 @@ def test_longest_context_sampled_rows(cuda_device):
     L = 16384
     inp = ipa_inputs(IpaDims(B=1, L=L, H=12), 0)
     gpu = run_gpu(inp)
-    t = inp["trans"][0] - inp["trans"][0].mean(0)
-    far = np.argsort(-np.linalg.norm(t, axis=1))[:16]
-    rows = np.unique(np.concatenate([far, [0, L // 3, L - 1]]))
+    rows = sampled_rows(inp, L, 32, 48)
+    assert len(rows) >= 64
     ref = ipa_dense_blocked(inp, rows=rows, block=32)
     assert_parity(gpu[:, rows], ref, what="L=16384")
 
@@ -192,14 +200,23 @@ def test_host_pipeline_matches_device_path_per_call(cuda_device):
         assert np.array_equal(out.numpy(), run_gpu(inp))
 
 
+@pytest.mark.parametrize("name", ["q", "z1", "z2", "w_bias"])
 @pytest.mark.parametrize("bad", [1e7, float("nan")])
-def test_operand_outside_fp16_range_is_reported(cuda_device, bad):
-    # a scalar channel that cannot be represented in the fp16 operands (or is
-    # NaN) is reported through the device error word, not silently used
-    inp = ipa_preset("tiny")
-    inp["q"][0, 5, 1, 3] = bad
+@pytest.mark.parametrize("Cz", [16, 64])     # R Cz = 32: single-CTA core; 128: CTA-pair core
+def test_operand_outside_fp16_range_is_reported(cuda_device, bad, name, Cz):
+    # a scalar channel, a pair factor or a pair-bias weight whose fp16 operand
+    # (for w_bias: the scaled Q_pair w_L log2(e) w_bias z1) cannot be
+    # represented (or is NaN) is reported through the device error word, not
+    # silently used
+    inp = ipa_inputs(IpaDims(B=1, L=64, H=4, Cz=Cz), 0)
+    if name == "q":
+        inp["q"][0, 5, 1, 3] = bad
+    elif name == "w_bias":
+        inp["w_bias"][3, 2] = bad
+    else:
+        inp[name][0, 7, 1, 2] = bad
     dev = to_dev({k: inp[k] for k in api.IPA_INPUTS})
-    plan = api.IpaPlan(1, 64, 4, 16, 4, 8, 2, 16, device="cuda")
+    plan = api.IpaPlan(1, 64, 4, 16, 4, 8, 2, Cz, device="cuda")
     plan(*[dev[n] for n in api.IPA_INPUTS])
     torch.cuda.synchronize()
     with pytest.raises(api.IpaError):
