@@ -11,6 +11,7 @@
 //
 // What it costs: the array below (GEO_STATIC_SCRATCH_BYTES) is reserved on
 // every GPU that loads this library, until the process exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -28,18 +29,43 @@ static __device__ __align__(256) unsigned char g_geo_scratch[GEO_STATIC_SCRATCH_
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
+// Per device ordinal: the context the address was looked up in, and the address.
+void* g_scratch_ctx[kMaxDevices] = {};
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the first call on a device does it).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
+
+// Device address of the scratch array on the current device.  It is looked
+// up (cudaGetSymbolAddress) on the first call in a device's context and again
+// whenever that context has changed since (after cudaDeviceReset the module
+// is loaded anew and the array may sit elsewhere).
 ipa_status_t scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return IPA_ERR_CUDA;
+  const CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (get_ctx == nullptr) return IPA_ERR_CUDA;
+  CUcontext ctx = nullptr;   // null until the runtime has set this device up in this thread
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return IPA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (ctx == nullptr || g_scratch_addr[dev] == nullptr || g_scratch_ctx[dev] != static_cast<void*>(ctx)) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_geo_scratch) != cudaSuccess || p == nullptr) return IPA_ERR_CUDA;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return IPA_ERR_CUDA;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = static_cast<void*>(ctx);
   }
   *out = g_scratch_addr[dev];
   return IPA_OK;
