@@ -79,6 +79,8 @@ struct PairArgs {
   const float4* frame;
   const float* z1f;     // [B, L, DZ]
   float* out;
+  float* lse;           // training forward: [B, H, L] log-sum-exp (natural log), else null
+  float* uagg;          // training forward: [B, L, H, R Cz] pair aggregate, else null
   int* err;
   int trace_cta0, trace_cta1;
 };
@@ -394,6 +396,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_QFULL), 0, abort_flag)) && lane == 0)
         fail(DEV_TIMEOUT_FULL);
       const float* wr = a.wqp + static_cast<int64_t>(h) * DZ;
+      float qmax = 0.f;   // largest |Q_pair| before rounding (NaN if any is NaN)
       for (int p = half * (np / 2); p < (half + 1) * (np / 2); ++p) {
         unsigned char* prow = smem + SP_QP + 16384 * p + r * 128;
 #pragma unroll
@@ -403,11 +406,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr + 64 * p + 8 * c));
           const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr + 64 * p + 8 * c + 4));
           const float2 z0 = unpack_half2(u.x), z1 = unpack_half2(u.y), z2 = unpack_half2(u.z), z3 = unpack_half2(u.w);
-          u = make_uint4(pack_half2(z0.x * w0.x, z0.y * w0.y), pack_half2(z1.x * w0.z, z1.y * w0.w),
-                         pack_half2(z2.x * w1.x, z2.y * w1.y), pack_half2(z3.x * w1.z, z3.y * w1.w));
+          const float e[8] = {z0.x * w0.x, z0.y * w0.y, z1.x * w0.z, z1.y * w0.w,
+                              z2.x * w1.x, z2.y * w1.y, z3.x * w1.z, z3.y * w1.w};
+#pragma unroll
+          for (int t = 0; t < 8; ++t) qmax = fmax_nan(qmax, fabsf(e[t]));
+          u = make_uint4(pack_half2(e[0], e[1]), pack_half2(e[2], e[3]), pack_half2(e[4], e[5]), pack_half2(e[6], e[7]));
           *ptr = u;
         }
       }
+      if (in_range && !(qmax < 65520.f)) record_error(a.err, DEV_NONFINITE);
       fence_proxy_async_smem();
       named_bar_sync(1, NSOFT);
       if (tid == 0) PAIR_SPAN(6);
@@ -542,6 +549,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     named_bar_sync(pair_bar, 64);
     const float lt = l + xch[512 + (1 - half) * 128 + r];
     const bool dead = !(in_range && f3.x != 0.f && lt > 0.f);
+    // training forward: log-sum-exp of the true logits; the pass left the row
+    // constant c sum_p |gq'_p|^2 (rowq.w) out of its logits
+    if (a.lse != nullptr && half == 0 && in_range)
+      a.lse[static_cast<int64_t>(bh) * L + row] = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
     const int pitch = stage_pitch(DZ);
     float* stage = reinterpret_cast<float*>(smem + SP_QP);
     if (all_ok) {
@@ -567,6 +578,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     if (tid == 0) PAIR_SPAN(11);
     if (!*abort_flag) {
       EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, row0, a.z1f, a.out};
+      ea.uagg = a.uagg;
 #ifdef IPA_TRACE
       ea.trace = (blockIdx.x < 4096 && warp == 0) ? &g_pair_span[blockIdx.x][16] : nullptr;
 #endif
@@ -624,7 +636,7 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
   t.wqp = reinterpret_cast<const float*>(ws + w.wqp);
   t.frame = reinterpret_cast<const float4*>(ws + w.frame);
   t.z1f = reinterpret_cast<const float*>(ws + w.z1f);
-  t.out = a.out; t.err = a.err;
+  t.out = a.out; t.err = a.err; t.lse = a.lse; t.uagg = a.uagg;
   const int pairs = static_cast<int>(bh) * t.nqp;
   t.trace_cta0 = 0;
   t.trace_cta1 = 1;   // the peer CTA of the first pair

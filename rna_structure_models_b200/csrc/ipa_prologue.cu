@@ -55,7 +55,13 @@ struct TileArgs {
   float* z1f;      // [B, L, DZ]
   __half* z1h;     // [B, L, DZ]
   __half* z2h;     // [B, L, DZ]
+  int* err;        // DEV_NONFINITE when a pair factor does not survive the fp16 rounding
 };
+
+// |x| >= 65520 (or NaN) does not survive the rounding to fp16
+__device__ __forceinline__ void check_fp16_range(const TileArgs& a, float vmax) {
+  if (!(vmax < 65520.f)) record_error(a.err, DEV_NONFINITE);
+}
 
 // Pair factors of 64 residues x one 64-column panel, zero-padded beyond
 // R*Cz and zero for masked residues: 4 residues x 64 columns per pass, all
@@ -82,6 +88,13 @@ __device__ __forceinline__ bool ipa_tile_copy_pairs_vec(const TileArgs& a, int b
       v2[q] = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(a.z2.p) + b * a.z2.s[0] + i * a.z2.s[1] + col));
     }
   }
+  float vmax = 0.f;
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    vmax = fmax_nan(vmax, fmax_nan(fmax_nan(fabsf(v1[q].x), fabsf(v1[q].y)), fmax_nan(fabsf(v1[q].z), fabsf(v1[q].w))));
+    vmax = fmax_nan(vmax, fmax_nan(fmax_nan(fabsf(v2[q].x), fabsf(v2[q].y)), fmax_nan(fabsf(v2[q].z), fabsf(v2[q].w))));
+  }
+  check_fp16_range(a, vmax);
 #pragma unroll
   for (int q = 0; q < NP; ++q) {
     const int i = i0 + 16 * q + (tid >> 4);
@@ -112,6 +125,10 @@ __device__ __forceinline__ void ipa_tile_copy_pairs(const TileArgs& a, int b, in
       v2[q] = ldf(a.z2, b * a.z2.s[0] + i * a.z2.s[1] + rr * a.z2.s[2] + cc * a.z2.s[3]);
     }
   }
+  float vmax = 0.f;
+#pragma unroll
+  for (int q = 0; q < NR; ++q) vmax = fmax_nan(vmax, fmax_nan(fabsf(v1[q]), fabsf(v2[q])));
+  check_fp16_range(a, vmax);
 #pragma unroll
   for (int q = 0; q < NR; ++q) {
     const int i = i0 + 4 * q + (tid >> 6);
@@ -186,7 +203,7 @@ struct RowArgs {
   uint4* qh;       // [B*H, L, 64] fp16 (8 x uint4 per row)
   uint4* kh;
   uint4* vh;
-  float4* rowq;    // [B*H, L]
+  float4* rowq;    // [B*H, L]: (sum_p gq'_p, c sum_p |gq'_p|^2)
   float4* colk;    // [B*H, L]
   int* err;
 };
@@ -206,13 +223,6 @@ __device__ __forceinline__ void load_row(const View& v, int64_t base, int64_t st
 #pragma unroll
     for (int e = 0; e < N; ++e) out[e] = p[e * st];
   }
-}
-
-// max that propagates NaN (so a NaN operand is reported like an overflow)
-__device__ __forceinline__ float fmax_nan(float a, float b) {
-  float d;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
-  return d;
 }
 
 // Origin (mean of the valid centred frame origins) of a run of 64-residue
@@ -345,12 +355,13 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
       gv[3 * p + x] = fmaf(Rm[3 * x], vp[3 * p], fmaf(Rm[3 * x + 1], vp[3 * p + 1], Rm[3 * x + 2] * vp[3 * p + 2])) + tc[x];
 
   // rows are built and stored one after the other to keep few values live
-  float sq[3] = {0.f, 0.f, 0.f}, sk[3] = {0.f, 0.f, 0.f}, nk = 0.f;
+  float sq[3] = {0.f, 0.f, 0.f}, sk[3] = {0.f, 0.f, 0.f}, nk = 0.f, nq = 0.f;
 #pragma unroll
   for (int e = 0; e < 3 * PQ; ++e) {
     sq[e % 3] += gq[e];
     sk[e % 3] += gk[e];
     nk = fmaf(gk[e], gk[e], nk);
+    nq = fmaf(gq[e], gq[e], nq);
   }
   float vmax = 0.f;   // largest |value| written (NaN if any value is NaN)
   auto store_row = [&](uint4* dst, auto value_of) {
@@ -404,8 +415,12 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   if (!valid) {
     sq[0] = sq[1] = sq[2] = 0.f;
     sk[0] = sk[1] = sk[2] = 0.f;
+    nq = 0.f;
   }
-  sterm[slot] = make_float4(sq[0], sq[1], sq[2], 0.f);
+  // .w: the row constant c sum_p |gq'_p|^2 that the fused pass leaves out of
+  // its logits (it cancels in the softmax); a training forward adds it back
+  // to report the log-sum-exp of the true logits
+  sterm[slot] = make_float4(sq[0], sq[1], sq[2], c * nq);
   sterm[H * rb + slot] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
   // |x| >= 65520 (or NaN) does not survive the fp16 rounding
   if (valid && !(vmax < 65520.f)) record_error(a.err, DEV_NONFINITE);
@@ -445,6 +460,7 @@ cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
   ta.z1f = reinterpret_cast<float*>(ws + w.z1f);
   ta.z2h = reinterpret_cast<__half*>(ws + w.z2);
   ta.z1h = reinterpret_cast<__half*>(ws + w.z1h);
+  ta.err = a.err;
   ipa_tile_kernel<<<dim3(a.nkt, a.B, a.DZ / 64), 256, 0, stream>>>(ta);
 
   RowArgs r{};

@@ -423,6 +423,13 @@ __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
   return d;
 }
 
+// Maximum that propagates NaN (a NaN operand is reported like an overflow).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // Three-input maximum.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
