@@ -117,3 +117,21 @@ def test_matches_float64_autograd_of_a_torch_restatement():
     grads = ipa_grad(inp, g)
     for key in KEYS:
         close(grads[key], t[key].grad.numpy(), 1e-10, key)
+
+
+def test_blocked_gradient_equals_the_dense_gradient():
+    # the row-blocked oracle (bounded memory, for long sequences) sums the
+    # same per-row steps; it must reproduce ipa_grad, including masked and
+    # dead rows and a ragged last block
+    from oracle.ipa_grad_blocked import ipa_grad_blocked
+    inp = as64(ipa_inputs(IpaDims(B=2, L=23, H=3, C=4, Pq=2, Pv=3, R=2, Cz=5), 7, jitter=0.5))
+    inp["mask"] = inp["mask"].copy()
+    inp["mask"][0, 4] = False
+    inp["mask"][1, :] = False
+    inp["mask"][1, 9] = True
+    g = upstream(inp, 17)
+    ref = ipa_grad(inp, g)
+    for block in (1, 5, 8, 64):
+        got = ipa_grad_blocked(inp, g, block=block)
+        for key in KEYS:
+            assert np.allclose(got[key], ref[key], rtol=1e-10, atol=1e-12), (block, key)
