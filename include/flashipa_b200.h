@@ -150,6 +150,68 @@ IPA_API ipa_status_t ipa_attn_core(const ipa_params_t* p, const ipa_tensor_t* ou
                            void* stream, int32_t* dev_err);
 
 /* --------------------------------------------------------------------------
+ * Training forward and gradients of the fused IPA core (Flash Invariant
+ * Point Attention trains the factorised IPA: TL;DR "drop-in replacement",
+ * Abstract "extends training to previously unattainable lengths", Figure 3).
+ *
+ * ipa_attn_fwd_train: ipa_attn_fwd plus two per-row results the gradient
+ * pass needs (same params, inputs, workspace and rules as ipa_attn_fwd):
+ *   lse    [B, H, L]        IPA_DTYPE_F32, contiguous: log sum_{allowed j}
+ *                           exp(logit_ij) (natural log); +inf for a row with
+ *                           no allowed key
+ *   u_agg  [B, L, H, R, Cz] IPA_DTYPE_F32, contiguous, 16-byte aligned:
+ *                           U_i = sum_j a_ij z2_j (the pair-value aggregate
+ *                           before its contraction with z1_i); 0 on rows with
+ *                           no allowed key
+ *
+ * ipa_attn_bwd: gradients of sum(g_out * out) with respect to every float
+ * input, for a caller-given upstream gradient g_out of the output layout.
+ * Inputs: the 13 forward inputs, the forward's out, lse and u_agg (from
+ * ipa_attn_fwd_train on the same inputs), g_out [B, L, H, C + 4 Pv + Cz]
+ * (all IPA_DTYPE_F32, any non-negative strides).  Outputs: ipa_grads_t,
+ * each IPA_DTYPE_F32, contiguous, with the shape of its input (mask has no
+ * gradient).  Readings: rows with no allowed key pass nothing on; the
+ * derivative of a point norm |o_pt| at o_pt = 0 is taken as 0.
+ * Method: flash-style recomputation on the forward's augmented fp16
+ * operands -- a query-side pass (dQ) and a key-side pass (dK, dV, dZ2) on
+ * tcgen05 tensor cores with fp32 accumulation, then per-residue kernels that
+ * map the augmented gradients back and sum over heads (fixed order, no
+ * atomics: bitwise reproducible).  No L x L array is stored; the workspace
+ * (ipa_attn_bwd_workspace_size bytes, 256-byte aligned) is linear in L.
+ * Same envelope as ipa_attn_fwd.
+ * ------------------------------------------------------------------------ */
+IPA_API ipa_status_t ipa_attn_fwd_train(const ipa_params_t* p,
+                          const ipa_tensor_t* q, const ipa_tensor_t* k, const ipa_tensor_t* v,
+                          const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                          const ipa_tensor_t* v_pts,
+                          const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                          const ipa_tensor_t* z1, const ipa_tensor_t* z2,
+                          const ipa_tensor_t* w_bias, const ipa_tensor_t* gamma,
+                          const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                          const ipa_tensor_t* lse, const ipa_tensor_t* u_agg,
+                          void* workspace, size_t workspace_bytes,
+                          void* stream, int32_t* dev_err);
+
+typedef struct {
+  ipa_tensor_t q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma;
+} ipa_grads_t;
+
+IPA_API size_t ipa_attn_bwd_workspace_size(const ipa_params_t* p);
+
+IPA_API ipa_status_t ipa_attn_bwd(const ipa_params_t* p,
+                          const ipa_tensor_t* q, const ipa_tensor_t* k, const ipa_tensor_t* v,
+                          const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                          const ipa_tensor_t* v_pts,
+                          const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                          const ipa_tensor_t* z1, const ipa_tensor_t* z2,
+                          const ipa_tensor_t* w_bias, const ipa_tensor_t* gamma,
+                          const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                          const ipa_tensor_t* lse, const ipa_tensor_t* u_agg,
+                          const ipa_tensor_t* g_out, const ipa_grads_t* grads,
+                          void* workspace, size_t workspace_bytes,
+                          void* stream, int32_t* dev_err);
+
+/* --------------------------------------------------------------------------
  * Geometric direction-and-distance attention ("Geometric direction-and-
  * distance attention", Required behavior).  For query i, key j, head h:
  *   qd = R_i q_direction_i, kd = R_j k_direction_j,
@@ -256,7 +318,9 @@ IPA_API ipa_status_t geo_attn_bwd(const geo_params_t* p,
  *     of 128 bytes for M = 4).
  *   - The first call on a device looks the array's device address up
  *     (cudaGetSymbolAddress); make that first call outside any stream
- *     capture.
+ *     capture.  The address is cached per device and context, and looked up
+ *     again when the device's current context differs from the cached one
+ *     (after cudaDeviceReset, for example).
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents: calls whose executions overlap on the GPU (other
  *     streams, other host threads) race on it and must be serialised by the
