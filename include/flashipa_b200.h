@@ -53,7 +53,8 @@ enum {
   IPA_DTYPE_F32 = 0,
   IPA_DTYPE_F64 = 1,
   IPA_DTYPE_BOOL = 2, /* one byte per element, 0 = false */
-  IPA_DTYPE_F16 = 3
+  IPA_DTYPE_F16 = 3,
+  IPA_DTYPE_I32 = 4
 };
 
 #define IPA_MAX_DIMS 6
@@ -148,6 +149,33 @@ IPA_API ipa_status_t ipa_attn_prologue(const ipa_params_t* p,
 IPA_API ipa_status_t ipa_attn_core(const ipa_params_t* p, const ipa_tensor_t* out,
                            void* workspace, size_t workspace_bytes,
                            void* stream, int32_t* dev_err);
+
+/* --------------------------------------------------------------------------
+ * ipa_attn_fwd on HOST buffers (end-to-end call for callers whose inputs and
+ * results live in host memory).  Same params and shapes as ipa_attn_fwd;
+ * every input and `out` must be a contiguous host buffer (page-locked, e.g.
+ * from cudaMallocHost, for the copies to be asynchronous).  On `stream` the
+ * call enqueues one cudaMemcpyAsync per input into `staging` (device memory
+ * of ipa_attn_host_staging_size(p) bytes, 256-byte aligned, caller-owned),
+ * the prologue and core kernels (using `workspace` as ipa_attn_fwd does) and
+ * one cudaMemcpyAsync of the result back into `out`.  The caller
+ * synchronises the stream before reading `out` or reusing the host inputs.
+ * Calls on different streams with their own staging and workspace overlap
+ * one call's copies with another's kernels.
+ * ------------------------------------------------------------------------ */
+IPA_API size_t ipa_attn_host_staging_size(const ipa_params_t* p);
+
+IPA_API ipa_status_t ipa_attn_fwd_host(const ipa_params_t* p,
+                          const ipa_tensor_t* q, const ipa_tensor_t* k, const ipa_tensor_t* v,
+                          const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                          const ipa_tensor_t* v_pts,
+                          const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                          const ipa_tensor_t* z1, const ipa_tensor_t* z2,
+                          const ipa_tensor_t* w_bias, const ipa_tensor_t* gamma,
+                          const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                          void* staging, size_t staging_bytes,
+                          void* workspace, size_t workspace_bytes,
+                          void* stream, int32_t* dev_err);
 
 /* --------------------------------------------------------------------------
  * Training forward and gradients of the fused IPA core (Flash Invariant
@@ -341,6 +369,34 @@ IPA_API ipa_status_t geo_attn_fwd_static(const geo_params_t* p,
                                  const ipa_tensor_t* out_vectors, const ipa_tensor_t* out_output,
                                  const ipa_tensor_t* out_attention,
                                  void* stream, int32_t* dev_err);
+
+/* --------------------------------------------------------------------------
+ * Local nearest-neighbour distogram of residue positions (Flash Invariant
+ * Point Attention, TL;DR: the pair representation is built from "a local
+ * nearest-neighbor distogram").  The page fixes neither the neighbour count
+ * nor the distance bins nor the map to pair factors, so the first two are
+ * arguments here and the third is left to the caller (e.g. a projection of
+ * the histogram with ipa_linear_fwd).  For batch b and valid residue i:
+ *   idx[b,i,:]   the k valid residues j != i nearest to i (|x_j - x_i|),
+ *                nearest first, equal distances in increasing j; -1 in
+ *                slots beyond the number of valid other residues
+ *   bins[b,i,:]  bin of each neighbour's distance: #{m : d >= edges[m]},
+ *                in [0, n_edges]; -1 in empty slots
+ *   hist[b,i,c]  number of neighbours in bin c (n_edges + 1 bins)
+ * and all slots -1 / 0 for a masked residue.  Distances are compared as
+ * float32 squared distances (dx*dx + dy*dy) + dz*dz against float32 squared
+ * edges, so the integer results are those of float32 arithmetic.
+ * Inputs: x [B, L, 3] IPA_DTYPE_F32 (C-alpha or frame origins, any strides),
+ * mask [B, L] IPA_DTYPE_BOOL, edges: HOST array of n_edges strictly
+ * increasing non-negative float32 values (validated on the host).
+ * Outputs (contiguous): idx, bins [B, L, k] IPA_DTYPE_I32, hist [B, L,
+ * n_edges + 1] IPA_DTYPE_F32.  Envelope: 1 <= k <= 32, 0 <= n_edges <= 63.
+ * No workspace.
+ * ------------------------------------------------------------------------ */
+IPA_API ipa_status_t ipa_knn_distogram(int32_t B, int32_t L, int32_t k, int32_t n_edges,
+                               const ipa_tensor_t* x, const ipa_tensor_t* mask,
+                               const float* edges, const ipa_tensor_t* idx,
+                               const ipa_tensor_t* bins, const ipa_tensor_t* hist, void* stream);
 
 /* --------------------------------------------------------------------------
  * Distance-aware attention (MEET, §2.2 "distance-aware attention",

@@ -17,16 +17,18 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libflashipa_b200.so")
 
-IPA_DTYPE_F32, IPA_DTYPE_F64, IPA_DTYPE_BOOL, IPA_DTYPE_F16 = 0, 1, 2, 3
+IPA_DTYPE_F32, IPA_DTYPE_F64, IPA_DTYPE_BOOL, IPA_DTYPE_F16, IPA_DTYPE_I32 = 0, 1, 2, 3, 4
 STATUS = {0: "IPA_OK", 1: "IPA_ERR_NULL", 2: "IPA_ERR_SHAPE", 3: "IPA_ERR_STRIDE_ALIGN",
           4: "IPA_ERR_DTYPE", 5: "IPA_ERR_WORKSPACE", 6: "IPA_ERR_UNSUPPORTED", 7: "IPA_ERR_CUDA",
           8: "IPA_ERR_TIMEOUT"}
 EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa_attn_core",
+            "ipa_attn_fwd_train", "ipa_attn_bwd_workspace_size", "ipa_attn_bwd",
+            "ipa_attn_host_staging_size", "ipa_attn_fwd_host",
             "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static",
             "geo_attn_bwd_workspace_size", "geo_attn_bwd",
             "meet_attn_workspace_size", "meet_attn_fwd", "ipa_frames_from_backbone", "ipa_linear_workspace_size",
             "ipa_linear_fwd", "ipa_module_workspace_size", "ipa_module_fwd", "ipa_status_string",
-            "ipa_device_error_status", "ipa_version")
+            "ipa_device_error_status", "ipa_version", "ipa_knn_distogram")
 
 
 class IpaTensor(ctypes.Structure):
@@ -52,6 +54,13 @@ GEO_GRADS = ("q_direction", "k_direction", "q_point", "k_point", "values", "dire
 
 class GeoGrads(ctypes.Structure):
     _fields_ = [(n, IpaTensor) for n in GEO_GRADS]
+
+
+IPA_GRADS = ("q", "k", "v", "q_pts", "k_pts", "v_pts", "rot", "trans", "z1", "z2", "w_bias", "gamma")
+
+
+class IpaGrads(ctypes.Structure):
+    _fields_ = [(n, IpaTensor) for n in IPA_GRADS]
 
 
 class MeetParams(ctypes.Structure):
@@ -93,6 +102,20 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ipa_attn_core.argtypes = [P(IpaParams), T, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                   ctypes.c_void_p]
     lib.ipa_attn_core.restype = ctypes.c_int
+    lib.ipa_attn_fwd_train.argtypes = [P(IpaParams)] + [T] * 16 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                                  ctypes.c_void_p, ctypes.c_void_p]
+    lib.ipa_attn_fwd_train.restype = ctypes.c_int
+    lib.ipa_attn_host_staging_size.argtypes = [P(IpaParams)]
+    lib.ipa_attn_host_staging_size.restype = ctypes.c_size_t
+    lib.ipa_attn_fwd_host.argtypes = [P(IpaParams)] + [T] * 14 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                                 ctypes.c_void_p, ctypes.c_size_t,
+                                                                 ctypes.c_void_p, ctypes.c_void_p]
+    lib.ipa_attn_fwd_host.restype = ctypes.c_int
+    lib.ipa_attn_bwd_workspace_size.argtypes = [P(IpaParams)]
+    lib.ipa_attn_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.ipa_attn_bwd.argtypes = [P(IpaParams)] + [T] * 17 + [P(IpaGrads), ctypes.c_void_p, ctypes.c_size_t,
+                                                            ctypes.c_void_p, ctypes.c_void_p]
+    lib.ipa_attn_bwd.restype = ctypes.c_int
     lib.geo_attn_workspace_size.argtypes = [P(GeoParams)]
     lib.geo_attn_workspace_size.restype = ctypes.c_size_t
     lib.geo_attn_fwd.argtypes = [P(GeoParams)] + [T] * 16 + [ctypes.c_void_p, ctypes.c_size_t,
@@ -120,6 +143,9 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ipa_module_fwd.argtypes = [P(ModuleParams)] + [T] * 14 + [ctypes.c_void_p, ctypes.c_size_t,
                                                                   ctypes.c_void_p, ctypes.c_void_p]
     lib.ipa_module_fwd.restype = ctypes.c_int
+    lib.ipa_knn_distogram.argtypes = [ctypes.c_int32] * 4 + [T, T, ctypes.POINTER(ctypes.c_float), T, T, T,
+                                                             ctypes.c_void_p]
+    lib.ipa_knn_distogram.restype = ctypes.c_int
     lib.ipa_status_string.argtypes = [ctypes.c_int]
     lib.ipa_status_string.restype = ctypes.c_char_p
     lib.ipa_device_error_status.argtypes = [ctypes.c_int32]
@@ -131,7 +157,7 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 _DT = {torch.float32: IPA_DTYPE_F32, torch.float64: IPA_DTYPE_F64, torch.bool: IPA_DTYPE_BOOL,
-       torch.uint8: IPA_DTYPE_BOOL, torch.float16: IPA_DTYPE_F16}
+       torch.uint8: IPA_DTYPE_BOOL, torch.float16: IPA_DTYPE_F16, torch.int32: IPA_DTYPE_I32}
 
 
 def tensor_desc(t: Optional[torch.Tensor]) -> IpaTensor:
@@ -239,8 +265,71 @@ class IpaPlan:
             raise IpaError(st, library().ipa_status_string(st).decode())
         return out
 
+    def train(self, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask,
+              out=None, lse=None, u_agg=None, stream=None):
+        """Training forward: the output plus the log-sum-exp of the logits
+        [B, H, L] and the pair aggregate U [B, L, H, R, Cz] that the gradient
+        pass needs.  Returns (out, lse, u_agg)."""
+        p = self.params
+        _require_cuda(q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask)
+        dev = q.device
+        if out is None:
+            out = torch.empty((p.B, p.L, p.H, self.F), dtype=torch.float32, device=dev)
+        if lse is None:
+            lse = torch.empty((p.B, p.H, p.L), dtype=torch.float32, device=dev)
+        if u_agg is None:
+            u_agg = torch.empty((p.B, p.L, p.H, p.R, p.Cz), dtype=torch.float32, device=dev)
+        descs = [tensor_desc(t) for t in (q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2,
+                                          w_bias, gamma, mask, out, lse, u_agg)]
+        st = library().ipa_attn_fwd_train(ctypes.byref(p), *[ctypes.byref(d) for d in descs],
+                                          ctypes.c_void_p(self.workspace.data_ptr()),
+                                          ctypes.c_size_t(self.workspace.numel()),
+                                          ctypes.c_void_p(_stream_ptr(stream)),
+                                          ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return out, lse, u_agg
+
     def check(self):
         """Synchronise and raise if a kernel reported a device-side error."""
+        v = int(self.dev_err.item())
+        if v != 0:
+            self.dev_err.zero_()
+            raise IpaError(int(library().ipa_device_error_status(v)), f"device error code {v}")
+
+
+class IpaGradPlan:
+    """Gradients of the fused IPA core for one problem shape; the plan owns
+    the workspace (linear in L) and a device error word."""
+
+    def __init__(self, B, L, H, C=16, Pq=4, Pv=8, R=2, Cz=128, device="cuda", **consts):
+        self.params = ipa_params(B, L, H, C, Pq, Pv, R, Cz, **consts)
+        nbytes = int(library().ipa_attn_bwd_workspace_size(ctypes.byref(self.params)))
+        if nbytes == 0:
+            raise IpaError(6, "dimensions outside the supported envelope")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def __call__(self, inp: dict, out, lse, u_agg, g_out, *, grads: Optional[dict] = None, stream=None) -> dict:
+        """inp: the forward inputs (IPA_INPUTS); out, lse, u_agg: the training
+        forward's results; g_out: upstream gradient of out.  Returns the
+        gradients of sum(g_out * out) keyed like IPA_GRADS."""
+        p = self.params
+        _require_cuda(*[inp[n] for n in IPA_INPUTS], out, lse, u_agg, g_out)
+        if grads is None:
+            grads = {n: torch.empty(tuple(inp[n].shape), dtype=torch.float32, device=out.device) for n in IPA_GRADS}
+        descs = [tensor_desc(inp[n]) for n in IPA_INPUTS] + [tensor_desc(t) for t in (out, lse, u_agg, g_out)]
+        gs = IpaGrads(*[tensor_desc(grads[n]) for n in IPA_GRADS])
+        st = library().ipa_attn_bwd(ctypes.byref(p), *[ctypes.byref(d) for d in descs], ctypes.byref(gs),
+                                    ctypes.c_void_p(self.workspace.data_ptr()),
+                                    ctypes.c_size_t(self.workspace.numel()),
+                                    ctypes.c_void_p(_stream_ptr(stream)),
+                                    ctypes.c_void_p(self.dev_err.data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+        return grads
+
+    def check(self):
         v = int(self.dev_err.item())
         if v != 0:
             self.dev_err.zero_()
@@ -259,6 +348,30 @@ def ipa_attn(inp: dict, *, out=None, stream=None, check: bool = True, **consts):
     R, Cz = inp["z1"].shape[2], inp["z1"].shape[3]
     plan = IpaPlan(B, L, H, C, Pq, Pv, R, Cz, device=q.device, **consts)
     res = plan(*[inp[n] for n in IPA_INPUTS], out=out, stream=stream)
+    if check:
+        plan.check()
+    return res
+
+
+def _dims_of(inp: dict):
+    q = inp["q"]
+    B, L, H, C = q.shape
+    return B, L, H, C, inp["q_pts"].shape[3], inp["v_pts"].shape[3], inp["z1"].shape[2], inp["z1"].shape[3]
+
+
+def ipa_attn_train(inp: dict, *, stream=None, check: bool = True, **consts):
+    """Training forward on CUDA tensors: (out, lse, u_agg)."""
+    plan = IpaPlan(*_dims_of(inp), device=inp["q"].device, **consts)
+    res = plan.train(*[inp[n] for n in IPA_INPUTS], stream=stream)
+    if check:
+        plan.check()
+    return res
+
+
+def ipa_attn_backward(inp: dict, out, lse, u_agg, g_out, *, stream=None, check: bool = True, **consts) -> dict:
+    """Gradients of sum(g_out * out) with respect to every float input."""
+    plan = IpaGradPlan(*_dims_of(inp), device=inp["q"].device, **consts)
+    res = plan(inp, out, lse, u_agg, g_out, stream=stream)
     if check:
         plan.check()
     return res
@@ -297,6 +410,55 @@ def ipa_attn_host(inp: dict, plan: Optional[IpaPlan] = None, device="cuda", stre
         out = cache[hkey]
     out.copy_(res, non_blocking=True)
     return out, plan
+
+
+class IpaHostCalls:
+    """Calls of the C entry point ipa_attn_fwd_host (host buffers in, host
+    result out; the copies and kernels are enqueued by the library) on
+    `slots` streams, each with its own device staging, workspace and error
+    word, so that one call's copies overlap another call's kernels."""
+
+    def __init__(self, B, L, H, C=16, Pq=4, Pv=8, R=2, Cz=128, slots=2, device="cuda", **consts):
+        self.params = ipa_params(B, L, H, C, Pq, Pv, R, Cz, **consts)
+        lib = library()
+        ns = int(lib.ipa_attn_host_staging_size(ctypes.byref(self.params)))
+        nw = int(lib.ipa_attn_workspace_size(ctypes.byref(self.params)))
+        if ns == 0 or nw == 0:
+            raise IpaError(6, "dimensions outside the supported envelope")
+        self.device = torch.device(device)
+        self.staging = [torch.empty(ns, dtype=torch.uint8, device=device) for _ in range(slots)]
+        self.workspace = [torch.empty(nw, dtype=torch.uint8, device=device) for _ in range(slots)]
+        self.dev_err = torch.zeros(slots, dtype=torch.int32, device=device)
+        self.streams = [torch.cuda.Stream(self.device) for _ in range(slots)]
+        self.F = C + 4 * Pv + Cz
+
+    def call(self, inp: dict, out, slot: int = 0):
+        """Enqueue one call on slot `slot`'s stream (host tensors, contiguous)."""
+        descs = [tensor_desc(inp[n]) for n in IPA_INPUTS] + [tensor_desc(out)]
+        st = library().ipa_attn_fwd_host(ctypes.byref(self.params), *[ctypes.byref(d) for d in descs],
+                                         ctypes.c_void_p(self.staging[slot].data_ptr()),
+                                         ctypes.c_size_t(self.staging[slot].numel()),
+                                         ctypes.c_void_p(self.workspace[slot].data_ptr()),
+                                         ctypes.c_size_t(self.workspace[slot].numel()),
+                                         ctypes.c_void_p(self.streams[slot].cuda_stream),
+                                         ctypes.c_void_p(self.dev_err[slot:].data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+
+    def run(self, inputs, outputs):
+        """Calls k = 0, 1, ... on slot k mod slots; waits for all of them."""
+        for k, (inp, out) in enumerate(zip(inputs, outputs)):
+            self.call(inp, out, k % len(self.streams))
+        for s in self.streams:
+            s.synchronize()
+        return outputs
+
+    def check(self):
+        v = self.dev_err.cpu()
+        if int(v.abs().sum()) != 0:
+            self.dev_err.zero_()
+            code = int(v[v != 0][0])
+            raise IpaError(int(library().ipa_device_error_status(code)), f"device error code {code}")
 
 
 class IpaHostPipeline:
@@ -530,6 +692,27 @@ def frames_from_backbone(n, ca, c, rot=None, trans=None, stream=None):
     if st != 0:
         raise IpaError(st, library().ipa_status_string(st).decode())
     return rot, trans
+
+
+# ------------------------------------------------------------------ distogram
+def knn_distogram(x, mask, k: int, edges, *, stream=None):
+    """Local nearest-neighbour distogram of positions x [B, L, 3] (CUDA
+    tensors): (idx [B, L, k] int32, bins [B, L, k] int32, hist [B, L, nb]
+    float32), nb = len(edges) + 1; `edges` is a host sequence of increasing
+    distances (Angstrom)."""
+    _require_cuda(x, mask)
+    B, L = x.shape[0], x.shape[1]
+    e = (ctypes.c_float * max(1, len(edges)))(*[float(v) for v in edges])
+    idx = torch.empty((B, L, k), dtype=torch.int32, device=x.device)
+    bins = torch.empty((B, L, k), dtype=torch.int32, device=x.device)
+    hist = torch.empty((B, L, len(edges) + 1), dtype=torch.float32, device=x.device)
+    descs = [tensor_desc(t) for t in (x, mask)]
+    outs = [tensor_desc(t) for t in (idx, bins, hist)]
+    st = library().ipa_knn_distogram(B, L, k, len(edges), *[ctypes.byref(d) for d in descs], e,
+                                     *[ctypes.byref(d) for d in outs], ctypes.c_void_p(_stream_ptr(stream)))
+    if st != 0:
+        raise IpaError(st, library().ipa_status_string(st).decode())
+    return idx, bins, hist
 
 
 # ------------------------------------------------------------------ projections

@@ -19,7 +19,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
          "--expt-relaxed-constexpr", "-Xcompiler", "-fvisibility=hidden"]
 SOURCES = ["api.cu", "ipa_prologue.cu", "ipa_attention.cu", "ipa_attention_pair.cu", "geo_kernels.cu",
-           "geo_static.cu", "meet.cu", "frames.cu", "geo_backward.cu", "linear.cu"]
+           "geo_static.cu", "meet.cu", "frames.cu", "geo_backward.cu", "linear.cu",
+           "ipa_backward.cu", "distogram.cu"]
 
 
 def nvcc() -> str:

@@ -268,6 +268,199 @@ ipa_status_t ipa_attn_fwd(const ipa_params_t* p, const ipa_tensor_t* q, const ip
   return IPA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Byte sizes of the 13 inputs and the output, in the order of ipa_attn_fwd.
+void ipa_host_sizes(const ipa_params_t* p, size_t sz[14]) {
+  const size_t B = p->B, L = p->L, H = p->H, C = p->C, Pq = p->Pq, Pv = p->Pv, R = p->R, Cz = p->Cz;
+  const size_t f = 4;
+  const size_t v[14] = {B * L * H * C * f, B * L * H * C * f, B * L * H * C * f, B * L * H * Pq * 3 * f,
+                        B * L * H * Pq * 3 * f, B * L * H * Pv * 3 * f, B * L * 9 * f, B * L * 3 * f,
+                        B * L * R * Cz * f, B * L * R * Cz * f, Cz * H * f, H * f, B * L,
+                        B * L * H * (C + 4 * Pv + Cz) * f};
+  for (int t = 0; t < 14; ++t) sz[t] = v[t];
+}
+
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool dense(const ipa_tensor_t* t) {
+  int64_t expect = 1;
+  for (int d = t->ndim - 1; d >= 0; --d) {
+    if (t->size[d] > 1 && t->stride[d] != expect) return false;
+    expect *= t->size[d];
+  }
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ipa_attn_host_staging_size(const ipa_params_t* p) {
+  ipa_status_t st;
+  if (!ipa_dims_ok(p, &st)) return 0;
+  size_t sz[14], total = 0;
+  ipa_host_sizes(p, sz);
+  for (int t = 0; t < 14; ++t) total += up256(sz[t]);
+  return total;
+}
+
+ipa_status_t ipa_attn_fwd_host(const ipa_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,
+                               const ipa_tensor_t* v, const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                               const ipa_tensor_t* v_pts, const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                               const ipa_tensor_t* z1, const ipa_tensor_t* z2, const ipa_tensor_t* w_bias,
+                               const ipa_tensor_t* gamma, const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                               void* staging, size_t staging_bytes, void* workspace, size_t workspace_bytes,
+                               void* stream, int32_t* dev_err) {
+  const ipa_tensor_t* in[14] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask, out};
+  if (out == nullptr) return IPA_ERR_NULL;
+  // shapes, dtypes and the workspace through the device entry point's checks
+  // (host pointers are only compared, never dereferenced, there)
+  IpaLaunch a;
+  ipa_status_t st = ipa_prepare(p, in, out, workspace, workspace_bytes, stream, dev_err, true, true, &a);
+  if (st != IPA_OK) return st;
+  for (int t = 0; t < 14; ++t)
+    if (!dense(in[t])) return IPA_ERR_STRIDE_ALIGN;
+  if (staging == nullptr) return IPA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(staging) % 256 != 0 || staging_bytes < ipa_attn_host_staging_size(p))
+    return IPA_ERR_WORKSPACE;
+  size_t sz[14];
+  ipa_host_sizes(p, sz);
+  unsigned char* sbase = static_cast<unsigned char*>(staging);
+  ipa_tensor_t dev[14];
+  size_t off = 0;
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  for (int t = 0; t < 14; ++t) {
+    dev[t] = *in[t];
+    dev[t].data = sbase + off;
+    if (t < 13 && cudaMemcpyAsync(sbase + off, in[t]->data, sz[t], cudaMemcpyHostToDevice, cs) != cudaSuccess)
+      return IPA_ERR_CUDA;
+    off += up256(sz[t]);
+  }
+  const ipa_tensor_t* din[13] = {&dev[0], &dev[1], &dev[2], &dev[3], &dev[4], &dev[5], &dev[6],
+                                 &dev[7], &dev[8], &dev[9], &dev[10], &dev[11], &dev[12]};
+  st = ipa_prepare(p, din, &dev[13], workspace, workspace_bytes, stream, dev_err, true, false, &a);
+  if (st != IPA_OK) return st;
+  if (ipa_launch_prologue(a, cs) != cudaSuccess || ipa_launch_core(a, cs) != cudaSuccess) return IPA_ERR_CUDA;
+  if (cudaMemcpyAsync(const_cast<void*>(out->data), dev[13].data, sz[13], cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
+ipa_status_t ipa_attn_fwd_train(const ipa_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,
+                                const ipa_tensor_t* v, const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                                const ipa_tensor_t* v_pts, const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                                const ipa_tensor_t* z1, const ipa_tensor_t* z2, const ipa_tensor_t* w_bias,
+                                const ipa_tensor_t* gamma, const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                                const ipa_tensor_t* lse, const ipa_tensor_t* u_agg, void* workspace,
+                                size_t workspace_bytes, void* stream, int32_t* dev_err) {
+  const ipa_tensor_t* in[13] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask};
+  IpaLaunch a;
+  if (out == nullptr) return IPA_ERR_NULL;
+  ipa_status_t st = ipa_prepare(p, in, out, workspace, workspace_bytes, stream, dev_err, true, true, &a);
+  if (st != IPA_OK) return st;
+  const int64_t s_l[3] = {p->B, p->H, p->L};
+  const int64_t s_u[5] = {p->B, p->L, p->H, p->R, p->Cz};
+  if (!check_contiguous_out(lse, 3, s_l, &st) || !check_contiguous_out(u_agg, 5, s_u, &st)) return st;
+  a.lse = static_cast<float*>(const_cast<void*>(lse->data));
+  a.uagg = static_cast<float*>(const_cast<void*>(u_agg->data));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ipa_launch_prologue(a, s) != cudaSuccess) return IPA_ERR_CUDA;
+  if (ipa_launch_core(a, s) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
+size_t ipa_attn_bwd_workspace_size(const ipa_params_t* p) {
+  ipa_status_t st;
+  if (!ipa_dims_ok(p, &st)) return 0;
+  return ipa_bwd_workspace_layout(p->B, p->L, p->H, pair_width(p), p->R * p->Cz).total;
+}
+
+ipa_status_t ipa_attn_bwd(const ipa_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,
+                          const ipa_tensor_t* v, const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                          const ipa_tensor_t* v_pts, const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                          const ipa_tensor_t* z1, const ipa_tensor_t* z2, const ipa_tensor_t* w_bias,
+                          const ipa_tensor_t* gamma, const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                          const ipa_tensor_t* lse, const ipa_tensor_t* u_agg, const ipa_tensor_t* g_out,
+                          const ipa_grads_t* grads, void* workspace, size_t workspace_bytes, void* stream,
+                          int32_t* dev_err) {
+  const ipa_tensor_t* in[13] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask};
+  if (grads == nullptr) return IPA_ERR_NULL;
+  ipa_status_t st = IPA_OK;
+  if (!ipa_dims_ok(p, &st)) return st;
+  const int64_t B = p->B, L = p->L, H = p->H, C = p->C, Pq = p->Pq, Pv = p->Pv, R = p->R, Cz = p->Cz;
+  const int64_t F = C + 4 * Pv + Cz;
+  const int64_t s_o[4] = {B, L, H, F};
+  const int64_t s_l[3] = {B, H, L};
+  const int64_t s_u[5] = {B, L, H, R, Cz};
+  if (!check_tensor(out, IPA_DTYPE_F32, 4, s_o, &st) || !check_tensor(lse, IPA_DTYPE_F32, 3, s_l, &st) ||
+      !check_tensor(u_agg, IPA_DTYPE_F32, 5, s_u, &st) || !check_tensor(g_out, IPA_DTYPE_F32, 4, s_o, &st))
+    return st;
+  const int64_t s_qkv[4] = {B, L, H, C}, s_qp[5] = {B, L, H, Pq, 3}, s_vp[5] = {B, L, H, Pv, 3};
+  const int64_t s_rot[4] = {B, L, 3, 3}, s_tr[3] = {B, L, 3}, s_z[4] = {B, L, R, Cz}, s_w[2] = {Cz, H};
+  const int64_t s_g[1] = {H};
+  if (!check_contiguous_out(&grads->q, 4, s_qkv, &st) || !check_contiguous_out(&grads->k, 4, s_qkv, &st) ||
+      !check_contiguous_out(&grads->v, 4, s_qkv, &st) || !check_contiguous_out(&grads->q_pts, 5, s_qp, &st) ||
+      !check_contiguous_out(&grads->k_pts, 5, s_qp, &st) || !check_contiguous_out(&grads->v_pts, 5, s_vp, &st) ||
+      !check_contiguous_out(&grads->rot, 4, s_rot, &st) || !check_contiguous_out(&grads->trans, 3, s_tr, &st) ||
+      !check_contiguous_out(&grads->z1, 4, s_z, &st) || !check_contiguous_out(&grads->z2, 4, s_z, &st) ||
+      !check_contiguous_out(&grads->w_bias, 2, s_w, &st) || !check_contiguous_out(&grads->gamma, 1, s_g, &st))
+    return st;
+  const int DZ = pair_width(p);
+  const IpaBwdWorkspace lay = ipa_bwd_workspace_layout(p->B, p->L, p->H, DZ, p->R * p->Cz);
+  if (workspace == nullptr) return IPA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
+  IpaBwdLaunch b{};
+  // inputs and the forward part of the workspace (prologue outputs) through the forward's checks
+  st = ipa_prepare(p, in, nullptr, workspace, lay.fwd.total, stream, dev_err, true, true, &b.f);
+  if (st != IPA_OK) return st;
+  b.out = view_of(out);
+  b.lse = view_of(lse);
+  b.uagg = view_of(u_agg);
+  b.g_out = view_of(g_out);
+  auto outp = [](const ipa_tensor_t& t) { return static_cast<float*>(const_cast<void*>(t.data)); };
+  b.d_q = outp(grads->q); b.d_k = outp(grads->k); b.d_v = outp(grads->v);
+  b.d_q_pts = outp(grads->q_pts); b.d_k_pts = outp(grads->k_pts); b.d_v_pts = outp(grads->v_pts);
+  b.d_rot = outp(grads->rot); b.d_trans = outp(grads->trans); b.d_z1 = outp(grads->z1); b.d_z2 = outp(grads->z2);
+  b.d_w_bias = outp(grads->w_bias); b.d_gamma = outp(grads->gamma);
+  b.lay = lay;
+  if (ipa_launch_bwd(b, static_cast<cudaStream_t>(stream)) != cudaSuccess) return IPA_ERR_CUDA;
+  return IPA_OK;
+}
+
+ipa_status_t ipa_knn_distogram(int32_t B, int32_t L, int32_t k, int32_t n_edges, const ipa_tensor_t* x,
+                               const ipa_tensor_t* mask, const float* edges, const ipa_tensor_t* idx,
+                               const ipa_tensor_t* bins, const ipa_tensor_t* hist, void* stream) {
+  if (B < 1 || L < 1 || k < 1 || n_edges < 0) return IPA_ERR_SHAPE;
+  if (k > DIST_MAX_K || n_edges > DIST_MAX_EDGES || L > (1 << 24) || static_cast<int64_t>(B) * L > (int64_t{1} << 31))
+    return IPA_ERR_UNSUPPORTED;
+  if (n_edges > 0 && edges == nullptr) return IPA_ERR_NULL;
+  for (int m = 0; m < n_edges; ++m)
+    if (!(edges[m] >= 0.f) || (m > 0 && !(edges[m] > edges[m - 1]))) return IPA_ERR_SHAPE;
+  ipa_status_t st = IPA_OK;
+  const int64_t s_x[3] = {B, L, 3}, s_m[2] = {B, L}, s_k[3] = {B, L, k}, s_h[3] = {B, L, n_edges + 1};
+  if (!check_tensor(x, IPA_DTYPE_F32, 3, s_x, &st) || !check_tensor(mask, IPA_DTYPE_BOOL, 2, s_m, &st)) return st;
+  auto check_i32_out = [&](const ipa_tensor_t* t) {
+    if (t == nullptr || t->data == nullptr) { st = IPA_ERR_NULL; return false; }
+    if (t->dtype != IPA_DTYPE_I32) { st = IPA_ERR_DTYPE; return false; }
+    ipa_tensor_t f = *t;
+    f.dtype = IPA_DTYPE_F32;                 // same size and alignment rules as an fp32 output
+    return check_contiguous_out(&f, 3, s_k, &st);
+  };
+  if (!check_i32_out(idx) || !check_i32_out(bins) || !check_contiguous_out(hist, 3, s_h, &st)) return st;
+  DistogramArgs a{};
+  a.B = B; a.L = L; a.k = k; a.nb = n_edges + 1;
+  a.x = view_of(x);
+  a.mask = view_of(mask);
+  for (int m = 0; m < n_edges; ++m) a.edge2[m] = edges[m] * edges[m];
+  a.idx = static_cast<int32_t*>(const_cast<void*>(idx->data));
+  a.bins = static_cast<int32_t*>(const_cast<void*>(bins->data));
+  a.hist = static_cast<float*>(const_cast<void*>(hist->data));
+  return distogram_launch(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? IPA_OK : IPA_ERR_CUDA;
+}
+
 size_t meet_attn_workspace_size(const meet_params_t* p) {
   if (p == nullptr || p->B < 1 || p->L < 1 || p->H < 1 || p->C != MEET_C || p->H > 128 || p->L > (1 << 20) ||
       static_cast<int64_t>(p->B) * p->H * p->L > (int64_t{1} << 31) / 64)

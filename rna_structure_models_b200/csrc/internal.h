@@ -35,6 +35,11 @@ struct IpaLaunch {
   float w_L, w_C, scalar_scale;
   View q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask;
   float* out;
+  // training forward only (else null): log-sum-exp of the logits per (b, h, i)
+  // in natural-log units (+inf for rows without an allowed key), [B, H, L];
+  // pair aggregate U_i = sum_j a_ij z2_j, [B, L, H, R Cz]
+  float* lse = nullptr;
+  float* uagg = nullptr;
   unsigned char* ws;
   IpaWorkspace lay;
   int* err;
@@ -43,6 +48,35 @@ struct IpaLaunch {
 // Stage launches; each returns the cudaError_t of its last launch.
 cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream);
 cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream);
+
+// Gradients of the IPA core (ipa_backward.cu).  The workspace holds the
+// forward prologue's outputs (recomputed) followed by the backward's.
+struct IpaBwdWorkspace {
+  IpaWorkspace fwd;
+  size_t doh, du, qp, rowd, dqh, dqp, rsq, dkh, dva, dz2, csk, wb_part, g_part, total;
+};
+IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz);
+
+struct IpaBwdLaunch {
+  IpaLaunch f;                 // forward inputs; f.ws / f.lay point at the backward workspace
+  View out, lse, uagg, g_out;  // forward output [B,L,H,F], lse [B,H,L], U [B,L,H,R,Cz], upstream [B,L,H,F]
+  // gradients (contiguous fp32, shapes of the inputs)
+  float *d_q, *d_k, *d_v, *d_q_pts, *d_k_pts, *d_v_pts, *d_rot, *d_trans, *d_z1, *d_z2, *d_w_bias, *d_gamma;
+  IpaBwdWorkspace lay;
+};
+cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream);
+
+// Local nearest-neighbour distogram (distogram.cu).
+constexpr int DIST_MAX_K = 32, DIST_MAX_EDGES = 63;
+struct DistogramArgs {
+  int B, L, k, nb;                 // nb = number of edges + 1
+  View x, mask;                    // [B, L, 3] f32, [B, L] u8
+  float edge2[DIST_MAX_EDGES];     // squared edges (float32 products)
+  int32_t* idx;                    // [B, L, k]
+  int32_t* bins;                   // [B, L, k]
+  float* hist;                     // [B, L, nb]
+};
+cudaError_t distogram_launch(const DistogramArgs& a, cudaStream_t stream);
 
 // Distance-aware attention (MEET) on the IPA core: C = 16, Pq = 4, Pv = 8,
 // one 16-channel pair factor (DZ = 64), output row F = 64.

@@ -316,9 +316,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     {
       const float4* zr = reinterpret_cast<const float4*>(a.z1f + (static_cast<int64_t>(b) * L + (in_range ? row : 0)) * DZ);
       const float4* wr = reinterpret_cast<const float4*>(a.wqp + static_cast<int64_t>(h) * DZ);
-      const int c_lo = half * (DZ / 4), c_hi = c_lo + DZ / 4;   // packed columns of this half
+      // 32-column chunks of the DZ / 2 packed columns, alternating between the
+      // two halves (every chunk lies inside the row's DZ pair factors)
       float qmax = 0.f;   // largest |Q_pair| before rounding (NaN if any is NaN)
-      for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+      for (int c0 = 32 * half; c0 < DZ / 2; c0 += 64) {
         uint32_t rg[32];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {

@@ -553,6 +553,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     // constant c sum_p |gq'_p|^2 (rowq.w) out of its logits
     if (a.lse != nullptr && half == 0 && in_range)
       a.lse[static_cast<int64_t>(bh) * L + row] = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
+    // direct output pass when the pair block has no padding and whole
+    // 64-column factors (the staged pass below handles every other shape)
+    if (a.RCz == DZ && (a.Cz & 63) == 0) {
+      if (all_ok && !*abort_flag) {
+        tc_fence_after();
+        const float inv = dead ? 0.f : 1.f / lt;
+        const int rrow = in_range ? row : 0;
+        const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
+        write_row_direct<IPA_C, IPA_PV>(tmem + lane_off, half, DZ, a.Cz, a.RCz / a.Cz, inv, dead, in_range,
+                                        a.z1f + (static_cast<int64_t>(b) * L + rrow) * DZ, a.out + orow * a.F,
+                                        a.uagg != nullptr ? a.uagg + orow * a.RCz : nullptr, g0, g1, g2, cn);
+      }
+    } else {
     const int pitch = stage_pitch(DZ);
     float* stage = reinterpret_cast<float*>(smem + SP_QP);
     if (all_ok) {
@@ -583,6 +596,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       ea.trace = (blockIdx.x < 4096 && warp == 0) ? &g_pair_span[blockIdx.x][16] : nullptr;
 #endif
       write_rows<IPA_C, IPA_PV>(ea, warp, lane);
+    }
     }
   }
 

@@ -1,0 +1,1171 @@
+// Gradients of the fused IPA core on sm_100a (Flash Invariant Point
+// Attention is a drop-in replacement for IPA in training: TL;DR, Abstract,
+// Figure 3).  Flash-style recomputation on the augmented operands of the
+// forward pass; no L x L array is stored.
+//
+// Notation (log2 units, per batch b and head h): x_ij = log2(e) l_ij is the
+// true logit, recomputed exactly as the forward pass computed it:
+//   x_ij = Q_h,i . K_h,j + Q_pair,i . Z2_j + col_j(I) + rt_i(J) - w_i
+// with the forward prologue's rows (Q_h unscaled tile-local query points,
+// K_h 2c-scaled tile-local key points, V_h centroid-relative value points),
+// col / rt the per-key / per-row tile-origin terms and w_i = c |gq'_i|^2 the
+// row constant the forward pass leaves out.  With lse2_i the training
+// forward's log-sum-exp (log2 units), p_ij = 2^(x_ij - lse2_i) = a_ij and
+//   dP_ij = dO_i . V_h,j + dU_i . Z2_j     dO_i = [g_o | R_i d_opt | R_i d_opt],
+//                                          dU_i = z1_i (.) g_pair_i
+//   dS_ij = ln 2 p_ij (dP_ij - D_i)        D_i = sum_j p_ij dP_ij, from the
+//                                          forward output and U
+// dS is dL/dx.  The kernels:
+//   ipa_bwd_rows_kernel  one warp per (b, i, h): dO, dU, Q_pair (fp16 rows),
+//                        the row constant -(w_i + lse2_i) and D_i;
+//   ipa_bwd_q_kernel     one CTA per (b, h, 128 queries), 64-key tiles:
+//                        S, dP (tcgen05, TMEM), dS (fp16, TMEM), then
+//                        dQ_h += dS K_h, dQ_pair += dS Z2 (A = dS from TMEM),
+//                        row sums rs_i = sum_j dS_ij, RSo_i = sum_j dS_ij o_J;
+//   ipa_bwd_k_kernel     one CTA per (b, h, 128 keys), 64-query tiles:
+//                        S^T, dP^T, then P^T and dS^T (fp16, in place in
+//                        TMEM) as A operands of dV += P^T dO,
+//                        dZ2 += P^T dU + dS^T Q_pair, dK_h += dS^T Q_h, column
+//                        sums cs_j, CSo_j = sum_i dS_ij o_I;
+//   ipa_bwd_map_kernel   per residue, all heads: the augmented gradients
+//                        mapped back to q, k, v, the local points, the frames,
+//                        z1, z2 (sums over heads) and per-block partial sums of
+//                        d w_bias and d gamma;
+//   ipa_bwd_reduce_kernel  fixed-order sums of those partials.
+// Every mbarrier wait is bounded (2 s) and reports into the error word.
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fipa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.69314718055994531f;
+
+struct BwdArgs {
+  int B, L, H, DZ, RCz, Cz, R, nqt, nkt, ns;
+  float qscale, w_L, w_C;
+  // forward prologue outputs (workspace)
+  const float4* rowq;    // [B*H, L] (sum_p gq', c |gq'|^2)
+  const float4* colk;    // [B*H, L] (2c sum_p gk', 0 or -inf)
+  const float4* oq;      // [B, nqt] 128-row tile origins
+  const float4* ok;      // [B, nkt] 64-row tile origins
+  const float4* cen;     // [B]
+  const float* headc;    // [H] c = log2(e) w_L gamma w_C / 2
+  const float* wqp;      // [H, DZ] log2(e) w_L w_bias
+  const float4* frame;   // [B, L, 4]
+  const float* z1f;      // [B, L, DZ]
+  const __half* z1h;     // [B, L, DZ]
+  // backward prologue outputs
+  const float2* rowd;    // [B*H, L] (-(w + lse2), D)
+  // pass outputs
+  float* dqh;            // [B*H, L, 64]
+  float* dqp;            // [B*H, L, DZ]
+  float4* rsq;           // [B*H, L] (rs, RSo)
+  float* dkh;            // [B*H, L, 64]
+  float* dva;            // [B*H, L, 64]
+  float* dz2;            // [B*H, L, DZ]
+  float4* csk;           // [B*H, L] (cs, CSo)
+  int* err;
+};
+
+__device__ __forceinline__ uint64_t kd128(uint32_t a) { return smem_desc(a, 16, 1024, 2); }      // K-major SW128
+__device__ __forceinline__ uint64_t mnd(uint32_t a, uint32_t panel) { return smem_desc(a, panel, 1024, 2); }  // MN-major SW128
+
+__device__ __forceinline__ float ldf(const View& v, int64_t off) {
+  return v.dtype == 1 ? static_cast<float>(reinterpret_cast<const double*>(v.p)[off])
+                      : reinterpret_cast<const float*>(v.p)[off];
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      SM100_W16(r, 0)
+      : "memory");
+}
+
+// ------------------------------------------------------------------ prologue
+struct RowsArgs {
+  int B, L, H, DZ, RCz, Cz, F;
+  bool z1_half;          // Q_pair from the fp16 z1 (as the CTA-pair forward core), else from fp32 z1
+  View g_out, out, lse, uagg;
+  const float4* frame;
+  const float4* cen;
+  const float4* rowq;
+  const float* wqp;
+  const float* z1f;
+  const __half* z1h;
+  __half* doh;           // [B*H, L, 64]
+  __half* du;            // [B*H, L, DZ]
+  __half* qp;            // [B*H, L, DZ]
+  float2* rowd;          // [B*H, L]
+};
+
+// One warp per (b, i, h), heads fastest.  Lane l: scalar channel l (< 16),
+// point coordinate l (< 24: point l / 3, axis l % 3), pair columns l + 32 k.
+__global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= static_cast<int64_t>(a.B) * a.L * a.H) return;
+  const int h = static_cast<int>(wid % a.H);
+  const int64_t bi = wid / a.H;
+  const int i = static_cast<int>(bi % a.L), b = static_cast<int>(bi / a.L);
+  const int64_t bhl = (static_cast<int64_t>(b) * a.H + h) * a.L + i;
+  const float4* fr = a.frame + bi * 4;
+  const float4 f0 = fr[0], f1 = fr[1], f2 = fr[2], f3 = fr[3];
+  const bool live = f3.x != 0.f;
+  const int C = IPA_C, PV = IPA_PV;
+  const int64_t gbase = b * a.g_out.s[0] + i * a.g_out.s[1] + h * a.g_out.s[2];
+  const int64_t obase = b * a.out.s[0] + i * a.out.s[1] + h * a.out.s[2];
+  float part = 0.f;   // this lane's share of D_i
+  // scalar channels
+  float g_o = 0.f;     // rounded to fp16 as the dP MMA sees it, in D too
+  if (lane < C && live) {
+    g_o = __half2float(__float2half_rn(ldf(a.g_out, gbase + lane * a.g_out.s[3])));
+    part = g_o * ldf(a.out, obase + lane * a.out.s[3]);
+  }
+  // value points: d_opt = g_pt + g_n unit(o_pt), dog = R d_opt (global frame)
+  const int l = lane < 3 * PV ? lane : 0;
+  const int x = l % 3, p3 = l - x;
+  float opt = 0.f, gpt = 0.f, gn = 0.f;
+  if (live) {
+    opt = ldf(a.out, obase + (C + l) * a.out.s[3]);
+    gpt = ldf(a.g_out, gbase + (C + l) * a.g_out.s[3]);
+    gn = ldf(a.g_out, gbase + (C + 3 * PV + l / 3) * a.g_out.s[3]);
+  }
+  const float o0 = __shfl_sync(0xffffffffu, opt, p3), o1 = __shfl_sync(0xffffffffu, opt, p3 + 1),
+              o2 = __shfl_sync(0xffffffffu, opt, p3 + 2);
+  const float nrm = sqrtf(o0 * o0 + o1 * o1 + o2 * o2);
+  const float dopt = gpt + (nrm > 0.f ? gn * opt / nrm : 0.f);
+  const float d0 = __shfl_sync(0xffffffffu, dopt, p3), d1 = __shfl_sync(0xffffffffu, dopt, p3 + 1),
+              d2 = __shfl_sync(0xffffffffu, dopt, p3 + 2);
+  const float Rm[9] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w, f2.x};
+  const float4 cn = a.cen[b];
+  const float tc[3] = {f2.y - cn.x, f2.z - cn.y, f2.w - cn.z};
+  const float dog = fmaf(Rm[3 * x], d0, fmaf(Rm[3 * x + 1], d1, Rm[3 * x + 2] * d2));
+  const float dog16 = __half2float(__float2half_rn(dog));
+  const float og = fmaf(Rm[3 * x], o0, fmaf(Rm[3 * x + 1], o1, Rm[3 * x + 2] * o2)) + tc[x];   // og - centroid
+  if (lane < 3 * PV && live) part = fmaf(dog16, og, part);
+  // dO row: column l and 32 + l; dog coordinate e is held by lane e
+  const float dg_a = __shfl_sync(0xffffffffu, dog16, (lane - 16) & 31);   // col l = 16 + e, e = l - 16
+  const float dg_b = __shfl_sync(0xffffffffu, dog16, lane < 8 ? lane + 16 : lane - 8);
+  const float c_lo = lane < C ? g_o : dg_a;
+  const float c_hi = dg_b;                 // col 32 + l: l < 8 -> dog[16 + l], else dog[l - 8]
+  __half* drow = a.doh + bhl * 64;
+  drow[lane] = __float2half_rn(live ? c_lo : 0.f);
+  drow[32 + lane] = __float2half_rn(live ? c_hi : 0.f);
+  // pair block: dU = z1 (.) g_pair (fp16), Q_pair = fp16(w_qp z1), D += dU . U
+  const float* z1r = a.z1f + bi * a.DZ;
+  const __half* z1hr = a.z1h + bi * a.DZ;
+  const float* wr = a.wqp + static_cast<int64_t>(h) * a.DZ;
+  __half* dur = a.du + bhl * a.DZ;
+  __half* qpr = a.qp + bhl * a.DZ;
+  const int64_t ubase = b * a.uagg.s[0] + i * a.uagg.s[1] + h * a.uagg.s[2];
+  for (int c = lane; c < a.DZ; c += 32) {
+    float duv = 0.f;
+    if (c < a.RCz && live) {
+      const int r = c / a.Cz, cc = c % a.Cz;
+      const float gp = ldf(a.g_out, gbase + (C + 4 * PV + cc) * a.g_out.s[3]);
+      const __half d16 = __float2half_rn(z1r[c] * gp);
+      duv = __half2float(d16);
+      part = fmaf(duv, ldf(a.uagg, ubase + r * a.uagg.s[3] + cc * a.uagg.s[4]), part);
+    }
+    dur[c] = __float2half_rn(duv);
+    const float zq = a.z1_half ? __half2float(z1hr[c]) : z1r[c];
+    qpr[c] = __float2half_rn(zq * wr[c]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+  if (lane == 0) {
+    float rowc = -INFINITY, D = 0.f;
+    if (live) {
+      const float lse = ldf(a.lse, b * a.lse.s[0] + h * a.lse.s[1] + i * a.lse.s[2]);
+      rowc = -(a.rowq[bhl].w + lse * kLog2e);
+      D = part;
+    }
+    a.rowd[bhl] = make_float2(rowc, D);
+  }
+}
+
+// --------------------------------------------------------------- query pass
+// Warps 0-7: two threads per query row (keys [32 half, 32 half + 32) of a
+// tile); warp 8: TMA producer and the per-key column terms; warp 9: tensor
+// memory and the MMA-issuing thread.
+constexpr int NTH = 320, NSOFT = 256, W_PROD = 8, W_MMA = 9;
+constexpr int MAX_NS = 3;
+
+// tensor memory (512 columns)
+constexpr uint32_t Q_TM_DQP = 0, Q_TM_DQH = 256, Q_TM_S = 320, Q_TM_DP = 384, Q_TM_DS = 448;
+
+struct QLayout {
+  uint32_t qh, qp, dO, du, stg, stg_bytes, aux, total;
+};
+__host__ __device__ inline QLayout q_layout(int DZ, int ns) {
+  QLayout s{};
+  const uint32_t np = DZ / 64;
+  s.qh = 0;
+  s.qp = 16384;
+  s.dO = s.qp + np * 16384;
+  s.du = s.dO + 16384;
+  s.stg = s.du + np * 16384;
+  s.stg_bytes = 16384 + np * 8192;          // K_h 8 KB | V_h 8 KB | Z2 np x 8 KB
+  s.aux = s.stg + ns * s.stg_bytes;
+  s.total = s.aux + 2048;
+  return s;
+}
+// aux area: col terms [MAX_NS][64] floats (768 B) | tile info [MAX_NS][2] float4 (96 B) | barriers
+constexpr uint32_t QA_COL = 0, QA_INFO = 768, QA_BAR = 896;
+enum { QB_QFULL = 0, QB_SFULL, QB_SFREE, QB_DSFULL, QB_DSFREE, QB_DRAIN, QB_FULL0, QB_EMPTY0 = QB_FULL0 + MAX_NS,
+       QB_COUNT = QB_EMPTY0 + MAX_NS };
+constexpr uint32_t QA_TMEM = QA_BAR + 8 * QB_COUNT, QA_ABORT = QA_TMEM + 8;
+
+__global__ void __launch_bounds__(NTH, 1)
+    ipa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_qp,
+                     const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_du,
+                     const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
+                     const __grid_constant__ CUtensorMap tm_z2, const BwdArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (sb - raw_u32);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int I = blockIdx.x % a.nqt;
+  const int bh = blockIdx.x / a.nqt;
+  const int b = bh / a.H, h = bh % a.H;
+  const int L = a.L, nt = a.nkt, DZ = a.DZ, np = DZ / 64, NS = a.ns;
+  const QLayout lay = q_layout(DZ, NS);
+  float* col_s = reinterpret_cast<float*>(smem + lay.aux + QA_COL);
+  float4* info = reinterpret_cast<float4*>(smem + lay.aux + QA_INFO);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + lay.aux + QA_ABORT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + lay.aux + QA_TMEM);
+  auto bar = [&](int k) -> uint32_t { return sb + lay.aux + QA_BAR + 8u * k; };
+
+  if (tid == 0) {
+    mbar_init(bar(QB_QFULL), 1);
+    mbar_init(bar(QB_SFULL), 1);
+    mbar_init(bar(QB_SFREE), NSOFT);
+    mbar_init(bar(QB_DSFULL), NSOFT);
+    mbar_init(bar(QB_DSFREE), 1);
+    mbar_init(bar(QB_DRAIN), 1);
+    for (int s = 0; s < MAX_NS; ++s) {
+      mbar_init(bar(QB_FULL0 + s), 1);
+      mbar_init(bar(QB_EMPTY0 + s), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == W_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&](int code) {
+    record_error(a.err, code);
+    *abort_flag = 1;
+  };
+
+  if (warp == W_PROD) {
+    const float4 oqv = a.oq[b * a.nqt + I];
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(QB_QFULL), 2u * 16384u * static_cast<uint32_t>(1 + np));
+      tma_load_3d(sb + lay.qh, &tm_qh, bar(QB_QFULL), 0, I * QT, bh);
+      tma_load_4d(sb + lay.qp, &tm_qp, bar(QB_QFULL), 0, I * QT, 0, bh);
+      tma_load_3d(sb + lay.dO, &tm_do, bar(QB_QFULL), 0, I * QT, bh);
+      tma_load_4d(sb + lay.du, &tm_du, bar(QB_QFULL), 0, I * QT, 0, bh);
+    }
+    int issued = 0;
+    for (int j = 0; j < nt; ++j) {
+      const int s = j % NS;
+      if (j >= NS) {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait_bounded(bar(QB_EMPTY0 + s), ((j / NS) - 1) & 1, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) fail(DEV_TIMEOUT_EMPTY);
+          break;
+        }
+      }
+      issued = j + 1;
+      const float4 okv = a.ok[b * nt + j];
+      const float dx = okv.x - oqv.x, dy = okv.y - oqv.y, dz = okv.z - oqv.z;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int key = j * KT + lane + 32 * t;
+        float cv = -INFINITY;
+        if (key < L) {
+          const float4 ck = a.colk[static_cast<int64_t>(bh) * L + key];
+          cv = ck.w - fmaf(ck.x, dx, fmaf(ck.y, dy, ck.z * dz));
+        }
+        col_s[s * 64 + lane + 32 * t] = cv;
+      }
+      if (lane == 0) {
+        info[2 * s] = make_float4(dx, dy, dz, fmaf(dx, dx, fmaf(dy, dy, dz * dz)));
+        info[2 * s + 1] = okv;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+        mbar_arrive_expect_tx(bar(QB_FULL0 + s), lay.stg_bytes);
+        tma_load_3d(st, &tm_kh, bar(QB_FULL0 + s), 0, j * KT, bh);
+        tma_load_3d(st + 8192, &tm_vh, bar(QB_FULL0 + s), 0, j * KT, bh);
+        tma_load_4d(st + 16384, &tm_z2, bar(QB_FULL0 + s), 0, j * KT, 0, b);
+      }
+      __syncwarp();
+    }
+    if (lane == 0 && *abort_flag) {
+      // copies still in flight must land before the CTA exits
+      mbar_wait_bounded(bar(QB_QFULL), 0, nullptr, 100000000ull);
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+        mbar_wait_bounded(bar(QB_FULL0 + j % NS), (j / NS) & 1, nullptr, 100000000ull);
+    }
+  } else if (warp == W_MMA) {
+    if (lane == 0) {
+      bool ok = mbar_wait_bounded(bar(QB_QFULL), 0, abort_flag);
+      if (!ok) fail(DEV_TIMEOUT_FULL);
+      tc_fence_after();
+      const uint32_t id64 = idesc_f16(128, 64, false);
+      const uint32_t id64mn = idesc_f16(128, 64, true);
+      const uint32_t idz = idesc_f16(128, DZ, true);
+      const uint32_t tS = tmem + Q_TM_S, tDP = tmem + Q_TM_DP, tDS = tmem + Q_TM_DS;
+      const uint32_t tDQH = tmem + Q_TM_DQH, tDQP = tmem + Q_TM_DQP;
+      bool issued_any = false;
+      auto issue_sdp = [&](int j) -> bool {
+        const int s = j % NS;
+        bool w = mbar_wait_bounded(bar(QB_FULL0 + s), (j / NS) & 1, abort_flag);
+        if (w && j > 0) w = mbar_wait_bounded(bar(QB_SFREE), (j - 1) & 1, abort_flag);
+        if (!w) { fail(DEV_TIMEOUT_FULL); return false; }
+        tc_fence_after();
+        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.qh + 32 * k), kd128(st + 32 * k), id64, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4 * np; ++kk)
+          umma_ss(tS, kd128(sb + lay.qp + 16384 * (kk >> 2) + 32 * (kk & 3)),
+                  kd128(st + 16384 + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, 1u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_ss(tDP, kd128(sb + lay.dO + 32 * k), kd128(st + 8192 + 32 * k), id64, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4 * np; ++kk)
+          umma_ss(tDP, kd128(sb + lay.du + 16384 * (kk >> 2) + 32 * (kk & 3)),
+                  kd128(st + 16384 + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, 1u);
+        umma_commit(bar(QB_SFULL));
+        issued_any = true;
+        return true;
+      };
+      auto issue_dq = [&](int jj) -> bool {
+        if (!mbar_wait_bounded(bar(QB_DSFULL), jj & 1, abort_flag)) { fail(DEV_TIMEOUT_SOFTMAX); return false; }
+        tc_fence_after();
+        const int s = jj % NS;
+        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
+          umma_ts(tDQH, tDS + 8 * k, mnd(st + 2048 * k, 8192), id64mn, acc);
+          umma_ts(tDQP, tDS + 8 * k, mnd(st + 16384 + 2048 * k, 8192), idz, acc);
+        }
+        umma_commit(bar(QB_DSFREE));
+        umma_commit(bar(QB_EMPTY0 + s));
+        return true;
+      };
+      // With one stage, dQ(j-1) must release the stage before tile j can
+      // load; with more, S(j) and dP(j) run while the threads work on j-1.
+      for (int j = 0; ok && j <= nt; ++j) {
+        if (NS == 1) {
+          if (j > 0) ok = issue_dq(j - 1);
+          if (ok && j < nt) ok = issue_sdp(j);
+        } else {
+          if (j < nt) ok = issue_sdp(j);
+          if (ok && j > 0) ok = issue_dq(j - 1);
+        }
+      }
+      if (!ok && issued_any) {
+        umma_commit(bar(QB_DRAIN));
+        mbar_wait_bounded(bar(QB_DRAIN), 0, nullptr, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const int row = I * QT + r;
+    const bool in_range = row < L;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float ch = a.headc[h];
+    const float4 sq = in_range ? a.rowq[static_cast<int64_t>(bh) * L + row] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float2 rd = in_range ? a.rowd[static_cast<int64_t>(bh) * L + row] : make_float2(-INFINITY, 0.f);
+    const float pq = static_cast<float>(IPA_PQ);
+    float rs = 0.f, ro0 = 0.f, ro1 = 0.f, ro2 = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt && ok; ++j) {
+      const int s = j % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(QB_SFULL), j & 1, abort_flag))) {
+        if (lane == 0) fail(DEV_TIMEOUT_MMA);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[32], dv[32];
+      tmem_ld32(tmem + Q_TM_S + 32 * half + lane_off, sv);
+      tmem_ld32(tmem + Q_TM_DP + 32 * half + lane_off, dv);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(QB_SFREE));
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(QB_FULL0 + s), (j / NS) & 1, abort_flag))) {
+        if (lane == 0) fail(DEV_TIMEOUT_FULL);
+        ok = false;
+        break;
+      }
+      const float4 dd = info[2 * s], oj = info[2 * s + 1];
+      const float rt = ch * (2.f * fmaf(sq.x, dd.x, fmaf(sq.y, dd.y, sq.z * dd.z)) - pq * dd.w);
+      const float base = rt + rd.x;                        // row terms - (w + lse2); -inf on dead rows
+      const float* cv = col_s + s * 64 + 32 * half;
+      uint32_t pk[16];
+      float tsum = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float x0 = __uint_as_float(sv[2 * k]) + cv[2 * k] + base;
+        const float x1 = __uint_as_float(sv[2 * k + 1]) + cv[2 * k + 1] + base;
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        const float g0 = p0 * (__uint_as_float(dv[2 * k]) - rd.y) * kLn2;
+        const float g1 = p1 * (__uint_as_float(dv[2 * k + 1]) - rd.y) * kLn2;
+        pk[k] = pack_half2(g0, g1);
+        tsum = add_half2_to_f32(pk[k], tsum);
+      }
+      rs += tsum;
+      ro0 = fmaf(tsum, oj.x, ro0);
+      ro1 = fmaf(tsum, oj.y, ro1);
+      ro2 = fmaf(tsum, oj.z, ro2);
+      // dQ(j-1) must have finished reading dS(j-1)
+      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(QB_DSFREE), (j - 1) & 1, abort_flag))) {
+        if (lane == 0) fail(DEV_TIMEOUT_MMA);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st16(tmem + Q_TM_DS + 16 * half + lane_off, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(QB_DSFULL));
+    }
+    if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(QB_DSFREE), (nt - 1) & 1, abort_flag))) {
+      if (lane == 0) fail(DEV_TIMEOUT_MMA);
+      ok = false;
+    }
+    const bool all_ok = __all_sync(0xffffffffu, ok);
+    // row sums of the two halves
+    // (the first stage's area is free: every MMA that read it has completed)
+    named_bar_sync(1, NSOFT);
+    if (half == 1) reinterpret_cast<float4*>(smem + lay.stg)[r] = make_float4(rs, ro0, ro1, ro2);
+    named_bar_sync(1, NSOFT);
+    if (all_ok && !*abort_flag) {
+      tc_fence_after();
+      if (half == 0 && in_range) {
+        const float4 o = reinterpret_cast<const float4*>(smem + lay.stg)[r];
+        a.rsq[static_cast<int64_t>(bh) * L + row] = make_float4(rs + o.x, ro0 + o.y, ro1 + o.z, ro2 + o.w);
+      }
+      // accumulators: dQ_h (64 columns, 32 per half) and dQ_pair (DZ, DZ / 2 per half)
+      {
+        uint32_t v[32];
+        tmem_ld32(tmem + Q_TM_DQH + 32 * half + lane_off, v);
+        tmem_ld_wait();
+        if (in_range) {
+          float4* dst = reinterpret_cast<float4*>(a.dqh + (static_cast<int64_t>(bh) * L + row) * 64 + 32 * half);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+      }
+      for (int c0 = half * (DZ / 2); c0 < (half + 1) * (DZ / 2); c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + Q_TM_DQP + c0 + lane_off, v);
+        tmem_ld_wait();
+        if (in_range) {
+          float4* dst = reinterpret_cast<float4*>(a.dqp + (static_cast<int64_t>(bh) * L + row) * DZ + c0);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == W_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------- key pass
+// Warps 0-7: two threads per key row (queries [32 half, 32 half + 32) of a
+// 64-query tile); warp 8: TMA producer and the per-query terms; warp 9: MMA.
+constexpr uint32_t K_TM_DZ2 = 0, K_TM_DKH = 256, K_TM_DVA = 320, K_TM_S = 384, K_TM_DP = 448;
+
+struct KLayout {
+  uint32_t kh, vh, z2, stg, stg_bytes, aux, total;
+};
+__host__ __device__ inline KLayout k_layout(int DZ, int ns) {
+  KLayout s{};
+  const uint32_t np = DZ / 64;
+  s.kh = 0;
+  s.vh = 16384;
+  s.z2 = 32768;
+  s.stg = s.z2 + np * 16384;
+  s.stg_bytes = 16384 + 2 * np * 8192;      // Q_h 8 KB | dO 8 KB | Q_pair np x 8 KB | dU np x 8 KB
+  s.aux = s.stg + ns * s.stg_bytes;
+  s.total = s.aux + 4096;
+  return s;
+}
+// aux: per-query terms [MAX_NS][64] float4 (3 KB) | stage query-tile origin [MAX_NS] float4 | barriers
+constexpr uint32_t KA_Q = 0, KA_OQ = 3072, KA_BAR = 3136;
+enum { KB_KFULL = 0, KB_SFULL, KB_PFULL, KB_ACC, KB_DRAIN, KB_FULL0, KB_EMPTY0 = KB_FULL0 + MAX_NS,
+       KB_COUNT = KB_EMPTY0 + MAX_NS };
+constexpr uint32_t KA_TMEM = KA_BAR + 8 * KB_COUNT, KA_ABORT = KA_TMEM + 8, KA_PAIR = KA_ABORT + 8;
+
+__global__ void __launch_bounds__(NTH, 1)
+    ipa_bwd_k_kernel(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
+                     const __grid_constant__ CUtensorMap tm_z2, const __grid_constant__ CUtensorMap tm_qh,
+                     const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_qp,
+                     const __grid_constant__ CUtensorMap tm_du, const BwdArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (sb - raw_u32);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nkp = (a.L + 127) / 128;
+  const int J2 = blockIdx.x % nkp;              // 128-key tile
+  const int bh = blockIdx.x / nkp;
+  const int b = bh / a.H, h = bh % a.H;
+  const int L = a.L, DZ = a.DZ, np = DZ / 64, NS = a.ns;
+  const int nq = (L + 63) / 64;                 // 64-query tiles
+  const KLayout lay = k_layout(DZ, NS);
+  float4* qinfo = reinterpret_cast<float4*>(smem + lay.aux + KA_Q);
+  float4* oqs = reinterpret_cast<float4*>(smem + lay.aux + KA_OQ);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + lay.aux + KA_ABORT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + lay.aux + KA_TMEM);
+  auto bar = [&](int k) -> uint32_t { return sb + lay.aux + KA_BAR + 8u * k; };
+
+  if (tid == 0) {
+    mbar_init(bar(KB_KFULL), 1);
+    mbar_init(bar(KB_SFULL), 1);
+    mbar_init(bar(KB_PFULL), NSOFT);
+    mbar_init(bar(KB_ACC), 1);
+    mbar_init(bar(KB_DRAIN), 1);
+    for (int s = 0; s < MAX_NS; ++s) {
+      mbar_init(bar(KB_FULL0 + s), 1);
+      mbar_init(bar(KB_EMPTY0 + s), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == W_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&](int code) {
+    record_error(a.err, code);
+    *abort_flag = 1;
+  };
+
+  if (warp == W_PROD) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(KB_KFULL), 2u * 16384u + static_cast<uint32_t>(np) * 16384u);
+      tma_load_3d(sb + lay.kh, &tm_kh, bar(KB_KFULL), 0, J2 * 128, bh);
+      tma_load_3d(sb + lay.vh, &tm_vh, bar(KB_KFULL), 0, J2 * 128, bh);
+      tma_load_4d(sb + lay.z2, &tm_z2, bar(KB_KFULL), 0, J2 * 128, 0, b);
+    }
+    const float ch = a.headc[h];
+    const float pq = static_cast<float>(IPA_PQ);
+    const int js0 = 2 * J2, js1 = 2 * J2 + 1;   // the two 64-key origin tiles of this CTA
+    const float4 ok0 = a.ok[b * a.nkt + js0];
+    const float4 ok1 = js1 < a.nkt ? a.ok[b * a.nkt + js1] : ok0;
+    int issued = 0;
+    for (int i = 0; i < nq; ++i) {
+      const int s = i % NS;
+      if (i >= NS) {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait_bounded(bar(KB_EMPTY0 + s), ((i / NS) - 1) & 1, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) fail(DEV_TIMEOUT_EMPTY);
+          break;
+        }
+      }
+      issued = i + 1;
+      const int Iq = (i * 64) / QT;
+      const float4 oqv = a.oq[b * a.nqt + Iq];
+      const float d0x = ok0.x - oqv.x, d0y = ok0.y - oqv.y, d0z = ok0.z - oqv.z;
+      const float d1x = ok1.x - oqv.x, d1y = ok1.y - oqv.y, d1z = ok1.z - oqv.z;
+      const float n0 = fmaf(d0x, d0x, fmaf(d0y, d0y, d0z * d0z)), n1 = fmaf(d1x, d1x, fmaf(d1y, d1y, d1z * d1z));
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int qi = i * 64 + lane + 32 * t;
+        float4 e = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
+        if (qi < L) {
+          const float4 sq = a.rowq[static_cast<int64_t>(bh) * L + qi];
+          const float2 rd = a.rowd[static_cast<int64_t>(bh) * L + qi];
+          const float rt0 = ch * (2.f * fmaf(sq.x, d0x, fmaf(sq.y, d0y, sq.z * d0z)) - pq * n0);
+          const float rt1 = ch * (2.f * fmaf(sq.x, d1x, fmaf(sq.y, d1y, sq.z * d1z)) - pq * n1);
+          e = make_float4(rt0 + rd.x, rt1 + rd.x, rd.y, 0.f);
+        }
+        qinfo[s * 64 + lane + 32 * t] = e;
+      }
+      if (lane == 0) oqs[s] = oqv;
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+        mbar_arrive_expect_tx(bar(KB_FULL0 + s), lay.stg_bytes);
+        tma_load_3d(st, &tm_qh, bar(KB_FULL0 + s), 0, i * 64, bh);
+        tma_load_3d(st + 8192, &tm_do, bar(KB_FULL0 + s), 0, i * 64, bh);
+        tma_load_4d(st + 16384, &tm_qp, bar(KB_FULL0 + s), 0, i * 64, 0, bh);
+        tma_load_4d(st + 16384 + np * 8192, &tm_du, bar(KB_FULL0 + s), 0, i * 64, 0, bh);
+      }
+      __syncwarp();
+    }
+    if (lane == 0 && *abort_flag) {
+      mbar_wait_bounded(bar(KB_KFULL), 0, nullptr, 100000000ull);
+      for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
+        mbar_wait_bounded(bar(KB_FULL0 + i % NS), (i / NS) & 1, nullptr, 100000000ull);
+    }
+  } else if (warp == W_MMA) {
+    if (lane == 0) {
+      bool ok = mbar_wait_bounded(bar(KB_KFULL), 0, abort_flag);
+      if (!ok) fail(DEV_TIMEOUT_FULL);
+      tc_fence_after();
+      const uint32_t id64 = idesc_f16(128, 64, false);
+      const uint32_t id64mn = idesc_f16(128, 64, true);
+      const uint32_t idz = idesc_f16(128, DZ, true);
+      const uint32_t tS = tmem + K_TM_S, tDP = tmem + K_TM_DP;
+      bool issued_any = false;
+      for (int i = 0; ok && i < nq; ++i) {
+        const int s = i % NS;
+        ok = mbar_wait_bounded(bar(KB_FULL0 + s), (i / NS) & 1, abort_flag);
+        // the accumulation MMAs of tile i-1 read P^T / dS^T from the columns S^T / dP^T(i) overwrite
+        if (ok && i > 0) ok = mbar_wait_bounded(bar(KB_ACC), (i - 1) & 1, abort_flag);
+        if (!ok) { fail(DEV_TIMEOUT_FULL); break; }
+        tc_fence_after();
+        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+        const uint32_t sQh = st, sDO = st + 8192, sQP = st + 16384, sDU = st + 16384 + np * 8192;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.kh + 32 * k), kd128(sQh + 32 * k), id64, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4 * np; ++kk)
+          umma_ss(tS, kd128(sb + lay.z2 + 16384 * (kk >> 2) + 32 * (kk & 3)),
+                  kd128(sQP + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, 1u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) umma_ss(tDP, kd128(sb + lay.vh + 32 * k), kd128(sDO + 32 * k), id64, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4 * np; ++kk)
+          umma_ss(tDP, kd128(sb + lay.z2 + 16384 * (kk >> 2) + 32 * (kk & 3)),
+                  kd128(sDU + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, 1u);
+        umma_commit(bar(KB_SFULL));
+        issued_any = true;
+        ok = mbar_wait_bounded(bar(KB_PFULL), i & 1, abort_flag);
+        if (!ok) { fail(DEV_TIMEOUT_SOFTMAX); break; }
+        tc_fence_after();
+        // P^T in columns [K_TM_S, +32), dS^T in [K_TM_DP, +32) (fp16, 64 queries)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
+          umma_ts(tmem + K_TM_DVA, tS + 8 * k, mnd(sDO + 2048 * k, 8192), id64mn, acc);
+          umma_ts(tmem + K_TM_DZ2, tS + 8 * k, mnd(sDU + 2048 * k, 8192), idz, acc);
+          umma_ts(tmem + K_TM_DZ2, tDP + 8 * k, mnd(sQP + 2048 * k, 8192), idz, 1u);
+          umma_ts(tmem + K_TM_DKH, tDP + 8 * k, mnd(sQh + 2048 * k, 8192), id64mn, acc);
+        }
+        umma_commit(bar(KB_ACC));
+        umma_commit(bar(KB_EMPTY0 + s));
+      }
+      if (!ok && issued_any) {
+        umma_commit(bar(KB_DRAIN));
+        mbar_wait_bounded(bar(KB_DRAIN), 0, nullptr, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const int key = J2 * 128 + r;
+    const bool in_range = key < L;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t pair_bar = 2 + quarter;
+    volatile int* pair_ok = reinterpret_cast<volatile int*>(smem + lay.aux + KA_PAIR);   // [2 parities][4][2]
+    const float4 ck = in_range ? a.colk[static_cast<int64_t>(bh) * L + key] : make_float4(0.f, 0.f, 0.f, -INFINITY);
+    const int sub = r >> 6;                      // which 64-key origin tile
+    const float4 okj = a.ok[b * a.nkt + (in_range ? key / 64 : 0)];
+    float cs = 0.f, co0 = 0.f, co1 = 0.f, co2 = 0.f;
+    bool ok = true;
+    for (int i = 0; i < nq && ok; ++i) {
+      const int s = i % NS;
+      // the two warps of these lanes decide together whether to go on, so
+      // that neither waits at their shared barrier for one that has left
+      const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_SFULL), i & 1, abort_flag));
+      uint32_t sv[32], dv[32];
+      if (got) {
+        tc_fence_after();
+        tmem_ld32(tmem + K_TM_S + 32 * half + lane_off, sv);
+        tmem_ld32(tmem + K_TM_DP + 32 * half + lane_off, dv);
+        tmem_ld_wait();
+        tc_fence_before();
+      }
+      if (lane == 0) pair_ok[(i & 1) * 8 + quarter * 2 + half] = got ? 1 : 0;
+      named_bar_sync(pair_bar, 64);           // both halves have read before either overwrites
+      if (!(pair_ok[(i & 1) * 8 + quarter * 2] && pair_ok[(i & 1) * 8 + quarter * 2 + 1])) {
+        if (lane == 0) fail(DEV_TIMEOUT_MMA);
+        ok = false;
+        break;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_FULL0 + s), (i / NS) & 1, abort_flag))) {
+        if (lane == 0) fail(DEV_TIMEOUT_FULL);
+        ok = false;
+        break;
+      }
+      const float4 oqv = oqs[s];
+      const float colv = ck.w - fmaf(ck.x, okj.x - oqv.x, fmaf(ck.y, okj.y - oqv.y, ck.z * (okj.z - oqv.z)));
+      const float4* qi = qinfo + s * 64 + 32 * half;
+      uint32_t pp[16], pd[16];
+      float tsum = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float4 e0 = qi[2 * k], e1 = qi[2 * k + 1];
+        const float x0 = __uint_as_float(sv[2 * k]) + colv + (sub ? e0.y : e0.x);
+        const float x1 = __uint_as_float(sv[2 * k + 1]) + colv + (sub ? e1.y : e1.x);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        pp[k] = pack_half2(p0, p1);
+        pd[k] = pack_half2(p0 * (__uint_as_float(dv[2 * k]) - e0.z) * kLn2,
+                           p1 * (__uint_as_float(dv[2 * k + 1]) - e1.z) * kLn2);
+        tsum = add_half2_to_f32(pd[k], tsum);
+      }
+      cs += tsum;
+      co0 = fmaf(tsum, oqv.x, co0);
+      co1 = fmaf(tsum, oqv.y, co1);
+      co2 = fmaf(tsum, oqv.z, co2);
+      tc_fence_after();
+      tmem_st16(tmem + K_TM_S + 16 * half + lane_off, pp);
+      tmem_st16(tmem + K_TM_DP + 16 * half + lane_off, pd);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(KB_PFULL));
+    }
+    if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_ACC), (nq - 1) & 1, abort_flag))) {
+      if (lane == 0) fail(DEV_TIMEOUT_MMA);
+      ok = false;
+    }
+    const bool all_ok = __all_sync(0xffffffffu, ok);
+    named_bar_sync(1, NSOFT);   // every thread is past its last read of the stage area
+    if (half == 1) reinterpret_cast<float4*>(smem + lay.stg)[r] = make_float4(cs, co0, co1, co2);
+    named_bar_sync(1, NSOFT);
+    if (all_ok && !*abort_flag) {
+      tc_fence_after();
+      if (half == 0 && in_range) {
+        const float4 o = reinterpret_cast<const float4*>(smem + lay.stg)[r];
+        a.csk[static_cast<int64_t>(bh) * L + key] = make_float4(cs + o.x, co0 + o.y, co1 + o.z, co2 + o.w);
+      }
+      auto store32 = [&](uint32_t tcol, float* dst_row) {
+        uint32_t v[32];
+        tmem_ld32(tmem + tcol + lane_off, v);
+        tmem_ld_wait();
+        if (in_range) {
+          float4* dst = reinterpret_cast<float4*>(dst_row);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+      };
+      const int64_t rowi = static_cast<int64_t>(bh) * L + (in_range ? key : 0);
+      store32(K_TM_DKH + 32 * half, a.dkh + rowi * 64 + 32 * half);
+      store32(K_TM_DVA + 32 * half, a.dva + rowi * 64 + 32 * half);
+      for (int c0 = half * (DZ / 2); c0 < (half + 1) * (DZ / 2); c0 += 32)
+        store32(K_TM_DZ2 + c0, a.dz2 + rowi * DZ + c0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == W_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ mapping
+struct MapArgs {
+  int B, L, H, DZ, RCz, Cz, R, rb, nblk;
+  float qscale, w_L, w_C;
+  View q_pts, k_pts, v_pts, g_out, out, uagg;
+  const float4* frame;
+  const float4* cen;
+  const float4* oq;
+  const float4* ok;
+  const float* headc;
+  const float* wqp;
+  const float* z1f;
+  const float* dqh;
+  const float* dqp;
+  const float4* rsq;
+  const float* dkh;
+  const float* dva;
+  const float* dz2;
+  const float4* csk;
+  int nqt, nkt;
+  // gradients (contiguous fp32)
+  float *d_q, *d_k, *d_v, *d_qpts, *d_kpts, *d_vpts, *d_rot, *d_trans, *d_z1, *d_z2;
+  float* wb_part;        // [nblk * B][H][DZ]
+  double* g_part;        // [nblk * B][H]
+};
+
+// Block: rb residues of one batch, all heads.  Phase 1: thread (residue,
+// head) -> scalar and point gradients, per-head frame contributions and
+// d gamma terms; phase 2: frame gradients summed over heads in a fixed
+// order; phase 3: thread per pair column -> d z1, d z2 (sums over heads)
+// and the block's partial sums of d w_bias.
+__global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
+  extern __shared__ float sm_map[];   // [rb][H][12] frame terms, then [rb][H] d gamma (double)
+  const int blk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int H = a.H, rb = a.rb;
+  const int i0 = blk * rb;
+  float* fterm = sm_map;
+  double* gterm = reinterpret_cast<double*>(sm_map + ((rb * H * 12 + 1) & ~1));
+  const int C = IPA_C, PQ = IPA_PQ, PV = IPA_PV;
+  const float4 cn = a.cen[b];
+  if (tid < rb * H) {
+    const int il = tid / H, h = tid % H;
+    const int i = i0 + il;
+    float fr[12];
+#pragma unroll
+    for (int e = 0; e < 12; ++e) fr[e] = 0.f;
+    double gsum = 0.0;
+    if (i < a.L) {
+      const int64_t bi = static_cast<int64_t>(b) * a.L + i;
+      const int64_t bhl = (static_cast<int64_t>(b) * H + h) * a.L + i;
+      const float4* fp = a.frame + bi * 4;
+      const float4 f0 = fp[0], f1 = fp[1], f2 = fp[2];
+      const float Rm[9] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w, f2.x};
+      const float tc[3] = {f2.y - cn.x, f2.z - cn.y, f2.w - cn.z};
+      const float c = a.headc[h];
+      const float* dq = a.dqh + bhl * 64;
+      const float* dk = a.dkh + bhl * 64;
+      const float* dv = a.dva + bhl * 64;
+      const float4 rq = a.rsq[bhl], ck = a.csk[bhl];
+      const int64_t o3 = bi * H + h;
+      for (int e = 0; e < C; ++e) {
+        a.d_q[o3 * C + e] = a.qscale * dq[e];
+        a.d_k[o3 * C + e] = dk[e];
+        a.d_v[o3 * C + e] = dv[e];
+      }
+      // query and key points: d gq = Gq2c + 2c (RSo - rs gq_c), d gk = 2c (Gk' + CSo - cs gk_c)
+      double g_q = 0.0, g_k = 0.0, g_x = 0.0;
+      for (int p = 0; p < PQ; ++p) {
+        float lq[3], lk[3], gqc[3], gkc[3], dgq[3], dgk[3];
+        for (int y = 0; y < 3; ++y) {
+          lq[y] = ldf(a.q_pts, b * a.q_pts.s[0] + i * a.q_pts.s[1] + h * a.q_pts.s[2] + p * a.q_pts.s[3] + y * a.q_pts.s[4]);
+          lk[y] = ldf(a.k_pts, b * a.k_pts.s[0] + i * a.k_pts.s[1] + h * a.k_pts.s[2] + p * a.k_pts.s[3] + y * a.k_pts.s[4]);
+        }
+        for (int x = 0; x < 3; ++x) {
+          gqc[x] = fmaf(Rm[3 * x], lq[0], fmaf(Rm[3 * x + 1], lq[1], Rm[3 * x + 2] * lq[2])) + tc[x];
+          gkc[x] = fmaf(Rm[3 * x], lk[0], fmaf(Rm[3 * x + 1], lk[1], Rm[3 * x + 2] * lk[2])) + tc[x];
+        }
+        const float rso[3] = {rq.y, rq.z, rq.w}, cso[3] = {ck.y, ck.z, ck.w};
+        for (int x = 0; x < 3; ++x) {
+          const int e = C + 3 * p + x;
+          const float gq2c = dq[e] + dq[e + 3 * PQ];                   // hi + lo key columns
+          const float gk1 = dk[e] + dk[e + 6 * PQ];                    // query hi + lo columns
+          dgq[x] = gq2c + 2.f * c * (rso[x] - rq.x * gqc[x]);
+          dgk[x] = 2.f * c * (gk1 + cso[x] - ck.x * gkc[x]);
+          g_q += static_cast<double>(rq.x) * gqc[x] * gqc[x];
+          g_k += static_cast<double>(ck.x) * gkc[x] * gkc[x];
+          g_x += static_cast<double>(gkc[x]) * (static_cast<double>(gk1) + cso[x]);
+        }
+        for (int y = 0; y < 3; ++y) {
+          a.d_qpts[(o3 * PQ + p) * 3 + y] = Rm[y] * dgq[0] + Rm[3 + y] * dgq[1] + Rm[6 + y] * dgq[2];
+          a.d_kpts[(o3 * PQ + p) * 3 + y] = Rm[y] * dgk[0] + Rm[3 + y] * dgk[1] + Rm[6 + y] * dgk[2];
+        }
+        for (int x = 0; x < 3; ++x) {
+          for (int y = 0; y < 3; ++y) fr[3 * x + y] += dgq[x] * lq[y] + dgk[x] * lk[y];
+          fr[9 + x] += dgq[x] + dgk[x];
+        }
+      }
+      gsum = -static_cast<double>(kLog2e) * a.w_L * a.w_C * 0.5 * (g_q + g_k - 2.0 * g_x);
+      // value points
+      for (int p = 0; p < PV; ++p) {
+        float lv[3], dgv[3];
+        for (int y = 0; y < 3; ++y)
+          lv[y] = ldf(a.v_pts, b * a.v_pts.s[0] + i * a.v_pts.s[1] + h * a.v_pts.s[2] + p * a.v_pts.s[3] + y * a.v_pts.s[4]);
+        for (int x = 0; x < 3; ++x) dgv[x] = dv[C + 3 * p + x];
+        for (int y = 0; y < 3; ++y)
+          a.d_vpts[(o3 * PV + p) * 3 + y] = Rm[y] * dgv[0] + Rm[3 + y] * dgv[1] + Rm[6 + y] * dgv[2];
+        for (int x = 0; x < 3; ++x) {
+          for (int y = 0; y < 3; ++y) fr[3 * x + y] += dgv[x] * lv[y];
+          fr[9 + x] += dgv[x];
+        }
+      }
+      // output side: o_pt = R^T (og - t): dR += (R o_pt) d_opt^T, dt -= R d_opt
+      if (fp[3].x != 0.f) {
+        const int64_t gb = b * a.g_out.s[0] + i * a.g_out.s[1] + h * a.g_out.s[2];
+        const int64_t ob = b * a.out.s[0] + i * a.out.s[1] + h * a.out.s[2];
+        for (int p = 0; p < PV; ++p) {
+          float op[3], dopt[3];
+          for (int y = 0; y < 3; ++y) op[y] = ldf(a.out, ob + (C + 3 * p + y) * a.out.s[3]);
+          const float nrm = sqrtf(op[0] * op[0] + op[1] * op[1] + op[2] * op[2]);
+          const float gn = ldf(a.g_out, gb + (C + 3 * PV + p) * a.g_out.s[3]);
+          for (int y = 0; y < 3; ++y)
+            dopt[y] = ldf(a.g_out, gb + (C + 3 * p + y) * a.g_out.s[3]) + (nrm > 0.f ? gn * op[y] / nrm : 0.f);
+          for (int x = 0; x < 3; ++x) {
+            const float rop = Rm[3 * x] * op[0] + Rm[3 * x + 1] * op[1] + Rm[3 * x + 2] * op[2];
+            const float rdo = Rm[3 * x] * dopt[0] + Rm[3 * x + 1] * dopt[1] + Rm[3 * x + 2] * dopt[2];
+            for (int y = 0; y < 3; ++y) fr[3 * x + y] += rop * dopt[y];
+            fr[9 + x] -= rdo;
+          }
+        }
+      }
+    }
+    for (int e = 0; e < 12; ++e) fterm[(il * H + h) * 12 + e] = fr[e];
+    gterm[il * H + h] = gsum;
+  }
+  __syncthreads();
+  // frame gradients: sum over heads in order
+  for (int t = tid; t < rb * 12; t += blockDim.x) {
+    const int il = t / 12, e = t % 12;
+    const int i = i0 + il;
+    if (i >= a.L) continue;
+    float s = 0.f;
+    for (int h = 0; h < H; ++h) s += fterm[(il * H + h) * 12 + e];
+    const int64_t bi = static_cast<int64_t>(b) * a.L + i;
+    if (e < 9) a.d_rot[bi * 9 + e] = s;
+    else a.d_trans[bi * 3 + (e - 9)] = s;
+  }
+  // d gamma partial of this block: residues in order
+  for (int h = tid; h < H; h += blockDim.x) {
+    double s = 0.0;
+    for (int il = 0; il < rb; ++il) s += gterm[il * H + h];
+    a.g_part[(static_cast<int64_t>(b) * a.nblk + blk) * H + h] = s;
+  }
+  // pair columns
+  for (int col = tid; col < a.DZ; col += blockDim.x) {
+    const int cc = col % a.Cz, rr = col / a.Cz;
+    const bool inpair = col < a.RCz;
+    for (int il = 0; il < rb; ++il) {
+      const int i = i0 + il;
+      if (i >= a.L) break;
+      if (!inpair) continue;
+      const int64_t bi = static_cast<int64_t>(b) * a.L + i;
+      float s1 = 0.f, s2 = 0.f;
+      for (int h = 0; h < H; ++h) {
+        const int64_t bhl = (static_cast<int64_t>(b) * H + h) * a.L + i;
+        const float gp = ldf(a.g_out, b * a.g_out.s[0] + i * a.g_out.s[1] + h * a.g_out.s[2] +
+                                          (C + 4 * PV + cc) * a.g_out.s[3]);
+        const float u = ldf(a.uagg, b * a.uagg.s[0] + i * a.uagg.s[1] + h * a.uagg.s[2] + rr * a.uagg.s[3] +
+                                        cc * a.uagg.s[4]);
+        const bool live = a.frame[bi * 4 + 3].x != 0.f;
+        s1 += a.wqp[h * a.DZ + col] * a.dqp[bhl * a.DZ + col] + (live ? gp * u : 0.f);
+        s2 += a.dz2[bhl * a.DZ + col];
+      }
+      a.d_z1[bi * a.RCz + col] = s1;
+      a.d_z2[bi * a.RCz + col] = s2;
+    }
+    for (int h = 0; h < H; ++h) {
+      float s = 0.f;
+      for (int il = 0; il < rb; ++il) {
+        const int i = i0 + il;
+        if (i >= a.L) break;
+        const int64_t bi = static_cast<int64_t>(b) * a.L + i;
+        const int64_t bhl = (static_cast<int64_t>(b) * H + h) * a.L + i;
+        s = fmaf(a.z1f[bi * a.DZ + col], a.dqp[bhl * a.DZ + col], s);
+      }
+      a.wb_part[((static_cast<int64_t>(b) * a.nblk + blk) * H + h) * a.DZ + col] = s;
+    }
+  }
+}
+
+// d w_bias[c, h] = log2(e) w_L sum over blocks and factors r of the partials;
+// d gamma[h] = sum over blocks.  One thread per output, fixed order.
+__global__ void ipa_bwd_reduce_kernel(const float* wb_part, const double* g_part, int nparts, int H, int DZ, int Cz,
+                                      int R, float scale, float* d_wb, float* d_gamma) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < Cz * H) {
+    const int c = t / H, h = t % H;
+    double s = 0.0;
+    for (int p = 0; p < nparts; ++p)
+      for (int r = 0; r < R; ++r) s += wb_part[(static_cast<int64_t>(p) * H + h) * DZ + r * Cz + c];
+    d_wb[c * H + h] = static_cast<float>(s * scale);
+  } else if (t < Cz * H + H) {
+    const int h = t - Cz * H;
+    double s = 0.0;
+    for (int p = 0; p < nparts; ++p) s += g_part[static_cast<int64_t>(p) * H + h];
+    d_gamma[h] = static_cast<float>(s);
+  }
+}
+
+int stages_for(uint32_t resident, uint32_t stage, uint32_t aux) {
+  const uint32_t budget = 227u * 1024u - 1024u - aux;
+  int ns = static_cast<int>((budget - resident) / stage);
+  return ns > MAX_NS ? MAX_NS : ns;
+}
+
+}  // namespace
+
+IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  IpaBwdWorkspace w{};
+  w.fwd = ipa_workspace_layout(B, L, H, DZ, RCz);
+  size_t o = up(w.fwd.total);
+  const size_t bhl = static_cast<size_t>(B) * H * L;
+  const int rb = 256 / H < 32 ? 256 / H : 32;
+  const size_t nblk = (L + rb - 1) / rb;
+  w.doh = o; o = up(o + bhl * 64 * 2);
+  w.du = o; o = up(o + bhl * DZ * 2);
+  w.qp = o; o = up(o + bhl * DZ * 2);
+  w.rowd = o; o = up(o + bhl * 8);
+  w.dqh = o; o = up(o + bhl * 64 * 4);
+  w.dqp = o; o = up(o + bhl * DZ * 4);
+  w.rsq = o; o = up(o + bhl * 16);
+  w.dkh = o; o = up(o + bhl * 64 * 4);
+  w.dva = o; o = up(o + bhl * 64 * 4);
+  w.dz2 = o; o = up(o + bhl * DZ * 4);
+  w.csk = o; o = up(o + bhl * 16);
+  w.wb_part = o; o = up(o + static_cast<size_t>(B) * nblk * H * DZ * 4);
+  w.g_part = o; o = up(o + static_cast<size_t>(B) * nblk * H * 8);
+  w.total = o;
+  return w;
+}
+
+cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
+  const IpaLaunch& f = a.f;
+  unsigned char* ws = f.ws;
+  const IpaBwdWorkspace& w = a.lay;
+  const IpaWorkspace& fw = w.fwd;
+  const int B = f.B, L = f.L, H = f.H, DZ = f.DZ, np = DZ / 64;
+  const uint64_t bh = static_cast<uint64_t>(B) * H;
+
+  // 1. the forward prologue again (frames, augmented rows, tile origins)
+  cudaError_t e = ipa_launch_prologue(f, stream);
+  if (e != cudaSuccess) return e;
+
+  // 2. backward rows
+  RowsArgs ra{};
+  ra.B = B; ra.L = L; ra.H = H; ra.DZ = DZ; ra.RCz = f.RCz; ra.Cz = f.Cz; ra.F = f.F;
+  ra.z1_half = ipa_pair_supported(DZ);
+  ra.g_out = a.g_out; ra.out = a.out; ra.lse = a.lse; ra.uagg = a.uagg;
+  ra.frame = reinterpret_cast<const float4*>(ws + fw.frame);
+  ra.cen = reinterpret_cast<const float4*>(ws + fw.cen);
+  ra.rowq = reinterpret_cast<const float4*>(ws + fw.rowq);
+  ra.wqp = reinterpret_cast<const float*>(ws + fw.wqp);
+  ra.z1f = reinterpret_cast<const float*>(ws + fw.z1f);
+  ra.z1h = reinterpret_cast<const __half*>(ws + fw.z1h);
+  ra.doh = reinterpret_cast<__half*>(ws + w.doh);
+  ra.du = reinterpret_cast<__half*>(ws + w.du);
+  ra.qp = reinterpret_cast<__half*>(ws + w.qp);
+  ra.rowd = reinterpret_cast<float2*>(ws + w.rowd);
+  const int64_t warps = static_cast<int64_t>(B) * L * H;
+  ipa_bwd_rows_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(ra);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  BwdArgs ba{};
+  ba.B = B; ba.L = L; ba.H = H; ba.DZ = DZ; ba.RCz = f.RCz; ba.Cz = f.Cz; ba.R = f.R;
+  ba.nqt = f.nqt; ba.nkt = f.nkt;
+  ba.qscale = kLog2e * f.w_L * f.scalar_scale; ba.w_L = f.w_L; ba.w_C = f.w_C;
+  ba.rowq = reinterpret_cast<const float4*>(ws + fw.rowq);
+  ba.colk = reinterpret_cast<const float4*>(ws + fw.colk);
+  ba.oq = reinterpret_cast<const float4*>(ws + fw.oq);
+  ba.ok = reinterpret_cast<const float4*>(ws + fw.ok);
+  ba.cen = reinterpret_cast<const float4*>(ws + fw.cen);
+  ba.headc = reinterpret_cast<const float*>(ws + fw.headc);
+  ba.wqp = reinterpret_cast<const float*>(ws + fw.wqp);
+  ba.frame = reinterpret_cast<const float4*>(ws + fw.frame);
+  ba.z1f = reinterpret_cast<const float*>(ws + fw.z1f);
+  ba.z1h = reinterpret_cast<const __half*>(ws + fw.z1h);
+  ba.rowd = reinterpret_cast<const float2*>(ws + w.rowd);
+  ba.dqh = reinterpret_cast<float*>(ws + w.dqh);
+  ba.dqp = reinterpret_cast<float*>(ws + w.dqp);
+  ba.rsq = reinterpret_cast<float4*>(ws + w.rsq);
+  ba.dkh = reinterpret_cast<float*>(ws + w.dkh);
+  ba.dva = reinterpret_cast<float*>(ws + w.dva);
+  ba.dz2 = reinterpret_cast<float*>(ws + w.dz2);
+  ba.csk = reinterpret_cast<float4*>(ws + w.csk);
+  ba.err = f.err;
+
+  const uint64_t rowb = static_cast<uint64_t>(L) * DH * 2;
+  // 3. query pass
+  {
+    CUtensorMap tqh, tqp, tdo, tdu, tkh, tvh, tz2;
+    bool ok = encode_tmap_f16_3d(&tqh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, 128) &&
+              encode_tmap_f16_panels(&tqp, ws + w.qp, DZ, L, bh, 128, np) &&
+              encode_tmap_f16_3d(&tdo, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, 128) &&
+              encode_tmap_f16_panels(&tdu, ws + w.du, DZ, L, bh, 128, np) &&
+              encode_tmap_f16_3d(&tkh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, 64) &&
+              encode_tmap_f16_3d(&tvh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, 64) &&
+              encode_tmap_f16_panels(&tz2, ws + fw.z2, DZ, L, B, 64, np);
+    if (!ok) return cudaErrorInvalidValue;
+    const QLayout l1 = q_layout(DZ, 1);
+    ba.ns = stages_for(l1.stg, l1.stg_bytes, 2048);
+    const QLayout lq = q_layout(DZ, ba.ns);
+    const uint32_t smem = lq.total + 1024;
+    e = cudaFuncSetAttribute(ipa_bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    ipa_bwd_q_kernel<<<static_cast<unsigned>(bh * f.nqt), NTH, smem, stream>>>(tqh, tqp, tdo, tdu, tkh, tvh, tz2, ba);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // 4. key pass
+  {
+    CUtensorMap tkh, tvh, tz2, tqh, tdo, tqp, tdu;
+    bool ok = encode_tmap_f16_3d(&tkh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, 128) &&
+              encode_tmap_f16_3d(&tvh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, 128) &&
+              encode_tmap_f16_panels(&tz2, ws + fw.z2, DZ, L, B, 128, np) &&
+              encode_tmap_f16_3d(&tqh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, 64) &&
+              encode_tmap_f16_3d(&tdo, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, 64) &&
+              encode_tmap_f16_panels(&tqp, ws + w.qp, DZ, L, bh, 64, np) &&
+              encode_tmap_f16_panels(&tdu, ws + w.du, DZ, L, bh, 64, np);
+    if (!ok) return cudaErrorInvalidValue;
+    const KLayout l1 = k_layout(DZ, 1);
+    BwdArgs kb = ba;
+    kb.ns = stages_for(l1.stg, l1.stg_bytes, 4096);
+    const KLayout lk = k_layout(DZ, kb.ns);
+    const uint32_t smem = lk.total + 1024;
+    e = cudaFuncSetAttribute(ipa_bwd_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int nkp = (L + 127) / 128;
+    ipa_bwd_k_kernel<<<static_cast<unsigned>(bh * nkp), NTH, smem, stream>>>(tkh, tvh, tz2, tqh, tdo, tqp, tdu, kb);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // 5. per-residue mapping and the reductions
+  MapArgs m{};
+  m.B = B; m.L = L; m.H = H; m.DZ = DZ; m.RCz = f.RCz; m.Cz = f.Cz; m.R = f.R;
+  m.rb = 256 / H < 32 ? 256 / H : 32;
+  m.nblk = (L + m.rb - 1) / m.rb;
+  m.qscale = ba.qscale; m.w_L = f.w_L; m.w_C = f.w_C;
+  m.q_pts = f.q_pts; m.k_pts = f.k_pts; m.v_pts = f.v_pts; m.g_out = a.g_out; m.out = a.out; m.uagg = a.uagg;
+  m.frame = ba.frame; m.cen = ba.cen; m.oq = ba.oq; m.ok = ba.ok; m.headc = ba.headc; m.wqp = ba.wqp;
+  m.z1f = ba.z1f; m.dqh = ba.dqh; m.dqp = ba.dqp; m.rsq = ba.rsq; m.dkh = ba.dkh; m.dva = ba.dva;
+  m.dz2 = ba.dz2; m.csk = ba.csk; m.nqt = f.nqt; m.nkt = f.nkt;
+  m.d_q = a.d_q; m.d_k = a.d_k; m.d_v = a.d_v; m.d_qpts = a.d_q_pts; m.d_kpts = a.d_k_pts; m.d_vpts = a.d_v_pts;
+  m.d_rot = a.d_rot; m.d_trans = a.d_trans; m.d_z1 = a.d_z1; m.d_z2 = a.d_z2;
+  m.wb_part = reinterpret_cast<float*>(ws + w.wb_part);
+  m.g_part = reinterpret_cast<double*>(ws + w.g_part);
+  const size_t msmem = static_cast<size_t>((m.rb * H * 12 + 1) & ~1) * 4 + static_cast<size_t>(m.rb) * H * 8;
+  ipa_bwd_map_kernel<<<dim3(static_cast<unsigned>(m.nblk), static_cast<unsigned>(B)), 256, msmem, stream>>>(m);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int nout = f.Cz * H + H;
+  ipa_bwd_reduce_kernel<<<(nout + 127) / 128, 128, 0, stream>>>(m.wb_part, m.g_part, B * m.nblk, H, DZ, f.Cz, f.R,
+                                                               kLog2e * f.w_L, a.d_w_bias, a.d_gamma);
+  return cudaGetLastError();
+}
+
+}  // namespace fipa

@@ -43,6 +43,7 @@ struct EpilogueArgs {
   int b, h, row0;        // first query row of the tile
   const float* z1f;      // [B, L, DZ] fp32, zero-padded
   float* out;            // [B, L, H, F]
+  float* uagg = nullptr; // training forward only: [B, L, H, R Cz] pair aggregate U (else null)
 #ifdef IPA_TRACE
   unsigned long long* trace = nullptr;   // phase clocks of warp 0 (tracing build only)
 #endif
@@ -161,6 +162,22 @@ static __device__ __noinline__ void fold_pairs_rows(const EpilogueArgs& e, int w
   }
 }
 
+// Training forward: the normalised pair aggregate U_i = sum_j a_ij z2_j of
+// the warp's 16 rows, R Cz floats per row, copied out of the stage before
+// phase A folds it with z1 (rows without an allowed key hold zeros).
+static __device__ __noinline__ void store_pair_aggregate(const EpilogueArgs& e, int warp, int lane) {
+  const int pitch = stage_pitch(e.DZ);
+  const int nq = e.RCz >> 2;                  // float4 per row (RCz % 16 == 0)
+  for (int rr = 0; rr < 16; ++rr) {
+    const int grow = e.row0 + warp * 16 + rr;
+    if (grow >= e.L) break;
+    const float4* src = reinterpret_cast<const float4*>(e.stage + (warp * 16 + rr) * pitch + 64);
+    float4* dst = reinterpret_cast<float4*>(e.uagg + ((static_cast<int64_t>(e.b) * e.L + grow) * e.H + e.h) * e.RCz);
+    for (int q = lane; q < nq; q += 32) dst[q] = src[q];
+  }
+  __syncwarp();
+}
+
 // Called by all 8 warps (warp = 0..7) after the staged rows are complete;
 // warp w handles rows 16 w .. 16 w + 15 of the tile: phase A (above), then
 // phase B: the output rows with coalesced stores.  No global load is issued after a global store.
@@ -178,6 +195,7 @@ __device__ __forceinline__ void write_rows(const EpilogueArgs& e, int warp, int 
   } while (0)
 #endif
   EPI_TR(0);
+  if (e.uagg != nullptr) store_pair_aggregate(e, warp, lane);
   fold_pairs_rows(e, warp, lane);
   EPI_TR(1);
 #pragma unroll 2
@@ -193,5 +211,94 @@ __device__ __forceinline__ void write_rows(const EpilogueArgs& e, int warp, int 
 }
 
 #undef EPI_TR
+
+// Direct output pass for the CTA-pair kernel, whose tensor memory holds
+// [O_pair (DZ) | O_v (64)] per row, when the pair block has no padding
+// (R Cz == DZ) and Cz is a multiple of 64.  Thread (row, half) folds z1
+// into the pair features c in [half Cz/2, (half + 1) Cz/2), 32 at a time,
+// straight from tensor memory (for each factor r: O_pair[r Cz + c] / l
+// times z1_i[r, c], summed over r in the order of the staged pass), and
+// writes them as 16-byte stores; half 0 also writes the scalar outputs, the
+// value points mapped back with R_i^T and their norms.  No shared-memory
+// stage and no per-warp pass over rows: the z1 loads of all rows are in
+// flight together.  tcgen05.ld is warp-collective, so every lane loads
+// and only the stores depend on the row being in range.
+template <int C, int PV>
+__device__ __forceinline__ void write_row_direct(uint32_t tmem_row, int half, int DZ, int Cz, int R, float inv,
+                                                 bool dead, bool in_range, const float* z1r, float* outr, float* ur,
+                                                 float4 g0, float4 g1, float4 g2, float4 cn) {
+  static_assert(C == 16 && PV == 8, "feature map written for the (16, 8) head shape");
+  for (int c0 = half * (Cz / 2); c0 < (half + 1) * (Cz / 2); c0 += 32) {
+    float acc[32];
+    for (int rf = 0; rf < R; ++rf) {
+      uint32_t o[32];
+      sm100::tmem_ld32(tmem_row + rf * Cz + c0, o);
+      float4 z[8];
+      const float4* zp = reinterpret_cast<const float4*>(z1r + rf * Cz + c0);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[e] = __ldg(zp + e);
+      sm100::tmem_ld_wait();
+      float u[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) u[e] = __uint_as_float(o[e]) * inv;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float zz[4] = {z[e].x, z[e].y, z[e].z, z[e].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[4 * e + k] = rf == 0 ? zz[k] * u[4 * e + k] : fmaf(zz[k], u[4 * e + k], acc[4 * e + k]);
+      }
+      if (ur != nullptr && in_range) {
+        float4* up = reinterpret_cast<float4*>(ur + rf * Cz + c0);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) up[e] = make_float4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
+      }
+    }
+    if (in_range) {
+      float4* op = reinterpret_cast<float4*>(outr + C + 4 * PV + c0);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) op[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+    }
+  }
+  if (half == 0) {
+    uint32_t v0[32], v1[32];
+    sm100::tmem_ld32(tmem_row + DZ, v0);
+    sm100::tmem_ld32(tmem_row + DZ + 32, v1);
+    sm100::tmem_ld_wait();
+    if (!in_range) return;
+    float4* op = reinterpret_cast<float4*>(outr);
+    if (dead) {
+#pragma unroll
+      for (int e = 0; e < (C + 4 * PV) / 4; ++e) op[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      return;
+    }
+    // O_v = [v (C) | gv hi (3 PV) | gv lo (3 PV)] relative to the centroid
+    float f[C + 4 * PV];
+#pragma unroll
+    for (int e = 0; e < C; ++e) f[e] = __uint_as_float(v0[e]) * inv;
+    const float Rm[9] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w, g2.x};
+    const float tp[3] = {g2.y - cn.x, g2.z - cn.y, g2.w - cn.z};
+#pragma unroll
+    for (int p = 0; p < PV; ++p) {
+      float g[3];
+#pragma unroll
+      for (int x = 0; x < 3; ++x) {
+        const int hi = C + 3 * p + x, lo = C + 3 * PV + 3 * p + x;
+        const float a = __uint_as_float(hi < 32 ? v0[hi & 31] : v1[hi & 31]) * inv;
+        const float bb = __uint_as_float(lo < 32 ? v0[lo & 31] : v1[lo & 31]) * inv;
+        g[x] = a + bb - tp[x];
+      }
+      float sqs = 0.f;
+#pragma unroll
+      for (int x = 0; x < 3; ++x) {
+        const float o = fmaf(Rm[x], g[0], fmaf(Rm[3 + x], g[1], Rm[6 + x] * g[2]));   // (R^T g)_x
+        f[C + 3 * p + x] = o;
+        sqs = x == 0 ? o * o : sqs + o * o;
+      }
+      f[C + 3 * PV + p] = sqrtf(sqs);
+    }
+#pragma unroll
+    for (int e = 0; e < (C + 4 * PV) / 4; ++e) op[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+  }
+}
 
 }  // namespace fipa

@@ -402,3 +402,89 @@ def test_module_rejects_bad_arguments_before_launch(case, expect):
     st = lib.ipa_module_fwd(ctypes.byref(p), *[ctypes.byref(ds[k]) if ds[k] is not None else None for k in order],
                             ctypes.c_void_p(FAKE), ctypes.c_size_t(ws), None, None)
     assert st == expect
+
+
+def ipa_bwd_call(p, ds, extra, grads, ws_bytes=None, ws_ptr=FAKE):
+    lib = api.library()
+    if ws_bytes is None:
+        ws_bytes = lib.ipa_attn_bwd_workspace_size(ctypes.byref(p))
+    gs = api.IpaGrads(*[grads[n] for n in api.IPA_GRADS])
+    return lib.ipa_attn_bwd(ctypes.byref(p), *[ctypes.byref(ds[k]) for k in ORDER],
+                            *[ctypes.byref(extra[k]) if extra[k] is not None else None
+                              for k in ("lse", "u_agg", "g_out")],
+                            ctypes.byref(gs), ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes), None,
+                            ctypes.c_void_p(FAKE))
+
+
+def bwd_args(B=1, L=64, H=4, R=2, Cz=16):
+    p, ds = ipa_args(B=B, L=L, H=H, R=R, Cz=Cz)
+    F = 16 + 32 + Cz
+    extra = {"lse": desc((B, H, L)), "u_agg": desc((B, L, H, R, Cz)), "g_out": desc((B, L, H, F))}
+    grads = {n: desc(tuple(ds[n].size[i] for i in range(ds[n].ndim))) for n in api.IPA_GRADS}
+    return p, ds, extra, grads
+
+
+def test_bwd_workspace_is_linear_in_L_and_zero_when_invalid():
+    lib = api.library()
+    per = []
+    for L in (2048, 4096, 8192, 16384):
+        p = api.ipa_params(1, L, 12, 16, 4, 8, 2, 128)
+        per.append(lib.ipa_attn_bwd_workspace_size(ctypes.byref(p)) / L)
+        assert lib.ipa_attn_bwd_workspace_size(ctypes.byref(p)) > lib.ipa_attn_workspace_size(ctypes.byref(p))
+    assert max(per) / min(per) < 1.02
+    bad = api.ipa_params(1, 64, 4, 16, 4, 8, 2, 20)      # Cz not a multiple of 16
+    assert lib.ipa_attn_bwd_workspace_size(ctypes.byref(bad)) == 0
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("ok_shape_check_only", None), ("null_grads", 1), ("lse_shape", 2), ("uagg_dtype", 4), ("g_out_shape", 2),
+    ("grad_noncontig", 3), ("grad_shape", 2), ("workspace", 5), ("ws_align", 5), ("unsupported", 6),
+])
+def test_ipa_bwd_rejects_bad_arguments_before_launch(case, expect):
+    p, ds, extra, grads = bwd_args()
+    ws, ws_ptr = None, FAKE
+    if case == "ok_shape_check_only":
+        return                                   # a valid call would launch: nothing to run without a GPU
+    if case == "null_grads":
+        lib = api.library()
+        st = lib.ipa_attn_bwd(ctypes.byref(p), *[ctypes.byref(ds[k]) for k in ORDER],
+                              *[ctypes.byref(extra[k]) for k in ("lse", "u_agg", "g_out")], None,
+                              ctypes.c_void_p(FAKE), ctypes.c_size_t(1 << 30), None, ctypes.c_void_p(FAKE))
+        assert st == expect
+        return
+    if case == "lse_shape":
+        extra["lse"] = desc((1, 64, 4))
+    elif case == "uagg_dtype":
+        extra["u_agg"] = desc((1, 64, 4, 2, 16), dtype=api.IPA_DTYPE_F64)
+    elif case == "g_out_shape":
+        extra["g_out"] = desc((1, 64, 4, 63))
+    elif case == "grad_noncontig":
+        grads["q"] = desc((1, 64, 4, 16), strides=(64 * 4 * 32, 4 * 32, 32, 1))
+    elif case == "grad_shape":
+        grads["z2"] = desc((1, 64, 2, 15))
+    elif case == "workspace":
+        ws = 1024
+    elif case == "ws_align":
+        ws_ptr = FAKE + 8
+    elif case == "unsupported":
+        p, ds, extra, grads = bwd_args()
+        p.C = 32
+    assert ipa_bwd_call(p, ds, extra, grads, ws, ws_ptr) == expect
+
+
+@pytest.mark.parametrize("case,expect", [("lse_shape", 2), ("uagg_align", 3), ("null_lse", 1)])
+def test_ipa_fwd_train_rejects_bad_outputs_before_launch(case, expect):
+    p, ds = ipa_args()
+    lse, uagg = desc((1, 4, 64)), desc((1, 64, 4, 2, 16))
+    if case == "lse_shape":
+        lse = desc((1, 64, 4))
+    elif case == "uagg_align":
+        uagg = desc((1, 64, 4, 2, 16), ptr=FAKE + 4)
+    elif case == "null_lse":
+        lse = desc((1, 4, 64), ptr=None)
+    lib = api.library()
+    ws = lib.ipa_attn_workspace_size(ctypes.byref(p))
+    st = lib.ipa_attn_fwd_train(ctypes.byref(p), *[ctypes.byref(ds[k]) for k in ORDER], ctypes.byref(lse),
+                                ctypes.byref(uagg), ctypes.c_void_p(FAKE), ctypes.c_size_t(ws), None,
+                                ctypes.c_void_p(FAKE))
+    assert st == expect
