@@ -49,12 +49,33 @@ NCU_TRAFFIC = {"kernel_sha256": "33c314293e9746ffee45dfd4781970575e1a13c1f721289
                "bytes_per_launch": 30.75e6}
 
 
-def ipa_flops(B, L, n_valid=None):
+def ipa_flops(B, L, n_valid=None, heads=H, rcz=R * CZ):
     """Algorithmic flops of the fused core (2 per multiply-add)."""
-    dqk = C + 3 * PQ + 1 + R * CZ
-    dv = C + 3 * PV + R * CZ
+    dqk = C + 3 * PQ + 1 + rcz
+    dv = C + 3 * PV + rcz
     pairs = B * L * L if n_valid is None else float(np.sum(np.asarray(n_valid, float) ** 2))
-    return 2.0 * pairs * H * (dqk + dv)
+    return 2.0 * pairs * heads * (dqk + dv)
+
+
+def ipa_bwd_flops(B, L, heads=H, rcz=R * CZ):
+    """Algorithmic flops of the gradient pass: the logits again (Dqk), dP
+    (Dv), dQ (Dqk), dK (Dqk) and dV (Dv) per (query, key, head)."""
+    dqk = C + 3 * PQ + 1 + rcz
+    dv = C + 3 * PV + rcz
+    return 2.0 * B * L * L * heads * (3 * dqk + 2 * dv)
+
+
+def host_threads():
+    """Cores this process may run on and the BLAS pool size (reported beside
+    the CPU oracle timings; the oracle's einsums themselves run on one)."""
+    cores = len(os.sched_getaffinity(0))
+    blas = None
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"), default=None)
+    except Exception:  # noqa: BLE001 -- reported as unknown
+        pass
+    return cores, blas
 
 
 def rank_inputs(rank, L):
@@ -165,6 +186,151 @@ def cpu_oracle_sample(L, seconds, max_rows, seed=0, inp=None):
     return flops / t_total / 1e12, rows_done, t_total
 
 
+def timed_graph(torch, fn, flush, n=20):
+    """Mean CUDA-event time (ms) of `fn` replayed as a CUDA graph, L2 flushed
+    (untimed) before each replay; direct launches if capture fails."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    run = fn
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        torch.cuda.synchronize()
+        run = gr.replay
+    except Exception:  # noqa: BLE001 -- fall back to direct launches
+        torch.cuda.synchronize()
+    ts = []
+    for _ in range(n):
+        flush.zero_()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        run()
+        a1.record()
+        torch.cuda.synchronize()
+        ts.append(a0.elapsed_time(a1))
+    return statistics.mean(ts)
+
+
+def fig2a_mb(L):
+    """The FlashIPA page's Fig. 2A memory fits (MB) at length L, as printed:
+    IPA 2.4e-3 L^2 + 1.4e-2 L, FlashIPA -7e-12 L^2 + 7.5e-2 L (context only;
+    their hardware and precision are not stated)."""
+    return {"ipa_MB": 2.4e-3 * L * L + 1.4e-2 * L, "flashipa_MB": -7e-12 * L * L + 7.5e-2 * L}
+
+
+def bench_configs(api, torch, dev, flush):
+    """Each configuration of the fused core on its own: step (prologue +
+    core) and core alone as CUDA-graph replays, algorithmic TFLOP/s of the
+    core (valid pairs only), fraction of the measured peak, and the device
+    bytes one call needs (inputs + output + workspace)."""
+    from rna_structure_models_b200.synth import IpaDims, ipa_inputs, ipa_preset
+    peaks, kind = measured_peaks()
+    peak = float(peaks["bf16_tflops"])
+    cases = [("AF2-sized, last 10% masked", ipa_preset("af2")),
+             ("batched generation-shaped, ragged 64..128", ipa_preset("batched"))]
+    cases += [(f"long-context L={Lc}", ipa_inputs(IpaDims(B=1, L=Lc, H=12), 0)) for Lc in (2048, 8192, 16384)]
+    res = []
+    for name, inp in cases:
+        Bc, Lc, Hc, _ = inp["q"].shape
+        Rc, Czc = inp["z1"].shape[2], inp["z1"].shape[3]
+        d = {n: torch.from_numpy(inp[n]).to(dev) for n in api.IPA_INPUTS}
+        plan = api.IpaPlan(Bc, Lc, Hc, C, PQ, PV, Rc, Czc, device=dev)
+        out = torch.empty((Bc, Lc, Hc, plan.F), dtype=torch.float32, device=dev)
+        args_in = [d[n] for n in api.IPA_INPUTS]
+
+        def step():
+            plan.prologue(*args_in)
+            plan.core(out)
+
+        ms_step = timed_graph(torch, step, flush)
+        ms_core = timed_graph(torch, lambda: plan.core(out), flush)
+        plan.check()
+        n_valid = inp["mask"].sum(axis=1)
+        flops = ipa_flops(Bc, Lc, n_valid=n_valid, heads=Hc, rcz=Rc * Czc)
+        in_bytes = sum(t.numel() * t.element_size() for t in args_in)
+        dbytes = in_bytes + out.numel() * 4 + plan.workspace.numel()
+        entry = {"config": name, "B": Bc, "L": Lc, "H": Hc, "R_Cz": Rc * Czc,
+                 "valid_pairs_per_head": float(np.sum(n_valid.astype(float) ** 2)),
+                 "gflop_algorithmic": flops / 1e9, "core_us": ms_core * 1e3, "step_us": ms_step * 1e3,
+                 "core_tflops": flops / (ms_core / 1e3) / 1e12, "step_tflops": flops / (ms_step / 1e3) / 1e12,
+                 "frac": flops / (ms_core / 1e3) / 1e12 / peak, "peak_source": f"{kind} bf16 dense (burst)",
+                 "device_bytes": dbytes, "workspace_bytes": plan.workspace.numel()}
+        if Bc == 1:
+            entry["fig2a_context"] = fig2a_mb(Lc)
+        res.append(entry)
+        del d, plan, out
+        torch.cuda.empty_cache()
+    return res
+
+
+def bench_backward(api, torch, dev, flush, L, dvc, names):
+    """Training forward and gradient pass at the headline workload."""
+    peaks, kind = measured_peaks()
+    peak = float(peaks["bf16_tflops"])
+    plan = api.IpaPlan(1, L, H, C, PQ, PV, R, CZ, device=dev)
+    gplan = api.IpaGradPlan(1, L, H, C, PQ, PV, R, CZ, device=dev)
+    args_in = [dvc[n] for n in names]
+    out, lse, U = plan.train(*args_in)
+    g = torch.randn(out.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(1))
+    grads = gplan(dvc, out, lse, U, g)
+    torch.cuda.synchronize()
+    plan.check()
+    gplan.check()
+    ms_train = timed_graph(torch, lambda: plan.train(*args_in, out=out, lse=lse, u_agg=U), flush)
+    ms_bwd = timed_graph(torch, lambda: gplan(dvc, out, lse, U, g, grads=grads), flush, n=10)
+    gplan.check()
+    fb = ipa_bwd_flops(1, L)
+    return {"workload": f"IPA core gradients B=1 L={L} H={H} C={C} Pq={PQ} Pv={PV} R={R} Cz={CZ}",
+            "train_forward_ms": ms_train, "backward_ms": ms_bwd,
+            "backward_gflop_algorithmic": fb / 1e9,
+            "backward_tflops": fb / (ms_bwd / 1e3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": fb / (ms_bwd / 1e3) / 1e12, "peak": peak,
+                         "unit": "TFLOP/s", "frac": fb / (ms_bwd / 1e3) / 1e12 / peak,
+                         "peak_source": f"{kind} bf16 dense (burst)",
+                         "note": "whole gradient call (prologue again, rows, query pass, key pass, mapping)"},
+            "issued_flops_per_triple": 4480, "algorithmic_flops_per_triple": 2 * (3 * 285 + 2 * 296),
+            "workspace_bytes": gplan.workspace.numel()}
+
+
+def cpu_oracle_configs(seconds):
+    """The float64 oracle on each configuration of the core: tiny, AF2 and
+    batched in full; the long-context lengths on 64-row blocks within a time
+    budget, extrapolated linearly in rows to the whole sequence."""
+    from oracle import ipa_dense
+    from rna_structure_models_b200.synth import IpaDims, ipa_inputs, ipa_preset
+    res = []
+    for name in ("tiny", "af2", "batched"):
+        inp = ipa_preset(name)
+        t0 = time.perf_counter()
+        if name == "batched":
+            for b in range(inp["q"].shape[0]):
+                ipa_dense({k: (v[b:b + 1] if isinstance(v, np.ndarray) and v.ndim >= 2 and k not in ("w_bias",)
+                               else v) for k, v in inp.items()})
+        else:
+            ipa_dense(inp)
+        res.append({"config": name, "seconds": time.perf_counter() - t0, "extrapolated": False})
+    for Lc in (2048, 4096, 8192, 16384):
+        inp = ipa_inputs(IpaDims(B=1, L=Lc, H=12), 0)
+        rows, t = 0, 0.0
+        while rows < Lc and t < seconds / 4:
+            r = np.arange(rows, min(rows + 64, Lc))
+            t0 = time.perf_counter()
+            ipa_dense(inp, rows=r)
+            t += time.perf_counter() - t0
+            rows += len(r)
+        res.append({"config": f"long-context L={Lc}", "seconds": t * Lc / rows, "extrapolated": rows < Lc,
+                    "rows_timed": rows})
+    return res
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -210,6 +376,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variant", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration timings")
+    ap.add_argument("--no-backward", action="store_true", help="skip the gradient-pass timing")
     ap.add_argument("--core-only", action="store_true", help="profiling aid: time only, print nothing else")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step's kernels directly instead of replaying a CUDA graph")
@@ -350,37 +518,42 @@ def main():
         h2d = sum(v.numel() * v.element_size() for v in pinned.values())
         res = torch.empty((1, L, H, plan.F), dtype=torch.float32, pin_memory=True)
         d2h = res.numel() * res.element_size()
-        for _ in range(max(1, min(args.warmup, 3))):
-            o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev, out=res)
-        torch.cuda.synchronize()
         ke = max(3, min(K, 50))
-        # one call at a time (ipa_attn_host): copies, kernels and the copy back in series
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        hc = api.IpaHostCalls(1, L, H, C, PQ, PV, R, CZ, slots=2, device=dev)
+        outs = [res, torch.empty_like(res).pin_memory()]
+        for _ in range(max(1, min(args.warmup, 3))):
+            hc.run([pinned] * 2, outs)
+        hc.check()
+        # one call at a time on one stream: copies, kernels and the copy back in series
+        s0, s1 = hc.streams
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        e0.record()
+        e0.record(s0)
         for _ in range(ke):
-            o, _ = api.ipa_attn_host(pinned, plan=plan, device=dev, out=res)
-        e1.record()
+            hc.call(pinned, res, 0)
+        e1.record(s0)
         torch.cuda.synchronize()
         t_serial = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
-        # ke calls through IpaHostPipeline: every call's inputs still go up and
-        # its result comes down inside the timed region, overlapped across calls
-        pipe = api.IpaHostPipeline(plan, device=dev)
-        pipe.run([pinned] * 3, [res] * 3)
-        torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        e0.record()
-        pipe.run([pinned] * ke, [res] * ke)
-        e1.record()
+        e0.record(s0)
+        s1.wait_event(e0)
+        for k in range(ke):
+            hc.call(pinned, outs[k & 1], k & 1)
+        done = torch.cuda.Event()
+        done.record(s1)
+        s0.wait_event(done)
+        e1.record(s0)
         torch.cuda.synchronize()
+        hc.check()
         te = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
         line["e2e"] = {"value": aggregate_tflops(world, flops, ke, te), "unit": UNIT,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
-                       "ms_per_step": te / ke, "api": "IpaHostPipeline (transfers overlapped across calls)",
+                       "ms_per_step": te / ke,
+                       "api": "C entry point ipa_attn_fwd_host, two streams (tests/c/e2e_host.c does the same)",
                        "serial_ms_per_step": t_serial / ke}
 
     # second hot-path row: direction/distance geometric attention (B=2, N=2048)
@@ -520,11 +693,28 @@ def main():
             "linear_note": "each call packs x and W to fp16 (two kernels) before the tcgen05 GEMM",
         }
 
+    # secondary sections: a failure there is reported in the line and does not
+    # take the headline with it
+    for key, enabled, fn in (("configs", not args.no_configs, lambda: bench_configs(api, torch, dev, flush)),
+                             ("backward", not args.no_backward,
+                              lambda: bench_backward(api, torch, dev, flush, L, dvc, names))):
+        if enabled and rank == 0:
+            try:
+                line[key] = fn()
+            except Exception as exc:  # noqa: BLE001
+                torch.cuda.synchronize()
+                line[key] = {"error": f"{type(exc).__name__}: {exc}"}
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, nrows, secs = cpu_oracle_sample(L, args.cpu_seconds, 4096)
+        cores, blas = host_threads()
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "host_cores": cores, "blas_threads": blas,
                                 "sample": f"{nrows} query rows x {L} keys x {H} heads of the same workload, "
-                                          f"{secs:.1f} s of numpy float64 (single-threaded einsum)"}
+                                          f"{secs:.1f} s of numpy float64 (einsum on one thread; "
+                                          f"{cores} host cores available)"}
+        if not args.no_configs:
+            line["cpu_configs"] = cpu_oracle_configs(args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -228,7 +228,7 @@ struct PairArgs {
   float4* dq;            // [B*H, N, 2]: (d qd, 0), (d qp, 0) in the global frame
   float4* dk;            // [B*H, N, 2]
   float* dvr;            // [B*H, N, VW]
-  float* acc;            // [2H]: sum ds <qd, kd>, sum ds |qp - kp|
+  float* acc;            // [B, H, row blocks, 4 warps, 2]: per-warp sums of ds <qd, kd> and ds |qp - kp|
 };
 
 __device__ __forceinline__ float g_att_at(const PairArgs& a, int b, int h, int i, int j) {
@@ -388,9 +388,10 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_ro
     s6 += __shfl_xor_sync(0xffffffffu, s6, o);
     s7 += __shfl_xor_sync(0xffffffffu, s7, o);
   }
-  if ((tid & 31) == 0) {
-    atomicAdd(a.acc + h, s6);
-    atomicAdd(a.acc + a.H + h, s7);
+  if ((tid & 31) == 0) {     // one slot per (b, h, row block, warp), summed in a fixed order later
+    const int64_t slot = ((bh * gridDim.x + blockIdx.x) * 4 + (tid >> 5)) * 2;
+    a.acc[slot] = s6;
+    a.acc[slot + 1] = s7;
   }
 }
 
@@ -501,7 +502,8 @@ struct FrameArgs {
   const float4* dq;
   const float4* dk;
   const float* dvr;
-  const float* acc;      // [2H]
+  const float* acc;      // [B, H, nrb, 4, 2] per-warp partial sums (geo_bwd_rows_kernel)
+  int nrb;               // row blocks per (b, h)
   float *d_qd, *d_kd, *d_qp, *d_kp, *d_val, *d_rot, *d_trans, *d_dscale, *d_xscale;
 };
 
@@ -511,8 +513,15 @@ __global__ void __launch_bounds__(128) geo_bwd_frame_kernel(const FrameArgs a) {
     for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
       // d scale = dA sigmoid(scale); dA = sum ds dot / sqrt3, dB = -sum ds dist / sqrt3
       const float xd = ldf(a.dscale, h * a.dscale.s[0]), xx = ldf(a.xscale, h * a.xscale.s[0]);
-      a.d_dscale[h] = a.acc[h] * kInvSqrt3 / (1.f + expf(-xd));
-      a.d_xscale[h] = -a.acc[a.H + h] * kInvSqrt3 / (1.f + expf(-xx));
+      double sd = 0.0, sx = 0.0;   // fixed summation order: batch, row block, warp
+      for (int b = 0; b < a.B; ++b)
+        for (int k = 0; k < a.nrb * 4; ++k) {
+          const int64_t slot = ((static_cast<int64_t>(b) * a.H + h) * a.nrb * 4 + k) * 2;
+          sd += a.acc[slot];
+          sx += a.acc[slot + 1];
+        }
+      a.d_dscale[h] = static_cast<float>(sd) * kInvSqrt3 / (1.f + expf(-xd));
+      a.d_xscale[h] = -static_cast<float>(sx) * kInvSqrt3 / (1.f + expf(-xx));
     }
   if (t >= static_cast<int64_t>(a.B) * a.N) return;
   const int b = static_cast<int>(t / a.N), n = static_cast<int>(t % a.N);
@@ -617,7 +626,7 @@ GeoBwdWorkspace geo_bwd_workspace_layout(int B, int N, int H, int M, int Cout) {
   w.dq = o; o = up(o + bhn * 32);
   w.dk = o; o = up(o + bhn * 32);
   w.dvr = o; o = up(o + bhn * VW * 4);
-  w.acc = o; o = up(o + static_cast<size_t>(H) * 8);
+  w.acc = o; o = up(o + static_cast<size_t>(B) * H * ((N + BW_ROWS - 1) / BW_ROWS) * 4 * 2 * 4);
   w.wt = o; o = up(o + HM3 * static_cast<size_t>(Cout) * 4);
   const size_t nchunk = (bn + 127) / 128;
   w.dwpart = o; o = up(o + nchunk * HM3 * static_cast<size_t>(Cout) * 4);
@@ -642,8 +651,6 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   f.out_agg = reinterpret_cast<float*>(ws + w.agg);
   f.skip_readout = true;
   cudaError_t e = geo_launch_all(f, st);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(ws + w.acc, 0, static_cast<size_t>(H) * 8, st);
   if (e != cudaSuccess) return e;
 
   {
@@ -717,7 +724,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   fa.qd = a.f.q_direction; fa.kd = a.f.k_direction; fa.qp = a.f.q_point; fa.kp = a.f.k_point;
   fa.val = a.f.values; fa.dscale = a.f.direction_scale; fa.xscale = a.f.distance_scale;
   fa.rotf = da.rotf; fa.agg = f.out_agg; fa.gvec = ga.gvec;
-  fa.dq = p.dq; fa.dk = p.dk; fa.dvr = p.dvr; fa.acc = p.acc;
+  fa.dq = p.dq; fa.dk = p.dk; fa.dvr = p.dvr; fa.acc = p.acc; fa.nrb = (N + BW_ROWS - 1) / BW_ROWS;
   fa.d_qd = a.d_q_direction; fa.d_kd = a.d_k_direction; fa.d_qp = a.d_q_point; fa.d_kp = a.d_k_point;
   fa.d_val = a.d_values; fa.d_rot = a.d_rotation; fa.d_trans = a.d_translation;
   fa.d_dscale = a.d_direction_scale; fa.d_xscale = a.d_distance_scale;

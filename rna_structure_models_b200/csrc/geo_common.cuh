@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace fipa {
 namespace geo {
@@ -25,9 +26,11 @@ __device__ __forceinline__ float softplus_stable(float x) {
   return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
 }
 
-// Score in the log2 domain and its parts.  The same instruction sequence is
-// used by the aggregation kernel, the attention-map kernel and the gradient
-// kernels so all of them see identical values.
+// Score in the log2 domain and its parts.  The same operation sequence is
+// used by the aggregation kernel (in packed pairs: fma.rn.f32x2 etc. round
+// each lane exactly like the scalar operation), the attention-map kernel and
+// the gradient kernels, so all of them see identical values.  The distance
+// is the hardware square-root approximation (sqrt.approx.f32, exact at 0).
 struct GeoPair {
   float s;            // log2(e) (A dot - B dist) / sqrt(3) + frame biases
   float dot, dist;    // <qd, kd>, |qp - kp|
@@ -42,7 +45,7 @@ __device__ __forceinline__ GeoPair geo_pair(const float4 q0, const float4 q1, co
   g.dy = __fsub_rn(q1.y, k1.y);
   g.dz = __fsub_rn(q1.z, k1.z);
   const float d2 = fmaf(g.dx, g.dx, fmaf(g.dy, g.dy, __fmul_rn(g.dz, g.dz)));
-  g.dist = __fsqrt_rn(d2);
+  g.dist = sm100::sqrt_approx(d2);
   g.s = __fadd_rn(__fadd_rn(fmaf(A, g.dot, -__fmul_rn(Bd, g.dist)), q0.w), k0.w);
   return g;
 }

@@ -9,11 +9,12 @@
 //   2. geo_prep_kernel    -- per (b, n, h): rotated directions, transformed
 //      points, R_j-rotated values (no translation), frame-mask bias.
 //   3. geo_attn_kernel<M> -- per (b, h, 128 queries) x 4 key splits (each split
-//      group of four warps stages its 32-key chunk in shared memory): online
-//      masked softmax in the log2 domain and aggregation of the rotated
-//      values; splits merged through shared memory; R_i^T back-rotation.
+//      group of four warps stages its 32-key chunks in shared memory, double
+//      buffered): scores and the value aggregation two keys per packed fp32
+//      instruction, online masked softmax in the log2 domain with lazy
+//      rescaling; splits merged through shared memory; R_i^T back-rotation.
 //   4. geo_map_kernel     -- optional: recomputes each score and writes the
-//      normalised attention row with coalesced stores.
+//      normalised attention map, 16 query rows per block, 16-byte stores.
 //   5. geo_readout_kernel -- output = flatten(vectors) . W (+ b), forced to
 //      zero for queries where no head has an allowed key.
 #include <cuda_fp16.h>
@@ -137,9 +138,25 @@ struct AttnArgs {
   float* agg;                // [B*H, N, VW] aggregated global-frame values, or null
 };
 
+// Staged chunk of 32 keys (one split group), laid out for packed pairs of
+// keys (a, b) = (2t, 2t + 1): per pair four float4
+//   (kd.x_a, kd.x_b, kd.y_a, kd.y_b) (kd.z_a, kd.z_b, bias_a, bias_b)
+//   (kp.x_a, kp.x_b, kp.y_a, kp.y_b) (kp.z_a, kp.z_b, 0, 0)
+// then the V rotated values as (v_e,a, v_e,b) pairs, padded to a multiple of
+// four floats so that every pair record starts 16-byte aligned.
+template <int V>
+struct GeoChunk {
+  static constexpr int PAIR = 16 + ((2 * V + 3) & ~3);   // floats per key pair, a multiple of 4 (float4 loads)
+  static constexpr int FLOATS = (GEO_CHUNK / 2) * PAIR;
+};
+
+// One 512-thread block per SM: the packed-pair loop keeps its working set in
+// registers without spilling (two blocks per SM at 64 registers spilled and
+// measured 9 % slower at B=2 N=2048 H=8 M=4, despite the single wave).
 template <int M>
-__global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, M <= 4 ? 2 : 1) geo_attn_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, 1) geo_attn_kernel(const AttnArgs a) {
   constexpr int V = 3 * M;
+  constexpr int PAIR = GeoChunk<V>::PAIR, CF = GeoChunk<V>::FLOATS;
   const int tid = threadIdx.x;
   const int r = tid % GEO_ROWS, split = tid / GEO_ROWS;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -157,31 +174,61 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, M <= 4 ? 2 : 1) geo_attn
   const unsigned char* pmrow =
       a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(in_range ? i : 0) * a.pms[2] : nullptr;
   const int64_t pj = a.pms[3];
+  const float2 qx = make_float2(q0.x, q0.x), qy = make_float2(q0.y, q0.y), qz = make_float2(q0.z, q0.z);
+  // a query whose frame is invalid (bias -inf) has no allowed key at all
+  const bool qdead = !(q0.w == 0.f);
+  const float2 px = make_float2(q1.x, q1.x), py = make_float2(q1.y, q1.y), pz = make_float2(q1.z, q1.z);
+  const float2 A2 = make_float2(sc.x, sc.x), nB2 = make_float2(-sc.y, -sc.y);
 
-  float m = -INFINITY, l = 0.f;
-  float acc[V];
+  float m = -INFINITY;
+  float2 l2 = make_float2(0.f, 0.f);
+  float2 acc[V];                                // (sum over even keys, sum over odd keys)
 #pragma unroll
-  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  for (int e = 0; e < V; ++e) acc[e] = make_float2(0.f, 0.f);
 
-  extern __shared__ float geo_merge[];  // [GEO_SPLIT][2 + V][GEO_ROWS], then the staged keys
-  // keys of one chunk staged per split group (four warps): [k0 | k1 | vr (padded)]
-  constexpr int SW = 8 + ((V + 3) & ~3);
-  float* stg = geo_merge + GEO_SPLIT * (2 + V) * GEO_ROWS + split * GEO_CHUNK * SW;
+  extern __shared__ float geo_merge[];  // [GEO_SPLIT][2 + V][GEO_ROWS], then 2 staged chunks per split
+  float* stg0 = geo_merge + GEO_SPLIT * (2 + V) * GEO_ROWS + split * 2 * CF;
   const uint32_t gbar = 1 + split;
   const int nchunk = (N + GEO_CHUNK - 1) / GEO_CHUNK;
+  // this thread's share of a chunk: source element e = (key, field) of the
+  // [32 keys][8 + V] chunk, staged into the packed-pair layout
+  constexpr int SRCW = 8 + V;
+  constexpr int PER = (GEO_CHUNK * SRCW + GEO_ROWS - 1) / GEO_ROWS;
+  auto fetch = [&](int ch, float (&vals)[PER]) {
+    const int j0 = ch * GEO_CHUNK;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int e = r + u * GEO_ROWS;
+      const int key = e / SRCW, f = e % SRCW, j = j0 + key;
+      float v = 0.f;
+      if (e < GEO_CHUNK * SRCW && ch < nchunk && j < N) {
+        if (f < 8) v = reinterpret_cast<const float*>(a.kg)[8 * (bh * N + j) + f];
+        else v = a.vg[(bh * N + j) * a.VW + (f - 8)];
+      }
+      vals[u] = v;
+    }
+  };
+  auto stage = [&](float* dst, const float (&vals)[PER]) {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int e = r + u * GEO_ROWS;
+      if (e >= GEO_CHUNK * SRCW) break;
+      const int key = e / SRCW, f = e % SRCW, t = key >> 1, q = key & 1;
+      // kg fields 0..7: kd.x kd.y kd.z bias kp.x kp.y kp.z 0
+      int pos;
+      if (f < 8) pos = (f >> 1) * 4 + (f & 1) * 2 + q;
+      else pos = 16 + 2 * (f - 8) + q;
+      dst[t * PAIR + pos] = vals[u];
+    }
+  };
+  float pre[PER];
+  int buf = 0;
+  fetch(split, pre);
+  stage(stg0, pre);
+  named_bar_sync(gbar, GEO_ROWS);
   for (int ch = split; ch < nchunk; ch += GEO_SPLIT) {
     const int j0 = ch * GEO_CHUNK;
-    named_bar_sync(gbar, GEO_ROWS);              // the previous chunk has been read
-    for (int e = r; e < GEO_CHUNK * SW; e += GEO_ROWS) {
-      const int it = e / SW, f = e % SW, j = j0 + it;
-      float v = 0.f;
-      if (j < N) {
-        if (f < 8) v = reinterpret_cast<const float*>(a.kg)[8 * (bh * N + j) + f];
-        else if (f - 8 < V) v = a.vg[(bh * N + j) * a.VW + (f - 8)];
-      }
-      stg[e] = v;
-    }
-    named_bar_sync(gbar, GEO_ROWS);
+    fetch(ch + GEO_SPLIT, pre);                   // the group's next chunk, in flight during this one
     uint32_t allowed = 0xffffffffu;
     if (pmrow) {
       allowed = 0u;
@@ -196,47 +243,67 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, M <= 4 ? 2 : 1) geo_attn
         for (int k = 0; k < GEO_CHUNK && j0 + k < N; ++k) allowed |= p[k * pj] ? (1u << k) : 0u;
       }
     }
-    float s[GEO_CHUNK];
-    float cm = -INFINITY;
+    if (j0 + GEO_CHUNK > N) allowed &= (N - j0 >= 32) ? 0xffffffffu : ((1u << (N - j0)) - 1u);
+    if (qdead) allowed = 0u;
+    const float* cur = stg0 + buf * CF;
+#pragma unroll 2
+    for (int t = 0; t < GEO_CHUNK / 2; ++t) {
+      const float4* kp4 = reinterpret_cast<const float4*>(cur + t * PAIR);
+      const float4 w0 = kp4[0], w1 = kp4[1], w2 = kp4[2], w3 = kp4[3];
+      // the score of geo_pair, two keys per instruction
+      const float2 dot = fma_f32x2(qx, make_float2(w0.x, w0.y),
+                                   fma_f32x2(qy, make_float2(w0.z, w0.w), mul_f32x2(qz, make_float2(w1.x, w1.y))));
+      const float2 dx = sub_f32x2(px, make_float2(w2.x, w2.y));
+      const float2 dy = sub_f32x2(py, make_float2(w2.z, w2.w));
+      const float2 dz = sub_f32x2(pz, make_float2(w3.x, w3.y));
+      const float2 d2 = fma_f32x2(dx, dx, fma_f32x2(dy, dy, mul_f32x2(dz, dz)));
+      const float2 dist = make_float2(sqrt_approx(d2.x), sqrt_approx(d2.y));
+      // (+ the query bias, 0 for a live query: the sum is unchanged)
+      float2 sv = add_f32x2(fma_f32x2(A2, dot, mul_f32x2(nB2, dist)), make_float2(w1.z, w1.w));
+      if (!((allowed >> (2 * t)) & 1u)) sv.x = -INFINITY;
+      if (!((allowed >> (2 * t + 1)) & 1u)) sv.y = -INFINITY;
+      const float cm = fmaxf(sv.x, sv.y);
+      if (cm > m + a.tau) {                         // lazy rescale: p stays below 2^tau
+        if (m != -INFINITY) {
+          const float f = ex2(m - cm);
+          const float2 f2 = make_float2(f, f);
+          l2 = mul_f32x2(l2, f2);
 #pragma unroll
-    for (int k = 0; k < GEO_CHUNK; ++k) {
-      const int j = j0 + k;
-      float v = -INFINITY;
-      if (j < N) {
-        const float4 k0 = *reinterpret_cast<const float4*>(stg + k * SW);
-        const float4 k1 = *reinterpret_cast<const float4*>(stg + k * SW + 4);
-        v = geo_score(q0, q1, k0, k1, sc.x, sc.y);
-        if (!((allowed >> k) & 1u)) v = -INFINITY;
+          for (int e = 0; e < V; ++e) acc[e] = mul_f32x2(acc[e], f2);
+        }
+        m = cm;
       }
-      s[k] = v;
-      cm = fmaxf(cm, v);
-    }
-    if (cm > m + a.tau) {
-      if (m != -INFINITY) {
-        const float f = ex2(m - cm);
-        l *= f;
+      const float mb = m == -INFINITY ? 0.f : m;    // while nothing is allowed every p is 0
+      const float2 y = sub_f32x2(sv, make_float2(mb, mb));
+      const float2 p2 = make_float2(ex2(y.x), ex2(y.y));
+      l2 = add_f32x2(l2, p2);
+      const float4* vp4 = reinterpret_cast<const float4*>(cur + t * PAIR + 16);
 #pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] *= f;
+      for (int e2 = 0; e2 < V / 2; ++e2) {
+        const float4 vv = vp4[e2];
+        acc[2 * e2] = fma_f32x2(p2, make_float2(vv.x, vv.y), acc[2 * e2]);
+        acc[2 * e2 + 1] = fma_f32x2(p2, make_float2(vv.z, vv.w), acc[2 * e2 + 1]);
       }
-      m = cm;
+      if (V & 1) {
+        const float2 vv = reinterpret_cast<const float2*>(cur + t * PAIR + 16)[V - 1];
+        acc[V - 1] = fma_f32x2(p2, vv, acc[V - 1]);
+      }
     }
-    if (m == -INFINITY) continue;
-#pragma unroll
-    for (int k = 0; k < GEO_CHUNK; ++k) {
-      const float p = ex2(s[k] - m);
-      l += p;
-      const float* vr = stg + k * SW + 8;
-#pragma unroll
-      for (int e = 0; e < V; ++e) acc[e] = fmaf(p, vr[e], acc[e]);
-    }
+    buf ^= 1;
+    stage(stg0 + buf * CF, pre);
+    named_bar_sync(gbar, GEO_ROWS);               // the next chunk is staged; this one is free
   }
+  const float l = l2.x + l2.y;
+  float accs[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) accs[e] = acc[e].x + acc[e].y;
 
   // merge the key splits
   auto sm_at = [&](int s2, int e) -> float& { return geo_merge[(s2 * (2 + V) + e) * GEO_ROWS + r]; };
   sm_at(split, 0) = m;
   sm_at(split, 1) = l;
 #pragma unroll
-  for (int e = 0; e < V; ++e) sm_at(split, 2 + e) = acc[e];
+  for (int e = 0; e < V; ++e) sm_at(split, 2 + e) = accs[e];
   __syncthreads();
   if (split != 0 || !in_range) return;
   float mf = -INFINITY;
@@ -287,27 +354,81 @@ struct MapArgs {
   float* att;   // [B, H, N, N]
 };
 
+// One block per (16 query rows, head, batch): each thread owns four
+// consecutive keys at a time, loads their terms once and writes the 16 rows'
+// probabilities for them as float4 stores (a warp writes 512 contiguous bytes
+// of a row).  Key terms are read N / 16 times per (b, h) instead of N times.
+constexpr int MAP_ROWS = 16;
+constexpr int MAP_KEYS = 4;
+
 __global__ void __launch_bounds__(256) geo_map_kernel(const MapArgs a) {
-  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int i0 = blockIdx.x * MAP_ROWS, h = blockIdx.y, b = blockIdx.z;
   const int N = a.N;
   const int64_t bh = static_cast<int64_t>(b) * a.H + h;
-  const float4 q0 = a.qg[2 * (bh * N + i)];
-  const float4 q1 = a.qg[2 * (bh * N + i) + 1];
-  const float2 sc = a.sc[h];
-  const float2 st = a.ml[bh * N + i];
-  const bool has = st.y > 0.f;
-  const float inv = has ? 1.f / st.y : 0.f;
-  float* dst = a.att + (bh * N + i) * static_cast<int64_t>(N);
-  const unsigned char* pmrow = a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] + static_cast<int64_t>(i) * a.pms[2] : nullptr;
-  for (int j = threadIdx.x; j < N; j += blockDim.x) {
-    float v = 0.f;
-    if (has && (!pmrow || pmrow[static_cast<int64_t>(j) * a.pms[3]])) {
-      const float4 k0 = a.kg[2 * (bh * N + j)];
-      const float4 k1 = a.kg[2 * (bh * N + j) + 1];
-      const float s = geo_score(q0, q1, k0, k1, sc.x, sc.y);
-      v = ex2(s - st.x) * inv;
+  __shared__ float4 qs[MAP_ROWS][2];
+  __shared__ float2 rs[MAP_ROWS];            // (running max m, 1 / l), l = 0 -> row of zeros
+  if (threadIdx.x < MAP_ROWS) {
+    const int i = i0 + threadIdx.x;
+    float4 q0 = make_float4(0.f, 0.f, 0.f, 0.f), q1 = q0;
+    float2 st = make_float2(0.f, 0.f);
+    if (i < N) {
+      q0 = a.qg[2 * (bh * N + i)];
+      q1 = a.qg[2 * (bh * N + i) + 1];
+      const float2 ml = a.ml[bh * N + i];
+      st = make_float2(ml.x, ml.y > 0.f ? 1.f / ml.y : 0.f);
     }
-    dst[j] = v;
+    qs[threadIdx.x][0] = q0;
+    qs[threadIdx.x][1] = q1;
+    rs[threadIdx.x] = st;
+  }
+  __syncthreads();
+  const float2 sc = a.sc[h];
+  const int nrows = N - i0 < MAP_ROWS ? N - i0 : MAP_ROWS;
+  const bool vec_store = (N & 3) == 0;
+  const unsigned char* pmb = a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] : nullptr;
+  const bool vec_mask = pmb != nullptr && a.pms[3] == 1 && (a.pms[2] & 3) == 0 &&
+                        (reinterpret_cast<uintptr_t>(pmb) & 3u) == 0;
+  for (int j0 = MAP_KEYS * threadIdx.x; j0 < N; j0 += MAP_KEYS * blockDim.x) {
+    float4 k0[MAP_KEYS], k1[MAP_KEYS];
+#pragma unroll
+    for (int t = 0; t < MAP_KEYS; ++t) {
+      const int j = j0 + t < N ? j0 + t : N - 1;
+      k0[t] = a.kg[2 * (bh * N + j)];
+      k1[t] = a.kg[2 * (bh * N + j) + 1];
+    }
+    const bool full = j0 + MAP_KEYS <= N;
+    for (int rr = 0; rr < nrows; ++rr) {
+      const int i = i0 + rr;
+      const float4 q0 = qs[rr][0], q1 = qs[rr][1];
+      const float2 st = rs[rr];
+      uint32_t allow = 0xffffffffu;
+      if (pmb) {
+        const unsigned char* pr = pmb + static_cast<int64_t>(i) * a.pms[2];
+        if (vec_mask && full) {
+          allow = *reinterpret_cast<const uint32_t*>(pr + j0);
+        } else {
+          allow = 0u;
+#pragma unroll
+          for (int t = 0; t < MAP_KEYS; ++t)
+            if (j0 + t < N && pr[static_cast<int64_t>(j0 + t) * a.pms[3]]) allow |= 0xffu << (8 * t);
+        }
+      }
+      float v[MAP_KEYS];
+#pragma unroll
+      for (int t = 0; t < MAP_KEYS; ++t) {
+        const float s = geo_score(q0, q1, k0[t], k1[t], sc.x, sc.y);
+        const bool ok = st.y > 0.f && ((allow >> (8 * t)) & 0xffu) != 0;
+        v[t] = ok ? ex2(s - st.x) * st.y : 0.f;
+      }
+      float* dst = a.att + (bh * N + i) * static_cast<int64_t>(N) + j0;
+      if (vec_store && full) {
+        *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+      } else {
+#pragma unroll
+        for (int t = 0; t < MAP_KEYS; ++t)
+          if (j0 + t < N) dst[t] = v[t];
+      }
+    }
   }
 }
 
@@ -359,7 +480,7 @@ __global__ void __launch_bounds__(256) geo_readout_kernel(const ReadArgs a) {
 template <int M>
 cudaError_t launch_attn(const AttnArgs& t, int B, int N, int H, cudaStream_t st) {
   dim3 grid((N + GEO_ROWS - 1) / GEO_ROWS, H, B);
-  const size_t smem = sizeof(float) * GEO_SPLIT * ((2 + 3 * M) * GEO_ROWS + GEO_CHUNK * (8 + ((3 * M + 3) & ~3)));
+  const size_t smem = sizeof(float) * GEO_SPLIT * ((2 + 3 * M) * GEO_ROWS + 2 * GeoChunk<3 * M>::FLOATS);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(geo_attn_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -453,7 +574,7 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
     ma.pm = t.pm;
     for (int d = 0; d < 4; ++d) ma.pms[d] = t.pms[d];
     ma.att = a.out_attention;
-    geo_map_kernel<<<dim3(a.N, a.H, a.B), 256, 0, st>>>(ma);
+    geo_map_kernel<<<dim3((a.N + MAP_ROWS - 1) / MAP_ROWS, a.H, a.B), 256, 0, st>>>(ma);
   }
 
   if (a.skip_readout) return cudaGetLastError();
