@@ -53,7 +53,7 @@ cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream);
 // forward prologue's outputs (recomputed) followed by the backward's.
 struct IpaBwdWorkspace {
   IpaWorkspace fwd;
-  size_t doh, du, qp, rowd, dqh, dqp, rsq, dkh, dva, dz2, csk, wb_part, g_part, total;
+  size_t doh, du, qp, rowd, dqh, dqp, rsq, dkh, dva, dz2, csk, pts, gsum, wb_part, g_part, total;
 };
 IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz);
 

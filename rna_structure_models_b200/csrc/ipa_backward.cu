@@ -18,15 +18,17 @@
 // dS is dL/dx.  The kernels:
 //   ipa_bwd_rows_kernel  one warp per (b, i, h): dO, dU, Q_pair (fp16 rows),
 //                        the row constant -(w_i + lse2_i) and D_i;
-//   ipa_bwd_q_kernel     one CTA per (b, h, 128 queries), 64-key tiles:
+//   query pass           one CTA per (b, h, 128 queries), 64-key tiles:
 //                        S, dP (tcgen05, TMEM), dS (fp16, TMEM), then
 //                        dQ_h += dS K_h, dQ_pair += dS Z2 (A = dS from TMEM),
 //                        row sums rs_i = sum_j dS_ij, RSo_i = sum_j dS_ij o_J;
-//   ipa_bwd_k_kernel     one CTA per (b, h, 128 keys), 64-query tiles:
+//   key pass             one CTA per (b, h, 128 keys), 64-query tiles:
 //                        S^T, dP^T, then P^T and dS^T (fp16, in place in
 //                        TMEM) as A operands of dV += P^T dO,
 //                        dZ2 += P^T dU + dS^T Q_pair, dK_h += dS^T Q_h, column
 //                        sums cs_j, CSo_j = sum_i dS_ij o_I;
+//   (both passes run as one grid, ipa_bwd_kernel, so that the key-pass CTAs
+//   fill the SMs the query pass leaves idle in its last wave)
 //   ipa_bwd_map_kernel   per residue, all heads: the augmented gradients
 //                        mapped back to q, k, v, the local points, the frames,
 //                        z1, z2 (sums over heads) and per-block partial sums of
@@ -74,6 +76,8 @@ struct BwdArgs {
   float* dva;            // [B*H, L, 64]
   float* dz2;            // [B*H, L, DZ]
   float4* csk;           // [B*H, L] (cs, CSo)
+  const float* pts;      // [B*H, L, 24]: tile-local query points gq' (12) | key points gk' (12), fp32
+  float* gsum;           // [B*H, L]: sum_i dS_ij |gq_i - gk_j|^2 per key (the d gamma sum, one side only)
   int* err;
 };
 
@@ -108,6 +112,11 @@ struct RowsArgs {
   __half* du;            // [B*H, L, DZ]
   __half* qp;            // [B*H, L, DZ]
   float2* rowd;          // [B*H, L]
+  View q_pts, k_pts;
+  const float4* oq;      // [B, nqt] 128-row query tile origins
+  const float4* ok;      // [B, nkt] 64-row key tile origins
+  int nqt, nkt;
+  float* pts;            // [B*H, L, 24]
 };
 
 // One warp per (b, i, h), heads fastest.  Lane l: scalar channel l (< 16),
@@ -183,6 +192,20 @@ __global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
     const float zq = a.z1_half ? __half2float(z1hr[c]) : z1r[c];
     qpr[c] = __float2half_rn(zq * wr[c]);
   }
+  // tile-local query and key points (the values the Q_h / K_h rows hold as
+  // hi + lo), for the key pass's d gamma sum: lane e < 12 query coordinate e,
+  // 12 <= lane < 24 key coordinate e - 12
+  if (lane < 24) {
+    const bool isq = lane < 12;
+    const int e = isq ? lane : lane - 12, pp = e / 3, xx = e % 3;
+    const View& pv = isq ? a.q_pts : a.k_pts;
+    const int64_t pb = b * pv.s[0] + i * pv.s[1] + h * pv.s[2] + pp * pv.s[3];
+    const float x0 = ldf(pv, pb), x1 = ldf(pv, pb + pv.s[4]), x2 = ldf(pv, pb + 2 * pv.s[4]);
+    const float4 og = isq ? a.oq[b * a.nqt + i / QT] : a.ok[b * a.nkt + i / KT];
+    const float ogx = xx == 0 ? og.x : xx == 1 ? og.y : og.z;
+    const float v = fmaf(Rm[3 * xx], x0, fmaf(Rm[3 * xx + 1], x1, Rm[3 * xx + 2] * x2)) + tc[xx] - ogx;
+    a.pts[bhl * 24 + lane] = live ? v : 0.f;
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
   if (lane == 0) {
@@ -228,18 +251,17 @@ enum { QB_QFULL = 0, QB_SFULL, QB_SFREE, QB_DSFULL, QB_DSFREE, QB_DRAIN, QB_FULL
        QB_COUNT = QB_EMPTY0 + MAX_NS };
 constexpr uint32_t QA_TMEM = QA_BAR + 8 * QB_COUNT, QA_ABORT = QA_TMEM + 8;
 
-__global__ void __launch_bounds__(NTH, 1)
-    ipa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_qp,
-                     const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_du,
-                     const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
-                     const __grid_constant__ CUtensorMap tm_z2, const BwdArgs a) {
+__device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_qh, const CUtensorMap& tm_qp,
+                                           const CUtensorMap& tm_do, const CUtensorMap& tm_du,
+                                           const CUtensorMap& tm_kh, const CUtensorMap& tm_vh,
+                                           const CUtensorMap& tm_z2, const BwdArgs& a) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (sb - raw_u32);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int I = blockIdx.x % a.nqt;
-  const int bh = blockIdx.x / a.nqt;
+  const int I = blk % a.nqt;
+  const int bh = blk / a.nqt;
   const int b = bh / a.H, h = bh % a.H;
   const int L = a.L, nt = a.nkt, DZ = a.DZ, np = DZ / 64, NS = a.ns;
   const QLayout lay = q_layout(DZ, NS);
@@ -526,28 +548,28 @@ __host__ __device__ inline KLayout k_layout(int DZ, int ns) {
   s.stg = s.z2 + np * 16384;
   s.stg_bytes = 16384 + 2 * np * 8192;      // Q_h 8 KB | dO 8 KB | Q_pair np x 8 KB | dU np x 8 KB
   s.aux = s.stg + ns * s.stg_bytes;
-  s.total = s.aux + 4096;
+  s.total = s.aux + 13312;
   return s;
 }
-// aux: per-query terms [MAX_NS][64] float4 (3 KB) | stage query-tile origin [MAX_NS] float4 | barriers
-constexpr uint32_t KA_Q = 0, KA_OQ = 3072, KA_BAR = 3136;
+// aux: per-query terms [MAX_NS][64] float4 (3 KB) | stage query-tile origin [MAX_NS] float4 | barriers |
+// per-stage query points [MAX_NS][64][12] floats (9 KB, from 4096)
+constexpr uint32_t KA_Q = 0, KA_OQ = 3072, KA_BAR = 3136, KA_QPTS = 4096;
 enum { KB_KFULL = 0, KB_SFULL, KB_PFULL, KB_ACC, KB_DRAIN, KB_FULL0, KB_EMPTY0 = KB_FULL0 + MAX_NS,
        KB_COUNT = KB_EMPTY0 + MAX_NS };
 constexpr uint32_t KA_TMEM = KA_BAR + 8 * KB_COUNT, KA_ABORT = KA_TMEM + 8, KA_PAIR = KA_ABORT + 8;
 
-__global__ void __launch_bounds__(NTH, 1)
-    ipa_bwd_k_kernel(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
-                     const __grid_constant__ CUtensorMap tm_z2, const __grid_constant__ CUtensorMap tm_qh,
-                     const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_qp,
-                     const __grid_constant__ CUtensorMap tm_du, const BwdArgs a) {
+__device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_kh, const CUtensorMap& tm_vh,
+                                           const CUtensorMap& tm_z2, const CUtensorMap& tm_qh,
+                                           const CUtensorMap& tm_do, const CUtensorMap& tm_qp,
+                                           const CUtensorMap& tm_du, const BwdArgs& a) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (sb - raw_u32);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nkp = (a.L + 127) / 128;
-  const int J2 = blockIdx.x % nkp;              // 128-key tile
-  const int bh = blockIdx.x / nkp;
+  const int J2 = blk % nkp;                     // 128-key tile
+  const int bh = blk / nkp;
   const int b = bh / a.H, h = bh % a.H;
   const int L = a.L, DZ = a.DZ, np = DZ / 64, NS = a.ns;
   const int nq = (L + 63) / 64;                 // 64-query tiles
@@ -628,6 +650,13 @@ __global__ void __launch_bounds__(NTH, 1)
         qinfo[s * 64 + lane + 32 * t] = e;
       }
       if (lane == 0) oqs[s] = oqv;
+      {
+        float* qp = reinterpret_cast<float*>(smem + lay.aux + KA_QPTS) + s * 64 * 12;
+        for (int e = lane; e < 64 * 12; e += 32) {
+          const int qq = i * 64 + e / 12;
+          qp[e] = qq < L ? a.pts[(static_cast<int64_t>(bh) * L + qq) * 24 + e % 12] : 0.f;
+        }
+      }
       __syncwarp();
       if (lane == 0) {
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
@@ -707,7 +736,10 @@ __global__ void __launch_bounds__(NTH, 1)
     const float4 ck = in_range ? a.colk[static_cast<int64_t>(bh) * L + key] : make_float4(0.f, 0.f, 0.f, -INFINITY);
     const int sub = r >> 6;                      // which 64-key origin tile
     const float4 okj = a.ok[b * a.nkt + (in_range ? key / 64 : 0)];
-    float cs = 0.f, co0 = 0.f, co1 = 0.f, co2 = 0.f;
+    float gk[12];                                // this key's tile-local points
+#pragma unroll
+    for (int e = 0; e < 12; ++e) gk[e] = in_range ? a.pts[(static_cast<int64_t>(bh) * L + key) * 24 + 12 + e] : 0.f;
+    float cs = 0.f, co0 = 0.f, co1 = 0.f, co2 = 0.f, gsum = 0.f;
     bool ok = true;
     for (int i = 0; i < nq && ok; ++i) {
       const int s = i % NS;
@@ -754,6 +786,32 @@ __global__ void __launch_bounds__(NTH, 1)
       co0 = fmaf(tsum, oqv.x, co0);
       co1 = fmaf(tsum, oqv.y, co1);
       co2 = fmaf(tsum, oqv.z, co2);
+      {
+        // sum_i dS_ij |gq_i - gk_j|^2 over this half's 32 queries, with the
+        // fp16 dS the MMAs multiply: gq_i - gk_j = gq'_i - (gk'_j + o_J - o_I)
+        const float ex = okj.x - oqv.x, ey = okj.y - oqv.y, ez = okj.z - oqv.z;
+        float e[12];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          e[3 * p] = gk[3 * p] + ex;
+          e[3 * p + 1] = gk[3 * p + 1] + ey;
+          e[3 * p + 2] = gk[3 * p + 2] + ez;
+        }
+        const float4* qp4 = reinterpret_cast<const float4*>(smem + lay.aux + KA_QPTS) + (s * 64 + 32 * half) * 3;
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+          const float4 g0 = qp4[3 * k], g1 = qp4[3 * k + 1], g2 = qp4[3 * k + 2];
+          const float q[12] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w, g2.x, g2.y, g2.z, g2.w};
+          float d2 = 0.f;
+#pragma unroll
+          for (int c = 0; c < 12; ++c) {
+            const float dd = q[c] - e[c];
+            d2 = fmaf(dd, dd, d2);
+          }
+          const float2 dsp = unpack_half2(pd[k >> 1]);
+          gsum = fmaf((k & 1) ? dsp.y : dsp.x, d2, gsum);
+        }
+      }
       tc_fence_after();
       tmem_st16(tmem + K_TM_S + 16 * half + lane_off, pp);
       tmem_st16(tmem + K_TM_DP + 16 * half + lane_off, pd);
@@ -767,13 +825,17 @@ __global__ void __launch_bounds__(NTH, 1)
     }
     const bool all_ok = __all_sync(0xffffffffu, ok);
     named_bar_sync(1, NSOFT);   // every thread is past its last read of the stage area
-    if (half == 1) reinterpret_cast<float4*>(smem + lay.stg)[r] = make_float4(cs, co0, co1, co2);
+    if (half == 1) {
+      reinterpret_cast<float4*>(smem + lay.stg)[r] = make_float4(cs, co0, co1, co2);
+      reinterpret_cast<float*>(smem + lay.stg + 2048)[r] = gsum;
+    }
     named_bar_sync(1, NSOFT);
     if (all_ok && !*abort_flag) {
       tc_fence_after();
       if (half == 0 && in_range) {
         const float4 o = reinterpret_cast<const float4*>(smem + lay.stg)[r];
         a.csk[static_cast<int64_t>(bh) * L + key] = make_float4(cs + o.x, co0 + o.y, co1 + o.z, co2 + o.w);
+        a.gsum[static_cast<int64_t>(bh) * L + key] = gsum + reinterpret_cast<const float*>(smem + lay.stg + 2048)[r];
       }
       auto store32 = [&](uint32_t tcol, float* dst_row) {
         uint32_t v[32];
@@ -802,6 +864,22 @@ __global__ void __launch_bounds__(NTH, 1)
   }
 }
 
+// Both passes in one grid: blocks [0, nqb) run the query pass, the rest the
+// key pass.  Each pass alone is 2.6 waves of one CTA per SM; in one grid the
+// key-pass CTAs fill the SMs the query pass leaves idle in its last wave.
+struct BwdMaps {
+  CUtensorMap q_qh, q_qp, q_do, q_du, q_kh, q_vh, q_z2;   // query pass
+  CUtensorMap k_kh, k_vh, k_z2, k_qh, k_do, k_qp, k_du;   // key pass
+};
+
+__global__ void __launch_bounds__(NTH, 1)
+    ipa_bwd_kernel(const __grid_constant__ BwdMaps m, const BwdArgs aq, const BwdArgs ak, const int nqb) {
+  if (static_cast<int>(blockIdx.x) < nqb)
+    bwd_q_body(blockIdx.x, m.q_qh, m.q_qp, m.q_do, m.q_du, m.q_kh, m.q_vh, m.q_z2, aq);
+  else
+    bwd_k_body(blockIdx.x - nqb, m.k_kh, m.k_vh, m.k_z2, m.k_qh, m.k_do, m.k_qp, m.k_du, ak);
+}
+
 // ------------------------------------------------------------------ mapping
 struct MapArgs {
   int B, L, H, DZ, RCz, Cz, R, rb, nblk;
@@ -821,6 +899,7 @@ struct MapArgs {
   const float* dva;
   const float* dz2;
   const float4* csk;
+  const float* gsum;     // [B*H, L] sum_i dS_ij |gq_i - gk_j|^2 per key
   int nqt, nkt;
   // gradients (contiguous fp32)
   float *d_q, *d_k, *d_v, *d_qpts, *d_kpts, *d_vpts, *d_rot, *d_trans, *d_z1, *d_z2;
@@ -868,7 +947,6 @@ __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
         a.d_v[o3 * C + e] = dv[e];
       }
       // query and key points: d gq = Gq2c + 2c (RSo - rs gq_c), d gk = 2c (Gk' + CSo - cs gk_c)
-      double g_q = 0.0, g_k = 0.0, g_x = 0.0;
       for (int p = 0; p < PQ; ++p) {
         float lq[3], lk[3], gqc[3], gkc[3], dgq[3], dgk[3];
         for (int y = 0; y < 3; ++y) {
@@ -886,9 +964,6 @@ __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
           const float gk1 = dk[e] + dk[e + 6 * PQ];                    // query hi + lo columns
           dgq[x] = gq2c + 2.f * c * (rso[x] - rq.x * gqc[x]);
           dgk[x] = 2.f * c * (gk1 + cso[x] - ck.x * gkc[x]);
-          g_q += static_cast<double>(rq.x) * gqc[x] * gqc[x];
-          g_k += static_cast<double>(ck.x) * gkc[x] * gkc[x];
-          g_x += static_cast<double>(gkc[x]) * (static_cast<double>(gk1) + cso[x]);
         }
         for (int y = 0; y < 3; ++y) {
           a.d_qpts[(o3 * PQ + p) * 3 + y] = Rm[y] * dgq[0] + Rm[3 + y] * dgq[1] + Rm[6 + y] * dgq[2];
@@ -899,7 +974,8 @@ __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
           fr[9 + x] += dgq[x] + dgk[x];
         }
       }
-      gsum = -static_cast<double>(kLog2e) * a.w_L * a.w_C * 0.5 * (g_q + g_k - 2.0 * g_x);
+      // d gamma: x_ij holds -(log2(e) w_L w_C / 2) gamma sum_p |gq_ip - gk_jp|^2
+      gsum = -static_cast<double>(kLog2e) * a.w_L * a.w_C * 0.5 * static_cast<double>(a.gsum[bhl]);
       // value points
       for (int p = 0; p < PV; ++p) {
         float lv[3], dgv[3];
@@ -1037,6 +1113,8 @@ IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz) {
   w.dva = o; o = up(o + bhl * 64 * 4);
   w.dz2 = o; o = up(o + bhl * DZ * 4);
   w.csk = o; o = up(o + bhl * 16);
+  w.pts = o; o = up(o + bhl * 24 * 4);
+  w.gsum = o; o = up(o + bhl * 4);
   w.wb_part = o; o = up(o + static_cast<size_t>(B) * nblk * H * DZ * 4);
   w.g_part = o; o = up(o + static_cast<size_t>(B) * nblk * H * 8);
   w.total = o;
@@ -1070,6 +1148,11 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   ra.du = reinterpret_cast<__half*>(ws + w.du);
   ra.qp = reinterpret_cast<__half*>(ws + w.qp);
   ra.rowd = reinterpret_cast<float2*>(ws + w.rowd);
+  ra.q_pts = f.q_pts; ra.k_pts = f.k_pts;
+  ra.oq = reinterpret_cast<const float4*>(ws + fw.oq);
+  ra.ok = reinterpret_cast<const float4*>(ws + fw.ok);
+  ra.nqt = f.nqt; ra.nkt = f.nkt;
+  ra.pts = reinterpret_cast<float*>(ws + w.pts);
   const int64_t warps = static_cast<int64_t>(B) * L * H;
   ipa_bwd_rows_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(ra);
   e = cudaGetLastError();
@@ -1097,50 +1180,41 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   ba.dva = reinterpret_cast<float*>(ws + w.dva);
   ba.dz2 = reinterpret_cast<float*>(ws + w.dz2);
   ba.csk = reinterpret_cast<float4*>(ws + w.csk);
+  ba.pts = reinterpret_cast<const float*>(ws + w.pts);
+  ba.gsum = reinterpret_cast<float*>(ws + w.gsum);
   ba.err = f.err;
 
   const uint64_t rowb = static_cast<uint64_t>(L) * DH * 2;
-  // 3. query pass
+  // 3.-4. query and key passes, one grid
   {
-    CUtensorMap tqh, tqp, tdo, tdu, tkh, tvh, tz2;
-    bool ok = encode_tmap_f16_3d(&tqh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, 128) &&
-              encode_tmap_f16_panels(&tqp, ws + w.qp, DZ, L, bh, 128, np) &&
-              encode_tmap_f16_3d(&tdo, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, 128) &&
-              encode_tmap_f16_panels(&tdu, ws + w.du, DZ, L, bh, 128, np) &&
-              encode_tmap_f16_3d(&tkh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, 64) &&
-              encode_tmap_f16_3d(&tvh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, 64) &&
-              encode_tmap_f16_panels(&tz2, ws + fw.z2, DZ, L, B, 64, np);
+    BwdMaps mp;
+    bool ok = encode_tmap_f16_3d(&mp.q_qh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, 128) &&
+              encode_tmap_f16_panels(&mp.q_qp, ws + w.qp, DZ, L, bh, 128, np) &&
+              encode_tmap_f16_3d(&mp.q_do, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, 128) &&
+              encode_tmap_f16_panels(&mp.q_du, ws + w.du, DZ, L, bh, 128, np) &&
+              encode_tmap_f16_3d(&mp.q_kh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, 64) &&
+              encode_tmap_f16_3d(&mp.q_vh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, 64) &&
+              encode_tmap_f16_panels(&mp.q_z2, ws + fw.z2, DZ, L, B, 64, np) &&
+              encode_tmap_f16_3d(&mp.k_kh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, 128) &&
+              encode_tmap_f16_3d(&mp.k_vh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, 128) &&
+              encode_tmap_f16_panels(&mp.k_z2, ws + fw.z2, DZ, L, B, 128, np) &&
+              encode_tmap_f16_3d(&mp.k_qh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, 64) &&
+              encode_tmap_f16_3d(&mp.k_do, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, 64) &&
+              encode_tmap_f16_panels(&mp.k_qp, ws + w.qp, DZ, L, bh, 64, np) &&
+              encode_tmap_f16_panels(&mp.k_du, ws + w.du, DZ, L, bh, 64, np);
     if (!ok) return cudaErrorInvalidValue;
     const QLayout l1 = q_layout(DZ, 1);
     ba.ns = stages_for(l1.stg, l1.stg_bytes, 2048);
-    const QLayout lq = q_layout(DZ, ba.ns);
-    const uint32_t smem = lq.total + 1024;
-    e = cudaFuncSetAttribute(ipa_bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    ipa_bwd_q_kernel<<<static_cast<unsigned>(bh * f.nqt), NTH, smem, stream>>>(tqh, tqp, tdo, tdu, tkh, tvh, tz2, ba);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  // 4. key pass
-  {
-    CUtensorMap tkh, tvh, tz2, tqh, tdo, tqp, tdu;
-    bool ok = encode_tmap_f16_3d(&tkh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, 128) &&
-              encode_tmap_f16_3d(&tvh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, 128) &&
-              encode_tmap_f16_panels(&tz2, ws + fw.z2, DZ, L, B, 128, np) &&
-              encode_tmap_f16_3d(&tqh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, 64) &&
-              encode_tmap_f16_3d(&tdo, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, 64) &&
-              encode_tmap_f16_panels(&tqp, ws + w.qp, DZ, L, bh, 64, np) &&
-              encode_tmap_f16_panels(&tdu, ws + w.du, DZ, L, bh, 64, np);
-    if (!ok) return cudaErrorInvalidValue;
-    const KLayout l1 = k_layout(DZ, 1);
+    const KLayout k1 = k_layout(DZ, 1);
     BwdArgs kb = ba;
-    kb.ns = stages_for(l1.stg, l1.stg_bytes, 4096);
-    const KLayout lk = k_layout(DZ, kb.ns);
-    const uint32_t smem = lk.total + 1024;
-    e = cudaFuncSetAttribute(ipa_bwd_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    kb.ns = stages_for(k1.stg, k1.stg_bytes, 13312);
+    const uint32_t sq = q_layout(DZ, ba.ns).total, sk = k_layout(DZ, kb.ns).total;
+    const uint32_t smem = (sq > sk ? sq : sk) + 1024;
+    e = cudaFuncSetAttribute(ipa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const int nkp = (L + 127) / 128;
-    ipa_bwd_k_kernel<<<static_cast<unsigned>(bh * nkp), NTH, smem, stream>>>(tkh, tvh, tz2, tqh, tdo, tqp, tdu, kb);
+    const int nqb = static_cast<int>(bh) * f.nqt;
+    const int nkb = static_cast<int>(bh) * ((L + 127) / 128);
+    ipa_bwd_kernel<<<static_cast<unsigned>(nqb + nkb), NTH, smem, stream>>>(mp, ba, kb, nqb);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -1153,7 +1227,7 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   m.q_pts = f.q_pts; m.k_pts = f.k_pts; m.v_pts = f.v_pts; m.g_out = a.g_out; m.out = a.out; m.uagg = a.uagg;
   m.frame = ba.frame; m.cen = ba.cen; m.oq = ba.oq; m.ok = ba.ok; m.headc = ba.headc; m.wqp = ba.wqp;
   m.z1f = ba.z1f; m.dqh = ba.dqh; m.dqp = ba.dqp; m.rsq = ba.rsq; m.dkh = ba.dkh; m.dva = ba.dva;
-  m.dz2 = ba.dz2; m.csk = ba.csk; m.nqt = f.nqt; m.nkt = f.nkt;
+  m.dz2 = ba.dz2; m.csk = ba.csk; m.gsum = ba.gsum; m.nqt = f.nqt; m.nkt = f.nkt;
   m.d_q = a.d_q; m.d_k = a.d_k; m.d_v = a.d_v; m.d_qpts = a.d_q_pts; m.d_kpts = a.d_k_pts; m.d_vpts = a.d_v_pts;
   m.d_rot = a.d_rot; m.d_trans = a.d_trans; m.d_z1 = a.d_z1; m.d_z2 = a.d_z2;
   m.wb_part = reinterpret_cast<float*>(ws + w.wb_part);
