@@ -37,7 +37,7 @@ import numpy as np
 
 from .ipa_dense import ipa_constants
 
-__all__ = ["ipa_grad"]
+__all__ = ["ipa_grad", "ipa_grad_gamma_scale"]
 
 
 def _f64(a):
@@ -138,3 +138,78 @@ def ipa_grad(inp: dict, g_out, *, w_L=None, w_C=None, scalar_scale=None) -> dict
     d_trans = d_trans + t1 + t2 + t3
     return {"q": d_q, "k": d_k, "v": d_v, "q_pts": d_qp, "k_pts": d_kp, "v_pts": d_vp, "rot": d_rot,
             "trans": d_trans, "z1": d_z1, "z2": d_z2, "w_bias": d_wb, "gamma": d_gamma}
+
+
+def ipa_grad_gamma_scale(inp: dict, g_out, *, w_L=None, w_C=None, scalar_scale=None) -> np.ndarray:
+    """Per head, the root-sum-square of the magnitudes of the terms that
+    d gamma sums (a tolerance scale, not a gradient).
+
+    Steps 5' and 4' above give d gamma_h = -w_L w_C / 2 sum_{b,i,j} dl d2 with
+    dl_ij = a_ij (da_ij - D_i), D_i = sum_k a_ik da_ik.  Each term is at most
+    t_ij = w_L w_C / 2 a_ij (|da_ij| + |D_i|) d2_ij in magnitude, and a d gamma
+    formed from rounded operands carries errors of about (unit roundoff) x t_ij
+    per term; errors without a common sign add in quadrature, so their sum is
+    of the size sqrt(sum t_ij^2), returned here [H].  The signed sum itself
+    cancels: |d gamma_h| is typically 10^-3 .. 10^-1 of this scale at a few
+    hundred residues.
+
+    da is taken with the value points relative to the mean translation of the
+    batch element's live residues: that shifts each row of da by a constant,
+    which dl does not see, and makes the scale independent of where the
+    structure sits (under a global rigid motion it is unchanged).
+
+    One (b, h) slice at a time, [L, L] arrays only (the forward of ipa_dense:
+    logits, masked softmax, outputs; then da and D as in ipa_grad)."""
+    q, k, v = _f64(inp["q"]), _f64(inp["k"]), _f64(inp["v"])
+    q_pts, k_pts, v_pts = _f64(inp["q_pts"]), _f64(inp["k_pts"]), _f64(inp["v_pts"])
+    rot, trans = _f64(inp["rot"]), _f64(inp["trans"])
+    z1, z2 = _f64(inp["z1"]), _f64(inp["z2"])
+    w_bias, gamma = _f64(inp["w_bias"]), _f64(inp["gamma"])
+    mask = np.asarray(inp["mask"], dtype=bool)
+    B, L, H, C = q.shape
+    Pq, Pv = q_pts.shape[3], v_pts.shape[3]
+    R, Cz = z1.shape[2], z1.shape[3]
+    consts = ipa_constants(C, Pq)
+    w_L = consts["w_L"] if w_L is None else w_L
+    w_C = consts["w_C"] if w_C is None else w_C
+    ss = consts["scalar_scale"] if scalar_scale is None else scalar_scale
+    g = _f64(g_out)
+    sq = np.zeros(H)
+    for b in range(B):
+        allowed = mask[b][:, None] & mask[b][None, :]
+        live = allowed.any(axis=1)
+        gq = np.einsum("lxy,lhpy->lhpx", rot[b], q_pts[b]) + trans[b][:, None, None, :]
+        gk = np.einsum("lxy,lhpy->lhpx", rot[b], k_pts[b]) + trans[b][:, None, None, :]
+        gv = np.einsum("lxy,lhpy->lhpx", rot[b], v_pts[b]) + trans[b][:, None, None, :]
+        cen = trans[b][mask[b]].mean(axis=0) if mask[b].any() else np.zeros(3)
+        for h in range(H):
+            d2 = np.zeros((L, L))
+            for p in range(Pq):
+                dd = gq[:, None, h, p, :] - gk[None, :, h, p, :]
+                d2 += np.einsum("ijx,ijx->ij", dd, dd)
+            wz1 = (z1[b] * w_bias[:, h][None, None, :]).reshape(L, R * Cz)
+            bias = wz1 @ z2[b].reshape(L, R * Cz).T                   # sum_c w_bias[c, h] z_ijc
+            logits = w_L * (ss * q[b, :, h] @ k[b, :, h].T + bias - gamma[h] * w_C / 2.0 * d2)
+            neg = np.where(allowed, logits, -np.inf)
+            mx = np.where(live, neg.max(axis=1), 0.0)
+            e = np.where(allowed, np.exp(neg - mx[:, None]), 0.0)
+            ssum = e.sum(axis=1)
+            a = np.where(ssum[:, None] > 0, e / np.where(ssum > 0, ssum, 1.0)[:, None], 0.0)
+            gh = np.where(live[:, None], g[b, :, h], 0.0)
+            g_o = gh[:, :C]
+            g_pt = gh[:, C:C + 3 * Pv].reshape(L, Pv, 3)
+            g_n = gh[:, C + 3 * Pv:C + 4 * Pv]
+            g_pair = gh[:, C + 4 * Pv:]
+            og = np.einsum("ij,jpx->ipx", a, gv[:, h])
+            o_pt = np.einsum("ixy,ipx->ipy", rot[b], og - trans[b][:, None, :])
+            nrm = np.sqrt(np.einsum("ipx,ipx->ip", o_pt, o_pt))
+            unit = np.where((nrm > 0)[..., None], o_pt / np.where(nrm > 0, nrm, 1.0)[..., None], 0.0)
+            d_og = np.einsum("ixy,ipy->ipx", rot[b], g_pt + g_n[..., None] * unit)
+            gz1 = (z1[b] * g_pair[:, None, :]).reshape(L, R * Cz)
+            gv_c = gv[:, h] - cen[None, None, :]
+            da = (g_o @ v[b, :, h].T + d_og.reshape(L, -1) @ gv_c.reshape(L, -1).T
+                  + gz1 @ z2[b].reshape(L, R * Cz).T)
+            D = np.sum(a * da, axis=1)
+            t = w_L * w_C / 2.0 * a * (np.abs(da) + np.abs(D)[:, None]) * d2
+            sq[h] += float(np.sum(t * t))
+    return np.sqrt(sq)

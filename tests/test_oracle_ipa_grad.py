@@ -135,3 +135,52 @@ def test_blocked_gradient_equals_the_dense_gradient():
         got = ipa_grad_blocked(inp, g, block=block)
         for key in KEYS:
             assert np.allclose(got[key], ref[key], rtol=1e-10, atol=1e-12), (block, key)
+
+
+# ---- the d gamma tolerance scale (root-sum-square of the summed terms' magnitudes)
+
+def test_gamma_scale_one_residue_closed_form():
+    # one live residue: the softmax has the single key j = i, a = 1 and D = da,
+    # so the one term's magnitude is w_L w_C |da| d2_ii, with d2_ii =
+    # sum_p |R (q_p - k_p)|^2 (R as stored: orthonormal to float32 precision
+    # only, so the rotation is kept).  With the translation at
+    # zero every output (o_pt = R^T a gv included) is homogeneous of degree 1
+    # in a, so da = <g, out>.  A second, masked residue contributes nothing.
+    from oracle import ipa_grad_gamma_scale
+    from oracle.ipa_dense import ipa_constants
+    inp = as64(ipa_inputs(IpaDims(B=1, L=2, H=3, C=4, Pq=2, Pv=3, R=2, Cz=3), 5, jitter=0.5))
+    inp["mask"] = inp["mask"].copy()
+    inp["mask"][0, 1] = False
+    inp["trans"] = np.zeros_like(inp["trans"])
+    g = upstream(inp, 6)
+    got = ipa_grad_gamma_scale(inp, g)
+    cst = ipa_constants(4, 2)
+    out = ipa_dense(inp)
+    for h in range(3):
+        da = float(np.sum(g[0, 0, h] * out[0, 0, h]))
+        d2 = float(np.sum((inp["rot"][0, 0] @ (inp["q_pts"][0, 0, h] - inp["k_pts"][0, 0, h]).T) ** 2))
+        want = cst["w_L"] * cst["w_C"] * abs(da) * d2
+        assert abs(got[h] - want) <= 1e-10 * max(1.0, want), (h, got[h], want)
+
+
+def test_gamma_scale_bounds_the_gradient_and_is_invariant():
+    # |d gamma_h| <= sum |terms| <= sqrt(n_h) * scale_h (Cauchy-Schwarz, since
+    # |dl| <= a (|da| + |D|)); the scale is even and of degree 1 in g_out and
+    # unchanged by a global rigid motion
+    from oracle import ipa_grad_gamma_scale
+    inp = as64(ipa_inputs(IpaDims(B=2, L=9, H=3, C=4, Pq=2, Pv=3, R=2, Cz=3), 7, jitter=0.5))
+    inp["mask"] = inp["mask"].copy()
+    inp["mask"][1, 5:] = False
+    g = upstream(inp, 8)
+    sc = ipa_grad_gamma_scale(inp, g)
+    n = int(sum(int(m.sum()) ** 2 for m in inp["mask"]))
+    dg = ipa_grad(inp, g)["gamma"]
+    assert np.all(sc > 0)
+    assert np.all(np.abs(dg) <= math.sqrt(n) * sc * (1 + 1e-12))
+    assert np.allclose(ipa_grad_gamma_scale(inp, -2.5 * g), 2.5 * sc, rtol=1e-12)
+    rng = np.random.default_rng(9)
+    G = random_rotations(rng, 1)[0]
+    moved = dict(inp)
+    moved["rot"] = np.einsum("xy,blyz->blxz", G, inp["rot"])
+    moved["trans"] = inp["trans"] @ G.T + rng.normal(size=3) * 5.0
+    assert np.allclose(ipa_grad_gamma_scale(moved, g), sc, rtol=1e-9)
