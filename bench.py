@@ -45,8 +45,8 @@ REF_BUDGET_S = 90.0
 # it was taken on (sha256 over the sources listed in CORE_SOURCES).
 CORE_KERNEL = "ipa_attention_pair_kernel"
 CORE_SOURCES = ("ipa_attention_pair.cu", "ipa_epilogue.cuh", "sm100.cuh")
-NCU_TRAFFIC = {"kernel_sha256": "33c314293e9746ffee45dfd4781970575e1a13c1f72128943478c88373d4423a",
-               "bytes_per_launch": 30.75e6}
+NCU_TRAFFIC = {"kernel_sha256": "16411912ce0b50670e6fe8fc3ae57a60a675ce0e4fad1e05e642468437fdad69",
+               "bytes_per_launch": 29.32e6}
 
 
 def ipa_flops(B, L, n_valid=None, heads=H, rcz=R * CZ):
@@ -328,6 +328,18 @@ def cpu_oracle_configs(seconds):
             rows += len(r)
         res.append({"config": f"long-context L={Lc}", "seconds": t * Lc / rows, "extrapolated": rows < Lc,
                     "rows_timed": rows})
+    # the direction/distance variant (B=2, N=2048): 64-row blocks, extrapolated in rows
+    from oracle import geo_dense_blocked
+    g = geo_inputs(GeoDims(B=2, N=2048, H=8, M=4, Cout=256), 0)
+    rows, t = 0, 0.0
+    while rows < 2048 and t < seconds / 4:
+        r = np.arange(rows, min(rows + 64, 2048))
+        t0 = time.perf_counter()
+        geo_dense_blocked(g, rows=r, block=64)
+        t += time.perf_counter() - t0
+        rows += len(r)
+    res.append({"config": "geometric variant B=2 N=2048", "seconds": t * 2048 / rows, "extrapolated": rows < 2048,
+                "rows_timed": rows})
     return res
 
 
@@ -520,13 +532,13 @@ def main():
         d2h = res.numel() * res.element_size()
         ke = max(3, min(K, 50))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        hc = api.IpaHostCalls(1, L, H, C, PQ, PV, R, CZ, slots=2, device=dev)
-        outs = [res, torch.empty_like(res).pin_memory()]
+        hc = api.IpaHostCalls(1, L, H, C, PQ, PV, R, CZ, slots=3, device=dev)
+        outs = [res] + [torch.empty_like(res).pin_memory() for _ in range(2)]
         for _ in range(max(1, min(args.warmup, 3))):
-            hc.run([pinned] * 2, outs)
+            hc.run([pinned] * 3, outs)
         hc.check()
         # one call at a time on one stream: copies, kernels and the copy back in series
-        s0, s1 = hc.streams
+        s0 = hc.streams[0]
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -540,12 +552,14 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
         e0.record(s0)
-        s1.wait_event(e0)
+        for st in hc.streams[1:]:
+            st.wait_event(e0)
         for k in range(ke):
-            hc.call(pinned, outs[k & 1], k & 1)
-        done = torch.cuda.Event()
-        done.record(s1)
-        s0.wait_event(done)
+            hc.call(pinned, outs[k % 3], k % 3)
+        for st in hc.streams[1:]:
+            done = torch.cuda.Event()
+            done.record(st)
+            s0.wait_event(done)
         e1.record(s0)
         torch.cuda.synchronize()
         hc.check()
@@ -553,7 +567,7 @@ def main():
         line["e2e"] = {"value": aggregate_tflops(world, flops, ke, te), "unit": UNIT,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
                        "ms_per_step": te / ke,
-                       "api": "C entry point ipa_attn_fwd_host, two streams (tests/c/e2e_host.c does the same)",
+                       "api": "C entry point ipa_attn_fwd_host, three streams (tests/c/e2e_host.c: the same call on two)",
                        "serial_ms_per_step": t_serial / ke}
 
     # second hot-path row: direction/distance geometric attention (B=2, N=2048)

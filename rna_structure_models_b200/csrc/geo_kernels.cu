@@ -246,11 +246,13 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, 1) geo_attn_kernel(const
     if (j0 + GEO_CHUNK > N) allowed &= (N - j0 >= 32) ? 0xffffffffu : ((1u << (N - j0)) - 1u);
     if (qdead) allowed = 0u;
     const float* cur = stg0 + buf * CF;
-#pragma unroll 2
+    // pass 1: the chunk's 32 scores (two per packed instruction) and their maximum
+    float2 sv2[GEO_CHUNK / 2];
+    float cm = -INFINITY;
+#pragma unroll
     for (int t = 0; t < GEO_CHUNK / 2; ++t) {
       const float4* kp4 = reinterpret_cast<const float4*>(cur + t * PAIR);
       const float4 w0 = kp4[0], w1 = kp4[1], w2 = kp4[2], w3 = kp4[3];
-      // the score of geo_pair, two keys per instruction
       const float2 dot = fma_f32x2(qx, make_float2(w0.x, w0.y),
                                    fma_f32x2(qy, make_float2(w0.z, w0.w), mul_f32x2(qz, make_float2(w1.x, w1.y))));
       const float2 dx = sub_f32x2(px, make_float2(w2.x, w2.y));
@@ -258,35 +260,41 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, 1) geo_attn_kernel(const
       const float2 dz = sub_f32x2(pz, make_float2(w3.x, w3.y));
       const float2 d2 = fma_f32x2(dx, dx, fma_f32x2(dy, dy, mul_f32x2(dz, dz)));
       const float2 dist = make_float2(sqrt_approx(d2.x), sqrt_approx(d2.y));
-      // (+ the query bias, 0 for a live query: the sum is unchanged)
       float2 sv = add_f32x2(fma_f32x2(A2, dot, mul_f32x2(nB2, dist)), make_float2(w1.z, w1.w));
       if (!((allowed >> (2 * t)) & 1u)) sv.x = -INFINITY;
       if (!((allowed >> (2 * t + 1)) & 1u)) sv.y = -INFINITY;
-      const float cm = fmaxf(sv.x, sv.y);
-      if (cm > m + a.tau) {                         // lazy rescale: p stays below 2^tau
-        if (m != -INFINITY) {
-          const float f = ex2(m - cm);
-          const float2 f2 = make_float2(f, f);
-          l2 = mul_f32x2(l2, f2);
+      sv2[t] = sv;
+      cm = fmax3(cm, sv.x, sv.y);
+    }
+    if (cm > m + a.tau) {                           // lazy rescale: p stays below 2^tau
+      if (m != -INFINITY) {
+        const float f = ex2(m - cm);
+        const float2 f2 = make_float2(f, f);
+        l2 = mul_f32x2(l2, f2);
 #pragma unroll
-          for (int e = 0; e < V; ++e) acc[e] = mul_f32x2(acc[e], f2);
+        for (int e = 0; e < V; ++e) acc[e] = mul_f32x2(acc[e], f2);
+      }
+      m = cm;
+    }
+    if (m != -INFINITY) {
+      // pass 2: probabilities and the value aggregation
+      const float2 mb = make_float2(m, m);
+#pragma unroll
+      for (int t = 0; t < GEO_CHUNK / 2; ++t) {
+        const float2 y = sub_f32x2(sv2[t], mb);
+        const float2 p2 = make_float2(ex2(y.x), ex2(y.y));
+        l2 = add_f32x2(l2, p2);
+        const float4* vp4 = reinterpret_cast<const float4*>(cur + t * PAIR + 16);
+#pragma unroll
+        for (int e2 = 0; e2 < V / 2; ++e2) {
+          const float4 vv = vp4[e2];
+          acc[2 * e2] = fma_f32x2(p2, make_float2(vv.x, vv.y), acc[2 * e2]);
+          acc[2 * e2 + 1] = fma_f32x2(p2, make_float2(vv.z, vv.w), acc[2 * e2 + 1]);
         }
-        m = cm;
-      }
-      const float mb = m == -INFINITY ? 0.f : m;    // while nothing is allowed every p is 0
-      const float2 y = sub_f32x2(sv, make_float2(mb, mb));
-      const float2 p2 = make_float2(ex2(y.x), ex2(y.y));
-      l2 = add_f32x2(l2, p2);
-      const float4* vp4 = reinterpret_cast<const float4*>(cur + t * PAIR + 16);
-#pragma unroll
-      for (int e2 = 0; e2 < V / 2; ++e2) {
-        const float4 vv = vp4[e2];
-        acc[2 * e2] = fma_f32x2(p2, make_float2(vv.x, vv.y), acc[2 * e2]);
-        acc[2 * e2 + 1] = fma_f32x2(p2, make_float2(vv.z, vv.w), acc[2 * e2 + 1]);
-      }
-      if (V & 1) {
-        const float2 vv = reinterpret_cast<const float2*>(cur + t * PAIR + 16)[V - 1];
-        acc[V - 1] = fma_f32x2(p2, vv, acc[V - 1]);
+        if (V & 1) {
+          const float2 vv = reinterpret_cast<const float2*>(cur + t * PAIR + 16)[V - 1];
+          acc[V - 1] = fma_f32x2(p2, vv, acc[V - 1]);
+        }
       }
     }
     buf ^= 1;

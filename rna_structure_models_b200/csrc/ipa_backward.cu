@@ -17,7 +17,8 @@
 //                                          forward output and U
 // dS is dL/dx.  The kernels:
 //   ipa_bwd_rows_kernel  one warp per (b, i, h): dO, dU, Q_pair (fp16 rows),
-//                        the row constant -(w_i + lse2_i) and D_i;
+//                        the row constant -(w_i + lse2_i), D_i and the query
+//                        and key points relative to the centroid (fp32);
 //   query pass           one CTA per (b, h, 128 queries), 64-key tiles:
 //                        S, dP (tcgen05, TMEM), dS (fp16, TMEM), then
 //                        dQ_h += dS K_h, dQ_pair += dS Z2 (A = dS from TMEM),
@@ -26,7 +27,9 @@
 //                        S^T, dP^T, then P^T and dS^T (fp16, in place in
 //                        TMEM) as A operands of dV += P^T dO,
 //                        dZ2 += P^T dU + dS^T Q_pair, dK_h += dS^T Q_h, column
-//                        sums cs_j, CSo_j = sum_i dS_ij o_I;
+//                        sums cs_j, CSo_j = sum_i dS_ij o_I, and the d gamma
+//                        sum_i dS_ij |gq_i - gk_j|^2 from fp32 points (CUDA
+//                        cores, inside the dS loop);
 //   (both passes run as one grid, ipa_bwd_kernel, so that the key-pass CTAs
 //   fill the SMs the query pass leaves idle in its last wave)
 //   ipa_bwd_map_kernel   per residue, all heads: the augmented gradients
@@ -76,7 +79,7 @@ struct BwdArgs {
   float* dva;            // [B*H, L, 64]
   float* dz2;            // [B*H, L, DZ]
   float4* csk;           // [B*H, L] (cs, CSo)
-  const float* pts;      // [B*H, L, 24]: tile-local query points gq' (12) | key points gk' (12), fp32
+  const float* pts;      // [B*H, L, 24]: query points gq - cen (12) | key points gk - cen (12), fp32
   float* gsum;           // [B*H, L]: sum_i dS_ij |gq_i - gk_j|^2 per key (the d gamma sum, one side only)
   int* err;
 };
@@ -113,9 +116,6 @@ struct RowsArgs {
   __half* qp;            // [B*H, L, DZ]
   float2* rowd;          // [B*H, L]
   View q_pts, k_pts;
-  const float4* oq;      // [B, nqt] 128-row query tile origins
-  const float4* ok;      // [B, nkt] 64-row key tile origins
-  int nqt, nkt;
   float* pts;            // [B*H, L, 24]
 };
 
@@ -192,18 +192,16 @@ __global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
     const float zq = a.z1_half ? __half2float(z1hr[c]) : z1r[c];
     qpr[c] = __float2half_rn(zq * wr[c]);
   }
-  // tile-local query and key points (the values the Q_h / K_h rows hold as
-  // hi + lo), for the key pass's d gamma sum: lane e < 12 query coordinate e,
-  // 12 <= lane < 24 key coordinate e - 12
+  // query and key points relative to the centroid (fp32), for the key
+  // pass's d gamma sum: lane e < 12 query coordinate e, 12 <= lane < 24 key
+  // coordinate e - 12
   if (lane < 24) {
     const bool isq = lane < 12;
     const int e = isq ? lane : lane - 12, pp = e / 3, xx = e % 3;
     const View& pv = isq ? a.q_pts : a.k_pts;
     const int64_t pb = b * pv.s[0] + i * pv.s[1] + h * pv.s[2] + pp * pv.s[3];
     const float x0 = ldf(pv, pb), x1 = ldf(pv, pb + pv.s[4]), x2 = ldf(pv, pb + 2 * pv.s[4]);
-    const float4 og = isq ? a.oq[b * a.nqt + i / QT] : a.ok[b * a.nkt + i / KT];
-    const float ogx = xx == 0 ? og.x : xx == 1 ? og.y : og.z;
-    const float v = fmaf(Rm[3 * xx], x0, fmaf(Rm[3 * xx + 1], x1, Rm[3 * xx + 2] * x2)) + tc[xx] - ogx;
+    const float v = fmaf(Rm[3 * xx], x0, fmaf(Rm[3 * xx + 1], x1, Rm[3 * xx + 2] * x2)) + tc[xx];
     a.pts[bhl * 24 + lane] = live ? v : 0.f;
   }
 #pragma unroll
@@ -736,9 +734,16 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
     const float4 ck = in_range ? a.colk[static_cast<int64_t>(bh) * L + key] : make_float4(0.f, 0.f, 0.f, -INFINITY);
     const int sub = r >> 6;                      // which 64-key origin tile
     const float4 okj = a.ok[b * a.nkt + (in_range ? key / 64 : 0)];
-    float gk[12];                                // this key's tile-local points
+    float2 kc[6];                                // this key's points relative to the centroid, in pairs
+    {
+      const float4* kp = reinterpret_cast<const float4*>(a.pts + (static_cast<int64_t>(bh) * L + (in_range ? key : 0)) * 24 + 12);
 #pragma unroll
-    for (int e = 0; e < 12; ++e) gk[e] = in_range ? a.pts[(static_cast<int64_t>(bh) * L + key) * 24 + 12 + e] : 0.f;
+      for (int u = 0; u < 3; ++u) {
+        const float4 w = in_range ? kp[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+        kc[2 * u] = make_float2(w.x, w.y);
+        kc[2 * u + 1] = make_float2(w.z, w.w);
+      }
+    }
     float cs = 0.f, co0 = 0.f, co1 = 0.f, co2 = 0.f, gsum = 0.f;
     bool ok = true;
     for (int i = 0; i < nq && ok; ++i) {
@@ -769,6 +774,22 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       const float4 oqv = oqs[s];
       const float colv = ck.w - fmaf(ck.x, okj.x - oqv.x, fmaf(ck.y, okj.y - oqv.y, ck.z * (okj.z - oqv.z)));
       const float4* qi = qinfo + s * 64 + 32 * half;
+      // this half's 32 query points relative to the centroid, 12 floats each
+      const float4* qc = reinterpret_cast<const float4*>(smem + lay.aux + KA_QPTS) + (s * 64 + 32 * half) * 3;
+      // |gq_i - gk_j|^2, two coordinates per packed instruction
+      auto dist2 = [&](const int k) {
+        const float4 g0 = qc[3 * k], g1 = qc[3 * k + 1], g2 = qc[3 * k + 2];
+        const float2 d0 = sub_f32x2(make_float2(g0.x, g0.y), kc[0]), d1 = sub_f32x2(make_float2(g0.z, g0.w), kc[1]);
+        const float2 d2 = sub_f32x2(make_float2(g1.x, g1.y), kc[2]), d3 = sub_f32x2(make_float2(g1.z, g1.w), kc[3]);
+        const float2 d4 = sub_f32x2(make_float2(g2.x, g2.y), kc[4]), d5 = sub_f32x2(make_float2(g2.z, g2.w), kc[5]);
+        float2 acc = mul_f32x2(d0, d0);
+        acc = fma_f32x2(d1, d1, acc);
+        acc = fma_f32x2(d2, d2, acc);
+        acc = fma_f32x2(d3, d3, acc);
+        acc = fma_f32x2(d4, d4, acc);
+        acc = fma_f32x2(d5, d5, acc);
+        return acc.x + acc.y;
+      };
       uint32_t pp[16], pd[16];
       float tsum = 0.f;
 #pragma unroll
@@ -778,40 +799,18 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         const float x1 = __uint_as_float(sv[2 * k + 1]) + colv + (sub ? e1.y : e1.x);
         const float p0 = ex2(x0), p1 = ex2(x1);
         pp[k] = pack_half2(p0, p1);
-        pd[k] = pack_half2(p0 * (__uint_as_float(dv[2 * k]) - e0.z) * kLn2,
-                           p1 * (__uint_as_float(dv[2 * k + 1]) - e1.z) * kLn2);
+        const float ds0 = p0 * (__uint_as_float(dv[2 * k]) - e0.z) * kLn2;
+        const float ds1 = p1 * (__uint_as_float(dv[2 * k + 1]) - e1.z) * kLn2;
+        pd[k] = pack_half2(ds0, ds1);
         tsum = add_half2_to_f32(pd[k], tsum);
+        // d gamma: sum_i dS_ij |gq_i - gk_j|^2 (dS before its fp16 rounding)
+        gsum = fmaf(ds0, dist2(2 * k), gsum);
+        gsum = fmaf(ds1, dist2(2 * k + 1), gsum);
       }
       cs += tsum;
       co0 = fmaf(tsum, oqv.x, co0);
       co1 = fmaf(tsum, oqv.y, co1);
       co2 = fmaf(tsum, oqv.z, co2);
-      {
-        // sum_i dS_ij |gq_i - gk_j|^2 over this half's 32 queries, with the
-        // fp16 dS the MMAs multiply: gq_i - gk_j = gq'_i - (gk'_j + o_J - o_I)
-        const float ex = okj.x - oqv.x, ey = okj.y - oqv.y, ez = okj.z - oqv.z;
-        float e[12];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          e[3 * p] = gk[3 * p] + ex;
-          e[3 * p + 1] = gk[3 * p + 1] + ey;
-          e[3 * p + 2] = gk[3 * p + 2] + ez;
-        }
-        const float4* qp4 = reinterpret_cast<const float4*>(smem + lay.aux + KA_QPTS) + (s * 64 + 32 * half) * 3;
-#pragma unroll 4
-        for (int k = 0; k < 32; ++k) {
-          const float4 g0 = qp4[3 * k], g1 = qp4[3 * k + 1], g2 = qp4[3 * k + 2];
-          const float q[12] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w, g2.x, g2.y, g2.z, g2.w};
-          float d2 = 0.f;
-#pragma unroll
-          for (int c = 0; c < 12; ++c) {
-            const float dd = q[c] - e[c];
-            d2 = fmaf(dd, dd, d2);
-          }
-          const float2 dsp = unpack_half2(pd[k >> 1]);
-          gsum = fmaf((k & 1) ? dsp.y : dsp.x, d2, gsum);
-        }
-      }
       tc_fence_after();
       tmem_st16(tmem + K_TM_S + 16 * half + lane_off, pp);
       tmem_st16(tmem + K_TM_DP + 16 * half + lane_off, pd);
@@ -872,6 +871,9 @@ struct BwdMaps {
   CUtensorMap k_kh, k_vh, k_z2, k_qh, k_do, k_qp, k_du;   // key pass
 };
 
+// One CTA of NTH = 320 threads per SM (shared memory).  Registers are
+// allocated to warps in groups of four, so the 10 warps count as 12 and the
+// bound is 65536 / (12 x 32) -> 168 per thread.
 __global__ void __launch_bounds__(NTH, 1)
     ipa_bwd_kernel(const __grid_constant__ BwdMaps m, const BwdArgs aq, const BwdArgs ak, const int nqb) {
   if (static_cast<int>(blockIdx.x) < nqb)
@@ -1149,9 +1151,6 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   ra.qp = reinterpret_cast<__half*>(ws + w.qp);
   ra.rowd = reinterpret_cast<float2*>(ws + w.rowd);
   ra.q_pts = f.q_pts; ra.k_pts = f.k_pts;
-  ra.oq = reinterpret_cast<const float4*>(ws + fw.oq);
-  ra.ok = reinterpret_cast<const float4*>(ws + fw.ok);
-  ra.nqt = f.nqt; ra.nkt = f.nkt;
   ra.pts = reinterpret_cast<float*>(ws + w.pts);
   const int64_t warps = static_cast<int64_t>(B) * L * H;
   ipa_bwd_rows_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(ra);

@@ -5,7 +5,7 @@
 //                        (R, t, valid), partial sums of the valid origins, and
 //                        the pair factors z2 (fp16) and z1 (fp32 and fp16)
 //                        padded to DZ.
-//   ipa_rows_kernel   -- three threads per (b, i, h) (Q, K, V rows), heads fastest: the
+//   ipa_rows_kernel   -- one thread per (b, i, h), heads fastest: the
 //                        centroid of the valid origins (each block reduces
 //                        the tile partial sums of its batches), query-tile
 //                        (128) and key-tile (64) origins relative to it, the
@@ -238,30 +238,25 @@ __device__ __forceinline__ float4 tile_origin(const float4* part, int J0, int J1
   return make_float4(s.x * inv - cen.x, s.y * inv - cen.y, s.z * inv - cen.z, 0.f);
 }
 
-constexpr int ROWS_THREADS = 3 * 128;   // three threads per (residue, head): Q_h, K_h, V_h rows
-
 template <int C, int PQ, int PV>
-__global__ void __launch_bounds__(ROWS_THREADS, 2) ipa_rows_kernel(const RowArgs a) {
+__global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   static_assert(C + 9 * PQ + 2 <= DH && C + 6 * PV <= DH, "augmented rows wider than 64");
   // a block owns rb consecutive residues of one batch, all heads (heads
   // fastest: the threads of a residue read its contiguous [H, ...] input
-  // rows together), three threads per (residue, head) -- kind 0 builds the
-  // Q_h row and the row term, kind 1 the K_h row and the column term, kind 2
-  // the V_h row; the rows are staged in shared memory and written as one
-  // contiguous run of rb rows per head plane
+  // rows together); its output rows are staged in shared memory and written
+  // as one contiguous run of rb rows per head plane
   extern __shared__ uint4 stage_rows[];    // [3][H][rb][8] fp16 rows, then [2][H][rb] float4 terms
   const int rb = a.rb, H = a.H;
   const int b = blockIdx.y;
   const int i0 = blockIdx.x * rb;
-  const int kind = threadIdx.x / 128, local = threadIdx.x % 128;
-  const int il = local / H, h = local % H;
+  const int il = threadIdx.x / H, h = threadIdx.x % H;
   const int i = i0 + il;
   const bool active = il < rb && i < a.L;
   const int nrow = a.L - i0 < rb ? a.L - i0 : rb;
 
   // centroid of the batch's valid origins (double sums over the per-tile
   // partial sums of the tile kernel)
-  __shared__ double red[ROWS_THREADS / 32][4];
+  __shared__ double red[4][4];
   __shared__ float4 cen_s;
   {
     double sx = 0, sy = 0, sz = 0, sn = 0;
@@ -283,7 +278,7 @@ __global__ void __launch_bounds__(ROWS_THREADS, 2) ipa_rows_kernel(const RowArgs
     __syncthreads();
     if (threadIdx.x == 0) {
       double tx = 0, ty = 0, tz = 0, tn = 0;
-      for (int w = 0; w < ROWS_THREADS / 32; ++w) { tx += red[w][0]; ty += red[w][1]; tz += red[w][2]; tn += red[w][3]; }
+      for (int w = 0; w < 4; ++w) { tx += red[w][0]; ty += red[w][1]; tz += red[w][2]; tn += red[w][3]; }
       const double inv = tn > 0 ? 1.0 / tn : 0.0;
       cen_s = make_float4(static_cast<float>(tx * inv), static_cast<float>(ty * inv), static_cast<float>(tz * inv),
                           static_cast<float>(tn));
@@ -291,144 +286,144 @@ __global__ void __launch_bounds__(ROWS_THREADS, 2) ipa_rows_kernel(const RowArgs
     __syncthreads();
   }
   const int slot = h * rb + il;                                   // row of this thread in a staged plane
-  uint4* srow = stage_rows + static_cast<size_t>(kind * H * rb + slot) * 8;
+  uint4* sq_rows = stage_rows + static_cast<size_t>(0 * H * rb + slot) * 8;
+  uint4* sk_rows = stage_rows + static_cast<size_t>(1 * H * rb + slot) * 8;
+  uint4* sv_rows = stage_rows + static_cast<size_t>(2 * H * rb + slot) * 8;
   float4* sterm = reinterpret_cast<float4*>(stage_rows + static_cast<size_t>(3 * H * rb) * 8);
   // the [H, DZ] pair-bias weights, one entry per thread of batch 0
-  if (b == 0 && active && kind == 0)
+  if (b == 0 && active)
     for (int64_t e = static_cast<int64_t>(i) * H + h; e < static_cast<int64_t>(H) * a.DZ;
          e += static_cast<int64_t>(H) * a.L) {
       const int he = static_cast<int>(e / a.DZ), col = static_cast<int>(e % a.DZ);
       a.wqp[e] = col < a.RCz ? kLog2e * a.w_L * ldf(a.w_bias, (col % a.Cz) * a.w_bias.s[0] + he * a.w_bias.s[1]) : 0.f;
     }
   if (active) {
-    const float4 cn = cen_s;
-    const float4* partb = a.part + static_cast<int64_t>(b) * a.nkt;
-    const float c = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
-    if (kind == 0 && h == 0) {
-      // the values the core kernel reads per batch / tile / head, one writer each
-      if (i == 0) a.cen[b] = cn;
-      if (i % QT == 0) {
-        const int Jq = (i / QT) * (QT / KT);
-        a.oq[b * a.nqt + i / QT] = tile_origin(partb, Jq, Jq + QT / KT < a.nkt ? Jq + QT / KT : a.nkt, cn);
-      }
-      if (i % KT == 0) a.ok[b * a.nkt + i / KT] = tile_origin(partb, i / KT, i / KT + 1, cn);
-    }
-    if (kind == 0 && b == 0 && i == 0) a.headc[h] = c;
+  const float4 cn = cen_s;
+  const float4* partb = a.part + static_cast<int64_t>(b) * a.nkt;
+  const int Jq = (i / QT) * (QT / KT);
+  const float4 oqv = tile_origin(partb, Jq, Jq + QT / KT < a.nkt ? Jq + QT / KT : a.nkt, cn);
+  const float4 okv = tile_origin(partb, i / KT, i / KT + 1, cn);
+  // the values the core kernel reads per batch / tile / head, one writer each
+  if (h == 0) {
+    if (i == 0) a.cen[b] = cn;
+    if (i % QT == 0) a.oq[b * a.nqt + i / QT] = oqv;
+    if (i % KT == 0) a.ok[b * a.nkt + i / KT] = okv;
+  }
+  if (b == 0 && i == 0) a.headc[h] = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
+  const float c = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
 
-    const float4* fr = a.frame + (static_cast<int64_t>(b) * a.L + i) * 4;
-    const float4 f0 = fr[0], f1 = fr[1], f2 = fr[2], f3 = fr[3];
-    const float Rm[9] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w, f2.x};
-    const float tc[3] = {f2.y - cn.x, f2.z - cn.y, f2.w - cn.z};
-    const bool valid = f3.x != 0.f;
-    auto load_pts = [&](const View& v, auto& dst) {
-      const int64_t base = b * v.s[0] + i * v.s[1] + h * v.s[2];
-      if (v.s[4] == 1 && v.s[3] == 3) {
-        load_row(v, base, 1, dst);             // [points, xyz] dense
-      } else {
-        constexpr int NP = sizeof(dst) / sizeof(float) / 3;
-#pragma unroll
-        for (int p = 0; p < NP; ++p)
-#pragma unroll
-          for (int y = 0; y < 3; ++y) dst[3 * p + y] = ldf(v, base + p * v.s[3] + y * v.s[4]);
-      }
-    };
-    auto hi_of = [](float x) { return __half2float(__float2half_rn(x)); };
-    float vmax = 0.f;   // largest |value| written (NaN if any value is NaN)
-    auto store_row = [&](auto value_of) {
-#pragma unroll
-      for (int u = 0; u < DH / 8; ++u) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = value_of(8 * u + 2 * e), x1 = value_of(8 * u + 2 * e + 1);
-          vmax = fmax_nan(vmax, fmax_nan(fabsf(x0), fabsf(x1)));
-          w[e] = valid ? pack_half2(x0, x1) : 0u;
-        }
-        srow[u] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    };
-    if (kind < 2) {
-      // query (kind 0) or key (kind 1) row: points relative to the tile origin
-      const View& sv = kind == 0 ? a.q : a.k;
-      const View& pv = kind == 0 ? a.q_pts : a.k_pts;
-      float4 og;
-      if (kind == 0) {
-        const int Jq = (i / QT) * (QT / KT);
-        og = tile_origin(partb, Jq, Jq + QT / KT < a.nkt ? Jq + QT / KT : a.nkt, cn);
-      } else {
-        og = tile_origin(partb, i / KT, i / KT + 1, cn);
-      }
-      float xs[C], pts[PQ * 3], g[PQ * 3];
-      load_row(sv, b * sv.s[0] + i * sv.s[1] + h * sv.s[2], sv.s[3], xs);
-      load_pts(pv, pts);
-      const float oa[3] = {og.x, og.y, og.z};
-#pragma unroll
-      for (int p = 0; p < PQ; ++p)
-#pragma unroll
-        for (int x = 0; x < 3; ++x)
-          g[3 * p + x] = fmaf(Rm[3 * x], pts[3 * p], fmaf(Rm[3 * x + 1], pts[3 * p + 1], Rm[3 * x + 2] * pts[3 * p + 2])) +
-                         tc[x] - oa[x];
-      float sg[3] = {0.f, 0.f, 0.f}, ng = 0.f;
-#pragma unroll
-      for (int e = 0; e < 3 * PQ; ++e) {
-        sg[e % 3] += g[e];
-        ng = fmaf(g[e], g[e], ng);
-      }
-      if (kind == 0) {
-        // Q_h: [ scaled q | gq' hi | gq' hi | gq' lo | -1 -1 | 0 ]
-        store_row([&](int col) -> float {
-          if (col < C) return a.qscale * xs[col];
-          if (col < C + 9 * PQ) {
-            const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
-            const float hi = hi_of(g[e]);
-            return part < 2 ? hi : g[e] - hi;
-          }
-          return col < C + 9 * PQ + 2 ? -1.f : 0.f;
-        });
-        // .w: the row constant c sum_p |gq'_p|^2 that the fused pass leaves out
-        // of its logits (it cancels in the softmax); a training forward adds it
-        // back to report the log-sum-exp of the true logits
-        sterm[slot] = valid ? make_float4(sg[0], sg[1], sg[2], c * ng) : make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        // K_h: [ k | 2c gk' hi | lo | hi | c|gk'|^2 hi, lo | 0 ]
-        store_row([&](int col) -> float {
-          if (col < C) return xs[col];
-          if (col < C + 9 * PQ) {
-            const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
-            const float gg = 2.f * c * g[e], hi = hi_of(gg);
-            return part == 1 ? gg - hi : hi;
-          }
-          if (col < C + 9 * PQ + 2) {
-            const float n = c * ng, hi = hi_of(n);
-            return col == C + 9 * PQ ? hi : n - hi;
-          }
-          return 0.f;
-        });
-        sterm[H * rb + slot] = valid ? make_float4(2.f * c * sg[0], 2.f * c * sg[1], 2.f * c * sg[2], 0.f)
-                                     : make_float4(0.f, 0.f, 0.f, -INFINITY);
-      }
+  const float4* fr = a.frame + (static_cast<int64_t>(b) * a.L + i) * 4;
+  const float4 f0 = fr[0], f1 = fr[1], f2 = fr[2], f3 = fr[3];
+  const float Rm[9] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w, f2.x};
+  const float tc[3] = {f2.y - cn.x, f2.z - cn.y, f2.w - cn.z};
+  const bool valid = f3.x != 0.f;
+  const float oqa[3] = {oqv.x, oqv.y, oqv.z}, oka[3] = {okv.x, okv.y, okv.z};
+
+  float qs[C], ks[C], vs[C], qp[PQ * 3], kp[PQ * 3], vp[PV * 3];
+  load_row(a.q, b * a.q.s[0] + i * a.q.s[1] + h * a.q.s[2], a.q.s[3], qs);
+  load_row(a.k, b * a.k.s[0] + i * a.k.s[1] + h * a.k.s[2], a.k.s[3], ks);
+  load_row(a.v, b * a.v.s[0] + i * a.v.s[1] + h * a.v.s[2], a.v.s[3], vs);
+  auto load_pts = [&](const View& v, auto& dst) {
+    const int64_t base = b * v.s[0] + i * v.s[1] + h * v.s[2];
+    if (v.s[4] == 1 && v.s[3] == 3) {
+      load_row(v, base, 1, dst);             // [points, xyz] dense
     } else {
-      // V_h: [ v | gv hi | gv lo ], value points relative to the centroid
-      float vs[C], vp[PV * 3], gv[PV * 3];
-      load_row(a.v, b * a.v.s[0] + i * a.v.s[1] + h * a.v.s[2], a.v.s[3], vs);
-      load_pts(a.v_pts, vp);
+      constexpr int NP = sizeof(dst) / sizeof(float) / 3;
 #pragma unroll
-      for (int p = 0; p < PV; ++p)
+      for (int p = 0; p < NP; ++p)
 #pragma unroll
-        for (int x = 0; x < 3; ++x)
-          gv[3 * p + x] = fmaf(Rm[3 * x], vp[3 * p], fmaf(Rm[3 * x + 1], vp[3 * p + 1], Rm[3 * x + 2] * vp[3 * p + 2])) + tc[x];
-      store_row([&](int col) -> float {
-        if (col < C) return vs[col];
-        if (col < C + 6 * PV) {
-          const int u = col - C, part = u / (3 * PV), e = u % (3 * PV);
-          const float hi = hi_of(gv[e]);
-          return part == 0 ? hi : gv[e] - hi;
-        }
-        return 0.f;
-      });
+        for (int y = 0; y < 3; ++y) dst[3 * p + y] = ldf(v, base + p * v.s[3] + y * v.s[4]);
     }
-    // |x| >= 65520 (or NaN) does not survive the fp16 rounding
-    if (valid && !(vmax < 65520.f)) record_error(a.err, DEV_NONFINITE);
+  };
+  load_pts(a.q_pts, qp);
+  load_pts(a.k_pts, kp);
+  load_pts(a.v_pts, vp);
+
+  // frames applied: gq' = R q + t' - o_I, gk' = R k + t' - o_J, gv = R v + t'
+  float gq[PQ * 3], gk[PQ * 3], gv[PV * 3];
+#pragma unroll
+  for (int p = 0; p < PQ; ++p)
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      gq[3 * p + x] = fmaf(Rm[3 * x], qp[3 * p], fmaf(Rm[3 * x + 1], qp[3 * p + 1], Rm[3 * x + 2] * qp[3 * p + 2])) + tc[x] - oqa[x];
+      gk[3 * p + x] = fmaf(Rm[3 * x], kp[3 * p], fmaf(Rm[3 * x + 1], kp[3 * p + 1], Rm[3 * x + 2] * kp[3 * p + 2])) + tc[x] - oka[x];
+    }
+#pragma unroll
+  for (int p = 0; p < PV; ++p)
+#pragma unroll
+    for (int x = 0; x < 3; ++x)
+      gv[3 * p + x] = fmaf(Rm[3 * x], vp[3 * p], fmaf(Rm[3 * x + 1], vp[3 * p + 1], Rm[3 * x + 2] * vp[3 * p + 2])) + tc[x];
+
+  // rows are built and stored one after the other to keep few values live
+  float sq[3] = {0.f, 0.f, 0.f}, sk[3] = {0.f, 0.f, 0.f}, nk = 0.f, nq = 0.f;
+#pragma unroll
+  for (int e = 0; e < 3 * PQ; ++e) {
+    sq[e % 3] += gq[e];
+    sk[e % 3] += gk[e];
+    nk = fmaf(gk[e], gk[e], nk);
+    nq = fmaf(gq[e], gq[e], nq);
+  }
+  float vmax = 0.f;   // largest |value| written (NaN if any value is NaN)
+  auto store_row = [&](uint4* dst, auto value_of) {
+#pragma unroll
+    for (int u = 0; u < DH / 8; ++u) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = value_of(8 * u + 2 * e), x1 = value_of(8 * u + 2 * e + 1);
+        vmax = fmax_nan(vmax, fmax_nan(fabsf(x0), fabsf(x1)));
+        w[e] = valid ? pack_half2(x0, x1) : 0u;
+      }
+      dst[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  };
+  auto hi_of = [](float x) { return __half2float(__float2half_rn(x)); };
+  // Q_h: [ scaled q | gq' hi | gq' hi | gq' lo | -1 -1 | 0 ]
+  store_row(sq_rows, [&](int col) -> float {
+    if (col < C) return a.qscale * qs[col];
+    if (col < C + 9 * PQ) {
+      const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
+      const float hi = hi_of(gq[e]);
+      return part < 2 ? hi : gq[e] - hi;
+    }
+    return col < C + 9 * PQ + 2 ? -1.f : 0.f;
+  });
+  // K_h: [ k | 2c gk' hi | lo | hi | c|gk'|^2 hi, lo | 0 ]
+  store_row(sk_rows, [&](int col) -> float {
+    if (col < C) return ks[col];
+    if (col < C + 9 * PQ) {
+      const int u = col - C, part = u / (3 * PQ), e = u % (3 * PQ);
+      const float g = 2.f * c * gk[e], hi = hi_of(g);
+      return part == 1 ? g - hi : hi;
+    }
+    if (col < C + 9 * PQ + 2) {
+      const float n = c * nk, hi = hi_of(n);
+      return col == C + 9 * PQ ? hi : n - hi;
+    }
+    return 0.f;
+  });
+  // V_h: [ v | gv hi | gv lo ]
+  store_row(sv_rows, [&](int col) -> float {
+    if (col < C) return vs[col];
+    if (col < C + 6 * PV) {
+      const int u = col - C, part = u / (3 * PV), e = u % (3 * PV);
+      const float hi = hi_of(gv[e]);
+      return part == 0 ? hi : gv[e] - hi;
+    }
+    return 0.f;
+  });
+  if (!valid) {
+    sq[0] = sq[1] = sq[2] = 0.f;
+    sk[0] = sk[1] = sk[2] = 0.f;
+    nq = 0.f;
+  }
+  // .w: the row constant c sum_p |gq'_p|^2 that the fused pass leaves out of
+  // its logits (it cancels in the softmax); a training forward adds it back
+  // to report the log-sum-exp of the true logits
+  sterm[slot] = make_float4(sq[0], sq[1], sq[2], c * nq);
+  sterm[H * rb + slot] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
+  // |x| >= 65520 (or NaN) does not survive the fp16 rounding
+  if (valid && !(vmax < 65520.f)) record_error(a.err, DEV_NONFINITE);
   }
   __syncthreads();
   // each head plane's run of nrow rows, 16-byte stores, consecutive threads on
@@ -436,11 +431,11 @@ __global__ void __launch_bounds__(ROWS_THREADS, 2) ipa_rows_kernel(const RowArgs
   uint4* const outs[3] = {a.qh, a.kh, a.vh};
   const int run = nrow * 8;                                        // uint4 per plane run
 #pragma unroll
-  for (int kd = 0; kd < 3; ++kd) {
-    const uint4* src = stage_rows + static_cast<size_t>(kd * H * rb) * 8;
+  for (int kind = 0; kind < 3; ++kind) {
+    const uint4* src = stage_rows + static_cast<size_t>(kind * H * rb) * 8;
     for (int e = threadIdx.x; e < H * run; e += blockDim.x) {
       const int hh = e / run, r = e % run;
-      outs[kd][(static_cast<int64_t>(b * H + hh) * a.L + i0) * 8 + r] = src[hh * rb * 8 + r];
+      outs[kind][(static_cast<int64_t>(b * H + hh) * a.L + i0) * 8 + r] = src[hh * rb * 8 + r];
     }
   }
   for (int e = threadIdx.x; e < 2 * H * nrow; e += blockDim.x) {
@@ -493,7 +488,7 @@ cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * (3 * DH * 2 + 2 * 16));
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>((a.L + r.rb - 1) / r.rb), static_cast<unsigned>(a.B));
-  ipa_rows_kernel<IPA_C, IPA_PQ, IPA_PV><<<grid, ROWS_THREADS, smem, stream>>>(r);
+  ipa_rows_kernel<IPA_C, IPA_PQ, IPA_PV><<<grid, 128, smem, stream>>>(r);
   return cudaGetLastError();
 }
 
