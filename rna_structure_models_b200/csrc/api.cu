@@ -131,6 +131,32 @@ bool encode_tmap_f16_panels(CUtensorMap* map, const void* base, uint64_t DZ, uin
   return r == CUDA_SUCCESS;
 }
 
+// fp32 tensor of rank 3 or 4 (dims innermost first, byte strides of dims 1..)
+// read or written in boxes whose inner extent is 32 elements (128 bytes) with
+// the 128-byte swizzle; out-of-range elements of a load are filled with zeros
+// and those of a store are dropped.
+bool encode_tmap_f32_sw128(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                           const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr || rank < 3 || rank > 4 || box[0] != 32) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
+  cuuint64_t d[4];
+  cuuint64_t st[3];
+  cuuint32_t bx[4], estr[4] = {1, 1, 1, 1};
+  for (int k = 0; k < rank; ++k) {
+    d[k] = dims[k];
+    bx[k] = box[k];
+    if (k + 1 < rank) {
+      st[k] = strides_bytes[k];
+      if (st[k] % 16 != 0) return false;
+    }
+  }
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+                        d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fipa
 
 using namespace fipa;

@@ -366,10 +366,13 @@ struct MapArgs {
 // consecutive keys at a time, loads their terms once and writes the 16 rows'
 // probabilities for them as float4 stores (a warp writes 512 contiguous bytes
 // of a row).  Key terms are read N / 16 times per (b, h) instead of N times.
+// The pair-mask words of all 16 rows are loaded before any score, so their
+// latency is paid once per four keys, and the scores are taken two keys per
+// packed instruction (each lane rounds as geo_pair does).
 constexpr int MAP_ROWS = 16;
 constexpr int MAP_KEYS = 4;
 
-__global__ void __launch_bounds__(256) geo_map_kernel(const MapArgs a) {
+__global__ void __launch_bounds__(256, 3) geo_map_kernel(const MapArgs a) {
   const int i0 = blockIdx.x * MAP_ROWS, h = blockIdx.y, b = blockIdx.z;
   const int N = a.N;
   const int64_t bh = static_cast<int64_t>(b) * a.H + h;
@@ -391,6 +394,7 @@ __global__ void __launch_bounds__(256) geo_map_kernel(const MapArgs a) {
   }
   __syncthreads();
   const float2 sc = a.sc[h];
+  const float2 A2 = make_float2(sc.x, sc.x), nB2 = make_float2(-sc.y, -sc.y);
   const int nrows = N - i0 < MAP_ROWS ? N - i0 : MAP_ROWS;
   const bool vec_store = (N & 3) == 0;
   const unsigned char* pmb = a.pm ? a.pm + b * a.pms[0] + h * a.pms[1] : nullptr;
@@ -405,28 +409,71 @@ __global__ void __launch_bounds__(256) geo_map_kernel(const MapArgs a) {
       k1[t] = a.kg[2 * (bh * N + j) + 1];
     }
     const bool full = j0 + MAP_KEYS <= N;
-    for (int rr = 0; rr < nrows; ++rr) {
+    // the four keys' mask bytes of every row, loaded together, kept as 4
+    // bits per row (bit 4 rr + t: key j0 + t allowed for row i0 + rr)
+    uint32_t wv[MAP_ROWS];
+#pragma unroll
+    for (int rr = 0; rr < MAP_ROWS; ++rr) {
+      wv[rr] = 0x01010101u;
+      if (pmb != nullptr && rr < nrows) {
+        const unsigned char* pr = pmb + static_cast<int64_t>(i0 + rr) * a.pms[2];
+        if (vec_mask && full) {
+          wv[rr] = *reinterpret_cast<const uint32_t*>(pr + j0);
+        } else {
+          uint32_t w = 0u;
+#pragma unroll
+          for (int t = 0; t < MAP_KEYS; ++t)
+            if (j0 + t < N && pr[static_cast<int64_t>(j0 + t) * a.pms[3]]) w |= 1u << (8 * t);
+          wv[rr] = w;
+        }
+      }
+    }
+    uint64_t allow = 0u;
+#pragma unroll
+    for (int rr = 0; rr < MAP_ROWS; ++rr) {
+      // one bit per nonzero byte: x = sum_t [byte t != 0] 2^(8 t); x * 0x01020408
+      // gathers bit t of the nibble at bits 24 + t (no carries between terms)
+      const uint32_t x = __vcmpne4(wv[rr], 0u) & 0x01010101u;
+      allow |= static_cast<uint64_t>(((x * 0x01020408u) >> 24) & 0xfu) << (4 * rr);
+    }
+    // key terms in lane pairs: keys (0, 1) and (2, 3)
+    float2 kx[2], ky[2], kz[2], px[2], py[2], pz[2], kb[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float4 a0 = k0[2 * u], a1 = k0[2 * u + 1], c0 = k1[2 * u], c1 = k1[2 * u + 1];
+      kx[u] = make_float2(a0.x, a1.x);
+      ky[u] = make_float2(a0.y, a1.y);
+      kz[u] = make_float2(a0.z, a1.z);
+      kb[u] = make_float2(a0.w, a1.w);
+      px[u] = make_float2(c0.x, c1.x);
+      py[u] = make_float2(c0.y, c1.y);
+      pz[u] = make_float2(c0.z, c1.z);
+    }
+#pragma unroll
+    for (int rr = 0; rr < MAP_ROWS; ++rr) {
+      if (rr >= nrows) break;
       const int i = i0 + rr;
       const float4 q0 = qs[rr][0], q1 = qs[rr][1];
       const float2 st = rs[rr];
-      uint32_t allow = 0xffffffffu;
-      if (pmb) {
-        const unsigned char* pr = pmb + static_cast<int64_t>(i) * a.pms[2];
-        if (vec_mask && full) {
-          allow = *reinterpret_cast<const uint32_t*>(pr + j0);
-        } else {
-          allow = 0u;
-#pragma unroll
-          for (int t = 0; t < MAP_KEYS; ++t)
-            if (j0 + t < N && pr[static_cast<int64_t>(j0 + t) * a.pms[3]]) allow |= 0xffu << (8 * t);
-        }
-      }
+      const uint32_t al = static_cast<uint32_t>(allow >> (4 * rr));
       float v[MAP_KEYS];
 #pragma unroll
-      for (int t = 0; t < MAP_KEYS; ++t) {
-        const float s = geo_score(q0, q1, k0[t], k1[t], sc.x, sc.y);
-        const bool ok = st.y > 0.f && ((allow >> (8 * t)) & 0xffu) != 0;
-        v[t] = ok ? ex2(s - st.x) * st.y : 0.f;
+      for (int u = 0; u < 2; ++u) {
+        // the operation sequence of geo_pair, two keys per instruction
+        const float2 dot = fma_f32x2(make_float2(q0.x, q0.x), kx[u],
+                                     fma_f32x2(make_float2(q0.y, q0.y), ky[u],
+                                               mul_f32x2(make_float2(q0.z, q0.z), kz[u])));
+        const float2 dx = sub_f32x2(make_float2(q1.x, q1.x), px[u]);
+        const float2 dy = sub_f32x2(make_float2(q1.y, q1.y), py[u]);
+        const float2 dz = sub_f32x2(make_float2(q1.z, q1.z), pz[u]);
+        const float2 d2 = fma_f32x2(dx, dx, fma_f32x2(dy, dy, mul_f32x2(dz, dz)));
+        const float2 dist = make_float2(sqrt_approx(d2.x), sqrt_approx(d2.y));
+        const float2 s = add_f32x2(add_f32x2(fma_f32x2(A2, dot, mul_f32x2(nB2, dist)), make_float2(q0.w, q0.w)), kb[u]);
+        const float2 y = sub_f32x2(s, make_float2(st.x, st.x));
+        const bool ok0 = st.y > 0.f && ((al >> (2 * u)) & 1u) != 0;
+        const bool ok1 = st.y > 0.f && ((al >> (2 * u + 1)) & 1u) != 0;
+        v[2 * u] = ok0 ? ex2(y.x) * st.y : 0.f;
+        v[2 * u + 1] = ok1 ? ex2(y.y) * st.y : 0.f;
       }
       float* dst = a.att + (bh * N + i) * static_cast<int64_t>(N) + j0;
       if (vec_store && full) {

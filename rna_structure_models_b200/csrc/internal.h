@@ -178,6 +178,8 @@ bool encode_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_
                         uint32_t box0, uint32_t box1, int swizzle_bytes = 128);
 bool encode_tmap_f16_panels(CUtensorMap* map, const void* base, uint64_t DZ, uint64_t L, uint64_t B,
                             uint32_t box_rows, uint32_t box_panels);
+bool encode_tmap_f32_sw128(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                           const uint64_t* strides_bytes, const uint32_t* box);
 
 // CTA-pair core kernel (cta_group::2): pair-dimension widths it supports and its launch.
 bool ipa_pair_supported(int DZ);

@@ -82,6 +82,7 @@ struct PairArgs {
   float* lse;           // training forward: [B, H, L] log-sum-exp (natural log), else null
   float* uagg;          // training forward: [B, L, H, R Cz] pair aggregate, else null
   int* err;
+  int tma_epi;          // 1: the output pass stages the pair features and stores them with TMA
   int trace_cta0, trace_cta1;
 };
 
@@ -112,7 +113,7 @@ enum {
   // local barriers (waited on in each CTA)
   P_QFULL = 0, P_SFULL, P_PFREE, P_KEMPTY0, P_COLFULL0 = P_KEMPTY0 + 2, P_DRAIN = P_COLFULL0 + NCOL,
   // barriers waited on by the MMA thread (used in CTA 0)
-  P_KFULL0, P_VFULL = P_KFULL0 + 2, P_SFREE, P_PFULL, P_QREADY, P_COUNT
+  P_KFULL0, P_VFULL = P_KFULL0 + 2, P_SFREE, P_PFULL, P_QREADY, P_ZFULL, P_COUNT
 };
 constexpr uint32_t AX_TMEM = AX_BAR + 8 * P_COUNT;
 constexpr uint32_t AX_ABORT = AX_TMEM + 8;
@@ -129,7 +130,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
                               const __grid_constant__ CUtensorMap tm_z2k,
                               const __grid_constant__ CUtensorMap tm_z2v,
                               const __grid_constant__ CUtensorMap tm_vh,
-                              const __grid_constant__ CUtensorMap tm_z1, const PairArgs a) {
+                              const __grid_constant__ CUtensorMap tm_z1,
+                              const __grid_constant__ CUtensorMap tm_z1f,
+                              const __grid_constant__ CUtensorMap tm_out, const PairArgs a) {
   extern __shared__ unsigned char smem_raw[];
 #ifdef IPA_TRACE
   if (threadIdx.x == 0 && blockIdx.x < 4096) {
@@ -179,6 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     mbar_init(bar(P_SFREE), 16);
     mbar_init(bar(P_PFULL), 16);
     mbar_init(bar(P_QREADY), 2);
+    mbar_init(bar(P_ZFULL), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -281,6 +285,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       if (!wait_local(P_KEMPTY0 + (j & 1), ((j - 2) >> 1) & 1, DEV_TIMEOUT_EMPTY)) break;
       if (lane == 0) PAIR_TR(j, 12);
       load_k(j);
+    }
+    // the epilogue's z1 rows (fp32, contiguous), brought into L2 while the
+    // last tiles run
+    if (lane == 0 && row0 < L) {
+      const int nrows = L - row0 < 128 ? L - row0 : 128;
+      bulk_prefetch_l2(a.z1f + (static_cast<int64_t>(b) * L + row0) * DZ, static_cast<uint32_t>(nrows * DZ * 4));
+    }
+    // staged output pass: the z1 rows into the Q_pair / K area (DZ / 32 boxes
+    // of 16 KB from SP_QP) once the last Q.K has completed and released both
+    if (a.tma_epi && !*abort_flag && wait_local(P_KEMPTY0 + ((nt - 1) & 1), ((nt - 1) >> 1) & 1, DEV_TIMEOUT_EMPTY) &&
+        lane == 0) {
+      mbar_arrive_expect_tx(bar(P_ZFULL), static_cast<uint32_t>(DZ / 32) * 16384u);
+      for (int k = 0; k < DZ / 32; ++k) tma_load_3d(sb + SP_QP + 16384u * k, &tm_z1f, bar(P_ZFULL), 32 * k, row0, b);
     }
   } else if (warp == W_VPROD) {
 #ifdef IPA_TRACE
@@ -547,6 +564,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     const bool all_ok = __all_sync(0xffffffffu, ok);
     xch[512 + half * 128 + r] = l;
     named_bar_sync(pair_bar, 64);
+    if (tid == 0) PAIR_SPAN(20);
     const float lt = l + xch[512 + (1 - half) * 128 + r];
     const bool dead = !(in_range && f3.x != 0.f && lt > 0.f);
     // training forward: log-sum-exp of the true logits; the pass left the row
@@ -555,15 +573,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       a.lse[static_cast<int64_t>(bh) * L + row] = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
     // direct output pass when the pair block has no padding and whole
     // 64-column factors (the staged pass below handles every other shape)
-    if (a.RCz == DZ && (a.Cz & 63) == 0) {
+    if (a.tma_epi) {
+      // staged pair features (z1 from the boxes the producer loaded, the
+      // output through staging boxes and a TMA store), scalars and points direct
+      const bool zok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(P_ZFULL), 0, abort_flag));
+      if (!zok && lane == 0) fail(DEV_TIMEOUT_FULL);
+      const int nz = DZ / 32;
+      if (all_ok && zok && !*abort_flag) {
+        tc_fence_after();
+        const float inv = dead ? 0.f : 1.f / lt;
+        const int rrow = in_range ? row : 0;
+        const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
+        auto z1box = [&](int k) -> const unsigned char* { return smem + SP_QP + 16384u * k; };
+        auto obox = [&](int k) -> unsigned char* {
+          return smem + (k == 0 ? SP_QH : SP_QP + 16384u * (nz + k - 1));
+        };
+        stage_row_pair(tmem + lane_off, half, a.Cz, a.RCz / a.Cz, inv, r,
+                       a.uagg != nullptr ? a.uagg + orow * a.RCz : nullptr, in_range, z1box, obox);
+        if (tid == 0) PAIR_SPAN(22);
+        if (half == 0)
+          write_row_points<IPA_C, IPA_PV>(tmem + DZ + lane_off, inv, dead, in_range, a.out + orow * a.F, g0, g1, g2, cn);
+        fence_proxy_async_smem();   // the staging writes, before the TMA store reads them
+      }
+      named_bar_sync(1, NSOFT);
+      if (tid == 0 && all_ok && zok && !*abort_flag) {
+        for (int k = 0; k < a.Cz / 32; ++k)
+          tma_store_4d(&tm_out, sb + (k == 0 ? SP_QH : SP_QP + 16384u * (nz + k - 1)), IPA_C + 4 * IPA_PV + 32 * k, h,
+                       row0, b);
+        bulk_commit_group();
+        bulk_wait_read_all();   // the staging boxes must outlive the reads, not the writes
+      }
+      if (tid == 0) PAIR_SPAN(21);
+    } else if (a.RCz == DZ && (a.Cz & 63) == 0) {
       if (all_ok && !*abort_flag) {
         tc_fence_after();
         const float inv = dead ? 0.f : 1.f / lt;
         const int rrow = in_range ? row : 0;
         const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
+        unsigned long long* etr = nullptr;
+#ifdef IPA_TRACE
+        if (tid == 0 && blockIdx.x < 4096) etr = &g_pair_span[blockIdx.x][22];
+#endif
         write_row_direct<IPA_C, IPA_PV>(tmem + lane_off, half, DZ, a.Cz, a.RCz / a.Cz, inv, dead, in_range,
                                         a.z1f + (static_cast<int64_t>(b) * L + rrow) * DZ, a.out + orow * a.F,
-                                        a.uagg != nullptr ? a.uagg + orow * a.RCz : nullptr, g0, g1, g2, cn);
+                                        a.uagg != nullptr ? a.uagg + orow * a.RCz : nullptr, g0, g1, g2, cn, etr);
+        if (tid == 0) PAIR_SPAN(21);
       }
     } else {
     const int pitch = stage_pitch(DZ);
@@ -651,10 +705,28 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
   t.frame = reinterpret_cast<const float4*>(ws + w.frame);
   t.z1f = reinterpret_cast<const float*>(ws + w.z1f);
   t.out = a.out; t.err = a.err; t.lse = a.lse; t.uagg = a.uagg;
+  // staged output pass: whole 32-column factors, the pair block unpadded, and
+  // the z1 boxes plus the staging boxes inside the freed operand area
+  CUtensorMap tz1f = tz1, tout = tz1;
+  t.tma_epi = 0;
+  if (a.RCz == a.DZ && a.Cz % 32 == 0 &&
+      SP_QP + 16384u * static_cast<uint32_t>(a.DZ / 32 + a.Cz / 32 - 1) <= SP_AUX) {
+    const uint64_t zd[3] = {static_cast<uint64_t>(a.DZ), static_cast<uint64_t>(a.L), static_cast<uint64_t>(a.B)};
+    const uint64_t zs[2] = {static_cast<uint64_t>(a.DZ) * 4, static_cast<uint64_t>(a.L) * a.DZ * 4};
+    const uint32_t zb[3] = {32, 128, 1};
+    const uint64_t od[4] = {static_cast<uint64_t>(a.F), static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.L),
+                            static_cast<uint64_t>(a.B)};
+    const uint64_t os[3] = {static_cast<uint64_t>(a.F) * 4, static_cast<uint64_t>(a.H) * a.F * 4,
+                            static_cast<uint64_t>(a.L) * a.H * a.F * 4};
+    const uint32_t ob[4] = {32, 1, 128, 1};
+    if (encode_tmap_f32_sw128(&tz1f, ws + w.z1f, 3, zd, zs, zb) && encode_tmap_f32_sw128(&tout, a.out, 4, od, os, ob))
+      t.tma_epi = 1;
+  }
   const int pairs = static_cast<int>(bh) * t.nqp;
   t.trace_cta0 = 0;
   t.trace_cta1 = 1;   // the peer CTA of the first pair
-  ipa_attention_pair_kernel<<<static_cast<unsigned>(2 * pairs), NT, SP_ALLOC, stream>>>(tqh, tkh, tz2k, tz2v, tvh, tz1, t);
+  ipa_attention_pair_kernel<<<static_cast<unsigned>(2 * pairs), NT, SP_ALLOC, stream>>>(tqh, tkh, tz2k, tz2v, tvh, tz1,
+                                                                                         tz1f, tout, t);
   return cudaGetLastError();
 }
 

@@ -649,11 +649,18 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       }
       if (lane == 0) oqs[s] = oqv;
       {
-        float* qp = reinterpret_cast<float*>(smem + lay.aux + KA_QPTS) + s * 64 * 12;
-        for (int e = lane; e < 64 * 12; e += 32) {
-          const int qq = i * 64 + e / 12;
-          qp[e] = qq < L ? a.pts[(static_cast<int64_t>(bh) * L + qq) * 24 + e % 12] : 0.f;
+        // the tile's 64 query points (12 floats = 3 float4 per query): six
+        // independent 16-byte loads per lane, all in flight together
+        float4* qp = reinterpret_cast<float4*>(smem + lay.aux + KA_QPTS) + s * 64 * 3;
+        const float4* src = reinterpret_cast<const float4*>(a.pts) + (static_cast<int64_t>(bh) * L + i * 64) * 6;
+        float4 v[6];
+#pragma unroll
+        for (int u = 0; u < 6; ++u) {
+          const int f = lane + 32 * u, row = f / 3;
+          v[u] = i * 64 + row < L ? src[row * 6 + f % 3] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+#pragma unroll
+        for (int u = 0; u < 6; ++u) qp[lane + 32 * u] = v[u];
       }
       __syncwarp();
       if (lane == 0) {

@@ -224,9 +224,14 @@ __device__ __forceinline__ void write_rows(const EpilogueArgs& e, int warp, int 
 // flight together.  tcgen05.ld is warp-collective, so every lane loads
 // and only the stores depend on the row being in range.
 template <int C, int PV>
+__device__ __forceinline__ void write_row_points(uint32_t tmem_v, float inv, bool dead, bool in_range, float* outr,
+                                                 float4 g0, float4 g1, float4 g2, float4 cn);
+
+template <int C, int PV>
 __device__ __forceinline__ void write_row_direct(uint32_t tmem_row, int half, int DZ, int Cz, int R, float inv,
                                                  bool dead, bool in_range, const float* z1r, float* outr, float* ur,
-                                                 float4 g0, float4 g1, float4 g2, float4 cn) {
+                                                 float4 g0, float4 g1, float4 g2, float4 cn,
+                                                 unsigned long long* trace = nullptr) {
   static_assert(C == 16 && PV == 8, "feature map written for the (16, 8) head shape");
   for (int c0 = half * (Cz / 2); c0 < (half + 1) * (Cz / 2); c0 += 32) {
     float acc[32];
@@ -259,10 +264,63 @@ __device__ __forceinline__ void write_row_direct(uint32_t tmem_row, int half, in
       for (int e = 0; e < 8; ++e) op[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
     }
   }
-  if (half == 0) {
+  if (trace != nullptr) trace[0] = clock64();   // tracing build: end of the pair part
+  if (half == 0) write_row_points<C, PV>(tmem_row + DZ, inv, dead, in_range, outr, g0, g1, g2, cn);
+}
+
+// Pair features of the CTA's rows through shared memory, for the layouts
+// the tensor-memory copy supports (R Cz = DZ, Cz a multiple of 32): z1 rows
+// come from TMA-loaded boxes and the folded features go to staging boxes
+// that one thread then stores with TMA.  Both are 128-row x 32-float boxes
+// with the 128-byte swizzle (16-byte chunk e of row r at byte 16 (e ^ (r & 7))
+// of the row), so thread-per-row float4 accesses are free of bank conflicts.
+// z1box(k): box k of the z1 row (columns 32 k ..); obox(k): staging box of
+// output pair features 32 k ..
+template <typename ZBox, typename OBox>
+__device__ __forceinline__ void stage_row_pair(uint32_t tmem_row, int half, int Cz, int R, float inv, int r,
+                                               float* ur, bool in_range, ZBox z1box, OBox obox) {
+  const int sw = r & 7;
+  for (int c0 = half * (Cz / 2); c0 < (half + 1) * (Cz / 2); c0 += 32) {
+    float acc[32];
+    for (int rf = 0; rf < R; ++rf) {
+      uint32_t o[32];
+      sm100::tmem_ld32(tmem_row + rf * Cz + c0, o);
+      const unsigned char* zrow = z1box((rf * Cz + c0) >> 5) + r * 128;
+      float4 z[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[e] = *reinterpret_cast<const float4*>(zrow + 16 * (e ^ sw));
+      sm100::tmem_ld_wait();
+      float u[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) u[e] = __uint_as_float(o[e]) * inv;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float zz[4] = {z[e].x, z[e].y, z[e].z, z[e].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[4 * e + k] = rf == 0 ? zz[k] * u[4 * e + k] : fmaf(zz[k], u[4 * e + k], acc[4 * e + k]);
+      }
+      if (ur != nullptr && in_range) {
+        float4* up = reinterpret_cast<float4*>(ur + rf * Cz + c0);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) up[e] = make_float4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
+      }
+    }
+    unsigned char* orow = obox(c0 >> 5) + r * 128;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      *reinterpret_cast<float4*>(orow + 16 * (e ^ sw)) = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+  }
+}
+
+// Scalar and point features of one row (the value aggregate O_v in tensor
+// memory at tmem_v): v / l, the value points mapped back with R^T, their norms.
+template <int C, int PV>
+__device__ __forceinline__ void write_row_points(uint32_t tmem_v, float inv, bool dead, bool in_range, float* outr,
+                                                 float4 g0, float4 g1, float4 g2, float4 cn) {
+  {
     uint32_t v0[32], v1[32];
-    sm100::tmem_ld32(tmem_row + DZ, v0);
-    sm100::tmem_ld32(tmem_row + DZ + 32, v1);
+    sm100::tmem_ld32(tmem_v, v0);
+    sm100::tmem_ld32(tmem_v + 32, v1);
     sm100::tmem_ld_wait();
     if (!in_range) return;
     float4* op = reinterpret_cast<float4*>(outr);
