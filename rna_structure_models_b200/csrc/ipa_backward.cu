@@ -33,10 +33,11 @@
 //   (both passes run as one grid, ipa_bwd_kernel, so that the key-pass CTAs
 //   fill the SMs the query pass leaves idle in its last wave)
 //   ipa_bwd_map_kernel   per residue, all heads: the augmented gradients
-//                        mapped back to q, k, v, the local points, the frames,
-//                        z1, z2 (sums over heads) and per-block partial sums of
-//                        d w_bias and d gamma;
-//   ipa_bwd_reduce_kernel  fixed-order sums of those partials.
+//                        mapped back to q, k, v, the local points and the
+//                        frames (sums over heads), per-block d gamma partials;
+//   ipa_bwd_pair_kernel  per pair column and residue: d z1, d z2
+//                        (sums over heads) and d w_bias partials;
+//   ipa_bwd_reduce_kernel  fixed-order sums of the partials, one block per head.
 // Every mbarrier wait is bounded (2 s) and reports into the error word.
 #include <cuda_fp16.h>
 
@@ -92,12 +93,10 @@ __device__ __forceinline__ float ldf(const View& v, int64_t off) {
                       : reinterpret_cast<const float*>(v.p)[off];
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      SM100_W16(r, 0)
-      : "memory");
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
 // ------------------------------------------------------------------ prologue
@@ -218,14 +217,19 @@ __global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
 }
 
 // --------------------------------------------------------------- query pass
-// Warps 0-7: two threads per query row (keys [32 half, 32 half + 32) of a
-// tile); warp 8: TMA producer and the per-key column terms; warp 9: tensor
-// memory and the MMA-issuing thread.
+// Warps 0-7: two threads per query row (keys [16 half, 16 half + 16) of a
+// 32-key tile); warp 8: TMA producer and the per-key column terms; warp 9:
+// tensor memory and the MMA-issuing thread.
 constexpr int NTH = 320, NSOFT = 256, W_PROD = 8, W_MMA = 9;
 constexpr int MAX_NS = 3;
+// Streamed tiles are 32 rows (keys in the query pass, queries in the key
+// pass): at R Cz = 256 a 64-row stage left room for one stage only, which put
+// every tile's load in series with its MMAs; 32-row stages fit two (query
+// pass) and three (key pass).
+constexpr int BT = 32;
 
 // tensor memory (512 columns)
-constexpr uint32_t Q_TM_DQP = 0, Q_TM_DQH = 256, Q_TM_S = 320, Q_TM_DP = 384, Q_TM_DS = 448;
+constexpr uint32_t Q_TM_DQP = 0, Q_TM_DQH = 256, Q_TM_S = 320, Q_TM_DP = 352, Q_TM_DS = 384;
 
 struct QLayout {
   uint32_t qh, qp, dO, du, stg, stg_bytes, aux, total;
@@ -238,12 +242,12 @@ __host__ __device__ inline QLayout q_layout(int DZ, int ns) {
   s.dO = s.qp + np * 16384;
   s.du = s.dO + 16384;
   s.stg = s.du + np * 16384;
-  s.stg_bytes = 16384 + np * 8192;          // K_h 8 KB | V_h 8 KB | Z2 np x 8 KB
+  s.stg_bytes = 8192 + np * 4096;           // K_h 4 KB | V_h 4 KB | Z2 np x 4 KB (32 keys)
   s.aux = s.stg + ns * s.stg_bytes;
   s.total = s.aux + 2048;
   return s;
 }
-// aux area: col terms [MAX_NS][64] floats (768 B) | tile info [MAX_NS][2] float4 (96 B) | barriers
+// aux area: col terms [MAX_NS][32] floats (384 B, from 0) | tile info [MAX_NS][2] float4 (96 B) | barriers
 constexpr uint32_t QA_COL = 0, QA_INFO = 768, QA_BAR = 896;
 enum { QB_QFULL = 0, QB_SFULL, QB_SFREE, QB_DSFULL, QB_DSFREE, QB_DRAIN, QB_FULL0, QB_EMPTY0 = QB_FULL0 + MAX_NS,
        QB_COUNT = QB_EMPTY0 + MAX_NS };
@@ -261,7 +265,7 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
   const int I = blk % a.nqt;
   const int bh = blk / a.nqt;
   const int b = bh / a.H, h = bh % a.H;
-  const int L = a.L, nt = a.nkt, DZ = a.DZ, np = DZ / 64, NS = a.ns;
+  const int L = a.L, nt = (a.L + BT - 1) / BT, DZ = a.DZ, np = DZ / 64, NS = a.ns;   // nt 32-key tiles
   const QLayout lay = q_layout(DZ, NS);
   float* col_s = reinterpret_cast<float*>(smem + lay.aux + QA_COL);
   float4* info = reinterpret_cast<float4*>(smem + lay.aux + QA_INFO);
@@ -318,17 +322,16 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         }
       }
       issued = j + 1;
-      const float4 okv = a.ok[b * nt + j];
+      const float4 okv = a.ok[b * a.nkt + j * BT / KT];   // the 64-key origin tile holding these keys
       const float dx = okv.x - oqv.x, dy = okv.y - oqv.y, dz = okv.z - oqv.z;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int key = j * KT + lane + 32 * t;
+      {
+        const int key = j * BT + lane;
         float cv = -INFINITY;
         if (key < L) {
           const float4 ck = a.colk[static_cast<int64_t>(bh) * L + key];
           cv = ck.w - fmaf(ck.x, dx, fmaf(ck.y, dy, ck.z * dz));
         }
-        col_s[s * 64 + lane + 32 * t] = cv;
+        col_s[s * BT + lane] = cv;
       }
       if (lane == 0) {
         info[2 * s] = make_float4(dx, dy, dz, fmaf(dx, dx, fmaf(dy, dy, dz * dz)));
@@ -338,9 +341,9 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
       if (lane == 0) {
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
         mbar_arrive_expect_tx(bar(QB_FULL0 + s), lay.stg_bytes);
-        tma_load_3d(st, &tm_kh, bar(QB_FULL0 + s), 0, j * KT, bh);
-        tma_load_3d(st + 8192, &tm_vh, bar(QB_FULL0 + s), 0, j * KT, bh);
-        tma_load_4d(st + 16384, &tm_z2, bar(QB_FULL0 + s), 0, j * KT, 0, b);
+        tma_load_3d(st, &tm_kh, bar(QB_FULL0 + s), 0, j * BT, bh);
+        tma_load_3d(st + 4096, &tm_vh, bar(QB_FULL0 + s), 0, j * BT, bh);
+        tma_load_4d(st + 8192, &tm_z2, bar(QB_FULL0 + s), 0, j * BT, 0, b);
       }
       __syncwarp();
     }
@@ -355,7 +358,7 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
       bool ok = mbar_wait_bounded(bar(QB_QFULL), 0, abort_flag);
       if (!ok) fail(DEV_TIMEOUT_FULL);
       tc_fence_after();
-      const uint32_t id64 = idesc_f16(128, 64, false);
+      const uint32_t id32 = idesc_f16(128, BT, false);
       const uint32_t id64mn = idesc_f16(128, 64, true);
       const uint32_t idz = idesc_f16(128, DZ, true);
       const uint32_t tS = tmem + Q_TM_S, tDP = tmem + Q_TM_DP, tDS = tmem + Q_TM_DS;
@@ -369,16 +372,16 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         tc_fence_after();
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.qh + 32 * k), kd128(st + 32 * k), id64, k > 0 ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.qh + 32 * k), kd128(st + 32 * k), id32, k > 0 ? 1u : 0u);
         for (int kk = 0; kk < 4 * np; ++kk)
           umma_ss(tS, kd128(sb + lay.qp + 16384 * (kk >> 2) + 32 * (kk & 3)),
-                  kd128(st + 16384 + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, 1u);
+                  kd128(st + 8192 + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma_ss(tDP, kd128(sb + lay.dO + 32 * k), kd128(st + 8192 + 32 * k), id64, k > 0 ? 1u : 0u);
+          umma_ss(tDP, kd128(sb + lay.dO + 32 * k), kd128(st + 4096 + 32 * k), id32, k > 0 ? 1u : 0u);
         for (int kk = 0; kk < 4 * np; ++kk)
           umma_ss(tDP, kd128(sb + lay.du + 16384 * (kk >> 2) + 32 * (kk & 3)),
-                  kd128(st + 16384 + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, 1u);
+                  kd128(st + 8192 + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
         umma_commit(bar(QB_SFULL));
         issued_any = true;
         return true;
@@ -389,10 +392,10 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         const int s = jj % NS;
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < BT / 16; ++k) {
           const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
-          umma_ts(tDQH, tDS + 8 * k, mnd(st + 2048 * k, 8192), id64mn, acc);
-          umma_ts(tDQP, tDS + 8 * k, mnd(st + 16384 + 2048 * k, 8192), idz, acc);
+          umma_ts(tDQH, tDS + 8 * k, mnd(st + 2048 * k, 4096), id64mn, acc);
+          umma_ts(tDQP, tDS + 8 * k, mnd(st + 8192 + 2048 * k, 4096), idz, acc);
         }
         umma_commit(bar(QB_DSFREE));
         umma_commit(bar(QB_EMPTY0 + s));
@@ -435,9 +438,9 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         break;
       }
       tc_fence_after();
-      uint32_t sv[32], dv[32];
-      tmem_ld32(tmem + Q_TM_S + 32 * half + lane_off, sv);
-      tmem_ld32(tmem + Q_TM_DP + 32 * half + lane_off, dv);
+      uint32_t sv[16], dv[16];
+      tmem_ld16(tmem + Q_TM_S + 16 * half + lane_off, sv);
+      tmem_ld16(tmem + Q_TM_DP + 16 * half + lane_off, dv);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(bar(QB_SFREE));
@@ -449,11 +452,11 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
       const float4 dd = info[2 * s], oj = info[2 * s + 1];
       const float rt = ch * (2.f * fmaf(sq.x, dd.x, fmaf(sq.y, dd.y, sq.z * dd.z)) - pq * dd.w);
       const float base = rt + rd.x;                        // row terms - (w + lse2); -inf on dead rows
-      const float* cv = col_s + s * 64 + 32 * half;
-      uint32_t pk[16];
+      const float* cv = col_s + s * BT + 16 * half;
+      uint32_t pk[8];
       float tsum = 0.f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < 8; ++k) {
         const float x0 = __uint_as_float(sv[2 * k]) + cv[2 * k] + base;
         const float x1 = __uint_as_float(sv[2 * k + 1]) + cv[2 * k + 1] + base;
         const float p0 = ex2(x0), p1 = ex2(x1);
@@ -473,7 +476,7 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         break;
       }
       tc_fence_after();
-      tmem_st16(tmem + Q_TM_DS + 16 * half + lane_off, pk);
+      tmem_st8(tmem + Q_TM_DS + 8 * half + lane_off, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(QB_DSFULL));
@@ -530,8 +533,10 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
 }
 
 // ----------------------------------------------------------------- key pass
-// Warps 0-7: two threads per key row (queries [32 half, 32 half + 32) of a
-// 64-query tile); warp 8: TMA producer and the per-query terms; warp 9: MMA.
+// Warps 0-7: two threads per key row (queries [16 half, 16 half + 16) of a
+// 32-query tile); warp 8: TMA producer and the per-query terms; warp 9: MMA.
+// S^T and dP^T are double-buffered (buffer i & 1, 32 columns each), so that
+// the MMAs of tile i + 1 run while the threads work on tile i.
 constexpr uint32_t K_TM_DZ2 = 0, K_TM_DKH = 256, K_TM_DVA = 320, K_TM_S = 384, K_TM_DP = 448;
 
 struct KLayout {
@@ -544,17 +549,18 @@ __host__ __device__ inline KLayout k_layout(int DZ, int ns) {
   s.vh = 16384;
   s.z2 = 32768;
   s.stg = s.z2 + np * 16384;
-  s.stg_bytes = 16384 + 2 * np * 8192;      // Q_h 8 KB | dO 8 KB | Q_pair np x 8 KB | dU np x 8 KB
+  s.stg_bytes = 8192 + 2 * np * 4096;       // Q_h 4 KB | dO 4 KB | Q_pair np x 4 KB | dU np x 4 KB (32 queries)
   s.aux = s.stg + ns * s.stg_bytes;
-  s.total = s.aux + 13312;
+  s.total = s.aux + 6656;
   return s;
 }
-// aux: per-query terms [MAX_NS][64] float4 (3 KB) | stage query-tile origin [MAX_NS] float4 | barriers |
-// per-stage query points [MAX_NS][64][12] floats (9 KB, from 4096)
-constexpr uint32_t KA_Q = 0, KA_OQ = 3072, KA_BAR = 3136, KA_QPTS = 4096;
-enum { KB_KFULL = 0, KB_SFULL, KB_PFULL, KB_ACC, KB_DRAIN, KB_FULL0, KB_EMPTY0 = KB_FULL0 + MAX_NS,
-       KB_COUNT = KB_EMPTY0 + MAX_NS };
+// aux: per-query terms [MAX_NS][32] float4 (1.5 KB) | stage query-tile origin [MAX_NS] float4 | barriers |
+// tensor-memory slot, abort flag, pair flags | per-stage query points [MAX_NS][32][12] floats (4.5 KB, from 2048)
+constexpr uint32_t KA_Q = 0, KA_OQ = 1536, KA_BAR = 1600, KA_QPTS = 2048;
+enum { KB_KFULL = 0, KB_SFULL0, KB_PFULL0 = KB_SFULL0 + 2, KB_ACC0 = KB_PFULL0 + 2, KB_DRAIN = KB_ACC0 + 2,
+       KB_FULL0, KB_EMPTY0 = KB_FULL0 + MAX_NS, KB_COUNT = KB_EMPTY0 + MAX_NS };
 constexpr uint32_t KA_TMEM = KA_BAR + 8 * KB_COUNT, KA_ABORT = KA_TMEM + 8, KA_PAIR = KA_ABORT + 8;
+static_assert(KA_PAIR + 64 <= KA_QPTS, "key-pass aux area overlaps the query points");
 
 __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_kh, const CUtensorMap& tm_vh,
                                            const CUtensorMap& tm_z2, const CUtensorMap& tm_qh,
@@ -570,7 +576,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
   const int bh = blk / nkp;
   const int b = bh / a.H, h = bh % a.H;
   const int L = a.L, DZ = a.DZ, np = DZ / 64, NS = a.ns;
-  const int nq = (L + 63) / 64;                 // 64-query tiles
+  const int nq = (L + BT - 1) / BT;             // 32-query tiles
   const KLayout lay = k_layout(DZ, NS);
   float4* qinfo = reinterpret_cast<float4*>(smem + lay.aux + KA_Q);
   float4* oqs = reinterpret_cast<float4*>(smem + lay.aux + KA_OQ);
@@ -580,9 +586,11 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
 
   if (tid == 0) {
     mbar_init(bar(KB_KFULL), 1);
-    mbar_init(bar(KB_SFULL), 1);
-    mbar_init(bar(KB_PFULL), NSOFT);
-    mbar_init(bar(KB_ACC), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(KB_SFULL0 + t), 1);
+      mbar_init(bar(KB_PFULL0 + t), NSOFT);
+      mbar_init(bar(KB_ACC0 + t), 1);
+    }
     mbar_init(bar(KB_DRAIN), 1);
     for (int s = 0; s < MAX_NS; ++s) {
       mbar_init(bar(KB_FULL0 + s), 1);
@@ -629,14 +637,13 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         }
       }
       issued = i + 1;
-      const int Iq = (i * 64) / QT;
+      const int Iq = (i * BT) / QT;
       const float4 oqv = a.oq[b * a.nqt + Iq];
       const float d0x = ok0.x - oqv.x, d0y = ok0.y - oqv.y, d0z = ok0.z - oqv.z;
       const float d1x = ok1.x - oqv.x, d1y = ok1.y - oqv.y, d1z = ok1.z - oqv.z;
       const float n0 = fmaf(d0x, d0x, fmaf(d0y, d0y, d0z * d0z)), n1 = fmaf(d1x, d1x, fmaf(d1y, d1y, d1z * d1z));
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int qi = i * 64 + lane + 32 * t;
+      {
+        const int qi = i * BT + lane;
         float4 e = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
         if (qi < L) {
           const float4 sq = a.rowq[static_cast<int64_t>(bh) * L + qi];
@@ -645,31 +652,31 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
           const float rt1 = ch * (2.f * fmaf(sq.x, d1x, fmaf(sq.y, d1y, sq.z * d1z)) - pq * n1);
           e = make_float4(rt0 + rd.x, rt1 + rd.x, rd.y, 0.f);
         }
-        qinfo[s * 64 + lane + 32 * t] = e;
+        qinfo[s * BT + lane] = e;
       }
       if (lane == 0) oqs[s] = oqv;
       {
-        // the tile's 64 query points (12 floats = 3 float4 per query): six
+        // the tile's 32 query points (12 floats = 3 float4 per query): three
         // independent 16-byte loads per lane, all in flight together
-        float4* qp = reinterpret_cast<float4*>(smem + lay.aux + KA_QPTS) + s * 64 * 3;
-        const float4* src = reinterpret_cast<const float4*>(a.pts) + (static_cast<int64_t>(bh) * L + i * 64) * 6;
-        float4 v[6];
+        float4* qp = reinterpret_cast<float4*>(smem + lay.aux + KA_QPTS) + s * BT * 3;
+        const float4* src = reinterpret_cast<const float4*>(a.pts) + (static_cast<int64_t>(bh) * L + i * BT) * 6;
+        float4 v[3];
 #pragma unroll
-        for (int u = 0; u < 6; ++u) {
+        for (int u = 0; u < 3; ++u) {
           const int f = lane + 32 * u, row = f / 3;
-          v[u] = i * 64 + row < L ? src[row * 6 + f % 3] : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[u] = i * BT + row < L ? src[row * 6 + f % 3] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 6; ++u) qp[lane + 32 * u] = v[u];
+        for (int u = 0; u < 3; ++u) qp[lane + 32 * u] = v[u];
       }
       __syncwarp();
       if (lane == 0) {
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
         mbar_arrive_expect_tx(bar(KB_FULL0 + s), lay.stg_bytes);
-        tma_load_3d(st, &tm_qh, bar(KB_FULL0 + s), 0, i * 64, bh);
-        tma_load_3d(st + 8192, &tm_do, bar(KB_FULL0 + s), 0, i * 64, bh);
-        tma_load_4d(st + 16384, &tm_qp, bar(KB_FULL0 + s), 0, i * 64, 0, bh);
-        tma_load_4d(st + 16384 + np * 8192, &tm_du, bar(KB_FULL0 + s), 0, i * 64, 0, bh);
+        tma_load_3d(st, &tm_qh, bar(KB_FULL0 + s), 0, i * BT, bh);
+        tma_load_3d(st + 4096, &tm_do, bar(KB_FULL0 + s), 0, i * BT, bh);
+        tma_load_4d(st + 8192, &tm_qp, bar(KB_FULL0 + s), 0, i * BT, 0, bh);
+        tma_load_4d(st + 8192 + np * 4096, &tm_du, bar(KB_FULL0 + s), 0, i * BT, 0, bh);
       }
       __syncwarp();
     }
@@ -683,46 +690,68 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       bool ok = mbar_wait_bounded(bar(KB_KFULL), 0, abort_flag);
       if (!ok) fail(DEV_TIMEOUT_FULL);
       tc_fence_after();
-      const uint32_t id64 = idesc_f16(128, 64, false);
+      const uint32_t id32 = idesc_f16(128, BT, false);
       const uint32_t id64mn = idesc_f16(128, 64, true);
       const uint32_t idz = idesc_f16(128, DZ, true);
-      const uint32_t tS = tmem + K_TM_S, tDP = tmem + K_TM_DP;
       bool issued_any = false;
-      for (int i = 0; ok && i < nq; ++i) {
-        const int s = i % NS;
-        ok = mbar_wait_bounded(bar(KB_FULL0 + s), (i / NS) & 1, abort_flag);
-        // the accumulation MMAs of tile i-1 read P^T / dS^T from the columns S^T / dP^T(i) overwrite
-        if (ok && i > 0) ok = mbar_wait_bounded(bar(KB_ACC), (i - 1) & 1, abort_flag);
-        if (!ok) { fail(DEV_TIMEOUT_FULL); break; }
+      // S^T(i), dP^T(i) into buffer i & 1, once stage i has landed and the
+      // accumulation MMAs of tile i - 2 (which read P^T / dS^T in place from
+      // that buffer) have completed
+      auto issue_sdp = [&](int i) -> bool {
+        const int s = i % NS, t = i & 1;
+        bool w = mbar_wait_bounded(bar(KB_FULL0 + s), (i / NS) & 1, abort_flag);
+        if (w && i >= 2) w = mbar_wait_bounded(bar(KB_ACC0 + t), ((i - 2) >> 1) & 1, abort_flag);
+        if (!w) { fail(DEV_TIMEOUT_FULL); return false; }
         tc_fence_after();
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
-        const uint32_t sQh = st, sDO = st + 8192, sQP = st + 16384, sDU = st + 16384 + np * 8192;
+        const uint32_t sQh = st, sDO = st + 4096, sQP = st + 8192, sDU = st + 8192 + np * 4096;
+        const uint32_t tS = tmem + K_TM_S + 32 * t, tDP = tmem + K_TM_DP + 32 * t;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.kh + 32 * k), kd128(sQh + 32 * k), id64, k > 0 ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.kh + 32 * k), kd128(sQh + 32 * k), id32, k > 0 ? 1u : 0u);
         for (int kk = 0; kk < 4 * np; ++kk)
           umma_ss(tS, kd128(sb + lay.z2 + 16384 * (kk >> 2) + 32 * (kk & 3)),
-                  kd128(sQP + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, 1u);
+                  kd128(sQP + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma_ss(tDP, kd128(sb + lay.vh + 32 * k), kd128(sDO + 32 * k), id64, k > 0 ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) umma_ss(tDP, kd128(sb + lay.vh + 32 * k), kd128(sDO + 32 * k), id32, k > 0 ? 1u : 0u);
         for (int kk = 0; kk < 4 * np; ++kk)
           umma_ss(tDP, kd128(sb + lay.z2 + 16384 * (kk >> 2) + 32 * (kk & 3)),
-                  kd128(sDU + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, 1u);
-        umma_commit(bar(KB_SFULL));
+                  kd128(sDU + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
+        umma_commit(bar(KB_SFULL0 + t));
         issued_any = true;
-        ok = mbar_wait_bounded(bar(KB_PFULL), i & 1, abort_flag);
-        if (!ok) { fail(DEV_TIMEOUT_SOFTMAX); break; }
+        return true;
+      };
+      // dV += P^T dO, dZ2 += P^T dU + dS^T Q_pair, dK_h += dS^T Q_h for tile
+      // i, once its threads have written P^T / dS^T (fp16, in place)
+      auto issue_acc = [&](int i) -> bool {
+        const int s = i % NS, t = i & 1;
+        if (!mbar_wait_bounded(bar(KB_PFULL0 + t), (i >> 1) & 1, abort_flag)) { fail(DEV_TIMEOUT_SOFTMAX); return false; }
         tc_fence_after();
-        // P^T in columns [K_TM_S, +32), dS^T in [K_TM_DP, +32) (fp16, 64 queries)
+        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+        const uint32_t sQh = st, sDO = st + 4096, sQP = st + 8192, sDU = st + 8192 + np * 4096;
+        const uint32_t tS = tmem + K_TM_S + 32 * t, tDP = tmem + K_TM_DP + 32 * t;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < BT / 16; ++k) {
           const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-          umma_ts(tmem + K_TM_DVA, tS + 8 * k, mnd(sDO + 2048 * k, 8192), id64mn, acc);
-          umma_ts(tmem + K_TM_DZ2, tS + 8 * k, mnd(sDU + 2048 * k, 8192), idz, acc);
-          umma_ts(tmem + K_TM_DZ2, tDP + 8 * k, mnd(sQP + 2048 * k, 8192), idz, 1u);
-          umma_ts(tmem + K_TM_DKH, tDP + 8 * k, mnd(sQh + 2048 * k, 8192), id64mn, acc);
+          umma_ts(tmem + K_TM_DVA, tS + 8 * k, mnd(sDO + 2048 * k, 4096), id64mn, acc);
+          umma_ts(tmem + K_TM_DZ2, tS + 8 * k, mnd(sDU + 2048 * k, 4096), idz, acc);
+          umma_ts(tmem + K_TM_DZ2, tDP + 8 * k, mnd(sQP + 2048 * k, 4096), idz, 1u);
+          umma_ts(tmem + K_TM_DKH, tDP + 8 * k, mnd(sQh + 2048 * k, 4096), id64mn, acc);
         }
-        umma_commit(bar(KB_ACC));
+        umma_commit(bar(KB_ACC0 + t));
         umma_commit(bar(KB_EMPTY0 + s));
+        return true;
+      };
+      // with two or more stages S^T / dP^T(i) are issued before the
+      // accumulation of tile i - 1; with one, tile i cannot load until that
+      // accumulation has released the stage
+      for (int i = 0; ok && i <= nq; ++i) {
+        if (NS == 1) {
+          if (i > 0) ok = issue_acc(i - 1);
+          if (ok && i < nq) ok = issue_sdp(i);
+        } else {
+          if (i < nq) ok = issue_sdp(i);
+          if (ok && i > 0) ok = issue_acc(i - 1);
+        }
       }
       if (!ok && issued_any) {
         umma_commit(bar(KB_DRAIN));
@@ -757,12 +786,13 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       const int s = i % NS;
       // the two warps of these lanes decide together whether to go on, so
       // that neither waits at their shared barrier for one that has left
-      const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_SFULL), i & 1, abort_flag));
-      uint32_t sv[32], dv[32];
+      const int tb = i & 1;                   // tensor-memory buffer of this tile
+      const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_SFULL0 + tb), (i >> 1) & 1, abort_flag));
+      uint32_t sv[16], dv[16];
       if (got) {
         tc_fence_after();
-        tmem_ld32(tmem + K_TM_S + 32 * half + lane_off, sv);
-        tmem_ld32(tmem + K_TM_DP + 32 * half + lane_off, dv);
+        tmem_ld16(tmem + K_TM_S + 32 * tb + 16 * half + lane_off, sv);
+        tmem_ld16(tmem + K_TM_DP + 32 * tb + 16 * half + lane_off, dv);
         tmem_ld_wait();
         tc_fence_before();
       }
@@ -780,9 +810,9 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       }
       const float4 oqv = oqs[s];
       const float colv = ck.w - fmaf(ck.x, okj.x - oqv.x, fmaf(ck.y, okj.y - oqv.y, ck.z * (okj.z - oqv.z)));
-      const float4* qi = qinfo + s * 64 + 32 * half;
-      // this half's 32 query points relative to the centroid, 12 floats each
-      const float4* qc = reinterpret_cast<const float4*>(smem + lay.aux + KA_QPTS) + (s * 64 + 32 * half) * 3;
+      const float4* qi = qinfo + s * BT + 16 * half;
+      // this half's 16 query points relative to the centroid, 12 floats each
+      const float4* qc = reinterpret_cast<const float4*>(smem + lay.aux + KA_QPTS) + (s * BT + 16 * half) * 3;
       // |gq_i - gk_j|^2, two coordinates per packed instruction
       auto dist2 = [&](const int k) {
         const float4 g0 = qc[3 * k], g1 = qc[3 * k + 1], g2 = qc[3 * k + 2];
@@ -797,10 +827,10 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         acc = fma_f32x2(d5, d5, acc);
         return acc.x + acc.y;
       };
-      uint32_t pp[16], pd[16];
+      uint32_t pp[8], pd[8];
       float tsum = 0.f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < 8; ++k) {
         const float4 e0 = qi[2 * k], e1 = qi[2 * k + 1];
         const float x0 = __uint_as_float(sv[2 * k]) + colv + (sub ? e0.y : e0.x);
         const float x1 = __uint_as_float(sv[2 * k + 1]) + colv + (sub ? e1.y : e1.x);
@@ -819,13 +849,14 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       co1 = fmaf(tsum, oqv.y, co1);
       co2 = fmaf(tsum, oqv.z, co2);
       tc_fence_after();
-      tmem_st16(tmem + K_TM_S + 16 * half + lane_off, pp);
-      tmem_st16(tmem + K_TM_DP + 16 * half + lane_off, pd);
+      tmem_st8(tmem + K_TM_S + 32 * tb + 8 * half + lane_off, pp);
+      tmem_st8(tmem + K_TM_DP + 32 * tb + 8 * half + lane_off, pd);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(KB_PFULL));
+      mbar_arrive(bar(KB_PFULL0 + tb));
     }
-    if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_ACC), (nq - 1) & 1, abort_flag))) {
+    // the commit after the last accumulation tracks every earlier MMA of the issuing thread
+    if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_ACC0 + ((nq - 1) & 1)), ((nq - 1) >> 1) & 1, abort_flag))) {
       if (lane == 0) fail(DEV_TIMEOUT_MMA);
       ok = false;
     }
@@ -912,15 +943,15 @@ struct MapArgs {
   int nqt, nkt;
   // gradients (contiguous fp32)
   float *d_q, *d_k, *d_v, *d_qpts, *d_kpts, *d_vpts, *d_rot, *d_trans, *d_z1, *d_z2;
-  float* wb_part;        // [nblk * B][H][DZ]
+  float* wb_part;        // [B][pair-column blocks][H][DZ]
   double* g_part;        // [nblk * B][H]
 };
 
 // Block: rb residues of one batch, all heads.  Phase 1: thread (residue,
 // head) -> scalar and point gradients, per-head frame contributions and
 // d gamma terms; phase 2: frame gradients summed over heads in a fixed
-// order; phase 3: thread per pair column -> d z1, d z2 (sums over heads)
-// and the block's partial sums of d w_bias.
+// order, and the block's d gamma partial (the pair columns are
+// ipa_bwd_pair_kernel's).
 __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
   extern __shared__ float sm_map[];   // [rb][H][12] frame terms, then [rb][H] d gamma (double)
   const int blk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
@@ -1039,59 +1070,96 @@ __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
     for (int il = 0; il < rb; ++il) s += gterm[il * H + h];
     a.g_part[(static_cast<int64_t>(b) * a.nblk + blk) * H + h] = s;
   }
-  // pair columns
-  for (int col = tid; col < a.DZ; col += blockDim.x) {
-    const int cc = col % a.Cz, rr = col / a.Cz;
-    const bool inpair = col < a.RCz;
-    for (int il = 0; il < rb; ++il) {
-      const int i = i0 + il;
-      if (i >= a.L) break;
-      if (!inpair) continue;
-      const int64_t bi = static_cast<int64_t>(b) * a.L + i;
-      float s1 = 0.f, s2 = 0.f;
-      for (int h = 0; h < H; ++h) {
-        const int64_t bhl = (static_cast<int64_t>(b) * H + h) * a.L + i;
-        const float gp = ldf(a.g_out, b * a.g_out.s[0] + i * a.g_out.s[1] + h * a.g_out.s[2] +
+}
+
+// Pair columns: a block covers 32 columns x PAIR_RB = 8 residues, one thread
+// per (column, residue): d z1 and d z2 (sums over heads, heads in order);
+// the per-residue terms z1 dQ_pair of every head are summed over the block's
+// residues in order through shared memory (d w_bias partials).  Warps read
+// 32 consecutive columns of one row.
+constexpr int PAIR_RB = 8;
+constexpr int PAIR_HC = 16;
+
+__global__ void __launch_bounds__(256) ipa_bwd_pair_kernel(const MapArgs a) {
+  __shared__ float wsm[PAIR_RB][PAIR_HC][33];
+  const int tid = threadIdx.x, cl = tid & 31, il = tid >> 5;
+  const int col = blockIdx.x * 32 + cl;
+  const int blk = blockIdx.y, b = blockIdx.z;
+  const int i = blk * PAIR_RB + il;
+  const int H = a.H, C = IPA_C, PV = IPA_PV;
+  const bool valid = i < a.L && col < a.DZ;
+  const int ic = valid ? i : 0, cc0 = col < a.DZ ? col : 0;
+  const int cc = cc0 % a.Cz, rr = cc0 / a.Cz;
+  const bool inpair = valid && col < a.RCz;
+  const int64_t bi = static_cast<int64_t>(b) * a.L + ic;
+  const bool live = valid && a.frame[bi * 4 + 3].x != 0.f;
+  const float z1 = valid ? a.z1f[bi * a.DZ + cc0] : 0.f;
+  float s1 = 0.f, s2 = 0.f;
+  for (int h0 = 0; h0 < H; h0 += PAIR_HC) {
+    const int nh = H - h0 < PAIR_HC ? H - h0 : PAIR_HC;
+#pragma unroll 4
+    for (int hh = 0; hh < nh; ++hh) {
+      const int h = h0 + hh;
+      const int64_t bhl = (static_cast<int64_t>(b) * H + h) * a.L + ic;
+      const float dq = valid ? a.dqp[bhl * a.DZ + cc0] : 0.f;
+      if (inpair) {
+        const float gp = ldf(a.g_out, b * a.g_out.s[0] + ic * a.g_out.s[1] + h * a.g_out.s[2] +
                                           (C + 4 * PV + cc) * a.g_out.s[3]);
-        const float u = ldf(a.uagg, b * a.uagg.s[0] + i * a.uagg.s[1] + h * a.uagg.s[2] + rr * a.uagg.s[3] +
+        const float u = ldf(a.uagg, b * a.uagg.s[0] + ic * a.uagg.s[1] + h * a.uagg.s[2] + rr * a.uagg.s[3] +
                                         cc * a.uagg.s[4]);
-        const bool live = a.frame[bi * 4 + 3].x != 0.f;
-        s1 += a.wqp[h * a.DZ + col] * a.dqp[bhl * a.DZ + col] + (live ? gp * u : 0.f);
-        s2 += a.dz2[bhl * a.DZ + col];
+        s1 += a.wqp[h * a.DZ + cc0] * dq + (live ? gp * u : 0.f);
+        s2 += a.dz2[bhl * a.DZ + cc0];
       }
-      a.d_z1[bi * a.RCz + col] = s1;
-      a.d_z2[bi * a.RCz + col] = s2;
+      wsm[il][hh][cl] = z1 * dq;
     }
-    for (int h = 0; h < H; ++h) {
-      float s = 0.f;
-      for (int il = 0; il < rb; ++il) {
-        const int i = i0 + il;
-        if (i >= a.L) break;
-        const int64_t bi = static_cast<int64_t>(b) * a.L + i;
-        const int64_t bhl = (static_cast<int64_t>(b) * H + h) * a.L + i;
-        s = fmaf(a.z1f[bi * a.DZ + col], a.dqp[bhl * a.DZ + col], s);
-      }
-      a.wb_part[((static_cast<int64_t>(b) * a.nblk + blk) * H + h) * a.DZ + col] = s;
+    __syncthreads();
+    for (int t = tid; t < nh * 32; t += blockDim.x) {
+      const int hh = t >> 5, c = t & 31;
+      float w = 0.f;
+#pragma unroll
+      for (int q = 0; q < PAIR_RB; ++q) w += wsm[q][hh][c];
+      if (blockIdx.x * 32 + c < a.DZ)
+        a.wb_part[((static_cast<int64_t>(b) * gridDim.y + blk) * H + h0 + hh) * a.DZ + blockIdx.x * 32 + c] = w;
     }
+    __syncthreads();
+  }
+  if (inpair) {
+    a.d_z1[bi * a.RCz + col] = s1;
+    a.d_z2[bi * a.RCz + col] = s2;
   }
 }
 
-// d w_bias[c, h] = log2(e) w_L sum over blocks and factors r of the partials;
-// d gamma[h] = sum over blocks.  One thread per output, fixed order.
-__global__ void ipa_bwd_reduce_kernel(const float* wb_part, const double* g_part, int nparts, int H, int DZ, int Cz,
-                                      int R, float scale, float* d_wb, float* d_gamma) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t < Cz * H) {
-    const int c = t / H, h = t % H;
-    double s = 0.0;
-    for (int p = 0; p < nparts; ++p)
-      for (int r = 0; r < R; ++r) s += wb_part[(static_cast<int64_t>(p) * H + h) * DZ + r * Cz + c];
-    d_wb[c * H + h] = static_cast<float>(s * scale);
-  } else if (t < Cz * H + H) {
-    const int h = t - Cz * H;
-    double s = 0.0;
-    for (int p = 0; p < nparts; ++p) s += g_part[static_cast<int64_t>(p) * H + h];
-    d_gamma[h] = static_cast<float>(s);
+// One block of 1024 threads per (head, 32 columns).  Thread (c, g): group g
+// of 32 sums parts g, g + 32, ... (factors r in order) for column c; the 32
+// group sums are then added in group order.  Warp 0 of the first column
+// block sums the d gamma parts, lane l taking parts l, l + 32, ..., then a
+// fixed shuffle tree.  The order of every sum depends on the sizes alone, so
+// the result is reproducible.
+constexpr int RED_THREADS = 1024;
+__global__ void __launch_bounds__(RED_THREADS) ipa_bwd_reduce_kernel(const float* wb_part, int nwb, const double* g_part,
+                                                                     int ng, int H, int DZ, int Cz, int R, float scale,
+                                                                     float* d_wb, float* d_gamma) {
+  __shared__ double red[32][33];
+  const int h = blockIdx.x, t = threadIdx.x, cl = t & 31, g = t >> 5;
+  const int c = blockIdx.y * 32 + cl;
+  double acc = 0.0;
+  if (c < Cz)
+    for (int p = g; p < nwb; p += 32)
+      for (int r = 0; r < R; ++r) acc += wb_part[(static_cast<int64_t>(p) * H + h) * DZ + r * Cz + c];
+  red[g][cl] = acc;
+  __syncthreads();
+  if (t < 32 && c < Cz) {
+    double sum = 0.0;
+    for (int q = 0; q < 32; ++q) sum += red[q][t];
+    d_wb[c * H + h] = static_cast<float>(sum * scale);
+  }
+  if (blockIdx.y == 0 && t >= 32 && t < 64) {
+    const int l = t - 32;
+    double gs = 0.0;
+    for (int p = l; p < ng; p += 32) gs += g_part[static_cast<int64_t>(p) * H + h];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, off);
+    if (l == 0) d_gamma[h] = static_cast<float>(gs);
   }
 }
 
@@ -1110,7 +1178,8 @@ IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz) {
   size_t o = up(w.fwd.total);
   const size_t bhl = static_cast<size_t>(B) * H * L;
   const int rb = 256 / H < 32 ? 256 / H : 32;
-  const size_t nblk = (L + rb - 1) / rb;
+  const size_t nblk = (L + rb - 1) / rb;                // per-residue mapping blocks
+  const size_t npb = (L + PAIR_RB - 1) / PAIR_RB;        // pair-column blocks
   w.doh = o; o = up(o + bhl * 64 * 2);
   w.du = o; o = up(o + bhl * DZ * 2);
   w.qp = o; o = up(o + bhl * DZ * 2);
@@ -1124,7 +1193,7 @@ IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz) {
   w.csk = o; o = up(o + bhl * 16);
   w.pts = o; o = up(o + bhl * 24 * 4);
   w.gsum = o; o = up(o + bhl * 4);
-  w.wb_part = o; o = up(o + static_cast<size_t>(B) * nblk * H * DZ * 4);
+  w.wb_part = o; o = up(o + static_cast<size_t>(B) * npb * H * DZ * 4);
   w.g_part = o; o = up(o + static_cast<size_t>(B) * nblk * H * 8);
   w.total = o;
   return w;
@@ -1198,22 +1267,22 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
               encode_tmap_f16_panels(&mp.q_qp, ws + w.qp, DZ, L, bh, 128, np) &&
               encode_tmap_f16_3d(&mp.q_do, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, 128) &&
               encode_tmap_f16_panels(&mp.q_du, ws + w.du, DZ, L, bh, 128, np) &&
-              encode_tmap_f16_3d(&mp.q_kh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, 64) &&
-              encode_tmap_f16_3d(&mp.q_vh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, 64) &&
-              encode_tmap_f16_panels(&mp.q_z2, ws + fw.z2, DZ, L, B, 64, np) &&
+              encode_tmap_f16_3d(&mp.q_kh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, BT) &&
+              encode_tmap_f16_3d(&mp.q_vh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, BT) &&
+              encode_tmap_f16_panels(&mp.q_z2, ws + fw.z2, DZ, L, B, BT, np) &&
               encode_tmap_f16_3d(&mp.k_kh, ws + fw.kh, DH, L, bh, DH * 2, rowb, 64, 128) &&
               encode_tmap_f16_3d(&mp.k_vh, ws + fw.vh, DH, L, bh, DH * 2, rowb, 64, 128) &&
               encode_tmap_f16_panels(&mp.k_z2, ws + fw.z2, DZ, L, B, 128, np) &&
-              encode_tmap_f16_3d(&mp.k_qh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, 64) &&
-              encode_tmap_f16_3d(&mp.k_do, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, 64) &&
-              encode_tmap_f16_panels(&mp.k_qp, ws + w.qp, DZ, L, bh, 64, np) &&
-              encode_tmap_f16_panels(&mp.k_du, ws + w.du, DZ, L, bh, 64, np);
+              encode_tmap_f16_3d(&mp.k_qh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, BT) &&
+              encode_tmap_f16_3d(&mp.k_do, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, BT) &&
+              encode_tmap_f16_panels(&mp.k_qp, ws + w.qp, DZ, L, bh, BT, np) &&
+              encode_tmap_f16_panels(&mp.k_du, ws + w.du, DZ, L, bh, BT, np);
     if (!ok) return cudaErrorInvalidValue;
     const QLayout l1 = q_layout(DZ, 1);
     ba.ns = stages_for(l1.stg, l1.stg_bytes, 2048);
     const KLayout k1 = k_layout(DZ, 1);
     BwdArgs kb = ba;
-    kb.ns = stages_for(k1.stg, k1.stg_bytes, 13312);
+    kb.ns = stages_for(k1.stg, k1.stg_bytes, 6656);
     const uint32_t sq = q_layout(DZ, ba.ns).total, sk = k_layout(DZ, kb.ns).total;
     const uint32_t smem = (sq > sk ? sq : sk) + 1024;
     e = cudaFuncSetAttribute(ipa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -1242,9 +1311,14 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   ipa_bwd_map_kernel<<<dim3(static_cast<unsigned>(m.nblk), static_cast<unsigned>(B)), 256, msmem, stream>>>(m);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int nout = f.Cz * H + H;
-  ipa_bwd_reduce_kernel<<<(nout + 127) / 128, 128, 0, stream>>>(m.wb_part, m.g_part, B * m.nblk, H, DZ, f.Cz, f.R,
-                                                               kLog2e * f.w_L, a.d_w_bias, a.d_gamma);
+  const int npb = (L + PAIR_RB - 1) / PAIR_RB;
+  ipa_bwd_pair_kernel<<<dim3(static_cast<unsigned>((DZ + 31) / 32), static_cast<unsigned>(npb), static_cast<unsigned>(B)),
+                        256, 0, stream>>>(m);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 rgrid(static_cast<unsigned>(H), static_cast<unsigned>((f.Cz + 31) / 32));
+  ipa_bwd_reduce_kernel<<<rgrid, RED_THREADS, 0, stream>>>(m.wb_part, B * npb, m.g_part, B * m.nblk, H, DZ, f.Cz, f.R,
+                                                          kLog2e * f.w_L, a.d_w_bias, a.d_gamma);
   return cudaGetLastError();
 }
 
