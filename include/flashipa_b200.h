@@ -177,6 +177,29 @@ IPA_API ipa_status_t ipa_attn_fwd_host(const ipa_params_t* p,
                           void* workspace, size_t workspace_bytes,
                           void* stream, int32_t* dev_err);
 
+/* Packed host inputs: the 13 inputs of ipa_attn_fwd_host, stored dense
+ * (C order, IPA_DTYPE_F32; mask one byte per element) in one host buffer in
+ * argument order, input t starting at byte offsets[t] (multiples of 256).
+ * ipa_attn_host_packed_layout fills offsets[13] and returns the buffer's
+ * size in bytes (0 for invalid params or a null offsets).  Pure host
+ * function.
+ *
+ * ipa_attn_fwd_host_packed is ipa_attn_fwd_host for such a buffer
+ * (`host_inputs`, `host_bytes` >= the layout size; page-locked for the copy
+ * to be asynchronous): one cudaMemcpyAsync of the whole buffer into
+ * `staging` instead of one per input (each copy has a fixed cost on the
+ * copy engine; thirteen cost ~0.3 ms per call at L = 4096), then the same
+ * kernels and the copy of the result into `out` (host, [B, L, H, C + 4 Pv +
+ * Cz] IPA_DTYPE_F32, contiguous).  Same staging, workspace, stream and error
+ * rules as ipa_attn_fwd_host; IPA_ERR_SHAPE if host_bytes is too small. */
+IPA_API size_t ipa_attn_host_packed_layout(const ipa_params_t* p, size_t offsets[13]);
+
+IPA_API ipa_status_t ipa_attn_fwd_host_packed(const ipa_params_t* p, const void* host_inputs,
+                          size_t host_bytes, const ipa_tensor_t* out,
+                          void* staging, size_t staging_bytes,
+                          void* workspace, size_t workspace_bytes,
+                          void* stream, int32_t* dev_err);
+
 /* --------------------------------------------------------------------------
  * Training forward and gradients of the fused IPA core (Flash Invariant
  * Point Attention trains the factorised IPA: TL;DR "drop-in replacement",

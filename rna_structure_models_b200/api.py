@@ -23,7 +23,8 @@ STATUS = {0: "IPA_OK", 1: "IPA_ERR_NULL", 2: "IPA_ERR_SHAPE", 3: "IPA_ERR_STRIDE
           8: "IPA_ERR_TIMEOUT"}
 EXPORTED = ("ipa_attn_workspace_size", "ipa_attn_fwd", "ipa_attn_prologue", "ipa_attn_core",
             "ipa_attn_fwd_train", "ipa_attn_bwd_workspace_size", "ipa_attn_bwd",
-            "ipa_attn_host_staging_size", "ipa_attn_fwd_host",
+            "ipa_attn_host_staging_size", "ipa_attn_fwd_host", "ipa_attn_host_packed_layout",
+            "ipa_attn_fwd_host_packed",
             "geo_attn_workspace_size", "geo_attn_fwd", "geo_attn_fwd_static",
             "geo_attn_bwd_workspace_size", "geo_attn_bwd",
             "meet_attn_workspace_size", "meet_attn_fwd", "ipa_frames_from_backbone", "ipa_linear_workspace_size",
@@ -111,6 +112,12 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                                  ctypes.c_void_p, ctypes.c_size_t,
                                                                  ctypes.c_void_p, ctypes.c_void_p]
     lib.ipa_attn_fwd_host.restype = ctypes.c_int
+    lib.ipa_attn_host_packed_layout.argtypes = [P(IpaParams), P(ctypes.c_size_t * 13)]
+    lib.ipa_attn_host_packed_layout.restype = ctypes.c_size_t
+    lib.ipa_attn_fwd_host_packed.argtypes = [P(IpaParams), ctypes.c_void_p, ctypes.c_size_t, T, ctypes.c_void_p,
+                                             ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                             ctypes.c_void_p]
+    lib.ipa_attn_fwd_host_packed.restype = ctypes.c_int
     lib.ipa_attn_bwd_workspace_size.argtypes = [P(IpaParams)]
     lib.ipa_attn_bwd_workspace_size.restype = ctypes.c_size_t
     lib.ipa_attn_bwd.argtypes = [P(IpaParams)] + [T] * 17 + [P(IpaGrads), ctypes.c_void_p, ctypes.c_size_t,
@@ -442,6 +449,44 @@ class IpaHostCalls:
                                          ctypes.c_size_t(self.workspace[slot].numel()),
                                          ctypes.c_void_p(self.streams[slot].cuda_stream),
                                          ctypes.c_void_p(self.dev_err[slot:].data_ptr()))
+        if st != 0:
+            raise IpaError(st, library().ipa_status_string(st).decode())
+
+    def packed_layout(self):
+        """(size in bytes, byte offsets of the 13 inputs) of the packed host
+        buffer ipa_attn_fwd_host_packed reads."""
+        offs = (ctypes.c_size_t * 13)()
+        n = int(library().ipa_attn_host_packed_layout(ctypes.byref(self.params), ctypes.byref(offs)))
+        if n == 0:
+            raise IpaError(2, "shape mismatch")
+        return n, [int(o) for o in offs]
+
+    def pack(self, inp: dict, buf=None):
+        """Copies the 13 host inputs (contiguous; fp32, mask bool / uint8) into
+        one page-locked byte buffer at the packed offsets (a host-side copy,
+        done once per set of inputs, outside any timed call)."""
+        n, offs = self.packed_layout()
+        if buf is None:
+            buf = torch.zeros(n, dtype=torch.uint8, pin_memory=True)
+        for name, off in zip(IPA_INPUTS, offs):
+            t = inp[name].contiguous()
+            if t.dtype == torch.bool:
+                t = t.to(torch.uint8)
+            b = t.reshape(-1).view(torch.uint8)
+            buf[off:off + b.numel()].copy_(b)
+        return buf
+
+    def call_packed(self, buf, out, slot: int = 0):
+        """Enqueue one ipa_attn_fwd_host_packed call on slot `slot`'s stream."""
+        od = tensor_desc(out)
+        st = library().ipa_attn_fwd_host_packed(ctypes.byref(self.params), ctypes.c_void_p(buf.data_ptr()),
+                                                ctypes.c_size_t(buf.numel()), ctypes.byref(od),
+                                                ctypes.c_void_p(self.staging[slot].data_ptr()),
+                                                ctypes.c_size_t(self.staging[slot].numel()),
+                                                ctypes.c_void_p(self.workspace[slot].data_ptr()),
+                                                ctypes.c_size_t(self.workspace[slot].numel()),
+                                                ctypes.c_void_p(self.streams[slot].cuda_stream),
+                                                ctypes.c_void_p(self.dev_err[slot:].data_ptr()))
         if st != 0:
             raise IpaError(st, library().ipa_status_string(st).decode())
 

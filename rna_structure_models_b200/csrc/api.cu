@@ -333,15 +333,23 @@ size_t ipa_attn_host_staging_size(const ipa_params_t* p) {
   return total;
 }
 
-ipa_status_t ipa_attn_fwd_host(const ipa_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,
-                               const ipa_tensor_t* v, const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
-                               const ipa_tensor_t* v_pts, const ipa_tensor_t* rot, const ipa_tensor_t* trans,
-                               const ipa_tensor_t* z1, const ipa_tensor_t* z2, const ipa_tensor_t* w_bias,
-                               const ipa_tensor_t* gamma, const ipa_tensor_t* mask, const ipa_tensor_t* out,
-                               void* staging, size_t staging_bytes, void* workspace, size_t workspace_bytes,
-                               void* stream, int32_t* dev_err) {
-  const ipa_tensor_t* in[14] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask, out};
+}  // extern "C"
+
+namespace {
+
+// Host-buffer call: the inputs up into `staging` (one copy per input, or,
+// when packed_bytes > 0, one copy of the packed buffer that starts at q's
+// data and holds the inputs at the staging offsets), the kernels, the result
+// down.
+ipa_status_t host_call(const ipa_params_t* p, const ipa_tensor_t* const in13[13], const ipa_tensor_t* out,
+                       void* staging, size_t staging_bytes, void* workspace, size_t workspace_bytes, void* stream,
+                       int32_t* dev_err, size_t packed_bytes) {
   if (out == nullptr) return IPA_ERR_NULL;
+  for (int t = 0; t < 13; ++t)
+    if (in13[t] == nullptr) return IPA_ERR_NULL;
+  const ipa_tensor_t* in[14];
+  for (int t = 0; t < 13; ++t) in[t] = in13[t];
+  in[13] = out;
   // shapes, dtypes and the workspace through the device entry point's checks
   // (host pointers are only compared, never dereferenced, there)
   IpaLaunch a;
@@ -358,10 +366,13 @@ ipa_status_t ipa_attn_fwd_host(const ipa_params_t* p, const ipa_tensor_t* q, con
   ipa_tensor_t dev[14];
   size_t off = 0;
   const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (packed_bytes > 0 && cudaMemcpyAsync(sbase, in[0]->data, packed_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    return IPA_ERR_CUDA;
   for (int t = 0; t < 14; ++t) {
     dev[t] = *in[t];
     dev[t].data = sbase + off;
-    if (t < 13 && cudaMemcpyAsync(sbase + off, in[t]->data, sz[t], cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    if (packed_bytes == 0 && t < 13 &&
+        cudaMemcpyAsync(sbase + off, in[t]->data, sz[t], cudaMemcpyHostToDevice, cs) != cudaSuccess)
       return IPA_ERR_CUDA;
     off += up256(sz[t]);
   }
@@ -373,6 +384,74 @@ ipa_status_t ipa_attn_fwd_host(const ipa_params_t* p, const ipa_tensor_t* q, con
   if (cudaMemcpyAsync(const_cast<void*>(out->data), dev[13].data, sz[13], cudaMemcpyDeviceToHost, cs) != cudaSuccess)
     return IPA_ERR_CUDA;
   return IPA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ipa_status_t ipa_attn_fwd_host(const ipa_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,
+                               const ipa_tensor_t* v, const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
+                               const ipa_tensor_t* v_pts, const ipa_tensor_t* rot, const ipa_tensor_t* trans,
+                               const ipa_tensor_t* z1, const ipa_tensor_t* z2, const ipa_tensor_t* w_bias,
+                               const ipa_tensor_t* gamma, const ipa_tensor_t* mask, const ipa_tensor_t* out,
+                               void* staging, size_t staging_bytes, void* workspace, size_t workspace_bytes,
+                               void* stream, int32_t* dev_err) {
+  const ipa_tensor_t* in[13] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, w_bias, gamma, mask};
+  return host_call(p, in, out, staging, staging_bytes, workspace, workspace_bytes, stream, dev_err, 0);
+}
+
+size_t ipa_attn_host_packed_layout(const ipa_params_t* p, size_t offsets[13]) {
+  ipa_status_t st;
+  if (offsets == nullptr || !ipa_dims_ok(p, &st)) return 0;
+  size_t sz[14], off = 0;
+  ipa_host_sizes(p, sz);
+  for (int t = 0; t < 13; ++t) {
+    offsets[t] = off;
+    off += up256(sz[t]);
+  }
+  return off;
+}
+
+ipa_status_t ipa_attn_fwd_host_packed(const ipa_params_t* p, const void* host_inputs, size_t host_bytes,
+                                      const ipa_tensor_t* out, void* staging, size_t staging_bytes,
+                                      void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err) {
+  if (host_inputs == nullptr || out == nullptr) return IPA_ERR_NULL;
+  size_t offs[13];
+  const size_t in_bytes = ipa_attn_host_packed_layout(p, offs);
+  if (in_bytes == 0) return IPA_ERR_SHAPE;
+  if (host_bytes < in_bytes) return IPA_ERR_SHAPE;
+  const int64_t B = p->B, L = p->L, H = p->H, C = p->C, Pq = p->Pq, Pv = p->Pv, R = p->R, Cz = p->Cz;
+  // the 13 inputs, dense, in argument order (the layout ipa_attn_host_packed_layout describes)
+  struct Shape {
+    int nd;
+    int64_t s[5];
+    int32_t dt;
+  };
+  const Shape shp[13] = {{4, {B, L, H, C}, IPA_DTYPE_F32},      {4, {B, L, H, C}, IPA_DTYPE_F32},
+                         {4, {B, L, H, C}, IPA_DTYPE_F32},      {5, {B, L, H, Pq, 3}, IPA_DTYPE_F32},
+                         {5, {B, L, H, Pq, 3}, IPA_DTYPE_F32},  {5, {B, L, H, Pv, 3}, IPA_DTYPE_F32},
+                         {4, {B, L, 3, 3}, IPA_DTYPE_F32},      {3, {B, L, 3}, IPA_DTYPE_F32},
+                         {4, {B, L, R, Cz}, IPA_DTYPE_F32},     {4, {B, L, R, Cz}, IPA_DTYPE_F32},
+                         {2, {Cz, H}, IPA_DTYPE_F32},           {1, {H}, IPA_DTYPE_F32},
+                         {2, {B, L}, IPA_DTYPE_BOOL}};
+  ipa_tensor_t host[13];
+  const ipa_tensor_t* hin[13];
+  for (int t = 0; t < 13; ++t) {
+    ipa_tensor_t& d = host[t];
+    d = ipa_tensor_t{};
+    d.data = static_cast<const unsigned char*>(host_inputs) + offs[t];
+    d.dtype = shp[t].dt;
+    d.ndim = shp[t].nd;
+    int64_t st = 1;
+    for (int k = shp[t].nd - 1; k >= 0; --k) {
+      d.size[k] = shp[t].s[k];
+      d.stride[k] = st;
+      st *= shp[t].s[k];
+    }
+    hin[t] = &host[t];
+  }
+  return host_call(p, hin, out, staging, staging_bytes, workspace, workspace_bytes, stream, dev_err, in_bytes);
 }
 
 ipa_status_t ipa_attn_fwd_train(const ipa_params_t* p, const ipa_tensor_t* q, const ipa_tensor_t* k,

@@ -363,7 +363,10 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     nk = fmaf(gk[e], gk[e], nk);
     nq = fmaf(gq[e], gq[e], nq);
   }
-  float vmax = 0.f;   // largest |value| written (NaN if any value is NaN)
+  // largest fp16 exponent field written, per half-word lane: a value that
+  // does not survive the rounding (|x| >= 65520 -> inf, or NaN) has all
+  // exponent bits set
+  uint32_t emax = 0u;
   auto store_row = [&](uint4* dst, auto value_of) {
 #pragma unroll
     for (int u = 0; u < DH / 8; ++u) {
@@ -371,8 +374,9 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float x0 = value_of(8 * u + 2 * e), x1 = value_of(8 * u + 2 * e + 1);
-        vmax = fmax_nan(vmax, fmax_nan(fabsf(x0), fabsf(x1)));
-        w[e] = valid ? pack_half2(x0, x1) : 0u;
+        const uint32_t pk = pack_half2(x0, x1);
+        emax = __vmaxu2(emax, pk & 0x7c007c00u);
+        w[e] = valid ? pk : 0u;
       }
       dst[u] = make_uint4(w[0], w[1], w[2], w[3]);
     }
@@ -423,7 +427,7 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   sterm[slot] = make_float4(sq[0], sq[1], sq[2], c * nq);
   sterm[H * rb + slot] = make_float4(2.f * c * sk[0], 2.f * c * sk[1], 2.f * c * sk[2], valid ? 0.f : -INFINITY);
   // |x| >= 65520 (or NaN) does not survive the fp16 rounding
-  if (valid && !(vmax < 65520.f)) record_error(a.err, DEV_NONFINITE);
+  if (valid && ((emax & 0xffffu) == 0x7c00u || (emax >> 16) == 0x7c00u)) record_error(a.err, DEV_NONFINITE);
   }
   __syncthreads();
   // each head plane's run of nrow rows, 16-byte stores, consecutive threads on

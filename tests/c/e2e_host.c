@@ -2,12 +2,15 @@
  * allocates page-locked host inputs and outputs, and device staging and
  * workspace for two in-flight calls, then times `calls` calls of
  * ipa_attn_fwd_host (copies up, prologue and core kernels, copy back, all
- * enqueued by the library) alternating over two streams, with CUDA events.
- * It also checks that one call's host result equals, bit for bit, what
+ * enqueued by the library) alternating over two streams, with CUDA events,
+ * and the same number of ipa_attn_fwd_host_packed calls (the inputs in one
+ * page-locked buffer at the offsets ipa_attn_host_packed_layout gives).
+ * It also checks that both host results equal, bit for bit, what
  * ipa_attn_fwd gives on the same inputs copied to the device by hand.
  *
  * Usage: e2e_host L [calls]   (B = 1, H = 12, C = 16, Pq = 4, Pv = 8, R = 2,
- * Cz = 128).  Prints "e2e ok ms_per_call=<t> h2d_bytes=<n> d2h_bytes=<n>". */
+ * Cz = 128).  Prints "e2e ok ms_per_call=<t> packed_ms_per_call=<t>
+ * h2d_bytes=<n> d2h_bytes=<n>". */
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdio.h>
@@ -70,8 +73,10 @@ int main(int argc, char** argv) {
   int32_t herr[3];
   cudaStream_t st[2];
   cudaEvent_t e0, e1;
-  float ms = 0.f;
+  float ms = 0.f, ms_packed = 0.f;
   ipa_status_t s;
+  size_t offs[13], packed_bytes;
+  unsigned char* packed;
 
   p.B = B; p.L = L; p.H = H; p.C = C; p.Pq = Pq; p.Pv = Pv; p.R = R; p.Cz = Cz;
   p.w_L = (float)sqrt(1.0 / 3.0);
@@ -136,32 +141,54 @@ int main(int argc, char** argv) {
     if (memcmp(host[13], hout2, bytes[13]) != 0) { fprintf(stderr, "host result differs\n"); return 1; }
   }
 
-  /* timed: `calls` calls alternating over the two streams */
+  /* the packed layout: the same inputs in one page-locked buffer */
+  packed_bytes = ipa_attn_host_packed_layout(&p, offs);
+  if (packed_bytes == 0) { fprintf(stderr, "packed layout rejected\n"); return 1; }
+  CK(cudaMallocHost((void**)&packed, packed_bytes));
+  memset(packed, 0, packed_bytes);
+  for (t = 0; t < 13; ++t) memcpy(packed + offs[t], host[t], bytes[t]);
+  for (slot = 0; slot < 2; ++slot) {
+    memset(host[13], 0, bytes[13]);
+    s = ipa_attn_fwd_host_packed(&p, packed, packed_bytes, &th[13], stg[slot], stg_bytes, ws[slot], ws_bytes,
+                                 st[slot], err + slot);
+    if (s != IPA_OK) { fprintf(stderr, "ipa_attn_fwd_host_packed: %s\n", ipa_status_string(s)); return 1; }
+    CK(cudaStreamSynchronize(st[slot]));
+    if (memcmp(host[13], hout2, bytes[13]) != 0) { fprintf(stderr, "packed host result differs\n"); return 1; }
+  }
+
+  /* timed: `calls` calls alternating over the two streams, per-input
+   * uploads first, then the packed layout */
   CK(cudaEventCreate(&e0));
   CK(cudaEventCreate(&e1));
-  CK(cudaDeviceSynchronize());
-  CK(cudaEventRecord(e0, st[0]));
-  CK(cudaStreamWaitEvent(st[1], e0, 0));
-  for (i = 0; i < calls; ++i) {
-    slot = i & 1;
-    s = ipa_attn_fwd_host(&p, &th[0], &th[1], &th[2], &th[3], &th[4], &th[5], &th[6], &th[7], &th[8], &th[9],
-                          &th[10], &th[11], &th[12], &th[13], stg[slot], stg_bytes, ws[slot], ws_bytes, st[slot],
-                          err + slot);
-    if (s != IPA_OK) { fprintf(stderr, "ipa_attn_fwd_host: %s\n", ipa_status_string(s)); return 1; }
+  for (d = 0; d < 2; ++d) {
+    CK(cudaDeviceSynchronize());
+    CK(cudaEventRecord(e0, st[0]));
+    CK(cudaStreamWaitEvent(st[1], e0, 0));
+    for (i = 0; i < calls; ++i) {
+      slot = i & 1;
+      if (d == 0)
+        s = ipa_attn_fwd_host(&p, &th[0], &th[1], &th[2], &th[3], &th[4], &th[5], &th[6], &th[7], &th[8], &th[9],
+                              &th[10], &th[11], &th[12], &th[13], stg[slot], stg_bytes, ws[slot], ws_bytes, st[slot],
+                              err + slot);
+      else
+        s = ipa_attn_fwd_host_packed(&p, packed, packed_bytes, &th[13], stg[slot], stg_bytes, ws[slot], ws_bytes,
+                                     st[slot], err + slot);
+      if (s != IPA_OK) { fprintf(stderr, "host call: %s\n", ipa_status_string(s)); return 1; }
+    }
+    {
+      cudaEvent_t done;
+      CK(cudaEventCreate(&done));
+      CK(cudaEventRecord(done, st[1]));
+      CK(cudaStreamWaitEvent(st[0], done, 0));
+      CK(cudaEventRecord(e1, st[0]));
+      CK(cudaEventSynchronize(e1));
+      CK(cudaEventDestroy(done));
+    }
+    CK(cudaEventElapsedTime(d == 0 ? &ms : &ms_packed, e0, e1));
   }
-  {
-    cudaEvent_t done;
-    CK(cudaEventCreate(&done));
-    CK(cudaEventRecord(done, st[1]));
-    CK(cudaStreamWaitEvent(st[0], done, 0));
-    CK(cudaEventRecord(e1, st[0]));
-    CK(cudaEventSynchronize(e1));
-    CK(cudaEventDestroy(done));
-  }
-  CK(cudaEventElapsedTime(&ms, e0, e1));
   CK(cudaMemcpy(herr, err, sizeof herr, cudaMemcpyDeviceToHost));
   if (herr[0] || herr[1] || herr[2]) { fprintf(stderr, "device error %d %d %d\n", herr[0], herr[1], herr[2]); return 1; }
-  printf("e2e ok ms_per_call=%.4f h2d_bytes=%lu d2h_bytes=%lu\n", ms / (float)calls, (unsigned long)h2d,
-         (unsigned long)bytes[13]);
+  printf("e2e ok ms_per_call=%.4f packed_ms_per_call=%.4f h2d_bytes=%lu d2h_bytes=%lu\n", ms / (float)calls,
+         ms_packed / (float)calls, (unsigned long)h2d, (unsigned long)bytes[13]);
   return 0;
 }

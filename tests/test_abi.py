@@ -488,3 +488,51 @@ def test_ipa_fwd_train_rejects_bad_outputs_before_launch(case, expect):
                                 ctypes.byref(uagg), ctypes.c_void_p(FAKE), ctypes.c_size_t(ws), None,
                                 ctypes.c_void_p(FAKE))
     assert st == expect
+
+
+def test_packed_host_layout_matches_the_staging_order():
+    # inputs in argument order, each at a multiple of 256 bytes, sized as the
+    # dense fp32 (mask: one byte) tensors; the staging area holds them at the
+    # same offsets, plus the result
+    lib = api.library()
+    p, ds = ipa_args(B=2, L=100, H=3, Cz=32)
+    offs = (ctypes.c_size_t * 13)()
+    n = lib.ipa_attn_host_packed_layout(ctypes.byref(p), ctypes.byref(offs))
+    sizes = []
+    for k in ORDER[:13]:
+        cnt = 1
+        for d in range(ds[k].ndim):
+            cnt *= ds[k].size[d]
+        sizes.append(cnt * (1 if k == "mask" else 4))
+    o = list(offs)
+    assert o[0] == 0 and all(x % 256 == 0 for x in o)
+    for t in range(12):
+        assert o[t + 1] == o[t] + (sizes[t] + 255) // 256 * 256
+    assert n == o[12] + (sizes[12] + 255) // 256 * 256
+    assert n < lib.ipa_attn_host_staging_size(ctypes.byref(p))
+    bad = api.ipa_params(1, 64, 4, 32, 4, 8, 2, 16)          # C outside the envelope
+    assert lib.ipa_attn_host_packed_layout(ctypes.byref(bad), ctypes.byref(offs)) == 0
+    assert lib.ipa_attn_host_packed_layout(ctypes.byref(p), None) == 0
+
+
+@pytest.mark.parametrize("case,expect", [("null_inputs", 1), ("short_buffer", 2), ("null_out", 1),
+                                         ("out_shape", 2)])
+def test_packed_host_call_rejects_bad_arguments_before_launch(case, expect):
+    lib = api.library()
+    p, ds = ipa_args()
+    offs = (ctypes.c_size_t * 13)()
+    n = lib.ipa_attn_host_packed_layout(ctypes.byref(p), ctypes.byref(offs))
+    host, nbytes, out = ctypes.c_void_p(FAKE), n, ds["out"]
+    if case == "null_inputs":
+        host = None
+    elif case == "short_buffer":
+        nbytes = n - 1
+    elif case == "out_shape":
+        out = desc((1, 64, 4, 7))
+    outp = None if case == "null_out" else ctypes.byref(out)
+    ws = lib.ipa_attn_workspace_size(ctypes.byref(p))
+    sz = lib.ipa_attn_host_staging_size(ctypes.byref(p))
+    st = lib.ipa_attn_fwd_host_packed(ctypes.byref(p), host, ctypes.c_size_t(nbytes), outp, ctypes.c_void_p(FAKE),
+                                      ctypes.c_size_t(sz), ctypes.c_void_p(FAKE), ctypes.c_size_t(ws), None,
+                                      ctypes.c_void_p(FAKE))
+    assert st == expect

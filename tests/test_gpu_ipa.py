@@ -188,6 +188,27 @@ def test_host_buffer_entry_matches_device_path_and_reuses_staging(cuda_device):
         assert np.array_equal(out_host.numpy(), ref)
 
 
+def test_packed_host_call_matches_the_per_input_host_call(cuda_device):
+    # ipa_attn_fwd_host_packed (one upload of the packed inputs) against
+    # ipa_attn_fwd_host (one upload per input) on the same slot: the same
+    # bytes reach the same staging offsets, so the results are identical;
+    # a second input set through the same slot must not see the first's
+    hc = api.IpaHostCalls(1, 300, 4, 16, 4, 8, 2, 64, slots=1, device="cuda")
+    buf = None
+    for seed in (13, 14):
+        inp = ipa_inputs(IpaDims(B=1, L=300, H=4, Cz=64), seed)
+        host = {k: torch.from_numpy(inp[k]).pin_memory() for k in api.IPA_INPUTS}
+        buf = hc.pack(host, buf)
+        a = torch.empty((1, 300, 4, hc.F), dtype=torch.float32, pin_memory=True)
+        b = torch.empty_like(a).pin_memory()
+        hc.call(host, a, 0)
+        hc.call_packed(buf, b, 0)
+        hc.streams[0].synchronize()
+        hc.check()
+        assert torch.equal(a, b)
+        assert np.array_equal(b.numpy(), run_gpu(inp))
+
+
 def test_host_pipeline_matches_device_path_per_call(cuda_device):
     # several calls with different inputs through the overlapped host
     # pipeline: every result equals that call's device-path result
