@@ -301,12 +301,22 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_ro
       }
     named_bar_sync(gbar, BW_ROWS);
   };
+  // bit k: key j0 + k allowed by the pair mask (a dense, 16-byte aligned
+  // row of 32 bytes is read as two 16-byte words)
   auto chunk_mask = [&](int j0) -> uint32_t {
     uint32_t allowed = 0xffffffffu;
     if (pmrow) {
       allowed = 0u;
       const unsigned char* pr = pmrow + static_cast<int64_t>(j0) * a.pms[3];
-      for (int k = 0; k < BW_CHUNK && j0 + k < N; ++k) allowed |= pr[k * a.pms[3]] ? (1u << k) : 0u;
+      if (a.pms[3] == 1 && j0 + BW_CHUNK <= N && (reinterpret_cast<uintptr_t>(pr) & 15u) == 0) {
+        const uint4 u0 = *reinterpret_cast<const uint4*>(pr);
+        const uint4 u1 = *reinterpret_cast<const uint4*>(pr + 16);
+        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int k = 0; k < BW_CHUNK; ++k) allowed |= ((w[k >> 2] >> (8 * (k & 3))) & 0xffu) ? (1u << k) : 0u;
+      } else {
+        for (int k = 0; k < BW_CHUNK && j0 + k < N; ++k) allowed |= pr[k * a.pms[3]] ? (1u << k) : 0u;
+      }
     }
     return allowed;
   };
@@ -443,12 +453,21 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_co
     }
     named_bar_sync(gbar, BW_ROWS);
     if (!active) continue;
+    // bit k: query i0 + k allowed with this key by the pair mask (the 32
+    // bytes down this key's column loaded together)
+    uint32_t allowed = 0xffffffffu;
+    if (pmcol) {
+      allowed = 0u;
+#pragma unroll
+      for (int k = 0; k < BW_CHUNK; ++k)
+        if (i0 + k < N && pmcol[static_cast<int64_t>(i0 + k) * a.pms[2]]) allowed |= 1u << k;
+    }
     for (int k = 0; k < BW_CHUNK; ++k) {
       const float* qq = stg + k * SW;
       const float4 info = *reinterpret_cast<const float4*>(qq);
       if (info.y == 0.f) continue;                 // query without an allowed key
       const int i = i0 + k;
-      if (pmcol && !pmcol[static_cast<int64_t>(i) * a.pms[2]]) continue;
+      if (!((allowed >> k) & 1u)) continue;
       const float4 q0 = *reinterpret_cast<const float4*>(qq + 4), q1 = *reinterpret_cast<const float4*>(qq + 8);
       const GeoPair g = geo_pair(q0, q1, k0, k1, sc.x, sc.y);
       const float p = ex2(g.s - info.x) * info.y;
