@@ -45,7 +45,9 @@ typedef enum {
   IPA_ERR_WORKSPACE = 5,    /* workspace too small or not 256-byte aligned      */
   IPA_ERR_UNSUPPORTED = 6,  /* dims outside the supported envelope (below)      */
   IPA_ERR_CUDA = 7,         /* a CUDA runtime call failed (launch, attribute)   */
-  IPA_ERR_TIMEOUT = 8       /* device: a bounded wait ran out (in dev_err only) */
+  IPA_ERR_TIMEOUT = 8,      /* device: a bounded wait ran out (in dev_err only) */
+  IPA_ERR_BOUNDS = 9        /* device, bounds-checked build only: a store index
+                               left its buffer (in dev_err only)                */
 } ipa_status_t;
 
 /* Element type codes. */
@@ -351,7 +353,8 @@ IPA_API ipa_status_t geo_attn_bwd(const geo_params_t* p,
                           const ipa_tensor_t* frame_mask, const ipa_tensor_t* pair_mask,
                           const ipa_tensor_t* g_output, const ipa_tensor_t* g_attention,
                           const ipa_tensor_t* g_vectors, const geo_grads_t* grads,
-                          void* workspace, size_t workspace_bytes, void* stream);
+                          void* workspace, size_t workspace_bytes, void* stream,
+                          int32_t* dev_err);
 
 /* --------------------------------------------------------------------------
  * geo_attn_fwd without a workspace argument (no counterpart on the pages:
@@ -540,7 +543,18 @@ IPA_API ipa_status_t ipa_module_fwd(const ipa_module_params_t* p, const ipa_tens
 IPA_API const char* ipa_status_string(ipa_status_t s);
 
 /* Translate a device error word written by the kernels into a status:
- * 0 -> IPA_OK, bounded-wait expiry -> IPA_ERR_TIMEOUT, else IPA_ERR_CUDA. */
+ * 0 -> IPA_OK, bounded-wait expiry -> IPA_ERR_TIMEOUT, a word with bit 16
+ * set -> IPA_ERR_BOUNDS, else IPA_ERR_CUDA.
+ *
+ * Bounds-checked build (the library compiled with -DIPA_BOUNDS_CHECK; its
+ * ipa_version() ends in "bounds-checked"): every kernel forms each pointer it
+ * stores through to global memory from a span [index, index + n) checked
+ * against the extent of the destination buffer (from the call's shapes).  A
+ * span outside its buffer writes 0x10000 | (source file tag << 12) | source
+ * line into dev_err (first error wins) and the stores go to a scratch area
+ * inside the library instead.  ipa_frames_from_backbone and ipa_knn_distogram
+ * have no error word: their spans are checked and redirected, not reported.
+ * The product build has none of these checks. */
 IPA_API ipa_status_t ipa_device_error_status(int32_t dev_err_value);
 
 /* Library build identifier, e.g. "flashipa_b200 sm_100a". */

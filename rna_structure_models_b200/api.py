@@ -138,7 +138,7 @@ def library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.geo_attn_bwd_workspace_size.argtypes = [P(GeoParams)]
     lib.geo_attn_bwd_workspace_size.restype = ctypes.c_size_t
     lib.geo_attn_bwd.argtypes = [P(GeoParams)] + [T] * 16 + [P(GeoGrads), ctypes.c_void_p, ctypes.c_size_t,
-                                                             ctypes.c_void_p]
+                                                             ctypes.c_void_p, ctypes.c_void_p]
     lib.geo_attn_bwd.restype = ctypes.c_int
     lib.ipa_linear_workspace_size.argtypes = [ctypes.c_int32] * 3
     lib.ipa_linear_workspace_size.restype = ctypes.c_size_t
@@ -636,6 +636,7 @@ class GeoGradPlan:
         if nbytes == 0:
             raise IpaError(6, "dimensions outside the supported envelope")
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
 
     def __call__(self, inp: dict, g_output, g_attention=None, g_vectors=None, *, out: Optional[dict] = None,
                  stream=None):
@@ -654,20 +655,31 @@ class GeoGradPlan:
         st = library().geo_attn_bwd(ctypes.byref(p), *[ctypes.byref(d) for d in descs], ctypes.byref(grads),
                                     ctypes.c_void_p(self.workspace.data_ptr()),
                                     ctypes.c_size_t(self.workspace.numel()),
-                                    ctypes.c_void_p(_stream_ptr(stream)))
+                                    ctypes.c_void_p(_stream_ptr(stream)),
+                                    ctypes.c_void_p(self.dev_err.data_ptr()))
         if st != 0:
             raise IpaError(st, library().ipa_status_string(st).decode())
         return out
 
+    def check(self):
+        v = int(self.dev_err.item())
+        if v != 0:
+            self.dev_err.zero_()
+            raise IpaError(int(library().ipa_device_error_status(v)), f"device error code {v}")
 
-def geo_attn_backward(inp: dict, g_output, g_attention=None, g_vectors=None, *, stream=None) -> dict:
+
+def geo_attn_backward(inp: dict, g_output, g_attention=None, g_vectors=None, *, stream=None,
+                      check: bool = True) -> dict:
     """Gradients of sum(g_output * output) + sum(g_attention * attention)
     + sum(g_vectors * vectors) with respect to every floating input (fp32)."""
     B, N, H, _ = inp["q_direction"].shape
     M = inp["values"].shape[3]
     Cout = inp["output_weight"].shape[1]
     plan = GeoGradPlan(B, N, H, M, Cout, device=inp["q_direction"].device)
-    return plan(inp, g_output, g_attention, g_vectors, stream=stream)
+    res = plan(inp, g_output, g_attention, g_vectors, stream=stream)
+    if check:
+        plan.check()
+    return res
 
 
 # ------------------------------------------------------------------ MEET

@@ -174,6 +174,7 @@ const char* ipa_status_string(ipa_status_t s) {
     case IPA_ERR_UNSUPPORTED: return "dimensions outside the supported envelope";
     case IPA_ERR_CUDA: return "CUDA runtime error";
     case IPA_ERR_TIMEOUT: return "device wait timed out";
+    case IPA_ERR_BOUNDS: return "device store index outside its buffer (bounds-checked build)";
   }
   return "unknown status";
 }
@@ -181,10 +182,15 @@ const char* ipa_status_string(ipa_status_t s) {
 ipa_status_t ipa_device_error_status(int32_t v) {
   if (v == 0) return IPA_OK;
   if (v >= 1 && v <= 5) return IPA_ERR_TIMEOUT;
+  if (v & 0x10000) return IPA_ERR_BOUNDS;
   return IPA_ERR_CUDA;
 }
 
+#ifdef IPA_BOUNDS_CHECK
+const char* ipa_version(void) { return "flashipa_b200 sm_100a 0.1 bounds-checked"; }
+#else
 const char* ipa_version(void) { return "flashipa_b200 sm_100a 0.1"; }
+#endif
 
 size_t ipa_attn_workspace_size(const ipa_params_t* p) {
   ipa_status_t st;
@@ -642,10 +648,11 @@ ipa_status_t meet_attn_fwd(const meet_params_t* p, const ipa_tensor_t* q, const 
     a.err = reinterpret_cast<int*>(a.ws + a.lay.err);
     if (cudaMemsetAsync(a.err, 0, sizeof(int), cs) != cudaSuccess) return IPA_ERR_CUDA;
   }
+  m.err = a.err;
   if (meet_launch_prep(m, cs) != cudaSuccess) return IPA_ERR_CUDA;
   if (ipa_launch_prologue(a, cs) != cudaSuccess) return IPA_ERR_CUDA;
   if (ipa_launch_core(a, cs) != cudaSuccess) return IPA_ERR_CUDA;
-  if (meet_launch_extract(a.out, static_cast<float*>(const_cast<void*>(out->data)), B * L * H, cs) != cudaSuccess)
+  if (meet_launch_extract(a.out, static_cast<float*>(const_cast<void*>(out->data)), B * L * H, a.err, cs) != cudaSuccess)
     return IPA_ERR_CUDA;
   return IPA_OK;
 }
@@ -971,7 +978,7 @@ ipa_status_t geo_attn_bwd(const geo_params_t* p, const ipa_tensor_t* q_direction
                           const ipa_tensor_t* frame_mask, const ipa_tensor_t* pair_mask,
                           const ipa_tensor_t* g_output, const ipa_tensor_t* g_attention,
                           const ipa_tensor_t* g_vectors, const geo_grads_t* grads, void* workspace,
-                          size_t workspace_bytes, void* stream) {
+                          size_t workspace_bytes, void* stream, int32_t* dev_err) {
   GeoBwdLaunch a{};
   int fdt = 0;
   ipa_status_t st = geo_inputs(p, q_direction, k_direction, q_point, k_point, values, direction_scale,
@@ -1027,7 +1034,12 @@ ipa_status_t geo_attn_bwd(const geo_params_t* p, const ipa_tensor_t* q_direction
   a.lay = lay;
   a.f.ws = a.ws;
   a.f.lay = lay.fwd;
-  a.f.err = reinterpret_cast<int*>(a.ws + lay.fwd.err);
+  if (dev_err != nullptr) {
+    a.f.err = dev_err;
+  } else {
+    a.f.err = reinterpret_cast<int*>(a.ws + lay.fwd.err);
+    if (cudaMemsetAsync(a.f.err, 0, sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess) return IPA_ERR_CUDA;
+  }
   if (geo_launch_bwd(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return IPA_ERR_CUDA;
   return IPA_OK;
 }

@@ -17,7 +17,10 @@
 
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
+
+#define IPA_FILE_TAG 12
 
 namespace fipa {
 
@@ -37,9 +40,10 @@ __global__ void __launch_bounds__(256) knn_distogram_kernel(const DistogramArgs 
   const int64_t xb = b * a.x.s[0], mbase = b * a.mask.s[0];
   auto X = [&](int r, int c) { return xp[xb + r * a.x.s[1] + c * a.x.s[2]]; };
   auto valid_at = [&](int r) { return mp[mbase + r * a.mask.s[1]] != 0; };
-  int32_t* idx = a.idx + wid * a.k;
-  int32_t* bins = a.bins + wid * a.k;
-  float* hist = a.hist + wid * a.nb;
+  const int64_t nres = static_cast<int64_t>(a.B) * a.L;
+  int32_t* idx = IPA_SPAN(a.idx, wid * a.k, a.k, nres * a.k, a.err);
+  int32_t* bins = IPA_SPAN(a.bins, wid * a.k, a.k, nres * a.k, a.err);
+  float* hist = IPA_SPAN(a.hist, wid * a.nb, a.nb, nres * a.nb, a.err);
   const bool valid = valid_at(i);
 
   uint64_t keys[KM];

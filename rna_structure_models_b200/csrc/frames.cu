@@ -5,7 +5,10 @@
 //   e3 = e1 x e2,  R = [e1 | e2 | e3] (columns),  t = CA.
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
+
+#define IPA_FILE_TAG 9
 
 namespace fipa {
 
@@ -37,14 +40,15 @@ __global__ void __launch_bounds__(256) frames_kernel(const FramesArgs a) {
   const float r2 = rsqrtf(fmaf(u2[0], u2[0], fmaf(u2[1], u2[1], u2[2] * u2[2])));
   float e2[3] = {u2[0] * r2, u2[1] * r2, u2[2] * r2};
   float e3[3] = {e1[1] * e2[2] - e1[2] * e2[1], e1[2] * e2[0] - e1[0] * e2[2], e1[0] * e2[1] - e1[1] * e2[0]};
-  float* R = a.rot + t * 9;
+  const int64_t n_res = static_cast<int64_t>(a.B) * a.L;
+  float* R = IPA_SPAN(a.rot, t * 9, 9, n_res * 9, a.err);
 #pragma unroll
   for (int x = 0; x < 3; ++x) {   // row x of R: (e1_x, e2_x, e3_x)
     R[3 * x] = e1[x];
     R[3 * x + 1] = e2[x];
     R[3 * x + 2] = e3[x];
   }
-  float* tr = a.trans + t * 3;
+  float* tr = IPA_SPAN(a.trans, t * 3, 3, n_res * 3, a.err);
   tr[0] = ca[0];
   tr[1] = ca[1];
   tr[2] = ca[2];

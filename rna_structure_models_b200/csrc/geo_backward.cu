@@ -32,9 +32,12 @@
 #include <cmath>
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "geo_common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+
+#define IPA_FILE_TAG 6
 
 namespace fipa {
 
@@ -56,6 +59,7 @@ struct GvecArgs {
   const float* wt;             // [Cout, HM3]
   float* gvec;                 // [B*N, HM3]
   unsigned char* rowlive;      // [B*N]
+  int* err;
 };
 
 // g_vec = g_vectors + [row live] g_output W^T.  Block: 32 k-columns x 8 row
@@ -72,7 +76,7 @@ __global__ void __launch_bounds__(256) geo_gvec_kernel(const GvecArgs a) {
     if (row < rows)
       for (int h = 0; h < a.H; ++h) l |= a.live[row * a.H + h] != 0;
     lv[q] = l;
-    if (blockIdx.y == 0 && threadIdx.x == 0 && row < rows) a.rowlive[row] = l ? 1 : 0;
+    if (blockIdx.y == 0 && threadIdx.x == 0 && row < rows) *IPA_AT(a.rowlive, row, rows, a.err) = l ? 1 : 0;
   }
   if (kx >= a.HM3) return;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -104,7 +108,7 @@ __global__ void __launch_bounds__(256) geo_gvec_kernel(const GvecArgs a) {
       const View& v = a.g_vectors;
       g += ldf(v, b * v.s[0] + n * v.s[1] + h * v.s[2] + m * v.s[3] + x * v.s[4]);
     }
-    a.gvec[row * a.HM3 + kx] = g;
+    *IPA_AT(a.gvec, row * a.HM3 + kx, rows * a.HM3, a.err) = g;
   }
 }
 
@@ -115,6 +119,7 @@ struct DaggArgs {
   const float* agg;    // [B*H, N, VW]
   float* dagg;         // [B*H, N, VW]
   float4* rowinfo;     // [B*H, N]: .z <- <dagg, agg>
+  int* err;
 };
 
 __global__ void __launch_bounds__(256) geo_dagg_kernel(const DaggArgs a) {
@@ -127,7 +132,8 @@ __global__ void __launch_bounds__(256) geo_dagg_kernel(const DaggArgs a) {
   const float* g = a.gvec + bn * a.HM3 + h * 3 * a.M;
   const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.N + n;
   const float* ag = a.agg + row * a.VW;
-  float* dst = a.dagg + row * a.VW;
+  const int64_t nbhn = static_cast<int64_t>(a.B) * a.N * a.H;
+  float* dst = IPA_SPAN(a.dagg, row * a.VW, 3 * a.M, nbhn * a.VW, a.err);
   float d1 = 0.f;
   for (int m = 0; m < a.M; ++m) {
 #pragma unroll
@@ -137,7 +143,7 @@ __global__ void __launch_bounds__(256) geo_dagg_kernel(const DaggArgs a) {
       d1 = fmaf(v, ag[3 * m + x], d1);
     }
   }
-  a.rowinfo[row] = make_float4(0.f, 0.f, d1, 0.f);
+  *IPA_AT(a.rowinfo, row, nbhn, a.err) = make_float4(0.f, 0.f, d1, 0.f);
 }
 
 constexpr int DW_ROWS = 128, DW_K = 32;
@@ -152,6 +158,7 @@ struct DwArgs {
   float* part_b;                   // [nchunk, Cout]
   float* d_w;                      // [HM3, Cout]
   float* d_b;                      // [Cout] or null
+  int* err;
 };
 
 // Partial dW over one chunk of 128 rows: a thread owns one output column c
@@ -189,11 +196,13 @@ __global__ void __launch_bounds__(256) geo_dw_part_kernel(const DwArgs a) {
 #pragma unroll
     for (int kk = 0; kk < DW_K; ++kk) acc[kk] = fmaf(vs[rr][kk], g, acc[kk]);
   }
-  float* pw = a.part_w + static_cast<int64_t>(blockIdx.z) * a.HM3 * a.Cout;
+  const int64_t nwc = static_cast<int64_t>(a.HM3) * a.Cout;
+  const int64_t pw0 = static_cast<int64_t>(blockIdx.z) * nwc;
 #pragma unroll
   for (int kk = 0; kk < DW_K; ++kk)
-    if (k0 + kk < a.HM3) pw[static_cast<int64_t>(k0 + kk) * a.Cout + c] = acc[kk];
-  if (blockIdx.y == 0) a.part_b[static_cast<int64_t>(blockIdx.z) * a.Cout + c] = accb;
+    if (k0 + kk < a.HM3) *IPA_AT(a.part_w, pw0 + static_cast<int64_t>(k0 + kk) * a.Cout + c, a.nchunk * nwc, a.err) = acc[kk];
+  if (blockIdx.y == 0)
+    *IPA_AT(a.part_b, static_cast<int64_t>(blockIdx.z) * a.Cout + c, static_cast<int64_t>(a.nchunk) * a.Cout, a.err) = accb;
 }
 
 // dW and db: the chunk partials summed in a fixed order (deterministic).
@@ -203,12 +212,12 @@ __global__ void __launch_bounds__(256) geo_dw_sum_kernel(const DwArgs a) {
   if (t < nw) {
     float s = 0.f;
     for (int z = 0; z < a.nchunk; ++z) s += a.part_w[z * nw + t];
-    a.d_w[t] = s;
+    *IPA_AT(a.d_w, t, nw, a.err) = s;
   }
   if (t < a.Cout && a.d_b) {
     float s = 0.f;
     for (int z = 0; z < a.nchunk; ++z) s += a.part_b[static_cast<int64_t>(z) * a.Cout + t];
-    a.d_b[t] = s;
+    *IPA_AT(a.d_b, t, a.Cout, a.err) = s;
   }
 }
 
@@ -229,6 +238,7 @@ struct PairArgs {
   float4* dk;            // [B*H, N, 2]
   float* dvr;            // [B*H, N, VW]
   float* acc;            // [B, H, row blocks, 4 warps, 2]: per-warp sums of ds <qd, kd> and ds |qp - kp|
+  int* err;
 };
 
 __device__ __forceinline__ float g_att_at(const PairArgs& a, int b, int h, int i, int j) {
@@ -387,9 +397,11 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_ro
   }
   const float Ar = sc.x / kLog2e, Br = sc.y / kLog2e;   // A / sqrt3, B / sqrt3
   if (in_range) {
-    a.dq[2 * (bh * N + i)] = make_float4(Ar * t[0], Ar * t[1], Ar * t[2], 0.f);
-    a.dq[2 * (bh * N + i) + 1] = make_float4(-Br * t[3], -Br * t[4], -Br * t[5], 0.f);
-    a.rowinfo[bh * N + i] = make_float4(m, inv, D, 0.f);
+    const int64_t nbhn = static_cast<int64_t>(a.B) * a.H * N;
+    float4* dq = IPA_SPAN(a.dq, 2 * (bh * N + i), 2, 2 * nbhn, a.err);
+    dq[0] = make_float4(Ar * t[0], Ar * t[1], Ar * t[2], 0.f);
+    dq[1] = make_float4(-Br * t[3], -Br * t[4], -Br * t[5], 0.f);
+    *IPA_AT(a.rowinfo, bh * N + i, nbhn, a.err) = make_float4(m, inv, D, 0.f);
   }
   // per-head sums over the block's rows (warps 0-3 hold split 0)
   float s6 = t[6], s7 = t[7];
@@ -400,8 +412,9 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_ro
   }
   if ((tid & 31) == 0) {     // one slot per (b, h, row block, warp), summed in a fixed order later
     const int64_t slot = ((bh * gridDim.x + blockIdx.x) * 4 + (tid >> 5)) * 2;
-    a.acc[slot] = s6;
-    a.acc[slot + 1] = s7;
+    float* ap = IPA_SPAN(a.acc, slot, 2, static_cast<int64_t>(a.B) * a.H * gridDim.x * 8, a.err);
+    ap[0] = s6;
+    ap[1] = s7;
   }
 }
 
@@ -506,10 +519,13 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_co
     for (int s2 = 0; s2 < BW_SPLIT; ++s2) t[e] += sm_at(s2, e);
   }
   const float Ar = sc.x / kLog2e, Br = sc.y / kLog2e;
-  a.dk[2 * (bh * N + j)] = make_float4(Ar * t[0], Ar * t[1], Ar * t[2], 0.f);
-  a.dk[2 * (bh * N + j) + 1] = make_float4(Br * t[3], Br * t[4], Br * t[5], 0.f);   // u points from kp to qp
+  const int64_t nbhn = static_cast<int64_t>(a.B) * a.H * N;
+  float4* dk = IPA_SPAN(a.dk, 2 * (bh * N + j), 2, 2 * nbhn, a.err);
+  dk[0] = make_float4(Ar * t[0], Ar * t[1], Ar * t[2], 0.f);
+  dk[1] = make_float4(Br * t[3], Br * t[4], Br * t[5], 0.f);   // u points from kp to qp
+  float* dvr = IPA_SPAN(a.dvr, (bh * N + j) * a.VW, V, nbhn * a.VW, a.err);
 #pragma unroll
-  for (int e = 0; e < V; ++e) a.dvr[(bh * N + j) * a.VW + e] = t[6 + e];
+  for (int e = 0; e < V; ++e) dvr[e] = t[6 + e];
 }
 
 struct FrameArgs {
@@ -524,6 +540,7 @@ struct FrameArgs {
   const float* acc;      // [B, H, nrb, 4, 2] per-warp partial sums (geo_bwd_rows_kernel)
   int nrb;               // row blocks per (b, h)
   float *d_qd, *d_kd, *d_qp, *d_kp, *d_val, *d_rot, *d_trans, *d_dscale, *d_xscale;
+  int* err;
 };
 
 __global__ void __launch_bounds__(128) geo_bwd_frame_kernel(const FrameArgs a) {
@@ -539,8 +556,8 @@ __global__ void __launch_bounds__(128) geo_bwd_frame_kernel(const FrameArgs a) {
           sd += a.acc[slot];
           sx += a.acc[slot + 1];
         }
-      a.d_dscale[h] = static_cast<float>(sd) * kInvSqrt3 / (1.f + expf(-xd));
-      a.d_xscale[h] = -static_cast<float>(sx) * kInvSqrt3 / (1.f + expf(-xx));
+      *IPA_AT(a.d_dscale, h, a.H, a.err) = static_cast<float>(sd) * kInvSqrt3 / (1.f + expf(-xd));
+      *IPA_AT(a.d_xscale, h, a.H, a.err) = -static_cast<float>(sx) * kInvSqrt3 / (1.f + expf(-xx));
     }
   if (t >= static_cast<int64_t>(a.B) * a.N) return;
   const int b = static_cast<int>(t / a.N), n = static_cast<int>(t % a.N);
@@ -566,17 +583,18 @@ __global__ void __launch_bounds__(128) geo_bwd_frame_kernel(const FrameArgs a) {
     const float4 q0 = a.dq[2 * row], q1 = a.dq[2 * row + 1], k0 = a.dk[2 * row], k1 = a.dk[2 * row + 1];
     const float gqd[3] = {q0.x, q0.y, q0.z}, gqp[3] = {q1.x, q1.y, q1.z};
     const float gkd[3] = {k0.x, k0.y, k0.z}, gkp[3] = {k1.x, k1.y, k1.z};
-    back(gqd, a.qd, b * a.qd.s[0] + n * a.qd.s[1] + h * a.qd.s[2], a.qd.s[3], a.d_qd + o3);
-    back(gkd, a.kd, b * a.kd.s[0] + n * a.kd.s[1] + h * a.kd.s[2], a.kd.s[3], a.d_kd + o3);
-    back(gqp, a.qp, b * a.qp.s[0] + n * a.qp.s[1] + h * a.qp.s[2], a.qp.s[3], a.d_qp + o3);
-    back(gkp, a.kp, b * a.kp.s[0] + n * a.kp.s[1] + h * a.kp.s[2], a.kp.s[3], a.d_kp + o3);
+    const int64_t n3 = static_cast<int64_t>(a.B) * a.N * a.H * 3;
+    back(gqd, a.qd, b * a.qd.s[0] + n * a.qd.s[1] + h * a.qd.s[2], a.qd.s[3], IPA_SPAN(a.d_qd, o3, 3, n3, a.err));
+    back(gkd, a.kd, b * a.kd.s[0] + n * a.kd.s[1] + h * a.kd.s[2], a.kd.s[3], IPA_SPAN(a.d_kd, o3, 3, n3, a.err));
+    back(gqp, a.qp, b * a.qp.s[0] + n * a.qp.s[1] + h * a.qp.s[2], a.qp.s[3], IPA_SPAN(a.d_qp, o3, 3, n3, a.err));
+    back(gkp, a.kp, b * a.kp.s[0] + n * a.kp.s[1] + h * a.kp.s[2], a.kp.s[3], IPA_SPAN(a.d_kp, o3, 3, n3, a.err));
 #pragma unroll
     for (int x = 0; x < 3; ++x) dT[x] += gqp[x] + gkp[x];
     for (int m = 0; m < a.M; ++m) {
       const float* dv = a.dvr + row * a.VW + 3 * m;
       const float gv[3] = {dv[0], dv[1], dv[2]};
       back(gv, a.val, b * a.val.s[0] + n * a.val.s[1] + h * a.val.s[2] + m * a.val.s[3], a.val.s[4],
-           a.d_val + (t * a.H + h) * a.VW + 3 * m);
+           IPA_SPAN(a.d_val, (t * a.H + h) * a.VW + 3 * m, 3, static_cast<int64_t>(a.B) * a.N * a.H * a.VW, a.err));
       // vectors = R^T agg: dR += agg g_vec^T
       const float* ag = a.agg + row * a.VW + 3 * m;
       const float* gq = a.gvec + t * a.HM3 + h * a.VW + 3 * m;
@@ -586,23 +604,26 @@ __global__ void __launch_bounds__(128) geo_bwd_frame_kernel(const FrameArgs a) {
         for (int y = 0; y < 3; ++y) dR[3 * x + y] = fmaf(ag[x], gq[y], dR[3 * x + y]);
     }
   }
+  float* drot = IPA_SPAN(a.d_rot, t * 9, 9, static_cast<int64_t>(a.B) * a.N * 9, a.err);
+  float* dtr = IPA_SPAN(a.d_trans, t * 3, 3, static_cast<int64_t>(a.B) * a.N * 3, a.err);
 #pragma unroll
-  for (int e = 0; e < 9; ++e) a.d_rot[t * 9 + e] = dR[e];
+  for (int e = 0; e < 9; ++e) drot[e] = dR[e];
 #pragma unroll
-  for (int x = 0; x < 3; ++x) a.d_trans[t * 3 + x] = dT[x];
+  for (int x = 0; x < 3; ++x) dtr[x] = dT[x];
 }
 
 struct TransposeArgs {
   int HM3, Cout;
   View w;
   float* wt;   // [Cout, HM3]
+  int* err;
 };
 
 __global__ void geo_wt_kernel(const TransposeArgs a) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= static_cast<int64_t>(a.HM3) * a.Cout) return;
   const int c = static_cast<int>(t / a.HM3), k = static_cast<int>(t % a.HM3);
-  a.wt[t] = ldf(a.w, k * a.w.s[0] + c * a.w.s[1]);
+  *IPA_AT(a.wt, t, static_cast<int64_t>(a.HM3) * a.Cout, a.err) = ldf(a.w, k * a.w.s[0] + c * a.w.s[1]);
 }
 
 template <int M>
@@ -673,7 +694,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
 
   {
-    TransposeArgs ta{HM3, Cout, a.f.output_weight, reinterpret_cast<float*>(ws + w.wt)};
+    TransposeArgs ta{HM3, Cout, a.f.output_weight, reinterpret_cast<float*>(ws + w.wt), a.f.err};
     const int64_t n = static_cast<int64_t>(HM3) * Cout;
     geo_wt_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(ta);
   }
@@ -684,6 +705,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   ga.wt = reinterpret_cast<const float*>(ws + w.wt);
   ga.gvec = reinterpret_cast<float*>(ws + w.gvec);
   ga.rowlive = ws + w.rowlive;
+  ga.err = a.f.err;
   geo_gvec_kernel<<<dim3(static_cast<unsigned>((rows + 31) / 32), (HM3 + 31) / 32), dim3(32, 8), 0, st>>>(ga);
 
   DaggArgs da{};
@@ -693,6 +715,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   da.agg = f.out_agg;
   da.dagg = reinterpret_cast<float*>(ws + w.dagg);
   da.rowinfo = reinterpret_cast<float4*>(ws + w.rowinfo);
+  da.err = a.f.err;
   geo_dagg_kernel<<<static_cast<unsigned>((rows * H + 255) / 256), 256, 0, st>>>(da);
 
   DwArgs dw{};
@@ -702,6 +725,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   dw.part_w = reinterpret_cast<float*>(ws + w.dwpart);
   dw.part_b = reinterpret_cast<float*>(ws + w.dbpart);
   dw.d_w = a.d_output_weight; dw.d_b = a.d_output_bias;
+  dw.err = a.f.err;
   geo_dw_part_kernel<<<dim3((Cout + 255) / 256, (HM3 + DW_K - 1) / DW_K, dw.nchunk), 256, 0, st>>>(dw);
   {
     int64_t n = static_cast<int64_t>(HM3) * Cout;
@@ -725,6 +749,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   p.dk = reinterpret_cast<float4*>(ws + w.dk);
   p.dvr = reinterpret_cast<float*>(ws + w.dvr);
   p.acc = reinterpret_cast<float*>(ws + w.acc);
+  p.err = a.f.err;
   switch (M) {
     case 1: e = launch_pairs<1>(p, B, N, H, st); break;
     case 2: e = launch_pairs<2>(p, B, N, H, st); break;
@@ -747,6 +772,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   fa.d_qd = a.d_q_direction; fa.d_kd = a.d_k_direction; fa.d_qp = a.d_q_point; fa.d_kp = a.d_k_point;
   fa.d_val = a.d_values; fa.d_rot = a.d_rotation; fa.d_trans = a.d_translation;
   fa.d_dscale = a.d_direction_scale; fa.d_xscale = a.d_distance_scale;
+  fa.err = a.f.err;
   geo_bwd_frame_kernel<<<static_cast<unsigned>((rows + 127) / 128), 128, 0, st>>>(fa);
   return cudaGetLastError();
 }

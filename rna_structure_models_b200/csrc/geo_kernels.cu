@@ -22,9 +22,12 @@
 #include <cmath>
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "geo_common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+
+#define IPA_FILE_TAG 5
 
 namespace fipa {
 
@@ -44,6 +47,7 @@ struct WArgs {
   float2* sc;   // [H]: (log2e softplus(direction)/sqrt3, log2e softplus(distance)/sqrt3)
   float* wf;    // [HM3, Cout]
   float* bf;    // [Cout]
+  int* err;
 };
 
 __global__ void geo_weights_kernel(const WArgs a) {
@@ -51,12 +55,12 @@ __global__ void geo_weights_kernel(const WArgs a) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t < n) {
     const int r = static_cast<int>(t / a.Cout), c = static_cast<int>(t % a.Cout);
-    a.wf[t] = ldf(a.w, r * a.w.s[0] + c * a.w.s[1]);
+    *IPA_AT(a.wf, t, n, a.err) = ldf(a.w, r * a.w.s[0] + c * a.w.s[1]);
   }
-  if (t < a.Cout) a.bf[t] = a.has_bias ? ldf(a.bias, t * a.bias.s[0]) : 0.f;
+  if (t < a.Cout) *IPA_AT(a.bf, t, a.Cout, a.err) = a.has_bias ? ldf(a.bias, t * a.bias.s[0]) : 0.f;
   if (t < a.H) {
     const float k = kLog2e * 0.57735026918962576f;  // log2(e) / sqrt(3)
-    a.sc[t] = make_float2(k * softplus_stable(ldf(a.dscale, t * a.dscale.s[0])),
+    *IPA_AT(a.sc, t, a.H, a.err) = make_float2(k * softplus_stable(ldf(a.dscale, t * a.dscale.s[0])),
                           k * softplus_stable(ldf(a.xscale, t * a.xscale.s[0])));
   }
 }
@@ -68,6 +72,7 @@ struct PrepArgs {
   float4* kg;   // [B*H, N, 2]: (kd, bias) (kp, 0)
   float* vg;    // [B*H, N, VW]
   float* rotf;  // [B, N, 9]
+  int* err;
 };
 
 __global__ void geo_prep_kernel(const PrepArgs a) {
@@ -99,11 +104,13 @@ __global__ void geo_prep_kernel(const PrepArgs a) {
   rot3(a.qp, b * a.qp.s[0] + n * a.qp.s[1] + h * a.qp.s[2], qp);
   rot3(a.kp, b * a.kp.s[0] + n * a.kp.s[1] + h * a.kp.s[2], kp);
   const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.N + n;
-  a.qg[2 * row] = make_float4(qd[0], qd[1], qd[2], bias);
-  a.qg[2 * row + 1] = make_float4(qp[0] + T[0], qp[1] + T[1], qp[2] + T[2], 0.f);
-  a.kg[2 * row] = make_float4(kd[0], kd[1], kd[2], bias);
-  a.kg[2 * row + 1] = make_float4(kp[0] + T[0], kp[1] + T[1], kp[2] + T[2], 0.f);
-  float* vo = a.vg + row * a.VW;
+  float4* qo = IPA_SPAN(a.qg, 2 * row, 2, 2 * total, a.err);
+  float4* ko = IPA_SPAN(a.kg, 2 * row, 2, 2 * total, a.err);
+  qo[0] = make_float4(qd[0], qd[1], qd[2], bias);
+  qo[1] = make_float4(qp[0] + T[0], qp[1] + T[1], qp[2] + T[2], 0.f);
+  ko[0] = make_float4(kd[0], kd[1], kd[2], bias);
+  ko[1] = make_float4(kp[0] + T[0], kp[1] + T[1], kp[2] + T[2], 0.f);
+  float* vo = IPA_SPAN(a.vg, row * a.VW, a.VW, total * a.VW, a.err);
   for (int m = 0; m < a.M; ++m) {
     float vr[3];
     const int64_t vb = b * a.val.s[0] + n * a.val.s[1] + h * a.val.s[2] + m * a.val.s[3];
@@ -116,7 +123,7 @@ __global__ void geo_prep_kernel(const PrepArgs a) {
   }
   for (int e = 3 * a.M; e < a.VW; ++e) vo[e] = 0.f;
   if (h == 0) {
-    float* rf = a.rotf + (static_cast<int64_t>(b) * a.N + n) * 9;
+    float* rf = IPA_SPAN(a.rotf, (static_cast<int64_t>(b) * a.N + n) * 9, 9, static_cast<int64_t>(a.B) * a.N * 9, a.err);
 #pragma unroll
     for (int e = 0; e < 9; ++e) rf[e] = R[e];
   }
@@ -136,6 +143,7 @@ struct AttnArgs {
   float2* ml;                // [B*H, N]
   unsigned char* live;       // [B, N, H]
   float* agg;                // [B*H, N, VW] aggregated global-frame values, or null
+  int* err;
 };
 
 // Staged chunk of 32 keys (one split group), laid out for packed pairs of
@@ -334,9 +342,10 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, 1) geo_attn_kernel(const
   const bool has = lf > 0.f;
   const float inv = has ? 1.f / lf : 0.f;
   const float* R = a.rotf + (static_cast<int64_t>(b) * N + i) * 9;
-  float* dst = a.out_vectors + ((static_cast<int64_t>(b) * N + i) * a.H + h) * V;
+  const int64_t nbhn = static_cast<int64_t>(a.B) * a.H * N;
+  float* dst = IPA_SPAN(a.out_vectors, ((static_cast<int64_t>(b) * N + i) * a.H + h) * V, V, nbhn * V, a.err);
   if (a.agg) {
-    float* ag = a.agg + (bh * N + i) * a.VW;
+    float* ag = IPA_SPAN(a.agg, (bh * N + i) * a.VW, V, nbhn * a.VW, a.err);
 #pragma unroll
     for (int e = 0; e < V; ++e) ag[e] = has ? af[e] * inv : 0.f;
   }
@@ -347,8 +356,8 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, 1) geo_attn_kernel(const
     for (int x = 0; x < 3; ++x)  // R^T g
       dst[3 * mm + x] = has ? fmaf(R[x], gx, fmaf(R[3 + x], gy, R[6 + x] * gz)) : 0.f;
   }
-  a.ml[bh * N + i] = make_float2(mf, lf);
-  a.live[(static_cast<int64_t>(b) * N + i) * a.H + h] = has ? 1 : 0;
+  *IPA_AT(a.ml, bh * N + i, nbhn, a.err) = make_float2(mf, lf);
+  *IPA_AT(a.live, (static_cast<int64_t>(b) * N + i) * a.H + h, nbhn, a.err) = has ? 1 : 0;
 }
 
 struct MapArgs {
@@ -360,6 +369,7 @@ struct MapArgs {
   const unsigned char* pm;
   int64_t pms[4];
   float* att;   // [B, H, N, N]
+  int* err;
 };
 
 // One block per (16 query rows, head, batch): each thread owns four
@@ -475,7 +485,9 @@ __global__ void __launch_bounds__(256, 3) geo_map_kernel(const MapArgs a) {
         v[2 * u] = ok0 ? ex2(y.x) * st.y : 0.f;
         v[2 * u + 1] = ok1 ? ex2(y.y) * st.y : 0.f;
       }
-      float* dst = a.att + (bh * N + i) * static_cast<int64_t>(N) + j0;
+      const int64_t nw = full ? MAP_KEYS : (N - j0 < MAP_KEYS ? N - j0 : MAP_KEYS);
+      float* dst = IPA_SPAN(a.att, (bh * N + i) * static_cast<int64_t>(N) + j0, nw,
+                            static_cast<int64_t>(a.B) * a.H * N * static_cast<int64_t>(N), a.err);
       if (vec_store && full) {
         *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
       } else {
@@ -494,6 +506,7 @@ struct ReadArgs {
   const float* wf;
   const float* bf;
   float* out;         // [B*N, Cout]
+  int* err;
 };
 
 constexpr int RD_ROWS = 32;
@@ -528,7 +541,7 @@ __global__ void __launch_bounds__(256) geo_readout_kernel(const ReadArgs a) {
 #pragma unroll
   for (int rr = 0; rr < RD_ROWS; ++rr) {
     const int64_t row = row0 + rr;
-    if (row < nrows) a.out[row * a.Cout + col] = any_live[rr] ? acc[rr] + bias : 0.f;
+    if (row < nrows) *IPA_AT(a.out, row * a.Cout + col, nrows * a.Cout, a.err) = any_live[rr] ? acc[rr] + bias : 0.f;
   }
 }
 
@@ -579,6 +592,7 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
   wa.sc = reinterpret_cast<float2*>(ws + w.sc);
   wa.wf = reinterpret_cast<float*>(ws + w.wf);
   wa.bf = reinterpret_cast<float*>(ws + w.bf);
+  wa.err = a.err;
   {
     int64_t n = static_cast<int64_t>(a.HM3) * a.Cout;
     if (n < a.Cout) n = a.Cout;
@@ -594,6 +608,7 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
   pa.kg = reinterpret_cast<float4*>(ws + w.kg);
   pa.vg = reinterpret_cast<float*>(ws + w.vg);
   pa.rotf = reinterpret_cast<float*>(ws + w.rotf);
+  pa.err = a.err;
   {
     const int64_t n = static_cast<int64_t>(a.B) * a.N * a.H;
     geo_prep_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(pa);
@@ -608,6 +623,7 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
   t.ml = reinterpret_cast<float2*>(ws + w.ml);
   t.live = ws + w.live;
   t.agg = a.out_agg;
+  t.err = a.err;
   cudaError_t le = cudaErrorInvalidValue;
   switch (a.M) {
     case 1: le = launch_attn<1>(t, a.B, a.N, a.H, st); break;
@@ -629,6 +645,7 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
     ma.pm = t.pm;
     for (int d = 0; d < 4; ++d) ma.pms[d] = t.pms[d];
     ma.att = a.out_attention;
+    ma.err = a.err;
     geo_map_kernel<<<dim3((a.N + MAP_ROWS - 1) / MAP_ROWS, a.H, a.B), 256, 0, st>>>(ma);
   }
 
@@ -637,6 +654,7 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
   ReadArgs ra{};
   ra.B = a.B; ra.N = a.N; ra.H = a.H; ra.HM3 = a.HM3; ra.Cout = a.Cout;
   ra.vec = a.out_vectors; ra.live = t.live; ra.wf = wa.wf; ra.bf = wa.bf; ra.out = a.out_output;
+  ra.err = a.err;
   {
     const int64_t rows = static_cast<int64_t>(a.B) * a.N;
     dim3 grid(static_cast<unsigned>((rows + RD_ROWS - 1) / RD_ROWS), (a.Cout + 255) / 256);

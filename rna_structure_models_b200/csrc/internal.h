@@ -75,6 +75,7 @@ struct DistogramArgs {
   int32_t* idx;                    // [B, L, k]
   int32_t* bins;                   // [B, L, k]
   float* hist;                     // [B, L, nb]
+  int* err;                        // bounds-checked build only; the call has no error word (null)
 };
 cudaError_t distogram_launch(const DistogramArgs& a, cudaStream_t stream);
 
@@ -93,9 +94,10 @@ struct MeetPrep {
   float* qs;       // [B, L, H, 16] rho_h q
   float* gamma;    // [H] rho_h s_h^2
   float* consts;   // MEET_ZEROS zeros, then the 3x3 identity
+  int* err;
 };
 cudaError_t meet_launch_prep(const MeetPrep& m, cudaStream_t stream);
-cudaError_t meet_launch_extract(const float* core_out, float* out, int64_t rows, cudaStream_t stream);
+cudaError_t meet_launch_extract(const float* core_out, float* out, int64_t rows, int* err, cudaStream_t stream);
 
 // Dense projection y = x W + b (tcgen05, fp16 operands, fp32 accumulation).
 struct LinearWorkspace {
@@ -121,6 +123,7 @@ struct FramesArgs {
   View n, ca, c;   // [B, L, 3]
   float* rot;      // [B, L, 3, 3]
   float* trans;    // [B, L, 3]
+  int* err;        // bounds-checked build only; the call has no error word (null)
 };
 cudaError_t frames_launch(const FramesArgs& a, cudaStream_t stream);
 

@@ -33,7 +33,10 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "bounds.cuh"
 #include "ipa_epilogue.cuh"
+
+#define IPA_FILE_TAG 2
 #include "sm100.cuh"
 
 #ifdef IPA_TRACE
@@ -472,7 +475,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // training forward: log-sum-exp of the true logits; the pass left the row
     // constant c sum_p |gq'_p|^2 (rowq.w) out of its logits
     if (a.lse != nullptr && half == 0 && in_range)
-      a.lse[static_cast<int64_t>(bh) * L + row] = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
+      *IPA_AT(a.lse, static_cast<int64_t>(bh) * L + row, static_cast<int64_t>(a.B) * a.H * L, a.err) = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
     const int pitch = stage_pitch(DZ);
     float* stage = reinterpret_cast<float*>(smem + SM_STG);
     if (all_ok) {
@@ -496,6 +499,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!*abort_flag) {
       EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, I * QT, a.z1f, a.out};
       ea.uagg = a.uagg;
+      ea.rows = static_cast<int64_t>(a.B) * L * a.H;
+      ea.err = a.err;
       write_rows<IPA_C, IPA_PV>(ea, warp, lane);
     }
   }

@@ -36,8 +36,11 @@
 #include <cmath>
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "ipa_epilogue.cuh"
+
+#define IPA_FILE_TAG 3
 #include "sm100.cuh"
 
 #ifdef IPA_TRACE
@@ -570,7 +573,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     // training forward: log-sum-exp of the true logits; the pass left the row
     // constant c sum_p |gq'_p|^2 (rowq.w) out of its logits
     if (a.lse != nullptr && half == 0 && in_range)
-      a.lse[static_cast<int64_t>(bh) * L + row] = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
+      *IPA_AT(a.lse, static_cast<int64_t>(bh) * L + row, static_cast<int64_t>(a.B) * a.H * L, a.err) = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
     // direct output pass when the pair block has no padding and whole
     // 64-column factors (the staged pass below handles every other shape)
     if (a.tma_epi) {
@@ -584,19 +587,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         const float inv = dead ? 0.f : 1.f / lt;
         const int rrow = in_range ? row : 0;
         const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
+        const int64_t nrows = static_cast<int64_t>(a.B) * L * a.H;
         auto z1box = [&](int k) -> const unsigned char* { return smem + SP_QP + 16384u * k; };
         auto obox = [&](int k) -> unsigned char* {
           return smem + (k == 0 ? SP_QH : SP_QP + 16384u * (nz + k - 1));
         };
         stage_row_pair(tmem + lane_off, half, a.Cz, a.RCz / a.Cz, inv, r,
-                       a.uagg != nullptr ? a.uagg + orow * a.RCz : nullptr, in_range, z1box, obox);
+                       a.uagg != nullptr ? IPA_SPAN(a.uagg, orow * a.RCz, a.RCz, nrows * a.RCz, a.err) : nullptr,
+                       in_range, z1box, obox);
         if (tid == 0) PAIR_SPAN(22);
         if (half == 0)
-          write_row_points<IPA_C, IPA_PV>(tmem + DZ + lane_off, inv, dead, in_range, a.out + orow * a.F, g0, g1, g2, cn);
+          write_row_points<IPA_C, IPA_PV>(tmem + DZ + lane_off, inv, dead, in_range,
+                                          IPA_SPAN(a.out, orow * a.F, a.F, nrows * a.F, a.err), g0, g1, g2, cn);
         fence_proxy_async_smem();   // the staging writes, before the TMA store reads them
       }
       named_bar_sync(1, NSOFT);
-      if (tid == 0 && all_ok && zok && !*abort_flag) {
+      // a tile past the last row (the pair's second CTA when L <= 128) has
+      // nothing to store; the tensor map clips the rest of a ragged tile
+      if (tid == 0 && all_ok && zok && !*abort_flag && row0 < L &&
+          IPA_CHECK(row0 >= 0 && b >= 0 && b < a.B && h >= 0 && h < a.H, a.err)) {
         for (int k = 0; k < a.Cz / 32; ++k)
           tma_store_4d(&tm_out, sb + (k == 0 ? SP_QH : SP_QP + 16384u * (nz + k - 1)), IPA_C + 4 * IPA_PV + 32 * k, h,
                        row0, b);
@@ -610,13 +619,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         const float inv = dead ? 0.f : 1.f / lt;
         const int rrow = in_range ? row : 0;
         const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
+        const int64_t nrows = static_cast<int64_t>(a.B) * L * a.H;
         unsigned long long* etr = nullptr;
 #ifdef IPA_TRACE
         if (tid == 0 && blockIdx.x < 4096) etr = &g_pair_span[blockIdx.x][22];
 #endif
         write_row_direct<IPA_C, IPA_PV>(tmem + lane_off, half, DZ, a.Cz, a.RCz / a.Cz, inv, dead, in_range,
-                                        a.z1f + (static_cast<int64_t>(b) * L + rrow) * DZ, a.out + orow * a.F,
-                                        a.uagg != nullptr ? a.uagg + orow * a.RCz : nullptr, g0, g1, g2, cn, etr);
+                                        a.z1f + (static_cast<int64_t>(b) * L + rrow) * DZ,
+                                        IPA_SPAN(a.out, orow * a.F, a.F, nrows * a.F, a.err),
+                                        a.uagg != nullptr ? IPA_SPAN(a.uagg, orow * a.RCz, a.RCz, nrows * a.RCz, a.err)
+                                                          : nullptr,
+                                        g0, g1, g2, cn, etr);
         if (tid == 0) PAIR_SPAN(21);
       }
     } else {
@@ -646,6 +659,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     if (!*abort_flag) {
       EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, row0, a.z1f, a.out};
       ea.uagg = a.uagg;
+      ea.rows = static_cast<int64_t>(a.B) * L * a.H;
+      ea.err = a.err;
 #ifdef IPA_TRACE
       ea.trace = (blockIdx.x < 4096 && warp == 0) ? &g_pair_span[blockIdx.x][16] : nullptr;
 #endif

@@ -44,8 +44,11 @@
 #include <cmath>
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+
+#define IPA_FILE_TAG 11
 
 namespace fipa {
 
@@ -116,6 +119,7 @@ struct RowsArgs {
   float2* rowd;          // [B*H, L]
   View q_pts, k_pts;
   float* pts;            // [B*H, L, 24]
+  int* err;
 };
 
 // One warp per (b, i, h), heads fastest.  Lane l: scalar channel l (< 16),
@@ -168,15 +172,16 @@ __global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
   const float dg_b = __shfl_sync(0xffffffffu, dog16, lane < 8 ? lane + 16 : lane - 8);
   const float c_lo = lane < C ? g_o : dg_a;
   const float c_hi = dg_b;                 // col 32 + l: l < 8 -> dog[16 + l], else dog[l - 8]
-  __half* drow = a.doh + bhl * 64;
+  const int64_t nbhl = static_cast<int64_t>(a.B) * a.H * a.L;
+  __half* drow = IPA_SPAN(a.doh, bhl * 64, 64, nbhl * 64, a.err);
   drow[lane] = __float2half_rn(live ? c_lo : 0.f);
   drow[32 + lane] = __float2half_rn(live ? c_hi : 0.f);
   // pair block: dU = z1 (.) g_pair (fp16), Q_pair = fp16(w_qp z1), D += dU . U
   const float* z1r = a.z1f + bi * a.DZ;
   const __half* z1hr = a.z1h + bi * a.DZ;
   const float* wr = a.wqp + static_cast<int64_t>(h) * a.DZ;
-  __half* dur = a.du + bhl * a.DZ;
-  __half* qpr = a.qp + bhl * a.DZ;
+  __half* dur = IPA_SPAN(a.du, bhl * a.DZ, a.DZ, nbhl * a.DZ, a.err);
+  __half* qpr = IPA_SPAN(a.qp, bhl * a.DZ, a.DZ, nbhl * a.DZ, a.err);
   const int64_t ubase = b * a.uagg.s[0] + i * a.uagg.s[1] + h * a.uagg.s[2];
   for (int c = lane; c < a.DZ; c += 32) {
     float duv = 0.f;
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
     const int64_t pb = b * pv.s[0] + i * pv.s[1] + h * pv.s[2] + pp * pv.s[3];
     const float x0 = ldf(pv, pb), x1 = ldf(pv, pb + pv.s[4]), x2 = ldf(pv, pb + 2 * pv.s[4]);
     const float v = fmaf(Rm[3 * xx], x0, fmaf(Rm[3 * xx + 1], x1, Rm[3 * xx + 2] * x2)) + tc[xx];
-    a.pts[bhl * 24 + lane] = live ? v : 0.f;
+    *IPA_AT(a.pts, bhl * 24 + lane, nbhl * 24, a.err) = live ? v : 0.f;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
@@ -212,7 +217,7 @@ __global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
       rowc = -(a.rowq[bhl].w + lse * kLog2e);
       D = part;
     }
-    a.rowd[bhl] = make_float2(rowc, D);
+    *IPA_AT(a.rowd, bhl, nbhl, a.err) = make_float2(rowc, D);
   }
 }
 
@@ -495,7 +500,8 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
       tc_fence_after();
       if (half == 0 && in_range) {
         const float4 o = reinterpret_cast<const float4*>(smem + lay.stg)[r];
-        a.rsq[static_cast<int64_t>(bh) * L + row] = make_float4(rs + o.x, ro0 + o.y, ro1 + o.z, ro2 + o.w);
+        *IPA_AT(a.rsq, static_cast<int64_t>(bh) * L + row, static_cast<int64_t>(a.B) * a.H * L, a.err) =
+            make_float4(rs + o.x, ro0 + o.y, ro1 + o.z, ro2 + o.w);
       }
       // accumulators: dQ_h (64 columns, 32 per half) and dQ_pair (DZ, DZ / 2 per half)
       {
@@ -503,7 +509,8 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         tmem_ld32(tmem + Q_TM_DQH + 32 * half + lane_off, v);
         tmem_ld_wait();
         if (in_range) {
-          float4* dst = reinterpret_cast<float4*>(a.dqh + (static_cast<int64_t>(bh) * L + row) * 64 + 32 * half);
+          float4* dst = reinterpret_cast<float4*>(IPA_SPAN(a.dqh, (static_cast<int64_t>(bh) * L + row) * 64 + 32 * half,
+                                                           32, static_cast<int64_t>(a.B) * a.H * L * 64, a.err));
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
@@ -515,7 +522,8 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         tmem_ld32(tmem + Q_TM_DQP + c0 + lane_off, v);
         tmem_ld_wait();
         if (in_range) {
-          float4* dst = reinterpret_cast<float4*>(a.dqp + (static_cast<int64_t>(bh) * L + row) * DZ + c0);
+          float4* dst = reinterpret_cast<float4*>(IPA_SPAN(a.dqp, (static_cast<int64_t>(bh) * L + row) * DZ + c0, 32,
+                                                           static_cast<int64_t>(a.B) * a.H * L * DZ, a.err));
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
@@ -871,8 +879,11 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       tc_fence_after();
       if (half == 0 && in_range) {
         const float4 o = reinterpret_cast<const float4*>(smem + lay.stg)[r];
-        a.csk[static_cast<int64_t>(bh) * L + key] = make_float4(cs + o.x, co0 + o.y, co1 + o.z, co2 + o.w);
-        a.gsum[static_cast<int64_t>(bh) * L + key] = gsum + reinterpret_cast<const float*>(smem + lay.stg + 2048)[r];
+        const int64_t nbhl = static_cast<int64_t>(a.B) * a.H * L;
+        *IPA_AT(a.csk, static_cast<int64_t>(bh) * L + key, nbhl, a.err) =
+            make_float4(cs + o.x, co0 + o.y, co1 + o.z, co2 + o.w);
+        *IPA_AT(a.gsum, static_cast<int64_t>(bh) * L + key, nbhl, a.err) =
+            gsum + reinterpret_cast<const float*>(smem + lay.stg + 2048)[r];
       }
       auto store32 = [&](uint32_t tcol, float* dst_row) {
         uint32_t v[32];
@@ -887,10 +898,11 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         }
       };
       const int64_t rowi = static_cast<int64_t>(bh) * L + (in_range ? key : 0);
-      store32(K_TM_DKH + 32 * half, a.dkh + rowi * 64 + 32 * half);
-      store32(K_TM_DVA + 32 * half, a.dva + rowi * 64 + 32 * half);
+      const int64_t nrow = static_cast<int64_t>(a.B) * a.H * L;
+      store32(K_TM_DKH + 32 * half, IPA_SPAN(a.dkh, rowi * 64 + 32 * half, 32, nrow * 64, a.err));
+      store32(K_TM_DVA + 32 * half, IPA_SPAN(a.dva, rowi * 64 + 32 * half, 32, nrow * 64, a.err));
       for (int c0 = half * (DZ / 2); c0 < (half + 1) * (DZ / 2); c0 += 32)
-        store32(K_TM_DZ2 + c0, a.dz2 + rowi * DZ + c0);
+        store32(K_TM_DZ2 + c0, IPA_SPAN(a.dz2, rowi * DZ + c0, 32, nrow * DZ, a.err));
     }
   }
   tc_fence_before();
@@ -945,6 +957,7 @@ struct MapArgs {
   float *d_q, *d_k, *d_v, *d_qpts, *d_kpts, *d_vpts, *d_rot, *d_trans, *d_z1, *d_z2;
   float* wb_part;        // [B][pair-column blocks][H][DZ]
   double* g_part;        // [nblk * B][H]
+  int* err;
 };
 
 // Block: rb residues of one batch, all heads.  Phase 1: thread (residue,
@@ -981,10 +994,17 @@ __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
       const float* dv = a.dva + bhl * 64;
       const float4 rq = a.rsq[bhl], ck = a.csk[bhl];
       const int64_t o3 = bi * H + h;
+      const int64_t nblh = static_cast<int64_t>(a.B) * a.L * H;
+      float* dqo = IPA_SPAN(a.d_q, o3 * C, C, nblh * C, a.err);
+      float* dko = IPA_SPAN(a.d_k, o3 * C, C, nblh * C, a.err);
+      float* dvo = IPA_SPAN(a.d_v, o3 * C, C, nblh * C, a.err);
+      float* dqpo = IPA_SPAN(a.d_qpts, o3 * PQ * 3, PQ * 3, nblh * PQ * 3, a.err);
+      float* dkpo = IPA_SPAN(a.d_kpts, o3 * PQ * 3, PQ * 3, nblh * PQ * 3, a.err);
+      float* dvpo = IPA_SPAN(a.d_vpts, o3 * PV * 3, PV * 3, nblh * PV * 3, a.err);
       for (int e = 0; e < C; ++e) {
-        a.d_q[o3 * C + e] = a.qscale * dq[e];
-        a.d_k[o3 * C + e] = dk[e];
-        a.d_v[o3 * C + e] = dv[e];
+        dqo[e] = a.qscale * dq[e];
+        dko[e] = dk[e];
+        dvo[e] = dv[e];
       }
       // query and key points: d gq = Gq2c + 2c (RSo - rs gq_c), d gk = 2c (Gk' + CSo - cs gk_c)
       for (int p = 0; p < PQ; ++p) {
@@ -1006,8 +1026,8 @@ __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
           dgk[x] = 2.f * c * (gk1 + cso[x] - ck.x * gkc[x]);
         }
         for (int y = 0; y < 3; ++y) {
-          a.d_qpts[(o3 * PQ + p) * 3 + y] = Rm[y] * dgq[0] + Rm[3 + y] * dgq[1] + Rm[6 + y] * dgq[2];
-          a.d_kpts[(o3 * PQ + p) * 3 + y] = Rm[y] * dgk[0] + Rm[3 + y] * dgk[1] + Rm[6 + y] * dgk[2];
+          dqpo[p * 3 + y] = Rm[y] * dgq[0] + Rm[3 + y] * dgq[1] + Rm[6 + y] * dgq[2];
+          dkpo[p * 3 + y] = Rm[y] * dgk[0] + Rm[3 + y] * dgk[1] + Rm[6 + y] * dgk[2];
         }
         for (int x = 0; x < 3; ++x) {
           for (int y = 0; y < 3; ++y) fr[3 * x + y] += dgq[x] * lq[y] + dgk[x] * lk[y];
@@ -1023,7 +1043,7 @@ __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
           lv[y] = ldf(a.v_pts, b * a.v_pts.s[0] + i * a.v_pts.s[1] + h * a.v_pts.s[2] + p * a.v_pts.s[3] + y * a.v_pts.s[4]);
         for (int x = 0; x < 3; ++x) dgv[x] = dv[C + 3 * p + x];
         for (int y = 0; y < 3; ++y)
-          a.d_vpts[(o3 * PV + p) * 3 + y] = Rm[y] * dgv[0] + Rm[3 + y] * dgv[1] + Rm[6 + y] * dgv[2];
+          dvpo[p * 3 + y] = Rm[y] * dgv[0] + Rm[3 + y] * dgv[1] + Rm[6 + y] * dgv[2];
         for (int x = 0; x < 3; ++x) {
           for (int y = 0; y < 3; ++y) fr[3 * x + y] += dgv[x] * lv[y];
           fr[9 + x] += dgv[x];
@@ -1061,14 +1081,15 @@ __global__ void __launch_bounds__(256) ipa_bwd_map_kernel(const MapArgs a) {
     float s = 0.f;
     for (int h = 0; h < H; ++h) s += fterm[(il * H + h) * 12 + e];
     const int64_t bi = static_cast<int64_t>(b) * a.L + i;
-    if (e < 9) a.d_rot[bi * 9 + e] = s;
-    else a.d_trans[bi * 3 + (e - 9)] = s;
+    const int64_t nbl = static_cast<int64_t>(a.B) * a.L;
+    if (e < 9) *IPA_AT(a.d_rot, bi * 9 + e, nbl * 9, a.err) = s;
+    else *IPA_AT(a.d_trans, bi * 3 + (e - 9), nbl * 3, a.err) = s;
   }
   // d gamma partial of this block: residues in order
   for (int h = tid; h < H; h += blockDim.x) {
     double s = 0.0;
     for (int il = 0; il < rb; ++il) s += gterm[il * H + h];
-    a.g_part[(static_cast<int64_t>(b) * a.nblk + blk) * H + h] = s;
+    *IPA_AT(a.g_part, (static_cast<int64_t>(b) * a.nblk + blk) * H + h, static_cast<int64_t>(a.B) * a.nblk * H, a.err) = s;
   }
 }
 
@@ -1119,13 +1140,15 @@ __global__ void __launch_bounds__(256) ipa_bwd_pair_kernel(const MapArgs a) {
 #pragma unroll
       for (int q = 0; q < PAIR_RB; ++q) w += wsm[q][hh][c];
       if (blockIdx.x * 32 + c < a.DZ)
-        a.wb_part[((static_cast<int64_t>(b) * gridDim.y + blk) * H + h0 + hh) * a.DZ + blockIdx.x * 32 + c] = w;
+        *IPA_AT(a.wb_part, ((static_cast<int64_t>(b) * gridDim.y + blk) * H + h0 + hh) * a.DZ + blockIdx.x * 32 + c,
+                static_cast<int64_t>(a.B) * gridDim.y * H * a.DZ, a.err) = w;
     }
     __syncthreads();
   }
   if (inpair) {
-    a.d_z1[bi * a.RCz + col] = s1;
-    a.d_z2[bi * a.RCz + col] = s2;
+    const int64_t nz = static_cast<int64_t>(a.B) * a.L * a.RCz;
+    *IPA_AT(a.d_z1, bi * a.RCz + col, nz, a.err) = s1;
+    *IPA_AT(a.d_z2, bi * a.RCz + col, nz, a.err) = s2;
   }
 }
 
@@ -1138,7 +1161,7 @@ __global__ void __launch_bounds__(256) ipa_bwd_pair_kernel(const MapArgs a) {
 constexpr int RED_THREADS = 1024;
 __global__ void __launch_bounds__(RED_THREADS) ipa_bwd_reduce_kernel(const float* wb_part, int nwb, const double* g_part,
                                                                      int ng, int H, int DZ, int Cz, int R, float scale,
-                                                                     float* d_wb, float* d_gamma) {
+                                                                     float* d_wb, float* d_gamma, int* err) {
   __shared__ double red[32][33];
   const int h = blockIdx.x, t = threadIdx.x, cl = t & 31, g = t >> 5;
   const int c = blockIdx.y * 32 + cl;
@@ -1151,7 +1174,7 @@ __global__ void __launch_bounds__(RED_THREADS) ipa_bwd_reduce_kernel(const float
   if (t < 32 && c < Cz) {
     double sum = 0.0;
     for (int q = 0; q < 32; ++q) sum += red[q][t];
-    d_wb[c * H + h] = static_cast<float>(sum * scale);
+    *IPA_AT(d_wb, c * H + h, static_cast<int64_t>(Cz) * H, err) = static_cast<float>(sum * scale);
   }
   if (blockIdx.y == 0 && t >= 32 && t < 64) {
     const int l = t - 32;
@@ -1159,7 +1182,7 @@ __global__ void __launch_bounds__(RED_THREADS) ipa_bwd_reduce_kernel(const float
     for (int p = l; p < ng; p += 32) gs += g_part[static_cast<int64_t>(p) * H + h];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, off);
-    if (l == 0) d_gamma[h] = static_cast<float>(gs);
+    if (l == 0) *IPA_AT(d_gamma, h, H, err) = static_cast<float>(gs);
   }
 }
 
@@ -1228,6 +1251,7 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   ra.rowd = reinterpret_cast<float2*>(ws + w.rowd);
   ra.q_pts = f.q_pts; ra.k_pts = f.k_pts;
   ra.pts = reinterpret_cast<float*>(ws + w.pts);
+  ra.err = f.err;
   const int64_t warps = static_cast<int64_t>(B) * L * H;
   ipa_bwd_rows_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(ra);
   e = cudaGetLastError();
@@ -1307,6 +1331,7 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   m.d_rot = a.d_rot; m.d_trans = a.d_trans; m.d_z1 = a.d_z1; m.d_z2 = a.d_z2;
   m.wb_part = reinterpret_cast<float*>(ws + w.wb_part);
   m.g_part = reinterpret_cast<double*>(ws + w.g_part);
+  m.err = f.err;
   const size_t msmem = static_cast<size_t>((m.rb * H * 12 + 1) & ~1) * 4 + static_cast<size_t>(m.rb) * H * 8;
   ipa_bwd_map_kernel<<<dim3(static_cast<unsigned>(m.nblk), static_cast<unsigned>(B)), 256, msmem, stream>>>(m);
   e = cudaGetLastError();
@@ -1318,7 +1343,7 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const dim3 rgrid(static_cast<unsigned>(H), static_cast<unsigned>((f.Cz + 31) / 32));
   ipa_bwd_reduce_kernel<<<rgrid, RED_THREADS, 0, stream>>>(m.wb_part, B * npb, m.g_part, B * m.nblk, H, DZ, f.Cz, f.R,
-                                                          kLog2e * f.w_L, a.d_w_bias, a.d_gamma);
+                                                          kLog2e * f.w_L, a.d_w_bias, a.d_gamma, f.err);
   return cudaGetLastError();
 }
 

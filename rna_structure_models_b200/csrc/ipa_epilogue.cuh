@@ -21,7 +21,12 @@
 
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "sm100.cuh"
+
+#pragma push_macro("IPA_FILE_TAG")
+#undef IPA_FILE_TAG
+#define IPA_FILE_TAG 4
 
 namespace fipa {
 
@@ -44,6 +49,8 @@ struct EpilogueArgs {
   const float* z1f;      // [B, L, DZ] fp32, zero-padded
   float* out;            // [B, L, H, F]
   float* uagg = nullptr; // training forward only: [B, L, H, R Cz] pair aggregate U (else null)
+  int64_t rows = 0;      // B L H: output rows (extent of out and uagg in rows; bounds-checked build)
+  int* err = nullptr;    // error word of the bounds-checked build
 #ifdef IPA_TRACE
   unsigned long long* trace = nullptr;   // phase clocks of warp 0 (tracing build only)
 #endif
@@ -172,7 +179,8 @@ static __device__ __noinline__ void store_pair_aggregate(const EpilogueArgs& e, 
     const int grow = e.row0 + warp * 16 + rr;
     if (grow >= e.L) break;
     const float4* src = reinterpret_cast<const float4*>(e.stage + (warp * 16 + rr) * pitch + 64);
-    float4* dst = reinterpret_cast<float4*>(e.uagg + ((static_cast<int64_t>(e.b) * e.L + grow) * e.H + e.h) * e.RCz);
+    float4* dst = reinterpret_cast<float4*>(IPA_SPAN(e.uagg, ((static_cast<int64_t>(e.b) * e.L + grow) * e.H + e.h) * e.RCz,
+                                                     e.RCz, e.rows * e.RCz, e.err));
     for (int q = lane; q < nq; q += 32) dst[q] = src[q];
   }
   __syncwarp();
@@ -203,7 +211,9 @@ __device__ __forceinline__ void write_rows(const EpilogueArgs& e, int warp, int 
     const int rloc = warp * 16 + rr;
     const int grow = e.row0 + rloc;
     if (grow < e.L)
-      write_row<C, PV>(e.stage + rloc * pitch, e.out + ((static_cast<int64_t>(e.b) * e.L + grow) * e.H + e.h) * e.F,
+      write_row<C, PV>(e.stage + rloc * pitch,
+                       IPA_SPAN(e.out, ((static_cast<int64_t>(e.b) * e.L + grow) * e.H + e.h) * e.F, e.F, e.rows * e.F,
+                                e.err),
                        lane, e.DZ, e.F);
     EPI_TR(3 + rr);
   }
@@ -360,3 +370,5 @@ __device__ __forceinline__ void write_row_points(uint32_t tmem_v, float inv, boo
 }
 
 }  // namespace fipa
+
+#pragma pop_macro("IPA_FILE_TAG")

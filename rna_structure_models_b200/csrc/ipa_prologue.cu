@@ -29,8 +29,11 @@
 #include <cmath>
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+
+#define IPA_FILE_TAG 1
 
 namespace fipa {
 
@@ -100,9 +103,12 @@ __device__ __forceinline__ bool ipa_tile_copy_pairs_vec(const TileArgs& a, int b
     const int i = i0 + 16 * q + (tid >> 4);
     if (i < a.L) {
       const int64_t o = (static_cast<int64_t>(b) * a.L + i) * a.DZ + col;
-      *reinterpret_cast<float4*>(a.z1f + o) = v1[q];
-      *reinterpret_cast<uint2*>(a.z1h + o) = make_uint2(pack_half2(v1[q].x, v1[q].y), pack_half2(v1[q].z, v1[q].w));
-      *reinterpret_cast<uint2*>(a.z2h + o) = make_uint2(pack_half2(v2[q].x, v2[q].y), pack_half2(v2[q].z, v2[q].w));
+      const int64_t ext = static_cast<int64_t>(a.B) * a.L * a.DZ;
+      *reinterpret_cast<float4*>(IPA_SPAN(a.z1f, o, 4, ext, a.err)) = v1[q];
+      *reinterpret_cast<uint2*>(IPA_SPAN(a.z1h, o, 4, ext, a.err)) =
+          make_uint2(pack_half2(v1[q].x, v1[q].y), pack_half2(v1[q].z, v1[q].w));
+      *reinterpret_cast<uint2*>(IPA_SPAN(a.z2h, o, 4, ext, a.err)) =
+          make_uint2(pack_half2(v2[q].x, v2[q].y), pack_half2(v2[q].z, v2[q].w));
     }
   }
   return true;
@@ -134,9 +140,10 @@ __device__ __forceinline__ void ipa_tile_copy_pairs(const TileArgs& a, int b, in
     const int i = i0 + 4 * q + (tid >> 6);
     if (i < a.L) {
       const int64_t o = (static_cast<int64_t>(b) * a.L + i) * a.DZ + col;
-      a.z1f[o] = v1[q];
-      a.z1h[o] = __float2half_rn(v1[q]);
-      a.z2h[o] = __float2half_rn(v2[q]);
+      const int64_t ext = static_cast<int64_t>(a.B) * a.L * a.DZ;
+      *IPA_AT(a.z1f, o, ext, a.err) = v1[q];
+      *IPA_AT(a.z1h, o, ext, a.err) = __float2half_rn(v1[q]);
+      *IPA_AT(a.z2h, o, ext, a.err) = __float2half_rn(v2[q]);
     }
   }
 }
@@ -162,7 +169,7 @@ __global__ void __launch_bounds__(256) ipa_tile_kernel(const TileArgs a) {
         for (int y = 0; y < 3; ++y) Rm[3 * x + y] = ldf(a.rot, ro + x * a.rot.s[2] + y * a.rot.s[3]);
       const int64_t to = b * a.trans.s[0] + i * a.trans.s[1];
       const float tx = ldf(a.trans, to), ty = ldf(a.trans, to + a.trans.s[2]), tz = ldf(a.trans, to + 2 * a.trans.s[2]);
-      float4* f = a.frame + (static_cast<int64_t>(b) * a.L + i) * 4;
+      float4* f = IPA_SPAN(a.frame, (static_cast<int64_t>(b) * a.L + i) * 4, 4, static_cast<int64_t>(a.B) * a.L * 4, a.err);
       f[0] = make_float4(Rm[0], Rm[1], Rm[2], Rm[3]);
       f[1] = make_float4(Rm[4], Rm[5], Rm[6], Rm[7]);
       f[2] = make_float4(Rm[8], tx, ty, tz);
@@ -182,8 +189,8 @@ __global__ void __launch_bounds__(256) ipa_tile_kernel(const TileArgs a) {
   }
   __syncthreads();
   if (tid == 0)
-    a.part[b * a.nkt + J] = make_float4(red[0][0] + red[1][0], red[0][1] + red[1][1],
-                                        red[0][2] + red[1][2], red[0][3] + red[1][3]);
+    *IPA_AT(a.part, b * a.nkt + J, static_cast<int64_t>(a.B) * a.nkt, a.err) =
+        make_float4(red[0][0] + red[1][0], red[0][1] + red[1][1], red[0][2] + red[1][2], red[0][3] + red[1][3]);
   ipa_tile_copy_pairs(a, b, i0, 0, tid);
 }
 
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     for (int64_t e = static_cast<int64_t>(i) * H + h; e < static_cast<int64_t>(H) * a.DZ;
          e += static_cast<int64_t>(H) * a.L) {
       const int he = static_cast<int>(e / a.DZ), col = static_cast<int>(e % a.DZ);
-      a.wqp[e] = col < a.RCz ? kLog2e * a.w_L * ldf(a.w_bias, (col % a.Cz) * a.w_bias.s[0] + he * a.w_bias.s[1]) : 0.f;
+      *IPA_AT(a.wqp, e, static_cast<int64_t>(H) * a.DZ, a.err) = col < a.RCz ? kLog2e * a.w_L * ldf(a.w_bias, (col % a.Cz) * a.w_bias.s[0] + he * a.w_bias.s[1]) : 0.f;
     }
   if (active) {
   const float4 cn = cen_s;
@@ -305,11 +312,11 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
   const float4 okv = tile_origin(partb, i / KT, i / KT + 1, cn);
   // the values the core kernel reads per batch / tile / head, one writer each
   if (h == 0) {
-    if (i == 0) a.cen[b] = cn;
-    if (i % QT == 0) a.oq[b * a.nqt + i / QT] = oqv;
-    if (i % KT == 0) a.ok[b * a.nkt + i / KT] = okv;
+    if (i == 0) *IPA_AT(a.cen, b, a.B, a.err) = cn;
+    if (i % QT == 0) *IPA_AT(a.oq, b * a.nqt + i / QT, static_cast<int64_t>(a.B) * a.nqt, a.err) = oqv;
+    if (i % KT == 0) *IPA_AT(a.ok, b * a.nkt + i / KT, static_cast<int64_t>(a.B) * a.nkt, a.err) = okv;
   }
-  if (b == 0 && i == 0) a.headc[h] = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
+  if (b == 0 && i == 0) *IPA_AT(a.headc, h, H, a.err) = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
   const float c = kLog2e * a.w_L * ldf(a.gamma, h * a.gamma.s[0]) * a.w_C * 0.5f;
 
   const float4* fr = a.frame + (static_cast<int64_t>(b) * a.L + i) * 4;
@@ -439,14 +446,16 @@ __global__ void __launch_bounds__(128, 4) ipa_rows_kernel(const RowArgs a) {
     const uint4* src = stage_rows + static_cast<size_t>(kind * H * rb) * 8;
     for (int e = threadIdx.x; e < H * run; e += blockDim.x) {
       const int hh = e / run, r = e % run;
-      outs[kind][(static_cast<int64_t>(b * H + hh) * a.L + i0) * 8 + r] = src[hh * rb * 8 + r];
+      *IPA_AT(outs[kind], (static_cast<int64_t>(b * H + hh) * a.L + i0) * 8 + r, static_cast<int64_t>(a.B) * H * a.L * 8,
+              a.err) = src[hh * rb * 8 + r];
     }
   }
   for (int e = threadIdx.x; e < 2 * H * nrow; e += blockDim.x) {
     const int which = e / (H * nrow), rem = e % (H * nrow);
     const int hh = rem / nrow, r = rem % nrow;
     float4* dst = which == 0 ? a.rowq : a.colk;
-    dst[static_cast<int64_t>(b * H + hh) * a.L + i0 + r] = sterm[which * H * rb + hh * rb + r];
+    *IPA_AT(dst, static_cast<int64_t>(b * H + hh) * a.L + i0 + r, static_cast<int64_t>(a.B) * H * a.L, a.err) =
+        sterm[which * H * rb + hh * rb + r];
   }
 }
 

@@ -18,8 +18,11 @@
 #include <cmath>
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+
+#define IPA_FILE_TAG 10
 
 namespace fipa {
 
@@ -142,7 +145,10 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int row = m0 + warp * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-      float* yr = a.y + static_cast<int64_t>(row < a.M ? row : 0) * a.ldy;
+      // this CTA's columns [n0, n0 + LBN) of the row, within [M - 1 rows of ldy, then N]
+      const int ncol = a.N - n0 < LBN ? a.N - n0 : LBN;
+      float* yr = IPA_SPAN(a.y, static_cast<int64_t>(row < a.M ? row : 0) * a.ldy + n0, ncol,
+                           static_cast<int64_t>(a.M - 1) * a.ldy + a.N, a.err) - n0;
       for (int c0 = 0; c0 < LBN; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + c0 + lane_off, v);
@@ -183,6 +189,7 @@ struct PackX {
   int M, K, Kp;
   View x;          // [M, K] fp32 (strides s[0], s[1])
   __half* out;     // [M, Kp]
+  int* err;
 };
 
 __global__ void linear_pack_x_kernel(const PackX a) {
@@ -192,13 +199,14 @@ __global__ void linear_pack_x_kernel(const PackX a) {
   const int m = static_cast<int>(t / (a.Kp / 2)), k = 2 * static_cast<int>(t % (a.Kp / 2));
   const float* x = static_cast<const float*>(a.x.p) + m * a.x.s[0];
   const float v0 = k < a.K ? x[k * a.x.s[1]] : 0.f, v1 = k + 1 < a.K ? x[(k + 1) * a.x.s[1]] : 0.f;
-  reinterpret_cast<__half2*>(a.out)[t] = __floats2half2_rn(v0, v1);
+  *IPA_AT(reinterpret_cast<__half2*>(a.out), t, n, a.err) = __floats2half2_rn(v0, v1);
 }
 
 struct PackW {
   int K, N, Kp;
   View w;          // [K, N] fp32
   __half* out;     // [N, Kp]
+  int* err;
 };
 
 // 32 x 32 tiles: read along n (contiguous in W), write along k (contiguous in W^T)
@@ -213,7 +221,9 @@ __global__ void __launch_bounds__(256) linear_pack_w_kernel(const PackW a) {
   __syncthreads();
   for (int r = threadIdx.y; r < 32; r += 8) {
     const int n = n0 + r, k = k0 + threadIdx.x;
-    if (n < a.N && k < a.Kp) a.out[static_cast<int64_t>(n) * a.Kp + k] = __float2half_rn(tile[threadIdx.x][r]);
+    if (n < a.N && k < a.Kp)
+      *IPA_AT(a.out, static_cast<int64_t>(n) * a.Kp + k, static_cast<int64_t>(a.N) * a.Kp, a.err) =
+          __float2half_rn(tile[threadIdx.x][r]);
   }
 }
 
@@ -235,12 +245,12 @@ cudaError_t linear_launch(const LinearLaunch& a, cudaStream_t st) {
   __half* x16 = reinterpret_cast<__half*>(a.ws + a.lay.x16);
   __half* w16 = reinterpret_cast<__half*>(a.ws + a.lay.w16);
   {
-    PackX p{a.M, a.K, Kp, a.x, x16};
+    PackX p{a.M, a.K, Kp, a.x, x16, a.err};
     const int64_t n = static_cast<int64_t>(a.M) * (Kp / 2);
     linear_pack_x_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p);
   }
   {
-    PackW p{a.K, a.N, Kp, a.w, w16};
+    PackW p{a.K, a.N, Kp, a.w, w16, a.err};
     linear_pack_w_kernel<<<dim3(Kp / 32, (a.N + 31) / 32), dim3(32, 8), 0, st>>>(p);
   }
   CUtensorMap tx, tw;

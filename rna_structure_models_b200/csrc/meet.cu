@@ -14,7 +14,10 @@
 // constant block in the workspace.
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
+
+#define IPA_FILE_TAG 8
 
 namespace fipa {
 
@@ -31,28 +34,28 @@ __global__ void __launch_bounds__(256) meet_prep_kernel(const MeetPrep m) {
     const int i = static_cast<int>(bi % m.L), b = static_cast<int>(bi / m.L);
     const float* q = static_cast<const float*>(m.q.p);
     const float rho = static_cast<const float*>(m.rho.p)[h * m.rho.s[0]];
-    m.qs[t] = rho * q[b * m.q.s[0] + i * m.q.s[1] + h * m.q.s[2] + c * m.q.s[3]];
+    *IPA_AT(m.qs, t, n, m.err) = rho * q[b * m.q.s[0] + i * m.q.s[1] + h * m.q.s[2] + c * m.q.s[3]];
   }
   if (blockIdx.x == 0) {
     for (int h = threadIdx.x; h < m.H; h += blockDim.x) {
       const float rho = static_cast<const float*>(m.rho.p)[h * m.rho.s[0]];
       const float s = static_cast<const float*>(m.s.p)[h * m.s.s[0]];
-      m.gamma[h] = rho * s * s;
+      *IPA_AT(m.gamma, h, m.H, m.err) = rho * s * s;
     }
     // constant block: MEET_ZEROS zeros, then the 3x3 identity
     for (int e = threadIdx.x; e < MEET_ZEROS + 9; e += blockDim.x)
-      m.consts[e] = e < MEET_ZEROS ? 0.f : ((e - MEET_ZEROS) % 4 == 0 ? 1.f : 0.f);
+      *IPA_AT(m.consts, e, MEET_ZEROS + 9, m.err) = e < MEET_ZEROS ? 0.f : ((e - MEET_ZEROS) % 4 == 0 ? 1.f : 0.f);
   }
 }
 
 // out[r, 0:16] = core_out[r, 0:16] for every (b, i, h) row r
 __global__ void __launch_bounds__(256) meet_extract_kernel(const float4* __restrict__ src, float4* __restrict__ dst,
-                                                           int64_t rows, int src_row_f4) {
+                                                           int64_t rows, int src_row_f4, int* err) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= rows * (MEET_C / 4)) return;
   const int64_t r = t / (MEET_C / 4);
   const int q = static_cast<int>(t % (MEET_C / 4));
-  dst[t] = src[r * src_row_f4 + q];
+  *IPA_AT(dst, t, rows * (MEET_C / 4), err) = src[r * src_row_f4 + q];
 }
 
 }  // namespace
@@ -79,10 +82,10 @@ cudaError_t meet_launch_prep(const MeetPrep& m, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-cudaError_t meet_launch_extract(const float* core_out, float* out, int64_t rows, cudaStream_t stream) {
+cudaError_t meet_launch_extract(const float* core_out, float* out, int64_t rows, int* err, cudaStream_t stream) {
   const int64_t n = rows * (MEET_C / 4);
   meet_extract_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
-      reinterpret_cast<const float4*>(core_out), reinterpret_cast<float4*>(out), rows, MEET_F / 4);
+      reinterpret_cast<const float4*>(core_out), reinterpret_cast<float4*>(out), rows, MEET_F / 4, err);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,6 @@
 """Helpers shared by the GPU tests: move seeded inputs to the device and
 compare against the oracle with the tolerances the fused path is held to."""
+import contextlib
 import os
 
 import numpy as np
@@ -45,3 +46,22 @@ def assert_parity(gpu, ref, max_abs=IPA_MAX_ABS, rel_fro=IPA_REL_FRO, what=""):
             f.write(f"{what}\tmax_abs={m:.3e}\trel_fro={r:.3e}\tbound=({max_abs}, {rel_fro})\n")
     assert m <= max_abs and r <= rel_fro, f"{what}: max-abs {m:.3e} (<= {max_abs}), rel-Fro {r:.3e} (<= {rel_fro})"
     return m, r
+
+
+@contextlib.contextmanager
+def checked_library():
+    """Route the binding's calls to the bounds-checked build of the library
+    (every global store index checked against its buffer; an index outside
+    it is reported as IPA_ERR_BOUNDS through the plans' error words).  The
+    build is compiled here when missing or older than a source."""
+    from rna_structure_models_b200 import api, build
+    if build.checked_is_stale():
+        build.build_checked()
+    saved = api._lib
+    api._lib = None
+    try:
+        lib = api.library(build.CHECKED_LIB)
+        assert lib.ipa_version().decode().endswith("bounds-checked")
+        yield lib
+    finally:
+        api._lib = saved

@@ -35,12 +35,26 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings_and_version():
     lib = api.library()
-    for code in range(9):
-        assert lib.ipa_status_string(code)
+    for code in range(10):
+        assert lib.ipa_status_string(code) != b"unknown status"
     assert b"sm_100a" in lib.ipa_version()
+    assert not lib.ipa_version().endswith(b"bounds-checked")   # the product build carries no checks
     assert lib.ipa_device_error_status(0) == 0
     assert lib.ipa_device_error_status(1) == 8       # bounded wait expired -> IPA_ERR_TIMEOUT
     assert lib.ipa_device_error_status(7) == 7
+    # bounds-checked build: 0x10000 | file tag << 12 | source line -> IPA_ERR_BOUNDS
+    assert lib.ipa_device_error_status(0x10000 | (11 << 12) | 873) == 9
+
+
+def test_checked_build_exports_the_same_symbols_and_reports_itself():
+    from rna_structure_models_b200 import build
+    if build.checked_is_stale():
+        pytest.skip("bounds-checked library not built (python -m rna_structure_models_b200.build)")
+    chk = ctypes.CDLL(build.CHECKED_LIB)
+    chk.ipa_version.restype = ctypes.c_char_p
+    assert chk.ipa_version().endswith(b"bounds-checked")
+    for name in api.EXPORTED:
+        assert hasattr(chk, name), name
 
 
 def desc(shape, dtype=api.IPA_DTYPE_F32, ptr=FAKE, strides=None):
@@ -286,7 +300,7 @@ def geo_bwd_call(p, ds, grads_over=None, ws_bytes=None, **up_over):
                             *[ctypes.byref(up[k]) if up[k] is not None else None
                               for k in ("g_output", "g_attention", "g_vectors")],
                             ctypes.byref(grads), ctypes.c_void_p(FAKE), ctypes.c_size_t(ws_bytes),
-                            ctypes.c_void_p(FAKE))
+                            ctypes.c_void_p(FAKE), None)
 
 
 def test_geo_bwd_workspace_grows_with_the_problem_and_is_zero_outside_envelope():

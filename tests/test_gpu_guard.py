@@ -8,6 +8,10 @@ filled with the byte 0x7F.  After a call on ragged sizes (tile remainders of
 itself starts filled with 0x7F too, so a kernel that read workspace it had
 not written first would also change its results, which are compared with a
 call on ordinary (zero-initialised) buffers.
+
+Every case runs twice: on the product library and on its bounds-checked
+build, where each store index is checked against its buffer and an index
+outside it raises IPA_ERR_BOUNDS from the plan's `check()`.
 """
 import numpy as np
 import pytest
@@ -16,9 +20,18 @@ import torch
 from rna_structure_models_b200 import api
 from rna_structure_models_b200.synth import (GeoDims, IpaDims, MeetDims, ModuleDims, backbone_inputs,
                                              geo_inputs, geo_upstream, ipa_inputs, meet_inputs, module_inputs)
-from tests.gpu_util import to_dev
+from tests.gpu_util import checked_library, to_dev
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(params=["product", "checked"], autouse=True)
+def library_build(request):
+    if request.param == "product":
+        yield request.param
+    else:
+        with checked_library():
+            yield request.param
 
 GUARD = 4096
 FILL = 0x7F
@@ -99,6 +112,7 @@ def test_variant_and_gradient_guard_bands(cuda_device, N):
     gout = {k: g2.like(v) for k, v in gref.items()}
     gplan(inp, up["g_output"], up.get("g_attention"), up.get("g_vectors"), out=gout)
     g2.check()
+    gplan.check()
     for k in gref:
         if gref[k] is not None:
             assert torch.equal(gout[k], gref[k]), k
