@@ -1057,5 +1057,8 @@ extern "C" __attribute__((visibility("default"))) int ipa_pair_trace_copy(void* 
 extern "C" __attribute__((visibility("default"))) int ipa_pair_span_copy(void* host, size_t bytes) {
   return fipa::ipa_pair_span_read(host, bytes) ? 0 : 1;
 }
+extern "C" __attribute__((visibility("default"))) int ipa_bwd_trace_copy(void* host, size_t bytes) {
+  return fipa::ipa_bwd_trace_read(host, bytes) ? 0 : 1;
+}
 extern "C" __attribute__((visibility("default"))) int ipa_pair_max_clusters() { return fipa::ipa_pair_max_clusters(); }
 #endif

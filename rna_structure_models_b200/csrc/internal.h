@@ -190,6 +190,7 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream);
 #ifdef IPA_TRACE
 bool ipa_pair_trace_read(void* host, size_t bytes);
 bool ipa_pair_span_read(void* host, size_t bytes);
+bool ipa_bwd_trace_read(void* host, size_t bytes);
 int ipa_pair_max_clusters();
 #endif
 

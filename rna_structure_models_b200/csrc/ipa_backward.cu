@@ -50,6 +50,20 @@
 
 #define IPA_FILE_TAG 11
 
+#ifdef IPA_TRACE
+// Tracing build only: per-tile event clocks of the first CTA of each pass,
+// [pass][tile][event] (events listed where they are taken).
+__device__ unsigned long long g_bwd_trace[2][256][16];
+#define BWD_TR(pass, j, ev)                                                         \
+  do {                                                                              \
+    if (blk == 0 && (j) >= 0 && (j) < 256) g_bwd_trace[(pass)][(j)][(ev)] = clock64(); \
+  } while (0)
+#else
+#define BWD_TR(pass, j, ev) \
+  do {                      \
+  } while (0)
+#endif
+
 namespace fipa {
 
 using namespace sm100;
@@ -286,7 +300,7 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
     mbar_init(bar(QB_DSFREE), 1);
     mbar_init(bar(QB_DRAIN), 1);
     for (int s = 0; s < MAX_NS; ++s) {
-      mbar_init(bar(QB_FULL0 + s), 1);
+      mbar_init(bar(QB_FULL0 + s), 2);   // the copy's expect-tx arrive and the column-term arrive
       mbar_init(bar(QB_EMPTY0 + s), 1);
     }
     *abort_flag = 0;
@@ -314,43 +328,52 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
       tma_load_3d(sb + lay.dO, &tm_do, bar(QB_QFULL), 0, I * QT, bh);
       tma_load_4d(sb + lay.du, &tm_du, bar(QB_QFULL), 0, I * QT, 0, bh);
     }
+    // A stage's copy is issued as soon as the stage is free.  The global
+    // values its column terms need (the key tile's origin, the keys' column
+    // terms) are loaded one tile ahead; FULL completes on the copy and on a
+    // second arrive after the terms are in shared memory.
     int issued = 0;
+    auto fetch = [&](int j, float4& okv, float4& ck) {
+      okv = a.ok[b * a.nkt + j * BT / KT];   // the 64-key origin tile holding these keys
+      const int key = j * BT + lane;
+      ck = key < L ? a.colk[static_cast<int64_t>(bh) * L + key] : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    float4 ok_next, ck_next;
+    fetch(0, ok_next, ck_next);
     for (int j = 0; j < nt; ++j) {
       const int s = j % NS;
       if (j >= NS) {
         int ok = 1;
         if (lane == 0) ok = mbar_wait_bounded(bar(QB_EMPTY0 + s), ((j / NS) - 1) & 1, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (lane == 0) BWD_TR(0, j, 10);   // stage free
         if (!ok) {
           if (lane == 0) fail(DEV_TIMEOUT_EMPTY);
           break;
         }
       }
       issued = j + 1;
-      const float4 okv = a.ok[b * a.nkt + j * BT / KT];   // the 64-key origin tile holding these keys
-      const float dx = okv.x - oqv.x, dy = okv.y - oqv.y, dz = okv.z - oqv.z;
-      {
-        const int key = j * BT + lane;
-        float cv = -INFINITY;
-        if (key < L) {
-          const float4 ck = a.colk[static_cast<int64_t>(bh) * L + key];
-          cv = ck.w - fmaf(ck.x, dx, fmaf(ck.y, dy, ck.z * dz));
-        }
-        col_s[s * BT + lane] = cv;
-      }
-      if (lane == 0) {
-        info[2 * s] = make_float4(dx, dy, dz, fmaf(dx, dx, fmaf(dy, dy, dz * dz)));
-        info[2 * s + 1] = okv;
-      }
-      __syncwarp();
       if (lane == 0) {
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
         mbar_arrive_expect_tx(bar(QB_FULL0 + s), lay.stg_bytes);
         tma_load_3d(st, &tm_kh, bar(QB_FULL0 + s), 0, j * BT, bh);
         tma_load_3d(st + 4096, &tm_vh, bar(QB_FULL0 + s), 0, j * BT, bh);
         tma_load_4d(st + 8192, &tm_z2, bar(QB_FULL0 + s), 0, j * BT, 0, b);
+        BWD_TR(0, j, 11);                  // copy issued
+      }
+      const float4 okv = ok_next, ck = ck_next;
+      if (j + 1 < nt) fetch(j + 1, ok_next, ck_next);
+      const float dx = okv.x - oqv.x, dy = okv.y - oqv.y, dz = okv.z - oqv.z;
+      col_s[s * BT + lane] = j * BT + lane < L ? ck.w - fmaf(ck.x, dx, fmaf(ck.y, dy, ck.z * dz)) : -INFINITY;
+      if (lane == 0) {
+        info[2 * s] = make_float4(dx, dy, dz, fmaf(dx, dx, fmaf(dy, dy, dz * dz)));
+        info[2 * s + 1] = okv;
       }
       __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(QB_FULL0 + s));
+        BWD_TR(0, j, 12);                  // column terms in
+      }
     }
     if (lane == 0 && *abort_flag) {
       // copies still in flight must land before the CTA exits
@@ -372,7 +395,9 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
       auto issue_sdp = [&](int j) -> bool {
         const int s = j % NS;
         bool w = mbar_wait_bounded(bar(QB_FULL0 + s), (j / NS) & 1, abort_flag);
+        BWD_TR(0, j, 0);                   // stage j landed
         if (w && j > 0) w = mbar_wait_bounded(bar(QB_SFREE), (j - 1) & 1, abort_flag);
+        BWD_TR(0, j, 1);                   // S(j-1), dP(j-1) read
         if (!w) { fail(DEV_TIMEOUT_FULL); return false; }
         tc_fence_after();
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
@@ -388,11 +413,13 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
           umma_ss(tDP, kd128(sb + lay.du + 16384 * (kk >> 2) + 32 * (kk & 3)),
                   kd128(st + 8192 + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
         umma_commit(bar(QB_SFULL));
+        BWD_TR(0, j, 2);                   // S(j), dP(j) issued
         issued_any = true;
         return true;
       };
       auto issue_dq = [&](int jj) -> bool {
         if (!mbar_wait_bounded(bar(QB_DSFULL), jj & 1, abort_flag)) { fail(DEV_TIMEOUT_SOFTMAX); return false; }
+        BWD_TR(0, jj, 3);                  // dS(jj) written
         tc_fence_after();
         const int s = jj % NS;
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
@@ -404,18 +431,17 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         }
         umma_commit(bar(QB_DSFREE));
         umma_commit(bar(QB_EMPTY0 + s));
+        BWD_TR(0, jj, 4);                  // dQ(jj) issued
         return true;
       };
-      // With one stage, dQ(j-1) must release the stage before tile j can
-      // load; with more, S(j) and dP(j) run while the threads work on j-1.
+      // dQ(j-1) before S(j), dP(j): tile j + 1 reuses the stage of tile j - 1
+      // (two stages), which dQ(j-1) releases, so its copy then overlaps S(j),
+      // dP(j) and the threads' work on j.  (Issuing S(j), dP(j) first kept the
+      // tensor pipe busy during that work but left each copy fully exposed:
+      // 2.567 -> 2.528 ms for the gradient call at L = 4096.)
       for (int j = 0; ok && j <= nt; ++j) {
-        if (NS == 1) {
-          if (j > 0) ok = issue_dq(j - 1);
-          if (ok && j < nt) ok = issue_sdp(j);
-        } else {
-          if (j < nt) ok = issue_sdp(j);
-          if (ok && j > 0) ok = issue_dq(j - 1);
-        }
+        if (j > 0) ok = issue_dq(j - 1);
+        if (ok && j < nt) ok = issue_sdp(j);
       }
       if (!ok && issued_any) {
         umma_commit(bar(QB_DRAIN));
@@ -443,17 +469,20 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         break;
       }
       tc_fence_after();
+      if (tid == 0) BWD_TR(0, j, 5);     // S(j), dP(j) complete
       uint32_t sv[16], dv[16];
       tmem_ld16(tmem + Q_TM_S + 16 * half + lane_off, sv);
       tmem_ld16(tmem + Q_TM_DP + 16 * half + lane_off, dv);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(bar(QB_SFREE));
+      if (tid == 0) BWD_TR(0, j, 6);     // read
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(QB_FULL0 + s), (j / NS) & 1, abort_flag))) {
         if (lane == 0) fail(DEV_TIMEOUT_FULL);
         ok = false;
         break;
       }
+      if (tid == 0) BWD_TR(0, j, 7);     // column terms visible
       const float4 dd = info[2 * s], oj = info[2 * s + 1];
       const float rt = ch * (2.f * fmaf(sq.x, dd.x, fmaf(sq.y, dd.y, sq.z * dd.z)) - pq * dd.w);
       const float base = rt + rd.x;                        // row terms - (w + lse2); -inf on dead rows
@@ -480,11 +509,13 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         ok = false;
         break;
       }
+      if (tid == 0) BWD_TR(0, j, 8);     // dQ(j-1) done with dS
       tc_fence_after();
       tmem_st8(tmem + Q_TM_DS + 8 * half + lane_off, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(QB_DSFULL));
+      if (tid == 0) BWD_TR(0, j, 9);     // dS(j) written
     }
     if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(QB_DSFREE), (nt - 1) & 1, abort_flag))) {
       if (lane == 0) fail(DEV_TIMEOUT_MMA);
@@ -601,7 +632,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
     }
     mbar_init(bar(KB_DRAIN), 1);
     for (int s = 0; s < MAX_NS; ++s) {
-      mbar_init(bar(KB_FULL0 + s), 1);
+      mbar_init(bar(KB_FULL0 + s), 2);   // the copy's expect-tx arrive and the row-term arrive
       mbar_init(bar(KB_EMPTY0 + s), 1);
     }
     *abort_flag = 0;
@@ -632,52 +663,43 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
     const int js0 = 2 * J2, js1 = 2 * J2 + 1;   // the two 64-key origin tiles of this CTA
     const float4 ok0 = a.ok[b * a.nkt + js0];
     const float4 ok1 = js1 < a.nkt ? a.ok[b * a.nkt + js1] : ok0;
+    // As in the query pass: each stage's copy goes out as soon as the stage
+    // is free, the global row values of a tile (its query-tile origin, row
+    // terms and the 32 query points, 12 floats = 3 float4 per query) are
+    // loaded one tile ahead, and FULL completes on the copy and on a second
+    // arrive after they are in shared memory.
     int issued = 0;
+    struct RowVals {
+      float4 oqv, sq, v[3];
+      float2 rd;
+    };
+    auto fetch = [&](int i, RowVals& r) {
+      r.oqv = a.oq[b * a.nqt + (i * BT) / QT];
+      const int qi = i * BT + lane;
+      r.sq = qi < L ? a.rowq[static_cast<int64_t>(bh) * L + qi] : make_float4(0.f, 0.f, 0.f, 0.f);
+      r.rd = qi < L ? a.rowd[static_cast<int64_t>(bh) * L + qi] : make_float2(0.f, 0.f);
+      const float4* src = reinterpret_cast<const float4*>(a.pts) + (static_cast<int64_t>(bh) * L + i * BT) * 6;
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const int f = lane + 32 * u, row = f / 3;
+        r.v[u] = i * BT + row < L ? src[row * 6 + f % 3] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    RowVals nxt;
+    fetch(0, nxt);
     for (int i = 0; i < nq; ++i) {
       const int s = i % NS;
       if (i >= NS) {
         int ok = 1;
         if (lane == 0) ok = mbar_wait_bounded(bar(KB_EMPTY0 + s), ((i / NS) - 1) & 1, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (lane == 0) BWD_TR(1, i, 10);
         if (!ok) {
           if (lane == 0) fail(DEV_TIMEOUT_EMPTY);
           break;
         }
       }
       issued = i + 1;
-      const int Iq = (i * BT) / QT;
-      const float4 oqv = a.oq[b * a.nqt + Iq];
-      const float d0x = ok0.x - oqv.x, d0y = ok0.y - oqv.y, d0z = ok0.z - oqv.z;
-      const float d1x = ok1.x - oqv.x, d1y = ok1.y - oqv.y, d1z = ok1.z - oqv.z;
-      const float n0 = fmaf(d0x, d0x, fmaf(d0y, d0y, d0z * d0z)), n1 = fmaf(d1x, d1x, fmaf(d1y, d1y, d1z * d1z));
-      {
-        const int qi = i * BT + lane;
-        float4 e = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
-        if (qi < L) {
-          const float4 sq = a.rowq[static_cast<int64_t>(bh) * L + qi];
-          const float2 rd = a.rowd[static_cast<int64_t>(bh) * L + qi];
-          const float rt0 = ch * (2.f * fmaf(sq.x, d0x, fmaf(sq.y, d0y, sq.z * d0z)) - pq * n0);
-          const float rt1 = ch * (2.f * fmaf(sq.x, d1x, fmaf(sq.y, d1y, sq.z * d1z)) - pq * n1);
-          e = make_float4(rt0 + rd.x, rt1 + rd.x, rd.y, 0.f);
-        }
-        qinfo[s * BT + lane] = e;
-      }
-      if (lane == 0) oqs[s] = oqv;
-      {
-        // the tile's 32 query points (12 floats = 3 float4 per query): three
-        // independent 16-byte loads per lane, all in flight together
-        float4* qp = reinterpret_cast<float4*>(smem + lay.aux + KA_QPTS) + s * BT * 3;
-        const float4* src = reinterpret_cast<const float4*>(a.pts) + (static_cast<int64_t>(bh) * L + i * BT) * 6;
-        float4 v[3];
-#pragma unroll
-        for (int u = 0; u < 3; ++u) {
-          const int f = lane + 32 * u, row = f / 3;
-          v[u] = i * BT + row < L ? src[row * 6 + f % 3] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int u = 0; u < 3; ++u) qp[lane + 32 * u] = v[u];
-      }
-      __syncwarp();
       if (lane == 0) {
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
         mbar_arrive_expect_tx(bar(KB_FULL0 + s), lay.stg_bytes);
@@ -685,8 +707,33 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         tma_load_3d(st + 4096, &tm_do, bar(KB_FULL0 + s), 0, i * BT, bh);
         tma_load_4d(st + 8192, &tm_qp, bar(KB_FULL0 + s), 0, i * BT, 0, bh);
         tma_load_4d(st + 8192 + np * 4096, &tm_du, bar(KB_FULL0 + s), 0, i * BT, 0, bh);
+        BWD_TR(1, i, 11);
       }
+      const RowVals cur = nxt;
+      if (i + 1 < nq) fetch(i + 1, nxt);
+      const float4 oqv = cur.oqv;
+      const float d0x = ok0.x - oqv.x, d0y = ok0.y - oqv.y, d0z = ok0.z - oqv.z;
+      const float d1x = ok1.x - oqv.x, d1y = ok1.y - oqv.y, d1z = ok1.z - oqv.z;
+      const float n0 = fmaf(d0x, d0x, fmaf(d0y, d0y, d0z * d0z)), n1 = fmaf(d1x, d1x, fmaf(d1y, d1y, d1z * d1z));
+      {
+        float4 e = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
+        if (i * BT + lane < L) {
+          const float4 sq = cur.sq;
+          const float rt0 = ch * (2.f * fmaf(sq.x, d0x, fmaf(sq.y, d0y, sq.z * d0z)) - pq * n0);
+          const float rt1 = ch * (2.f * fmaf(sq.x, d1x, fmaf(sq.y, d1y, sq.z * d1z)) - pq * n1);
+          e = make_float4(rt0 + cur.rd.x, rt1 + cur.rd.x, cur.rd.y, 0.f);
+        }
+        qinfo[s * BT + lane] = e;
+      }
+      if (lane == 0) oqs[s] = oqv;
+      float4* qp = reinterpret_cast<float4*>(smem + lay.aux + KA_QPTS) + s * BT * 3;
+#pragma unroll
+      for (int u = 0; u < 3; ++u) qp[lane + 32 * u] = cur.v[u];
       __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(KB_FULL0 + s));
+        BWD_TR(1, i, 12);
+      }
     }
     if (lane == 0 && *abort_flag) {
       mbar_wait_bounded(bar(KB_KFULL), 0, nullptr, 100000000ull);
@@ -708,7 +755,9 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       auto issue_sdp = [&](int i) -> bool {
         const int s = i % NS, t = i & 1;
         bool w = mbar_wait_bounded(bar(KB_FULL0 + s), (i / NS) & 1, abort_flag);
+        BWD_TR(1, i, 0);
         if (w && i >= 2) w = mbar_wait_bounded(bar(KB_ACC0 + t), ((i - 2) >> 1) & 1, abort_flag);
+        BWD_TR(1, i, 1);
         if (!w) { fail(DEV_TIMEOUT_FULL); return false; }
         tc_fence_after();
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
@@ -725,6 +774,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
           umma_ss(tDP, kd128(sb + lay.z2 + 16384 * (kk >> 2) + 32 * (kk & 3)),
                   kd128(sDU + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
         umma_commit(bar(KB_SFULL0 + t));
+        BWD_TR(1, i, 2);
         issued_any = true;
         return true;
       };
@@ -733,6 +783,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       auto issue_acc = [&](int i) -> bool {
         const int s = i % NS, t = i & 1;
         if (!mbar_wait_bounded(bar(KB_PFULL0 + t), (i >> 1) & 1, abort_flag)) { fail(DEV_TIMEOUT_SOFTMAX); return false; }
+        BWD_TR(1, i, 3);
         tc_fence_after();
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
         const uint32_t sQh = st, sDO = st + 4096, sQP = st + 8192, sDU = st + 8192 + np * 4096;
@@ -747,6 +798,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         }
         umma_commit(bar(KB_ACC0 + t));
         umma_commit(bar(KB_EMPTY0 + s));
+        BWD_TR(1, i, 4);
         return true;
       };
       // with two or more stages S^T / dP^T(i) are issued before the
@@ -796,6 +848,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       // that neither waits at their shared barrier for one that has left
       const int tb = i & 1;                   // tensor-memory buffer of this tile
       const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_SFULL0 + tb), (i >> 1) & 1, abort_flag));
+      if (tid == 0) BWD_TR(1, i, 5);
       uint32_t sv[16], dv[16];
       if (got) {
         tc_fence_after();
@@ -804,6 +857,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         tmem_ld_wait();
         tc_fence_before();
       }
+      if (tid == 0) BWD_TR(1, i, 6);
       if (lane == 0) pair_ok[(i & 1) * 8 + quarter * 2 + half] = got ? 1 : 0;
       named_bar_sync(pair_bar, 64);           // both halves have read before either overwrites
       if (!(pair_ok[(i & 1) * 8 + quarter * 2] && pair_ok[(i & 1) * 8 + quarter * 2 + 1])) {
@@ -816,6 +870,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         ok = false;
         break;
       }
+      if (tid == 0) BWD_TR(1, i, 7);
       const float4 oqv = oqs[s];
       const float colv = ck.w - fmaf(ck.x, okj.x - oqv.x, fmaf(ck.y, okj.y - oqv.y, ck.z * (okj.z - oqv.z)));
       const float4* qi = qinfo + s * BT + 16 * half;
@@ -856,12 +911,14 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       co0 = fmaf(tsum, oqv.x, co0);
       co1 = fmaf(tsum, oqv.y, co1);
       co2 = fmaf(tsum, oqv.z, co2);
+      if (tid == 0) BWD_TR(1, i, 8);
       tc_fence_after();
       tmem_st8(tmem + K_TM_S + 32 * tb + 8 * half + lane_off, pp);
       tmem_st8(tmem + K_TM_DP + 32 * tb + 8 * half + lane_off, pd);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(KB_PFULL0 + tb));
+      if (tid == 0) BWD_TR(1, i, 9);
     }
     // the commit after the last accumulation tracks every earlier MMA of the issuing thread
     if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(KB_ACC0 + ((nq - 1) & 1)), ((nq - 1) >> 1) & 1, abort_flag))) {
@@ -1193,6 +1250,13 @@ int stages_for(uint32_t resident, uint32_t stage, uint32_t aux) {
 }
 
 }  // namespace
+
+#ifdef IPA_TRACE
+bool ipa_bwd_trace_read(void* host, size_t bytes) {
+  if (bytes < sizeof(g_bwd_trace)) return false;
+  return cudaMemcpyFromSymbol(host, g_bwd_trace, sizeof(g_bwd_trace)) == cudaSuccess;
+}
+#endif
 
 IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
