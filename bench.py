@@ -583,11 +583,13 @@ def main():
         outs = {"vectors": torch.empty((2, 2048, 8, 4, 3), device=dev),
                 "output": torch.empty((2, 2048, 256), device=dev),
                 "attention": torch.empty((2, 8, 2048, 2048), device=dev)}
-        res = {}
+        res, resg = {}, {}
         for with_att in (False, True):
             o2 = dict(outs)
             if not with_att:
                 o2["attention"] = None
+            # device time of the call's kernels (CUDA-graph replay), next to the direct call
+            resg[with_att] = timed_graph(torch, lambda o2=o2: gp(gd, out=o2), flush)
             for _ in range(3):
                 gp(gd, out=o2)
             torch.cuda.synchronize()
@@ -604,12 +606,34 @@ def main():
         gp.check()
         pairs = 2 * 8 * 2048 * 2048
         att_bytes = pairs * 4 + pairs * 1          # attention map written + pair mask read
+        map_gbs = att_bytes / ((resg[True] - resg[False]) / 1e3) / 1e9 if resg[True] > resg[False] else None
+        peaks, psrc = measured_peaks()
+        # scores and aggregation: per (i, j, h) 27 fp32-pipe operations (the
+        # direction dot product 3, displacement 3, squared distance 3, score
+        # 4, subtraction of the running maximum 1, row sum 1, 3 M = 12 value
+        # products) and 2 MUFU (square root, exp2); the fp32 pipe bounds it
+        # at 148 SMs x 128 lanes x 1.965 GHz
+        alu_ops = 27
+        alu_peak = 148 * 128 * 1.965e9 / 1e12
+        alu_achieved = pairs * alu_ops / (resg[False] / 1e3) / 1e12
         line["variant"] = {
             "workload": "geometric attention B=2 N=2048 H=8 M=4 Cout=256, 20% pair mask, 5% invalid frames",
-            "ms_no_attention_map": res[False], "ms_with_attention_map": res[True],
-            "pair_heads_per_s": pairs / (res[False] / 1e3),
-            "attention_map_GBps": att_bytes / ((res[True] - res[False]) / 1e3) / 1e9
-            if res[True] > res[False] else None,
+            "ms_no_attention_map": resg[False], "ms_with_attention_map": resg[True],
+            "direct_call_ms": {"no_attention_map": res[False], "with_attention_map": res[True]},
+            "timing": "ms_*: CUDA-graph replay of the call's kernels (device time); direct_call_ms: one "
+                      "call from Python per step, host work included",
+            "pair_heads_per_s": pairs / (resg[False] / 1e3),
+            "attention_map_GBps": map_gbs,
+            "roofline": [
+                {"kernel": "geo_attn_kernel", "bound": "alu", "achieved": alu_achieved, "peak": alu_peak,
+                 "unit": "Top/s (fp32 pipe)", "frac": alu_achieved / alu_peak,
+                 "note": f"{alu_ops} fp32 operations per (query, key, head), 2 MUFU; timed as the whole call "
+                         "without the map (weights, prep and readout kernels included), CUDA-graph replay"},
+                {"kernel": "geo_map_kernel", "bound": "hbm", "achieved": map_gbs, "peak": peaks["hbm_gbs"],
+                 "unit": "GB/s", "frac": map_gbs / peaks["hbm_gbs"] if map_gbs else None,
+                 "peak_source": psrc,
+                 "note": "268 MB map written + 67 MB pair mask read, over the time the map adds to the call"},
+            ],
         }
         # gradients of the variant (forward statistics recomputed inside the call)
         from rna_structure_models_b200.synth import geo_upstream
@@ -617,9 +641,11 @@ def main():
               for k, v in geo_upstream(g["dims"], 1).items()}
         gg = api.GeoGradPlan(2, 2048, 8, 4, 256, device=dev)
         gout = {n: torch.empty(tuple(gd[n].shape), device=dev) for n in api.GEO_GRADS}
-        bres = {}
+        bres, bresg = {}, {}
         for with_ga in (False, True):
             ga = ug["g_attention"] if with_ga else None
+            bresg[with_ga] = timed_graph(torch, lambda ga=ga: gg(gd, ug["g_output"], ga, ug["g_vectors"], out=gout),
+                                         flush, n=10)
             for _ in range(3):
                 gg(gd, ug["g_output"], ga, ug["g_vectors"], out=gout)
             torch.cuda.synchronize()
@@ -634,8 +660,9 @@ def main():
                 times.append(a0.elapsed_time(a1))
             bres[with_ga] = statistics.mean(times)
         line["variant"].update({
-            "backward_ms": bres[False], "backward_ms_with_attention_grad": bres[True],
-            "backward_pair_heads_per_s": pairs / (bres[False] / 1e3),
+            "backward_ms": bresg[False], "backward_ms_with_attention_grad": bresg[True],
+            "backward_direct_call_ms": {"no_attention_grad": bres[False], "with_attention_grad": bres[True]},
+            "backward_pair_heads_per_s": pairs / (bresg[False] / 1e3),
         })
 
     # distance-aware attention of MEET (§2.2) on the same core (B=1, L=4096, H=8)
@@ -658,11 +685,15 @@ def main():
             torch.cuda.synchronize()
             mt.append(a0.elapsed_time(a1))
         mp.check()
-        ms_meet = statistics.mean(mt)
+        ms_meet_direct = statistics.mean(mt)
+        ms_meet = timed_graph(torch, lambda: mp(*[md[n] for n in api.MEET_INPUTS], out=mout), flush)
+        mp.check()
         triples = L * L * 8
         line["meet"] = {
             "workload": f"MEET distance-aware attention B=1 L={L} H=8 C=16 (all four kernels of a call)",
-            "ms": ms_meet, "pair_heads_per_s": triples / (ms_meet / 1e3),
+            "ms": ms_meet, "direct_call_ms": ms_meet_direct,
+            "timing": "ms: CUDA-graph replay of the call's kernels; direct_call_ms: one call from Python per step",
+            "pair_heads_per_s": triples / (ms_meet / 1e3),
             "tflops_algorithmic": triples * 2 * (2 * 16 + 9) / (ms_meet / 1e3) / 1e12,
         }
 
@@ -690,7 +721,8 @@ def main():
                 ts.append(a0.elapsed_time(a1))
             return statistics.mean(ts)
 
-        ms_layer = timed(lambda: mplan(mdev, out=mo))
+        ms_layer_direct = timed(lambda: mplan(mdev, out=mo))
+        ms_layer = timed_graph(torch, lambda: mplan(mdev, out=mo), flush)
         mplan.check()
         width = 12 * (3 * 16 + 3 * (2 * 4 + 8))
         HF = 12 * (16 + 32 + 128)
@@ -698,14 +730,19 @@ def main():
         lin_out = api.LinearPlan(L, HF, 384, device=dev)
         xo = torch.randn((L, HF), device=dev)
         wo = torch.randn((HF, 384), device=dev)
-        ms_in = timed(lambda: lin_in(mdev["s"].view(L, 384), mdev["w_in"], mdev["b_in"]))
-        ms_out = timed(lambda: lin_out(xo, wo, mdev["b_out"]))
+        ms_in_direct = timed(lambda: lin_in(mdev["s"].view(L, 384), mdev["w_in"], mdev["b_in"]))
+        ms_out_direct = timed(lambda: lin_out(xo, wo, mdev["b_out"]))
+        ms_in = timed_graph(torch, lambda: lin_in(mdev["s"].view(L, 384), mdev["w_in"], mdev["b_in"]), flush)
+        ms_out = timed_graph(torch, lambda: lin_out(xo, wo, mdev["b_out"]), flush)
         lin_in.check()
         lin_out.check()
         f_in, f_out = 2.0 * L * 384 * width, 2.0 * L * HF * 384
         line["layer"] = {
             "workload": f"IPA layer B=1 L={L} H=12 Cz=128 c_s=384: input projection, core, output projection",
             "ms": ms_layer,
+            "direct_call_ms": {"layer": ms_layer_direct, "linear_in": ms_in_direct, "linear_out": ms_out_direct},
+            "timing": "ms and linear_*_ms: CUDA-graph replay of the calls' kernels (device time); "
+                      "direct_call_ms: one call from Python per step, host work (tensor-map encoding) included",
             "linear_in_ms": ms_in, "linear_in_tflops": f_in / (ms_in / 1e3) / 1e12,
             "linear_out_ms": ms_out, "linear_out_tflops": f_out / (ms_out / 1e3) / 1e12,
             "linear_note": "each call packs x and W to fp16 (two kernels) before the tcgen05 GEMM",

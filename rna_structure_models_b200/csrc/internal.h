@@ -101,7 +101,7 @@ cudaError_t meet_launch_extract(const float* core_out, float* out, int64_t rows,
 
 // Dense projection y = x W + b (tcgen05, fp16 operands, fp32 accumulation).
 struct LinearWorkspace {
-  size_t x16, w16, total;
+  size_t x16, w16, w32, total;
 };
 LinearWorkspace linear_workspace_layout(int M, int K, int N);
 
