@@ -745,7 +745,8 @@ def main():
                       "direct_call_ms: one call from Python per step, host work (tensor-map encoding) included",
             "linear_in_ms": ms_in, "linear_in_tflops": f_in / (ms_in / 1e3) / 1e12,
             "linear_out_ms": ms_out, "linear_out_tflops": f_out / (ms_out / 1e3) / 1e12,
-            "linear_note": "each call packs x and W to fp16 (two kernels) before the tcgen05 GEMM",
+            "linear_note": "tf32 tcgen05 GEMM on the caller's fp32 x (TMA); each call transposes W to fp32 W^T "
+                           "(one small kernel) first",
         }
 
     # secondary sections: a failure there is reported in the line and does not
