@@ -62,53 +62,52 @@ struct GvecArgs {
   int* err;
 };
 
-// g_vec = g_vectors + [row live] g_output W^T.  Block: 32 k-columns x 8 row
-// groups; each thread covers 4 rows of one column.
+// g_vec = g_vectors + [row live] g_output W^T: a 64-row x 32-column tile of
+// g_vec per block (tile_product over the Cout columns of g_output); rows with
+// no live head pass no g_output on.
+constexpr int GV_TM = 64, GV_TN = 32;
 __global__ void __launch_bounds__(256) geo_gvec_kernel(const GvecArgs a) {
-  const int kx = blockIdx.y * 32 + threadIdx.x;
+  __shared__ int64_t goff[GV_TM];   // g_output offset of each row, -1 if it passes nothing on
   const int64_t rows = static_cast<int64_t>(a.B) * a.N;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32 + threadIdx.y * 4;
-  bool lv[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int64_t row = row0 + q;
-    bool l = false;
+  const int r0 = blockIdx.x * GV_TM, c0 = blockIdx.y * GV_TN;
+  if (threadIdx.x < GV_TM) {
+    const int64_t row = r0 + static_cast<int>(threadIdx.x);
+    int l = 0;
     if (row < rows)
       for (int h = 0; h < a.H; ++h) l |= a.live[row * a.H + h] != 0;
-    lv[q] = l;
-    if (blockIdx.y == 0 && threadIdx.x == 0 && row < rows) *IPA_AT(a.rowlive, row, rows, a.err) = l ? 1 : 0;
+    const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
+    goff[threadIdx.x] = (row < rows && l) ? b * a.g_output.s[0] + n * a.g_output.s[1] : -1;
+    if (blockIdx.y == 0 && row < rows) *IPA_AT(a.rowlive, row, rows, a.err) = l ? 1 : 0;
   }
-  if (kx >= a.HM3) return;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  int64_t go[4];   // g_output offset of each row (its live rows only)
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int64_t row = row0 + q;
-    go[q] = -1;
-    if (row < rows && lv[q]) {
-      const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
-      go[q] = b * a.g_output.s[0] + n * a.g_output.s[1];
-    }
-  }
+  __syncthreads();
   const int64_t sc = a.g_output.s[2];
-  for (int c = 0; c < a.Cout; ++c) {
-    const float w = a.wt[static_cast<int64_t>(c) * a.HM3 + kx];
+  float acc[GV_TM / 16][GV_TN / 16];
+  tile_product<GV_TM, GV_TN>(
+      r0, c0, a.Cout,
+      [&](int r, int c) {
+        const int64_t off = goff[r - r0];
+        return (c < a.Cout && off >= 0) ? ldf(a.g_output, off + c * sc) : 0.f;
+      },
+      [&](int c, int kx) { return (c < a.Cout && kx < a.HM3) ? a.wt[static_cast<int64_t>(c) * a.HM3 + kx] : 0.f; },
+      acc);
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (go[q] >= 0) acc[q] = fmaf(ldf(a.g_output, go[q] + c * sc), w, acc[q]);
-  }
-  const int h = kx / (a.HM3 / a.H), mx = kx % (a.HM3 / a.H), m = mx / 3, x = mx % 3;
+  for (int j = 0; j < GV_TN / 16; ++j) {
+    const int kx = c0 + tx + 16 * j;
+    if (kx >= a.HM3) continue;
+    const int h = kx / (a.HM3 / a.H), mx = kx % (a.HM3 / a.H), m = mx / 3, x = mx % 3;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int64_t row = row0 + q;
-    if (row >= rows) continue;
-    float g = acc[q];
-    if (a.has_g_vectors) {
-      const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
-      const View& v = a.g_vectors;
-      g += ldf(v, b * v.s[0] + n * v.s[1] + h * v.s[2] + m * v.s[3] + x * v.s[4]);
+    for (int i = 0; i < GV_TM / 16; ++i) {
+      const int64_t row = r0 + ty + 16 * i;
+      if (row >= rows) continue;
+      float g = acc[i][j];
+      if (a.has_g_vectors) {
+        const int b = static_cast<int>(row / a.N), n = static_cast<int>(row % a.N);
+        const View& v = a.g_vectors;
+        g += ldf(v, b * v.s[0] + n * v.s[1] + h * v.s[2] + m * v.s[3] + x * v.s[4]);
+      }
+      *IPA_AT(a.gvec, row * a.HM3 + kx, rows * a.HM3, a.err) = g;
     }
-    *IPA_AT(a.gvec, row * a.HM3 + kx, rows * a.HM3, a.err) = g;
   }
 }
 
@@ -146,7 +145,7 @@ __global__ void __launch_bounds__(256) geo_dagg_kernel(const DaggArgs a) {
   *IPA_AT(a.rowinfo, row, nbhn, a.err) = make_float4(0.f, 0.f, d1, 0.f);
 }
 
-constexpr int DW_ROWS = 128, DW_K = 32;
+constexpr int DW_ROWS = 128;
 
 struct DwArgs {
   int64_t rows;
@@ -161,19 +160,15 @@ struct DwArgs {
   int* err;
 };
 
-// Partial dW over one chunk of 128 rows: a thread owns one output column c
-// and 32 rows k of W; the chunk's vec values sit in shared memory.
+// Partial dW over one chunk of 128 rows: the 32 x 64 tile (k, c) of
+// vec^T g_output summed over the chunk's rows in order (tile_product, rows
+// that pass nothing on contribute zeros); the first k tile also sums the
+// chunk's g_output rows for db.
+constexpr int DW_TM = 32, DW_TN = 64;
 __global__ void __launch_bounds__(256) geo_dw_part_kernel(const DwArgs a) {
-  __shared__ float vs[DW_ROWS][DW_K];
   __shared__ int64_t goff[DW_ROWS];   // g_output offset of each row, -1 if it passes nothing on
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  const int k0 = blockIdx.y * DW_K;
+  const int k0 = blockIdx.x * DW_TM, c0 = blockIdx.y * DW_TN;
   const int64_t r0 = static_cast<int64_t>(blockIdx.z) * DW_ROWS;
-  for (int e = threadIdx.x; e < DW_ROWS * DW_K; e += blockDim.x) {
-    const int rr = e / DW_K, kk = e % DW_K;
-    const int64_t row = r0 + rr;
-    vs[rr][kk] = (row < a.rows && k0 + kk < a.HM3) ? a.vec[row * a.HM3 + k0 + kk] : 0.f;
-  }
   for (int rr = threadIdx.x; rr < DW_ROWS; rr += blockDim.x) {
     const int64_t row = r0 + rr;
     int64_t off = -1;
@@ -184,25 +179,33 @@ __global__ void __launch_bounds__(256) geo_dw_part_kernel(const DwArgs a) {
     goff[rr] = off;
   }
   __syncthreads();
-  if (c >= a.Cout) return;
-  float acc[DW_K], accb = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < DW_K; ++kk) acc[kk] = 0.f;
-  const int64_t sc = static_cast<int64_t>(c) * a.g_output.s[2];
-  for (int rr = 0; rr < DW_ROWS; ++rr) {
-    if (goff[rr] < 0) continue;
-    const float g = ldf(a.g_output, goff[rr] + sc);
-    accb += g;
-#pragma unroll
-    for (int kk = 0; kk < DW_K; ++kk) acc[kk] = fmaf(vs[rr][kk], g, acc[kk]);
-  }
+  const int64_t sc = a.g_output.s[2];
+  float acc[DW_TM / 16][DW_TN / 16];
+  tile_product<DW_TM, DW_TN>(
+      k0, c0, DW_ROWS,
+      [&](int k, int rr) { return (k < a.HM3 && r0 + rr < a.rows) ? a.vec[(r0 + rr) * a.HM3 + k] : 0.f; },
+      [&](int rr, int c) { return (c < a.Cout && goff[rr] >= 0) ? ldf(a.g_output, goff[rr] + c * sc) : 0.f; },
+      acc);
   const int64_t nwc = static_cast<int64_t>(a.HM3) * a.Cout;
   const int64_t pw0 = static_cast<int64_t>(blockIdx.z) * nwc;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 #pragma unroll
-  for (int kk = 0; kk < DW_K; ++kk)
-    if (k0 + kk < a.HM3) *IPA_AT(a.part_w, pw0 + static_cast<int64_t>(k0 + kk) * a.Cout + c, a.nchunk * nwc, a.err) = acc[kk];
-  if (blockIdx.y == 0)
+  for (int i = 0; i < DW_TM / 16; ++i) {
+    const int k = k0 + ty + 16 * i;
+    if (k >= a.HM3) continue;
+#pragma unroll
+    for (int j = 0; j < DW_TN / 16; ++j) {
+      const int c = c0 + tx + 16 * j;
+      if (c < a.Cout) *IPA_AT(a.part_w, pw0 + static_cast<int64_t>(k) * a.Cout + c, a.nchunk * nwc, a.err) = acc[i][j];
+    }
+  }
+  if (blockIdx.x == 0 && threadIdx.x < DW_TN && c0 + static_cast<int>(threadIdx.x) < a.Cout) {
+    const int c = c0 + threadIdx.x;
+    float accb = 0.f;
+    for (int rr = 0; rr < DW_ROWS; ++rr)
+      if (goff[rr] >= 0) accb += ldf(a.g_output, goff[rr] + c * sc);
     *IPA_AT(a.part_b, static_cast<int64_t>(blockIdx.z) * a.Cout + c, static_cast<int64_t>(a.nchunk) * a.Cout, a.err) = accb;
+  }
 }
 
 // dW and db: the chunk partials summed in a fixed order (deterministic).
@@ -706,7 +709,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   ga.gvec = reinterpret_cast<float*>(ws + w.gvec);
   ga.rowlive = ws + w.rowlive;
   ga.err = a.f.err;
-  geo_gvec_kernel<<<dim3(static_cast<unsigned>((rows + 31) / 32), (HM3 + 31) / 32), dim3(32, 8), 0, st>>>(ga);
+  geo_gvec_kernel<<<dim3(static_cast<unsigned>((rows + GV_TM - 1) / GV_TM), (HM3 + GV_TN - 1) / GV_TN), 256, 0, st>>>(ga);
 
   DaggArgs da{};
   da.B = B; da.N = N; da.H = H; da.M = M; da.VW = VW; da.HM3 = HM3;
@@ -726,7 +729,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   dw.part_b = reinterpret_cast<float*>(ws + w.dbpart);
   dw.d_w = a.d_output_weight; dw.d_b = a.d_output_bias;
   dw.err = a.f.err;
-  geo_dw_part_kernel<<<dim3((Cout + 255) / 256, (HM3 + DW_K - 1) / DW_K, dw.nchunk), 256, 0, st>>>(dw);
+  geo_dw_part_kernel<<<dim3((HM3 + DW_TM - 1) / DW_TM, (Cout + DW_TN - 1) / DW_TN, dw.nchunk), 256, 0, st>>>(dw);
   {
     int64_t n = static_cast<int64_t>(HM3) * Cout;
     geo_dw_sum_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(dw);

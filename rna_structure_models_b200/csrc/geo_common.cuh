@@ -55,5 +55,69 @@ __device__ __forceinline__ float geo_score(const float4 q0, const float4 q1, con
   return geo_pair(q0, q1, k0, k1, A, Bd).s;
 }
 
+// Register-tiled fp32 product on the CUDA cores for the small dense products
+// of the variant (the readout, and the two products of its gradient): a
+// 256-thread block computes the TM x TN tile at (r0, c0) of C = A B.  Thread
+// (ty, tx) = (tid / 16, tid % 16) owns rows r0 + ty + 16 i and columns
+// c0 + tx + 16 j.  K is staged 32 at a time in shared memory (A transposed,
+// so that a k-column of the tile is contiguous); the next 32 are loaded into
+// registers while the current ones are multiplied.  Every output accumulates
+// fmaf(a_k, b_k, acc) in increasing k, the order of a plain loop over k.
+// load_a(r, k) and load_b(k, c) return the operands, 0 outside the matrices.
+template <int TM, int TN, class LoadA, class LoadB>
+__device__ __forceinline__ void tile_product(int r0, int c0, int K, LoadA load_a, LoadB load_b,
+                                             float (&acc)[TM / 16][TN / 16]) {
+  static_assert(TM % 16 == 0 && TN % 16 == 0 && TM <= 64 && TN <= 64, "tile of 16-multiples up to 64");
+  constexpr int NA = 32 * TM / 256, NB = 32 * TN / 256;   // staged values per thread
+  __shared__ float As[32][TM + 1];
+  __shared__ float Bs[32][TN + 1];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+#pragma unroll
+  for (int i = 0; i < TM / 16; ++i)
+#pragma unroll
+    for (int j = 0; j < TN / 16; ++j) acc[i][j] = 0.f;
+  float ra[NA], rb[NB];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < NA; ++u) {   // A[r0 + r][k0 + k], k fastest across threads
+      const int e = tid + 256 * u, r = e >> 5, k = e & 31;
+      ra[u] = load_a(r0 + r, k0 + k);
+    }
+#pragma unroll
+    for (int u = 0; u < NB; ++u) {   // B[k0 + k][c0 + c], c fastest
+      const int e = tid + 256 * u, k = e / TN, c = e % TN;
+      rb[u] = load_b(k0 + k, c0 + c);
+    }
+  };
+  fetch(0);
+  for (int k0 = 0; k0 < K; k0 += 32) {
+#pragma unroll
+    for (int u = 0; u < NA; ++u) {
+      const int e = tid + 256 * u;
+      As[e & 31][e >> 5] = ra[u];
+    }
+#pragma unroll
+    for (int u = 0; u < NB; ++u) {
+      const int e = tid + 256 * u;
+      Bs[e / TN][e % TN] = rb[u];
+    }
+    __syncthreads();
+    if (k0 + 32 < K) fetch(k0 + 32);
+    const int kn = K - k0 < 32 ? K - k0 : 32;
+    for (int k = 0; k < kn; ++k) {
+      float av[TM / 16], bv[TN / 16];
+#pragma unroll
+      for (int i = 0; i < TM / 16; ++i) av[i] = As[k][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < TN / 16; ++j) bv[j] = Bs[k][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < TM / 16; ++i)
+#pragma unroll
+        for (int j = 0; j < TN / 16; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace geo
 }  // namespace fipa

@@ -509,39 +509,39 @@ struct ReadArgs {
   int* err;
 };
 
-constexpr int RD_ROWS = 32;
+constexpr int RD_TM = 64, RD_TN = 64;
 
+// out[row, :] = vec[row, :] W + b over a 64 x 64 tile per block; rows whose
+// heads all lacked an allowed key are forced to 0.
 __global__ void __launch_bounds__(256) geo_readout_kernel(const ReadArgs a) {
-  extern __shared__ float vs[];  // [RD_ROWS][HM3]
-  __shared__ int any_live[RD_ROWS];
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * RD_ROWS;
+  __shared__ int any_live[RD_TM];
   const int64_t nrows = static_cast<int64_t>(a.B) * a.N;
-  for (int t = threadIdx.x; t < RD_ROWS * a.HM3; t += blockDim.x) {
-    const int rr = t / a.HM3, k = t % a.HM3;
-    vs[t] = row0 + rr < nrows ? a.vec[(row0 + rr) * a.HM3 + k] : 0.f;
-  }
-  if (threadIdx.x < RD_ROWS) {
+  const int r0 = blockIdx.x * RD_TM, c0 = blockIdx.y * RD_TN;
+  if (threadIdx.x < RD_TM) {
     int anyl = 0;
-    if (row0 + threadIdx.x < nrows)
-      for (int h = 0; h < a.H; ++h) anyl |= a.live[(row0 + threadIdx.x) * a.H + h];
+    const int64_t row = r0 + static_cast<int>(threadIdx.x);
+    if (row < nrows)
+      for (int h = 0; h < a.H; ++h) anyl |= a.live[row * a.H + h];
     any_live[threadIdx.x] = anyl;
   }
-  __syncthreads();
-  const int col = blockIdx.y * blockDim.x + threadIdx.x;
-  if (col >= a.Cout) return;
-  float acc[RD_ROWS];
+  float acc[RD_TM / 16][RD_TN / 16];
+  tile_product<RD_TM, RD_TN>(
+      r0, c0, a.HM3,
+      [&](int r, int k) { return (r < nrows && k < a.HM3) ? a.vec[static_cast<int64_t>(r) * a.HM3 + k] : 0.f; },
+      [&](int k, int c) { return (k < a.HM3 && c < a.Cout) ? a.wf[static_cast<int64_t>(k) * a.Cout + c] : 0.f; },
+      acc);
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 #pragma unroll
-  for (int rr = 0; rr < RD_ROWS; ++rr) acc[rr] = 0.f;
-  for (int k = 0; k < a.HM3; ++k) {
-    const float w = a.wf[static_cast<int64_t>(k) * a.Cout + col];
+  for (int i = 0; i < RD_TM / 16; ++i) {
+    const int64_t row = r0 + ty + 16 * i;
+    if (row >= nrows) continue;
 #pragma unroll
-    for (int rr = 0; rr < RD_ROWS; ++rr) acc[rr] = fmaf(vs[rr * a.HM3 + k], w, acc[rr]);
-  }
-  const float bias = a.bf[col];
-#pragma unroll
-  for (int rr = 0; rr < RD_ROWS; ++rr) {
-    const int64_t row = row0 + rr;
-    if (row < nrows) *IPA_AT(a.out, row * a.Cout + col, nrows * a.Cout, a.err) = any_live[rr] ? acc[rr] + bias : 0.f;
+    for (int j = 0; j < RD_TN / 16; ++j) {
+      const int col = c0 + tx + 16 * j;
+      if (col < a.Cout)
+        *IPA_AT(a.out, row * a.Cout + col, nrows * a.Cout, a.err) =
+            any_live[ty + 16 * i] ? acc[i][j] + a.bf[col] : 0.f;
+    }
   }
 }
 
@@ -657,14 +657,8 @@ cudaError_t geo_launch_all(const GeoLaunch& a, cudaStream_t st) {
   ra.err = a.err;
   {
     const int64_t rows = static_cast<int64_t>(a.B) * a.N;
-    dim3 grid(static_cast<unsigned>((rows + RD_ROWS - 1) / RD_ROWS), (a.Cout + 255) / 256);
-    const size_t smem = static_cast<size_t>(RD_ROWS) * a.HM3 * sizeof(float);
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(geo_readout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-    }
-    geo_readout_kernel<<<grid, 256, smem, st>>>(ra);
+    dim3 grid(static_cast<unsigned>((rows + RD_TM - 1) / RD_TM), static_cast<unsigned>((a.Cout + RD_TN - 1) / RD_TN));
+    geo_readout_kernel<<<grid, 256, 0, st>>>(ra);
   }
   return cudaGetLastError();
 }
