@@ -546,58 +546,70 @@ struct FrameArgs {
   int* err;
 };
 
+// Block: rb = 128 / H residues x all heads, thread (residue, head): the
+// local-frame gradients of its head's inputs and that head's terms of the
+// frame gradient, which are then summed over heads in order (through shared
+// memory) into d R and d t of the residue.  Block 0 also finishes the two
+// scale gradients.
 __global__ void __launch_bounds__(128) geo_bwd_frame_kernel(const FrameArgs a) {
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  __shared__ float fterm[128 * 12];   // [rb][H][12]: d R (9), d t (3) per head
+  const int H = a.H, rb = 128 / H;
+  const int il = threadIdx.x / H, h = threadIdx.x % H;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.N;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * rb + il;
+  const bool active = il < rb && t < rows;
   if (blockIdx.x == 0)
-    for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+    for (int hh = threadIdx.x; hh < H; hh += blockDim.x) {
       // d scale = dA sigmoid(scale); dA = sum ds dot / sqrt3, dB = -sum ds dist / sqrt3
-      const float xd = ldf(a.dscale, h * a.dscale.s[0]), xx = ldf(a.xscale, h * a.xscale.s[0]);
+      const float xd = ldf(a.dscale, hh * a.dscale.s[0]), xx = ldf(a.xscale, hh * a.xscale.s[0]);
       double sd = 0.0, sx = 0.0;   // fixed summation order: batch, row block, warp
       for (int b = 0; b < a.B; ++b)
         for (int k = 0; k < a.nrb * 4; ++k) {
-          const int64_t slot = ((static_cast<int64_t>(b) * a.H + h) * a.nrb * 4 + k) * 2;
+          const int64_t slot = ((static_cast<int64_t>(b) * H + hh) * a.nrb * 4 + k) * 2;
           sd += a.acc[slot];
           sx += a.acc[slot + 1];
         }
-      *IPA_AT(a.d_dscale, h, a.H, a.err) = static_cast<float>(sd) * kInvSqrt3 / (1.f + expf(-xd));
-      *IPA_AT(a.d_xscale, h, a.H, a.err) = -static_cast<float>(sx) * kInvSqrt3 / (1.f + expf(-xx));
+      *IPA_AT(a.d_dscale, hh, H, a.err) = static_cast<float>(sd) * kInvSqrt3 / (1.f + expf(-xd));
+      *IPA_AT(a.d_xscale, hh, H, a.err) = -static_cast<float>(sx) * kInvSqrt3 / (1.f + expf(-xx));
     }
-  if (t >= static_cast<int64_t>(a.B) * a.N) return;
-  const int b = static_cast<int>(t / a.N), n = static_cast<int>(t % a.N);
-  const float* R = a.rotf + t * 9;
-  float dR[9], dT[3] = {0.f, 0.f, 0.f};
+  if (active) {
+    const int b = static_cast<int>(t / a.N), n = static_cast<int>(t % a.N);
+    const float* R = a.rotf + t * 9;
+    float Rm[9];
 #pragma unroll
-  for (int e = 0; e < 9; ++e) dR[e] = 0.f;
-  // local gradient R^T g and dR += g x^T for one rotated 3-vector x
-  auto back = [&](const float g[3], const View& v, int64_t base, int64_t sx, float* out) {
-    const float x0 = ldf(v, base), x1 = ldf(v, base + sx), x2 = ldf(v, base + 2 * sx);
+    for (int e = 0; e < 9; ++e) Rm[e] = R[e];
+    float dR[9], dT[3];
 #pragma unroll
-    for (int y = 0; y < 3; ++y) out[y] = fmaf(R[y], g[0], fmaf(R[3 + y], g[1], R[6 + y] * g[2]));
+    for (int e = 0; e < 9; ++e) dR[e] = 0.f;
+    // local gradient R^T g and dR += g x^T for one rotated 3-vector x
+    auto back = [&](const float g[3], const View& v, int64_t base, int64_t sx, float* out) {
+      const float x0 = ldf(v, base), x1 = ldf(v, base + sx), x2 = ldf(v, base + 2 * sx);
 #pragma unroll
-    for (int x = 0; x < 3; ++x) {
-      dR[3 * x] = fmaf(g[x], x0, dR[3 * x]);
-      dR[3 * x + 1] = fmaf(g[x], x1, dR[3 * x + 1]);
-      dR[3 * x + 2] = fmaf(g[x], x2, dR[3 * x + 2]);
-    }
-  };
-  for (int h = 0; h < a.H; ++h) {
-    const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.N + n;
-    const int64_t o3 = (t * a.H + h) * 3;
+      for (int y = 0; y < 3; ++y) out[y] = fmaf(Rm[y], g[0], fmaf(Rm[3 + y], g[1], Rm[6 + y] * g[2]));
+#pragma unroll
+      for (int x = 0; x < 3; ++x) {
+        dR[3 * x] = fmaf(g[x], x0, dR[3 * x]);
+        dR[3 * x + 1] = fmaf(g[x], x1, dR[3 * x + 1]);
+        dR[3 * x + 2] = fmaf(g[x], x2, dR[3 * x + 2]);
+      }
+    };
+    const int64_t row = (static_cast<int64_t>(b) * H + h) * a.N + n;
+    const int64_t o3 = (t * H + h) * 3;
     const float4 q0 = a.dq[2 * row], q1 = a.dq[2 * row + 1], k0 = a.dk[2 * row], k1 = a.dk[2 * row + 1];
     const float gqd[3] = {q0.x, q0.y, q0.z}, gqp[3] = {q1.x, q1.y, q1.z};
     const float gkd[3] = {k0.x, k0.y, k0.z}, gkp[3] = {k1.x, k1.y, k1.z};
-    const int64_t n3 = static_cast<int64_t>(a.B) * a.N * a.H * 3;
+    const int64_t n3 = rows * H * 3;
     back(gqd, a.qd, b * a.qd.s[0] + n * a.qd.s[1] + h * a.qd.s[2], a.qd.s[3], IPA_SPAN(a.d_qd, o3, 3, n3, a.err));
     back(gkd, a.kd, b * a.kd.s[0] + n * a.kd.s[1] + h * a.kd.s[2], a.kd.s[3], IPA_SPAN(a.d_kd, o3, 3, n3, a.err));
     back(gqp, a.qp, b * a.qp.s[0] + n * a.qp.s[1] + h * a.qp.s[2], a.qp.s[3], IPA_SPAN(a.d_qp, o3, 3, n3, a.err));
     back(gkp, a.kp, b * a.kp.s[0] + n * a.kp.s[1] + h * a.kp.s[2], a.kp.s[3], IPA_SPAN(a.d_kp, o3, 3, n3, a.err));
 #pragma unroll
-    for (int x = 0; x < 3; ++x) dT[x] += gqp[x] + gkp[x];
+    for (int x = 0; x < 3; ++x) dT[x] = gqp[x] + gkp[x];
     for (int m = 0; m < a.M; ++m) {
       const float* dv = a.dvr + row * a.VW + 3 * m;
       const float gv[3] = {dv[0], dv[1], dv[2]};
       back(gv, a.val, b * a.val.s[0] + n * a.val.s[1] + h * a.val.s[2] + m * a.val.s[3], a.val.s[4],
-           IPA_SPAN(a.d_val, (t * a.H + h) * a.VW + 3 * m, 3, static_cast<int64_t>(a.B) * a.N * a.H * a.VW, a.err));
+           IPA_SPAN(a.d_val, (t * H + h) * a.VW + 3 * m, 3, rows * H * a.VW, a.err));
       // vectors = R^T agg: dR += agg g_vec^T
       const float* ag = a.agg + row * a.VW + 3 * m;
       const float* gq = a.gvec + t * a.HM3 + h * a.VW + 3 * m;
@@ -606,13 +618,23 @@ __global__ void __launch_bounds__(128) geo_bwd_frame_kernel(const FrameArgs a) {
 #pragma unroll
         for (int y = 0; y < 3; ++y) dR[3 * x + y] = fmaf(ag[x], gq[y], dR[3 * x + y]);
     }
+    float* ft = fterm + (il * H + h) * 12;
+#pragma unroll
+    for (int e = 0; e < 9; ++e) ft[e] = dR[e];
+#pragma unroll
+    for (int x = 0; x < 3; ++x) ft[9 + x] = dT[x];
   }
-  float* drot = IPA_SPAN(a.d_rot, t * 9, 9, static_cast<int64_t>(a.B) * a.N * 9, a.err);
-  float* dtr = IPA_SPAN(a.d_trans, t * 3, 3, static_cast<int64_t>(a.B) * a.N * 3, a.err);
-#pragma unroll
-  for (int e = 0; e < 9; ++e) drot[e] = dR[e];
-#pragma unroll
-  for (int x = 0; x < 3; ++x) dtr[x] = dT[x];
+  __syncthreads();
+  // sums over heads in order, one (residue, entry) per thread
+  for (int e = threadIdx.x; e < rb * 12; e += blockDim.x) {
+    const int r = e / 12, k = e % 12;
+    const int64_t tr = static_cast<int64_t>(blockIdx.x) * rb + r;
+    if (tr >= rows) continue;
+    float sum = 0.f;
+    for (int hh = 0; hh < H; ++hh) sum += fterm[(r * H + hh) * 12 + k];
+    if (k < 9) *IPA_AT(a.d_rot, tr * 9 + k, rows * 9, a.err) = sum;
+    else *IPA_AT(a.d_trans, tr * 3 + (k - 9), rows * 3, a.err) = sum;
+  }
 }
 
 struct TransposeArgs {
@@ -776,7 +798,7 @@ cudaError_t geo_launch_bwd(const GeoBwdLaunch& a, cudaStream_t st) {
   fa.d_val = a.d_values; fa.d_rot = a.d_rotation; fa.d_trans = a.d_translation;
   fa.d_dscale = a.d_direction_scale; fa.d_xscale = a.d_distance_scale;
   fa.err = a.f.err;
-  geo_bwd_frame_kernel<<<static_cast<unsigned>((rows + 127) / 128), 128, 0, st>>>(fa);
+  geo_bwd_frame_kernel<<<static_cast<unsigned>((rows + 128 / H - 1) / (128 / H)), 128, 0, st>>>(fa);
   return cudaGetLastError();
 }
 
