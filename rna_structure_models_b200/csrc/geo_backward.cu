@@ -372,8 +372,18 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_ro
       const float p = ex2(g.s - m) * inv;
       if (p == 0.f) continue;
       float da = a.has_g_att ? gst[r * GP + k] : 0.f;
+      {
+        // the key's V rotated values as 16-byte loads (rows of SW floats, SW % 4 == 0)
+        const float4* kv = reinterpret_cast<const float4*>(kk + 8);
 #pragma unroll
-      for (int e = 0; e < V; ++e) da = fmaf(dg[e], kk[8 + e], da);
+        for (int e4 = 0; e4 < (V + 3) / 4; ++e4) {
+          const float4 w = kv[e4];
+          const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (4 * e4 + u < V) da = fmaf(dg[4 * e4 + u], wv[u], da);
+        }
+      }
       const float ds = p * (da - D);
       cq[0] = fmaf(ds, k0.x, cq[0]);
       cq[1] = fmaf(ds, k0.y, cq[1]);
@@ -489,8 +499,15 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_co
       const float p = ex2(g.s - info.x) * info.y;
       if (p == 0.f) continue;
       float da = a.has_g_att ? g_att_at(a, b, h, i, j) : 0.f;
+      // the query's V dagg values as 16-byte loads (rows of SW floats, SW % 4 == 0)
+      float dq[(V + 3) & ~3];
 #pragma unroll
-      for (int e = 0; e < V; ++e) da = fmaf(qq[12 + e], vr[e], da);
+      for (int e4 = 0; e4 < (V + 3) / 4; ++e4) {
+        const float4 w = reinterpret_cast<const float4*>(qq + 12)[e4];
+        dq[4 * e4] = w.x; dq[4 * e4 + 1] = w.y; dq[4 * e4 + 2] = w.z; dq[4 * e4 + 3] = w.w;
+      }
+#pragma unroll
+      for (int e = 0; e < V; ++e) da = fmaf(dq[e], vr[e], da);
       const float ds = p * (da - info.z);
       ck[0] = fmaf(ds, q0.x, ck[0]);
       ck[1] = fmaf(ds, q0.y, ck[1]);
@@ -500,7 +517,7 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_co
       cp[1] = fmaf(ru, g.dy, cp[1]);
       cp[2] = fmaf(ru, g.dz, cp[2]);
 #pragma unroll
-      for (int e = 0; e < V; ++e) dv[e] = fmaf(p, qq[12 + e], dv[e]);
+      for (int e = 0; e < V; ++e) dv[e] = fmaf(p, dq[e], dv[e]);
     }
   }
   __syncthreads();
