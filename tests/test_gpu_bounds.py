@@ -116,6 +116,21 @@ def test_ipa_forward_training_and_gradients(cuda_device, L, Cz):
     assert_same(*both_builds(run), "ipa")
 
 
+def test_ipa_production_width_at_length_2048(cuda_device):
+    """The pair kernel's production shape (R Cz = 256, TMA output pass) and
+    the gradient passes at a length spanning many tiles, in both builds."""
+    inp = ipa_inputs(IpaDims(B=1, L=2048, H=4, Cz=128), 31)
+    inp["mask"][0, 2000:] = False
+    dev = to_dev({k: inp[k] for k in api.IPA_INPUTS})
+
+    def run():
+        o, lse, u = api.ipa_attn_train(dev)
+        g_out = torch.randn(o.shape, device="cuda", generator=torch.Generator(device="cuda").manual_seed(5))
+        return {"train": [o, lse, u], "grads": api.ipa_attn_backward(dev, o, lse, u, g_out)}
+
+    assert_same(*both_builds(run), "ipa L=2048")
+
+
 @pytest.mark.parametrize("N", [1, 65, 383])
 def test_variant_forward_and_gradients(cuda_device, N):
     dims = GeoDims(B=2, N=N, H=3, M=4, Cout=40)
