@@ -609,10 +609,10 @@ ipa_status_t meet_attn_fwd(const meet_params_t* p, const ipa_tensor_t* q, const 
   m.gamma = reinterpret_cast<float*>(ws + lay.gamma);
   m.consts = reinterpret_cast<float*>(ws + lay.consts);
 
-  // the IPA problem: C = 16, Pq = 4, Pv = 8, R = 1, Cz = 16; w_L = 1,
-  // w_C = 1/2, scalar scale 1
+  // the IPA problem: C = 16, Pq = 4, Pv = 8, no pair block (R = 0 factors of
+  // width 16); w_L = 1, w_C = 1/2, scalar scale 1
   IpaLaunch a{};
-  a.B = p->B; a.L = p->L; a.H = p->H; a.C = MEET_C; a.Pq = IPA_PQ; a.Pv = IPA_PV; a.R = 1; a.Cz = MEET_RCZ;
+  a.B = p->B; a.L = p->L; a.H = p->H; a.C = MEET_C; a.Pq = IPA_PQ; a.Pv = IPA_PV; a.R = 0; a.Cz = 16;
   a.DZ = MEET_DZ; a.RCz = MEET_RCZ; a.F = MEET_F;
   a.nqt = (p->L + QT - 1) / QT; a.nkt = (p->L + KT - 1) / KT;
   a.w_L = 1.f; a.w_C = 0.5f; a.scalar_scale = 1.f;

@@ -79,11 +79,10 @@ struct DistogramArgs {
 };
 cudaError_t distogram_launch(const DistogramArgs& a, cudaStream_t stream);
 
-// Distance-aware attention (MEET) on the IPA core: C = 16, Pq = 4, Pv = 8, a
-// zero pair block of 128 columns (the narrowest width of the CTA-pair core,
-// which runs this shape faster than the one-CTA core at 64), output row
-// F = C + 4 Pv + 128.
-constexpr int MEET_C = 16, MEET_RCZ = 128, MEET_DZ = 128, MEET_F = 16 + 4 * 8 + 128, MEET_ZEROS = 128;
+// Distance-aware attention (MEET) on the IPA core: C = 16, Pq = 4, Pv = 8 and
+// no pair block (pair width 0, which the one-CTA core and the prologue skip),
+// output row F = C + 4 Pv.
+constexpr int MEET_C = 16, MEET_RCZ = 0, MEET_DZ = 0, MEET_F = 16 + 4 * 8, MEET_ZEROS = 128;
 
 struct MeetWorkspace {
   size_t ipa, qs, gamma, consts, out, total;

@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int k = 0; k < 4; ++k) {
             const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
             umma_ss(tO, kdesc(pbase + 32 * k), mndesc(st + 8192 + 2048 * k), idv1, acc);
-            umma_ss(tO + 64, kdesc(pbase + 32 * k), mndesc(st + 16384 + 2048 * k), idv2, acc);
+            if (DZ > 0) umma_ss(tO + 64, kdesc(pbase + 32 * k), mndesc(st + 16384 + 2048 * k), idv2, acc);
           }
           umma_commit(bar(B_PFREE0 + pb));
           umma_commit(bar(B_EMPTY0 + s2));
@@ -526,8 +526,9 @@ cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream) {
   bool ok = encode_tmap_f16_3d(&tqh, ws + w.qh, DH, a.L, bh, DH * 2, rowb, 64, QT) &&
             encode_tmap_f16_3d(&tkh, ws + w.kh, DH, a.L, bh, DH * 2, rowb, 64, KT) &&
             encode_tmap_f16_3d(&tvh, ws + w.vh, DH, a.L, bh, DH * 2, rowb, 64, KT) &&
-            encode_tmap_f16_3d(&tz2, ws + w.z2, a.DZ, a.L, a.B, static_cast<uint64_t>(a.DZ) * 2,
-                               static_cast<uint64_t>(a.L) * a.DZ * 2, 64, KT);
+            (a.DZ == 0 ? (tz2 = tvh, true) :   // no pair block: the Z2 map is never read
+             encode_tmap_f16_3d(&tz2, ws + w.z2, a.DZ, a.L, a.B, static_cast<uint64_t>(a.DZ) * 2,
+                                static_cast<uint64_t>(a.L) * a.DZ * 2, 64, KT));
   if (!ok) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(ipa_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(SMEM_ALLOC));

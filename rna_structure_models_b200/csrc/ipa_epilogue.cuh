@@ -113,6 +113,7 @@ __device__ __forceinline__ void write_row(const float* O, float* dst, int lane, 
 // a pair feature sit on one lane and fold in registers; otherwise the
 // products are written in place and reduced in a second, float4 pass.
 static __device__ __noinline__ void fold_pairs_rows(const EpilogueArgs& e, int warp, int lane) {
+  if (e.RCz == 0) return;                     // no pair block (distance-aware attention)
   const int pitch = stage_pitch(e.DZ);
   const int nq = e.RCz >> 2;                  // float4 columns holding pair factors (RCz % 16 == 0)
   const int R = e.RCz / e.Cz, cq = e.Cz >> 2;

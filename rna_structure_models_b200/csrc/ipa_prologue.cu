@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(256) ipa_tile_kernel(const TileArgs a) {
     ipa_tile_copy_pairs(a, b, i0, panel, tid);
     return;
   }
+  const bool pairs = a.DZ > 0;   // no pair block (distance-aware attention): frames and sums only
   if (tid < KT) {
     const int i = i0 + tid;
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(256) ipa_tile_kernel(const TileArgs a) {
   if (tid == 0)
     *IPA_AT(a.part, b * a.nkt + J, static_cast<int64_t>(a.B) * a.nkt, a.err) =
         make_float4(red[0][0] + red[1][0], red[0][1] + red[1][1], red[0][2] + red[1][2], red[0][3] + red[1][3]);
-  ipa_tile_copy_pairs(a, b, i0, 0, tid);
+  if (pairs) ipa_tile_copy_pairs(a, b, i0, 0, tid);
 }
 
 struct RowArgs {
@@ -474,7 +475,7 @@ cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
   ta.z2h = reinterpret_cast<__half*>(ws + w.z2);
   ta.z1h = reinterpret_cast<__half*>(ws + w.z1h);
   ta.err = a.err;
-  ipa_tile_kernel<<<dim3(a.nkt, a.B, a.DZ / 64), 256, 0, stream>>>(ta);
+  ipa_tile_kernel<<<dim3(a.nkt, a.B, a.DZ > 0 ? a.DZ / 64 : 1), 256, 0, stream>>>(ta);
 
   RowArgs r{};
   r.B = a.B; r.L = a.L; r.H = a.H; r.nqt = a.nqt; r.nkt = a.nkt; r.Cz = a.Cz; r.RCz = a.RCz; r.DZ = a.DZ;
