@@ -16,19 +16,23 @@
 // Launches (all fp32 on CUDA cores; the per-pair terms are recomputed, no
 // N x N array is stored):
 //   0. the forward statistics (scales, rotated inputs, row max / sum, agg)
-//   1. geo_gvec_kernel     -- per (b, n): g_vec and whether any head is live
+//   1. geo_gvec_kernel     -- g_vec (a register-tiled product, 64 rows x 32
+//                             columns per block) and whether any head is live
 //   2. geo_dagg_kernel     -- per (b, n, h): dagg = R g_vec, <dagg, agg>
 //   3. geo_dw_part_kernel / geo_dw_sum_kernel -- dW = vec^T g_output and
 //                             db = sum g_output over live rows, per 128-row
-//                             chunk, then summed in a fixed order
+//                             chunk (register-tiled), then summed in a fixed
+//                             order
 //   4. geo_bwd_rows_kernel -- per (b, h, 128 queries) x 4 key splits: D_i,
 //                             then d qd, d qp and the per-head sums of
 //                             ds <qd, kd> and ds |qp - kp|
 //   5. geo_bwd_cols_kernel -- per (b, h, 128 keys) x 4 query splits: d kd,
 //                             d kp, d vr
-//   6. geo_bwd_frame_kernel -- per (b, n): local gradients R^T (...), the
-//                             rotation and translation gradients summed over
-//                             heads; block 0 also writes the scale gradients.
+//   6. geo_bwd_frame_kernel -- per (b, n, h): local gradients R^T (...) and
+//                             the head's frame terms, summed over heads in
+//                             order into the rotation and translation
+//                             gradients; block 0 also writes the scale
+//                             gradients.
 #include <cmath>
 #include <cstdint>
 

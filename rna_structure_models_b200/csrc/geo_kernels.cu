@@ -15,8 +15,9 @@
 //      rescaling; splits merged through shared memory; R_i^T back-rotation.
 //   4. geo_map_kernel     -- optional: recomputes each score and writes the
 //      normalised attention map, 16 query rows per block, 16-byte stores.
-//   5. geo_readout_kernel -- output = flatten(vectors) . W (+ b), forced to
-//      zero for queries where no head has an allowed key.
+//   5. geo_readout_kernel -- output = flatten(vectors) . W (+ b) as a
+//      register-tiled product (64 x 64 per block), forced to zero for
+//      queries where no head has an allowed key.
 #include <cuda_fp16.h>
 
 #include <cmath>

@@ -1,12 +1,13 @@
 // Fused attention pass of the IPA core for sm_100a: one CTA per
 // (batch, head, 128-query tile), a flash-style loop over 64-key tiles.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax and epilogue, one query row per thread (tensor-memory
-//              lane = row);
-//   warp 4     producer: per key tile, the fp32 column term and the TMA loads
+// Warp roles (320 threads):
+//   warps 0-7  softmax and epilogue, two threads per query row (column halves
+//              of S; tensor-memory lane = row);
+//   warp 8     producer: per key tile, the fp32 column term and the TMA loads
 //              of K_h, V_h and the shared Z2 tile into a 3-stage ring;
-//   warp 5     tensor-memory allocation and the single MMA-issuing thread.
+//   warp 9     tensor-memory allocation and the single MMA-issuing thread.
+// A pair width of 0 (no pair block) skips every Q_pair / Z2 step.
 //
 // Per key tile j (MMA issue order QK(0), QK(1), PV(0), QK(2), PV(1), ...):
 //   S  = Q_h . K_h^T (A from shared memory, K = 64)

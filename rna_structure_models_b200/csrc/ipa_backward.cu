@@ -19,11 +19,11 @@
 //   ipa_bwd_rows_kernel  one warp per (b, i, h): dO, dU, Q_pair (fp16 rows),
 //                        the row constant -(w_i + lse2_i), D_i and the query
 //                        and key points relative to the centroid (fp32);
-//   query pass           one CTA per (b, h, 128 queries), 64-key tiles:
+//   query pass           one CTA per (b, h, 128 queries), 32-key tiles:
 //                        S, dP (tcgen05, TMEM), dS (fp16, TMEM), then
 //                        dQ_h += dS K_h, dQ_pair += dS Z2 (A = dS from TMEM),
 //                        row sums rs_i = sum_j dS_ij, RSo_i = sum_j dS_ij o_J;
-//   key pass             one CTA per (b, h, 128 keys), 64-query tiles:
+//   key pass             one CTA per (b, h, 128 keys), 32-query tiles:
 //                        S^T, dP^T, then P^T and dS^T (fp16, in place in
 //                        TMEM) as A operands of dV += P^T dO,
 //                        dZ2 += P^T dU + dS^T Q_pair, dK_h += dS^T Q_h, column
@@ -37,7 +37,8 @@
 //                        frames (sums over heads), per-block d gamma partials;
 //   ipa_bwd_pair_kernel  per pair column and residue: d z1, d z2
 //                        (sums over heads) and d w_bias partials;
-//   ipa_bwd_reduce_kernel  fixed-order sums of the partials, one block per head.
+//   ipa_bwd_reduce_kernel  fixed-order sums of the partials, one block per
+//                        (head, 32 pair columns).
 // Every mbarrier wait is bounded (2 s) and reports into the error word.
 #include <cuda_fp16.h>
 
