@@ -577,7 +577,9 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
 // 32-query tile); warp 8: TMA producer and the per-query terms; warp 9: MMA.
 // S^T and dP^T are double-buffered (buffer i & 1, 32 columns each), so that
 // the MMAs of tile i + 1 run while the threads work on tile i.
-constexpr uint32_t K_TM_DZ2 = 0, K_TM_DKH = 256, K_TM_DVA = 320, K_TM_S = 384, K_TM_DP = 448;
+// S^T / dP^T buffer t: S^T at K_TM_SD + 64 t, dP^T right after it (one N = 64
+// accumulator for their pair parts)
+constexpr uint32_t K_TM_DZ2 = 0, K_TM_DKH = 256, K_TM_DVA = 320, K_TM_SD = 384;
 
 struct KLayout {
   uint32_t kh, vh, z2, stg, stg_bytes, aux, total;
@@ -589,7 +591,9 @@ __host__ __device__ inline KLayout k_layout(int DZ, int ns) {
   s.vh = 16384;
   s.z2 = 32768;
   s.stg = s.z2 + np * 16384;
-  s.stg_bytes = 8192 + 2 * np * 4096;       // Q_h 4 KB | dO 4 KB | Q_pair np x 4 KB | dU np x 4 KB (32 queries)
+  // Q_h 4 KB | dO 4 KB | np x (Q_pair panel 4 KB | dU panel 4 KB) (32 queries): each
+  // Q_pair panel with its dU panel is one 64-row K-major B operand
+  s.stg_bytes = 8192 + 2 * np * 4096;
   s.aux = s.stg + ns * s.stg_bytes;
   s.total = s.aux + 6656;
   return s;
@@ -706,8 +710,10 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         mbar_arrive_expect_tx(bar(KB_FULL0 + s), lay.stg_bytes);
         tma_load_3d(st, &tm_qh, bar(KB_FULL0 + s), 0, i * BT, bh);
         tma_load_3d(st + 4096, &tm_do, bar(KB_FULL0 + s), 0, i * BT, bh);
-        tma_load_4d(st + 8192, &tm_qp, bar(KB_FULL0 + s), 0, i * BT, 0, bh);
-        tma_load_4d(st + 8192 + np * 4096, &tm_du, bar(KB_FULL0 + s), 0, i * BT, 0, bh);
+        for (int p = 0; p < np; ++p) {   // interleaved panels: Q_pair p, then dU p
+          tma_load_4d(st + 8192 + 8192 * p, &tm_qp, bar(KB_FULL0 + s), 0, i * BT, p, bh);
+          tma_load_4d(st + 8192 + 8192 * p + 4096, &tm_du, bar(KB_FULL0 + s), 0, i * BT, p, bh);
+        }
         BWD_TR(1, i, 11);
       }
       const RowVals cur = nxt;
@@ -748,6 +754,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       tc_fence_after();
       const uint32_t id32 = idesc_f16(128, BT, false);
       const uint32_t id64mn = idesc_f16(128, 64, true);
+      const uint32_t id64 = idesc_f16(128, 2 * BT, false);   // [Q_pair ; dU] rows of a stage
       const uint32_t idz = idesc_f16(128, DZ, true);
       bool issued_any = false;
       // S^T(i), dP^T(i) into buffer i & 1, once stage i has landed and the
@@ -762,18 +769,17 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         if (!w) { fail(DEV_TIMEOUT_FULL); return false; }
         tc_fence_after();
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
-        const uint32_t sQh = st, sDO = st + 4096, sQP = st + 8192, sDU = st + 8192 + np * 4096;
-        const uint32_t tS = tmem + K_TM_S + 32 * t, tDP = tmem + K_TM_DP + 32 * t;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.kh + 32 * k), kd128(sQh + 32 * k), id32, k > 0 ? 1u : 0u);
+        const uint32_t sQh = st, sDO = st + 4096, sPair = st + 8192;
+        const uint32_t tS = tmem + K_TM_SD + 64 * t, tDP = tS + 32;
+        // the pair parts of S^T and dP^T share their A operand (Z2): one
+        // N = 64 MMA per K-step against [Q_pair ; dU], into [S^T | dP^T]
         for (int kk = 0; kk < 4 * np; ++kk)
           umma_ss(tS, kd128(sb + lay.z2 + 16384 * (kk >> 2) + 32 * (kk & 3)),
-                  kd128(sQP + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
+                  kd128(sPair + 8192 * (kk >> 2) + 32 * (kk & 3)), id64, kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma_ss(tDP, kd128(sb + lay.vh + 32 * k), kd128(sDO + 32 * k), id32, k > 0 ? 1u : 0u);
-        for (int kk = 0; kk < 4 * np; ++kk)
-          umma_ss(tDP, kd128(sb + lay.z2 + 16384 * (kk >> 2) + 32 * (kk & 3)),
-                  kd128(sDU + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
+        for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.kh + 32 * k), kd128(sQh + 32 * k), id32, 1u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) umma_ss(tDP, kd128(sb + lay.vh + 32 * k), kd128(sDO + 32 * k), id32, 1u);
         umma_commit(bar(KB_SFULL0 + t));
         BWD_TR(1, i, 2);
         issued_any = true;
@@ -787,14 +793,14 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
         BWD_TR(1, i, 3);
         tc_fence_after();
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
-        const uint32_t sQh = st, sDO = st + 4096, sQP = st + 8192, sDU = st + 8192 + np * 4096;
-        const uint32_t tS = tmem + K_TM_S + 32 * t, tDP = tmem + K_TM_DP + 32 * t;
+        const uint32_t sQh = st, sDO = st + 4096, sQP = st + 8192, sDU = st + 8192 + 4096;   // panels 8 KB apart
+        const uint32_t tS = tmem + K_TM_SD + 64 * t, tDP = tS + 32;
 #pragma unroll
         for (int k = 0; k < BT / 16; ++k) {
           const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
           umma_ts(tmem + K_TM_DVA, tS + 8 * k, mnd(sDO + 2048 * k, 4096), id64mn, acc);
-          umma_ts(tmem + K_TM_DZ2, tS + 8 * k, mnd(sDU + 2048 * k, 4096), idz, acc);
-          umma_ts(tmem + K_TM_DZ2, tDP + 8 * k, mnd(sQP + 2048 * k, 4096), idz, 1u);
+          umma_ts(tmem + K_TM_DZ2, tS + 8 * k, mnd(sDU + 2048 * k, 8192), idz, acc);
+          umma_ts(tmem + K_TM_DZ2, tDP + 8 * k, mnd(sQP + 2048 * k, 8192), idz, 1u);
           umma_ts(tmem + K_TM_DKH, tDP + 8 * k, mnd(sQh + 2048 * k, 4096), id64mn, acc);
         }
         umma_commit(bar(KB_ACC0 + t));
@@ -853,8 +859,8 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       uint32_t sv[16], dv[16];
       if (got) {
         tc_fence_after();
-        tmem_ld16(tmem + K_TM_S + 32 * tb + 16 * half + lane_off, sv);
-        tmem_ld16(tmem + K_TM_DP + 32 * tb + 16 * half + lane_off, dv);
+        tmem_ld16(tmem + K_TM_SD + 64 * tb + 16 * half + lane_off, sv);
+        tmem_ld16(tmem + K_TM_SD + 64 * tb + 32 + 16 * half + lane_off, dv);
         tmem_ld_wait();
         tc_fence_before();
       }
@@ -914,8 +920,8 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       co2 = fmaf(tsum, oqv.z, co2);
       if (tid == 0) BWD_TR(1, i, 8);
       tc_fence_after();
-      tmem_st8(tmem + K_TM_S + 32 * tb + 8 * half + lane_off, pp);
-      tmem_st8(tmem + K_TM_DP + 32 * tb + 8 * half + lane_off, pd);
+      tmem_st8(tmem + K_TM_SD + 64 * tb + 8 * half + lane_off, pp);
+      tmem_st8(tmem + K_TM_SD + 64 * tb + 32 + 8 * half + lane_off, pd);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(KB_PFULL0 + tb));
@@ -1364,8 +1370,8 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
               encode_tmap_f16_panels(&mp.k_z2, ws + fw.z2, DZ, L, B, 128, np) &&
               encode_tmap_f16_3d(&mp.k_qh, ws + fw.qh, DH, L, bh, DH * 2, rowb, 64, BT) &&
               encode_tmap_f16_3d(&mp.k_do, ws + w.doh, DH, L, bh, DH * 2, rowb, 64, BT) &&
-              encode_tmap_f16_panels(&mp.k_qp, ws + w.qp, DZ, L, bh, BT, np) &&
-              encode_tmap_f16_panels(&mp.k_du, ws + w.du, DZ, L, bh, BT, np);
+              encode_tmap_f16_panels(&mp.k_qp, ws + w.qp, DZ, L, bh, BT, 1) &&
+              encode_tmap_f16_panels(&mp.k_du, ws + w.du, DZ, L, bh, BT, 1);
     if (!ok) return cudaErrorInvalidValue;
     const QLayout l1 = q_layout(DZ, 1);
     ba.ns = stages_for(l1.stg, l1.stg_bytes, 2048);
