@@ -76,6 +76,7 @@ constexpr float kLn2 = 0.69314718055994531f;
 
 struct BwdArgs {
   int B, L, H, DZ, RCz, Cz, R, nqt, nkt, ns;
+  int qp_stage;          // query pass: 1 if its last stage lives in the Q_pair area (free once Q_pair is in TMEM)
   float qscale, w_L, w_C;
   // forward prologue outputs (workspace)
   const float4* rowq;    // [B*H, L] (sum_p gq', c |gq'|^2)
@@ -249,7 +250,11 @@ constexpr int MAX_NS = 3;
 constexpr int BT = 32;
 
 // tensor memory (512 columns)
-constexpr uint32_t Q_TM_DQP = 0, Q_TM_DQH = 256, Q_TM_S = 320, Q_TM_DP = 352, Q_TM_DS = 384;
+// Q_TM_QPT: the first QPT_COLS columns of the Q_pair rows (fp16 pairs), the
+// A operand of most of S's pair part, so that its MMAs read only the key
+// tile from shared memory
+constexpr uint32_t Q_TM_DQP = 0, Q_TM_DQH = 256, Q_TM_S = 320, Q_TM_DP = 352, Q_TM_DS = 384, Q_TM_QPT = 400;
+constexpr int QPT_COLS = 112;
 
 struct QLayout {
   uint32_t qh, qp, dO, du, stg, stg_bytes, aux, total;
@@ -269,7 +274,7 @@ __host__ __device__ inline QLayout q_layout(int DZ, int ns) {
 }
 // aux area: col terms [MAX_NS][32] floats (384 B, from 0) | tile info [MAX_NS][2] float4 (96 B) | barriers
 constexpr uint32_t QA_COL = 0, QA_INFO = 768, QA_BAR = 896;
-enum { QB_QFULL = 0, QB_SFULL, QB_SFREE, QB_DSFULL, QB_DSFREE, QB_DRAIN, QB_FULL0, QB_EMPTY0 = QB_FULL0 + MAX_NS,
+enum { QB_QFULL = 0, QB_QTM, QB_SFULL, QB_SFREE, QB_DSFULL, QB_DSFREE, QB_DRAIN, QB_FULL0, QB_EMPTY0 = QB_FULL0 + MAX_NS,
        QB_COUNT = QB_EMPTY0 + MAX_NS };
 constexpr uint32_t QA_TMEM = QA_BAR + 8 * QB_COUNT, QA_ABORT = QA_TMEM + 8;
 
@@ -286,7 +291,9 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
   const int bh = blk / a.nqt;
   const int b = bh / a.H, h = bh % a.H;
   const int L = a.L, nt = (a.L + BT - 1) / BT, DZ = a.DZ, np = DZ / 64, NS = a.ns;   // nt 32-key tiles
-  const QLayout lay = q_layout(DZ, NS);
+  const int nreg = NS - a.qp_stage;   // stages in the stage area; stage nreg (if any) in the Q_pair area
+  const QLayout lay = q_layout(DZ, nreg);
+  auto stage_at = [&](int s) -> uint32_t { return s < nreg ? sb + lay.stg + s * lay.stg_bytes : sb + lay.qp; };
   float* col_s = reinterpret_cast<float*>(smem + lay.aux + QA_COL);
   float4* info = reinterpret_cast<float4*>(smem + lay.aux + QA_INFO);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + lay.aux + QA_ABORT);
@@ -295,6 +302,7 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
 
   if (tid == 0) {
     mbar_init(bar(QB_QFULL), 1);
+    mbar_init(bar(QB_QTM), NSOFT);
     mbar_init(bar(QB_SFULL), 1);
     mbar_init(bar(QB_SFREE), NSOFT);
     mbar_init(bar(QB_DSFULL), NSOFT);
@@ -355,7 +363,17 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
       }
       issued = j + 1;
       if (lane == 0) {
-        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+        // the Q_pair-area stage is first filled once every thread has copied
+        // its Q_pair row into tensor memory
+        if (s == nreg && j == nreg && !mbar_wait_bounded(bar(QB_QTM), 0, abort_flag)) {
+          fail(DEV_TIMEOUT_EMPTY);
+          issued = j;
+        }
+      }
+      issued = __shfl_sync(0xffffffffu, issued, 0);
+      if (issued == j) break;
+      if (lane == 0) {
+        const uint32_t st = stage_at(s);
         mbar_arrive_expect_tx(bar(QB_FULL0 + s), lay.stg_bytes);
         tma_load_3d(st, &tm_kh, bar(QB_FULL0 + s), 0, j * BT, bh);
         tma_load_3d(st + 4096, &tm_vh, bar(QB_FULL0 + s), 0, j * BT, bh);
@@ -384,12 +402,13 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
     }
   } else if (warp == W_MMA) {
     if (lane == 0) {
-      bool ok = mbar_wait_bounded(bar(QB_QFULL), 0, abort_flag);
+      bool ok = mbar_wait_bounded(bar(QB_QFULL), 0, abort_flag) && mbar_wait_bounded(bar(QB_QTM), 0, abort_flag);
       if (!ok) fail(DEV_TIMEOUT_FULL);
       tc_fence_after();
       const uint32_t id32 = idesc_f16(128, BT, false);
       const uint32_t id64mn = idesc_f16(128, 64, true);
       const uint32_t idz = idesc_f16(128, DZ, true);
+      const int ntm = 4 * np < 2 * QPT_COLS / 16 ? 4 * np : 2 * QPT_COLS / 16;   // S pair K-steps with A in TMEM
       const uint32_t tS = tmem + Q_TM_S, tDP = tmem + Q_TM_DP, tDS = tmem + Q_TM_DS;
       const uint32_t tDQH = tmem + Q_TM_DQH, tDQP = tmem + Q_TM_DQP;
       bool issued_any = false;
@@ -401,10 +420,12 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         BWD_TR(0, j, 1);                   // S(j-1), dP(j-1) read
         if (!w) { fail(DEV_TIMEOUT_FULL); return false; }
         tc_fence_after();
-        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+        const uint32_t st = stage_at(s);
 #pragma unroll
         for (int k = 0; k < 4; ++k) umma_ss(tS, kd128(sb + lay.qh + 32 * k), kd128(st + 32 * k), id32, k > 0 ? 1u : 0u);
-        for (int kk = 0; kk < 4 * np; ++kk)
+        for (int kk = 0; kk < ntm; ++kk)
+          umma_ts(tS, tmem + Q_TM_QPT + 8 * kk, kd128(st + 8192 + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
+        for (int kk = ntm; kk < 4 * np; ++kk)
           umma_ss(tS, kd128(sb + lay.qp + 16384 * (kk >> 2) + 32 * (kk & 3)),
                   kd128(st + 8192 + 4096 * (kk >> 2) + 32 * (kk & 3)), id32, 1u);
 #pragma unroll
@@ -423,7 +444,7 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         BWD_TR(0, jj, 3);                  // dS(jj) written
         tc_fence_after();
         const int s = jj % NS;
-        const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
+        const uint32_t st = stage_at(s);
 #pragma unroll
         for (int k = 0; k < BT / 16; ++k) {
           const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
@@ -435,14 +456,19 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
         BWD_TR(0, jj, 4);                  // dQ(jj) issued
         return true;
       };
-      // dQ(j-1) before S(j), dP(j): tile j + 1 reuses the stage of tile j - 1
-      // (two stages), which dQ(j-1) releases, so its copy then overlaps S(j),
-      // dP(j) and the threads' work on j.  (Issuing S(j), dP(j) first kept the
-      // tensor pipe busy during that work but left each copy fully exposed:
-      // 2.567 -> 2.528 ms for the gradient call at L = 4096.)
+      // Three stages (the third in the Q_pair area): S(j), dP(j) before
+      // dQ(j-1), so the tensor pipe works on tile j while the threads finish
+      // j - 1, and the copy of tile j + 2 has a whole tile to land.  Two
+      // stages: dQ(j-1) first, since tile j + 1 reuses the stage dQ(j-1)
+      // releases (S(j), dP(j) first left each copy exposed).
       for (int j = 0; ok && j <= nt; ++j) {
-        if (j > 0) ok = issue_dq(j - 1);
-        if (ok && j < nt) ok = issue_sdp(j);
+        if (NS >= 3) {
+          if (j < nt) ok = issue_sdp(j);
+          if (ok && j > 0) ok = issue_dq(j - 1);
+        } else {
+          if (j > 0) ok = issue_dq(j - 1);
+          if (ok && j < nt) ok = issue_sdp(j);
+        }
       }
       if (!ok && issued_any) {
         umma_commit(bar(QB_DRAIN));
@@ -462,6 +488,25 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
     const float pq = static_cast<float>(IPA_PQ);
     float rs = 0.f, ro0 = 0.f, ro1 = 0.f, ro2 = 0.f;
     bool ok = true;
+    // the first QPT_COLS columns of this row's Q_pair into tensor memory
+    // (from the 128-byte swizzled panels TMA wrote: 16-byte chunk c of row r
+    // at 16 (c ^ (r & 7))), half 0 the first half of them
+    if (__all_sync(0xffffffffu, mbar_wait_bounded(bar(QB_QFULL), 0, abort_flag))) {
+      const int nw = DZ / 2 < QPT_COLS ? DZ / 2 : QPT_COLS;   // words (fp16 pairs) in tensor memory
+      for (int w0 = half * (QPT_COLS / 2); w0 < (half + 1) * (QPT_COLS / 2) && w0 < nw; w0 += 8) {
+        const int pnl = w0 >> 5, c0 = (w0 & 31) >> 2;
+        const unsigned char* rowp = smem + lay.qp + 16384u * pnl + r * 128;
+        const uint4 u0 = *reinterpret_cast<const uint4*>(rowp + ((c0 ^ (r & 7)) << 4));
+        const uint4 u1 = *reinterpret_cast<const uint4*>(rowp + (((c0 + 1) ^ (r & 7)) << 4));
+        const uint32_t v[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        tmem_st8(tmem + Q_TM_QPT + w0 + lane_off, v);
+      }
+      tmem_st_wait();
+    } else {
+      if (lane == 0) fail(DEV_TIMEOUT_FULL);
+    }
+    tc_fence_before();
+    mbar_arrive(bar(QB_QTM));
     for (int j = 0; j < nt && ok; ++j) {
       const int s = j % NS;
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(QB_SFULL), j & 1, abort_flag))) {
@@ -1374,11 +1419,17 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
               encode_tmap_f16_panels(&mp.k_du, ws + w.du, DZ, L, bh, BT, 1);
     if (!ok) return cudaErrorInvalidValue;
     const QLayout l1 = q_layout(DZ, 1);
-    ba.ns = stages_for(l1.stg, l1.stg_bytes, 2048);
+    const int nreg = stages_for(l1.stg, l1.stg_bytes, 2048);
+    // one more stage in the Q_pair area: the columns in tensor memory free at
+    // least its first stg_bytes (all of it when every K-step is there, the
+    // first three panels at DZ = 256)
+    ba.qp_stage = nreg < MAX_NS ? 1 : 0;
+    ba.ns = nreg + ba.qp_stage;
     const KLayout k1 = k_layout(DZ, 1);
     BwdArgs kb = ba;
     kb.ns = stages_for(k1.stg, k1.stg_bytes, 6656);
-    const uint32_t sq = q_layout(DZ, ba.ns).total, sk = k_layout(DZ, kb.ns).total;
+    kb.qp_stage = 0;
+    const uint32_t sq = q_layout(DZ, nreg).total, sk = k_layout(DZ, kb.ns).total;
     const uint32_t smem = (sq > sk ? sq : sk) + 1024;
     e = cudaFuncSetAttribute(ipa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
