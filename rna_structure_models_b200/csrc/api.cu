@@ -195,7 +195,7 @@ const char* ipa_version(void) { return "flashipa_b200 sm_100a 0.1"; }
 size_t ipa_attn_workspace_size(const ipa_params_t* p) {
   ipa_status_t st;
   if (!ipa_dims_ok(p, &st)) return 0;
-  return ipa_workspace_layout(p->B, p->L, p->H, pair_width(p), p->R * p->Cz).total;
+  return ipa_workspace_layout(p->B, p->L, p->H, pair_width(p), p->R * p->Cz, true).total;
 }
 
 }  // extern "C"
@@ -204,9 +204,11 @@ namespace {
 
 // Validation + launch description shared by the three IPA entry points.
 // inputs == false: only the params, `out` and the workspace are checked.
+// with_split == false: the layout without the core's key-split reserve (the
+// gradient call's recomputed prologue).
 ipa_status_t ipa_prepare(const ipa_params_t* p, const ipa_tensor_t* const* in, const ipa_tensor_t* out,
                          void* workspace, size_t workspace_bytes, void* stream, int32_t* dev_err,
-                         bool inputs, bool reset_err, IpaLaunch* a) {
+                         bool inputs, bool reset_err, IpaLaunch* a, bool with_split = true) {
   ipa_status_t st = IPA_OK;
   if (!ipa_dims_ok(p, &st)) return st;
   const int64_t B = p->B, L = p->L, H = p->H, C = p->C, Pq = p->Pq, Pv = p->Pv, R = p->R, Cz = p->Cz;
@@ -231,7 +233,7 @@ ipa_status_t ipa_prepare(const ipa_params_t* p, const ipa_tensor_t* const* in, c
     if (!check_contiguous_out(out, 4, s_o, &st)) return st;
   }
   const int DZ = pair_width(p);
-  const IpaWorkspace lay = ipa_workspace_layout(p->B, p->L, p->H, DZ, p->R * p->Cz);
+  const IpaWorkspace lay = ipa_workspace_layout(p->B, p->L, p->H, DZ, p->R * p->Cz, with_split);
   if (workspace == nullptr) return IPA_ERR_NULL;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
 
@@ -525,7 +527,7 @@ ipa_status_t ipa_attn_bwd(const ipa_params_t* p, const ipa_tensor_t* q, const ip
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < lay.total) return IPA_ERR_WORKSPACE;
   IpaBwdLaunch b{};
   // inputs and the forward part of the workspace (prologue outputs) through the forward's checks
-  st = ipa_prepare(p, in, nullptr, workspace, lay.fwd.total, stream, dev_err, true, true, &b.f);
+  st = ipa_prepare(p, in, nullptr, workspace, lay.fwd.total, stream, dev_err, true, true, &b.f, false);
   if (st != IPA_OK) return st;
   b.out = view_of(out);
   b.lse = view_of(lse);

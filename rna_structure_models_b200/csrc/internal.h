@@ -25,10 +25,26 @@ struct View {
 };
 
 struct IpaWorkspace {
-  size_t qh, kh, vh, z2, z1h, z1f, rowq, colk, frame, part, cen, oq, ok, headc, wqp, err, total;
+  size_t qh, kh, vh, z2, z1h, z1f, rowq, colk, frame, part, cen, oq, ok, headc, wqp, err;
+  // key-split tail of the CTA-pair core (with_split): partial accumulators
+  // of up to split_chunks chunks (two CTAs each, [DZ + 67][128] floats) and
+  // a ticket per (tile, CTA) for up to split_tiles tiles; 0 without
+  size_t split, ticket;
+  int64_t split_tiles, split_chunks;
+  size_t total;
 };
 
-IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz);
+// Resident CTA pairs of the core on a B200 (148 SMs, one CTA per SM): the
+// key-split reserve holds two chunks per pair and a ticket per pair.
+constexpr int kSplitPairs = 74;
+
+IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz, bool with_split = false);
+
+struct SplitPlan {
+  int first;   // pair tiles before this run whole
+  int S;       // chunks per later tile (1: no split)
+};
+SplitPlan ipa_split_plan(int T, int nkp, int P, int64_t max_tiles, int64_t max_chunks);
 
 struct IpaLaunch {
   int B, L, H, C, Pq, Pv, R, Cz, DZ, RCz, F, nqt, nkt;

@@ -86,6 +86,13 @@ struct PairArgs {
   float* uagg;          // training forward: [B, L, H, R Cz] pair aggregate, else null
   int* err;
   int tma_epi;          // 1: the output pass stages the pair features and stores them with TMA
+  // key-split tail: pair tiles [split_first, T) are each run as split_s
+  // chunks of consecutive key tiles by split_s CTA pairs (split_s == 1: none)
+  int split_first, split_s;
+  int64_t part_extent;  // floats in part (bounds-checked build)
+  int ticket_extent;    // ints in ticket
+  float* part;          // per (chunk, CTA rank): [DZ + 64 + 3][128] partial accumulators, max, two half sums
+  int* ticket;          // per (split tile, CTA rank): chunks finished (zero between calls)
   int trace_cta0, trace_cta1;
 };
 
@@ -93,6 +100,7 @@ constexpr int NT = 352;            // 8 softmax warps, K producer, MMA issuer, V
 constexpr int NSOFT = 256;
 constexpr int W_PROD = 8, W_MMA = 9, W_VPROD = 10;
 constexpr int NCOL = 4;            // column-term ring
+constexpr int MAX_SPLIT = 5;       // key chunks of a split tile
 
 // shared memory (offsets from a 1024-byte aligned base)
 constexpr uint32_t SP_QH = 0;
@@ -120,6 +128,7 @@ enum {
 };
 constexpr uint32_t AX_TMEM = AX_BAR + 8 * P_COUNT;
 constexpr uint32_t AX_ABORT = AX_TMEM + 8;
+constexpr uint32_t AX_LAST = AX_ABORT + 4;        // int: this CTA finishes its split tile
 
 constexpr uint32_t TM_S = 320, TM_P = 448, TM_COLS = 512;
 
@@ -153,10 +162,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
-  const int I2 = pair % a.nqp;
-  const int bh = pair / a.nqp;
+  // a split tile's chunk c covers key tiles [c nkp / S, (c + 1) nkp / S)
+  int tile = pair, chunk = -1, kbeg = 0, nt = a.nkp;
+  if (pair >= a.split_first) {
+    const int q = pair - a.split_first;
+    tile = a.split_first + q / a.split_s;
+    chunk = q % a.split_s;
+    kbeg = chunk * a.nkp / a.split_s;
+    nt = (chunk + 1) * a.nkp / a.split_s - kbeg;
+  }
+  const int I2 = tile % a.nqp;
+  const int bh = tile / a.nqp;
   const int b = bh / a.H, h = bh % a.H;
-  const int L = a.L, nt = a.nkp, DZ = a.DZ, np = DZ / 64;
+  const int L = a.L, DZ = a.DZ, np = DZ / 64;
   const int row0 = 256 * I2 + 128 * static_cast<int>(rank);   // first query row of this CTA
   const int I = row0 / QT;                                      // its 128-row query tile
 #ifdef IPA_TRACE
@@ -212,7 +230,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     record_error(a.err, code);
     *abort_flag = 1;
   };
-  const int start = (2 * I2) % nt;   // diagonal key tile first
+  const int start = chunk < 0 ? (2 * I2) % a.nkp : kbeg;   // a whole tile starts at its diagonal key tile
 
   if (warp == W_PROD) {
     // ------------------------------------------------ producer (each CTA)
@@ -228,7 +246,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     // that their global-load latency overlaps the wait for a free K slot
     float4 ckn[4], okn[4], odn = make_float4(0.f, 0.f, 0.f, 0.f);
     auto fetch_cols = [&](int j) {
-      const int J2 = (start + j) % nt;
+      const int J2 = (start + j) % a.nkp;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int key = J2 * 128 + lane + 32 * t;
@@ -240,7 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       odn = (j < nt && jt < a.nkt) ? a.ok[b * a.nkt + jt] : make_float4(0.f, 0.f, 0.f, 0.f);
     };
     auto load_k = [&](int j) {
-      const int J2 = (start + j) % nt;
+      const int J2 = (start + j) % a.nkp;
       const int s = j & 1;
       if (lane == 0) {
         const uint32_t kf = bar0(P_KFULL0 + s);
@@ -324,7 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           break;
         }
         PAIR_TR(j, 15);
-        const int J2 = (start + j) % nt;
+        const int J2 = (start + j) % a.nkp;
         const uint32_t vf = bar0(P_VFULL);
         const uint32_t st = sb + SP_V;
         mbar_arrive_expect_tx_remote(vf, vbytes);
@@ -565,107 +583,201 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     }
     if (tid == 0) PAIR_SPAN(10);
     const bool all_ok = __all_sync(0xffffffffu, ok);
-    xch[512 + half * 128 + r] = l;
-    named_bar_sync(pair_bar, 64);
-    if (tid == 0) PAIR_SPAN(20);
-    const float lt = l + xch[512 + (1 - half) * 128 + r];
-    const bool dead = !(in_range && f3.x != 0.f && lt > 0.f);
-    // training forward: log-sum-exp of the true logits; the pass left the row
-    // constant c sum_p |gq'_p|^2 (rowq.w) out of its logits
-    if (a.lse != nullptr && half == 0 && in_range)
-      *IPA_AT(a.lse, static_cast<int64_t>(bh) * L + row, static_cast<int64_t>(a.B) * a.H * L, a.err) = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
-    // direct output pass when the pair block has no padding and whole
-    // 64-column factors (the staged pass below handles every other shape)
-    if (a.tma_epi) {
-      // staged pair features (z1 from the boxes the producer loaded, the
-      // output through staging boxes and a TMA store), scalars and points direct
-      const bool zok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(P_ZFULL), 0, abort_flag));
-      if (!zok && lane == 0) fail(DEV_TIMEOUT_FULL);
-      const int nz = DZ / 32;
-      if (all_ok && zok && !*abort_flag) {
+    // key-split tail: each chunk stores its partial accumulators, row
+    // maximum and half sums; the chunk that finishes its tile last (ticket)
+    // merges all chunks in chunk order into tensor memory, so the result does
+    // not depend on which chunk that is, and runs the output pass
+    bool epi = true;
+    if (chunk >= 0) {
+      const int OW3 = OW + 3;
+      const int64_t qc = pair - a.split_first;   // (split tile) S + chunk
+      const int64_t blk_floats = static_cast<int64_t>(OW3) * 128;
+      float* mine = IPA_SPAN(a.part, (2 * qc + rank) * blk_floats, blk_floats, a.part_extent, a.err);
+      if (all_ok) {
         tc_fence_after();
-        const float inv = dead ? 0.f : 1.f / lt;
-        const int rrow = in_range ? row : 0;
-        const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
-        const int64_t nrows = static_cast<int64_t>(a.B) * L * a.H;
-        auto z1box = [&](int k) -> const unsigned char* { return smem + SP_QP + 16384u * k; };
-        auto obox = [&](int k) -> unsigned char* {
-          return smem + (k == 0 ? SP_QH : SP_QP + 16384u * (nz + k - 1));
-        };
-        stage_row_pair(tmem + lane_off, half, a.Cz, a.RCz / a.Cz, inv, r,
-                       a.uagg != nullptr ? IPA_SPAN(a.uagg, orow * a.RCz, a.RCz, nrows * a.RCz, a.err) : nullptr,
-                       in_range, z1box, obox);
-        if (tid == 0) PAIR_SPAN(22);
-        if (half == 0)
-          write_row_points<IPA_C, IPA_PV>(tmem + DZ + lane_off, inv, dead, in_range,
-                                          IPA_SPAN(a.out, orow * a.F, a.F, nrows * a.F, a.err), g0, g1, g2, cn);
-        fence_proxy_async_smem();   // the staging writes, before the TMA store reads them
+        for (int c0 = o_lo; c0 < o_hi; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tmem + c0 + lane_off, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mine[(c0 + e) * 128 + r] = __uint_as_float(o[e]);
+        }
+        if (half == 0) mine[OW * 128 + r] = m_used;
+        mine[(OW + 1 + half) * 128 + r] = l;
+      }
+      __threadfence();
+      named_bar_sync(1, NSOFT);
+      volatile int* last = reinterpret_cast<volatile int*>(smem + SP_AUX + AX_LAST);
+      if (tid == 0) {
+        int* tk = IPA_AT(a.ticket, 2 * (qc / a.split_s) + rank, a.ticket_extent, a.err);
+        const bool fin = atomicAdd(tk, 1) == a.split_s - 1;
+        if (fin) *tk = 0;   // every chunk of the tile has counted: ready for the next call
+        *last = fin ? 1 : 0;
       }
       named_bar_sync(1, NSOFT);
-      // a tile past the last row (the pair's second CTA when L <= 128) has
-      // nothing to store; the tensor map clips the rest of a ragged tile
-      if (tid == 0 && all_ok && zok && !*abort_flag && row0 < L &&
-          IPA_CHECK(row0 >= 0 && b >= 0 && b < a.B && h >= 0 && h < a.H, a.err)) {
-        for (int k = 0; k < a.Cz / 32; ++k)
-          tma_store_4d(&tm_out, sb + (k == 0 ? SP_QH : SP_QP + 16384u * (nz + k - 1)), IPA_C + 4 * IPA_PV + 32 * k, h,
-                       row0, b);
-        bulk_commit_group();
-        bulk_wait_read_all();   // the staging boxes must outlive the reads, not the writes
-      }
-      if (tid == 0) PAIR_SPAN(21);
-    } else if (a.RCz == DZ && (a.Cz & 63) == 0) {
-      if (all_ok && !*abort_flag) {
-        tc_fence_after();
-        const float inv = dead ? 0.f : 1.f / lt;
-        const int rrow = in_range ? row : 0;
-        const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
-        const int64_t nrows = static_cast<int64_t>(a.B) * L * a.H;
-        unsigned long long* etr = nullptr;
-#ifdef IPA_TRACE
-        if (tid == 0 && blockIdx.x < 4096) etr = &g_pair_span[blockIdx.x][22];
-#endif
-        write_row_direct<IPA_C, IPA_PV>(tmem + lane_off, half, DZ, a.Cz, a.RCz / a.Cz, inv, dead, in_range,
-                                        a.z1f + (static_cast<int64_t>(b) * L + rrow) * DZ,
-                                        IPA_SPAN(a.out, orow * a.F, a.F, nrows * a.F, a.err),
-                                        a.uagg != nullptr ? IPA_SPAN(a.uagg, orow * a.RCz, a.RCz, nrows * a.RCz, a.err)
-                                                          : nullptr,
-                                        g0, g1, g2, cn, etr);
-        if (tid == 0) PAIR_SPAN(21);
-      }
-    } else {
-    const int pitch = stage_pitch(DZ);
-    float* stage = reinterpret_cast<float*>(smem + SP_QP);
-    if (all_ok) {
-      tc_fence_after();
-      const float inv = dead ? 0.f : 1.f / lt;
-      float* orow = stage + r * pitch;
-      // tensor memory holds [O_pair | O_v]; the stage row is [O_v | O_pair | frame]
-      for (int c0 = o_lo; c0 < o_hi; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tmem + c0 + lane_off, o);
-        tmem_ld_wait();
-        const int dstc = c0 < DZ ? 64 + c0 : c0 - DZ;
+      epi = *last != 0;
+      if (epi) {
+        __threadfence();
+        const float* c0p = a.part + (2 * (qc - chunk) + rank) * blk_floats;   // chunk 0 of this tile
+        const int S = a.split_s;
+        float ms[MAX_SPLIT], wt[MAX_SPLIT];
+        float M = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(orow + dstc + e) =
-              make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                          __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+        for (int s = 0; s < MAX_SPLIT; ++s) {
+          ms[s] = s < S ? (s == chunk ? m_used : __ldcg(c0p + 2 * s * blk_floats + OW * 128 + r)) : -INFINITY;
+          M = fmaxf(M, ms[s]);
+        }
+        float ln = 0.f;
+#pragma unroll
+        for (int s = 0; s < MAX_SPLIT; ++s) {
+          wt[s] = (s < S && M != -INFINITY) ? ex2(ms[s] - M) : 0.f;
+          if (s < S) ln = fmaf(wt[s], s == chunk ? l : __ldcg(c0p + 2 * s * blk_floats + (OW + 1 + half) * 128 + r), ln);
+        }
+        tc_fence_after();
+        // 16 columns at a time: the loads of every other chunk are issued
+        // together (one L2 round trip per group), then summed in chunk order
+        for (int c0 = o_lo; c0 < o_hi; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(tmem + c0 + lane_off, o);
+          float v[MAX_SPLIT][16];
+#pragma unroll
+          for (int s = 0; s < MAX_SPLIT; ++s) {
+            const float* src = c0p + 2 * s * blk_floats + c0 * 128 + r;
+            const bool other = s < S && s != chunk;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[s][e] = other ? __ldcg(src + e * 128) : 0.f;
+          }
+          tmem_ld_wait();
+          float acc[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+#pragma unroll
+          for (int s = 0; s < MAX_SPLIT; ++s) {
+            if (s < S) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) acc[e] = fmaf(wt[s], s == chunk ? __uint_as_float(o[e]) : v[s][e], acc[e]);
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(acc[e]);
+          tmem_st16(tmem + c0 + lane_off, o);
+        }
+        tmem_st_wait();
+        m_used = M;
+        l = ln;
+        // the output pass reads columns of both halves of a row
+        tc_fence_before();
+        named_bar_sync(pair_bar, 64);
+        tc_fence_after();
       }
-      if (half == 0) stage_frame(orow + 64 + DZ, g0, g1, g2, cn, dead);
     }
-    tc_fence_before();
-    named_bar_sync(1, NSOFT);
-    if (tid == 0) PAIR_SPAN(11);
-    if (!*abort_flag) {
-      EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, row0, a.z1f, a.out};
-      ea.uagg = a.uagg;
-      ea.rows = static_cast<int64_t>(a.B) * L * a.H;
-      ea.err = a.err;
+    if (epi) {
+      xch[512 + half * 128 + r] = l;
+      named_bar_sync(pair_bar, 64);
+      if (tid == 0) PAIR_SPAN(20);
+      const float lt = l + xch[512 + (1 - half) * 128 + r];
+      const bool dead = !(in_range && f3.x != 0.f && lt > 0.f);
+      // training forward: log-sum-exp of the true logits; the pass left the row
+      // constant c sum_p |gq'_p|^2 (rowq.w) out of its logits
+      if (a.lse != nullptr && half == 0 && in_range)
+        *IPA_AT(a.lse, static_cast<int64_t>(bh) * L + row, static_cast<int64_t>(a.B) * a.H * L, a.err) = dead ? INFINITY : (m_used + log2f(lt) - sq.w) * 0.69314718055994531f;
+      // direct output pass when the pair block has no padding and whole
+      // 64-column factors (the staged pass below handles every other shape)
+      if (a.tma_epi) {
+        // staged pair features (z1 from the boxes the producer loaded, the
+        // output through staging boxes and a TMA store), scalars and points direct
+        const bool zok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(P_ZFULL), 0, abort_flag));
+        if (!zok && lane == 0) fail(DEV_TIMEOUT_FULL);
+        const int nz = DZ / 32;
+        if (all_ok && zok && !*abort_flag) {
+          tc_fence_after();
+          const float inv = dead ? 0.f : 1.f / lt;
+          const int rrow = in_range ? row : 0;
+          const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
+          const int64_t nrows = static_cast<int64_t>(a.B) * L * a.H;
+          auto z1box = [&](int k) -> const unsigned char* { return smem + SP_QP + 16384u * k; };
+          auto obox = [&](int k) -> unsigned char* {
+            return smem + (k == 0 ? SP_QH : SP_QP + 16384u * (nz + k - 1));
+          };
+          stage_row_pair(tmem + lane_off, half, a.Cz, a.RCz / a.Cz, inv, r,
+                         a.uagg != nullptr ? IPA_SPAN(a.uagg, orow * a.RCz, a.RCz, nrows * a.RCz, a.err) : nullptr,
+                         in_range, z1box, obox);
+          if (tid == 0) PAIR_SPAN(22);
+          if (half == 0)
+            write_row_points<IPA_C, IPA_PV>(tmem + DZ + lane_off, inv, dead, in_range,
+                                            IPA_SPAN(a.out, orow * a.F, a.F, nrows * a.F, a.err), g0, g1, g2, cn);
+          fence_proxy_async_smem();   // the staging writes, before the TMA store reads them
+        }
+        named_bar_sync(1, NSOFT);
+        // a tile past the last row (the pair's second CTA when L <= 128) has
+        // nothing to store; the tensor map clips the rest of a ragged tile
+        if (tid == 0 && all_ok && zok && !*abort_flag && row0 < L &&
+            IPA_CHECK(row0 >= 0 && b >= 0 && b < a.B && h >= 0 && h < a.H, a.err)) {
+          for (int k = 0; k < a.Cz / 32; ++k)
+            tma_store_4d(&tm_out, sb + (k == 0 ? SP_QH : SP_QP + 16384u * (nz + k - 1)), IPA_C + 4 * IPA_PV + 32 * k, h,
+                         row0, b);
+          bulk_commit_group();
+          bulk_wait_read_all();   // the staging boxes must outlive the reads, not the writes
+        }
+        if (tid == 0) PAIR_SPAN(21);
+      } else if (a.RCz == DZ && (a.Cz & 63) == 0) {
+        if (all_ok && !*abort_flag) {
+          tc_fence_after();
+          const float inv = dead ? 0.f : 1.f / lt;
+          const int rrow = in_range ? row : 0;
+          const int64_t orow = (static_cast<int64_t>(b) * L + rrow) * a.H + h;
+          const int64_t nrows = static_cast<int64_t>(a.B) * L * a.H;
+          unsigned long long* etr = nullptr;
 #ifdef IPA_TRACE
-      ea.trace = (blockIdx.x < 4096 && warp == 0) ? &g_pair_span[blockIdx.x][16] : nullptr;
+          if (tid == 0 && blockIdx.x < 4096) etr = &g_pair_span[blockIdx.x][22];
 #endif
-      write_rows<IPA_C, IPA_PV>(ea, warp, lane);
-    }
+          write_row_direct<IPA_C, IPA_PV>(tmem + lane_off, half, DZ, a.Cz, a.RCz / a.Cz, inv, dead, in_range,
+                                          a.z1f + (static_cast<int64_t>(b) * L + rrow) * DZ,
+                                          IPA_SPAN(a.out, orow * a.F, a.F, nrows * a.F, a.err),
+                                          a.uagg != nullptr ? IPA_SPAN(a.uagg, orow * a.RCz, a.RCz, nrows * a.RCz, a.err)
+                                                            : nullptr,
+                                          g0, g1, g2, cn, etr);
+          if (tid == 0) PAIR_SPAN(21);
+        }
+      } else {
+        const int pitch = stage_pitch(DZ);
+        float* stage = reinterpret_cast<float*>(smem + SP_QP);
+        if (all_ok) {
+          tc_fence_after();
+          const float inv = dead ? 0.f : 1.f / lt;
+          float* orow = stage + r * pitch;
+          // tensor memory holds [O_pair | O_v]; the stage row is [O_v | O_pair | frame]
+          for (int c0 = o_lo; c0 < o_hi; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tmem + c0 + lane_off, o);
+            tmem_ld_wait();
+            const int dstc = c0 < DZ ? 64 + c0 : c0 - DZ;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(orow + dstc + e) =
+                  make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                              __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          }
+          if (half == 0) stage_frame(orow + 64 + DZ, g0, g1, g2, cn, dead);
+        }
+        tc_fence_before();
+        named_bar_sync(1, NSOFT);
+        if (tid == 0) PAIR_SPAN(11);
+        if (!*abort_flag) {
+          EpilogueArgs ea{stage, DZ, a.Cz, a.RCz, a.F, a.H, L, b, h, row0, a.z1f, a.out};
+          ea.uagg = a.uagg;
+          ea.rows = static_cast<int64_t>(a.B) * L * a.H;
+          ea.err = a.err;
+#ifdef IPA_TRACE
+          ea.trace = (blockIdx.x < 4096 && warp == 0) ? &g_pair_span[blockIdx.x][16] : nullptr;
+#endif
+          write_rows<IPA_C, IPA_PV>(ea, warp, lane);
+        }
+      }
+    } else if (a.tma_epi) {
+      // the z1 boxes the producer loaded must land before the CTA ends
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(P_ZFULL), 0, abort_flag)) && lane == 0)
+        fail(DEV_TIMEOUT_FULL);
     }
   }
 
@@ -690,6 +802,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
 }  // namespace
 
 bool ipa_pair_supported(int DZ) { return DZ == 128 || DZ == 256; }
+
+// Key split of the last, partial wave.  T pair tiles on P resident CTA pairs
+// run floor(T / P) full waves and a tail of r = T mod P tiles that leaves
+// P - r pairs idle for a whole tile.  Splitting each tail tile's nkp key
+// tiles into S chunks runs the tail as ceil(r S / P) rounds of
+// ceil(nkp / S) key tiles.  In units of one key tile's time, a CTA pair's
+// set-up, Q load and output pass cost about 5 (event clocks of the tracing
+// build: ~10 us against ~2 us per key tile), and the merge about
+// 1 + (S - 1) / 2.  S is the cheapest of 2 .. MAX_SPLIT under that cost,
+// taken when it saves at least a tenth of the tail and the partials fit the
+// workspace's reserve.
+SplitPlan ipa_split_plan(int T, int nkp, int P, int64_t max_tiles, int64_t max_chunks) {
+  SplitPlan none{T, 1};
+  if (T <= 0 || P <= 0 || nkp < 2) return none;
+  const int r = T % P;
+  if (r == 0) return none;
+  constexpr double kFixed = 5.0;
+  double best = 0.9 * (nkp + kFixed);
+  int bs = 1;
+  for (int S = 2; S <= MAX_SPLIT && S <= nkp; ++S) {
+    if (r > max_tiles || static_cast<int64_t>(r) * S > max_chunks) break;
+    const int rounds = (r * S + P - 1) / P;
+    const double cost = rounds * ((nkp + S - 1) / S + kFixed) + 1.0 + 0.5 * (S - 1);
+    if (cost < best) {
+      best = cost;
+      bs = S;
+    }
+  }
+  return bs == 1 ? none : SplitPlan{T - r, bs};
+}
 
 cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
   unsigned char* ws = a.ws;
@@ -738,10 +880,26 @@ cudaError_t ipa_launch_core_pair(const IpaLaunch& a, cudaStream_t stream) {
       t.tma_epi = 1;
   }
   const int pairs = static_cast<int>(bh) * t.nqp;
+  // one CTA per SM (shared memory), so P = SMs / 2 resident pairs; the
+  // training forward (log-sum-exp and pair aggregate of whole rows) is not split
+  SplitPlan plan{pairs, 1};
+  if (a.lse == nullptr && a.uagg == nullptr && w.split_tiles > 0) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      plan = ipa_split_plan(pairs, t.nkp, sms / 2, w.split_tiles, w.split_chunks);
+  }
+  t.split_first = plan.first;
+  t.split_s = plan.S;
+  t.part = reinterpret_cast<float*>(ws + w.split);
+  t.ticket = reinterpret_cast<int*>(ws + w.ticket);
+  t.part_extent = w.split_chunks * 2 * (a.DZ + 67) * 128;
+  t.ticket_extent = static_cast<int>(2 * w.split_tiles);
+  const int blocks = plan.first + (pairs - plan.first) * plan.S;
   t.trace_cta0 = 0;
   t.trace_cta1 = 1;   // the peer CTA of the first pair
-  ipa_attention_pair_kernel<<<static_cast<unsigned>(2 * pairs), NT, SP_ALLOC, stream>>>(tqh, tkh, tz2k, tz2v, tvh, tz1,
-                                                                                         tz1f, tout, t);
+  ipa_attention_pair_kernel<<<static_cast<unsigned>(2 * blocks), NT, SP_ALLOC, stream>>>(tqh, tkh, tz2k, tz2v, tvh, tz1,
+                                                                                          tz1f, tout, t);
   return cudaGetLastError();
 }
 

@@ -59,6 +59,8 @@ struct TileArgs {
   __half* z1h;     // [B, L, DZ]
   __half* z2h;     // [B, L, DZ]
   int* err;        // DEV_NONFINITE when a pair factor does not survive the fp16 rounding
+  int* ticket;     // the core's key-split tickets, zeroed here (nticket ints)
+  int nticket;
 };
 
 // |x| >= 65520 (or NaN) does not survive the rounding to fp16
@@ -152,6 +154,8 @@ __global__ void __launch_bounds__(256) ipa_tile_kernel(const TileArgs a) {
   const int J = blockIdx.x, b = blockIdx.y, panel = blockIdx.z, tid = threadIdx.x;
   const int i0 = J * KT;
   __shared__ float red[2][4];
+  if ((J | b | panel) == 0)
+    for (int e = tid; e < a.nticket; e += blockDim.x) *IPA_AT(a.ticket, e, a.nticket, a.err) = 0;
   if (panel > 0) {
     ipa_tile_copy_pairs(a, b, i0, panel, tid);
     return;
@@ -475,6 +479,8 @@ cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
   ta.z2h = reinterpret_cast<__half*>(ws + w.z2);
   ta.z1h = reinterpret_cast<__half*>(ws + w.z1h);
   ta.err = a.err;
+  ta.ticket = reinterpret_cast<int*>(ws + w.ticket);
+  ta.nticket = static_cast<int>(2 * w.split_tiles);
   ipa_tile_kernel<<<dim3(a.nkt, a.B, a.DZ > 0 ? a.DZ / 64 : 1), 256, 0, stream>>>(ta);
 
   RowArgs r{};
@@ -506,7 +512,7 @@ cudaError_t ipa_launch_prologue(const IpaLaunch& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz) {
+IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz, bool with_split) {
   (void)RCz;
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   IpaWorkspace w{};
@@ -529,6 +535,14 @@ IpaWorkspace ipa_workspace_layout(int B, int L, int H, int DZ, int RCz) {
   w.headc = o; o = up(o + static_cast<size_t>(H) * 4);
   w.wqp = o; o = up(o + static_cast<size_t>(H) * DZ * 4);
   w.err = o; o = up(o + 16);
+  w.split = w.ticket = o;
+  if (with_split && ipa_pair_supported(DZ)) {
+    const int64_t T = static_cast<int64_t>(B) * H * ((L + 255) / 256);
+    w.split_tiles = T < kSplitPairs ? T : kSplitPairs;
+    w.split_chunks = 2 * w.split_tiles;
+    w.split = o; o = up(o + static_cast<size_t>(w.split_chunks) * 2 * (DZ + 67) * 128 * 4);
+    w.ticket = o; o = up(o + static_cast<size_t>(w.split_tiles) * 2 * 4);
+  }
   w.total = o;
   return w;
 }

@@ -88,8 +88,15 @@ def test_training_forward_statistics(cuda_device, name):
     dev = to_dev({k: inp[k] for k in api.IPA_INPUTS})
     out, lse, U = api.ipa_attn_train(dev)
     torch.cuda.synchronize()
-    # the training forward's output is the inference forward's, bit for bit
-    assert torch.equal(out, api.ipa_attn(dev))
+    # the training forward runs every pair tile whole; the inference forward
+    # may run the last, partial wave as key chunks whose P is rounded against
+    # each chunk's own maximum, so the two agree within the rounding of P
+    # (bit for bit where no tile is split, as in the tiny preset)
+    inf = api.ipa_attn(dev)
+    rel = float((out - inf).norm() / out.norm())
+    assert rel < 1e-3, rel
+    if name == "tiny":
+        assert torch.equal(out, inf)
     lse_ref, U_ref = ipa_forward_stats(inp)
     lse_g = lse.cpu().numpy()
     live = np.isfinite(lse_ref)
