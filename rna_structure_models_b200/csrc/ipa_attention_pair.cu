@@ -586,38 +586,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     // key-split tail: each chunk stores its partial accumulators, row
     // maximum and half sums; the chunk that finishes its tile last (ticket)
     // merges all chunks in chunk order into tensor memory, so the result does
-    // not depend on which chunk that is, and runs the output pass
+    // not depend on which chunk that is, and runs the output pass.  A chunk's
+    // block holds the accumulators as groups of four columns,
+    // [OW / 4][128 rows][4] (a warp's float4 stores cover 512 contiguous
+    // bytes), then the row maximum and the two half sums, [3][128].
     bool epi = true;
     if (chunk >= 0) {
       const int OW3 = OW + 3;
       const int64_t qc = pair - a.split_first;   // (split tile) S + chunk
       const int64_t blk_floats = static_cast<int64_t>(OW3) * 128;
-      float* mine = IPA_SPAN(a.part, (2 * qc + rank) * blk_floats, blk_floats, a.part_extent, a.err);
+      const int64_t mine = (2 * qc + rank) * blk_floats;   // this chunk-CTA's block in part
       if (all_ok) {
         tc_fence_after();
         for (int c0 = o_lo; c0 < o_hi; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tmem + c0 + lane_off, o);
           tmem_ld_wait();
+          float4* m4 = IPA_SPAN(reinterpret_cast<float4*>(a.part), mine / 4 + (c0 / 4) * 128, 8 * 128,
+                                a.part_extent / 4, a.err);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mine[(c0 + e) * 128 + r] = __uint_as_float(o[e]);
+          for (int g = 0; g < 8; ++g)
+            m4[g * 128 + r] = make_float4(__uint_as_float(o[4 * g]), __uint_as_float(o[4 * g + 1]),
+                                          __uint_as_float(o[4 * g + 2]), __uint_as_float(o[4 * g + 3]));
         }
-        if (half == 0) mine[OW * 128 + r] = m_used;
-        mine[(OW + 1 + half) * 128 + r] = l;
+        if (half == 0) *IPA_AT(a.part, mine + OW * 128 + r, a.part_extent, a.err) = m_used;
+        *IPA_AT(a.part, mine + (OW + 1 + half) * 128 + r, a.part_extent, a.err) = l;
       }
-      __threadfence();
+      // the barrier orders every thread's stores before thread 0's device-
+      // scope fence, which orders them before the ticket (fences are
+      // cumulative); the merging CTA fences after reading the ticket
       named_bar_sync(1, NSOFT);
       volatile int* last = reinterpret_cast<volatile int*>(smem + SP_AUX + AX_LAST);
       if (tid == 0) {
         int* tk = IPA_AT(a.ticket, 2 * (qc / a.split_s) + rank, a.ticket_extent, a.err);
+        __threadfence();
         const bool fin = atomicAdd(tk, 1) == a.split_s - 1;
-        if (fin) *tk = 0;   // every chunk of the tile has counted: ready for the next call
+        if (fin) {
+          *tk = 0;   // every chunk of the tile has counted: ready for the next call
+          __threadfence();
+        }
         *last = fin ? 1 : 0;
       }
       named_bar_sync(1, NSOFT);
       epi = *last != 0;
       if (epi) {
-        __threadfence();
         const float* c0p = a.part + (2 * (qc - chunk) + rank) * blk_floats;   // chunk 0 of this tile
         const int S = a.split_s;
         float ms[MAX_SPLIT], wt[MAX_SPLIT];
@@ -642,10 +654,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           float v[MAX_SPLIT][16];
 #pragma unroll
           for (int s = 0; s < MAX_SPLIT; ++s) {
-            const float* src = c0p + 2 * s * blk_floats + c0 * 128 + r;
+            const float4* src = reinterpret_cast<const float4*>(c0p + 2 * s * blk_floats) + (c0 / 4) * 128 + r;
             const bool other = s < S && s != chunk;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[s][e] = other ? __ldcg(src + e * 128) : 0.f;
+            for (int g = 0; g < 4; ++g) {
+              const float4 x = other ? __ldcg(src + g * 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+              v[s][4 * g] = x.x;
+              v[s][4 * g + 1] = x.y;
+              v[s][4 * g + 2] = x.z;
+              v[s][4 * g + 3] = x.w;
+            }
           }
           tmem_ld_wait();
           float acc[16];

@@ -117,8 +117,9 @@ def test_ipa_forward_training_and_gradients(cuda_device, L, Cz):
 
 
 def test_ipa_production_width_at_length_2048(cuda_device):
-    """The pair kernel's production shape (R Cz = 256, TMA output pass) and
-    the gradient passes at a length spanning many tiles, in both builds."""
+    """The pair kernel's production shape (R Cz = 256, TMA output pass), its
+    key-split tail and the gradient passes at a length spanning many tiles,
+    in both builds."""
     inp = ipa_inputs(IpaDims(B=1, L=2048, H=4, Cz=128), 31)
     inp["mask"][0, 2000:] = False
     dev = to_dev({k: inp[k] for k in api.IPA_INPUTS})
@@ -126,7 +127,10 @@ def test_ipa_production_width_at_length_2048(cuda_device):
     def run():
         o, lse, u = api.ipa_attn_train(dev)
         g_out = torch.randn(o.shape, device="cuda", generator=torch.Generator(device="cuda").manual_seed(5))
-        return {"train": [o, lse, u], "grads": api.ipa_attn_backward(dev, o, lse, u, g_out)}
+        # the inference call splits its tiles' keys in two chunks (partial
+        # accumulators, tickets, merge), the training call does not
+        return {"infer": api.ipa_attn(dev), "train": [o, lse, u],
+                "grads": api.ipa_attn_backward(dev, o, lse, u, g_out)}
 
     assert_same(*both_builds(run), "ipa L=2048")
 
