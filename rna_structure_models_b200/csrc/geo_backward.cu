@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(BW_ROWS * BW_SPLIT, M <= 4 ? 2 : 1) geo_bwd_ro
         const uint4 u1 = *reinterpret_cast<const uint4*>(pr + 16);
         const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-        for (int k = 0; k < BW_CHUNK; ++k) allowed |= ((w[k >> 2] >> (8 * (k & 3))) & 0xffu) ? (1u << k) : 0u;
+        for (int q = 0; q < BW_CHUNK / 4; ++q) allowed |= nonzero_byte_bits(w[q]) << (4 * q);
       } else {
         for (int k = 0; k < BW_CHUNK && j0 + k < N; ++k) allowed |= pr[k * a.pms[3]] ? (1u << k) : 0u;
       }

@@ -30,7 +30,25 @@ __device__ __forceinline__ float softplus_stable(float x) {
 // used by the aggregation kernel (in packed pairs: fma.rn.f32x2 etc. round
 // each lane exactly like the scalar operation), the attention-map kernel and
 // the gradient kernels, so all of them see identical values.  The distance
-// is the hardware square-root approximation (sqrt.approx.f32, exact at 0).
+// is the hardware square-root approximation with subnormals flushed
+// (sqrt.approx.ftz.f32: exact at 0; a squared distance below the smallest
+// normal float, |d| < 1.1e-19, counts as 0).
+__device__ __forceinline__ float dist_sqrt(float d2) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d2));
+  return y;
+}
+
+// Bit t (t < 4) set iff byte t of w is nonzero.  ((b & 0x7f) + 0x7f) | b has
+// its top bit set iff the byte b is nonzero, with no carry into the next byte
+// ((b & 0x7f) + 0x7f <= 0xfe); shifted to bit 8 t, the four flags are
+// gathered into bits 24 .. 27 by one multiplication by 2^24 + 2^17 + 2^10 +
+// 2^3, whose sixteen partial products land on distinct bits.
+__device__ __forceinline__ uint32_t nonzero_byte_bits(uint32_t w) {
+  const uint32_t h = ((((w & 0x7f7f7f7fu) + 0x7f7f7f7fu) | w) & 0x80808080u) >> 7;
+  return ((h * 0x01020408u) >> 24) & 0xfu;
+}
+
 struct GeoPair {
   float s;            // log2(e) (A dot - B dist) / sqrt(3) + frame biases
   float dot, dist;    // <qd, kd>, |qp - kp|
@@ -45,7 +63,7 @@ __device__ __forceinline__ GeoPair geo_pair(const float4 q0, const float4 q1, co
   g.dy = __fsub_rn(q1.y, k1.y);
   g.dz = __fsub_rn(q1.z, k1.z);
   const float d2 = fmaf(g.dx, g.dx, fmaf(g.dy, g.dy, __fmul_rn(g.dz, g.dz)));
-  g.dist = sm100::sqrt_approx(d2);
+  g.dist = dist_sqrt(d2);
   g.s = __fadd_rn(__fadd_rn(fmaf(A, g.dot, -__fmul_rn(Bd, g.dist)), q0.w), k0.w);
   return g;
 }

@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, 1) geo_attn_kernel(const
         const uint4 u1 = *reinterpret_cast<const uint4*>(p + 16);
         const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-        for (int k = 0; k < 32; ++k) allowed |= ((w[k >> 2] >> (8 * (k & 3))) & 0xffu) ? (1u << k) : 0u;
+        for (int q = 0; q < 8; ++q) allowed |= nonzero_byte_bits(w[q]) << (4 * q);
       } else {
         for (int k = 0; k < GEO_CHUNK && j0 + k < N; ++k) allowed |= p[k * pj] ? (1u << k) : 0u;
       }
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(GEO_ROWS * GEO_SPLIT, 1) geo_attn_kernel(const
       const float2 dy = sub_f32x2(py, make_float2(w2.z, w2.w));
       const float2 dz = sub_f32x2(pz, make_float2(w3.x, w3.y));
       const float2 d2 = fma_f32x2(dx, dx, fma_f32x2(dy, dy, mul_f32x2(dz, dz)));
-      const float2 dist = make_float2(sqrt_approx(d2.x), sqrt_approx(d2.y));
+      const float2 dist = make_float2(dist_sqrt(d2.x), dist_sqrt(d2.y));
       float2 sv = add_f32x2(fma_f32x2(A2, dot, mul_f32x2(nB2, dist)), make_float2(w1.z, w1.w));
       if (!((allowed >> (2 * t)) & 1u)) sv.x = -INFINITY;
       if (!((allowed >> (2 * t + 1)) & 1u)) sv.y = -INFINITY;
@@ -442,10 +442,7 @@ __global__ void __launch_bounds__(256, 3) geo_map_kernel(const MapArgs a) {
     uint64_t allow = 0u;
 #pragma unroll
     for (int rr = 0; rr < MAP_ROWS; ++rr) {
-      // one bit per nonzero byte: x = sum_t [byte t != 0] 2^(8 t); x * 0x01020408
-      // gathers bit t of the nibble at bits 24 + t (no carries between terms)
-      const uint32_t x = __vcmpne4(wv[rr], 0u) & 0x01010101u;
-      allow |= static_cast<uint64_t>(((x * 0x01020408u) >> 24) & 0xfu) << (4 * rr);
+      allow |= static_cast<uint64_t>(nonzero_byte_bits(wv[rr])) << (4 * rr);
     }
     // key terms in lane pairs: keys (0, 1) and (2, 3)
     float2 kx[2], ky[2], kz[2], px[2], py[2], pz[2], kb[2];
@@ -478,7 +475,7 @@ __global__ void __launch_bounds__(256, 3) geo_map_kernel(const MapArgs a) {
         const float2 dy = sub_f32x2(make_float2(q1.y, q1.y), py[u]);
         const float2 dz = sub_f32x2(make_float2(q1.z, q1.z), pz[u]);
         const float2 d2 = fma_f32x2(dx, dx, fma_f32x2(dy, dy, mul_f32x2(dz, dz)));
-        const float2 dist = make_float2(sqrt_approx(d2.x), sqrt_approx(d2.y));
+        const float2 dist = make_float2(dist_sqrt(d2.x), dist_sqrt(d2.y));
         const float2 s = add_f32x2(add_f32x2(fma_f32x2(A2, dot, mul_f32x2(nB2, dist)), make_float2(q0.w, q0.w)), kb[u]);
         const float2 y = sub_f32x2(s, make_float2(st.x, st.x));
         const bool ok0 = st.y > 0.f && ((al >> (2 * u)) & 1u) != 0;
