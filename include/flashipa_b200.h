@@ -114,7 +114,12 @@ typedef struct {
 } ipa_params_t;
 
 /* Bytes of device workspace ipa_attn_fwd needs for these params (0 if the
- * params are invalid).  Pure host function. */
+ * params are invalid).  Pure host function.  Linear in B L H plus, for pair
+ * widths 128 and 256, a bounded reserve for the key-split tail of the core:
+ * the last, partial wave of (batch, head, 256-query) tiles may run as
+ * chunks of consecutive key tiles whose partial accumulators are stored
+ * there and merged by the chunk that finishes last (at most 2 x 74 chunks,
+ * 49 MB at a pair width of 256). */
 IPA_API size_t ipa_attn_workspace_size(const ipa_params_t* p);
 
 /* Enqueue the fused IPA core on `stream` (a cudaStream_t, NULL = legacy
@@ -137,7 +142,10 @@ IPA_API ipa_status_t ipa_attn_fwd(const ipa_params_t* p,
  * fp16 operands into the workspace; ipa_attn_core runs the fused attention
  * pass from that workspace into `out`.  The core reads only the workspace,
  * so it must follow a prologue with the same params and workspace on the
- * same stream.  ipa_attn_fwd == prologue then core. */
+ * same stream; it may run several times after one prologue.  After a call
+ * that reported an error through dev_err, run the prologue again before the
+ * next core (the prologue also resets the key-split tickets in the
+ * workspace).  ipa_attn_fwd == prologue then core. */
 IPA_API ipa_status_t ipa_attn_prologue(const ipa_params_t* p,
                                const ipa_tensor_t* q, const ipa_tensor_t* k, const ipa_tensor_t* v,
                                const ipa_tensor_t* q_pts, const ipa_tensor_t* k_pts,
