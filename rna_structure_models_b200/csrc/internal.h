@@ -69,8 +69,17 @@ cudaError_t ipa_launch_core(const IpaLaunch& a, cudaStream_t stream);
 // forward prologue's outputs (recomputed) followed by the backward's.
 struct IpaBwdWorkspace {
   IpaWorkspace fwd;
-  size_t doh, du, qp, rowd, dqh, dqp, rsq, dkh, dva, dz2, csk, pts, gsum, wb_part, g_part, total;
+  size_t doh, du, qp, rowd, dqh, dqp, rsq, dkh, dva, dz2, csk, pts, gsum, wb_part, g_part;
+  // query split of the key pass's last wave: partials of up to ksplit_chunks
+  // chunks ([DZ + 138][128] floats each) and a ticket per split key tile
+  size_t kpart, kticket;
+  int64_t ksplit_tiles, ksplit_chunks;
+  size_t total;
 };
+
+// Resident CTAs of the gradient passes on a B200 (148 SMs, one CTA per SM):
+// the key-pass split runs its chunks in one round, at most this many.
+constexpr int kBwdSlots = 148;
 IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz);
 
 struct IpaBwdLaunch {

@@ -102,6 +102,13 @@ struct BwdArgs {
   const float* pts;      // [B*H, L, 24]: query points gq - cen (12) | key points gk - cen (12), fp32
   float* gsum;           // [B*H, L]: sum_i dS_ij |gq_i - gk_j|^2 per key (the d gamma sum, one side only)
   int* err;
+  // key pass, query split of the last wave: key tiles [split_first, nkb) run
+  // as split_s chunks of consecutive 32-query tiles (split_s == 1: none)
+  int split_first, split_s;
+  float* part;           // per chunk: [DZ + 128][128] accumulators (float4 groups), [2][5][128] half sums
+  int64_t part_extent;   // floats in part
+  int* ticket;           // per split key tile: chunks finished (zero between calls)
+  int ticket_extent;
 };
 
 __device__ __forceinline__ uint64_t kd128(uint32_t a) { return smem_desc(a, 16, 1024, 2); }      // K-major SW128
@@ -122,6 +129,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
 struct RowsArgs {
   int B, L, H, DZ, RCz, Cz, F;
   bool z1_half;          // Q_pair from the fp16 z1 (as the CTA-pair forward core), else from fp32 z1
+  int pair_cpl;          // 4 or 8: pair columns per lane from 16-byte loads (contiguous fp32 rows, R Cz = DZ); 0: per element
   View g_out, out, lse, uagg;
   const float4* frame;
   const float4* cen;
@@ -136,13 +144,87 @@ struct RowsArgs {
   View q_pts, k_pts;
   float* pts;            // [B*H, L, 24]
   int* err;
+  int* kticket;          // the key pass's split tickets, zeroed here (nkticket ints)
+  int nkticket;
 };
 
+// Pair block of one row when its rows are contiguous fp32 and R Cz = DZ:
+// lane l owns the CPL = DZ / 32 consecutive columns [CPL l, CPL l + CPL) (one
+// factor r, features cc .. cc + CPL - 1), every operand read with 16-byte
+// loads issued together; the same per-element arithmetic as the general loop.
+template <int CPL>
+__device__ __forceinline__ void bwd_pair_cols(const RowsArgs& a, int lane, bool live, int64_t gbase, int64_t ubase,
+                                              int64_t bi, int h, __half* dur, __half* qpr, float& part) {
+  const int c0 = CPL * lane, r = c0 / a.Cz, cc = c0 % a.Cz;
+  float z[CPL], w[CPL], gp[CPL], u[CPL], zh[CPL];
+  const float4* z4 = reinterpret_cast<const float4*>(a.z1f + bi * a.DZ + c0);
+  const float4* w4 = reinterpret_cast<const float4*>(a.wqp + static_cast<int64_t>(h) * a.DZ + c0);
+  const float4* g4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.g_out.p) + gbase +
+                                                     (IPA_C + 4 * IPA_PV + cc));
+  const float4* u4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.uagg.p) + ubase +
+                                                     r * a.uagg.s[3] + cc);
+#pragma unroll
+  for (int q = 0; q < CPL / 4; ++q) {
+    const float4 zv = z4[q], wv = w4[q];
+    const float4 gv = live ? g4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 uv = live ? u4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+    z[4 * q] = zv.x; z[4 * q + 1] = zv.y; z[4 * q + 2] = zv.z; z[4 * q + 3] = zv.w;
+    w[4 * q] = wv.x; w[4 * q + 1] = wv.y; w[4 * q + 2] = wv.z; w[4 * q + 3] = wv.w;
+    gp[4 * q] = gv.x; gp[4 * q + 1] = gv.y; gp[4 * q + 2] = gv.z; gp[4 * q + 3] = gv.w;
+    u[4 * q] = uv.x; u[4 * q + 1] = uv.y; u[4 * q + 2] = uv.z; u[4 * q + 3] = uv.w;
+  }
+  if (a.z1_half) {
+    const __half* zr = a.z1h + bi * a.DZ + c0;
+    uint32_t hw[CPL / 2];
+    if constexpr (CPL == 8) {
+      const uint4 t = *reinterpret_cast<const uint4*>(zr);
+      hw[0] = t.x; hw[1] = t.y; hw[2] = t.z; hw[3] = t.w;
+    } else {
+      const uint2 t = *reinterpret_cast<const uint2*>(zr);
+      hw[0] = t.x; hw[1] = t.y;
+    }
+#pragma unroll
+    for (int e = 0; e < CPL / 2; ++e) {
+      const float2 f = unpack_half2(hw[e]);
+      zh[2 * e] = f.x;
+      zh[2 * e + 1] = f.y;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) zh[e] = z[e];
+  }
+  uint32_t dw[CPL / 2], qw[CPL / 2];
+#pragma unroll
+  for (int e = 0; e < CPL; e += 2) {
+    float d2v[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      d2v[k] = 0.f;
+      if (live) {
+        d2v[k] = __half2float(__float2half_rn(z[e + k] * gp[e + k]));
+        part = fmaf(d2v[k], u[e + k], part);
+      }
+    }
+    dw[e / 2] = pack_half2(d2v[0], d2v[1]);
+    qw[e / 2] = pack_half2(zh[e] * w[e], zh[e + 1] * w[e + 1]);
+  }
+  if constexpr (CPL == 8) {
+    *reinterpret_cast<uint4*>(dur + c0) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+    *reinterpret_cast<uint4*>(qpr + c0) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+  } else {
+    *reinterpret_cast<uint2*>(dur + c0) = make_uint2(dw[0], dw[1]);
+    *reinterpret_cast<uint2*>(qpr + c0) = make_uint2(qw[0], qw[1]);
+  }
+}
+
 // One warp per (b, i, h), heads fastest.  Lane l: scalar channel l (< 16),
-// point coordinate l (< 24: point l / 3, axis l % 3), pair columns l + 32 k.
+// point coordinate l (< 24: point l / 3, axis l % 3), pair columns l + 32 k
+// (or, for contiguous fp32 rows, the lane's run of DZ / 32 columns).
 __global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e < a.nkticket; e += blockDim.x) *IPA_AT(a.kticket, e, a.nkticket, a.err) = 0;
   if (wid >= static_cast<int64_t>(a.B) * a.L * a.H) return;
   const int h = static_cast<int>(wid % a.H);
   const int64_t bi = wid / a.H;
@@ -199,7 +281,9 @@ __global__ void __launch_bounds__(256) ipa_bwd_rows_kernel(const RowsArgs a) {
   __half* dur = IPA_SPAN(a.du, bhl * a.DZ, a.DZ, nbhl * a.DZ, a.err);
   __half* qpr = IPA_SPAN(a.qp, bhl * a.DZ, a.DZ, nbhl * a.DZ, a.err);
   const int64_t ubase = b * a.uagg.s[0] + i * a.uagg.s[1] + h * a.uagg.s[2];
-  for (int c = lane; c < a.DZ; c += 32) {
+  if (a.pair_cpl == 8) bwd_pair_cols<8>(a, lane, live, gbase, ubase, bi, h, dur, qpr, part);
+  else if (a.pair_cpl == 4) bwd_pair_cols<4>(a, lane, live, gbase, ubase, bi, h, dur, qpr, part);
+  else for (int c = lane; c < a.DZ; c += 32) {
     float duv = 0.f;
     if (c < a.RCz && live) {
       const int r = c / a.Cz, cc = c % a.Cz;
@@ -625,6 +709,7 @@ __device__ __forceinline__ void bwd_q_body(const int blk, const CUtensorMap& tm_
 // S^T / dP^T buffer t: S^T at K_TM_SD + 64 t, dP^T right after it (one N = 64
 // accumulator for their pair parts)
 constexpr uint32_t K_TM_DZ2 = 0, K_TM_DKH = 256, K_TM_DVA = 320, K_TM_SD = 384;
+constexpr int MAX_KSPLIT = 5;   // query chunks of a split key tile
 
 struct KLayout {
   uint32_t kh, vh, z2, stg, stg_bytes, aux, total;
@@ -649,7 +734,8 @@ constexpr uint32_t KA_Q = 0, KA_OQ = 1536, KA_BAR = 1600, KA_QPTS = 2048;
 enum { KB_KFULL = 0, KB_SFULL0, KB_PFULL0 = KB_SFULL0 + 2, KB_ACC0 = KB_PFULL0 + 2, KB_DRAIN = KB_ACC0 + 2,
        KB_FULL0, KB_EMPTY0 = KB_FULL0 + MAX_NS, KB_COUNT = KB_EMPTY0 + MAX_NS };
 constexpr uint32_t KA_TMEM = KA_BAR + 8 * KB_COUNT, KA_ABORT = KA_TMEM + 8, KA_PAIR = KA_ABORT + 8;
-static_assert(KA_PAIR + 64 <= KA_QPTS, "key-pass aux area overlaps the query points");
+constexpr uint32_t KA_LAST = KA_PAIR + 64;   // int: this CTA finishes its split key tile
+static_assert(KA_LAST + 4 <= KA_QPTS, "key-pass aux area overlaps the query points");
 
 __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_kh, const CUtensorMap& tm_vh,
                                            const CUtensorMap& tm_z2, const CUtensorMap& tm_qh,
@@ -661,11 +747,20 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
   unsigned char* smem = smem_raw + (sb - raw_u32);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nkp = (a.L + 127) / 128;
-  const int J2 = blk % nkp;                     // 128-key tile
-  const int bh = blk / nkp;
+  // a split key tile's chunk c covers query tiles [c nqa / S, (c + 1) nqa / S)
+  const int nqa = (a.L + BT - 1) / BT;          // 32-query tiles in all
+  int tile = blk, chunk = -1, ib = 0, nq = nqa;  // nq: query tiles this CTA runs, from ib
+  if (blk >= a.split_first) {
+    const int q = blk - a.split_first;
+    tile = a.split_first + q / a.split_s;
+    chunk = q % a.split_s;
+    ib = chunk * nqa / a.split_s;
+    nq = (chunk + 1) * nqa / a.split_s - ib;
+  }
+  const int J2 = tile % nkp;                    // 128-key tile
+  const int bh = tile / nkp;
   const int b = bh / a.H, h = bh % a.H;
   const int L = a.L, DZ = a.DZ, np = DZ / 64, NS = a.ns;
-  const int nq = (L + BT - 1) / BT;             // 32-query tiles
   const KLayout lay = k_layout(DZ, NS);
   float4* qinfo = reinterpret_cast<float4*>(smem + lay.aux + KA_Q);
   float4* oqs = reinterpret_cast<float4*>(smem + lay.aux + KA_OQ);
@@ -723,7 +818,8 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       float4 oqv, sq, v[3];
       float2 rd;
     };
-    auto fetch = [&](int i, RowVals& r) {
+    auto fetch = [&](int il, RowVals& r) {
+      const int i = ib + il;                    // global 32-query tile
       r.oqv = a.oq[b * a.nqt + (i * BT) / QT];
       const int qi = i * BT + lane;
       r.sq = qi < L ? a.rowq[static_cast<int64_t>(bh) * L + qi] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -753,11 +849,12 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       if (lane == 0) {
         const uint32_t st = sb + lay.stg + s * lay.stg_bytes;
         mbar_arrive_expect_tx(bar(KB_FULL0 + s), lay.stg_bytes);
-        tma_load_3d(st, &tm_qh, bar(KB_FULL0 + s), 0, i * BT, bh);
-        tma_load_3d(st + 4096, &tm_do, bar(KB_FULL0 + s), 0, i * BT, bh);
+        const int q0 = (ib + i) * BT;
+        tma_load_3d(st, &tm_qh, bar(KB_FULL0 + s), 0, q0, bh);
+        tma_load_3d(st + 4096, &tm_do, bar(KB_FULL0 + s), 0, q0, bh);
         for (int p = 0; p < np; ++p) {   // interleaved panels: Q_pair p, then dU p
-          tma_load_4d(st + 8192 + 8192 * p, &tm_qp, bar(KB_FULL0 + s), 0, i * BT, p, bh);
-          tma_load_4d(st + 8192 + 8192 * p + 4096, &tm_du, bar(KB_FULL0 + s), 0, i * BT, p, bh);
+          tma_load_4d(st + 8192 + 8192 * p, &tm_qp, bar(KB_FULL0 + s), 0, q0, p, bh);
+          tma_load_4d(st + 8192 + 8192 * p + 4096, &tm_du, bar(KB_FULL0 + s), 0, q0, p, bh);
         }
         BWD_TR(1, i, 11);
       }
@@ -769,7 +866,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       const float n0 = fmaf(d0x, d0x, fmaf(d0y, d0y, d0z * d0z)), n1 = fmaf(d1x, d1x, fmaf(d1y, d1y, d1z * d1z));
       {
         float4 e = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
-        if (i * BT + lane < L) {
+        if ((ib + i) * BT + lane < L) {
           const float4 sq = cur.sq;
           const float rt0 = ch * (2.f * fmaf(sq.x, d0x, fmaf(sq.y, d0y, sq.z * d0z)) - pq * n0);
           const float rt1 = ch * (2.f * fmaf(sq.x, d1x, fmaf(sq.y, d1y, sq.z * d1z)) - pq * n1);
@@ -978,6 +1075,111 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       ok = false;
     }
     const bool all_ok = __all_sync(0xffffffffu, ok);
+    // query split: each chunk stores its accumulators (partial column pc:
+    // dZ2 [0, DZ) | dK_h [DZ, DZ + 64) | dV [DZ + 64, DZ + 128), as float4
+    // groups of columns, [(DZ + 128) / 4][128 rows][4]) and its five half
+    // sums ([2 halves][5][128]); the chunk that takes the last ticket adds the
+    // chunks in chunk order (its own from tensor memory and registers), so
+    // the result does not depend on which chunk that is, and writes the rows
+    // as a whole tile does.  No CTA waits for another.
+    bool epi = true;
+    if (chunk >= 0) {
+      constexpr int NSUM = 5;
+      const int OWK = DZ + 128;
+      const int64_t qc = blk - a.split_first;   // (split tile) S + chunk
+      const int64_t blk_floats = static_cast<int64_t>(OWK + 2 * NSUM) * 128;
+      const int64_t mine = qc * blk_floats;
+      auto tcol = [&](int pc) -> uint32_t {
+        return pc < DZ ? K_TM_DZ2 + pc : pc < DZ + 64 ? K_TM_DKH + (pc - DZ) : K_TM_DVA + (pc - DZ - 64);
+      };
+      // this thread's 32-column groups: its half of dZ2, of dK_h and of dV
+      const int ngrp = DZ / 64 + 2;
+      auto grp = [&](int g) -> int { return g < DZ / 64 ? half * (DZ / 2) + 32 * g : DZ + 64 * (g - DZ / 64) + 32 * half; };
+      float sums[NSUM] = {cs, co0, co1, co2, gsum};
+      if (all_ok) {
+        tc_fence_after();
+        for (int g = 0; g < ngrp; ++g) {
+          const int pc0 = grp(g);
+          uint32_t v[32];
+          tmem_ld32(tmem + tcol(pc0) + lane_off, v);
+          tmem_ld_wait();
+          float4* m4 = IPA_SPAN(reinterpret_cast<float4*>(a.part), mine / 4 + (pc0 / 4) * 128, 8 * 128,
+                                a.part_extent / 4, a.err);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            m4[e * 128 + r] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                          __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+#pragma unroll
+        for (int k = 0; k < NSUM; ++k)
+          *IPA_AT(a.part, mine + (OWK + half * NSUM + k) * 128 + r, a.part_extent, a.err) = sums[k];
+      }
+      // the barrier orders every thread's stores before thread 0's device-
+      // scope fence and ticket; the merging CTA fences after its ticket
+      named_bar_sync(1, NSOFT);
+      volatile int* last = reinterpret_cast<volatile int*>(smem + lay.aux + KA_LAST);
+      if (tid == 0) {
+        int* tk = IPA_AT(a.ticket, qc / a.split_s, a.ticket_extent, a.err);
+        __threadfence();
+        const bool fin = atomicAdd(tk, 1) == a.split_s - 1;
+        if (fin) {
+          *tk = 0;   // every chunk of the tile has counted: ready for the next call
+          __threadfence();
+        }
+        *last = fin ? 1 : 0;
+      }
+      named_bar_sync(1, NSOFT);
+      epi = *last != 0;
+      if (epi && all_ok) {
+        const float* c0p = a.part + (qc - chunk) * blk_floats;   // chunk 0 of this tile
+        const int S = a.split_s;
+#pragma unroll
+        for (int k = 0; k < NSUM; ++k) {
+          float acc = 0.f;
+#pragma unroll
+          for (int sc = 0; sc < MAX_KSPLIT; ++sc)
+            if (sc < S) acc += sc == chunk ? sums[k] : __ldcg(c0p + sc * blk_floats + (OWK + half * NSUM + k) * 128 + r);
+          sums[k] = acc;
+        }
+        cs = sums[0]; co0 = sums[1]; co1 = sums[2]; co2 = sums[3]; gsum = sums[4];
+        tc_fence_after();
+        for (int g = 0; g < ngrp; ++g) {
+#pragma unroll
+          for (int hsub = 0; hsub < 2; ++hsub) {   // 16 columns at a time, the other chunks' loads together
+            const int pc0 = grp(g) + 16 * hsub;
+            uint32_t o[16];
+            tmem_ld16(tmem + tcol(pc0) + lane_off, o);
+            float v[MAX_KSPLIT][16];
+#pragma unroll
+            for (int sc = 0; sc < MAX_KSPLIT; ++sc) {
+              const float4* src = reinterpret_cast<const float4*>(c0p + sc * blk_floats) + (pc0 / 4) * 128 + r;
+              const bool other = sc < S && sc != chunk;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float4 x = other ? __ldcg(src + q * 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[sc][4 * q] = x.x; v[sc][4 * q + 1] = x.y; v[sc][4 * q + 2] = x.z; v[sc][4 * q + 3] = x.w;
+              }
+            }
+            tmem_ld_wait();
+            float acc[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+#pragma unroll
+            for (int sc = 0; sc < MAX_KSPLIT; ++sc)
+              if (sc < S) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc[e] += sc == chunk ? __uint_as_float(o[e]) : v[sc][e];
+              }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(acc[e]);
+            tmem_st16(tmem + tcol(pc0) + lane_off, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+    }
+    if (epi) {
     named_bar_sync(1, NSOFT);   // every thread is past its last read of the stage area
     if (half == 1) {
       reinterpret_cast<float4*>(smem + lay.stg)[r] = make_float4(cs, co0, co1, co2);
@@ -1012,6 +1214,7 @@ __device__ __forceinline__ void bwd_k_body(const int blk, const CUtensorMap& tm_
       store32(K_TM_DVA + 32 * half, IPA_SPAN(a.dva, rowi * 64 + 32 * half, 32, nrow * 64, a.err));
       for (int c0 = half * (DZ / 2); c0 < (half + 1) * (DZ / 2); c0 += 32)
         store32(K_TM_DZ2 + c0, IPA_SPAN(a.dz2, rowi * DZ + c0, 32, nrow * DZ, a.err));
+    }
     }
   }
   tc_fence_before();
@@ -1334,8 +1537,39 @@ IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz) {
   w.gsum = o; o = up(o + bhl * 4);
   w.wb_part = o; o = up(o + static_cast<size_t>(B) * npb * H * DZ * 4);
   w.g_part = o; o = up(o + static_cast<size_t>(B) * nblk * H * 8);
+  const int64_t nkb = static_cast<int64_t>(B) * H * ((L + 127) / 128);
+  w.ksplit_chunks = nkb < kBwdSlots ? nkb : kBwdSlots;
+  w.ksplit_tiles = w.ksplit_chunks / 2;
+  w.kpart = o; o = up(o + static_cast<size_t>(w.ksplit_chunks) * (DZ + 138) * 128 * 4);
+  w.kticket = o; o = up(o + static_cast<size_t>(w.ksplit_tiles) * 4 + 4);
   w.total = o;
   return w;
+}
+
+// Query split of the key pass.  The grid is nqb query-pass CTAs, then nkb
+// key-pass CTAs, one per SM at a time (P resident).  When the last, partial
+// wave (r = (nqb + nkb) mod P CTAs) holds key-pass CTAs only, each of them
+// can run as S chunks of consecutive 32-query tiles, all chunks in one round
+// (r S <= P).  Cost in units of one 32-query tile (~2 us): a chunk pays
+// ceil(nq / S) tiles plus ~5 of set-up and output; the merging one ~1 + S / 2
+// more.  S is the cheapest of 2 .. MAX_KSPLIT when it saves a tenth.
+SplitPlan ipa_bwd_split_plan(int nqb, int nkb, int nq, int P, int64_t max_tiles, int64_t max_chunks) {
+  const int T = nqb + nkb;
+  SplitPlan none{nkb, 1};
+  if (P <= 0 || T < P || nq < 2) return none;
+  const int r = T % P;
+  if (r == 0 || r > nkb || r > max_tiles) return none;
+  constexpr double kFixed = 5.0;
+  double best = 0.9 * (nq + kFixed);
+  int bs = 1;
+  for (int S = 2; S <= MAX_KSPLIT && S <= nq && static_cast<int64_t>(r) * S <= max_chunks && r * S <= P; ++S) {
+    const double cost = (nq + S - 1) / S + kFixed + 1.0 + 0.5 * S;
+    if (cost < best) {
+      best = cost;
+      bs = S;
+    }
+  }
+  return bs == 1 ? none : SplitPlan{nkb - r, bs};
 }
 
 cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
@@ -1355,6 +1589,19 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   ra.B = B; ra.L = L; ra.H = H; ra.DZ = DZ; ra.RCz = f.RCz; ra.Cz = f.Cz; ra.F = f.F;
   ra.z1_half = ipa_pair_supported(DZ);
   ra.g_out = a.g_out; ra.out = a.out; ra.lse = a.lse; ra.uagg = a.uagg;
+  {
+    // 16-byte pair-block loads: fp32 rows with unit feature stride, every
+    // row start and factor start on a 16-byte boundary, whole columns per lane
+    auto al16 = [](const View& v, int n) {
+      bool ok = (reinterpret_cast<uintptr_t>(v.p) & 15u) == 0;
+      for (int d = 0; d < n; ++d) ok = ok && (v.s[d] % 4 == 0);
+      return ok;
+    };
+    const bool vec = f.RCz == DZ && (DZ == 128 || DZ == 256) && f.Cz % 8 == 0 && a.g_out.dtype == 0 &&
+                     a.g_out.s[3] == 1 && al16(a.g_out, 3) && (IPA_C + 4 * IPA_PV) % 4 == 0 && a.uagg.dtype == 0 &&
+                     a.uagg.s[4] == 1 && al16(a.uagg, 4);
+    ra.pair_cpl = vec ? DZ / 32 : 0;
+  }
   ra.frame = reinterpret_cast<const float4*>(ws + fw.frame);
   ra.cen = reinterpret_cast<const float4*>(ws + fw.cen);
   ra.rowq = reinterpret_cast<const float4*>(ws + fw.rowq);
@@ -1368,6 +1615,8 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   ra.q_pts = f.q_pts; ra.k_pts = f.k_pts;
   ra.pts = reinterpret_cast<float*>(ws + w.pts);
   ra.err = f.err;
+  ra.kticket = reinterpret_cast<int*>(ws + w.kticket);
+  ra.nkticket = static_cast<int>(w.ksplit_tiles);
   const int64_t warps = static_cast<int64_t>(B) * L * H;
   ipa_bwd_rows_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(ra);
   e = cudaGetLastError();
@@ -1398,6 +1647,8 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   ba.pts = reinterpret_cast<const float*>(ws + w.pts);
   ba.gsum = reinterpret_cast<float*>(ws + w.gsum);
   ba.err = f.err;
+  ba.split_first = 1 << 30;   // the query pass runs whole tiles
+  ba.split_s = 1;
 
   const uint64_t rowb = static_cast<uint64_t>(L) * DH * 2;
   // 3.-4. query and key passes, one grid
@@ -1435,7 +1686,19 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const int nqb = static_cast<int>(bh) * f.nqt;
     const int nkb = static_cast<int>(bh) * ((L + 127) / 128);
-    ipa_bwd_kernel<<<static_cast<unsigned>(nqb + nkb), NTH, smem, stream>>>(mp, ba, kb, nqb);
+    int dev = 0, sms = 0;
+    SplitPlan plan{nkb, 1};
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      plan = ipa_bwd_split_plan(nqb, nkb, (L + BT - 1) / BT, sms, w.ksplit_tiles, w.ksplit_chunks);
+    kb.split_first = plan.first;
+    kb.split_s = plan.S;
+    kb.part = reinterpret_cast<float*>(ws + w.kpart);
+    kb.part_extent = w.ksplit_chunks * (DZ + 138) * 128;
+    kb.ticket = reinterpret_cast<int*>(ws + w.kticket);
+    kb.ticket_extent = static_cast<int>(w.ksplit_tiles);
+    const int kblocks = plan.first + (nkb - plan.first) * plan.S;
+    ipa_bwd_kernel<<<static_cast<unsigned>(nqb + kblocks), NTH, smem, stream>>>(mp, ba, kb, nqb);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

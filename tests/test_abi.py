@@ -446,12 +446,18 @@ def bwd_args(B=1, L=64, H=4, R=2, Cz=16):
 
 def test_bwd_workspace_is_linear_in_L_and_zero_when_invalid():
     lib = api.library()
-    per = []
+    sizes = []
     for L in (2048, 4096, 8192, 16384):
         p = api.ipa_params(1, L, 12, 16, 4, 8, 2, 128)
-        per.append(lib.ipa_attn_bwd_workspace_size(ctypes.byref(p)) / L)
+        sizes.append(lib.ipa_attn_bwd_workspace_size(ctypes.byref(p)))
         assert lib.ipa_attn_bwd_workspace_size(ctypes.byref(p)) > lib.ipa_attn_workspace_size(ctypes.byref(p))
-    assert max(per) / min(per) < 1.02
+    Ls = np.array([2048, 4096, 8192, 16384], float)
+    marg = np.diff(np.array(sizes, float)) / np.diff(Ls)     # bytes per added residue
+    assert marg.max() / marg.min() < 1.02, marg
+    # plus a bounded constant: the key pass's split reserve (one round of
+    # chunks on the resident CTAs) and the per-block reduction rounding
+    const = sizes[0] - marg[0] * Ls[0]
+    assert abs(const) < 64 * 2 ** 20, const
     bad = api.ipa_params(1, 64, 4, 16, 4, 8, 2, 20)      # Cz not a multiple of 16
     assert lib.ipa_attn_bwd_workspace_size(ctypes.byref(bad)) == 0
 

@@ -182,6 +182,23 @@ def test_gradients_are_reproducible(cuda_device):
         assert np.array_equal(a[key], b[key]), key
 
 
+def test_gradients_with_the_key_pass_split(cuda_device):
+    """B = 2, L = 512, H = 12: 96 query-pass and 96 key-pass CTAs, one per SM
+    on 148 SMs, leave a last wave of 44 key-pass CTAs.  Each of those runs as
+    three chunks of its 16 query tiles; the chunk that finishes last adds the
+    partial sums in chunk order.  Every gradient against the oracle, and the
+    same bits on a second call whichever chunk finishes last."""
+    inp = ipa_inputs(IpaDims(B=2, L=512, H=12, Cz=128), 47)
+    inp["mask"][1, 400:] = False
+    g = upstream((2, 512, 12, 176), 48)
+    got = run_gpu(inp, g)[3]
+    again = run_gpu(inp, g)[3]
+    for key in api.IPA_GRADS:
+        assert np.array_equal(got[key], again[key]), key
+    ref = ipa_grad_blocked(inp, g, block=32)
+    assert_grads(got, ref, "key-pass split", gamma_scale=ipa_grad_gamma_scale(inp, g))
+
+
 def sampled_query_rows(inp, L, n):
     t = inp["trans"][0] - inp["trans"][0].mean(0)
     far = np.argsort(-np.linalg.norm(t, axis=1))[:8]
