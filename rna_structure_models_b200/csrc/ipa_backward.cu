@@ -1464,6 +1464,74 @@ __global__ void __launch_bounds__(256) ipa_bwd_pair_kernel(const MapArgs a) {
   }
 }
 
+// The same sums with 16-byte accesses, when every operand row is contiguous
+// fp32 on 16-byte boundaries and the pair block has no padding (R Cz = DZ,
+// DZ % 128 == 0): thread (residue il, lane) owns columns [128 x + 4 lane,
+// +4) of block column x, so a warp reads 512 contiguous bytes per operand.
+// The per-element arithmetic and every summation order are those of
+// ipa_bwd_pair_kernel (heads in order for d z1 / d z2, the block's residues
+// in order for the d w_bias partials), eight heads per shared-memory round.
+constexpr int PAIR4_HC = 8;
+__global__ void __launch_bounds__(256) ipa_bwd_pair4_kernel(const MapArgs a) {
+  __shared__ float4 wsm4[PAIR_RB][PAIR4_HC][33];
+  const int tid = threadIdx.x, cl = tid & 31, il = tid >> 5;
+  const int col = blockIdx.x * 128 + 4 * cl;
+  const int blk = blockIdx.y, b = blockIdx.z;
+  const int i = blk * PAIR_RB + il;
+  const int H = a.H, C = IPA_C, PV = IPA_PV;
+  const bool valid = i < a.L;
+  const int ic = valid ? i : 0;
+  const int cc = col % a.Cz, rr = col / a.Cz;
+  const int64_t bi = static_cast<int64_t>(b) * a.L + ic;
+  const bool live = valid && a.frame[bi * 4 + 3].x != 0.f;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4 z1 = valid ? *reinterpret_cast<const float4*>(a.z1f + bi * a.DZ + col) : zero;
+  const float* gbase = reinterpret_cast<const float*>(a.g_out.p) + b * a.g_out.s[0] + ic * a.g_out.s[1] + (C + 4 * PV + cc);
+  const float* ubase = reinterpret_cast<const float*>(a.uagg.p) + b * a.uagg.s[0] + ic * a.uagg.s[1] + rr * a.uagg.s[3] + cc;
+  float4 s1 = zero, s2 = zero;
+  for (int h0 = 0; h0 < H; h0 += PAIR4_HC) {
+    const int nh = H - h0 < PAIR4_HC ? H - h0 : PAIR4_HC;
+#pragma unroll 4
+    for (int hh = 0; hh < nh; ++hh) {
+      const int h = h0 + hh;
+      const int64_t bhl = (static_cast<int64_t>(b) * H + h) * a.L + ic;
+      const float4 dq = valid ? *reinterpret_cast<const float4*>(a.dqp + bhl * a.DZ + col) : zero;
+      if (valid) {
+        const float4 gp = *reinterpret_cast<const float4*>(gbase + h * a.g_out.s[2]);
+        const float4 u = *reinterpret_cast<const float4*>(ubase + h * a.uagg.s[2]);
+        const float4 w = *reinterpret_cast<const float4*>(a.wqp + h * a.DZ + col);
+        const float4 d2 = *reinterpret_cast<const float4*>(a.dz2 + bhl * a.DZ + col);
+        s1.x += w.x * dq.x + (live ? gp.x * u.x : 0.f);
+        s1.y += w.y * dq.y + (live ? gp.y * u.y : 0.f);
+        s1.z += w.z * dq.z + (live ? gp.z * u.z : 0.f);
+        s1.w += w.w * dq.w + (live ? gp.w * u.w : 0.f);
+        s2.x += d2.x; s2.y += d2.y; s2.z += d2.z; s2.w += d2.w;
+      }
+      wsm4[il][hh][cl] = make_float4(z1.x * dq.x, z1.y * dq.y, z1.z * dq.z, z1.w * dq.w);
+    }
+    __syncthreads();
+    for (int t = tid; t < nh * 32; t += blockDim.x) {
+      const int hh = t >> 5, c = t & 31;
+      float4 w = zero;
+#pragma unroll
+      for (int q = 0; q < PAIR_RB; ++q) {
+        const float4 v = wsm4[q][hh][c];
+        w.x += v.x; w.y += v.y; w.z += v.z; w.w += v.w;
+      }
+      float4* dst = reinterpret_cast<float4*>(
+          IPA_SPAN(a.wb_part, ((static_cast<int64_t>(b) * gridDim.y + blk) * H + h0 + hh) * a.DZ + blockIdx.x * 128 + 4 * c,
+                   4, static_cast<int64_t>(a.B) * gridDim.y * H * a.DZ, a.err));
+      *dst = w;
+    }
+    __syncthreads();
+  }
+  if (valid) {
+    const int64_t nz = static_cast<int64_t>(a.B) * a.L * a.RCz;
+    *reinterpret_cast<float4*>(IPA_SPAN(a.d_z1, bi * a.RCz + col, 4, nz, a.err)) = s1;
+    *reinterpret_cast<float4*>(IPA_SPAN(a.d_z2, bi * a.RCz + col, 4, nz, a.err)) = s2;
+  }
+}
+
 // One block of 1024 threads per (head, 32 columns).  Thread (c, g): group g
 // of 32 sums parts g, g + 32, ... (factors r in order) for column c; the 32
 // group sums are then added in group order.  Warp 0 of the first column
@@ -1722,8 +1790,15 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int npb = (L + PAIR_RB - 1) / PAIR_RB;
-  ipa_bwd_pair_kernel<<<dim3(static_cast<unsigned>((DZ + 31) / 32), static_cast<unsigned>(npb), static_cast<unsigned>(B)),
-                        256, 0, stream>>>(m);
+  if (ra.pair_cpl != 0 && (reinterpret_cast<uintptr_t>(a.d_z1) & 15u) == 0 &&
+      (reinterpret_cast<uintptr_t>(a.d_z2) & 15u) == 0)
+    // the rows kernel's 16-byte conditions (fp32 rows on 16-byte boundaries,
+    // R Cz = DZ, DZ = 128 or 256) and aligned gradient outputs
+    ipa_bwd_pair4_kernel<<<dim3(static_cast<unsigned>(DZ / 128), static_cast<unsigned>(npb), static_cast<unsigned>(B)),
+                           256, 0, stream>>>(m);
+  else
+    ipa_bwd_pair_kernel<<<dim3(static_cast<unsigned>((DZ + 31) / 32), static_cast<unsigned>(npb), static_cast<unsigned>(B)),
+                          256, 0, stream>>>(m);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const dim3 rgrid(static_cast<unsigned>(H), static_cast<unsigned>((f.Cz + 31) / 32));
