@@ -1581,13 +1581,22 @@ bool ipa_bwd_trace_read(void* host, size_t bytes) {
 }
 #endif
 
+// Residues per block of ipa_bwd_map_kernel (one thread per residue and
+// head): about 64 threads, so that a long sequence spreads as many small
+// blocks evenly over the SMs (with 256-thread blocks, L = 4096 and H = 12
+// gave 196 blocks on 148 SMs, and the SMs holding two set the time).
+static int map_residues_per_block(int H) {
+  const int rb = 64 / H;
+  return rb < 1 ? 1 : rb > 32 ? 32 : rb;
+}
+
 IpaBwdWorkspace ipa_bwd_workspace_layout(int B, int L, int H, int DZ, int RCz) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   IpaBwdWorkspace w{};
   w.fwd = ipa_workspace_layout(B, L, H, DZ, RCz);
   size_t o = up(w.fwd.total);
   const size_t bhl = static_cast<size_t>(B) * H * L;
-  const int rb = 256 / H < 32 ? 256 / H : 32;
+  const int rb = map_residues_per_block(H);
   const size_t nblk = (L + rb - 1) / rb;                // per-residue mapping blocks
   const size_t npb = (L + PAIR_RB - 1) / PAIR_RB;        // pair-column blocks
   w.doh = o; o = up(o + bhl * 64 * 2);
@@ -1773,7 +1782,7 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   // 5. per-residue mapping and the reductions
   MapArgs m{};
   m.B = B; m.L = L; m.H = H; m.DZ = DZ; m.RCz = f.RCz; m.Cz = f.Cz; m.R = f.R;
-  m.rb = 256 / H < 32 ? 256 / H : 32;
+  m.rb = map_residues_per_block(H);
   m.nblk = (L + m.rb - 1) / m.rb;
   m.qscale = ba.qscale; m.w_L = f.w_L; m.w_C = f.w_C;
   m.q_pts = f.q_pts; m.k_pts = f.k_pts; m.v_pts = f.v_pts; m.g_out = a.g_out; m.out = a.out; m.uagg = a.uagg;
@@ -1786,7 +1795,8 @@ cudaError_t ipa_launch_bwd(const IpaBwdLaunch& a, cudaStream_t stream) {
   m.g_part = reinterpret_cast<double*>(ws + w.g_part);
   m.err = f.err;
   const size_t msmem = static_cast<size_t>((m.rb * H * 12 + 1) & ~1) * 4 + static_cast<size_t>(m.rb) * H * 8;
-  ipa_bwd_map_kernel<<<dim3(static_cast<unsigned>(m.nblk), static_cast<unsigned>(B)), 256, msmem, stream>>>(m);
+  const unsigned mthreads = static_cast<unsigned>((m.rb * H + 31) / 32 * 32);
+  ipa_bwd_map_kernel<<<dim3(static_cast<unsigned>(m.nblk), static_cast<unsigned>(B)), mthreads, msmem, stream>>>(m);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int npb = (L + PAIR_RB - 1) / PAIR_RB;
