@@ -31,6 +31,13 @@
 //
 // The softmax, lazy rescaling, rounded row sums, tile-local point terms and
 // the epilogue are those of the single-CTA kernel (ipa_attention.cu).
+//
+// Key-split tail (inference only): the pair tiles of the last, partial wave
+// may each run as 2-5 CTA pairs over consecutive key-tile ranges.  Each
+// stores its un-normalised accumulators, row maximum and half sums; the one
+// that takes the last ticket merges the chunks in chunk order into tensor
+// memory (flash-decoding style rescale by 2^(m_s - max m)) and runs the
+// output pass.  ipa_split_plan chooses the chunk count on the host.
 #include <cuda_fp16.h>
 
 #include <cmath>

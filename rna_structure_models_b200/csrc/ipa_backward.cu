@@ -16,7 +16,9 @@
 //   dS_ij = ln 2 p_ij (dP_ij - D_i)        D_i = sum_j p_ij dP_ij, from the
 //                                          forward output and U
 // dS is dL/dx.  The kernels:
-//   ipa_bwd_rows_kernel  one warp per (b, i, h): dO, dU, Q_pair (fp16 rows),
+//   ipa_bwd_rows_kernel  one warp per (b, i, h): dO, dU, Q_pair (fp16 rows;
+//                        DZ / 32 columns per lane with 16-byte accesses for
+//                        contiguous fp32 rows),
 //                        the row constant -(w_i + lse2_i), D_i and the query
 //                        and key points relative to the centroid (fp32);
 //   query pass           one CTA per (b, h, 128 queries), 32-key tiles:
@@ -31,12 +33,17 @@
 //                        sum_i dS_ij |gq_i - gk_j|^2 from fp32 points (CUDA
 //                        cores, inside the dS loop);
 //   (both passes run as one grid, ipa_bwd_kernel, so that the key-pass CTAs
-//   fill the SMs the query pass leaves idle in its last wave)
+//   fill the SMs the query pass leaves idle in its last wave; key-pass CTAs
+//   of the grid's last, partial wave may run as chunks of consecutive query
+//   tiles whose partial sums the chunk with the last ticket adds in chunk
+//   order, ipa_bwd_split_plan)
 //   ipa_bwd_map_kernel   per residue, all heads: the augmented gradients
 //                        mapped back to q, k, v, the local points and the
 //                        frames (sums over heads), per-block d gamma partials;
 //   ipa_bwd_pair_kernel  per pair column and residue: d z1, d z2
-//                        (sums over heads) and d w_bias partials;
+//                        (sums over heads) and d w_bias partials
+//                        (ipa_bwd_pair4_kernel: four columns per thread,
+//                        16-byte accesses, for contiguous fp32 rows);
 //   ipa_bwd_reduce_kernel  fixed-order sums of the partials, one block per
 //                        (head, 32 pair columns).
 // Every mbarrier wait is bounded (2 s) and reports into the error word.
