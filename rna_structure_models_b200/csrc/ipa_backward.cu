@@ -1540,8 +1540,9 @@ __global__ void __launch_bounds__(256) ipa_bwd_pair4_kernel(const MapArgs a) {
 }
 
 // One block of 1024 threads per (head, 32 columns).  Thread (c, g): group g
-// of 32 sums parts g, g + 32, ... (factors r in order) for column c; the 32
-// group sums are then added in group order.  Warp 0 of the first column
+// of 32 sums parts g, g + 32, ... (factors r in order, four running sums
+// over parts 128 apart) for column c; the 32 group sums are then added in
+// group order.  Warp 0 of the first column
 // block sums the d gamma parts, lane l taking parts l, l + 32, ..., then a
 // fixed shuffle tree.  The order of every sum depends on the sizes alone, so
 // the result is reproducible.
@@ -1552,11 +1553,25 @@ __global__ void __launch_bounds__(RED_THREADS) ipa_bwd_reduce_kernel(const float
   __shared__ double red[32][33];
   const int h = blockIdx.x, t = threadIdx.x, cl = t & 31, g = t >> 5;
   const int c = blockIdx.y * 32 + cl;
-  double acc = 0.0;
-  if (c < Cz)
-    for (int p = g; p < nwb; p += 32)
-      for (int r = 0; r < R; ++r) acc += wb_part[(static_cast<int64_t>(p) * H + h) * DZ + r * Cz + c];
-  red[g][cl] = acc;
+  // four independent running sums (parts p, p + 32, p + 64, p + 96 of each
+  // step of 128), so that four loads are in flight; combined in a fixed order
+  double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
+  if (c < Cz) {
+    const int64_t pstride = static_cast<int64_t>(H) * DZ;
+    const float* col = wb_part + static_cast<int64_t>(h) * DZ + c;
+    int p = g;
+    for (; p + 96 < nwb; p += 128)
+      for (int r = 0; r < R; ++r) {
+        const float* q = col + r * Cz + p * pstride;
+        acc0 += q[0];
+        acc1 += q[32 * pstride];
+        acc2 += q[64 * pstride];
+        acc3 += q[96 * pstride];
+      }
+    for (; p < nwb; p += 32)
+      for (int r = 0; r < R; ++r) acc0 += col[r * Cz + p * pstride];
+  }
+  red[g][cl] = (acc0 + acc1) + (acc2 + acc3);
   __syncthreads();
   if (t < 32 && c < Cz) {
     double sum = 0.0;
@@ -1565,8 +1580,16 @@ __global__ void __launch_bounds__(RED_THREADS) ipa_bwd_reduce_kernel(const float
   }
   if (blockIdx.y == 0 && t >= 32 && t < 64) {
     const int l = t - 32;
-    double gs = 0.0;
-    for (int p = l; p < ng; p += 32) gs += g_part[static_cast<int64_t>(p) * H + h];
+    double g0 = 0.0, g1 = 0.0, g2 = 0.0, g3 = 0.0;
+    int p = l;
+    for (; p + 96 < ng; p += 128) {
+      g0 += g_part[static_cast<int64_t>(p) * H + h];
+      g1 += g_part[static_cast<int64_t>(p + 32) * H + h];
+      g2 += g_part[static_cast<int64_t>(p + 64) * H + h];
+      g3 += g_part[static_cast<int64_t>(p + 96) * H + h];
+    }
+    for (; p < ng; p += 32) g0 += g_part[static_cast<int64_t>(p) * H + h];
+    double gs = (g0 + g1) + (g2 + g3);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, off);
     if (l == 0) *IPA_AT(d_gamma, h, H, err) = static_cast<float>(gs);
