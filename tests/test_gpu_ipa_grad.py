@@ -185,8 +185,8 @@ def test_gradients_are_reproducible(cuda_device):
 def test_gradients_with_the_key_pass_split(cuda_device):
     """B = 2, L = 512, H = 12: 96 query-pass and 96 key-pass CTAs, one per SM
     on 148 SMs, leave a last wave of 44 key-pass CTAs.  Each of those runs as
-    three chunks of its 16 query tiles; the chunk that finishes last adds the
-    partial sums in chunk order.  Every gradient against the oracle, and the
+    two chunks of its 16 query tiles (the reserve holds 96 chunks); the chunk
+    that finishes last adds the partial sums in chunk order.  Every gradient against the oracle, and the
     same bits on a second call whichever chunk finishes last."""
     inp = ipa_inputs(IpaDims(B=2, L=512, H=12, Cz=128), 47)
     inp["mask"][1, 400:] = False
